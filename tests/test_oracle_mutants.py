@@ -1,0 +1,52 @@
+"""The pins must catch plausible mistakes in the oracle.
+
+Each case plants one mistake in a copy of the oracle source (a dropped term, a wrong sign, a
+wrong divisor, a dropped index, a flipped comparison), builds it with gcc, and runs the pin
+suite against that build in a subprocess: the suite has to fail. CPU only.
+"""
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "ekv_oracle.c")
+
+MUTANTS = {
+    "bound_takes_min": ("acc += a > b ? a : b;", "acc += a < b ? a : b;"),
+    "variance_divides_by_n_minus_1": ("var[(size_t)j * d + c] = ss / n;",
+                                      "var[(size_t)j * d + c] = ss / (n > 1 ? n - 1 : 1);"),
+    "meta_ignores_head": ("return (((size_t)block * H_kv + h) * P + t) * d + c;",
+                          "return (((size_t)block * H_kv) * P + t) * d + c; (void)h;"),
+    "entmax15_wrong_root": ("tk = mean - sqrt(disc);", "tk = mean + sqrt(disc);"),
+    "sparsemax_wrong_sign": ("tk = (sum - 1.0) / k;", "tk = (sum + 1.0) / k;"),
+    "trunc_moment_drops_pdf_term": ("return r * Phi + b * phi;", "return r * Phi;"),
+    "trunc_moment15_drops_variance": ("return (r * r + b * b) * Phi + r * b * phi;",
+                                      "return (r * r) * Phi + r * b * phi;"),
+    "topk_ties_to_higher_index": ("return a < b ? -1 : (a > b);\n}\n\nstatic int cmp_int_asc",
+                                  "return a > b ? -1 : (a < b);\n}\n\nstatic int cmp_int_asc"),
+    "gauss_v_not_squared": ("b += qc * qc * var[(size_t)j * d + c];",
+                            "b += qc * var[(size_t)j * d + c];"),
+    "gauss_select_not_strict": ("> tau_hat[g] - delta)", ">= tau_hat[g] - delta)"),
+    "softmax_stat_drops_max": ("stat[g] = mx + log(l);", "stat[g] = log(l);"),
+    "attention_reads_invalid_tokens": (
+        "n_tok += seq_len - j * P < P ? seq_len - j * P : P;", "n_tok += P;"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_planted_mistake(name, tmp_path):
+    old, new = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(old) == 1, "mutation anchor not found: " + name
+    mut = tmp_path / "mutant.c"
+    mut.write_text(src.replace(old, new))
+    lib = tmp_path / "libmutant.so"
+    subprocess.check_call(["gcc", "-std=c11", "-D_DEFAULT_SOURCE", "-O2", "-fPIC", "-shared",
+                           "-o", str(lib), str(mut), "-lm"])
+    env = dict(os.environ, EKV_ORACLE_LIB=str(lib))
+    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+                        os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode != 0, "planted mistake %s went unnoticed:\n%s" % (name, r.stdout[-2000:])

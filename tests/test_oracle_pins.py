@@ -1,0 +1,504 @@
+"""Pins for the CPU oracle: each check ties it to something other than itself.
+
+Sources: EntmaxKV technical summary (gist.science) §2.A (page metadata and bound), §2.B
+(top-k and Gaussian-aware selection), §2.C (exact sparse entmax attention), §3 (error bound
+2*B*delta, support recovery). Pins are closed forms, hand-worked fixtures under tests/golden/,
+library routines (numpy/scipy) on the defining equations, brute force on tiny inputs, and the
+invariants the summary states.
+"""
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+from scipy import integrate, optimize, special, stats
+
+import oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# ----------------------------------------------------------------------------- helpers
+def rand_cache(rng, nb, H_kv, P, d, dist=None):
+    if dist is None:
+        return rng.standard_normal((nb, H_kv, P, d)).astype(np.float32)
+    return dist(rng, (nb, H_kv, P, d)).astype(np.float32)
+
+
+def parse_golden(name):
+    out = {}
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.split("#", 1)[0].strip()
+            if not line:
+                continue
+            key, val = (s.strip() for s in line.split("=", 1))
+            rows = [[float(Fraction(x)) for x in r.split()] for r in val.split(";")]
+            out[key] = np.array(rows if len(rows) > 1 else rows[0])
+    return out
+
+
+def page_cache_from_keys(keys, P=None):
+    """One sequence, one KV head, one block holding `keys` [n, d]."""
+    n, d = keys.shape
+    P = P or n
+    k = np.zeros((1, 1, P, d), dtype=np.float32)
+    k[0, 0, :n] = keys
+    return k
+
+
+# ----------------------------------------------------------------------------- §2.A metadata
+def test_meta_golden_fixture():
+    g = parse_golden("bbox_page_example.txt")
+    k = page_cache_from_keys(g["keys"])
+    kmin, kmax, mean, var = O.page_meta_head(k, [0], 3, 0)
+    np.testing.assert_array_equal(kmin[0], g["kmin"])
+    np.testing.assert_array_equal(kmax[0], g["kmax"])
+    np.testing.assert_allclose(mean[0], g["mean"], rtol=0, atol=1e-15)
+    np.testing.assert_allclose(var[0], g["var"], rtol=1e-15, atol=1e-15)
+
+
+@pytest.mark.parametrize("n,P", [(16, 16), (5, 16), (1, 8), (64, 64)])
+def test_meta_arithmetic_progression_closed_form(n, P):
+    # k_t = a_c + t * b_c: min/max at the ends, mean a + b(n-1)/2, variance b^2 (n^2-1)/12.
+    d = 8
+    a = np.array([-3.0, -1.5, 0.25, 2.0, -0.75, 1.0, 0.5, -2.0])  # dyadic: exact in float32
+    b = np.array([0.5, -0.25, 1.0, -1.0, 0.125, 2.0, -0.5, 0.0])
+    keys = a[None, :] + np.arange(n)[:, None] * b[None, :]
+    k = page_cache_from_keys(keys, P)
+    kmin, kmax, mean, var = O.page_meta_head(k, [0], n, 0)
+    ends = np.stack([a, a + (n - 1) * b])
+    np.testing.assert_array_equal(kmin[0], ends.min(0))
+    np.testing.assert_array_equal(kmax[0], ends.max(0))
+    np.testing.assert_allclose(mean[0], a + b * (n - 1) / 2, atol=1e-12)
+    np.testing.assert_allclose(var[0], b * b * (n * n - 1) / 12.0, rtol=1e-12, atol=1e-12)
+
+
+def test_meta_constant_page():
+    keys = np.full((7, 4), 1.25)
+    kmin, kmax, mean, var = O.page_meta_head(page_cache_from_keys(keys, 16), [0], 7, 0)
+    assert np.all(kmin == 1.25) and np.all(kmax == 1.25) and np.all(mean == 1.25)
+    assert np.all(var == 0.0)
+
+
+def test_meta_paged_layout_against_numpy():
+    # Several sequences, scattered blocks, partial last pages: numpy reductions over the
+    # valid tokens of block page_table[b, j], head h, must agree.
+    rng = np.random.default_rng(1)
+    nb, H_kv, P, d = 40, 3, 8, 6
+    k = rand_cache(rng, nb, H_kv, P, d)
+    perm = rng.permutation(nb).astype(np.int32)
+    seq_lens = [37, 8, 1]
+    pt = np.full((3, 5), -1, np.int32)
+    nxt = 0
+    for b, L in enumerate(seq_lens):
+        n = O.pages_of(L, P)
+        pt[b, :n] = perm[nxt:nxt + n]
+        nxt += n
+    for b, L in enumerate(seq_lens):
+        for h in range(H_kv):
+            kmin, kmax, mean, var = O.page_meta_head(k, pt[b], L, h)
+            for j in range(O.pages_of(L, P)):
+                rows = k[pt[b, j], h, :min(P, L - j * P)].astype(np.float64)
+                np.testing.assert_array_equal(kmin[j], rows.min(0))
+                np.testing.assert_array_equal(kmax[j], rows.max(0))
+                np.testing.assert_allclose(mean[j], rows.mean(0), atol=1e-14)
+                np.testing.assert_allclose(var[j], rows.var(0), atol=1e-14)
+
+
+def test_meta_bf16_widening_is_exact():
+    # bf16 bit patterns widen to the float32 with the same upper half.
+    rng = np.random.default_rng(2)
+    f = rng.standard_normal((1, 1, 4, 8)).astype(np.float32)
+    bits = (f.view(np.uint32) >> 16).astype(np.uint16)
+    exact = (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    kmin, kmax, _, _ = O.page_meta_head(bits, [0], 4, 0)
+    np.testing.assert_array_equal(kmin[0], exact[0, 0].min(0))
+    np.testing.assert_array_equal(kmax[0], exact[0, 0].max(0))
+
+
+def test_meta_rejects_bad_block():
+    k = np.zeros((2, 1, 4, 2), np.float32)
+    with pytest.raises(ValueError):
+        O.page_meta_head(k, [0, 2], 8, 0)
+
+
+# ----------------------------------------------------------------------------- §2.A bound
+def test_bound_golden_fixture():
+    g = parse_golden("bbox_page_example.txt")
+    ub, S = O.score_head(g["q"], 1.0, g["kmin"][None], g["kmax"][None])
+    np.testing.assert_array_equal(ub[:, 0], g["ub"])
+    assert S[0] == g["S"]
+    best = (g["q"] @ g["keys"].T).max(1)
+    np.testing.assert_array_equal(best, g["best"])
+    m, v = O.gauss_stats_head(g["q"], 1.0, g["mean"][None], g["var"][None])
+    np.testing.assert_allclose(m[:, 0], g["m"], atol=1e-15)
+    np.testing.assert_allclose(v[:, 0], g["v"], rtol=1e-15)
+
+
+def test_bound_dominates_every_token_brute_force():
+    # §2.A: the bound is an upper bound on the score of every token in the page.
+    rng = np.random.default_rng(3)
+    for trial in range(30):
+        P, d, G = rng.choice([1, 3, 16]), rng.choice([2, 5, 64]), rng.choice([1, 4])
+        n = rng.integers(1, P + 1)
+        keys = rng.standard_normal((n, d)) * rng.choice([0.1, 1, 10])
+        k = page_cache_from_keys(keys.astype(np.float32), P)
+        kmin, kmax, _, _ = O.page_meta_head(k, [0], n, 0)
+        q = rng.standard_normal((G, d))
+        scale = float(rng.choice([1.0, 0.125, 3.0]))
+        ub, S = O.score_head(q, scale, kmin, kmax)
+        s = scale * q @ k[0, 0, :n].astype(np.float64).T
+        assert np.all(ub[:, 0] >= s.max(1) - 1e-12 * np.abs(s).max())
+        np.testing.assert_allclose(S[0], ub[:, 0].sum(), rtol=1e-14)
+
+
+def test_bound_tight_for_single_token_page():
+    rng = np.random.default_rng(4)
+    keys = rng.standard_normal((1, 16))
+    kmin, kmax, _, _ = O.page_meta_head(page_cache_from_keys(keys.astype(np.float32)), [0], 1, 0)
+    q = rng.standard_normal((3, 16))
+    ub, _ = O.score_head(q, 0.5, kmin, kmax)
+    np.testing.assert_allclose(ub[:, 0], 0.5 * q @ keys.astype(np.float32).astype(np.float64)[0],
+                               rtol=1e-13)
+
+
+def test_bound_sign_split_closed_form():
+    # For q >= 0 coordinate-wise the bound is q.kmax; for q <= 0 it is q.kmin.
+    rng = np.random.default_rng(5)
+    kmin = -np.abs(rng.standard_normal((3, 8)))
+    kmax = np.abs(rng.standard_normal((3, 8)))
+    qp = np.abs(rng.standard_normal((1, 8)))
+    ub, _ = O.score_head(qp, 1.0, kmin, kmax)
+    np.testing.assert_allclose(ub[0], kmax @ qp[0], rtol=1e-14)
+    ub, _ = O.score_head(-qp, 1.0, kmin, kmax)
+    np.testing.assert_allclose(ub[0], kmin @ -qp[0], rtol=1e-14)
+
+
+def test_gauss_stats_are_mean_and_variance_of_the_scores():
+    # m = q.mean and v = sum_c q_c^2 var_c are the exact mean and variance of q.k over a
+    # page whose coordinates are independent: check on an outer-product page where they are.
+    rng = np.random.default_rng(6)
+    d = 3
+    vals = [rng.standard_normal(2) for _ in range(d)]
+    import itertools
+    keys = np.array(list(itertools.product(*vals)))  # every combination: coordinates independent
+    k = page_cache_from_keys(keys.astype(np.float32))
+    _, _, mean, var = O.page_meta_head(k, [0], len(keys), 0)
+    q = rng.standard_normal((2, d))
+    m, v = O.gauss_stats_head(q, 1.0, mean, var)
+    s = q @ k[0, 0].astype(np.float64).T
+    np.testing.assert_allclose(m[:, 0], s.mean(1), atol=1e-13)
+    np.testing.assert_allclose(v[:, 0], s.var(1), atol=1e-13)
+
+
+# ----------------------------------------------------------------------------- §2.B.1 top-k
+@pytest.mark.parametrize("seed", range(8))
+def test_topk_matches_library_sort(seed):
+    rng = np.random.default_rng(seed)
+    n = int(rng.integers(1, 300))
+    S = rng.integers(-5, 5, size=n).astype(np.float64) if seed % 2 else rng.standard_normal(n)
+    for k in [1, 2, n // 3 + 1, n, n + 7]:
+        ref = sorted(sorted(range(n), key=lambda j: (-S[j], j))[:k])
+        np.testing.assert_array_equal(O.topk(S, k), ref)
+
+
+def test_topk_tie_storm_prefers_lower_index():
+    S = np.zeros(100)
+    np.testing.assert_array_equal(O.topk(S, 10), np.arange(10))
+    S[50:] = 1.0
+    np.testing.assert_array_equal(O.topk(S, 55), np.r_[np.arange(5), np.arange(50, 100)])
+
+
+# ----------------------------------------------------------------------------- §2.C entmax
+def entmax_objective(p, z, alpha):
+    # Peters et al. (2019): alpha-entmax(s) = argmax_p p.s + H_alpha(p) over the simplex, with
+    # the Tsallis entropy H_alpha(p) = sum_j (p_j - p_j^alpha) / (alpha (alpha - 1)). The
+    # oracle works in the z = (alpha - 1) s domain, so the logits here are s = z / (alpha - 1).
+    s = np.asarray(z) / (alpha - 1.0)
+    return p @ s + np.sum(p - p ** alpha) / (alpha * (alpha - 1.0))
+
+
+@pytest.mark.parametrize("alpha", [1.5, 2.0])
+def test_entmax_closed_forms(alpha):
+    np.testing.assert_allclose(O.entmax([3.7], alpha), [1.0])
+    np.testing.assert_allclose(O.entmax(np.zeros(5), alpha), np.full(5, 0.2), atol=1e-15)
+    np.testing.assert_allclose(O.entmax([1.0, 0.0], alpha), [1.0, 0.0])       # gap >= 1
+    np.testing.assert_allclose(O.entmax([2.0, 0.5, -3.0], alpha), [1.0, 0.0, 0.0])
+    d = 0.5
+    if alpha == 2.0:
+        ref = [(1 + d) / 2, (1 - d) / 2]
+    else:
+        x = (d + math.sqrt(2 - d * d)) / 2  # x^2 + (x - d)^2 = 1, both positive for d < 1
+        ref = [x * x, (x - d) ** 2]
+    np.testing.assert_allclose(O.entmax([d, 0.0], alpha), ref, atol=1e-15)
+
+
+@pytest.mark.parametrize("alpha", [1.5, 2.0])
+def test_entmax_tau_solves_the_normalisation_equation(alpha):
+    # tau is the root of sum_i [z_i - tau]_+^(1/(alpha-1)) = 1, found here by scipy's brentq.
+    rng = np.random.default_rng(7)
+    for n in [1, 2, 3, 10, 100, 2000]:
+        z = rng.standard_normal(n) * rng.choice([0.1, 1.0, 5.0])
+        pw = 1.0 / (alpha - 1.0)
+        f = lambda t: np.sum(np.maximum(z - t, 0.0) ** pw) - 1.0
+        ref = optimize.brentq(f, z.max() - 1.0, z.max(), xtol=1e-15, rtol=1e-15)
+        tau = O.entmax_tau(z, alpha)
+        assert abs(tau - ref) <= 1e-12 * max(1.0, abs(ref))
+        p = O.entmax(z, alpha)
+        assert abs(p.sum() - 1.0) <= 1e-12
+        assert np.all(p >= 0)
+
+
+@pytest.mark.parametrize("alpha", [1.5, 2.0])
+def test_entmax_is_the_variational_maximiser(alpha):
+    rng = np.random.default_rng(8)
+    for _ in range(10):
+        n = int(rng.integers(2, 7))
+        z = rng.standard_normal(n)
+        p = O.entmax(z, alpha)
+        best = entmax_objective(p, z, alpha)
+        res = optimize.minimize(lambda x: -entmax_objective(x, z, alpha),
+                                np.full(n, 1.0 / n), method="SLSQP", bounds=[(0.0, 1.0)] * n,
+                                constraints=[{"type": "eq", "fun": lambda x: x.sum() - 1}],
+                                options={"ftol": 1e-14, "maxiter": 500})
+        x = np.maximum(res.x, 0.0)
+        x /= x.sum()  # a feasible simplex point near the optimiser's answer
+        assert best >= entmax_objective(x, z, alpha) - 1e-12
+        assert np.abs(x - p).max() < 1e-4  # and the optimiser lands on the same distribution
+        for _ in range(200):
+            r = rng.dirichlet(np.ones(n) * rng.choice([0.2, 1.0, 5.0]))
+            assert best >= entmax_objective(r, z, alpha) - 1e-12
+
+
+@pytest.mark.parametrize("alpha", [1.5, 2.0])
+def test_entmax_shift_invariance_and_kkt(alpha):
+    rng = np.random.default_rng(9)
+    z = rng.standard_normal(64) * 2
+    tau = O.entmax_tau(z, alpha)
+    assert abs(O.entmax_tau(z + 3.25, alpha) - (tau + 3.25)) <= 1e-12
+    p = O.entmax(z, alpha)
+    on = p > 0
+    # KKT: in the support z_i - tau = p_i^(alpha-1); outside it z_i <= tau.
+    np.testing.assert_allclose(z[on] - tau, p[on] ** (alpha - 1.0), rtol=1e-12)
+    assert np.all(z[~on] <= tau)
+
+
+# ----------------------------------------------------------------------------- §2.B.2 Gaussian
+@pytest.mark.parametrize("alpha", [1.5, 2.0])
+def test_trunc_moment_against_quadrature(alpha):
+    pw = 1.0 / (alpha - 1.0)
+    for a, b, tau in [(0.3, 1.0, 0.0), (-2.0, 0.5, 1.0), (1.0, 0.01, 0.5), (4.0, 3.0, 9.0),
+                      (0.0, 2.0, -5.0)]:
+        f = lambda x: (x - tau) ** pw * stats.norm.pdf(x, loc=a, scale=b)
+        ref, _ = integrate.quad(f, tau, np.inf, epsabs=1e-14, epsrel=1e-12)
+        assert abs(O.trunc_moment(a, b, tau, alpha) - ref) <= 1e-10 * max(1.0, ref)
+    assert O.trunc_moment(1.0, 0.0, 0.25, alpha) == 0.75 ** pw
+    assert O.trunc_moment(1.0, 0.0, 1.5, alpha) == 0.0
+
+
+@pytest.mark.parametrize("alpha", [1.5, 2.0])
+def test_gauss_tau_zero_variance_reduces_to_exact_entmax(alpha):
+    # With all page variances zero, page j is n_j copies of one score: F(tau) = 1 is exactly
+    # the entmax normalisation over that multiset, so tau-hat is the exact entmax threshold.
+    rng = np.random.default_rng(10)
+    for _ in range(5):
+        n = int(rng.integers(1, 40))
+        m = rng.standard_normal(n) * 2
+        cnt = rng.integers(1, 17, size=n).astype(np.int32)
+        th = O.gauss_tau(m, np.zeros(n), cnt, alpha)
+        z = np.repeat((alpha - 1.0) * m, cnt)
+        pw = 1.0 / (alpha - 1.0)
+        ref = optimize.brentq(lambda t: np.sum(np.maximum(z - t, 0) ** pw) - 1.0,
+                              z.max() - 1, z.max(), xtol=1e-15, rtol=1e-15)
+        assert abs(th - ref) <= 1e-11 * max(1.0, abs(ref))
+        assert abs(th - O.entmax_tau(z, alpha)) <= 1e-11 * max(1.0, abs(ref))
+
+
+@pytest.mark.parametrize("alpha", [1.5, 2.0])
+def test_gauss_tau_monte_carlo(alpha):
+    # F(tau-hat) = 1 in expectation: draw n_j iid N(m_j, v_j) scores per page and average the
+    # entmax mass sum_i [(alpha-1) s_i - tau-hat]_+^(1/(alpha-1)) over many draws.
+    rng = np.random.default_rng(11)
+    n = 12
+    m = rng.standard_normal(n)
+    v = rng.uniform(0.05, 1.0, n)
+    cnt = rng.integers(1, 33, size=n).astype(np.int32)
+    th = O.gauss_tau(m, v, cnt, alpha)
+    assert abs(O.gauss_F(m, v, cnt, alpha, th) - 1.0) <= 1e-10
+    draws = 20000
+    tot = np.zeros(draws)
+    pw = 1.0 / (alpha - 1.0)
+    for j in range(n):
+        s = rng.normal(m[j], math.sqrt(v[j]), size=(draws, cnt[j]))
+        tot += np.sum(np.maximum((alpha - 1.0) * s - th, 0.0) ** pw, axis=1)
+    se = tot.std() / math.sqrt(draws)
+    assert abs(tot.mean() - 1.0) <= 5 * se
+
+
+def test_gauss_F_is_decreasing():
+    rng = np.random.default_rng(12)
+    m, v = rng.standard_normal(20), rng.uniform(0, 1, 20)
+    cnt = np.full(20, 16, np.int32)
+    taus = np.linspace(-5, 5, 200)
+    F = [O.gauss_F(m, v, cnt, 1.5, t) for t in taus]
+    assert np.all(np.diff(F) <= 0)
+
+
+def test_gauss_select_rule():
+    # keep j iff some query g has (alpha - 1) UB_gj > tau_hat_g - delta (strict)
+    ub = np.array([[1.0, 2.0, 3.0, 0.0], [0.0, 0.0, 0.0, 2.1]])
+    tau_hat = np.array([1.1, 1.0])
+    # alpha 1.5: thresholds 1.0 / 0.9; page 1 gives 0.5*2 = 1.0, not strictly above -> dropped
+    np.testing.assert_array_equal(O.gauss_select(ub, tau_hat, 1.5, 0.1), [2, 3])
+    np.testing.assert_array_equal(O.gauss_select(ub, tau_hat, 2.0, 0.1), [1, 2, 3])
+    np.testing.assert_array_equal(O.gauss_select(ub, tau_hat, 2.0, 0.0), [1, 2, 3])
+    np.testing.assert_array_equal(O.gauss_select(ub, np.array([2.0, 1.0]), 2.0, 0.0), [2, 3])
+
+
+# ----------------------------------------------------------------------------- §2.C / §3 attention
+def make_seq(rng, P=8, d=16, H_kv=2, L=61, nb=20, dist_scale=1.0):
+    k = (rng.standard_normal((nb, H_kv, P, d)) * dist_scale).astype(np.float32)
+    v = rng.standard_normal((nb, H_kv, P, d)).astype(np.float32)
+    pt = rng.permutation(nb)[:O.pages_of(L, P)].astype(np.int32)
+    return k, v, pt
+
+
+def dense_tokens(cache, pt, L, h):
+    P = cache.shape[2]
+    rows = [cache[pt[j], h, t] for j in range(O.pages_of(L, P)) for t in range(min(P, L - j * P))]
+    return np.array(rows, dtype=np.float64)
+
+
+def test_softmax_all_pages_equals_dense_attention():
+    rng = np.random.default_rng(13)
+    k, v, pt = make_seq(rng)
+    L, h, scale = 61, 1, 0.3
+    q = rng.standard_normal((3, 16))
+    allp = np.arange(O.pages_of(L, 8))
+    out, stat, _ = O.attend_head(k, v, pt, L, h, q, scale, O.SOFTMAX, allp)
+    K, V = dense_tokens(k, pt, L, h), dense_tokens(v, pt, L, h)
+    s = scale * q @ K.T
+    ref = special.softmax(s, axis=1) @ V
+    np.testing.assert_allclose(out, ref, atol=1e-13)
+    np.testing.assert_allclose(stat, special.logsumexp(s, axis=1), atol=1e-13)
+
+
+@pytest.mark.parametrize("mode", [O.ENTMAX15, O.SPARSEMAX])
+def test_entmax_all_pages_equals_dense_entmax(mode):
+    rng = np.random.default_rng(14)
+    k, v, pt = make_seq(rng, dist_scale=3.0)
+    L, h, scale = 61, 0, 0.5
+    alpha = O.ALPHA_OF_MODE[mode]
+    q = rng.standard_normal((2, 16))
+    out, stat, _ = O.attend_head(k, v, pt, L, h, q, scale, mode, np.arange(8))
+    K, V = dense_tokens(k, pt, L, h), dense_tokens(v, pt, L, h)
+    pw = 1.0 / (alpha - 1.0)
+    for g in range(2):
+        z = (alpha - 1.0) * scale * K @ q[g]
+        tau = optimize.brentq(lambda t: np.sum(np.maximum(z - t, 0) ** pw) - 1.0,
+                              z.max() - 1, z.max(), xtol=1e-15, rtol=1e-15)
+        p = np.maximum(z - tau, 0) ** pw
+        np.testing.assert_allclose(out[g], p @ V, atol=1e-11)
+        assert abs(stat[g] - tau) <= 1e-12 * max(1, abs(tau))
+
+
+def full_support_pages(k, v, pt, L, h, q, scale, mode):
+    P = k.shape[2]
+    allp = np.arange(O.pages_of(L, P))
+    out, _, w = O.attend_head(k, v, pt, L, h, q, scale, mode, allp, want_weights=True)
+    tok_page = np.concatenate([[j] * min(P, L - j * P) for j in allp])
+    support = sorted(set(tok_page[np.any(w > 0, axis=0)]))
+    return out, w, support, tok_page
+
+
+@pytest.mark.parametrize("mode", [O.ENTMAX15, O.SPARSEMAX])
+def test_support_superset_gives_the_full_cache_output(mode):
+    # §3 support recovery: if the kept pages contain the whole entmax support, delta = 0 and
+    # the sparse output equals the full-cache output.
+    rng = np.random.default_rng(15)
+    for trial in range(10):
+        k, v, pt = make_seq(rng, L=int(rng.integers(20, 160)), nb=24, dist_scale=3.0)
+        L = int(rng.integers(20, 160))
+        pt = rng.permutation(24)[:O.pages_of(L, 8)].astype(np.int32)
+        q = rng.standard_normal((2, 16))
+        full, _, support, _ = full_support_pages(k, v, pt, L, 1, q, 0.7, mode)
+        n = O.pages_of(L, 8)
+        extra = rng.choice(n, size=int(rng.integers(0, n)), replace=False)
+        keep = np.array(sorted(set(support) | set(extra.tolist())), dtype=np.int32)
+        out, _, _ = O.attend_head(k, v, pt, L, 1, q, 0.7, mode, keep)
+        np.testing.assert_allclose(out, full, atol=1e-12)
+        if len(keep) < n and len(support) > 0:
+            # dropping a support page changes the output
+            drop = np.array([j for j in keep if j != support[0]], dtype=np.int32)
+            o2, _, _ = O.attend_head(k, v, pt, L, 1, q, 0.7, mode, drop)
+            assert np.abs(o2 - full).max() > 0
+
+
+@pytest.mark.parametrize("mode", [O.SOFTMAX, O.ENTMAX15, O.SPARSEMAX])
+def test_error_bound_two_B_delta(mode):
+    # §3: ||o - o_sparse|| <= 2 B delta, B = max ||v_i||, delta = full-cache mass of the
+    # dropped tokens.
+    rng = np.random.default_rng(16)
+    for trial in range(20):
+        L = int(rng.integers(9, 120))
+        k, v, pt = make_seq(rng, L=L, nb=16, dist_scale=float(rng.choice([0.5, 2.0])))
+        pt = rng.permutation(16)[:O.pages_of(L, 8)].astype(np.int32)
+        q = rng.standard_normal((2, 16))
+        full, w, _, tok_page = full_support_pages(k, v, pt, L, 0, q, 0.5, mode)
+        n = O.pages_of(L, 8)
+        keep = np.sort(rng.choice(n, size=int(rng.integers(1, n + 1)), replace=False))
+        out, _, _ = O.attend_head(k, v, pt, L, 0, q, 0.5, mode, keep.astype(np.int32))
+        B = np.linalg.norm(dense_tokens(v, pt, L, 0), axis=1).max()
+        kept_tok = np.isin(tok_page, keep)
+        for g in range(2):
+            delta = w[g, ~kept_tok].sum()
+            err = np.linalg.norm(out[g] - full[g])
+            assert err <= 2 * B * delta + 1e-12
+
+
+def test_entmax_drops_less_mass_than_softmax_on_needle_heads():
+    # §3/§4 comparison, on a planted-needle head: for the same kept set (the needle pages)
+    # the entmax full-cache mass outside it is below softmax's.
+    rng = np.random.default_rng(17)
+    P, d, nb, L = 16, 64, 64, 1024
+    k = rng.standard_normal((nb, 1, P, d)).astype(np.float32)
+    v = rng.standard_normal((nb, 1, P, d)).astype(np.float32)
+    pt = np.arange(nb, dtype=np.int32)
+    q = rng.standard_normal((1, d)) / 8
+    qh = q[0] / np.linalg.norm(q[0])
+    for blk in [3, 17, 40]:
+        k[blk, 0, 5] = (math.sqrt(d) * qh).astype(np.float32)
+    keep = np.array([3, 17, 40], np.int32)
+    masses = {}
+    for mode in [O.SOFTMAX, O.ENTMAX15]:
+        _, w, _, tok_page = full_support_pages(k, v, pt, L, 0, q, 1.0, mode)
+        masses[mode] = w[0, ~np.isin(tok_page, keep)].sum()
+    assert masses[O.ENTMAX15] < masses[O.SOFTMAX]
+
+
+def test_empty_selection():
+    rng = np.random.default_rng(18)
+    k, v, pt = make_seq(rng)
+    out, stat, _ = O.attend_head(k, v, pt, 61, 0, rng.standard_normal((2, 16)), 1.0,
+                                 O.ENTMAX15, np.zeros(0, np.int32))
+    assert np.all(out == 0) and np.all(np.isneginf(stat))
+
+
+def test_partial_last_page_only_reads_valid_tokens():
+    # Tokens at positions >= seq_len must not count: poison them and compare.
+    rng = np.random.default_rng(19)
+    k, v, pt = make_seq(rng, L=61)
+    q = rng.standard_normal((2, 16))
+    sel = np.arange(8, dtype=np.int32)
+    a = O.attend_head(k, v, pt, 61, 0, q, 1.0, O.SOFTMAX, sel)[0]
+    k2, v2 = k.copy(), v.copy()
+    k2[pt[7], 0, 5:] = 1e6
+    v2[pt[7], 0, 5:] = 1e6
+    b = O.attend_head(k2, v2, pt, 61, 0, q, 1.0, O.SOFTMAX, sel)[0]
+    np.testing.assert_array_equal(a, b)
+    m1 = O.page_meta_head(k, pt, 61, 0)
+    m2 = O.page_meta_head(k2, pt, 61, 0)
+    for x, y in zip(m1, m2):
+        np.testing.assert_array_equal(x, y)
