@@ -1,0 +1,185 @@
+/*
+ * ekv.h -- C ABI of libekv: query-aware sparse decode attention over a paged KV cache on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The method ("EntmaxKV: support-aware decoding for alpha-entmax attention", technical
+ * summary on gist.science): the KV cache is split into pages (§2); per-page key metadata --
+ * a coordinate-wise kmin/kmax bounding box and the key mean/variance -- is kept up to date as
+ * pages fill (§2.A); each decode step scores every page with a query-aware bound before any
+ * key or value is loaded (§2.A), selects candidate pages either as a fixed top-k budget
+ * (§2.B.1) or as the pages whose estimated maximum score clears a Gaussian-estimated entmax
+ * threshold tau-hat less a margin Delta (§2.B.2), and runs exact alpha-entmax (or softmax)
+ * attention over only those pages (§2.C).
+ *
+ * Conventions shared by every call
+ *  - All pointers are caller-owned DEVICE memory, except `c` itself (a host struct) and the
+ *    host outputs of ekv_device_status. The library never allocates or frees memory.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the legacy default
+ *    stream) and returns an ekv_status. Only ekv_device_status synchronises.
+ *  - Host-side validation failures return before any launch and leave every output
+ *    untouched. Supported shapes: head_dim d in {64, 128}; page size P in {16, 32, 64};
+ *    K/V/q/bbox dtype fp32 or bf16; num_q_heads a multiple of num_kv_heads with group size
+ *    G = num_q_heads / num_kv_heads in {1, 2, 4, 8}.
+ *  - Device-side bad input (a page-table entry outside [0, num_blocks), a sequence length
+ *    outside [0, max_pages * P], a selected page outside the sequence, ...) never traps:
+ *    the offending page is skipped and an EKV_DEV_* bit is OR-ed into *c->dev_status.
+ *    Read it with ekv_device_status.
+ *  - Logits are s = scale * q.k. The alpha-entmax weights are p_i = [z_i - tau]_+^(1/(alpha-1))
+ *    with z = (alpha - 1) s and sum_i p_i = 1 (alpha = 1.5 or alpha = 2, sparsemax).
+ *  - Page j of sequence b holds tokens j*P .. j*P+P-1; only tokens t < seq_lens[b] exist, so
+ *    the last page of a sequence may be partly filled. Pages j >= ceil(seq_lens[b] / P) do
+ *    not exist.
+ */
+#ifndef EKV_H
+#define EKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    EKV_OK = 0,
+    EKV_ERR_INVALID_ARG = 1, /* a null pointer, a negative size, a size mismatch         */
+    EKV_ERR_UNSUPPORTED = 2, /* a shape / dtype / mode outside the supported set          */
+    EKV_ERR_WORKSPACE = 3,   /* workspace smaller than ekv_decode_workspace_bytes()        */
+    EKV_ERR_CUDA = 4,        /* a CUDA launch or copy failed                              */
+    EKV_ERR_DEVICE = 5       /* ekv_device_status: a kernel flagged bad input             */
+} ekv_status;
+
+typedef enum { EKV_F32 = 0, EKV_BF16 = 1 } ekv_dtype;
+
+/* attention over the selected pages (§2.C); alpha = 1, 1.5, 2 */
+typedef enum { EKV_SOFTMAX = 0, EKV_ENTMAX15 = 1, EKV_SPARSEMAX = 2 } ekv_attn;
+
+/* candidate selection policy (§2.B) */
+typedef enum { EKV_SEL_TOPK = 0, EKV_SEL_GAUSS = 1 } ekv_policy;
+
+/* bits OR-ed into *dev_status by kernels that meet bad input */
+#define EKV_DEV_BAD_BLOCK 0x1u    /* page-table entry outside [0, num_blocks)            */
+#define EKV_DEV_BAD_LEN 0x2u      /* seq_lens[b] outside [0, max_pages * P]               */
+#define EKV_DEV_BAD_SEL 0x4u      /* selected page outside [0, ceil(seq_len / P))         */
+#define EKV_DEV_SEL_OVERFLOW 0x8u /* Gaussian policy kept more than max_sel pages         */
+#define EKV_DEV_BAD_RANGE 0x10u   /* meta update range outside [0, seq_len] or > max_new   */
+
+/*
+ * The paged cache and its metadata (§2, §2.A). Plain data; every pointer is device memory.
+ *   k_cache, v_cache  [num_blocks][H_kv][P][d] in `dtype`: one (block, head) is P*d
+ *                     contiguous elements, so a page of one KV head is one contiguous span.
+ *   meta_bbox         [num_blocks][H_kv][2][d] in `dtype`: row 0 kmin, row 1 kmax of the
+ *                     page's valid keys (exact: min/max of stored values).
+ *   meta_mom          [num_blocks][H_kv][2][d] fp32: row 0 mean, row 1 population variance of
+ *                     the page's valid keys. NULL is allowed unless EKV_SEL_GAUSS is used.
+ *   page_table        [batch][max_pages] int32: logical page j of sequence b is block
+ *                     page_table[b * max_pages + j].
+ *   seq_lens          [batch] int32: tokens in each sequence.
+ *   dev_status        one uint32 word of device memory; kernels OR EKV_DEV_* bits into it.
+ */
+typedef struct {
+    int32_t dtype;        /* ekv_dtype of K, V, q and meta_bbox       */
+    int32_t head_dim;     /* d                                        */
+    int32_t page_size;    /* P                                        */
+    int32_t num_kv_heads; /* H_kv                                     */
+    int32_t num_blocks;   /* physical blocks in the pool              */
+    int32_t batch;        /* B                                        */
+    int32_t max_pages;    /* row length of page_table                 */
+    int32_t reserved;     /* must be 0                                */
+    void *k_cache;
+    void *v_cache;
+    void *meta_bbox;
+    float *meta_mom;
+    const int32_t *page_table;
+    const int32_t *seq_lens;
+    uint32_t *dev_status;
+} ekv_cache;
+
+/*
+ * §2.A "metadata kept up to date as pages fill": recompute kmin/kmax (and, when meta_mom is
+ * not NULL, mean and population variance) of every page touched by the token range
+ * [new_start[b], new_start[b] + new_count[b]) of each sequence b, from all of that page's
+ * valid tokens (t < seq_lens[b]; seq_lens must already count the new tokens).
+ *   new_start, new_count  [batch] int32 device arrays (they stay on the device so a decode
+ *                         loop never synchronises). new_count[b] = 0 touches nothing.
+ *   max_new               host upper bound on every new_count[b]; sizes the launch. A range
+ *                         longer than max_new, or outside [0, seq_lens[b]], is clamped and
+ *                         flagged EKV_DEV_BAD_RANGE.
+ * Prefill: new_start = 0, new_count = seq_lens, max_new = max(seq_lens).
+ */
+ekv_status ekv_page_meta_update(const ekv_cache *c, const int32_t *new_start,
+                                const int32_t *new_count, int32_t max_new, void *stream);
+
+/*
+ * §2.A query-aware page scores, computed from the metadata only.
+ *   q       [batch][num_q_heads][d] in c->dtype; query head hq belongs to KV head hq / G.
+ *   scale   logit scale (> 0): s = scale * q.k.
+ *   policy  EKV_SEL_TOPK: scores is [batch][H_kv][max_pages] fp32 and holds the group bound
+ *             S_j = sum_{g in group} UB_{g,j},  UB_{g,j} = scale * sum_c max(q_gc kmin_jc, q_gc kmax_jc).
+ *           EKV_SEL_GAUSS: scores is [batch][num_q_heads][3][max_pages] fp32 and holds, per
+ *             query, UB_{g,j}, m_{g,j} = scale * q_g.mean_j and
+ *             v_{g,j} = scale^2 * sum_c q_gc^2 var_jc (needs c->meta_mom).
+ * Entries for pages j >= ceil(seq_lens[b] / P) are not written. A page whose page-table entry
+ * is out of range scores -inf (and m = v = 0) and is flagged.
+ */
+ekv_status ekv_score_pages(const ekv_cache *c, const void *q, int32_t num_q_heads, float scale,
+                           int32_t policy, float *scores, void *stream);
+
+/*
+ * §2.B candidate selection, per (sequence, KV head).
+ *   EKV_SEL_TOPK (§2.B.1): the min(topk, n_pages) pages with the largest S_j; equal scores go
+ *     to the lower page index. alpha, delta, tau_hat are ignored (tau_hat may be NULL).
+ *     Requires max_sel >= min(topk, max_pages).
+ *   EKV_SEL_GAUSS (§2.B.2): per query g, tau_hat_g solves
+ *       sum_j n_j E[((alpha-1) s - tau)_+^(1/(alpha-1))] = 1,  s ~ N(m_{g,j}, v_{g,j}),
+ *     n_j the valid tokens of page j (alpha in {1.5, 2}); page j is kept iff some query g of
+ *     the group has (alpha-1) * UB_{g,j} > tau_hat_g - delta. tau_hat: [batch][num_q_heads]
+ *     fp32 output (-inf for an empty sequence). More than max_sel kept pages: the first
+ *     max_sel (ascending) are emitted, sel_count holds max_sel, EKV_DEV_SEL_OVERFLOW is set.
+ *   scores     as written by ekv_score_pages with the same policy.
+ *   sel_idx    [batch][H_kv][max_sel] int32 output: logical page indices, ascending, then -1.
+ *   sel_count  [batch][H_kv] int32 output.
+ */
+ekv_status ekv_select_pages(const ekv_cache *c, int32_t num_q_heads, int32_t policy,
+                            int32_t topk, float alpha, float delta, const float *scores,
+                            int32_t *sel_idx, int32_t *sel_count, int32_t max_sel,
+                            float *tau_hat, void *stream);
+
+/*
+ * §2.C attention over the selected pages only, read in place from the paged cache (no gather
+ * copy). For each query head: s_i = scale * q.k_i over the valid tokens of the pages of its
+ * KV head listed in sel_idx[b][h][0 .. min(sel_count, max_sel));
+ *   EKV_SOFTMAX:   p = softmax(s);                        stat = log sum_i exp(s_i)
+ *   EKV_ENTMAX15, EKV_SPARSEMAX: z = (alpha-1) s, exact tau with sum_i [z_i - tau]_+^(1/(alpha-1)) = 1,
+ *                  p_i = [z_i - tau]_+^(1/(alpha-1));    stat = tau
+ *   out[b][hq][:] = sum_i p_i v_i (fp32);  an empty selection gives out = 0, stat = -inf.
+ *   q          [batch][num_q_heads][d] in c->dtype.
+ *   out        [batch][num_q_heads][d] fp32.   stat [batch][num_q_heads] fp32.
+ *   ws         scratch of at least ekv_decode_workspace_bytes(c, num_q_heads, max_sel)
+ *              bytes. It must be zero-filled once before its first use; every call leaves
+ *              it ready for the next. Calls that share one ws must not overlap on the GPU.
+ */
+ekv_status ekv_sparse_decode(const ekv_cache *c, const void *q, int32_t num_q_heads,
+                             float scale, int32_t attn, const int32_t *sel_idx,
+                             const int32_t *sel_count, int32_t max_sel, float *out, float *stat,
+                             void *ws, size_t ws_bytes, void *stream);
+
+/* Scratch bytes ekv_sparse_decode needs for this cache geometry, num_q_heads and max_sel
+ * (0 on invalid arguments). */
+size_t ekv_decode_workspace_bytes(const ekv_cache *c, int32_t num_q_heads, int32_t max_sel);
+
+/* Synchronise `stream`, copy *c->dev_status to *bits (host pointer, may be NULL) and return
+ * EKV_ERR_DEVICE if any bit is set, else EKV_OK (EKV_ERR_CUDA if the copy fails). */
+ekv_status ekv_device_status(const ekv_cache *c, uint32_t *bits, void *stream);
+
+/* Clear *c->dev_status (asynchronous). */
+ekv_status ekv_clear_device_status(const ekv_cache *c, void *stream);
+
+/* A static, human-readable name for a status code. */
+const char *ekv_status_str(ekv_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EKV_H */

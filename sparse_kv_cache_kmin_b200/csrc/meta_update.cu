@@ -1,0 +1,103 @@
+// meta_update.cu -- per-page key metadata upkeep (EntmaxKV technical summary, §2.A: the
+// bounding box kmin/kmax and the Gaussian statistics mean/variance of each page's keys,
+// kept up to date as pages fill).
+//
+// One warp per (touched page, KV head). A warp reads the page's valid key rows of its head
+// (P rows of d elements, contiguous in the [block][head][P][d] layout) with lane l owning
+// coordinates [l * d/32, (l+1) * d/32): min, max and sum in one pass, then the squared
+// deviations from the fp32 mean in a second pass over the same rows (two-pass variance; the
+// rows are still in L1/L2). kmin/kmax are stored in the cache dtype (exact: they are stored
+// values); mean and population variance in fp32.
+#include "ekv_device.cuh"
+
+namespace ekv {
+
+template <int DT, int D>
+__global__ void __launch_bounds__(256)
+page_meta_update_kernel(ekv_cache c, const int32_t *__restrict__ new_start,
+                        const int32_t *__restrict__ new_count, int max_new)
+{
+    pdl_wait();
+    constexpr int VEC = D / 32;
+    const int lane = threadIdx.x & 31;
+    const int h = blockIdx.z * 8 + (threadIdx.x >> 5);
+    const int b = blockIdx.y;
+    const int P = c.page_size;
+    if (h >= c.num_kv_heads) return;
+
+    int len;
+    seq_pages(c.seq_lens, b, P, c.max_pages, c.dev_status, &len);
+    int s = new_start[b], n = new_count[b];
+    if (n <= 0) return;
+    if (s < 0 || s + n > len || n > max_new) {
+        if (blockIdx.x == 0 && threadIdx.x == 0) flag(c.dev_status, EKV_DEV_BAD_RANGE);
+        s = s < 0 ? 0 : (s > len ? len : s);
+        int e = s + n > len ? len : s + n;
+        n = e - s > max_new ? max_new : e - s;
+        if (n <= 0) return;
+    }
+    const int p = s / P + blockIdx.x;
+    if (p > (s + n - 1) / P) return;
+    const int blk = c.page_table[(size_t)b * c.max_pages + p];
+    if (blk < 0 || blk >= c.num_blocks) {
+        if (lane == 0) flag(c.dev_status, EKV_DEV_BAD_BLOCK);
+        return;
+    }
+    const int cnt = len - p * P < P ? len - p * P : P;
+    const size_t row0 = ((size_t)blk * c.num_kv_heads + h) * P;
+
+    float mn[VEC], mx[VEC], sum[VEC];
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) { mn[e] = INFINITY; mx[e] = -INFINITY; sum[e] = 0.f; }
+    for (int t = 0; t < cnt; ++t) {
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) {
+            float x = load_elem<DT>(c.k_cache, (row0 + t) * D + lane * VEC + e);
+            mn[e] = fminf(mn[e], x);
+            mx[e] = fmaxf(mx[e], x);
+            sum[e] += x;
+        }
+    }
+    const size_t mbase = ((size_t)blk * c.num_kv_heads + h) * 2 * D;
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) {
+        store_exact<DT>(c.meta_bbox, mbase + lane * VEC + e, mn[e]);
+        store_exact<DT>(c.meta_bbox, mbase + D + lane * VEC + e, mx[e]);
+    }
+    if (c.meta_mom) {
+        float mean[VEC], ss[VEC];
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) { mean[e] = sum[e] / (float)cnt; ss[e] = 0.f; }
+        for (int t = 0; t < cnt; ++t) {
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) {
+                float x = load_elem<DT>(c.k_cache, (row0 + t) * D + lane * VEC + e) - mean[e];
+                ss[e] = fmaf(x, x, ss[e]);
+            }
+        }
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) {
+            c.meta_mom[mbase + lane * VEC + e] = mean[e];
+            c.meta_mom[mbase + D + lane * VEC + e] = ss[e] / (float)cnt;
+        }
+    }
+}
+
+cudaError_t launch_page_meta_update(const ekv_cache &c, const int32_t *new_start,
+                                    const int32_t *new_count, int max_new, cudaStream_t st)
+{
+    // A range of max_new tokens starting anywhere touches at most ceil(max_new / P) + 1 pages.
+    const int P = c.page_size;
+    dim3 grid((max_new + P - 1) / P + 1, c.batch, (c.num_kv_heads + 7) / 8);
+    if (max_new == 0) return cudaSuccess;
+#define EKV_META(DT, D) page_meta_update_kernel<DT, D><<<grid, 256, 0, st>>>(c, new_start, new_count, max_new)
+    if (c.dtype == EKV_BF16) {
+        if (c.head_dim == 128) EKV_META(EKV_BF16, 128); else EKV_META(EKV_BF16, 64);
+    } else {
+        if (c.head_dim == 128) EKV_META(EKV_F32, 128); else EKV_META(EKV_F32, 64);
+    }
+#undef EKV_META
+    return cudaGetLastError();
+}
+
+}  // namespace ekv

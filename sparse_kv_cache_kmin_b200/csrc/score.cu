@@ -1,0 +1,299 @@
+// score.cu -- query-aware page scoring from the page metadata only (EntmaxKV technical
+// summary, §2.A), before any key or value is read.
+//
+// Top-k policy: the group bound S_j = sum_g scale * sum_c max(q_gc kmin_jc, q_gc kmax_jc).
+// Because kmin <= kmax coordinate-wise, max(q kmin, q kmax) = q+ kmax + q- kmin with
+// q+ = max(q, 0), q- = min(q, 0); summed over the group this is
+//     S_j = scale * (Q+ . kmax_j + Q- . kmin_j),   Q+- = sum_g q_g+-,
+// two FMAs per coordinate per page whatever the group size: the scan is bound by HBM.
+//
+// Layout and traffic: a page's bbox row for one KV head is 2*d contiguous elements (512 B for
+// bf16 d=128). A warp streams whole rows with 16-byte loads (lane l owns the l-th 16 bytes,
+// i.e. eight kmin or eight kmax coordinates, and holds the matching eight Q- or Q+
+// coefficients in registers), eight pages per step so that each lane has eight independent
+// loads in flight, then a transposing butterfly reduces the eight per-page partial dots in
+// nine shuffles. The grid is persistent (a few CTAs per SM); the flattened work list of
+// (sequence, KV head, 8-page group) is split evenly over CTAs, so ragged batches balance.
+//
+// Gaussian policy: per query, UB_gj (as above but unsummed), m_gj = scale * q_g . mean_j and
+// v_gj = scale^2 * sum_c q_gc^2 var_jc; each page reads its bbox row and its fp32 moment row.
+#include "ekv_device.cuh"
+
+namespace ekv {
+
+// Prefix over sequences of the work groups each contributes: H_kv * ceil(n_pages / PG).
+template <int PG>
+__device__ __forceinline__ int build_group_prefix(const ekv_cache &c, int *pre, int *warp_tot)
+{
+    const int B = c.batch;
+    int run = 0;
+    for (int b0 = 0; b0 < B; b0 += 256) {
+        const int b = b0 + (int)threadIdx.x;
+        int v = 0;
+        if (b < B) {
+            int np = seq_pages(c.seq_lens, b, c.page_size, c.max_pages,
+                               blockIdx.x == 0 ? c.dev_status : nullptr, nullptr);
+            v = c.num_kv_heads * ((np + PG - 1) / PG);
+        }
+        int tot;
+        int incl = block_incl_scan<256>(v, warp_tot, &tot);
+        if (b < B) pre[b] = run + incl - v;
+        run += tot;
+    }
+    if (threadIdx.x == 0) pre[B] = run;
+    __syncthreads();
+    return run;
+}
+
+// Largest b with pre[b] <= gi (pre non-decreasing, pre[0] = 0 <= gi < pre[B]).
+__device__ __forceinline__ int find_seq(const int *pre, int B, long gi)
+{
+    int lo = 0, hi = B;
+    while (hi - lo > 1) {
+        int mid = (lo + hi) >> 1;
+        if (pre[mid] <= gi) lo = mid; else hi = mid;
+    }
+    return lo;
+}
+
+template <int DT, int D, int G>
+__global__ void __launch_bounds__(256)
+score_topk_kernel(ekv_cache c, const void *__restrict__ q, int H_q, float scale,
+                  float *__restrict__ scores)
+{
+    extern __shared__ int pre[];  // [B + 1]
+    __shared__ int warp_tot[8];
+    constexpr int EPC = Chunk<DT>::N;
+    constexpr int CPR = 2 * D * Chunk<DT>::kBytes / 16;  // 16-byte chunks per bbox row
+    constexpr int W = CPR < 32 ? CPR : 32;                 // lanes per row
+    constexpr int LPL = CPR / W;                           // chunks per lane per row
+    constexpr int RPI = 32 / W;                            // rows per warp instruction
+    constexpr int PG = 8;                                  // pages per work group
+    constexpr int NPL = PG / RPI;                          // page slots per lane
+    static_assert(NPL <= W, "one result per lane group");
+
+    pdl_wait();
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int H = c.num_kv_heads, B = c.batch, P = c.page_size;
+    const long TG = build_group_prefix<PG>(c, pre, warp_tot);
+    const long lo = (long)blockIdx.x * TG / gridDim.x;
+    const long hi = (long)(blockIdx.x + 1) * TG / gridDim.x;
+    const char *bbox = static_cast<const char *>(c.meta_bbox);
+
+    int cur_bh = -1, np = 0, bb = 0, hh = 0;
+    float coef[LPL][EPC];
+    for (long gi = lo + warp; gi < hi; gi += 8) {
+        bb = find_seq(pre, B, gi);
+        int len = c.seq_lens[bb];
+        len = len < 0 ? 0 : (len > c.max_pages * P ? c.max_pages * P : len);
+        np = (len + P - 1) / P;
+        const int ng = (np + PG - 1) / PG;
+        const int r = (int)(gi - pre[bb]);
+        hh = r / ng;
+        const int j0 = (r % ng) * PG;
+        const int bh = bb * H + hh;
+        if (bh != cur_bh) {
+            cur_bh = bh;
+#pragma unroll
+            for (int k = 0; k < LPL; ++k) {
+                const int ci = k * W + lane % W;
+                const bool upper = ci >= CPR / 2;
+                const int cb = (ci % (CPR / 2)) * EPC;
+#pragma unroll
+                for (int e = 0; e < EPC; ++e) {
+                    float a = 0.f;
+#pragma unroll
+                    for (int g = 0; g < G; ++g) {
+                        float qv = load_elem<DT>(q, ((size_t)bb * H_q + hh * G + g) * D + cb + e);
+                        a += upper ? fmaxf(qv, 0.f) : fminf(qv, 0.f);
+                    }
+                    coef[k][e] = a;
+                }
+            }
+        }
+        // block id of page j0 + (lane & 7): -1 past the end, -2 out of range
+        int myblk = -1;
+        const int jl = j0 + (lane & (PG - 1));
+        if (jl < np) {
+            myblk = c.page_table[(size_t)bb * c.max_pages + jl];
+            if (myblk < 0 || myblk >= c.num_blocks) {
+                flag(c.dev_status, EKV_DEV_BAD_BLOCK);
+                myblk = -2;
+            }
+        }
+        uint4 x[NPL][LPL];
+#pragma unroll
+        for (int i = 0; i < NPL; ++i) {
+            const int blk = __shfl_sync(kFull, myblk, i * RPI + lane / W);
+#pragma unroll
+            for (int k = 0; k < LPL; ++k) {
+                if (blk >= 0)
+                    x[i][k] = ld_stream16(bbox + (((size_t)blk * H + hh) * CPR + k * W + lane % W) * 16);
+                else
+                    x[i][k] = make_uint4(0, 0, 0, 0);
+            }
+        }
+        float part[NPL];
+#pragma unroll
+        for (int i = 0; i < NPL; ++i) {
+            part[i] = 0.f;
+#pragma unroll
+            for (int k = 0; k < LPL; ++k) {
+                float f[EPC];
+                Chunk<DT>::unpack(x[i][k], f);
+#pragma unroll
+                for (int e = 0; e < EPC; ++e) part[i] = fmaf(coef[k][e], f[e], part[i]);
+            }
+        }
+        transpose_reduce<NPL, W>(part, lane);
+        const int po = transpose_index<NPL, W>(lane, 0) * RPI + lane / W;
+        const int blk = __shfl_sync(kFull, myblk, po);
+        if (((lane % W) % (W / NPL)) == 0 && j0 + po < np)
+            scores[(size_t)bh * c.max_pages + j0 + po] = blk >= 0 ? scale * part[0] : -INFINITY;
+    }
+    pdl_trigger();
+}
+
+template <int DT, int D, int G>
+__global__ void __launch_bounds__(256)
+score_gauss_kernel(ekv_cache c, const void *__restrict__ q, int H_q, float scale,
+                   float *__restrict__ scores)
+{
+    // Lane l owns coordinates [l * VEC, (l + 1) * VEC) of all four metadata rows of a page
+    // (kmin, kmax, mean, variance), so the query coefficients it needs are just q_g there.
+    extern __shared__ int pre[];
+    __shared__ int warp_tot[8];
+    constexpr int VEC = D / 32;
+    constexpr int PGG = G >= 8 ? 1 : 8 / G;  // pages per work group
+    constexpr int NV = PGG * G;              // 8 values per output kind per lane
+
+    pdl_wait();
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int H = c.num_kv_heads, B = c.batch, P = c.page_size;
+    const long TG = build_group_prefix<PGG>(c, pre, warp_tot);
+    const long lo = (long)blockIdx.x * TG / gridDim.x;
+    const long hi = (long)(blockIdx.x + 1) * TG / gridDim.x;
+
+    int cur_bh = -1;
+    float qv[G][VEC];
+    for (long gi = lo + warp; gi < hi; gi += 8) {
+        const int bb = find_seq(pre, B, gi);
+        int len = c.seq_lens[bb];
+        len = len < 0 ? 0 : (len > c.max_pages * P ? c.max_pages * P : len);
+        const int np = (len + P - 1) / P;
+        const int ng = (np + PGG - 1) / PGG;
+        const int r = (int)(gi - pre[bb]);
+        const int hh = r / ng;
+        const int j0 = (r % ng) * PGG;
+        const int bh = bb * H + hh;
+        if (bh != cur_bh) {
+            cur_bh = bh;
+#pragma unroll
+            for (int g = 0; g < G; ++g)
+#pragma unroll
+                for (int e = 0; e < VEC; ++e)
+                    qv[g][e] = load_elem<DT>(q, ((size_t)bb * H_q + hh * G + g) * D + lane * VEC + e);
+        }
+        int myblk = -1;
+        const int jl = j0 + lane % PGG;
+        if (jl < np) {
+            myblk = c.page_table[(size_t)bb * c.max_pages + jl];
+            if (myblk < 0 || myblk >= c.num_blocks) {
+                flag(c.dev_status, EKV_DEV_BAD_BLOCK);
+                myblk = -2;
+            }
+        }
+        float kn[PGG][VEC], kx[PGG][VEC], mu[PGG][VEC], vr[PGG][VEC];
+#pragma unroll
+        for (int i = 0; i < PGG; ++i) {
+            const int blk = __shfl_sync(kFull, myblk, i);
+            const size_t base = ((size_t)(blk < 0 ? 0 : blk) * H + hh) * 2 * D + lane * VEC;
+            if (blk >= 0) {
+                load_vec_nc<DT, VEC>(static_cast<const char *>(c.meta_bbox) + base * Chunk<DT>::kBytes, kn[i]);
+                load_vec_nc<DT, VEC>(static_cast<const char *>(c.meta_bbox) + (base + D) * Chunk<DT>::kBytes, kx[i]);
+                load_vec_nc<EKV_F32, VEC>(c.meta_mom + base, mu[i]);
+                load_vec_nc<EKV_F32, VEC>(c.meta_mom + base + D, vr[i]);
+            } else {
+#pragma unroll
+                for (int e = 0; e < VEC; ++e) { kn[i][e] = 0.f; kx[i][e] = 0.f; mu[i][e] = 0.f; vr[i][e] = 0.f; }
+            }
+        }
+        float pu[NV], pm[NV], pv[NV];
+#pragma unroll
+        for (int i = 0; i < PGG; ++i)
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                float u = 0.f, m = 0.f, v = 0.f;
+#pragma unroll
+                for (int e = 0; e < VEC; ++e) {
+                    const float qe = qv[g][e];
+                    u += fmaxf(qe * kn[i][e], qe * kx[i][e]);
+                    m = fmaf(qe, mu[i][e], m);
+                    v = fmaf(qe * qe, vr[i][e], v);
+                }
+                pu[i * G + g] = u; pm[i * G + g] = m; pv[i * G + g] = v;
+            }
+        transpose_reduce<NV, 32>(pu, lane);
+        transpose_reduce<NV, 32>(pm, lane);
+        transpose_reduce<NV, 32>(pv, lane);
+        const int idx = transpose_index<NV, 32>(lane, 0);
+        const int i = idx / G, g = idx % G;
+        const int blk = __shfl_sync(kFull, myblk, i);
+        if ((lane & (32 / NV - 1)) == 0 && j0 + i < np) {
+            float *out = scores + ((size_t)bb * H_q + hh * G + g) * 3 * c.max_pages + j0 + i;
+            const bool ok = blk >= 0;
+            out[0] = ok ? scale * pu[0] : -INFINITY;
+            out[c.max_pages] = ok ? scale * pm[0] : 0.f;
+            out[2 * (size_t)c.max_pages] = ok ? scale * scale * pv[0] : 0.f;
+        }
+    }
+    pdl_trigger();
+}
+
+template <int DT, int D, int G>
+static cudaError_t launch_score_t(const ekv_cache &c, const void *q, int H_q, float scale,
+                                  int policy, float *scores, cudaStream_t st, bool pdl)
+{
+    const size_t smem = sizeof(int) * (c.batch + 1);
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    if (policy == EKV_SEL_TOPK) {
+        auto k = score_topk_kernel<DT, D, G>;
+        cfg.gridDim = dim3(persistent_grid_size((const void *)k, 256, smem));
+        return cudaLaunchKernelEx(&cfg, k, c, q, H_q, scale, scores);
+    }
+    auto k = score_gauss_kernel<DT, D, G>;
+    cfg.gridDim = dim3(persistent_grid_size((const void *)k, 256, smem));
+    return cudaLaunchKernelEx(&cfg, k, c, q, H_q, scale, scores);
+}
+
+template <int DT, int D>
+static cudaError_t launch_score_g(const ekv_cache &c, const void *q, int H_q, float scale,
+                                  int policy, float *scores, cudaStream_t st, bool pdl)
+{
+    switch (H_q / c.num_kv_heads) {
+    case 1: return launch_score_t<DT, D, 1>(c, q, H_q, scale, policy, scores, st, pdl);
+    case 2: return launch_score_t<DT, D, 2>(c, q, H_q, scale, policy, scores, st, pdl);
+    case 4: return launch_score_t<DT, D, 4>(c, q, H_q, scale, policy, scores, st, pdl);
+    default: return launch_score_t<DT, D, 8>(c, q, H_q, scale, policy, scores, st, pdl);
+    }
+}
+
+cudaError_t launch_score_pages(const ekv_cache &c, const void *q, int H_q, float scale,
+                               int policy, float *scores, cudaStream_t st, bool pdl)
+{
+    if (c.dtype == EKV_BF16)
+        return c.head_dim == 128 ? launch_score_g<EKV_BF16, 128>(c, q, H_q, scale, policy, scores, st, pdl)
+                                 : launch_score_g<EKV_BF16, 64>(c, q, H_q, scale, policy, scores, st, pdl);
+    return c.head_dim == 128 ? launch_score_g<EKV_F32, 128>(c, q, H_q, scale, policy, scores, st, pdl)
+                             : launch_score_g<EKV_F32, 64>(c, q, H_q, scale, policy, scores, st, pdl);
+}
+
+}  // namespace ekv

@@ -1,0 +1,301 @@
+// select.cu -- candidate page selection (EntmaxKV technical summary, §2.B).
+//
+// Top-k (§2.B.1), one 1024-thread CTA per (sequence, KV head): an exact radix select over
+// order-preserving 32-bit keys of the fp32 scores (11 + 11 + 10 bits; histograms with
+// warp-aggregated shared-memory increments, so a run of nearly equal scores does not serialise
+// on one counter) finds the k-th largest key T and how many keys equal to T are taken; a
+// block scan then emits the kept pages in ascending order, equal scores going to the lower
+// page index.
+//
+// Gaussian-aware (§2.B.2), one CTA per (sequence, KV head), one warp per query of the group:
+// tau-hat solves F(tau) = sum_j n_j E[(X_j - tau)_+^(1/(alpha-1))] = 1 with
+// X_j ~ N((alpha-1) m_j, (alpha-1)^2 v_j). F is convex and decreasing, so Newton's method
+// started at max_j a_j - 1 (where F >= 1 by Jensen) climbs monotonically to the root. Pages
+// with a_j + 8 b_j <= max_j a_j - 1 contribute less than 1e-16 n_j b_j^2 to F at every tau on
+// that path and are dropped before the iterations; the rest are kept in shared memory. Then a
+// block scan keeps page j iff some query g has (alpha-1) UB_gj > tau_hat_g - Delta.
+#include "ekv_device.cuh"
+
+namespace ekv {
+
+__device__ __forceinline__ uint32_t order_key(float x)
+{
+    if (x != x) return 0u;                  // NaN sorts below everything
+    uint32_t u = __float_as_uint(x + 0.0f);  // -0 -> +0
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__global__ void __launch_bounds__(1024)
+select_topk_kernel(const float *__restrict__ scores, int H, int max_pages, int P,
+                   const int32_t *__restrict__ seq_lens, int k, int32_t *__restrict__ sel_idx,
+                   int32_t *__restrict__ sel_count, int max_sel, uint32_t *status)
+{
+    constexpr int NT = 1024;
+    __shared__ int hist[2048];
+    __shared__ int warp_tot[32];
+    __shared__ int s_bin, s_above;
+    pdl_wait();
+    const int tid = threadIdx.x, lane = tid & 31;
+    const int h = blockIdx.x, b = blockIdx.y;
+    const int bh = b * H + h;
+    const int n = seq_pages(seq_lens, b, P, max_pages, h == 0 ? status : nullptr, nullptr);
+    const float *S = scores + (size_t)bh * max_pages;
+    int32_t *out = sel_idx + (size_t)bh * max_sel;
+    const int kk = k < n ? k : n;
+
+    if (kk == n) {  // every page is kept
+        for (int j = tid; j < max_sel; j += NT) out[j] = j < n ? j : -1;
+        if (tid == 0) sel_count[bh] = n;
+        pdl_trigger();
+        return;
+    }
+
+    uint32_t prefix = 0, mask = 0;
+    int remaining = kk;
+    const int shifts[3] = {21, 10, 0};
+    const int widths[3] = {11, 11, 10};
+#pragma unroll 1
+    for (int pass = 0; pass < 3; ++pass) {
+        const int shift = shifts[pass], nb = 1 << widths[pass];
+        for (int i = tid; i < 2048; i += NT) hist[i] = 0;
+        __syncthreads();
+        for (int j0 = 0; j0 < n; j0 += NT) {
+            const int j = j0 + tid;
+            int bin = -1;
+            if (j < n) {
+                const uint32_t u = order_key(S[j]);
+                if ((u & mask) == prefix) bin = (int)((u >> shift) & (uint32_t)(nb - 1));
+            }
+            const unsigned peers = __match_any_sync(kFull, bin);
+            if (bin >= 0 && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
+        }
+        __syncthreads();
+        // counts in descending bin order: thread t owns positions 2t and 2t+1
+        const int b0 = nb - 1 - 2 * tid, b1 = nb - 2 - 2 * tid;
+        const int c0 = b0 >= 0 ? hist[b0] : 0, c1 = b1 >= 0 ? hist[b1] : 0;
+        const int incl = block_incl_scan<NT>(c0 + c1, warp_tot, nullptr);
+        const int excl = incl - c0 - c1;
+        if (c0 > 0 && excl < remaining && remaining <= excl + c0) { s_bin = b0; s_above = excl; }
+        if (c1 > 0 && excl + c0 < remaining && remaining <= incl) { s_bin = b1; s_above = excl + c0; }
+        __syncthreads();
+        remaining -= s_above;
+        prefix |= (uint32_t)s_bin << shift;
+        mask |= (uint32_t)(nb - 1) << shift;
+        __syncthreads();
+    }
+    // prefix is now the k-th largest key T; `remaining` keys equal to T are kept (lowest
+    // page indices first).
+    const uint32_t T = prefix;
+    const int E = (n + NT - 1) / NT;
+    const int j0 = tid * E, j1 = j0 + E < n ? j0 + E : n;
+    int eq = 0;
+    for (int j = j0; j < j1; ++j) eq += order_key(S[j]) == T;
+    const int eq_before = block_incl_scan<NT>(eq, warp_tot, nullptr) - eq;
+    int mine = 0, seen = eq_before;
+    for (int j = j0; j < j1; ++j) {
+        const uint32_t u = order_key(S[j]);
+        if (u > T) ++mine;
+        else if (u == T && seen++ < remaining) ++mine;
+    }
+    int pos = block_incl_scan<NT>(mine, warp_tot, nullptr) - mine;
+    seen = eq_before;
+    for (int j = j0; j < j1; ++j) {
+        const uint32_t u = order_key(S[j]);
+        if (u > T || (u == T && seen++ < remaining)) out[pos++] = j;
+    }
+    for (int j = kk + tid; j < max_sel; j += NT) out[j] = -1;
+    if (tid == 0) sel_count[bh] = kk;
+    pdl_trigger();
+}
+
+// ---------------------------------------------------------------------------- Gaussian-aware
+// E[(X - tau)_+^p] for X ~ N(a, b^2), p = 1 (alpha = 2) or 2 (alpha = 1.5), and its
+// derivative in tau. Phi(u) = erfc(-u / sqrt 2) / 2, phi(u) = exp(-u^2 / 2) / sqrt(2 pi).
+__device__ __forceinline__ void trunc_moment(double a, double b, double tau, bool sparsemax,
+                                             double &E, double &dE)
+{
+    const double r = a - tau;
+    if (b <= 0.0) {
+        const double rp = r > 0.0 ? r : 0.0;
+        E = sparsemax ? rp : rp * rp;
+        dE = sparsemax ? (r > 0.0 ? -1.0 : 0.0) : -2.0 * rp;
+        return;
+    }
+    const double u = r / b;
+    const double Phi = 0.5 * erfc(-u * 0.70710678118654752440);
+    const double phi = 0.39894228040143267794 * exp(-0.5 * u * u);
+    if (sparsemax) {
+        E = r * Phi + b * phi;
+        dE = -Phi;
+    } else {
+        E = (r * r + b * b) * Phi + r * b * phi;
+        dE = -2.0 * (r * Phi + b * phi);
+    }
+}
+
+template <int G>
+__global__ void __launch_bounds__(256)
+select_gauss_kernel(const float *__restrict__ scores, int H, int max_pages, int P,
+                    const int32_t *__restrict__ seq_lens, float alpha, float delta,
+                    int32_t *__restrict__ sel_idx, int32_t *__restrict__ sel_count, int max_sel,
+                    float *__restrict__ tau_hat, uint32_t *status)
+{
+    constexpr int NT = 256;
+    constexpr int CAP = 2048 / G;  // survivors kept in shared memory per query
+    __shared__ float s_a[G][CAP], s_b[G][CAP];
+    __shared__ int s_n[G][CAP];
+    __shared__ double s_tau[G];
+    __shared__ int warp_tot[8];
+    pdl_wait();
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int h = blockIdx.x, b = blockIdx.y, bh = b * H + h;
+    const int H_q = H * G;
+    int len;
+    const int n = seq_pages(seq_lens, b, P, max_pages, h == 0 ? status : nullptr, &len);
+    const bool sparsemax = alpha == 2.0f;
+    const double am1 = (double)alpha - 1.0;
+
+    if (warp < G) {
+        const int g = warp, hq = h * G + g;
+        const float *sc = scores + ((size_t)b * H_q + hq) * 3 * max_pages;
+        const float *m = sc + max_pages, *v = sc + 2 * (size_t)max_pages;
+        double amax = -INFINITY;
+        for (int j = lane; j < n; j += 32) amax = fmax(amax, am1 * (double)m[j]);
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) amax = fmax(amax, __shfl_xor_sync(kFull, amax, o));
+        double tau = amax - 1.0;
+        // survivors: pages that can still contribute at tau >= amax - 1
+        int cnt = 0;
+        for (int j0 = 0; j0 < n; j0 += 32) {
+            const int j = j0 + lane;
+            float aj = 0.f, bj = 0.f;
+            bool keep = false;
+            if (j < n) {
+                aj = (float)(am1 * (double)m[j]);
+                bj = (float)(am1 * sqrt(fmax((double)v[j], 0.0)));
+                keep = (double)aj + 8.0 * (double)bj > tau;
+            }
+            const unsigned bal = __ballot_sync(kFull, keep);
+            const int pos = cnt + __popc(bal & ((1u << lane) - 1u));
+            if (keep && pos < CAP) {
+                s_a[g][pos] = aj;
+                s_b[g][pos] = bj;
+                s_n[g][pos] = len - j * P < P ? len - j * P : P;
+            }
+            cnt += __popc(bal);
+        }
+        __syncwarp();
+        if (n == 0) {
+            tau = -INFINITY;
+        } else {
+#pragma unroll 1
+            for (int it = 0; it < 64; ++it) {
+                double F = 0.0, dF = 0.0;
+                if (cnt <= CAP) {
+                    for (int i = lane; i < cnt; i += 32) {
+                        double E, dE;
+                        trunc_moment(s_a[g][i], s_b[g][i], tau, sparsemax, E, dE);
+                        F += s_n[g][i] * E;
+                        dF += s_n[g][i] * dE;
+                    }
+                } else {  // too many survivors for shared memory: walk every page
+                    for (int j = lane; j < n; j += 32) {
+                        double E, dE;
+                        const double aj = (float)(am1 * (double)m[j]);
+                        const double bj = (float)(am1 * sqrt(fmax((double)v[j], 0.0)));
+                        trunc_moment(aj, bj, tau, sparsemax, E, dE);
+                        const int nj = len - j * P < P ? len - j * P : P;
+                        F += nj * E;
+                        dF += nj * dE;
+                    }
+                }
+                F = warp_sum(F);
+                dF = warp_sum(dF);
+                if (!(dF < 0.0)) break;
+                const double step = (F - 1.0) / -dF;
+                if (!(step > 1e-13 * fmax(1.0, fabs(tau)))) break;
+                tau += step;
+            }
+        }
+        if (lane == 0) {
+            s_tau[g] = tau;
+            tau_hat[(size_t)b * H_q + hq] = (float)tau;
+        }
+    }
+    __syncthreads();
+
+    // union over the group, ascending page order
+    const int E = (n + NT - 1) / NT;
+    const int j0 = tid * E, j1 = j0 + E < n ? j0 + E : n;
+    int mine = 0;
+    for (int j = j0; j < j1; ++j) {
+        bool keep = false;
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            const float ub = scores[((size_t)b * H_q + h * G + g) * 3 * max_pages + j];
+            keep |= am1 * (double)ub > s_tau[g] - (double)delta;
+        }
+        mine += keep;
+    }
+    int total;
+    int pos = block_incl_scan<NT>(mine, warp_tot, &total) - mine;
+    int32_t *out = sel_idx + (size_t)bh * max_sel;
+    for (int j = j0; j < j1 && pos < max_sel; ++j) {
+        bool keep = false;
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            const float ub = scores[((size_t)b * H_q + h * G + g) * 3 * max_pages + j];
+            keep |= am1 * (double)ub > s_tau[g] - (double)delta;
+        }
+        if (keep) out[pos++] = j;
+    }
+    for (int j = total + tid; j < max_sel; j += NT) out[j] = -1;
+    if (tid == 0) {
+        if (total > max_sel) flag(status, EKV_DEV_SEL_OVERFLOW);
+        sel_count[bh] = total < max_sel ? total : max_sel;
+    }
+    pdl_trigger();
+}
+
+static cudaLaunchConfig_t pdl_config(dim3 grid, dim3 block, cudaStream_t st, bool pdl,
+                                     cudaLaunchAttribute *attr)
+{
+    cudaLaunchConfig_t cfg = {};
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cfg;
+}
+
+cudaError_t launch_select_pages(const ekv_cache &c, int H_q, int policy, int topk, float alpha,
+                                float delta, const float *scores, int32_t *sel_idx,
+                                int32_t *sel_count, int max_sel, float *tau_hat, cudaStream_t st,
+                                bool pdl)
+{
+    cudaLaunchAttribute attr[1];
+    const dim3 grid(c.num_kv_heads, c.batch);
+    if (policy == EKV_SEL_TOPK) {
+        cudaLaunchConfig_t cfg = pdl_config(grid, dim3(1024), st, pdl, attr);
+        return cudaLaunchKernelEx(&cfg, select_topk_kernel, scores, c.num_kv_heads, c.max_pages,
+                                  c.page_size, c.seq_lens, topk, sel_idx, sel_count, max_sel,
+                                  c.dev_status);
+    }
+    cudaLaunchConfig_t cfg = pdl_config(grid, dim3(256), st, pdl, attr);
+#define EKV_GSEL(G)                                                                            \
+    cudaLaunchKernelEx(&cfg, select_gauss_kernel<G>, scores, c.num_kv_heads, c.max_pages,      \
+                       c.page_size, c.seq_lens, alpha, delta, sel_idx, sel_count, max_sel,     \
+                       tau_hat, c.dev_status)
+    switch (H_q / c.num_kv_heads) {
+    case 1: return EKV_GSEL(1);
+    case 2: return EKV_GSEL(2);
+    case 4: return EKV_GSEL(4);
+    default: return EKV_GSEL(8);
+    }
+#undef EKV_GSEL
+}
+
+}  // namespace ekv

@@ -1,0 +1,54 @@
+"""One decode step = [page metadata update] -> page scores -> page selection -> sparse attention.
+
+SparseDecoder owns the per-step device buffers (scores, selection, outputs, workspace) for a
+fixed cache geometry and policy, and issues the four libekv calls on one stream. It adds no
+computation of its own.
+"""
+from __future__ import annotations
+
+from typing import Optional
+
+import torch
+
+from . import ekv
+
+
+class SparseDecoder:
+    def __init__(self, cache: ekv.PagedKVCache, num_q_heads: int, policy: int, attn: int,
+                 topk: int = 0, alpha: float = 1.5, delta: float = 0.0, scale: float = 1.0,
+                 max_sel: Optional[int] = None):
+        self.cache, self.num_q_heads, self.policy, self.attn = cache, num_q_heads, policy, attn
+        self.topk, self.alpha, self.delta, self.scale = topk, alpha, delta, scale
+        B, H, P, d = cache.batch, cache.num_kv_heads, cache.page_size, cache.head_dim
+        mp = cache.max_pages
+        if max_sel is None:
+            max_sel = min(topk, mp) if policy == ekv.EKV_SEL_TOPK else mp
+        self.max_sel = max_sel
+        dev = cache.k_cache.device
+        if policy == ekv.EKV_SEL_TOPK:
+            self.scores = torch.empty((B, H, mp), dtype=torch.float32, device=dev)
+        else:
+            self.scores = torch.empty((B, num_q_heads, 3, mp), dtype=torch.float32, device=dev)
+        self.sel_idx = torch.empty((B, H, max_sel), dtype=torch.int32, device=dev)
+        self.sel_count = torch.empty((B, H), dtype=torch.int32, device=dev)
+        self.tau_hat = torch.empty((B, num_q_heads), dtype=torch.float32, device=dev)
+        self.out = torch.empty((B, num_q_heads, d), dtype=torch.float32, device=dev)
+        self.stat = torch.empty((B, num_q_heads), dtype=torch.float32, device=dev)
+        nbytes = ekv.ekv_decode_workspace_bytes(cache, num_q_heads, max_sel)
+        if nbytes == 0:
+            raise ValueError("unsupported decoder geometry")
+        self.ws = torch.empty((nbytes,), dtype=torch.uint8, device=dev)
+
+    def update_metadata(self, new_start: torch.Tensor, new_count: torch.Tensor, max_new: int,
+                        stream=None):
+        ekv.ekv_page_meta_update(self.cache, new_start, new_count, max_new, stream)
+
+    def step(self, q: torch.Tensor, stream=None):
+        c = self.cache
+        ekv.ekv_score_pages(c, q, self.num_q_heads, self.scale, self.policy, self.scores, stream)
+        ekv.ekv_select_pages(c, self.num_q_heads, self.policy, self.topk, self.alpha, self.delta,
+                             self.scores, self.sel_idx, self.sel_count, self.max_sel,
+                             self.tau_hat, stream)
+        ekv.ekv_sparse_decode(c, q, self.num_q_heads, self.scale, self.attn, self.sel_idx,
+                              self.sel_count, self.max_sel, self.out, self.stat, self.ws, stream)
+        return self.out, self.stat

@@ -1,0 +1,148 @@
+"""The C ABI without a GPU: the library loads, exports every entry point include/ekv.h
+declares, its struct layout matches the binding's, and host-side validation answers with the
+documented status codes before any launch."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ekv.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from sparse_kv_cache_kmin_b200 import build, ekv
+    build.build_library()
+    return ekv.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*(ekv_[a-z_0-9]+)\s*\(",
+                                 text, re.M)))
+
+
+def test_header_declares_the_four_calls_and_helpers():
+    names = declared_functions()
+    for n in ["ekv_page_meta_update", "ekv_score_pages", "ekv_select_pages", "ekv_sparse_decode",
+              "ekv_decode_workspace_bytes", "ekv_device_status", "ekv_clear_device_status",
+              "ekv_status_str"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    from sparse_kv_cache_kmin_b200 import build
+    out = subprocess.run(["nm", "-D", "--defined-only", build.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (ekv_\w+)", out))
+    for n in declared_functions():
+        assert n in exported, n
+        assert hasattr(lib, n)
+
+
+def test_struct_layout_matches_header(tmp_path):
+    from sparse_kv_cache_kmin_b200.ekv import EkvCacheStruct
+    src = tmp_path / "layout.c"
+    fields = [f for f, _ in EkvCacheStruct._fields_]
+    body = "".join('printf("%%s %%zu\\n", "%s", offsetof(ekv_cache, %s));' % (f, f) for f in fields)
+    src.write_text('#include <stdio.h>\n#include <stddef.h>\n#include "ekv.h"\nint main(void){%s'
+                   'printf("sizeof %%zu\\n", sizeof(ekv_cache));return 0;}\n' % body)
+    exe = tmp_path / "layout"
+    subprocess.check_call(["gcc", "-std=c11", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)])
+    got = dict(line.split() for line in subprocess.check_output([str(exe)], text=True).splitlines())
+    for f in fields:
+        assert int(got[f]) == getattr(EkvCacheStruct, f).offset, f
+    assert int(got["sizeof"]) == ctypes.sizeof(EkvCacheStruct)
+
+
+def test_status_strings(lib):
+    from sparse_kv_cache_kmin_b200 import ekv
+    assert lib.ekv_status_str(ekv.EKV_OK) == b"EKV_OK"
+    assert lib.ekv_status_str(ekv.EKV_ERR_WORKSPACE) == b"EKV_ERR_WORKSPACE"
+    assert lib.ekv_status_str(99) == b"EKV_UNKNOWN_STATUS"
+
+
+def fake_cache(**over):
+    """A struct with non-null placeholder pointers: host validation only reads sizes and
+    checks pointers for NULL, so no device memory is touched by the failing calls below."""
+    from sparse_kv_cache_kmin_b200.ekv import EkvCacheStruct
+    c = EkvCacheStruct()
+    c.dtype, c.head_dim, c.page_size, c.num_kv_heads = 1, 128, 16, 8
+    c.num_blocks, c.batch, c.max_pages, c.reserved = 1024, 4, 256, 0
+    for f in ["k_cache", "v_cache", "meta_bbox", "meta_mom", "page_table", "seq_lens", "dev_status"]:
+        setattr(c, f, 0x1000)
+    for k, v in over.items():
+        setattr(c, k, v)
+    return c
+
+
+@pytest.mark.parametrize("over,status", [
+    ({"head_dim": 96}, 2), ({"page_size": 8}, 2), ({"dtype": 7}, 2),
+    ({"num_kv_heads": 0}, 1), ({"k_cache": None}, 1), ({"dev_status": None}, 1),
+    ({"batch": 9000}, 2),
+])
+def test_score_validation(lib, over, status):
+    c = fake_cache(**over)
+    assert lib.ekv_score_pages(ctypes.byref(c), 0x1000, 32, 1.0, 0, 0x1000, None) == status
+
+
+def test_head_count_and_policy_validation(lib):
+    c = fake_cache()
+    assert lib.ekv_score_pages(ctypes.byref(c), 0x1000, 30, 1.0, 0, 0x1000, None) == 1   # H_q % H_kv
+    assert lib.ekv_score_pages(ctypes.byref(c), 0x1000, 8 * 16, 1.0, 0, 0x1000, None) == 2  # G = 16
+    assert lib.ekv_score_pages(ctypes.byref(c), 0x1000, 32, 0.0, 0, 0x1000, None) == 1   # scale
+    assert lib.ekv_score_pages(ctypes.byref(c), 0x1000, 32, 1.0, 5, 0x1000, None) == 2   # policy
+    c2 = fake_cache(meta_mom=None)
+    assert lib.ekv_score_pages(ctypes.byref(c2), 0x1000, 32, 1.0, 1, 0x1000, None) == 1  # gauss w/o moments
+
+
+def test_select_validation(lib):
+    c = fake_cache()
+    P = 0x1000
+    assert lib.ekv_select_pages(ctypes.byref(c), 32, 0, 0, 1.5, 0.1, P, P, P, 16, None, None) == 1
+    assert lib.ekv_select_pages(ctypes.byref(c), 32, 0, 64, 1.5, 0.1, P, P, P, 16, None, None) == 1
+    assert lib.ekv_select_pages(ctypes.byref(c), 32, 1, 0, 1.2, 0.1, P, P, P, 16, P, None) == 2
+    assert lib.ekv_select_pages(ctypes.byref(c), 32, 1, 0, 1.5, 0.1, P, P, P, 16, None, None) == 1
+
+
+def test_decode_validation_and_workspace(lib):
+    c = fake_cache()
+    P = 0x1000
+    need = lib.ekv_decode_workspace_bytes(ctypes.byref(c), 32, 256)
+    assert need > 0
+    # [B*H_q][NC][2] + [B*H_q][NC][D] + [B*H_q][NC*CP*P] floats, each 256-byte aligned
+    assert need >= 4 * 32 * 256 * 16 * 4
+    assert lib.ekv_decode_workspace_bytes(ctypes.byref(c), 30, 256) == 0
+    assert lib.ekv_sparse_decode(ctypes.byref(c), P, 32, 1.0, 1, P, P, 256, P, P, P, need - 1, None) == 3
+    assert lib.ekv_sparse_decode(ctypes.byref(c), P, 32, 1.0, 1, P, P, 256, P, P, None, need, None) == 3
+    assert lib.ekv_sparse_decode(ctypes.byref(c), P, 32, 1.0, 9, P, P, 256, P, P, P, need, None) == 2
+    c2 = fake_cache(v_cache=None)
+    assert lib.ekv_sparse_decode(ctypes.byref(c2), P, 32, 1.0, 1, P, P, 256, P, P, P, need, None) == 1
+
+
+def test_meta_update_validation(lib):
+    c = fake_cache()
+    assert lib.ekv_page_meta_update(ctypes.byref(c), None, 0x1000, 16, None) == 1
+    assert lib.ekv_page_meta_update(ctypes.byref(c), 0x1000, 0x1000, -1, None) == 1
+    assert lib.ekv_page_meta_update(ctypes.byref(c), 0x1000, 0x1000, 256 * 16 + 1, None) == 1
+
+
+def test_binding_refuses_host_tensors():
+    import torch
+    from sparse_kv_cache_kmin_b200 import ekv
+    with pytest.raises(ValueError):
+        ekv._ptr(torch.zeros(4))
+
+
+def test_product_path_does_not_import_the_oracle():
+    # The package must not reach the CPU oracle: no import of it anywhere in the product.
+    pkg = os.path.join(ROOT, "sparse_kv_cache_kmin_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert not re.search(r"^\s*(from|import)\s+oracle\b", text, re.M), f
+                assert "ekv_oracle" not in text, f

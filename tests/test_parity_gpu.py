@@ -1,0 +1,247 @@
+"""GPU parity: the CUDA path, called through the C ABI, against the CPU oracle on the same
+seeded inputs -- every stage (metadata, scores, selection, attention) of every (sequence, KV
+head) on small ragged cases that span several tiles, and sampled heads of the full-size
+workloads in the launch configuration the benchmark times."""
+import itertools
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from sparse_kv_cache_kmin_b200 import ekv
+from sparse_kv_cache_kmin_b200.workloads import GAUSS, TOPK, make, make_random
+from parity_utils import HostCopy, check_head, close, make_cache, prefill_metadata, run_gpu, widen
+
+pytestmark = pytest.mark.gpu
+
+ATTN = [ekv.EKV_SOFTMAX, ekv.EKV_ENTMAX15, ekv.EKV_SPARSEMAX]
+
+
+def assert_status_ok(cache):
+    st, bits = ekv.ekv_device_status(cache)
+    assert st == ekv.EKV_OK, hex(bits)
+
+
+TOPK_CASES = list(itertools.product([torch.float32, torch.bfloat16], [64, 128], [16, 32, 64],
+                                    [1, 2, 4, 8]))
+
+
+@pytest.mark.parametrize("dtype,d,P,G", TOPK_CASES,
+                         ids=["%s-d%d-P%d-G%d" % (str(t)[6:], d, P, G) for t, d, P, G in TOPK_CASES])
+def test_topk_small_ragged(cuda_device, dtype, d, P, G):
+    lens = (1000 + 7 * P, 517, 33, 2 * P)
+    wl = make_random(B=4, H_kv=2, G=G, d=d, P=P, lens=lens, dtype=dtype, device="cuda",
+                     seed=d + P + G, kv_scale=2.0, topk=9)
+    for attn in ATTN:
+        cache, dec = run_gpu(wl, attn)
+        assert_status_ok(cache)
+        for b in range(wl.batch):
+            for h in range(wl.num_kv_heads):
+                check_head(wl, cache, dec, b, h, attn)
+
+
+GAUSS_CASES = list(itertools.product([torch.float32, torch.bfloat16], [64, 128], [16, 32],
+                                     [1, 4, 8], [ekv.EKV_ENTMAX15, ekv.EKV_SPARSEMAX]))
+
+
+@pytest.mark.parametrize("dtype,d,P,G,attn", GAUSS_CASES,
+                         ids=["%s-d%d-P%d-G%d-a%d" % (str(t)[6:], d, P, G, a) for t, d, P, G, a in GAUSS_CASES])
+def test_gauss_small_ragged(cuda_device, dtype, d, P, G, attn):
+    lens = (3000 + 5, 700, 64 * 3 + 1)
+    alpha = 1.5 if attn == ekv.EKV_ENTMAX15 else 2.0
+    wl = make_random(B=3, H_kv=2, G=G, d=d, P=P, lens=lens, dtype=dtype, device="cuda",
+                     seed=100 + d + P + G, kv_scale=1.0, q_scale=0.6, policy=GAUSS, alpha=alpha,
+                     delta=0.1)
+    cache, dec = run_gpu(wl, attn)
+    assert_status_ok(cache)
+    for b in range(wl.batch):
+        for h in range(wl.num_kv_heads):
+            check_head(wl, cache, dec, b, h, attn)
+
+
+def test_multi_chunk_pages(cuda_device):
+    # enough selected pages that each (sequence, head) spans several multi-page chunks
+    wl = make_random(B=4, H_kv=8, G=4, d=128, P=16, lens=(8000, 8000 - 3, 4100, 8000),
+                     dtype=torch.bfloat16, device="cuda", seed=7, topk=200)
+    for attn in ATTN:
+        cache, dec = run_gpu(wl, attn)
+        assert_status_ok(cache)
+        for b, h in [(0, 0), (1, 7), (2, 3), (3, 5)]:
+            check_head(wl, cache, dec, b, h, attn)
+
+
+# ------------------------------------------------------------------ the five named workloads
+def test_tiny_full_and_support_invariant(cuda_device):
+    wl = make("tiny", device="cuda")
+    for attn in [ekv.EKV_SOFTMAX, ekv.EKV_ENTMAX15]:
+        cache, dec = run_gpu(wl, attn)
+        assert_status_ok(cache)
+        check_head(wl, cache, dec, 0, 0, attn)
+    # full-cache 1.5-entmax on the GPU (every page selected) against the oracle
+    n_pages = wl.max_pages
+    wl.topk = n_pages
+    cache, full = run_gpu(wl, ekv.EKV_ENTMAX15)
+    hc = HostCopy(wl, 0)
+    out_o, stat_o, w = O.attend_head(hc.k, hc.v, hc.pt, hc.L, 0, hc.q[0], 1.0, O.ENTMAX15,
+                                     np.arange(n_pages), want_weights=True)
+    close(full.out[0].double().cpu().numpy(), out_o, False)
+    # support invariant: a selection containing the full-cache support gives the same output
+    support = sorted(set((np.nonzero(w[0] > 0)[0] // wl.page_size).tolist()))
+    wl.topk = 32
+    _, sparse = run_gpu(wl, ekv.EKV_ENTMAX15)
+    sel = set(sparse.sel_idx[0, 0, :int(sparse.sel_count[0, 0])].cpu().numpy().tolist())
+    if set(support) <= sel:
+        close(sparse.out[0].double().cpu().numpy(), out_o, False)
+    # and by construction: select support pages plus others directly
+    keep = sorted(set(support) | set(range(0, n_pages, 11)))
+    sel_idx = torch.full((1, 1, len(keep)), -1, dtype=torch.int32, device="cuda")
+    sel_idx[0, 0] = torch.tensor(keep, dtype=torch.int32)
+    cnt = torch.tensor([[len(keep)]], dtype=torch.int32, device="cuda")
+    out = torch.empty((1, 1, 64), device="cuda")
+    stat = torch.empty((1, 1), device="cuda")
+    ws = torch.empty(ekv.ekv_decode_workspace_bytes(cache, 1, len(keep)), dtype=torch.uint8, device="cuda")
+    ekv.ekv_sparse_decode(cache, wl.q, 1, 1.0, ekv.EKV_ENTMAX15, sel_idx, cnt, len(keep), out, stat, ws)
+    torch.cuda.synchronize()
+    close(out[0].double().cpu().numpy(), out_o, False)
+
+
+@pytest.mark.parametrize("name,heads", [
+    ("gqa32k", [(0, 0), (3, 7)]),
+    ("needle128k", [(0, 0), (5, 3), (7, 7)]),
+    ("gauss", [(0, 0), (9, 4), (15, 7)]),
+    ("long1m", [(0, 0), (0, 5)]),
+])
+def test_named_workload_sampled_heads(cuda_device, name, heads):
+    wl = make(name, device="cuda")
+    cache = make_cache(wl)
+    prefill_metadata(cache, wl)
+    if wl.append is not None:  # the decode step appends the last page and refreshes its metadata
+        start, count = wl.append
+        st = torch.full((wl.batch,), start, dtype=torch.int32, device="cuda")
+        ct = torch.full((wl.batch,), count, dtype=torch.int32, device="cuda")
+        ekv.ekv_page_meta_update(cache, st, ct, count)
+    for attn in wl.attn_modes:
+        _, dec = run_gpu(wl, attn, cache=cache)
+        assert_status_ok(cache)
+        hcs = {}
+        for b, h in heads:
+            hc = hcs.setdefault(b, HostCopy(wl, b))
+            check_head(wl, cache, dec, b, h, attn, hc=hc)
+
+
+# ------------------------------------------------------------------ edge cases
+def test_edge_lengths_and_budgets(cuda_device):
+    # empty sequence, one token, exactly one page, k >= n_pages
+    wl = make_random(B=4, H_kv=2, G=2, d=64, P=16, lens=(0, 1, 16, 40), dtype=torch.float32,
+                     device="cuda", seed=11, topk=3)
+    for attn in ATTN:
+        cache, dec = run_gpu(wl, attn)
+        assert_status_ok(cache)
+        assert dec.sel_count[0].tolist() == [0, 0]
+        assert torch.all(dec.out[0] == 0) and torch.all(torch.isinf(dec.stat[0]))
+        for b in (1, 2, 3):
+            for h in range(2):
+                check_head(wl, cache, dec, b, h, attn)
+
+
+def test_tie_storm_prefers_lower_pages(cuda_device):
+    wl = make_random(B=2, H_kv=2, G=4, d=128, P=16, lens=(4096, 3000), dtype=torch.bfloat16,
+                     device="cuda", seed=12, topk=37)
+    wl.k_cache.fill_(0.5)  # every page has the same bound
+    cache, dec = run_gpu(wl, ekv.EKV_ENTMAX15)
+    assert_status_ok(cache)
+    for b in range(2):
+        for h in range(2):
+            np.testing.assert_array_equal(dec.sel_idx[b, h, :37].cpu().numpy(), np.arange(37))
+            check_head(wl, cache, dec, b, h, ekv.EKV_ENTMAX15)
+
+
+def test_bad_page_table_entry_is_flagged_not_trapped(cuda_device):
+    wl = make_random(B=2, H_kv=2, G=2, d=64, P=16, lens=(300, 200), dtype=torch.float32,
+                     device="cuda", seed=13, topk=4)
+    cache = make_cache(wl)
+    prefill_metadata(cache, wl)
+    assert_status_ok(cache)
+    wl.page_table[1, 3] = wl.k_cache.shape[0] + 5  # out of range
+    _, dec = run_gpu(wl, ekv.EKV_SOFTMAX, cache=cache)
+    st, bits = ekv.ekv_device_status(cache)
+    assert st == ekv.EKV_ERR_DEVICE and bits & ekv.EKV_DEV_BAD_BLOCK
+    ekv.ekv_clear_device_status(cache)
+    assert ekv.ekv_device_status(cache)[0] == ekv.EKV_OK
+    # sequence 0 is untouched by the bad entry
+    check_head(wl, cache, dec, 0, 1, ekv.EKV_SOFTMAX)
+
+
+def test_bad_selection_is_flagged(cuda_device):
+    wl = make_random(B=1, H_kv=1, G=1, d=64, P=16, lens=(100,), dtype=torch.float32,
+                     device="cuda", seed=14)
+    cache = make_cache(wl)
+    prefill_metadata(cache, wl)
+    sel = torch.tensor([[[0, 99]]], dtype=torch.int32, device="cuda")
+    cnt = torch.tensor([[2]], dtype=torch.int32, device="cuda")
+    out = torch.empty((1, 1, 64), device="cuda")
+    stat = torch.empty((1, 1), device="cuda")
+    ws = torch.empty(ekv.ekv_decode_workspace_bytes(cache, 1, 2), dtype=torch.uint8, device="cuda")
+    ekv.ekv_sparse_decode(cache, wl.q, 1, 1.0, ekv.EKV_SOFTMAX, sel, cnt, 2, out, stat, ws)
+    st, bits = ekv.ekv_device_status(cache)
+    assert st == ekv.EKV_ERR_DEVICE and bits & ekv.EKV_DEV_BAD_SEL
+    hc = HostCopy(wl, 0)
+    ref, _, _ = O.attend_head(hc.k, hc.v, hc.pt, hc.L, 0, hc.q[0], 1.0, O.SOFTMAX, [0])
+    close(out[0].double().cpu().numpy(), ref, False)
+
+
+def test_small_workspace_and_unsupported_shapes_are_refused(cuda_device):
+    wl = make_random(B=1, H_kv=1, G=1, d=64, P=16, lens=(64,), dtype=torch.float32,
+                     device="cuda", seed=15)
+    cache = make_cache(wl)
+    sel = torch.zeros((1, 1, 4), dtype=torch.int32, device="cuda")
+    cnt = torch.zeros((1, 1), dtype=torch.int32, device="cuda")
+    out = torch.empty((1, 1, 64), device="cuda")
+    stat = torch.empty((1, 1), device="cuda")
+    need = ekv.ekv_decode_workspace_bytes(cache, 1, 4)
+    ws = torch.empty(need - 256, dtype=torch.uint8, device="cuda")
+    with pytest.raises(ekv.EkvError) as e:
+        ekv.ekv_sparse_decode(cache, wl.q, 1, 1.0, ekv.EKV_SOFTMAX, sel, cnt, 4, out, stat, ws)
+    assert e.value.status == ekv.EKV_ERR_WORKSPACE
+    with pytest.raises(ekv.EkvError) as e:  # group size 3 is not a supported shape
+        ekv.ekv_score_pages(cache, wl.q, 3, 1.0, ekv.EKV_SEL_TOPK,
+                            torch.empty(64, device="cuda"))
+    assert e.value.status == ekv.EKV_ERR_UNSUPPORTED
+    wl2 = make_random(B=1, H_kv=2, G=1, d=64, P=16, lens=(64,), dtype=torch.float32,
+                      device="cuda", seed=15)
+    with pytest.raises(ekv.EkvError) as e:  # 3 query heads do not split over 2 KV heads
+        ekv.ekv_score_pages(make_cache(wl2), wl2.q, 3, 1.0, ekv.EKV_SEL_TOPK,
+                            torch.empty(64, device="cuda"))
+    assert e.value.status == ekv.EKV_ERR_INVALID_ARG
+
+
+def test_meta_update_append_equals_from_scratch(cuda_device):
+    # grow sequences token by token in uneven increments; incremental upkeep must equal a
+    # from-scratch build (and the oracle)
+    wl = make_random(B=3, H_kv=2, G=2, d=128, P=16, lens=(150, 77, 16), dtype=torch.bfloat16,
+                     device="cuda", seed=16, policy=GAUSS)
+    full = wl.seq_lens.clone()
+    cache = make_cache(wl)
+    cur = torch.zeros_like(full)
+    rng = np.random.default_rng(0)
+    while bool((cur < full).any()):
+        inc = torch.as_tensor(rng.integers(0, 23, size=3), dtype=torch.int32, device="cuda")
+        new = torch.minimum(cur + inc, full)
+        wl.seq_lens.copy_(new)
+        ekv.ekv_page_meta_update(cache, cur, new - cur, 22)
+        cur = new
+    assert_status_ok(cache)
+    ref = make_cache(wl)
+    prefill_metadata(ref, wl)
+    torch.cuda.synchronize()
+    for b in range(3):
+        n = (int(full[b]) + 15) // 16
+        blocks = wl.page_table[b, :n].long()
+        assert torch.equal(cache.meta_bbox[blocks], ref.meta_bbox[blocks])
+        assert torch.allclose(cache.meta_mom[blocks], ref.meta_mom[blocks], rtol=1e-6, atol=1e-6)
+    from parity_utils import check_meta
+    for b in range(3):
+        hc = HostCopy(wl, b)
+        for h in range(2):
+            check_meta(cache, hc, h, O.page_meta_head(hc.k, hc.pt, hc.L, h))
