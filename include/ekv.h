@@ -164,6 +164,31 @@ ekv_status ekv_sparse_decode(const ekv_cache *c, const void *q, int32_t num_q_he
                              const int32_t *sel_count, int32_t max_sel, float *out, float *stat,
                              void *ws, size_t ws_bytes, void *stream);
 
+/* Scratch that ekv_sparse_decode_noalloc draws on: 16 MiB, held by every GPU that loads the
+ * library until the process exits. */
+#define EKV_NOALLOC_WS_BYTES (16u << 20)
+
+/*
+ * ekv_sparse_decode without a workspace argument. (The paper has no counterpart: this is a
+ * library convenience.)
+ * For callers that cannot allocate device memory -- an engine whose allocator has already
+ * reserved all of HBM for the KV cache and its own pools, a latency-critical loop that must
+ * not risk a synchronising cudaMalloc/cudaFree, a plug-in that is handed only its inputs and
+ * outputs. The scratch is a fixed array inside the library; this call allocates nothing.
+ *   Arguments and results are those of ekv_sparse_decode (minus ws / ws_bytes).
+ *   A geometry whose ekv_decode_workspace_bytes() exceeds EKV_NOALLOC_WS_BYTES returns
+ *   EKV_ERR_WORKSPACE and launches nothing.
+ *   The first call on a device looks up the array's device address (once per device, with
+ *   that device current); make that first call before any stream capture.
+ *   Every call on a device shares the one array, which keeps the last call's contents
+ *   (nothing in it has to start at zero): calls that overlap on the GPU -- concurrent streams,
+ *   or several host threads -- race on it and must be serialised by the caller.
+ */
+ekv_status ekv_sparse_decode_noalloc(const ekv_cache *c, const void *q, int32_t num_q_heads,
+                                     float scale, int32_t attn, const int32_t *sel_idx,
+                                     const int32_t *sel_count, int32_t max_sel, float *out,
+                                     float *stat, void *stream);
+
 /* Scratch bytes ekv_sparse_decode needs for this cache geometry, num_q_heads and max_sel
  * (0 on invalid arguments). */
 size_t ekv_decode_workspace_bytes(const ekv_cache *c, int32_t num_q_heads, int32_t max_sel);

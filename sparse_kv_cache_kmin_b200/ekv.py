@@ -247,3 +247,22 @@ def ekv_clear_device_status(cache: PagedKVCache, stream=None):
     c = cache.struct()
     _check(load_library().ekv_clear_device_status(ctypes.byref(c), _stream(stream)),
            "ekv_clear_device_status")
+
+
+def ekv_sparse_decode_noalloc(cache: PagedKVCache, q: torch.Tensor, num_q_heads: int,
+                              scale: float, attn: int, sel_idx: torch.Tensor,
+                              sel_count: torch.Tensor, max_sel: int, out: torch.Tensor,
+                              stat: torch.Tensor, stream=None):
+    """ekv_sparse_decode with the library's fixed scratch (no workspace argument): for callers
+    that cannot allocate device memory. Its first call on a device should precede any stream
+    capture; calls that overlap on the GPU share the scratch and must be serialised."""
+    lib = load_library()
+    fn = lib.ekv_sparse_decode_noalloc
+    if fn.restype is not ctypes.c_int or fn.argtypes is None:
+        P, I32, F = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float
+        fn.argtypes = [ctypes.POINTER(EkvCacheStruct), P, I32, F, I32, P, P, I32, P, P, P]
+        fn.restype = ctypes.c_int
+    c = cache.struct()
+    _check(fn(ctypes.byref(c), _ptr(q), int(num_q_heads), float(scale), int(attn), _ptr(sel_idx),
+              _ptr(sel_count), int(max_sel), _ptr(out), _ptr(stat), _stream(stream)),
+           "ekv_sparse_decode_noalloc")
