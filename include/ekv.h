@@ -63,6 +63,8 @@ typedef enum { EKV_SEL_TOPK = 0, EKV_SEL_GAUSS = 1 } ekv_policy;
 #define EKV_DEV_BAD_SEL 0x4u      /* selected page outside [0, ceil(seq_len / P))         */
 #define EKV_DEV_SEL_OVERFLOW 0x8u /* Gaussian policy kept more than max_sel pages         */
 #define EKV_DEV_BAD_RANGE 0x10u   /* meta update range outside [0, seq_len] or > max_new   */
+#define EKV_DEV_TIMEOUT 0x20u     /* a bounded on-chip wait gave up (the call's outputs are
+                                     incomplete); not expected in normal operation          */
 
 /*
  * The paged cache and its metadata (§2, §2.A). Plain data; every pointer is device memory.
@@ -153,7 +155,9 @@ ekv_status ekv_select_pages(const ekv_cache *c, int32_t num_q_heads, int32_t pol
  *   EKV_ENTMAX15, EKV_SPARSEMAX: z = (alpha-1) s, exact tau with sum_i [z_i - tau]_+^(1/(alpha-1)) = 1,
  *                  p_i = [z_i - tau]_+^(1/(alpha-1));    stat = tau
  *   out[b][hq][:] = sum_i p_i v_i (fp32);  an empty selection gives out = 0, stat = -inf.
- *   q          [batch][num_q_heads][d] in c->dtype.
+ *   q          [batch][num_q_heads][d] in c->dtype. q, c->k_cache and c->v_cache must be
+ *              16-byte aligned (pages and query rows are moved with bulk copies), else
+ *              EKV_ERR_INVALID_ARG.
  *   out        [batch][num_q_heads][d] fp32.   stat [batch][num_q_heads] fp32.
  *   ws         scratch of at least ekv_decode_workspace_bytes(c, num_q_heads, max_sel)
  *              bytes. It must be zero-filled once before its first use; every call leaves

@@ -42,6 +42,7 @@ struct DecodeArgs {
     int NC;         // chunks per (sequence, KV head) at most
     int LS;         // logits row stride: NC * CP * P
     int Pshift;     // log2(P)
+    int stages;     // pipeline stages of the chunk kernel (2 or 3)
     float *part_ml; // [B * H_q][NC][2]   softmax (m, l); entmax (max z, unused)
     float *part_o;  // [B * H_q][NC][D]   softmax sum p v
     float *logits;  // [B * H_q][LS]       entmax z
@@ -49,83 +50,203 @@ struct DecodeArgs {
     float *stat;
 };
 
-constexpr int kChunkTok = 256;  // tokens per chunk at most
-constexpr int kNW = 8;          // warps per CTA
+constexpr int kNW = 8;         // consumer warps per CTA
+constexpr int kMaxCP = 16;     // pages per chunk at most
+constexpr int kThreads = (kNW + 1) * 32;
 
+// Tokens per chunk: a K tile (entmax) or a K + V tile (softmax) of about 32 KiB per pipeline
+// stage, at least one page, at most 256 tokens, a whole number of pages.
+__host__ __device__ constexpr int chunk_tokens(int row_bytes, int P, bool softmax)
+{
+    int t = (softmax ? 16384 : 32768) / row_bytes;
+    t = t > 256 ? 256 : t;
+    t = (t / P) * P;
+    return t < P ? P : t;
+}
+
+constexpr int kStages = 3;  // pipeline depth (shared-memory stages per CTA)
+
+// Bytes of one pipeline stage: the group's query rows (rounded to 128 B), then the K tile
+// (and the V tile for softmax).
+__host__ __device__ constexpr int stage_q_bytes(int G, int D, int esz) { return (G * D * esz + 127) / 128 * 128; }
+
+// Producer/consumer pipeline over the flattened (chunk, sequence, KV head) items of a
+// persistent grid. Warp kNW (the producer) walks the CTA's items, skips empty ones, resolves
+// the next item's pages (selection -> page table, validated) while the previous copies are in
+// flight, then waits for a free stage and issues one bulk copy per page span -- K rows, and V
+// rows for softmax -- plus one for the group's query rows, all completing on the stage's
+// `full` barrier. The eight consumer warps wait on `full`, compute from shared memory and
+// release the stage through its `empty` barrier. Every wait is bounded by the global timer:
+// on expiry the kernel flags EKV_DEV_TIMEOUT and stops.
 template <int DT, int D, int G, bool SOFTMAX>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(kThreads)
 decode_chunk_kernel(DecodeArgs a)
 {
     constexpr int EPC = Chunk<DT>::N;
     constexpr int ESZ = Chunk<DT>::kBytes;
-    constexpr int W = D * ESZ / 16;  // lanes per token row
+    constexpr int RB = D * ESZ;      // bytes per token row
+    constexpr int W = RB / 16;       // lanes per token row
     constexpr int RPI = 32 / W;      // rows per warp instruction
     constexpr int TPL = 4;           // rows per lane per step
     constexpr int TW = TPL * RPI;    // rows per warp step
     constexpr int NQK = TPL * G;
     constexpr int OUTN = NQK >= W ? NQK / W : 1;
-    __shared__ float z_s[G][kChunkTok];
-    __shared__ int blk_s[kChunkTok / 16], ntok_s[kChunkTok / 16];
+    constexpr int QB = stage_q_bytes(G, D, ESZ);
+    extern __shared__ __align__(128) unsigned char smem[];
+    __shared__ uint64_t bar_full[kStages], bar_empty[kStages];
+    __shared__ int blk_s[kStages][kMaxCP], ntok_s[kStages][kMaxCP];
+    __shared__ long long item_s[kStages];
     __shared__ float m_s[G], l_s[G];
-    extern __shared__ float o_s[];  // softmax: [kNW][G][D]
+    __shared__ int ok_s;
 
-    pdl_wait();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const ekv_cache &c = a.c;
     const int H = c.num_kv_heads, P = c.page_size, BH = c.batch * H;
-    const int CPP = a.CP * P;
-    const int cidx = lane % W;
-    const long items = (long)BH * a.NC;
-    const char *kc = static_cast<const char *>(c.k_cache);
-    const char *vc = static_cast<const char *>(c.v_cache);
+    const int CT = a.CP * P;                         // tokens per chunk
+    const int stage_bytes = QB + CT * RB * (SOFTMAX ? 2 : 1);
+    unsigned char *stage0 = smem;
+    const int NS = a.stages;
+    float *z_s = reinterpret_cast<float *>(smem + NS * stage_bytes);        // [G][CT]
+    float *o_s = z_s + G * CT;                                              // softmax: [kNW][G][D]
+    const long long items = (long long)BH * a.NC;
 
-    for (long it = blockIdx.x; it < items; it += gridDim.x) {
-        const int ci = (int)(it / BH), bh = (int)(it % BH);
-        const int b = bh / H, h = bh % H;
-        int len;
-        const int np = seq_pages(c.seq_lens, b, P, c.max_pages, nullptr, &len);
-        int nsel = a.sel_count[bh];
-        nsel = nsel < 0 ? 0 : (nsel > a.max_sel ? a.max_sel : nsel);
-        if (ci >= (nsel + a.CP - 1) / a.CP) continue;  // uniform over the CTA
+    if (tid == 0) {
+        for (int i = 0; i < NS; ++i) {
+            mbar_init(&bar_full[i], 1);
+            mbar_init(&bar_empty[i], kNW * 32);
+        }
+        fence_mbar_init();
+    }
+    __syncthreads();
+    pdl_wait();
 
-        if (tid < a.CP) {
-            const int i = ci * a.CP + tid;
-            int blk = 0, nt = 0;
+    if (warp == kNW) {
+        // ------------------------------------------------------------------ producer
+        const char *kc = static_cast<const char *>(c.k_cache);
+        const char *vc = static_cast<const char *>(c.v_cache);
+        const char *qc = static_cast<const char *>(a.q);
+        // the next non-empty item at or after `it`, with this lane's page of it resolved
+        long long it = blockIdx.x;
+        int ci = 0, bh = 0, blk = 0, nt = 0;
+        auto advance = [&]() {
+            int nsel = 0;
+            for (; it < items; it += gridDim.x) {
+                ci = (int)(it / BH);
+                bh = (int)(it % BH);
+                nsel = a.sel_count[bh];
+                nsel = nsel < 0 ? 0 : (nsel > a.max_sel ? a.max_sel : nsel);
+                if (ci * a.CP < nsel) break;
+            }
+            blk = 0;
+            nt = 0;
+            if (it >= items || lane >= a.CP) return;
+            const int b = bh / H;
+            int len;
+            const int np = seq_pages(c.seq_lens, b, P, c.max_pages, nullptr, &len);
+            const int i = ci * a.CP + lane;
             if (i < nsel) {
                 const int j = a.sel_idx[(size_t)bh * a.max_sel + i];
                 if (j < 0 || j >= np) {
                     flag(c.dev_status, EKV_DEV_BAD_SEL);
                 } else {
-                    blk = c.page_table[(size_t)b * c.max_pages + j];
-                    if (blk < 0 || blk >= c.num_blocks) {
+                    const int bk = c.page_table[(size_t)b * c.max_pages + j];
+                    if (bk < 0 || bk >= c.num_blocks) {
                         flag(c.dev_status, EKV_DEV_BAD_BLOCK);
-                        blk = 0;
                     } else {
+                        blk = bk;
                         nt = len - j * P < P ? len - j * P : P;
                     }
                 }
             }
-            blk_s[tid] = blk;
-            ntok_s[tid] = nt;
+        };
+        advance();
+        for (int k = 0;; ++k) {
+            const int buf = k % NS;
+            const uint32_t ph = (k / NS) & 1;
+            int free_ok = lane == 0 ? (int)mbar_wait_bounded(&bar_empty[buf], ph ^ 1) : 0;
+            free_ok = __shfl_sync(kFull, free_ok, 0);
+            if (!free_ok) {
+                if (lane == 0) flag(c.dev_status, EKV_DEV_TIMEOUT);
+                break;
+            }
+            mbar_try_wait(&bar_empty[buf], ph ^ 1);  // observe the release in every lane
+            if (it >= items) {
+                if (lane == 0) {
+                    item_s[buf] = -1;
+                    mbar_arrive(&bar_full[buf]);
+                }
+                break;
+            }
+            if (lane < a.CP) {
+                blk_s[buf][lane] = blk;
+                ntok_s[buf][lane] = nt;
+            }
+            const uint32_t bytes = (uint32_t)(nt * RB) * (SOFTMAX ? 2u : 1u);
+            const uint32_t total = (uint32_t)warp_sum((int)bytes) + (uint32_t)(G * D * ESZ);
+            if (lane == 0) item_s[buf] = it;
+            __syncwarp();
+            if (lane == 0) mbar_arrive_expect_tx(&bar_full[buf], total);
+            __syncwarp();
+            unsigned char *st = stage0 + buf * stage_bytes;
+            fence_proxy_async();
+            if (lane == 0) {
+                const int b = bh / H, h = bh % H;
+                bulk_copy_g2s(st, qc + ((size_t)b * a.H_q + (size_t)h * G) * D * ESZ,
+                              (uint32_t)(G * D * ESZ), &bar_full[buf]);
+            }
+            if (lane < a.CP && nt > 0) {
+                const int h = bh % H;
+                unsigned char *dst = st + QB + lane * P * RB;
+                const size_t off = ((size_t)blk * H + h) * P * RB;
+                bulk_copy_g2s(dst, kc + off, (uint32_t)(nt * RB), &bar_full[buf]);
+                if (SOFTMAX) bulk_copy_g2s(dst + CT * RB, vc + off, (uint32_t)(nt * RB), &bar_full[buf]);
+            }
+            it += gridDim.x;
+            advance();  // resolve the next item while this one's copies are in flight
         }
+        pdl_trigger();
+        return;
+    }
+
+    // ---------------------------------------------------------------------- consumers
+    const int cidx = lane % W;
+    for (int k = 0;; ++k) {
+        const int buf = k % NS;
+        const uint32_t ph = (k / NS) & 1;
+        if (tid == 0) ok_s = (int)mbar_wait_bounded(&bar_full[buf], ph);
+        named_sync(1, kNW * 32);
+        if (!ok_s) {
+            if (tid == 0) {
+                flag(c.dev_status, EKV_DEV_TIMEOUT);
+                mbar_wait_bounded(&bar_full[buf], ph);  // let any copy still in flight land
+            }
+            break;
+        }
+        mbar_try_wait(&bar_full[buf], ph);  // observe the completed phase in every thread
+        const long long it = item_s[buf];
+        if (it < 0) break;
+        const int ci = (int)(it / BH), bh = (int)(it % BH);
+        const int b = bh / H, h = bh % H;
+        const unsigned char *st = stage0 + buf * stage_bytes;
+        const unsigned char *tile = st + QB;
+        const int *ntok = ntok_s[buf];
+
         float qv[G][EPC];
 #pragma unroll
-        for (int g = 0; g < G; ++g)
+        for (int g = 0; g < G; ++g) {
+            float f[EPC];
+            Chunk<DT>::unpack(*reinterpret_cast<const uint4 *>(st + g * RB + cidx * 16), f);
 #pragma unroll
-            for (int e = 0; e < EPC; ++e)
-                qv[g][e] = a.qscale * load_elem<DT>(a.q, ((size_t)b * a.H_q + h * G + g) * D + cidx * EPC + e);
-        __syncthreads();
+            for (int e = 0; e < EPC; ++e) qv[g][e] = a.qscale * f[e];
+        }
 
-        // ---- logits of the chunk's tokens
-        for (int base = warp * TW; base < CPP; base += kNW * TW) {
+        // ---- logits of the chunk's tokens, from shared memory
+        for (int base = warp * TW; base < CT; base += kNW * TW) {
             uint4 x[TPL];
 #pragma unroll
             for (int i = 0; i < TPL; ++i) {
                 const int slot = base + i * RPI + lane / W;
-                const int pi = slot >> a.Pshift, t = slot & (P - 1);
-                x[i] = t < ntok_s[pi]
-                           ? ld_stream16(kc + ((((size_t)blk_s[pi] * H + h) * P + t) * D) * ESZ + cidx * 16)
-                           : make_uint4(0, 0, 0, 0);
+                x[i] = *reinterpret_cast<const uint4 *>(tile + slot * RB + cidx * 16);
             }
             float part[NQK];
 #pragma unroll
@@ -148,96 +269,98 @@ decode_chunk_kernel(DecodeArgs a)
                     const int i = idx / G, g = idx % G;
                     const int slot = base + i * RPI + lane / W;
                     const int pi = slot >> a.Pshift, t = slot & (P - 1);
-                    z_s[g][slot] = t < ntok_s[pi] ? part[r] : -INFINITY;
+                    z_s[g * CT + slot] = t < ntok[pi] ? part[r] : -INFINITY;
                 }
             }
         }
-        __syncthreads();
+        named_sync(1, kNW * 32);
         if (warp < G) {
             float m = -INFINITY;
-            for (int s = lane; s < CPP; s += 32) m = fmaxf(m, z_s[warp][s]);
+            for (int s = lane; s < CT; s += 32) m = fmaxf(m, z_s[warp * CT + s]);
             m = warp_max(m);
             if (lane == 0) m_s[warp] = m;
         }
-        __syncthreads();
+        named_sync(1, kNW * 32);
         const size_t bq0 = (size_t)b * a.H_q + h * G;
 
         if constexpr (!SOFTMAX) {
-            for (int i = tid; i < G * CPP; i += 256) {
-                const int g = i / CPP, s = i - g * CPP;
-                a.logits[(bq0 + g) * (size_t)a.LS + (size_t)ci * CPP + s] = z_s[g][s];
+            mbar_arrive(&bar_empty[buf]);  // the stage is no longer read
+            for (int i = tid; i < G * CT; i += kNW * 32) {
+                const int g = i / CT, s = i - g * CT;
+                a.logits[(bq0 + g) * (size_t)a.LS + (size_t)ci * CT + s] = z_s[g * CT + s];
             }
             if (tid < G) a.part_ml[((bq0 + tid) * a.NC + ci) * 2] = m_s[tid];
-            __syncthreads();
+            named_sync(1, kNW * 32);
             continue;
-        }
-
-        // ---- softmax partial: p = 2^(z - m), l = sum p, o = sum p v
-        for (int i = tid; i < G * CPP; i += 256) {
-            const int g = i / CPP, s = i - g * CPP;
-            const float z = z_s[g][s];
-            z_s[g][s] = z == -INFINITY ? 0.f : exp2f(z - m_s[g]);
-        }
-        __syncthreads();
-        if (warp < G) {
-            float l = 0.f;
-            for (int s = lane; s < CPP; s += 32) l += z_s[warp][s];
-            l = warp_sum(l);
-            if (lane == 0) l_s[warp] = l;
-        }
-        float acc[G][EPC];
-#pragma unroll
-        for (int g = 0; g < G; ++g)
-#pragma unroll
-            for (int e = 0; e < EPC; ++e) acc[g][e] = 0.f;
-        for (int base = warp * TW; base < CPP; base += kNW * TW) {
-            uint4 x[TPL];
-#pragma unroll
-            for (int i = 0; i < TPL; ++i) {
-                const int slot = base + i * RPI + lane / W;
-                const int pi = slot >> a.Pshift, t = slot & (P - 1);
-                x[i] = t < ntok_s[pi]
-                           ? ld_stream16(vc + ((((size_t)blk_s[pi] * H + h) * P + t) * D) * ESZ + cidx * 16)
-                           : make_uint4(0, 0, 0, 0);
+        } else {
+            // ---- softmax partial: p = 2^(z - m), l = sum p, o = sum p v (V tile after K)
+            for (int i = tid; i < G * CT; i += kNW * 32) {
+                const int g = i / CT;
+                const float z = z_s[i];
+                z_s[i] = z == -INFINITY ? 0.f : exp2f(z - m_s[g]);
             }
+            named_sync(1, kNW * 32);
+            if (warp < G) {
+                float l = 0.f;
+                for (int s = lane; s < CT; s += 32) l += z_s[warp * CT + s];
+                l = warp_sum(l);
+                if (lane == 0) l_s[warp] = l;
+            }
+            float acc[G][EPC];
 #pragma unroll
-            for (int i = 0; i < TPL; ++i) {
-                const int slot = base + i * RPI + lane / W;
-                float f[EPC];
-                Chunk<DT>::unpack(x[i], f);
+            for (int g = 0; g < G; ++g)
 #pragma unroll
-                for (int g = 0; g < G; ++g) {
-                    const float p = z_s[g][slot];
+                for (int e = 0; e < EPC; ++e) acc[g][e] = 0.f;
+            const unsigned char *vt = tile + CT * RB;
+            for (int base = warp * TW; base < CT; base += kNW * TW) {
+                uint4 x[TPL];
 #pragma unroll
-                    for (int e = 0; e < EPC; ++e) acc[g][e] = fmaf(p, f[e], acc[g][e]);
+                for (int i = 0; i < TPL; ++i) {
+                    const int slot = base + i * RPI + lane / W;
+                    x[i] = *reinterpret_cast<const uint4 *>(vt + slot * RB + cidx * 16);
+                }
+#pragma unroll
+                for (int i = 0; i < TPL; ++i) {
+                    const int slot = base + i * RPI + lane / W;
+                    float f[EPC];
+                    Chunk<DT>::unpack(x[i], f);
+#pragma unroll
+                    for (int g = 0; g < G; ++g) {
+                        const float p = z_s[g * CT + slot];
+                        if (p != 0.f) {  // rows past a page's valid tokens hold stale data
+#pragma unroll
+                            for (int e = 0; e < EPC; ++e) acc[g][e] = fmaf(p, f[e], acc[g][e]);
+                        }
+                    }
                 }
             }
+            mbar_arrive(&bar_empty[buf]);  // the stage is no longer read
+#pragma unroll
+            for (int o = W; o < 32; o <<= 1)
+#pragma unroll
+                for (int g = 0; g < G; ++g)
+#pragma unroll
+                    for (int e = 0; e < EPC; ++e) acc[g][e] += __shfl_xor_sync(kFull, acc[g][e], o);
+            if (lane < W) {
+#pragma unroll
+                for (int g = 0; g < G; ++g)
+#pragma unroll
+                    for (int e = 0; e < EPC; ++e) o_s[(warp * G + g) * D + cidx * EPC + e] = acc[g][e];
+            }
+            named_sync(1, kNW * 32);
+            for (int i = tid; i < G * D; i += kNW * 32) {
+                float s = 0.f;
+#pragma unroll
+                for (int w = 0; w < kNW; ++w) s += o_s[w * G * D + i];
+                const int g = i / D, dd = i - g * D;
+                a.part_o[((bq0 + g) * a.NC + ci) * D + dd] = s;
+            }
+            if (tid < G) {
+                a.part_ml[((bq0 + tid) * a.NC + ci) * 2] = m_s[tid];
+                a.part_ml[((bq0 + tid) * a.NC + ci) * 2 + 1] = l_s[tid];
+            }
+            named_sync(1, kNW * 32);
         }
-#pragma unroll
-        for (int o = W; o < 32; o <<= 1)
-#pragma unroll
-            for (int g = 0; g < G; ++g)
-#pragma unroll
-                for (int e = 0; e < EPC; ++e) acc[g][e] += __shfl_xor_sync(kFull, acc[g][e], o);
-        if (lane < W) {
-#pragma unroll
-            for (int g = 0; g < G; ++g)
-#pragma unroll
-                for (int e = 0; e < EPC; ++e) o_s[(warp * G + g) * D + cidx * EPC + e] = acc[g][e];
-        }
-        __syncthreads();
-        for (int i = tid; i < G * D; i += 256) {
-            float s = 0.f;
-#pragma unroll
-            for (int w = 0; w < kNW; ++w) s += o_s[w * G * D + i];
-            const int g = i / D, dd = i - g * D;
-            a.part_o[((bq0 + g) * a.NC + ci) * D + dd] = s;
-        }
-        if (tid < G) {
-            a.part_ml[((bq0 + tid) * a.NC + ci) * 2] = m_s[tid];
-            a.part_ml[((bq0 + tid) * a.NC + ci) * 2 + 1] = l_s[tid];
-        }
-        __syncthreads();
     }
     pdl_trigger();
 }
@@ -275,6 +398,7 @@ __device__ void finish_softmax(const DecodeArgs &a, int b, int hq, int nchunks)
     const int dd = tid % D, part = tid / D;
     float acc = 0.f;
     if (M != -INFINITY) {
+#pragma unroll 8
         for (int ch = part; ch < nchunks; ch += SPLIT) {
             const float m = __ldcg(ml + 2 * ch);
             if (m != -INFINITY)
@@ -292,23 +416,73 @@ __device__ void finish_softmax(const DecodeArgs &a, int b, int hq, int nchunks)
     if (tid == 0) a.stat[bq] = M == -INFINITY ? -INFINITY : (M + log2f(L)) * 0.69314718055994530942f;
 }
 
-template <int DT, int D>
-__device__ void finish_entmax(const DecodeArgs &a, int b, int hq, int h, int nsel, int nchunks)
+constexpr int kCapW = 512;  // gathered logits per warp kept in shared memory
+
+// Exact threshold of <= 32 candidates, one per lane (x = z - zmax, -inf padding): sort
+// descending across the warp, prefix sums of x and x^2, then the largest k whose closed-form
+// tau(k) satisfies tau(k) <= x_(k) (1.5-entmax also needs a real root).
+__device__ __forceinline__ double warp_exact_tau(float x, int cnt, bool sparsemax)
 {
-    constexpr int CAPW = 256;  // gathered logits per warp
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int k = 2; k <= 32; k <<= 1)
+#pragma unroll
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            const float o = __shfl_xor_sync(kFull, x, j);
+            const bool up = (lane & k) == 0, lower = (lane & j) == 0;
+            x = (lower == up) ? fmaxf(x, o) : fminf(x, o);
+        }
+    const bool in = lane < cnt;
+    const double xd = in ? (double)x : 0.0;
+    double s1 = xd, s2 = xd * xd;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const double t1 = __shfl_up_sync(kFull, s1, o), t2 = __shfl_up_sync(kFull, s2, o);
+        if (lane >= o) { s1 += t1; s2 += t2; }
+    }
+    const double k = lane + 1;
+    double tk;
+    bool ok = in;
+    if (sparsemax) {
+        tk = (s1 - 1.0) / k;
+    } else {
+        const double mean = s1 / k;
+        const double m2 = s2 - s1 * mean;  // sum of squared deviations of the top k
+        const double disc = (1.0 - m2) / k;
+        ok = ok && disc >= 0.0;
+        tk = mean - sqrt(disc > 0.0 ? disc : 0.0);
+    }
+    ok = ok && tk <= (double)x;
+    const unsigned bal = __ballot_sync(kFull, ok);
+    const int K = 31 - __clz(bal);  // lane 0 is always valid: tau(1) = x_(1) - 1
+    return __shfl_sync(kFull, tk, K);
+}
+
+// Entmax finish for one (sequence, query head), one CTA: the eight warps gather the logits
+// above max z - 1 (only those can carry weight) from contiguous slot ranges into per-warp lists
+// in shared memory; warp 0 finds tau (exact sort for <= 32 candidates, else fp32 Newton then a
+// closed-form fp64 polish over the support); then every warp accumulates p_i v_i over the
+// support entries of its own list, resolving their page-table look-ups 32 at a time and
+// keeping several V rows in flight. A warp whose list overflows walks its slot range in global
+// memory instead (correct, slower).
+template <int DT, int D>
+__device__ void finish_entmax_cta(const DecodeArgs &a, int b, int h, int hq, int nsel, int nchunks)
+{
     constexpr int EPC = Chunk<DT>::N;
     constexpr int ESZ = Chunk<DT>::kBytes;
     constexpr int W = D * ESZ / 16;
     constexpr int RPI = 32 / W;
-    __shared__ float cz[kNW][CAPW];
-    __shared__ int cs[kNW][CAPW];
+    constexpr int UNRV = 4;  // V rows in flight per lane group
+    constexpr int UNR = 8;   // logits in flight per lane while gathering
+    __shared__ float cz[kNW][kCapW];
+    __shared__ int cs[kNW][kCapW];
     __shared__ int cn[kNW];
     __shared__ float red[kNW];
     __shared__ double s_tau;
     __shared__ float o_w[kNW][D];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const ekv_cache &c = a.c;
-    const int P = c.page_size;
+    const int P = c.page_size, H = c.num_kv_heads;
     const size_t bq = (size_t)b * a.H_q + hq;
     const float *z = a.logits + bq * (size_t)a.LS;
     const bool sparsemax = a.alpha == 2.0f;
@@ -326,119 +500,166 @@ __device__ void finish_entmax(const DecodeArgs &a, int b, int hq, int h, int nse
         if (tid == 0) a.stat[bq] = -INFINITY;
         return;
     }
-    const float thr = zmax - 1.0f;
+    const float thr = zmax - 1.0f;  // the largest weight is at most 1, so tau >= zmax - 1
 
-    // gather the logits above thr: warp w scans a contiguous slot range, in slot order
+    // gather: warp w owns slots [s0, s1)
     const int nslots = nsel * P;
-    const int per_warp = ((nslots + kNW - 1) / kNW + 31) / 32 * 32;
-    const int s0 = warp * per_warp, s1 = min(s0 + per_warp, nslots);
+    const int per = (nslots + kNW - 1) / kNW;
+    const int s0 = warp * per, s1 = min(s0 + per, nslots);
     int cnt = 0;
-    for (int s = s0; s < s1; s += 32) {
-        const int sl = s + lane;
-        const float v = sl < s1 ? __ldcg(z + sl) : -INFINITY;
-        const bool keep = v > thr;
-        const unsigned bal = __ballot_sync(kFull, keep);
-        const int pos = cnt + __popc(bal & ((1u << lane) - 1u));
-        if (keep && pos < CAPW) { cz[warp][pos] = v; cs[warp][pos] = sl; }
-        cnt += __popc(bal);
+    for (int s = s0; s < s1; s += 32 * UNR) {
+        float v[UNR];
+#pragma unroll
+        for (int u = 0; u < UNR; ++u) {
+            const int sl = s + u * 32 + lane;
+            v[u] = sl < s1 ? __ldcg(z + sl) : -INFINITY;
+        }
+#pragma unroll
+        for (int u = 0; u < UNR; ++u) {
+            const bool keep = v[u] > thr;
+            const unsigned bal = __ballot_sync(kFull, keep);
+            const int pos = cnt + __popc(bal & ((1u << lane) - 1u));
+            if (keep && pos < kCapW) { cz[warp][pos] = v[u]; cs[warp][pos] = s + u * 32 + lane; }
+            cnt += __popc(bal);
+        }
     }
     if (lane == 0) cn[warp] = cnt;
     __syncthreads();
-    bool overflow = false;
-#pragma unroll
-    for (int w = 0; w < kNW; ++w) overflow |= cn[w] > CAPW;
 
-    // threshold: warp 0, Newton from the left, then closed form on the support
     if (warp == 0) {
+        int total = 0;
+        bool any_over = false;
+#pragma unroll
+        for (int w = 0; w < kNW; ++w) { total += cn[w]; any_over |= cn[w] > kCapW; }
+        // every gathered logit, shifted by zmax
         auto visit = [&](auto &&fn) {
-            if (!overflow) {
-                for (int w = 0; w < kNW; ++w)
-                    for (int i = lane; i < cn[w]; i += 32) fn(cz[w][i]);
-            } else {
-                for (int s = lane; s < nslots; s += 32) {
-                    const float v = __ldcg(z + s);
-                    if (v > thr) fn(v);
+            for (int w = 0; w < kNW; ++w) {
+                if (cn[w] <= kCapW) {
+                    for (int i = lane; i < cn[w]; i += 32) fn(cz[w][i] - zmax);
+                } else {
+                    const int a0 = w * per, a1 = min(a0 + per, nslots);
+                    for (int sl = a0 + lane; sl < a1; sl += 32) {
+                        const float v = __ldcg(z + sl);
+                        if (v > thr) fn(v - zmax);
+                    }
                 }
             }
         };
-        double tau = thr;
-#pragma unroll 1
-        for (int it = 0; it < 100; ++it) {
-            double f = 0.0, df = 0.0;
-            visit([&](float v) {
-                const double r = (double)v - tau;
-                if (r > 0.0) {
-                    f += sparsemax ? r : r * r;
-                    df += sparsemax ? 1.0 : 2.0 * r;
-                }
-            });
-            f = warp_sum(f) - 1.0;
-            df = warp_sum(df);
-            if (!(df > 0.0) || !(f > 0.0)) break;
-            const double step = f / df;
-            if (!(step > 1e-12 * fmax(1.0, fabs(tau)))) break;
-            tau += step;
-        }
-        // exact closed form over the support, until the support is stable
-#pragma unroll 1
-        for (int round = 0; round < 8; ++round) {
-            double n = 0.0, s1v = 0.0;
-            visit([&](float v) { if ((double)v > tau) { n += 1.0; s1v += v; } });
-            n = warp_sum(n);
-            s1v = warp_sum(s1v);
-            if (n < 1.0) break;
-            double t2;
-            if (sparsemax) {
-                t2 = (s1v - 1.0) / n;
-            } else {
-                const double mean = s1v / n;
-                double m2 = 0.0;
-                visit([&](float v) { if ((double)v > tau) m2 += ((double)v - mean) * ((double)v - mean); });
-                m2 = warp_sum(m2);
-                const double disc = (1.0 - m2) / n;
-                if (disc < 0.0) break;
-                t2 = mean - sqrt(disc);
+        double tau;  // in the shifted domain x = z - zmax
+        if (!any_over && total <= 32) {
+            // lane i takes the i-th candidate in warp order
+            float x = -INFINITY;
+            int base = 0;
+#pragma unroll
+            for (int w = 0; w < kNW; ++w) {
+                if (lane >= base && lane < base + cn[w]) x = cz[w][lane - base] - zmax;
+                base += cn[w];
             }
-            // stable iff {v > t2} == {v > tau}
-            int changed = 0;
-            visit([&](float v) { changed |= ((double)v > t2) != ((double)v > tau); });
-            changed = __any_sync(kFull, changed);
-            tau = t2;
-            if (!changed) break;
+            tau = warp_exact_tau(x, total, sparsemax);
+        } else {
+            float t = -1.0f;
+#pragma unroll 1
+            for (int it = 0; it < 40; ++it) {
+                float f = 0.f, df = 0.f;
+                visit([&](float x) {
+                    const float r = x - t;
+                    if (r > 0.f) { f += sparsemax ? r : r * r; df += sparsemax ? 1.f : 2.f * r; }
+                });
+                f = warp_sum(f) - 1.0f;
+                df = warp_sum(df);
+                if (!(f > 0.f) || !(df > 0.f)) break;
+                const float step = f / df;
+                t += step;
+                if (!(step > 1e-6f)) break;
+            }
+            tau = t;
+#pragma unroll 1
+            for (int round = 0; round < 4; ++round) {
+                double n = 0.0, s1d = 0.0;
+                visit([&](float x) { if ((double)x > tau) { n += 1.0; s1d += x; } });
+                n = warp_sum(n);
+                s1d = warp_sum(s1d);
+                if (n < 1.0) break;
+                double t2;
+                if (sparsemax) {
+                    t2 = (s1d - 1.0) / n;
+                } else {
+                    const double mean = s1d / n;
+                    double m2 = 0.0;
+                    visit([&](float x) { if ((double)x > tau) m2 += ((double)x - mean) * ((double)x - mean); });
+                    m2 = warp_sum(m2);
+                    const double disc = (1.0 - m2) / n;
+                    if (disc < 0.0) break;
+                    t2 = mean - sqrt(disc);
+                }
+                int changed = 0;
+                visit([&](float x) { changed |= ((double)x > t2) != ((double)x > tau); });
+                changed = __any_sync(kFull, changed);
+                tau = t2;
+                if (!changed) break;
+            }
         }
-        if (lane == 0) s_tau = tau;
+        if (lane == 0) s_tau = tau + (double)zmax;
     }
     __syncthreads();
-    const double tau = s_tau;
+    const double tau_z = s_tau;
 
-    // o = sum over the support of p_i v_i; warp w takes its own gathered entries (or, on
-    // overflow, every slot s with s % kNW == w)
+    // o = sum over the support of p_i v_i, each warp over its own entries
     const char *vc = static_cast<const char *>(c.v_cache);
-    const int H = c.num_kv_heads;
     const int cidx = lane % W, row = lane / W;
     float acc[EPC];
 #pragma unroll
     for (int e = 0; e < EPC; ++e) acc[e] = 0.f;
-    const int nmine = overflow ? (nslots + kNW - 1 - warp) / kNW : cn[warp];
-    for (int k0 = 0; k0 < nmine; k0 += RPI) {
-        const int k = k0 + row;
+    const bool over = cnt > kCapW;
+    float *sp = cz[warp];  // compacted support weights, in place over the gathered list
+    int *sr = cs[warp];    // and rows as blk * P + t
+    const int total = over ? s1 - s0 : cnt;
+    for (int i0 = 0; i0 < total; i0 += 32) {
+        const int i = i0 + lane;
         float v = -INFINITY;
         int slot = 0;
-        if (k < nmine) {
-            if (overflow) { slot = warp + k * kNW; v = __ldcg(z + slot); }
-            else { slot = cs[warp][k]; v = cz[warp][k]; }
+        if (i < total) {
+            if (over) { slot = s0 + i; v = __ldcg(z + slot); }
+            else { slot = cs[warp][i]; v = cz[warp][i]; }
         }
-        const double r = (double)v - tau;
-        if (r > 0.0) {
-            const float p = (float)(sparsemax ? r : r * r);
+        const double r = (double)v - tau_z;
+        const bool keep = r > 0.0;
+        const unsigned bal = __ballot_sync(kFull, keep);
+        const int nb = __popc(bal);
+        __syncwarp();
+        if (keep) {
+            const int pos = __popc(bal & ((1u << lane) - 1u));
             const int pi = slot >> a.Pshift, t = slot & (P - 1);
             const int j = a.sel_idx[((size_t)b * H + h) * a.max_sel + pi];
             const int blk = c.page_table[(size_t)b * c.max_pages + j];
-            float f[EPC];
-            Chunk<DT>::unpack(ld_stream16(vc + ((((size_t)blk * H + h) * P + t) * D) * ESZ + cidx * 16), f);
-#pragma unroll
-            for (int e = 0; e < EPC; ++e) acc[e] = fmaf(p, f[e], acc[e]);
+            sp[pos] = (float)(sparsemax ? r : r * r);
+            sr[pos] = blk * P + t;
         }
+        __syncwarp();
+        for (int k0 = 0; k0 < nb; k0 += RPI * UNRV) {
+            uint4 x[UNRV];
+            float p[UNRV];
+#pragma unroll
+            for (int u = 0; u < UNRV; ++u) {
+                const int k = k0 + u * RPI + row;
+                p[u] = 0.f;
+                x[u] = make_uint4(0, 0, 0, 0);
+                if (k < nb) {
+                    p[u] = sp[k];
+                    const int br = sr[k];
+                    const size_t rowi = ((size_t)(br >> a.Pshift) * H + h) * P + (br & (P - 1));
+                    x[u] = ld_stream16(vc + rowi * D * ESZ + cidx * 16);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < UNRV; ++u) {
+                float f[EPC];
+                Chunk<DT>::unpack(x[u], f);
+#pragma unroll
+                for (int e = 0; e < EPC; ++e) acc[e] = fmaf(p[u], f[e], acc[e]);
+            }
+        }
+        __syncwarp();
     }
 #pragma unroll
     for (int o = W; o < 32; o <<= 1)
@@ -450,18 +671,19 @@ __device__ void finish_entmax(const DecodeArgs &a, int b, int hq, int h, int nse
     }
     __syncthreads();
     for (int i = tid; i < D; i += 256) {
-        float s = 0.f;
+        float sum = 0.f;
 #pragma unroll
-        for (int w = 0; w < kNW; ++w) s += o_w[w][i];
-        a.out[bq * D + i] = s;
+        for (int w = 0; w < kNW; ++w) sum += o_w[w][i];
+        a.out[bq * D + i] = sum;
     }
-    if (tid == 0) a.stat[bq] = (float)tau;
+    if (tid == 0) a.stat[bq] = (float)tau_z;
 }
 
 template <int DT, int D, int G, bool SOFTMAX>
 __global__ void __launch_bounds__(256)
 decode_finish_kernel(DecodeArgs a)
 {
+    // one CTA per (sequence, query head)
     pdl_wait();
     const int hq = blockIdx.x, b = blockIdx.y;
     const int h = hq / G, bh = b * a.c.num_kv_heads + h;
@@ -472,32 +694,24 @@ decode_finish_kernel(DecodeArgs a)
     if (nchunks == 0) {
         for (int i = threadIdx.x; i < D; i += 256) a.out[bq * D + i] = 0.f;
         if (threadIdx.x == 0) a.stat[bq] = -INFINITY;
-        pdl_trigger();
-        return;
+    } else if constexpr (SOFTMAX) {
+        finish_softmax<D>(a, b, hq, nchunks);
+    } else {
+        finish_entmax_cta<DT, D>(a, b, h, hq, nsel, nchunks);
     }
-    if constexpr (SOFTMAX) finish_softmax<D>(a, b, hq, nchunks);
-    else finish_entmax<DT, D>(a, b, hq, h, nsel, nchunks);
     pdl_trigger();
 }
 
 // ------------------------------------------------------------------------------ host side
-// Pages per chunk: enough chunks to give every SM a few CTAs, at most 256 tokens per chunk.
-int decode_pages_per_chunk(int batch, int H_kv, int max_sel, int P)
-{
-    long units = (long)batch * H_kv * max_sel;
-    long cp = units / (148L * 4);
-    const int cap = kChunkTok / P;
-    if (cp > cap) cp = cap;
-    if (cp < 1) cp = 1;
-    return (int)cp;
-}
-
 static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-size_t decode_workspace_layout(int batch, int H_q, int H_kv, int D, int P, int max_sel,
-                               size_t *off_o, size_t *off_logits, int *CP, int *NC)
+// Workspace layout of one attention mode: [B*H_q][NC][2] chunk (m, l) | [B*H_q][NC][D] chunk
+// sums (softmax) | [B*H_q][NC*CP*P] logits (entmax), each 256-byte aligned.
+static size_t mode_layout(int batch, int H_q, int D, int P, int dtype, int max_sel, bool softmax,
+                          size_t *off_o, size_t *off_logits, int *CP, int *NC)
 {
-    const int cp = decode_pages_per_chunk(batch, H_kv, max_sel, P);
+    const int rb = D * (dtype == EKV_BF16 ? 2 : 4);
+    const int cp = chunk_tokens(rb, P, softmax) / P;
     const int nc = (max_sel + cp - 1) / cp;
     const size_t BQ = (size_t)batch * H_q;
     size_t off = align256(BQ * nc * 2 * sizeof(float));
@@ -510,6 +724,39 @@ size_t decode_workspace_layout(int batch, int H_q, int H_kv, int D, int P, int m
     return off;
 }
 
+// Bytes that cover every attention mode.
+size_t decode_workspace_bytes_all_modes(int batch, int H_q, int D, int P, int dtype, int max_sel)
+{
+    const size_t a = mode_layout(batch, H_q, D, P, dtype, max_sel, true, nullptr, nullptr, nullptr, nullptr);
+    const size_t b = mode_layout(batch, H_q, D, P, dtype, max_sel, false, nullptr, nullptr, nullptr, nullptr);
+    return a > b ? a : b;
+}
+
+template <int DT, int D, int G, bool SOFTMAX>
+static cudaError_t launch_chunk(const DecodeArgs &a, cudaLaunchConfig_t cfg)
+{
+    constexpr int RB = D * Chunk<DT>::kBytes;
+    auto k = decode_chunk_kernel<DT, D, G, SOFTMAX>;
+    const int CT = a.CP * a.c.page_size;
+    const size_t stage = (size_t)stage_q_bytes(G, D, Chunk<DT>::kBytes) + (size_t)CT * RB * (SOFTMAX ? 2 : 1);
+    const size_t fixed = sizeof(float) * G * CT + (SOFTMAX ? sizeof(float) * kNW * G * D : 0);
+    DecodeArgs a2 = a;
+    a2.stages = kStages * stage + fixed <= 220 * 1024 ? kStages : 2;
+    const size_t smem = a2.stages * stage + fixed;
+    static bool attr_set = false;  // per instantiation
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, 220 * 1024);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    const long long items = (long long)a.c.batch * a.c.num_kv_heads * a.NC;
+    const long long grid = persistent_grid_size((const void *)k, kThreads, smem);
+    cfg.gridDim = dim3((unsigned)(items < grid ? items : grid));
+    return cudaLaunchKernelEx(&cfg, k, a2);
+}
+
 template <int DT, int D, int G>
 static cudaError_t launch_decode_t(const DecodeArgs &a, bool softmax, cudaStream_t st, bool pdl)
 {
@@ -517,26 +764,12 @@ static cudaError_t launch_decode_t(const DecodeArgs &a, bool softmax, cudaStream
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cudaLaunchConfig_t cfg = {};
-    cfg.blockDim = dim3(256);
     cfg.stream = st;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    const long items = (long)a.c.batch * a.c.num_kv_heads * a.NC;
-    cudaError_t e;
-    if (softmax) {
-        auto k = decode_chunk_kernel<DT, D, G, true>;
-        cfg.dynamicSmemBytes = sizeof(float) * kNW * G * D;
-        const long grid = persistent_grid_size((const void *)k, 256, cfg.dynamicSmemBytes);
-        cfg.gridDim = dim3((unsigned)(items < grid ? items : grid));
-        e = cudaLaunchKernelEx(&cfg, k, a);
-    } else {
-        auto k = decode_chunk_kernel<DT, D, G, false>;
-        cfg.dynamicSmemBytes = 0;
-        const long grid = persistent_grid_size((const void *)k, 256, 0);
-        cfg.gridDim = dim3((unsigned)(items < grid ? items : grid));
-        e = cudaLaunchKernelEx(&cfg, k, a);
-    }
+    cudaError_t e = softmax ? launch_chunk<DT, D, G, true>(a, cfg) : launch_chunk<DT, D, G, false>(a, cfg);
     if (e != cudaSuccess) return e;
+    cfg.blockDim = dim3(256);
     cfg.dynamicSmemBytes = 0;
     cfg.gridDim = dim3(a.H_q, a.c.batch);
     cfg.numAttrs = 1;  // the finish kernel always waits on the chunk kernel programmatically
@@ -562,8 +795,8 @@ cudaError_t launch_sparse_decode(const ekv_cache &c, const void *q, int H_q, flo
 {
     DecodeArgs a;
     size_t off_o, off_logits;
-    decode_workspace_layout(c.batch, H_q, c.num_kv_heads, c.head_dim, c.page_size, max_sel,
-                            &off_o, &off_logits, &a.CP, &a.NC);
+    mode_layout(c.batch, H_q, c.head_dim, c.page_size, c.dtype, max_sel, attn == EKV_SOFTMAX,
+                &off_o, &off_logits, &a.CP, &a.NC);
     a.LS = a.NC * a.CP * c.page_size;
     a.Pshift = c.page_size == 16 ? 4 : (c.page_size == 32 ? 5 : 6);
     a.c = c;

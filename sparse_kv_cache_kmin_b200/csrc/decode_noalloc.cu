@@ -64,7 +64,7 @@ extern "C" ekv_status ekv_sparse_decode_noalloc(const ekv_cache *c, const void *
     if (attn != EKV_SOFTMAX && attn != EKV_ENTMAX15 && attn != EKV_SPARSEMAX)
         return EKV_ERR_UNSUPPORTED;
     if (!q || !sel_idx || !sel_count || !out || !stat || !c->v_cache || !(scale > 0.0f) ||
-        !(scale < INFINITY))
+        !(scale < INFINITY) || (((uintptr_t)q | (uintptr_t)c->k_cache | (uintptr_t)c->v_cache) & 15u))
         return EKV_ERR_INVALID_ARG;
     void *ws = nullptr;
     if (noalloc_workspace(&ws) != cudaSuccess) return EKV_ERR_CUDA;

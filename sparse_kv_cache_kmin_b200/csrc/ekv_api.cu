@@ -23,8 +23,7 @@ cudaError_t launch_sparse_decode(const ekv_cache &c, const void *q, int H_q, flo
                                  int attn, const int32_t *sel_idx, const int32_t *sel_count,
                                  int max_sel, float *out, float *stat, void *ws, cudaStream_t st,
                                  bool pdl);
-size_t decode_workspace_layout(int batch, int H_q, int H_kv, int D, int P, int max_sel,
-                               size_t *off_o, size_t *off_logits, int *CP, int *NC);
+size_t decode_workspace_bytes_all_modes(int batch, int H_q, int D, int P, int dtype, int max_sel);
 
 int persistent_grid_size(const void *kernel, int threads, size_t smem)
 {
@@ -141,8 +140,8 @@ size_t ekv_decode_workspace_bytes(const ekv_cache *c, int32_t num_q_heads, int32
 {
     if (check_cache(c, false) != EKV_OK || check_heads(c, num_q_heads) != EKV_OK || max_sel < 1)
         return 0;
-    return decode_workspace_layout(c->batch, num_q_heads, c->num_kv_heads, c->head_dim,
-                                   c->page_size, max_sel, nullptr, nullptr, nullptr, nullptr);
+    return decode_workspace_bytes_all_modes(c->batch, num_q_heads, c->head_dim, c->page_size,
+                                            c->dtype, max_sel);
 }
 
 ekv_status ekv_sparse_decode(const ekv_cache *c, const void *q, int32_t num_q_heads,
@@ -157,6 +156,9 @@ ekv_status ekv_sparse_decode(const ekv_cache *c, const void *q, int32_t num_q_he
         return EKV_ERR_UNSUPPORTED;
     if (!q || !sel_idx || !sel_count || !out || !stat || max_sel < 1 || !(scale > 0.0f) ||
         !std::isfinite(scale))
+        return EKV_ERR_INVALID_ARG;
+    // K/V page spans and the query rows are moved with bulk copies: 16-byte aligned bases
+    if (((uintptr_t)q | (uintptr_t)c->k_cache | (uintptr_t)c->v_cache) & 15u)
         return EKV_ERR_INVALID_ARG;
     if (!ws || ws_bytes < ekv_decode_workspace_bytes(c, num_q_heads, max_sel))
         return EKV_ERR_WORKSPACE;

@@ -80,18 +80,64 @@ score_topk_kernel(ekv_cache c, const void *__restrict__ q, int H_q, float scale,
     const long hi = (long)(blockIdx.x + 1) * TG / gridDim.x;
     const char *bbox = static_cast<const char *>(c.meta_bbox);
 
-    int cur_bh = -1, np = 0, bb = 0, hh = 0;
-    float coef[LPL][EPC];
-    for (long gi = lo + warp; gi < hi; gi += 8) {
-        bb = find_seq(pre, B, gi);
-        int len = c.seq_lens[bb];
+    // Work group gi -> (sequence, KV head, first page); its page-table entries are fetched
+    // one group ahead, so each group's bbox loads wait on one memory latency, not two.
+    struct Grp { int bb, hh, j0, np; };
+    auto locate = [&](long gi) {
+        Grp g;
+        g.bb = find_seq(pre, B, gi);
+        int len = c.seq_lens[g.bb];
         len = len < 0 ? 0 : (len > c.max_pages * P ? c.max_pages * P : len);
-        np = (len + P - 1) / P;
-        const int ng = (np + PG - 1) / PG;
-        const int r = (int)(gi - pre[bb]);
-        hh = r / ng;
-        const int j0 = (r % ng) * PG;
-        const int bh = bb * H + hh;
+        g.np = (len + P - 1) / P;
+        const int ng = (g.np + PG - 1) / PG;
+        const int r = (int)(gi - pre[g.bb]);
+        g.hh = r / ng;
+        g.j0 = (r % ng) * PG;
+        return g;
+    };
+    // block id of page j0 + (lane & 7): -1 past the end, -2 out of range
+    auto fetch_blk = [&](const Grp &g) {
+        int blk = -1;
+        const int jl = g.j0 + (lane & (PG - 1));
+        if (jl < g.np) {
+            blk = c.page_table[(size_t)g.bb * c.max_pages + jl];
+            if (blk < 0 || blk >= c.num_blocks) {
+                flag(c.dev_status, EKV_DEV_BAD_BLOCK);
+                blk = -2;
+            }
+        }
+        return blk;
+    };
+
+    int cur_bh = -1;
+    float coef[LPL][EPC];
+    long gi = lo + warp;
+    Grp nxt = {0, 0, 0, 0};
+    int nxt_blk = -1;
+    if (gi < hi) {
+        nxt = locate(gi);
+        nxt_blk = fetch_blk(nxt);
+    }
+    for (; gi < hi; gi += 8) {
+        const Grp cur = nxt;
+        const int myblk = nxt_blk;
+        const int bh = cur.bb * H + cur.hh;
+        uint4 x[NPL][LPL];
+#pragma unroll
+        for (int i = 0; i < NPL; ++i) {
+            const int blk = __shfl_sync(kFull, myblk, i * RPI + lane / W);
+#pragma unroll
+            for (int k = 0; k < LPL; ++k) {
+                if (blk >= 0)
+                    x[i][k] = ld_stream16(bbox + (((size_t)blk * H + cur.hh) * CPR + k * W + lane % W) * 16);
+                else
+                    x[i][k] = make_uint4(0, 0, 0, 0);
+            }
+        }
+        if (gi + 8 < hi) {
+            nxt = locate(gi + 8);
+            nxt_blk = fetch_blk(nxt);
+        }
         if (bh != cur_bh) {
             cur_bh = bh;
 #pragma unroll
@@ -104,33 +150,11 @@ score_topk_kernel(ekv_cache c, const void *__restrict__ q, int H_q, float scale,
                     float a = 0.f;
 #pragma unroll
                     for (int g = 0; g < G; ++g) {
-                        float qv = load_elem<DT>(q, ((size_t)bb * H_q + hh * G + g) * D + cb + e);
+                        float qv = load_elem<DT>(q, ((size_t)cur.bb * H_q + cur.hh * G + g) * D + cb + e);
                         a += upper ? fmaxf(qv, 0.f) : fminf(qv, 0.f);
                     }
                     coef[k][e] = a;
                 }
-            }
-        }
-        // block id of page j0 + (lane & 7): -1 past the end, -2 out of range
-        int myblk = -1;
-        const int jl = j0 + (lane & (PG - 1));
-        if (jl < np) {
-            myblk = c.page_table[(size_t)bb * c.max_pages + jl];
-            if (myblk < 0 || myblk >= c.num_blocks) {
-                flag(c.dev_status, EKV_DEV_BAD_BLOCK);
-                myblk = -2;
-            }
-        }
-        uint4 x[NPL][LPL];
-#pragma unroll
-        for (int i = 0; i < NPL; ++i) {
-            const int blk = __shfl_sync(kFull, myblk, i * RPI + lane / W);
-#pragma unroll
-            for (int k = 0; k < LPL; ++k) {
-                if (blk >= 0)
-                    x[i][k] = ld_stream16(bbox + (((size_t)blk * H + hh) * CPR + k * W + lane % W) * 16);
-                else
-                    x[i][k] = make_uint4(0, 0, 0, 0);
             }
         }
         float part[NPL];
@@ -148,8 +172,8 @@ score_topk_kernel(ekv_cache c, const void *__restrict__ q, int H_q, float scale,
         transpose_reduce<NPL, W>(part, lane);
         const int po = transpose_index<NPL, W>(lane, 0) * RPI + lane / W;
         const int blk = __shfl_sync(kFull, myblk, po);
-        if (((lane % W) % (W / NPL)) == 0 && j0 + po < np)
-            scores[(size_t)bh * c.max_pages + j0 + po] = blk >= 0 ? scale * part[0] : -INFINITY;
+        if (((lane % W) % (W / NPL)) == 0 && cur.j0 + po < cur.np)
+            scores[(size_t)bh * c.max_pages + cur.j0 + po] = blk >= 0 ? scale * part[0] : -INFINITY;
     }
     pdl_trigger();
 }

@@ -25,17 +25,109 @@ __device__ __forceinline__ uint32_t order_key(float x)
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-__global__ void __launch_bounds__(1024)
+constexpr int kSelThreads = 1024;
+constexpr int kSmemKeys = 16384;  // keys staged in shared memory (larger n reads them from L2)
+constexpr int kBoundaryMax = 256; // boundary-bin entries resolved by rank counting
+
+// Exact radix select on the order-preserving keys (11 + 11 + 10 bits) and emission of the
+// kept pages in ascending order. `key(j)` returns the key of page j.
+template <class KeyFn>
+__device__ void radix_select_emit(int n, int kk, KeyFn key, int *hist, int *warp_tot, int *s_bin,
+                                  int *s_above, int32_t *out)
+{
+    constexpr int NT = kSelThreads;
+    const int tid = threadIdx.x, lane = tid & 31;
+    uint32_t prefix = 0, mask = 0;
+    int remaining = kk;
+#pragma unroll 1
+    for (int pass = 0; pass < 3; ++pass) {
+        const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
+        const int nb = pass == 2 ? 1024 : 2048;
+        for (int i = tid; i < 2048; i += NT) hist[i] = 0;
+        __syncthreads();
+        for (int j0 = 0; j0 < n; j0 += NT) {
+            const int j = j0 + tid;
+            int bin = -1;
+            if (j < n) {
+                const uint32_t u = key(j);
+                if ((u & mask) == prefix) bin = (int)((u >> shift) & (uint32_t)(nb - 1));
+            }
+            const unsigned peers = __match_any_sync(kFull, bin);
+            if (bin >= 0 && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
+        }
+        __syncthreads();
+        const int b0 = nb - 1 - 2 * tid, b1 = nb - 2 - 2 * tid;
+        const int c0 = b0 >= 0 ? hist[b0] : 0, c1 = b1 >= 0 ? hist[b1] : 0;
+        const int incl = block_incl_scan<NT>(c0 + c1, warp_tot, nullptr);
+        const int excl = incl - c0 - c1;
+        if (c0 > 0 && excl < remaining && remaining <= excl + c0) { *s_bin = b0; *s_above = excl; }
+        if (c1 > 0 && excl + c0 < remaining && remaining <= incl) { *s_bin = b1; *s_above = excl + c0; }
+        __syncthreads();
+        remaining -= *s_above;
+        prefix |= (uint32_t)*s_bin << shift;
+        mask |= (uint32_t)(nb - 1) << shift;
+        const bool whole_bin = remaining == hist[*s_bin];
+        __syncthreads();
+        if (whole_bin) break;  // every key matching the prefix is kept: lower bits cannot matter
+    }
+    const uint32_t T = prefix;
+    auto cmp = [&](uint32_t u) -> int { const uint32_t um = u & mask; return um > T ? 1 : (um == T ? 0 : -1); };
+    // emission in page order: warp w owns a contiguous page range; ties at T are kept while
+    // their rank among all ties (in page order) is below `remaining`
+    const int warp = tid >> 5;
+    const int per = (n + 31) / 32;
+    const int j0 = warp * per, j1 = j0 + per < n ? j0 + per : n;
+    int n_above = 0, n_tie = 0;
+    for (int j = j0 + lane; j - lane < j1; j += 32) {
+        const int c = j < j1 ? cmp(key(j)) : -1;
+        n_above += __popc(__ballot_sync(kFull, c > 0));
+        n_tie += __popc(__ballot_sync(kFull, c == 0));
+    }
+    if (lane == 0) { hist[warp] = n_above; hist[32 + warp] = n_tie; }
+    __syncthreads();
+    if (warp == 0) {
+        const int a = hist[lane], t = hist[32 + lane];
+        const int ia = warp_incl_scan(a), it = warp_incl_scan(t);
+        hist[64 + lane] = ia - a;   // kept-above before this warp
+        hist[96 + lane] = it - t;   // ties before this warp
+    }
+    __syncthreads();
+    int tie_rank = hist[96 + warp];
+    int pos = hist[64 + warp] + (tie_rank < remaining ? tie_rank : remaining);
+    for (int j = j0 + lane; j - lane < j1; j += 32) {
+        const int c = j < j1 ? cmp(key(j)) : -1;
+        const unsigned tb = __ballot_sync(kFull, c == 0);
+        const bool keep = c > 0 || (c == 0 && tie_rank + __popc(tb & ((1u << lane) - 1u)) < remaining);
+        const unsigned kb = __ballot_sync(kFull, keep);
+        if (keep) out[pos + __popc(kb & ((1u << lane) - 1u))] = j;
+        pos += __popc(kb);
+        tie_rank += __popc(tb);
+    }
+    __syncthreads();
+}
+
+__global__ void __launch_bounds__(kSelThreads)
 select_topk_kernel(const float *__restrict__ scores, int H, int max_pages, int P,
                    const int32_t *__restrict__ seq_lens, int k, int32_t *__restrict__ sel_idx,
                    int32_t *__restrict__ sel_count, int max_sel, uint32_t *status)
 {
-    constexpr int NT = 1024;
+    // The keys of one (sequence, KV head) go to shared memory once (all loads in flight
+    // together). One histogram pass over 2048 bins that split the [min, max] key range evenly
+    // finds the bin holding the k-th largest key; the few keys of that bin are ranked exactly
+    // by (key descending, page ascending). Heavy ties (a large boundary bin) or more than
+    // kSmemKeys pages take the three-pass radix select instead.
+    constexpr int NT = kSelThreads;
+    constexpr int NB = 2048;
+    extern __shared__ uint32_t keys[];  // [min(n, kSmemKeys)]
     __shared__ int hist[2048];
     __shared__ int warp_tot[32];
-    __shared__ int s_bin, s_above;
+    __shared__ int s_bin, s_above, s_cnt;
+    __shared__ uint32_t s_umin, s_umax;
+    __shared__ uint32_t bu[kBoundaryMax];
+    __shared__ int bj[kBoundaryMax];
+    __shared__ uint32_t kept_bits[kSmemKeys / 32];
     pdl_wait();
-    const int tid = threadIdx.x, lane = tid & 31;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int h = blockIdx.x, b = blockIdx.y;
     const int bh = b * H + h;
     const int n = seq_pages(seq_lens, b, P, max_pages, h == 0 ? status : nullptr, nullptr);
@@ -49,59 +141,118 @@ select_topk_kernel(const float *__restrict__ scores, int H, int max_pages, int P
         pdl_trigger();
         return;
     }
+    if (n > kSmemKeys) {
+        radix_select_emit(n, kk, [&](int j) { return order_key(__ldcg(S + j)); }, hist, warp_tot,
+                          &s_bin, &s_above, out);
+        for (int j = kk + tid; j < max_sel; j += NT) out[j] = -1;
+        if (tid == 0) sel_count[bh] = kk;
+        pdl_trigger();
+        return;
+    }
 
-    uint32_t prefix = 0, mask = 0;
-    int remaining = kk;
-    const int shifts[3] = {21, 10, 0};
-    const int widths[3] = {11, 11, 10};
-#pragma unroll 1
-    for (int pass = 0; pass < 3; ++pass) {
-        const int shift = shifts[pass], nb = 1 << widths[pass];
-        for (int i = tid; i < 2048; i += NT) hist[i] = 0;
-        __syncthreads();
-        for (int j0 = 0; j0 < n; j0 += NT) {
-            const int j = j0 + tid;
-            int bin = -1;
-            if (j < n) {
-                const uint32_t u = order_key(S[j]);
-                if ((u & mask) == prefix) bin = (int)((u >> shift) & (uint32_t)(nb - 1));
+    uint32_t umin = 0xffffffffu, umax = 0;
+    if ((max_pages & 3) == 0) {
+        const float4 *S4 = reinterpret_cast<const float4 *>(S);
+        const int n4 = n >> 2;
+#pragma unroll 4
+        for (int i = tid; i < n4; i += NT) {
+            const float4 v = __ldcg(S4 + i);
+            const uint32_t u0 = order_key(v.x), u1 = order_key(v.y), u2 = order_key(v.z), u3 = order_key(v.w);
+            keys[4 * i] = u0; keys[4 * i + 1] = u1; keys[4 * i + 2] = u2; keys[4 * i + 3] = u3;
+            umin = min(min(umin, u0), min(u1, min(u2, u3)));
+            umax = max(max(umax, u0), max(u1, max(u2, u3)));
+        }
+        for (int j = 4 * n4 + tid; j < n; j += NT) {
+            const uint32_t u = order_key(__ldcg(S + j));
+            keys[j] = u;
+            umin = min(umin, u);
+            umax = max(umax, u);
+        }
+    } else {
+#pragma unroll 4
+        for (int j = tid; j < n; j += NT) {
+            const uint32_t u = order_key(__ldcg(S + j));
+            keys[j] = u;
+            umin = min(umin, u);
+            umax = max(umax, u);
+        }
+    }
+    for (int i = tid; i < NB; i += NT) hist[i] = 0;
+    for (int i = tid; i < kSmemKeys / 32; i += NT) kept_bits[i] = 0;
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+        umin = min(umin, __shfl_xor_sync(kFull, umin, o));
+        umax = max(umax, __shfl_xor_sync(kFull, umax, o));
+    }
+    if (tid == 0) { s_umin = 0xffffffffu; s_umax = 0; s_cnt = 0; }
+    __syncthreads();
+    if (lane == 0) { atomicMin(&s_umin, umin); atomicMax(&s_umax, umax); }
+    __syncthreads();
+    umin = s_umin;
+    umax = s_umax;
+    // monotone bin of a key: floor((u - umin) * NB / (umax - umin + 1)) in fp32 (rounding is
+    // monotone, so equal keys share a bin and bin order never contradicts key order)
+    const float bscale = (float)NB / ((float)(umax - umin) + 1.0f);
+    auto bin_of = [&](uint32_t u) {
+        const int bb = (int)((float)(u - umin) * bscale);
+        return bb < NB - 1 ? bb : NB - 1;
+    };
+
+    for (int j = tid; j < n; j += NT) atomicAdd(&hist[bin_of(keys[j])], 1);
+    __syncthreads();
+    // counts in descending bin order: thread t owns bins NB-1-2t and NB-2-2t
+    const int b0 = NB - 1 - 2 * tid, b1 = NB - 2 - 2 * tid;
+    const int c0 = b0 >= 0 ? hist[b0] : 0, c1 = b1 >= 0 ? hist[b1] : 0;
+    const int incl = block_incl_scan<NT>(c0 + c1, warp_tot, nullptr);
+    const int excl = incl - c0 - c1;
+    if (c0 > 0 && excl < kk && kk <= excl + c0) { s_bin = b0; s_above = excl; }
+    if (c1 > 0 && excl + c0 < kk && kk <= incl) { s_bin = b1; s_above = excl + c0; }
+    __syncthreads();
+    const int B = s_bin, r = kk - s_above, cB = hist[B];
+
+    if (cB > kBoundaryMax) {  // heavy ties around the k-th key
+        radix_select_emit(n, kk, [&](int j) { return keys[j]; }, hist, warp_tot, &s_bin,
+                          &s_above, out);
+    } else {
+        for (int j = tid; j < n; j += NT)
+            if (bin_of(keys[j]) == B) {
+                const int pos = atomicAdd(&s_cnt, 1);
+                bu[pos] = keys[j];
+                bj[pos] = j;
             }
-            const unsigned peers = __match_any_sync(kFull, bin);
-            if (bin >= 0 && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
+        __syncthreads();
+        if (tid < cB) {
+            const uint32_t u = bu[tid];
+            const int j = bj[tid];
+            int rank = 0;
+            for (int m = 0; m < cB; ++m) rank += bu[m] > u || (bu[m] == u && bj[m] < j);
+            if (rank < r) atomicOr(&kept_bits[j >> 5], 1u << (j & 31));
         }
         __syncthreads();
-        // counts in descending bin order: thread t owns positions 2t and 2t+1
-        const int b0 = nb - 1 - 2 * tid, b1 = nb - 2 - 2 * tid;
-        const int c0 = b0 >= 0 ? hist[b0] : 0, c1 = b1 >= 0 ? hist[b1] : 0;
-        const int incl = block_incl_scan<NT>(c0 + c1, warp_tot, nullptr);
-        const int excl = incl - c0 - c1;
-        if (c0 > 0 && excl < remaining && remaining <= excl + c0) { s_bin = b0; s_above = excl; }
-        if (c1 > 0 && excl + c0 < remaining && remaining <= incl) { s_bin = b1; s_above = excl + c0; }
+        // emission in page order: warp w owns a contiguous page range
+        const int per = (n + 31) / 32;
+        const int j0 = warp * per, j1 = j0 + per < n ? j0 + per : n;
+        auto kept = [&](int j) {
+            const int bb = bin_of(keys[j]);
+            return bb > B || (bb == B && (kept_bits[j >> 5] >> (j & 31) & 1u));
+        };
+        int mine = 0;
+        for (int j = j0 + lane; j - lane < j1; j += 32)
+            mine += __popc(__ballot_sync(kFull, j < j1 && kept(j)));
+        if (lane == 0) warp_tot[warp] = mine;
         __syncthreads();
-        remaining -= s_above;
-        prefix |= (uint32_t)s_bin << shift;
-        mask |= (uint32_t)(nb - 1) << shift;
+        if (warp == 0) {
+            const int v = warp_tot[lane];
+            warp_tot[lane] = warp_incl_scan(v) - v;
+        }
         __syncthreads();
-    }
-    // prefix is now the k-th largest key T; `remaining` keys equal to T are kept (lowest
-    // page indices first).
-    const uint32_t T = prefix;
-    const int E = (n + NT - 1) / NT;
-    const int j0 = tid * E, j1 = j0 + E < n ? j0 + E : n;
-    int eq = 0;
-    for (int j = j0; j < j1; ++j) eq += order_key(S[j]) == T;
-    const int eq_before = block_incl_scan<NT>(eq, warp_tot, nullptr) - eq;
-    int mine = 0, seen = eq_before;
-    for (int j = j0; j < j1; ++j) {
-        const uint32_t u = order_key(S[j]);
-        if (u > T) ++mine;
-        else if (u == T && seen++ < remaining) ++mine;
-    }
-    int pos = block_incl_scan<NT>(mine, warp_tot, nullptr) - mine;
-    seen = eq_before;
-    for (int j = j0; j < j1; ++j) {
-        const uint32_t u = order_key(S[j]);
-        if (u > T || (u == T && seen++ < remaining)) out[pos++] = j;
+        int pos = warp_tot[warp];
+        for (int j = j0 + lane; j - lane < j1; j += 32) {
+            const bool keep = j < j1 && kept(j);
+            const unsigned kb = __ballot_sync(kFull, keep);
+            if (keep) out[pos + __popc(kb & ((1u << lane) - 1u))] = j;
+            pos += __popc(kb);
+        }
     }
     for (int j = kk + tid; j < max_sel; j += NT) out[j] = -1;
     if (tid == 0) sel_count[bh] = kk;
@@ -280,6 +431,14 @@ cudaError_t launch_select_pages(const ekv_cache &c, int H_q, int policy, int top
     const dim3 grid(c.num_kv_heads, c.batch);
     if (policy == EKV_SEL_TOPK) {
         cudaLaunchConfig_t cfg = pdl_config(grid, dim3(1024), st, pdl, attr);
+        const int keys = c.max_pages < kSmemKeys ? c.max_pages : kSmemKeys;
+        cfg.dynamicSmemBytes = sizeof(uint32_t) * keys;
+        static bool attr_set = false;
+        if (!attr_set) {
+            cudaFuncSetAttribute(select_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kSmemKeys * (int)sizeof(uint32_t));
+            attr_set = true;
+        }
         return cudaLaunchKernelEx(&cfg, select_topk_kernel, scores, c.num_kv_heads, c.max_pages,
                                   c.page_size, c.seq_lens, topk, sel_idx, sel_count, max_sel,
                                   c.dev_status);

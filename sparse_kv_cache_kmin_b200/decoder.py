@@ -43,6 +43,18 @@ class SparseDecoder:
                         stream=None):
         ekv.ekv_page_meta_update(self.cache, new_start, new_count, max_new, stream)
 
+    def capture(self, q_static: torch.Tensor, pre_step=None) -> torch.cuda.CUDAGraph:
+        """Capture one decode step reading `q_static` into a CUDA graph (one launch per step
+        on replay instead of one host call per kernel). `pre_step`, if given, is called inside
+        the capture first (e.g. a metadata update of an appended page). Run one eager step
+        before capturing so that one-time set-up happens outside the capture."""
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            if pre_step is not None:
+                pre_step()
+            self.step(q_static)
+        return g
+
     def step(self, q: torch.Tensor, stream=None):
         c = self.cache
         ekv.ekv_score_pages(c, q, self.num_q_heads, self.scale, self.policy, self.scores, stream)

@@ -28,6 +28,7 @@ EKV_SOFTMAX, EKV_ENTMAX15, EKV_SPARSEMAX = 0, 1, 2
 EKV_SEL_TOPK, EKV_SEL_GAUSS = 0, 1
 EKV_DEV_BAD_BLOCK, EKV_DEV_BAD_LEN, EKV_DEV_BAD_SEL, EKV_DEV_SEL_OVERFLOW, EKV_DEV_BAD_RANGE = \
     0x1, 0x2, 0x4, 0x8, 0x10
+EKV_DEV_TIMEOUT = 0x20
 ALPHA = {EKV_SOFTMAX: 1.0, EKV_ENTMAX15: 1.5, EKV_SPARSEMAX: 2.0}
 
 EXPORTED = ["ekv_page_meta_update", "ekv_score_pages", "ekv_select_pages", "ekv_sparse_decode",
@@ -160,6 +161,18 @@ class PagedKVCache:
         return self.page_table.shape[1]
 
     def struct(self) -> EkvCacheStruct:
+        """The C view of the cache; rebuilt only when a tensor of it is replaced."""
+        key = tuple((t.data_ptr(), tuple(t.shape), t.dtype) if t is not None else None
+                    for t in (self.k_cache, self.v_cache, self.meta_bbox, self.meta_mom,
+                              self.page_table, self.seq_lens, self.dev_status))
+        cached = self.__dict__.get("_struct_cache")
+        if cached is not None and cached[0] == key:
+            return cached[1]
+        s = self._build_struct()
+        self.__dict__["_struct_cache"] = (key, s)
+        return s
+
+    def _build_struct(self) -> EkvCacheStruct:
         if self.k_cache.dtype == torch.float32:
             dt = EKV_F32
         elif self.k_cache.dtype == torch.bfloat16:
