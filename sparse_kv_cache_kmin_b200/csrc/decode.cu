@@ -25,33 +25,11 @@
 //            the support S = {z > tau} and recomputes tau in closed form over S in fp64
 //            (sparsemax: (sum_S z - 1) / |S|; 1.5-entmax: mean_S - sqrt((1 - sum_S (z -
 //            mean_S)^2) / |S|)), repeating until S is stable. Only the V rows of S are read.
-#include "ekv_device.cuh"
+#include "decode.cuh"
 
 namespace ekv {
 
-struct DecodeArgs {
-    ekv_cache c;
-    const void *q;
-    int H_q;
-    float qscale;  // softmax: scale * log2(e); entmax: scale * (alpha - 1)
-    float alpha;
-    const int32_t *sel_idx;
-    const int32_t *sel_count;
-    int max_sel;
-    int CP;         // pages per chunk
-    int NC;         // chunks per (sequence, KV head) at most
-    int LS;         // logits row stride: NC * CP * P
-    int Pshift;     // log2(P)
-    int stages;     // pipeline stages of the chunk kernel (2 or 3)
-    float *part_ml; // [B * H_q][NC][2]   softmax (m, l); entmax (max z, unused)
-    float *part_o;  // [B * H_q][NC][D]   softmax sum p v
-    float *logits;  // [B * H_q][LS]       entmax z
-    float *out;
-    float *stat;
-};
-
 constexpr int kNW = 8;         // consumer warps per CTA
-constexpr int kMaxCP = 16;     // pages per chunk at most
 constexpr int kThreads = (kNW + 1) * 32;
 
 // Tokens per chunk: a K tile (entmax) or a K + V tile (softmax) of about 32 KiB per pipeline
@@ -418,53 +396,89 @@ __device__ void finish_softmax(const DecodeArgs &a, int b, int hq, int nchunks)
 
 constexpr int kCapW = 512;  // gathered logits per warp kept in shared memory
 
-// Exact threshold of <= 32 candidates, one per lane (x = z - zmax, -inf padding): sort
-// descending across the warp, prefix sums of x and x^2, then the largest k whose closed-form
-// tau(k) satisfies tau(k) <= x_(k) (1.5-entmax also needs a real root).
-__device__ __forceinline__ double warp_exact_tau(float x, int cnt, bool sparsemax)
+// Exact threshold of at most 32*R candidates held R per lane (element e = r*32 + lane; x =
+// z - zmax, -inf padding): bitonic sort descending across registers and lanes, prefix sums of
+// x and x^2 in sorted order, then the largest k whose closed-form tau(k) satisfies
+// tau(k) <= x_(k) (1.5-entmax also needs a real root).
+template <int R>
+__device__ __forceinline__ double warp_exact_tau(float (&v)[R], int cnt, bool sparsemax)
 {
     const int lane = threadIdx.x & 31;
+    constexpr int N = 32 * R;
 #pragma unroll
-    for (int k = 2; k <= 32; k <<= 1)
+    for (int k = 2; k <= N; k <<= 1) {
 #pragma unroll
         for (int j = k >> 1; j > 0; j >>= 1) {
-            const float o = __shfl_xor_sync(kFull, x, j);
-            const bool up = (lane & k) == 0, lower = (lane & j) == 0;
-            x = (lower == up) ? fmaxf(x, o) : fminf(x, o);
-        }
-    const bool in = lane < cnt;
-    const double xd = in ? (double)x : 0.0;
-    double s1 = xd, s2 = xd * xd;
+            if (j >= 32) {
+                const int rj = j / 32;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const double t1 = __shfl_up_sync(kFull, s1, o), t2 = __shfl_up_sync(kFull, s2, o);
-        if (lane >= o) { s1 += t1; s2 += t2; }
+                for (int r = 0; r < R; ++r) {
+                    if (r & rj) continue;
+                    const int e = r * 32 + lane;
+                    const bool up = (e & k) == 0;
+                    const float hi = fmaxf(v[r], v[r | rj]), lo = fminf(v[r], v[r | rj]);
+                    v[r] = up ? hi : lo;
+                    v[r | rj] = up ? lo : hi;
+                }
+            } else {
+#pragma unroll
+                for (int r = 0; r < R; ++r) {
+                    const int e = r * 32 + lane;
+                    const float o = __shfl_xor_sync(kFull, v[r], j);
+                    const bool up = (e & k) == 0, lower = (lane & j) == 0;
+                    v[r] = (lower == up) ? fmaxf(v[r], o) : fminf(v[r], o);
+                }
+            }
+        }
     }
-    const double k = lane + 1;
-    double tk;
-    bool ok = in;
-    if (sparsemax) {
-        tk = (s1 - 1.0) / k;
-    } else {
-        const double mean = s1 / k;
-        const double m2 = s2 - s1 * mean;  // sum of squared deviations of the top k
-        const double disc = (1.0 - m2) / k;
-        ok = ok && disc >= 0.0;
-        tk = mean - sqrt(disc > 0.0 ? disc : 0.0);
+    double carry1 = 0.0, carry2 = 0.0;
+    int best = -1;
+    double best_t = 0.0;
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        const int e = r * 32 + lane;
+        const bool in = e < cnt;
+        const double xd = in ? (double)v[r] : 0.0;
+        double s1 = xd, s2 = xd * xd;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const double t1 = __shfl_up_sync(kFull, s1, o), t2 = __shfl_up_sync(kFull, s2, o);
+            if (lane >= o) { s1 += t1; s2 += t2; }
+        }
+        s1 += carry1;
+        s2 += carry2;
+        carry1 = __shfl_sync(kFull, s1, 31);
+        carry2 = __shfl_sync(kFull, s2, 31);
+        const double kk = e + 1;
+        double tk;
+        bool ok = in;
+        if (sparsemax) {
+            tk = (s1 - 1.0) / kk;
+        } else {
+            const double mean = s1 / kk;
+            const double m2 = s2 - s1 * mean;  // sum of squared deviations of the top k
+            const double disc = (1.0 - m2) / kk;
+            ok = ok && disc >= 0.0;
+            tk = mean - sqrt(disc > 0.0 ? disc : 0.0);
+        }
+        ok = ok && tk <= (double)v[r];
+        const unsigned bal = __ballot_sync(kFull, ok);
+        if (bal) {  // a later row's valid k beats an earlier one
+            const int K = 31 - __clz(bal);
+            best = r * 32 + K;
+            best_t = __shfl_sync(kFull, tk, K);
+        }
     }
-    ok = ok && tk <= (double)x;
-    const unsigned bal = __ballot_sync(kFull, ok);
-    const int K = 31 - __clz(bal);  // lane 0 is always valid: tau(1) = x_(1) - 1
-    return __shfl_sync(kFull, tk, K);
+    return best_t;  // element 0 is always valid: tau(1) = x_(1) - 1
 }
 
-// Entmax finish for one (sequence, query head), one CTA: the eight warps gather the logits
-// above max z - 1 (only those can carry weight) from contiguous slot ranges into per-warp lists
-// in shared memory; warp 0 finds tau (exact sort for <= 32 candidates, else fp32 Newton then a
-// closed-form fp64 polish over the support); then every warp accumulates p_i v_i over the
-// support entries of its own list, resolving their page-table look-ups 32 at a time and
-// keeping several V rows in flight. A warp whose list overflows walks its slot range in global
-// memory instead (correct, slower).
+// Exact threshold of <= 32 candidates, one per lane.
+__device__ __forceinline__ double warp_exact_tau(float x, int cnt, bool sparsemax)
+{
+    float v[1] = {x};
+    return warp_exact_tau<1>(v, cnt, sparsemax);
+}
+
 template <int DT, int D>
 __device__ void finish_entmax_cta(const DecodeArgs &a, int b, int h, int hq, int nsel, int nchunks)
 {
@@ -526,16 +540,68 @@ __device__ void finish_entmax_cta(const DecodeArgs &a, int b, int h, int hq, int
     if (lane == 0) cn[warp] = cnt;
     __syncthreads();
 
+    // tau: the exact threshold of any subset of the logits is a lower bound on the threshold of
+    // all of them (adding tokens can only raise it), so each warp solves exactly over up to 32
+    // of its surviving candidates, the largest of these bounds filters every list, and once at
+    // most 32 candidates survive, warp 0 solves exactly over them -- which is the threshold of
+    // the whole set, as everything filtered out lies at or below it.
+    const bool over = cnt > kCapW;
+    bool any_over = false;
+#pragma unroll
+    for (int w = 0; w < kNW; ++w) any_over |= cn[w] > kCapW;
+    __shared__ float lb_w[kNW];
+    if (!any_over) {
+        for (int i = lane; i < cnt; i += 32) cz[warp][i] -= zmax;  // lists now hold x = z - zmax
+        __syncthreads();
+#pragma unroll 1
+        for (int round = 0; round < 6; ++round) {
+            // lower bound from this warp's first (up to) 32 candidates
+            const int nw = cn[warp];
+            const float xv = lane < nw ? cz[warp][lane] : -INFINITY;
+            const double tw = nw > 0 ? warp_exact_tau(xv, nw < 32 ? nw : 32, sparsemax) : -INFINITY;
+            if (lane == 0) lb_w[warp] = (float)tw;
+            __syncthreads();
+            float lb = -1.0f;
+#pragma unroll
+            for (int w = 0; w < kNW; ++w) lb = fmaxf(lb, lb_w[w]);
+            // keep x > lb (rounded down a little so fp32 rounding of the bound never drops a
+            // support member)
+            lb = lb - 1e-6f * fmaxf(1.0f, fabsf(lb));
+            int kept = 0;
+            for (int i0 = 0; i0 < nw; i0 += 32) {
+                const int i = i0 + lane;
+                const float x = i < nw ? cz[warp][i] : -INFINITY;
+                const int sl = i < nw ? cs[warp][i] : 0;
+                const bool keep = x > lb;
+                const unsigned bal = __ballot_sync(kFull, keep);
+                __syncwarp();
+                if (keep) {
+                    const int pos = kept + __popc(bal & ((1u << lane) - 1u));
+                    cz[warp][pos] = x;
+                    cs[warp][pos] = sl;
+                }
+                kept += __popc(bal);
+                __syncwarp();
+            }
+            __syncthreads();
+            if (lane == 0) cn[warp] = kept;
+            __syncthreads();
+            int total = 0;
+#pragma unroll
+            for (int w = 0; w < kNW; ++w) total += cn[w];
+            if (total <= 128) break;
+            if (round == 5) break;
+        }
+    }
     if (warp == 0) {
         int total = 0;
-        bool any_over = false;
 #pragma unroll
-        for (int w = 0; w < kNW; ++w) { total += cn[w]; any_over |= cn[w] > kCapW; }
-        // every gathered logit, shifted by zmax
+        for (int w = 0; w < kNW; ++w) total += cn[w];
+        // every candidate, shifted by zmax
         auto visit = [&](auto &&fn) {
             for (int w = 0; w < kNW; ++w) {
                 if (cn[w] <= kCapW) {
-                    for (int i = lane; i < cn[w]; i += 32) fn(cz[w][i] - zmax);
+                    for (int i = lane; i < cn[w]; i += 32) fn(any_over ? cz[w][i] - zmax : cz[w][i]);
                 } else {
                     const int a0 = w * per, a1 = min(a0 + per, nslots);
                     for (int sl = a0 + lane; sl < a1; sl += 32) {
@@ -546,20 +612,26 @@ __device__ void finish_entmax_cta(const DecodeArgs &a, int b, int h, int hq, int
             }
         };
         double tau;  // in the shifted domain x = z - zmax
-        if (!any_over && total <= 32) {
-            // lane i takes the i-th candidate in warp order
-            float x = -INFINITY;
-            int base = 0;
+        if (!any_over && total <= 128) {
+            // element e = r * 32 + lane takes the e-th candidate in warp order
+            float x[4];
 #pragma unroll
-            for (int w = 0; w < kNW; ++w) {
-                if (lane >= base && lane < base + cn[w]) x = cz[w][lane - base] - zmax;
-                base += cn[w];
+            for (int r = 0; r < 4; ++r) {
+                const int e = r * 32 + lane;
+                x[r] = -INFINITY;
+                int base = 0;
+#pragma unroll
+                for (int w = 0; w < kNW; ++w) {
+                    if (e >= base && e < base + cn[w]) x[r] = cz[w][e - base];
+                    base += cn[w];
+                }
             }
-            tau = warp_exact_tau(x, total, sparsemax);
+            tau = total <= 32 ? warp_exact_tau(x[0], total, sparsemax)
+                              : warp_exact_tau<4>(x, total, sparsemax);
         } else {
             float t = -1.0f;
 #pragma unroll 1
-            for (int it = 0; it < 40; ++it) {
+            for (int it = 0; it < 24; ++it) {
                 float f = 0.f, df = 0.f;
                 visit([&](float x) {
                     const float r = x - t;
@@ -570,11 +642,11 @@ __device__ void finish_entmax_cta(const DecodeArgs &a, int b, int h, int hq, int
                 if (!(f > 0.f) || !(df > 0.f)) break;
                 const float step = f / df;
                 t += step;
-                if (!(step > 1e-6f)) break;
+                if (!(step > 1e-5f * fmaxf(1.0f, fabsf(t)))) break;
             }
             tau = t;
 #pragma unroll 1
-            for (int round = 0; round < 4; ++round) {
+            for (int round = 0; round < 3; ++round) {
                 double n = 0.0, s1d = 0.0;
                 visit([&](float x) { if ((double)x > tau) { n += 1.0; s1d += x; } });
                 n = warp_sum(n);
@@ -610,17 +682,17 @@ __device__ void finish_entmax_cta(const DecodeArgs &a, int b, int h, int hq, int
     float acc[EPC];
 #pragma unroll
     for (int e = 0; e < EPC; ++e) acc[e] = 0.f;
-    const bool over = cnt > kCapW;
     float *sp = cz[warp];  // compacted support weights, in place over the gathered list
     int *sr = cs[warp];    // and rows as blk * P + t
-    const int total = over ? s1 - s0 : cnt;
+    const int total = over ? s1 - s0 : cn[warp];
     for (int i0 = 0; i0 < total; i0 += 32) {
         const int i = i0 + lane;
         float v = -INFINITY;
         int slot = 0;
         if (i < total) {
             if (over) { slot = s0 + i; v = __ldcg(z + slot); }
-            else { slot = cs[warp][i]; v = cz[warp][i]; }
+            else if (any_over) { slot = cs[warp][i]; v = cz[warp][i]; }
+            else { slot = cs[warp][i]; v = cz[warp][i] + zmax; }
         }
         const double r = (double)v - tau_z;
         const bool keep = r > 0.0;
@@ -711,7 +783,8 @@ static size_t mode_layout(int batch, int H_q, int D, int P, int dtype, int max_s
                           size_t *off_o, size_t *off_logits, int *CP, int *NC)
 {
     const int rb = D * (dtype == EKV_BF16 ? 2 : 4);
-    const int cp = chunk_tokens(rb, P, softmax) / P;
+    // bf16 entmax chunks are one 128-token tensor-core tile
+    const int cp = (dtype == EKV_BF16 && !softmax) ? 128 / P : chunk_tokens(rb, P, softmax) / P;
     const int nc = (max_sel + cp - 1) / cp;
     const size_t BQ = (size_t)batch * H_q;
     size_t off = align256(BQ * nc * 2 * sizeof(float));
@@ -757,6 +830,9 @@ static cudaError_t launch_chunk(const DecodeArgs &a, cudaLaunchConfig_t cfg)
     return cudaLaunchKernelEx(&cfg, k, a2);
 }
 
+bool tc_chunk_supported(const ekv_cache &c, int H_q, bool softmax);
+cudaError_t launch_chunk_tc(const DecodeArgs &a, int G, cudaLaunchConfig_t cfg);
+
 template <int DT, int D, int G>
 static cudaError_t launch_decode_t(const DecodeArgs &a, bool softmax, cudaStream_t st, bool pdl)
 {
@@ -767,7 +843,13 @@ static cudaError_t launch_decode_t(const DecodeArgs &a, bool softmax, cudaStream
     cfg.stream = st;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    cudaError_t e = softmax ? launch_chunk<DT, D, G, true>(a, cfg) : launch_chunk<DT, D, G, false>(a, cfg);
+    cudaError_t e;
+    if (softmax)
+        e = launch_chunk<DT, D, G, true>(a, cfg);
+    else if (DT == EKV_BF16 && tc_chunk_supported(a.c, a.H_q, false))
+        e = launch_chunk_tc(a, G, cfg);
+    else
+        e = launch_chunk<DT, D, G, false>(a, cfg);
     if (e != cudaSuccess) return e;
     cfg.blockDim = dim3(256);
     cfg.dynamicSmemBytes = 0;
