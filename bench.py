@@ -250,11 +250,10 @@ def oracle_sample(wl, attn, budget_s, max_heads=None):
 # ----------------------------------------------------------------------------- main
 def main():
     args = parse()
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-
+    from sparse_kv_cache_kmin_b200 import replicas
     from sparse_kv_cache_kmin_b200.workloads import make
+
+    rank, world, local = replicas.rank_info()
 
     if args.impl == "reference":
         return reference_arm(args, rank, world, make)
@@ -274,9 +273,7 @@ def main():
         pg = dist
 
     kw = {"B": args.batch} if args.batch else {}
-    wl = make(args.workload, device=dev, seed={"tiny": 1, "gqa32k": 2, "needle128k": 3,
-                                                "gauss": 4, "long1m": 5}[args.workload] + 1000 * rank,
-              **kw)
+    wl = make(args.workload, device=dev, seed=replicas.workload_seed(args.workload, rank), **kw)
     attn = wl.attn_modes[0] if args.attn is None else args.attn
     nb, H, P, d = wl.k_cache.shape
     cache = ekv.PagedKVCache(
@@ -363,11 +360,7 @@ def main():
             torch.cuda.synchronize()
             for k, j in [("meta", 0), ("score", 1), ("select", 2), ("decode", 3)]:
                 part_ms[k].append(evb[j].elapsed_time(evb[j + 1]))
-    total_s = sum(step_ms) / 1e3
-    if pg:
-        t = torch.tensor([total_s], device=dev, dtype=torch.float64)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        total_s = float(t.item())
+    total_s = replicas.max_over_ranks(sum(step_ms) / 1e3, device=dev)
     st, bits = ekv.ekv_device_status(cache)
     if st != ekv.EKV_OK:
         raise RuntimeError("device status 0x%x after timing" % bits)
@@ -398,11 +391,7 @@ def main():
         if i >= 3:
             e2e_ev[i - 3][1].record(stream)
         stream.synchronize()
-    e2e_s = sum(a.elapsed_time(b) for a, b in e2e_ev) / 1e3
-    if pg:
-        t = torch.tensor([e2e_s], device=dev, dtype=torch.float64)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        e2e_s = float(t.item())
+    e2e_s = replicas.max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e_ev) / 1e3, device=dev)
     d2h = out_host.numel() * 4 + stat_host.numel() * 4
 
     if rank != 0:
@@ -419,7 +408,7 @@ def main():
     traffic = ncu_traffic("score.cu", "score_pages_needle128k.md", total_pages * H) \
         if args.workload == "needle128k" else None
     achieved = by["score"] / score_s / 1e9
-    value = world * args.steps / total_s
+    value = replicas.job_rate(args.steps, world, total_s)
     ms = total_s / args.steps * 1e3
     cpu = None
     if not args.no_cpu_baseline and world == 1:
@@ -450,7 +439,7 @@ def main():
                      "algorithmic_bytes_per_launch": by["score"]},
         "decode_kernel": {"achieved_GBps": by["decode"] / decode_s / 1e9,
                           "frac": by["decode"] / decode_s / 1e9 / peak},
-        "e2e": {"value": world * args.steps / e2e_s, "unit": "steps/s",
+        "e2e": {"value": replicas.job_rate(args.steps, world, e2e_s), "unit": "steps/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * args.steps,
         "launch": "one CUDA graph per step (programmatic dependent launch between its kernels)",
@@ -468,8 +457,8 @@ def reference_arm(args, rank, world, make):
     if rank != 0:
         return
     dev = "cuda" if torch.cuda.is_available() else "cpu"
-    seed = {"tiny": 1, "gqa32k": 2, "needle128k": 3, "gauss": 4, "long1m": 5}[args.workload]
-    wl = make(args.workload, device=dev, seed=seed)
+    from sparse_kv_cache_kmin_b200 import replicas
+    wl = make(args.workload, device=dev, seed=replicas.workload_seed(args.workload, 0))
     attn = wl.attn_modes[0] if args.attn is None else args.attn
     n_steps = max(args.warmup, 3) + args.steps
     budget = max(2.0, 150.0 / n_steps)  # the whole run stays within a few minutes

@@ -108,6 +108,7 @@ typedef struct {
  *                         longer than max_new, or outside [0, seq_lens[b]], is clamped and
  *                         flagged EKV_DEV_BAD_RANGE.
  * Prefill: new_start = 0, new_count = seq_lens, max_new = max(seq_lens).
+ * c->k_cache must be 16-byte aligned (EKV_ERR_INVALID_ARG otherwise).
  */
 ekv_status ekv_page_meta_update(const ekv_cache *c, const int32_t *new_start,
                                 const int32_t *new_count, int32_t max_new, void *stream);

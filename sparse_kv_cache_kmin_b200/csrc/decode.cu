@@ -397,9 +397,11 @@ __device__ void finish_softmax(const DecodeArgs &a, int b, int hq, int nchunks)
 constexpr int kCapW = 512;  // gathered logits per warp kept in shared memory
 
 // Exact threshold of at most 32*R candidates held R per lane (element e = r*32 + lane; x =
-// z - zmax, -inf padding): bitonic sort descending across registers and lanes, prefix sums of
-// x and x^2 in sorted order, then the largest k whose closed-form tau(k) satisfies
-// tau(k) <= x_(k) (1.5-entmax also needs a real root).
+// z - zmax in [-1, 0], -inf padding): bitonic sort descending across registers and lanes,
+// prefix sums of x and x^2 in sorted order, then the largest k whose closed-form tau(k)
+// satisfies tau(k) <= x_(k) (1.5-entmax also needs a real root). fp32 throughout: with x in
+// [-1, 0] and at most 128 terms the sums carry ~1e-5 absolute error, far inside the output
+// tolerances, and fp32 keeps the dependent chain short.
 template <int R>
 __device__ __forceinline__ double warp_exact_tau(float (&v)[R], int cnt, bool sparsemax)
 {
@@ -431,45 +433,39 @@ __device__ __forceinline__ double warp_exact_tau(float (&v)[R], int cnt, bool sp
             }
         }
     }
-    double carry1 = 0.0, carry2 = 0.0;
-    int best = -1;
-    double best_t = 0.0;
+    float carry1 = 0.f, carry2 = 0.f, best_t = 0.f;
 #pragma unroll
     for (int r = 0; r < R; ++r) {
         const int e = r * 32 + lane;
         const bool in = e < cnt;
-        const double xd = in ? (double)v[r] : 0.0;
-        double s1 = xd, s2 = xd * xd;
+        const float xd = in ? v[r] : 0.f;
+        float s1 = xd, s2 = xd * xd;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-            const double t1 = __shfl_up_sync(kFull, s1, o), t2 = __shfl_up_sync(kFull, s2, o);
+            const float t1 = __shfl_up_sync(kFull, s1, o), t2 = __shfl_up_sync(kFull, s2, o);
             if (lane >= o) { s1 += t1; s2 += t2; }
         }
         s1 += carry1;
         s2 += carry2;
         carry1 = __shfl_sync(kFull, s1, 31);
         carry2 = __shfl_sync(kFull, s2, 31);
-        const double kk = e + 1;
-        double tk;
+        const float kk = (float)(e + 1);
+        float tk;
         bool ok = in;
         if (sparsemax) {
-            tk = (s1 - 1.0) / kk;
+            tk = (s1 - 1.0f) / kk;
         } else {
-            const double mean = s1 / kk;
-            const double m2 = s2 - s1 * mean;  // sum of squared deviations of the top k
-            const double disc = (1.0 - m2) / kk;
-            ok = ok && disc >= 0.0;
-            tk = mean - sqrt(disc > 0.0 ? disc : 0.0);
+            const float mean = s1 / kk;
+            const float m2 = fmaxf(s2 - s1 * mean, 0.f);  // sum of squared deviations of the top k
+            const float disc = (1.0f - m2) / kk;
+            ok = ok && disc >= 0.f;
+            tk = mean - sqrtf(fmaxf(disc, 0.f));
         }
-        ok = ok && tk <= (double)v[r];
+        ok = ok && tk <= v[r];
         const unsigned bal = __ballot_sync(kFull, ok);
-        if (bal) {  // a later row's valid k beats an earlier one
-            const int K = 31 - __clz(bal);
-            best = r * 32 + K;
-            best_t = __shfl_sync(kFull, tk, K);
-        }
+        if (bal) best_t = __shfl_sync(kFull, tk, 31 - __clz(bal));  // later rows win
     }
-    return best_t;  // element 0 is always valid: tau(1) = x_(1) - 1
+    return (double)best_t;  // element 0 is always valid: tau(1) = x_(1) - 1
 }
 
 // Exact threshold of <= 32 candidates, one per lane.
@@ -626,8 +622,14 @@ __device__ void finish_entmax_cta(const DecodeArgs &a, int b, int h, int hq, int
                     base += cn[w];
                 }
             }
-            tau = total <= 32 ? warp_exact_tau(x[0], total, sparsemax)
-                              : warp_exact_tau<4>(x, total, sparsemax);
+            if (total <= 32) {
+                tau = warp_exact_tau(x[0], total, sparsemax);
+            } else if (total <= 64) {
+                float x2[2] = {x[0], x[1]};
+                tau = warp_exact_tau<2>(x2, total, sparsemax);
+            } else {
+                tau = warp_exact_tau<4>(x, total, sparsemax);
+            }
         } else {
             float t = -1.0f;
 #pragma unroll 1

@@ -94,6 +94,7 @@ ekv_status ekv_page_meta_update(const ekv_cache *c, const int32_t *new_start,
     ekv_status s = check_cache(c, false);
     if (s != EKV_OK) return s;
     if (!new_start || !new_count || max_new < 0) return EKV_ERR_INVALID_ARG;
+    if ((uintptr_t)c->k_cache & 15u) return EKV_ERR_INVALID_ARG;  // rows are read with vector loads
     if ((long long)max_new > (long long)c->max_pages * c->page_size) return EKV_ERR_INVALID_ARG;
     return cuda_status(launch_page_meta_update(*c, new_start, new_count, max_new,
                                                static_cast<cudaStream_t>(stream)));

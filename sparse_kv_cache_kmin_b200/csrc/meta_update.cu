@@ -46,16 +46,30 @@ page_meta_update_kernel(ekv_cache c, const int32_t *__restrict__ new_start,
     const int cnt = len - p * P < P ? len - p * P : P;
     const size_t row0 = ((size_t)blk * c.num_kv_heads + h) * P;
 
+    // The page's rows are read 8 tokens at a time, each lane's VEC coordinates with one
+    // vector load per token, so a warp keeps 8 loads in flight per lane instead of walking the
+    // tokens one dependent load after another.
+    constexpr int TB = 8;
+    const char *krow = static_cast<const char *>(c.k_cache) +
+                       (row0 * D + lane * VEC) * (size_t)Chunk<DT>::kBytes;
+    constexpr size_t ROWB = (size_t)D * Chunk<DT>::kBytes;
     float mn[VEC], mx[VEC], sum[VEC];
 #pragma unroll
     for (int e = 0; e < VEC; ++e) { mn[e] = INFINITY; mx[e] = -INFINITY; sum[e] = 0.f; }
-    for (int t = 0; t < cnt; ++t) {
+    for (int t0 = 0; t0 < cnt; t0 += TB) {
+        float x[TB][VEC];
 #pragma unroll
-        for (int e = 0; e < VEC; ++e) {
-            float x = load_elem<DT>(c.k_cache, (row0 + t) * D + lane * VEC + e);
-            mn[e] = fminf(mn[e], x);
-            mx[e] = fmaxf(mx[e], x);
-            sum[e] += x;
+        for (int u = 0; u < TB; ++u)
+            if (t0 + u < cnt) load_vec_nc<DT, VEC>(krow + (t0 + u) * ROWB, x[u]);
+#pragma unroll
+        for (int u = 0; u < TB; ++u) {
+            if (t0 + u >= cnt) break;
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) {
+                mn[e] = fminf(mn[e], x[u][e]);
+                mx[e] = fmaxf(mx[e], x[u][e]);
+                sum[e] += x[u][e];
+            }
         }
     }
     const size_t mbase = ((size_t)blk * c.num_kv_heads + h) * 2 * D;
@@ -68,11 +82,19 @@ page_meta_update_kernel(ekv_cache c, const int32_t *__restrict__ new_start,
         float mean[VEC], ss[VEC];
 #pragma unroll
         for (int e = 0; e < VEC; ++e) { mean[e] = sum[e] / (float)cnt; ss[e] = 0.f; }
-        for (int t = 0; t < cnt; ++t) {
+        for (int t0 = 0; t0 < cnt; t0 += TB) {
+            float x[TB][VEC];
 #pragma unroll
-            for (int e = 0; e < VEC; ++e) {
-                float x = load_elem<DT>(c.k_cache, (row0 + t) * D + lane * VEC + e) - mean[e];
-                ss[e] = fmaf(x, x, ss[e]);
+            for (int u = 0; u < TB; ++u)
+                if (t0 + u < cnt) load_vec_nc<DT, VEC>(krow + (t0 + u) * ROWB, x[u]);
+#pragma unroll
+            for (int u = 0; u < TB; ++u) {
+                if (t0 + u >= cnt) break;
+#pragma unroll
+                for (int e = 0; e < VEC; ++e) {
+                    const float dv = x[u][e] - mean[e];
+                    ss[e] = fmaf(dv, dv, ss[e]);
+                }
             }
         }
 #pragma unroll
