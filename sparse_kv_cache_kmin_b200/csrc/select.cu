@@ -261,26 +261,26 @@ select_topk_kernel(const float *__restrict__ scores, int H, int max_pages, int P
 
 // ---------------------------------------------------------------------------- Gaussian-aware
 // E[(X - tau)_+^p] for X ~ N(a, b^2), p = 1 (alpha = 2) or 2 (alpha = 1.5), and its
-// derivative in tau. Phi(u) = erfc(-u / sqrt 2) / 2, phi(u) = exp(-u^2 / 2) / sqrt(2 pi).
-__device__ __forceinline__ void trunc_moment(double a, double b, double tau, bool sparsemax,
-                                             double &E, double &dE)
+// derivative in tau, in fp32. Phi(u) = erfc(-u / sqrt 2) / 2, phi(u) = exp(-u^2 / 2) / sqrt(2 pi).
+__device__ __forceinline__ void trunc_moment(float a, float b, float tau, bool sparsemax,
+                                             float &E, float &dE)
 {
-    const double r = a - tau;
-    if (b <= 0.0) {
-        const double rp = r > 0.0 ? r : 0.0;
+    const float r = a - tau;
+    if (b <= 0.f) {
+        const float rp = r > 0.f ? r : 0.f;
         E = sparsemax ? rp : rp * rp;
-        dE = sparsemax ? (r > 0.0 ? -1.0 : 0.0) : -2.0 * rp;
+        dE = sparsemax ? (r > 0.f ? -1.f : 0.f) : -2.f * rp;
         return;
     }
-    const double u = r / b;
-    const double Phi = 0.5 * erfc(-u * 0.70710678118654752440);
-    const double phi = 0.39894228040143267794 * exp(-0.5 * u * u);
+    const float u = r / b;
+    const float Phi = 0.5f * erfcf(-u * 0.70710678118654752f);
+    const float phi = 0.39894228040143268f * __expf(-0.5f * u * u);
     if (sparsemax) {
         E = r * Phi + b * phi;
         dE = -Phi;
     } else {
         E = (r * r + b * b) * Phi + r * b * phi;
-        dE = -2.0 * (r * Phi + b * phi);
+        dE = -2.f * (r * Phi + b * phi);
     }
 }
 
@@ -340,32 +340,55 @@ select_gauss_kernel(const float *__restrict__ scores, int H, int max_pages, int 
             tau = -INFINITY;
         } else {
 #pragma unroll 1
-            for (int it = 0; it < 64; ++it) {
-                double F = 0.0, dF = 0.0;
+            for (int it = 0; it < 48; ++it) {
+                float F = 0.f, dF = 0.f;
+                const float tf = (float)tau;
                 if (cnt <= CAP) {
                     for (int i = lane; i < cnt; i += 32) {
-                        double E, dE;
-                        trunc_moment(s_a[g][i], s_b[g][i], tau, sparsemax, E, dE);
-                        F += s_n[g][i] * E;
-                        dF += s_n[g][i] * dE;
+                        float E, dE;
+                        trunc_moment(s_a[g][i], s_b[g][i], tf, sparsemax, E, dE);
+                        F = fmaf((float)s_n[g][i], E, F);
+                        dF = fmaf((float)s_n[g][i], dE, dF);
                     }
                 } else {  // too many survivors for shared memory: walk every page
                     for (int j = lane; j < n; j += 32) {
-                        double E, dE;
-                        const double aj = (float)(am1 * (double)m[j]);
-                        const double bj = (float)(am1 * sqrt(fmax((double)v[j], 0.0)));
-                        trunc_moment(aj, bj, tau, sparsemax, E, dE);
+                        float E, dE;
+                        const float aj = (float)(am1 * (double)m[j]);
+                        const float bj = (float)(am1 * sqrt(fmax((double)v[j], 0.0)));
+                        trunc_moment(aj, bj, tf, sparsemax, E, dE);
                         const int nj = len - j * P < P ? len - j * P : P;
-                        F += nj * E;
-                        dF += nj * dE;
+                        F = fmaf((float)nj, E, F);
+                        dF = fmaf((float)nj, dE, dF);
                     }
                 }
-                F = warp_sum(F);
-                dF = warp_sum(dF);
-                if (!(dF < 0.0)) break;
-                const double step = (F - 1.0) / -dF;
-                if (!(step > 1e-13 * fmax(1.0, fabs(tau)))) break;
+                const double Fs = warp_sum((double)F), dFs = warp_sum((double)dF);
+                if (!(dFs < 0.0)) break;
+                const double step = (Fs - 1.0) / -dFs;
+                if (!(step > 1e-7 * fmax(1.0, fabs(tau)))) break;
                 tau += step;
+                // pages with a + 8 b below the (rising) threshold contribute nothing any more
+                if (cnt <= CAP && (it & 3) == 3) {
+                    int kept = 0;
+                    for (int i0 = 0; i0 < cnt; i0 += 32) {
+                        const int i = i0 + lane;
+                        float ai = 0.f, bi = 0.f;
+                        int ni = 0;
+                        bool keep = false;
+                        if (i < cnt) {
+                            ai = s_a[g][i]; bi = s_b[g][i]; ni = s_n[g][i];
+                            keep = (double)ai + 8.0 * (double)bi > tau;
+                        }
+                        const unsigned bal = __ballot_sync(kFull, keep);
+                        __syncwarp();
+                        if (keep) {
+                            const int pos = kept + __popc(bal & ((1u << lane) - 1u));
+                            s_a[g][pos] = ai; s_b[g][pos] = bi; s_n[g][pos] = ni;
+                        }
+                        kept += __popc(bal);
+                        __syncwarp();
+                    }
+                    cnt = kept;
+                }
             }
         }
         if (lane == 0) {
