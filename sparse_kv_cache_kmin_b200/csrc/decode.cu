@@ -394,16 +394,14 @@ __device__ void finish_softmax(const DecodeArgs &a, int b, int hq, int nchunks)
     if (tid == 0) a.stat[bq] = M == -INFINITY ? -INFINITY : (M + log2f(L)) * 0.69314718055994530942f;
 }
 
-constexpr int kCapW = 512;  // gathered logits per warp kept in shared memory
+constexpr int kCapW = 512;       // gathered logits per warp kept in shared memory
+constexpr int kHistBins = 512;   // bins per level of the threshold bracket (two per thread)
+constexpr int kHistLevels = 3;   // bracket levels: bin widths 2^-9, 2^-18, 2^-27
+constexpr int kHistExact = 128;  // a bracket bin with at most this many logits is solved exactly
 
-// Exact threshold of at most 32*R candidates held R per lane (element e = r*32 + lane; x =
-// z - zmax in [-1, 0], -inf padding): bitonic sort descending across registers and lanes,
-// prefix sums of x and x^2 in sorted order, then the largest k whose closed-form tau(k)
-// satisfies tau(k) <= x_(k) (1.5-entmax also needs a real root). fp32 throughout: with x in
-// [-1, 0] and at most 128 terms the sums carry ~1e-5 absolute error, far inside the output
-// tolerances, and fp32 keeps the dependent chain short.
+// Bitonic sort, descending, of 32*R values held R per lane (element e = r*32 + lane).
 template <int R>
-__device__ __forceinline__ double warp_exact_tau(float (&v)[R], int cnt, bool sparsemax)
+__device__ __forceinline__ void warp_sort_desc(float (&v)[R])
 {
     const int lane = threadIdx.x & 31;
     constexpr int N = 32 * R;
@@ -433,6 +431,18 @@ __device__ __forceinline__ double warp_exact_tau(float (&v)[R], int cnt, bool sp
             }
         }
     }
+}
+
+// Exact threshold of at most 32*R candidates held R per lane (x = z - zmax in [-1, 0], -inf
+// padding): sort descending, prefix sums of x and x^2 in sorted order, then the largest k whose
+// closed-form tau(k) satisfies tau(k) <= x_(k) (1.5-entmax also needs a real root). fp32
+// throughout: with x in [-1, 0] and at most 128 terms the sums carry ~1e-5 absolute error, far
+// inside the output tolerances, and fp32 keeps the dependent chain short.
+template <int R>
+__device__ __forceinline__ double warp_exact_tau(float (&v)[R], int cnt, bool sparsemax)
+{
+    const int lane = threadIdx.x & 31;
+    warp_sort_desc<R>(v);
     float carry1 = 0.f, carry2 = 0.f, best_t = 0.f;
 #pragma unroll
     for (int r = 0; r < R; ++r) {
@@ -468,11 +478,251 @@ __device__ __forceinline__ double warp_exact_tau(float (&v)[R], int cnt, bool sp
     return (double)best_t;  // element 0 is always valid: tau(1) = x_(1) - 1
 }
 
-// Exact threshold of <= 32 candidates, one per lane.
-__device__ __forceinline__ double warp_exact_tau(float x, int cnt, bool sparsemax)
+// Closed-form threshold of a support with n members, sum s1 and sum of squares s2 (x space):
+// sparsemax sum (x - tau) = 1; 1.5-entmax sum (x - tau)^2 = 1 (smaller root). Returns false when
+// the quadratic has no real root (the support is too wide).
+__device__ __forceinline__ bool closed_form_tau(double n, double s1, double s2, bool sparsemax,
+                                                double &tau)
 {
-    float v[1] = {x};
-    return warp_exact_tau<1>(v, cnt, sparsemax);
+    if (sparsemax) {
+        tau = (s1 - 1.0) / n;
+        return true;
+    }
+    const double mean = s1 / n;
+    const double disc = (1.0 - fmax(s2 - s1 * mean, 0.0)) / n;
+    tau = mean - sqrt(fmax(disc, 0.0));
+    return disc >= 0.0;
+}
+
+// Exact threshold over a known part of the support -- n0 logits with sums a0 = sum x,
+// b0 = sum x^2, every one above all candidates -- plus at most 32*R candidates held R per lane
+// as y = x - lo >= 0 (-inf padding). Same rule as warp_exact_tau on the merged sorted order: the
+// support is the largest k with tau(k) <= x_(k); if no candidate qualifies it is the known part.
+template <int R>
+__device__ double warp_exact_tau_based(float (&y)[R], int cnt, double lo, double n0, double a0,
+                                       double b0, bool sparsemax)
+{
+    const int lane = threadIdx.x & 31;
+    warp_sort_desc<R>(y);
+    double best = 0.0;
+    bool found = false;
+    if (n0 > 0.0) found = closed_form_tau(n0, a0, b0, sparsemax, best) || sparsemax;
+    float carry1 = 0.f, carry2 = 0.f;
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        const int e = r * 32 + lane;
+        const bool in = e < cnt;
+        const float yd = in ? y[r] : 0.f;
+        float s1 = yd, s2 = yd * yd;  // small: y lies within one bracket bin
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float t1 = __shfl_up_sync(kFull, s1, o), t2 = __shfl_up_sync(kFull, s2, o);
+            if (lane >= o) { s1 += t1; s2 += t2; }
+        }
+        s1 += carry1;
+        s2 += carry2;
+        carry1 = __shfl_sync(kFull, s1, 31);
+        carry2 = __shfl_sync(kFull, s2, 31);
+        const double k = (double)(e + 1);
+        const double sx = k * lo + (double)s1;
+        const double sxx = k * lo * lo + 2.0 * lo * (double)s1 + (double)s2;
+        double tk = 0.0;
+        const bool real = closed_form_tau(n0 + k, a0 + sx, b0 + sxx, sparsemax, tk);
+        const bool ok = in && real && tk <= lo + (double)yd;
+        const unsigned bal = __ballot_sync(kFull, ok);
+        if (bal) {
+            best = __shfl_sync(kFull, tk, 31 - __clz(bal));  // later rows win
+            found = true;
+        }
+    }
+    return found ? best : lo;
+}
+
+// Block-wide suffix sums (inclusive, from the highest thread down) of three doubles.
+__device__ __forceinline__ void block_suffix3(double (&v)[3], double (*wtot)[3])
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+#pragma unroll
+        for (int i = 0; i < 3; ++i) {
+            const double t = __shfl_down_sync(kFull, v[i], o);
+            if (lane + o < 32) v[i] += t;
+        }
+    }
+    if (lane == 0) {
+#pragma unroll
+        for (int i = 0; i < 3; ++i) wtot[warp][i] = v[i];
+    }
+    __syncthreads();
+    for (int w = warp + 1; w < kNW; ++w) {
+#pragma unroll
+        for (int i = 0; i < 3; ++i) v[i] += wtot[w][i];
+    }
+}
+
+struct HistScratch {
+    int c[kHistBins];
+    float t1[kHistBins], t2[kHistBins];  // per bin: sum and sum of squares of x - bin edge
+    double base[3];                      // count, sum x, sum x^2 of logits above the range
+    double wtot[kNW][3];
+    float list[kHistExact];
+    int nlist;
+    int jstar;
+};
+
+// Exact threshold of a candidate set too large for one warp's sort, in the domain x = z - zmax
+// (candidates in (-1, 0]). F(t) = sum (x - t)_+^p (p = 2 for 1.5-entmax, 1 for sparsemax) is
+// decreasing and tau solves F(tau) = 1 with tau >= -1. Each level bins the candidates in the
+// current range [lo, lo + width) into kHistBins bins holding count, sum and sum of squares of the
+// offset from the bin edge, evaluates F at every edge from suffix sums in fp64, and keeps the
+// last bin whose lower edge has F >= 1: tau lies inside it, everything above it is in the
+// support (it joins the known part) and everything below is not. Once the bracketing bin holds
+// at most kHistExact logits one warp solves exactly over them plus the known part; if after
+// kHistLevels levels it still holds more (ties to within 2^-27), support-refinement rounds from
+// the lower edge (each takes the closed-form tau of the logits above the current tau, which
+// rises monotonically to the exact one) finish the job. `visit(fn)` calls fn(x) for every
+// candidate of the calling warp; every thread of the block must call this.
+template <typename Visit>
+__device__ double cta_hist_tau(Visit &&visit, bool sparsemax, HistScratch &H)
+{
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    double lo = -1.0, width = 1.0;
+    if (tid == 0) H.base[0] = H.base[1] = H.base[2] = 0.0;
+    for (int level = 0;; ++level) {
+        for (int i = tid; i < kHistBins; i += 256) { H.c[i] = 0; H.t1[i] = 0.f; H.t2[i] = 0.f; }
+        if (tid == 0) { H.jstar = -1; H.nlist = 0; }
+        __syncthreads();
+        const double bw = width / kHistBins, inv = kHistBins / width, hi = lo + width;
+        // bin of x in this level's range, or -1 (the top level's last bin also takes x = 0)
+        auto bin_of = [&](double xd) -> int {
+            if (xd < lo || (level > 0 && xd >= hi)) return -1;
+            const int k = (int)((xd - lo) * inv);
+            return k < kHistBins - 1 ? k : kHistBins - 1;
+        };
+        visit([&](float x) {
+            const double xd = x;
+            const int k = bin_of(xd);
+            if (k < 0) return;
+            const float u = (float)(xd - (lo + k * bw));
+            atomicAdd(&H.c[k], 1);
+            atomicAdd(&H.t1[k], u);
+            atomicAdd(&H.t2[k], u * u);
+        });
+        __syncthreads();
+        // this thread's bins 2*tid and 2*tid+1 as (count, sum, sum of squares) of x - lo
+        double own[2][3], suf[3];
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            const int k = 2 * tid + r;
+            const double cc = H.c[k], e = k * bw, t1 = H.t1[k], t2 = H.t2[k];
+            own[r][0] = cc;
+            own[r][1] = cc * e + t1;
+            own[r][2] = cc * e * e + 2.0 * e * t1 + t2;
+        }
+#pragma unroll
+        for (int i = 0; i < 3; ++i) suf[i] = own[0][i] + own[1][i];
+        block_suffix3(suf, H.wtot);
+        const double n0 = H.base[0], a0 = H.base[1], b0 = H.base[2];
+        // F at an edge lo + e from the suffix (C, S1, S2) of the bins at and above it
+        auto F_at = [&](double e, const double (&s)[3]) {
+            const double t = lo + e;
+            if (sparsemax) return (a0 - t * n0) + (s[1] - e * s[0]);
+            return (b0 - 2.0 * t * a0 + t * t * n0) + (s[2] - 2.0 * e * s[1] + e * e * s[0]);
+        };
+        double suf1[3];  // suffix from bin 2*tid+1
+#pragma unroll
+        for (int i = 0; i < 3; ++i) suf1[i] = suf[i] - own[0][i];
+        int jm = -1;
+        if (F_at((2 * tid + 1) * bw, suf1) >= 1.0) jm = 2 * tid + 1;
+        else if (F_at(2 * tid * bw, suf) >= 1.0) jm = 2 * tid;
+        if (jm >= 0) atomicMax(&H.jstar, jm);
+        __syncthreads();
+        const int j = H.jstar < 0 ? 0 : H.jstar;
+        const int cj = H.c[j];
+        // the bins above j join the known part of the support
+        if (j + 1 < kHistBins && tid == (j + 1) / 2) {
+            const double *s = ((j + 1) & 1) ? suf1 : suf;
+            H.base[0] = n0 + s[0];
+            H.base[1] = a0 + s[1] + s[0] * lo;
+            H.base[2] = b0 + s[2] + 2.0 * lo * s[1] + lo * lo * s[0];
+        }
+        if (cj <= kHistExact || level == kHistLevels - 1) {
+            // collect the bracketing bin's logits as offsets from its lower edge
+            const double flo = lo + j * bw;
+            visit([&](float x) {
+                const double xd = x;
+                if (bin_of(xd) != j) return;
+                const int pos = atomicAdd(&H.nlist, 1);
+                if (pos < kHistExact) H.list[pos] = (float)(xd - flo);
+            });
+            __syncthreads();
+            const double N0 = H.base[0], A0 = H.base[1], B0 = H.base[2];
+            if (cj <= kHistExact) {
+                double tau = 0.0;
+                if (warp == 0) {
+                    const int n = H.nlist < kHistExact ? H.nlist : kHistExact;
+                    float y[4];
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) {
+                        const int e = r * 32 + lane;
+                        y[r] = e < n ? H.list[e] : -INFINITY;
+                    }
+                    if (n <= 32) {
+                        float y1[1] = {y[0]};
+                        tau = warp_exact_tau_based<1>(y1, n, flo, N0, A0, B0, sparsemax);
+                    } else if (n <= 64) {
+                        float y2[2] = {y[0], y[1]};
+                        tau = warp_exact_tau_based<2>(y2, n, flo, N0, A0, B0, sparsemax);
+                    } else {
+                        tau = warp_exact_tau_based<4>(y, n, flo, N0, A0, B0, sparsemax);
+                    }
+                    if (lane == 0) H.wtot[0][0] = tau;
+                }
+                __syncthreads();
+                tau = H.wtot[0][0];
+                __syncthreads();
+                return tau;
+            }
+            // more than kHistExact logits within 2^-27: refine the support from the lower edge
+            double tau = flo;
+            double prev = -1.0;
+#pragma unroll 1
+            for (int round = 0; round < 16; ++round) {
+                double acc[3] = {0.0, 0.0, 0.0};
+                visit([&](float x) {
+                    const double xd = x;
+                    if (bin_of(xd) == j && xd > tau) { acc[0] += 1.0; acc[1] += xd; acc[2] += xd * xd; }
+                });
+#pragma unroll
+                for (int i = 0; i < 3; ++i) acc[i] = warp_sum(acc[i]);
+                __syncthreads();
+                if (lane == 0) {
+#pragma unroll
+                    for (int i = 0; i < 3; ++i) H.wtot[warp][i] = acc[i];
+                }
+                __syncthreads();
+                double tot[3] = {0.0, 0.0, 0.0};
+#pragma unroll
+                for (int w = 0; w < kNW; ++w)
+#pragma unroll
+                    for (int i = 0; i < 3; ++i) tot[i] += H.wtot[w][i];
+                if (tot[0] == prev) break;
+                prev = tot[0];
+                double t2 = tau;
+                if (N0 + tot[0] > 0.0 &&
+                    closed_form_tau(N0 + tot[0], A0 + tot[1], B0 + tot[2], sparsemax, t2))
+                    tau = fmax(tau, t2);
+                else
+                    break;
+            }
+            __syncthreads();
+            return tau;
+        }
+        __syncthreads();
+        lo = lo + j * bw;
+        width = bw;
+    }
 }
 
 template <int DT, int D>
@@ -483,13 +733,14 @@ __device__ void finish_entmax_cta(const DecodeArgs &a, int b, int h, int hq, int
     constexpr int W = D * ESZ / 16;
     constexpr int RPI = 32 / W;
     constexpr int UNRV = 4;  // V rows in flight per lane group
-    constexpr int UNR = 8;   // logits in flight per lane while gathering
+    constexpr int UNR = 4;   // float4 logit loads in flight per lane while gathering
     __shared__ float cz[kNW][kCapW];
     __shared__ int cs[kNW][kCapW];
     __shared__ int cn[kNW];
     __shared__ float red[kNW];
     __shared__ double s_tau;
     __shared__ float o_w[kNW][D];
+    __shared__ HistScratch hist;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const ekv_cache &c = a.c;
     const int P = c.page_size, H = c.num_kv_heads;
@@ -512,104 +763,61 @@ __device__ void finish_entmax_cta(const DecodeArgs &a, int b, int h, int hq, int
     }
     const float thr = zmax - 1.0f;  // the largest weight is at most 1, so tau >= zmax - 1
 
-    // gather: warp w owns slots [s0, s1)
+    // gather: warp w owns slots [s0, s1), a multiple of 4 wide so rows are read as float4
     const int nslots = nsel * P;
-    const int per = (nslots + kNW - 1) / kNW;
-    const int s0 = warp * per, s1 = min(s0 + per, nslots);
+    const int per = ((nslots + kNW - 1) / kNW + 3) & ~3;
+    const int s0 = min(warp * per, nslots), s1 = min(s0 + per, nslots);
     int cnt = 0;
-    for (int s = s0; s < s1; s += 32 * UNR) {
-        float v[UNR];
+    for (int s = s0; s < s1; s += 128 * UNR) {
+        float4 v[UNR];
 #pragma unroll
         for (int u = 0; u < UNR; ++u) {
-            const int sl = s + u * 32 + lane;
-            v[u] = sl < s1 ? __ldcg(z + sl) : -INFINITY;
+            const int sl = s + (u * 32 + lane) * 4;
+            v[u] = sl < s1 ? __ldcg(reinterpret_cast<const float4 *>(z + sl))
+                           : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
         }
 #pragma unroll
         for (int u = 0; u < UNR; ++u) {
-            const bool keep = v[u] > thr;
-            const unsigned bal = __ballot_sync(kFull, keep);
-            const int pos = cnt + __popc(bal & ((1u << lane) - 1u));
-            if (keep && pos < kCapW) { cz[warp][pos] = v[u]; cs[warp][pos] = s + u * 32 + lane; }
-            cnt += __popc(bal);
+            const float e4[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const bool keep = e4[e] > thr;
+                const unsigned bal = __ballot_sync(kFull, keep);
+                const int pos = cnt + __popc(bal & ((1u << lane) - 1u));
+                if (keep && pos < kCapW) {
+                    cz[warp][pos] = e4[e] - zmax;  // lists hold x = z - zmax
+                    cs[warp][pos] = s + (u * 32 + lane) * 4 + e;
+                }
+                cnt += __popc(bal);
+            }
         }
     }
     if (lane == 0) cn[warp] = cnt;
     __syncthreads();
-
-    // tau: the exact threshold of any subset of the logits is a lower bound on the threshold of
-    // all of them (adding tokens can only raise it), so each warp solves exactly over up to 32
-    // of its surviving candidates, the largest of these bounds filters every list, and once at
-    // most 32 candidates survive, warp 0 solves exactly over them -- which is the threshold of
-    // the whole set, as everything filtered out lies at or below it.
     const bool over = cnt > kCapW;
     bool any_over = false;
+    int total = 0;
 #pragma unroll
-    for (int w = 0; w < kNW; ++w) any_over |= cn[w] > kCapW;
-    __shared__ float lb_w[kNW];
-    if (!any_over) {
-        for (int i = lane; i < cnt; i += 32) cz[warp][i] -= zmax;  // lists now hold x = z - zmax
-        __syncthreads();
-#pragma unroll 1
-        for (int round = 0; round < 6; ++round) {
-            // lower bound from this warp's first (up to) 32 candidates
-            const int nw = cn[warp];
-            const float xv = lane < nw ? cz[warp][lane] : -INFINITY;
-            const double tw = nw > 0 ? warp_exact_tau(xv, nw < 32 ? nw : 32, sparsemax) : -INFINITY;
-            if (lane == 0) lb_w[warp] = (float)tw;
-            __syncthreads();
-            float lb = -1.0f;
-#pragma unroll
-            for (int w = 0; w < kNW; ++w) lb = fmaxf(lb, lb_w[w]);
-            // keep x > lb (rounded down a little so fp32 rounding of the bound never drops a
-            // support member)
-            lb = lb - 1e-6f * fmaxf(1.0f, fabsf(lb));
-            int kept = 0;
-            for (int i0 = 0; i0 < nw; i0 += 32) {
-                const int i = i0 + lane;
-                const float x = i < nw ? cz[warp][i] : -INFINITY;
-                const int sl = i < nw ? cs[warp][i] : 0;
-                const bool keep = x > lb;
-                const unsigned bal = __ballot_sync(kFull, keep);
-                __syncwarp();
-                if (keep) {
-                    const int pos = kept + __popc(bal & ((1u << lane) - 1u));
-                    cz[warp][pos] = x;
-                    cs[warp][pos] = sl;
-                }
-                kept += __popc(bal);
-                __syncwarp();
-            }
-            __syncthreads();
-            if (lane == 0) cn[warp] = kept;
-            __syncthreads();
-            int total = 0;
-#pragma unroll
-            for (int w = 0; w < kNW; ++w) total += cn[w];
-            if (total <= 128) break;
-            if (round == 5) break;
-        }
+    for (int w = 0; w < kNW; ++w) {
+        any_over |= cn[w] > kCapW;
+        total += cn[w];
     }
-    if (warp == 0) {
-        int total = 0;
-#pragma unroll
-        for (int w = 0; w < kNW; ++w) total += cn[w];
-        // every candidate, shifted by zmax
-        auto visit = [&](auto &&fn) {
-            for (int w = 0; w < kNW; ++w) {
-                if (cn[w] <= kCapW) {
-                    for (int i = lane; i < cn[w]; i += 32) fn(any_over ? cz[w][i] - zmax : cz[w][i]);
-                } else {
-                    const int a0 = w * per, a1 = min(a0 + per, nslots);
-                    for (int sl = a0 + lane; sl < a1; sl += 32) {
-                        const float v = __ldcg(z + sl);
-                        if (v > thr) fn(v - zmax);
-                    }
-                }
+    // this warp's candidates: its list, or its slot range again when the list overflowed
+    auto visit_own = [&](auto &&fn) {
+        if (!over) {
+            for (int i = lane; i < cnt; i += 32) fn(cz[warp][i]);
+        } else {
+            for (int sl = s0 + lane; sl < s1; sl += 32) {
+                const float v = __ldcg(z + sl);
+                if (v > thr) fn(v - zmax);
             }
-        };
-        double tau;  // in the shifted domain x = z - zmax
-        if (!any_over && total <= 128) {
-            // element e = r * 32 + lane takes the e-th candidate in warp order
+        }
+    };
+
+    double tau;  // in the shifted domain x = z - zmax
+    if (!any_over && total <= 128) {
+        // one warp sorts every candidate: element e = r * 32 + lane is the e-th in warp order
+        if (warp == 0) {
             float x[4];
 #pragma unroll
             for (int r = 0; r < 4; ++r) {
@@ -622,61 +830,23 @@ __device__ void finish_entmax_cta(const DecodeArgs &a, int b, int h, int hq, int
                     base += cn[w];
                 }
             }
+            double t;
             if (total <= 32) {
-                tau = warp_exact_tau(x[0], total, sparsemax);
+                float x1[1] = {x[0]};
+                t = warp_exact_tau<1>(x1, total, sparsemax);
             } else if (total <= 64) {
                 float x2[2] = {x[0], x[1]};
-                tau = warp_exact_tau<2>(x2, total, sparsemax);
+                t = warp_exact_tau<2>(x2, total, sparsemax);
             } else {
-                tau = warp_exact_tau<4>(x, total, sparsemax);
+                t = warp_exact_tau<4>(x, total, sparsemax);
             }
-        } else {
-            float t = -1.0f;
-#pragma unroll 1
-            for (int it = 0; it < 24; ++it) {
-                float f = 0.f, df = 0.f;
-                visit([&](float x) {
-                    const float r = x - t;
-                    if (r > 0.f) { f += sparsemax ? r : r * r; df += sparsemax ? 1.f : 2.f * r; }
-                });
-                f = warp_sum(f) - 1.0f;
-                df = warp_sum(df);
-                if (!(f > 0.f) || !(df > 0.f)) break;
-                const float step = f / df;
-                t += step;
-                if (!(step > 1e-5f * fmaxf(1.0f, fabsf(t)))) break;
-            }
-            tau = t;
-#pragma unroll 1
-            for (int round = 0; round < 3; ++round) {
-                double n = 0.0, s1d = 0.0;
-                visit([&](float x) { if ((double)x > tau) { n += 1.0; s1d += x; } });
-                n = warp_sum(n);
-                s1d = warp_sum(s1d);
-                if (n < 1.0) break;
-                double t2;
-                if (sparsemax) {
-                    t2 = (s1d - 1.0) / n;
-                } else {
-                    const double mean = s1d / n;
-                    double m2 = 0.0;
-                    visit([&](float x) { if ((double)x > tau) m2 += ((double)x - mean) * ((double)x - mean); });
-                    m2 = warp_sum(m2);
-                    const double disc = (1.0 - m2) / n;
-                    if (disc < 0.0) break;
-                    t2 = mean - sqrt(disc);
-                }
-                int changed = 0;
-                visit([&](float x) { changed |= ((double)x > t2) != ((double)x > tau); });
-                changed = __any_sync(kFull, changed);
-                tau = t2;
-                if (!changed) break;
-            }
+            if (lane == 0) s_tau = t;
         }
-        if (lane == 0) s_tau = tau + (double)zmax;
+        __syncthreads();
+        tau = s_tau;
+    } else {
+        tau = cta_hist_tau(visit_own, sparsemax, hist);
     }
-    __syncthreads();
-    const double tau_z = s_tau;
 
     // o = sum over the support of p_i v_i, each warp over its own entries
     const char *vc = static_cast<const char *>(c.v_cache);
@@ -686,17 +856,22 @@ __device__ void finish_entmax_cta(const DecodeArgs &a, int b, int h, int hq, int
     for (int e = 0; e < EPC; ++e) acc[e] = 0.f;
     float *sp = cz[warp];  // compacted support weights, in place over the gathered list
     int *sr = cs[warp];    // and rows as blk * P + t
-    const int total = over ? s1 - s0 : cn[warp];
-    for (int i0 = 0; i0 < total; i0 += 32) {
+    const int nitems = over ? s1 - s0 : cnt;
+    for (int i0 = 0; i0 < nitems; i0 += 32) {
         const int i = i0 + lane;
-        float v = -INFINITY;
+        float x = -INFINITY;
         int slot = 0;
-        if (i < total) {
-            if (over) { slot = s0 + i; v = __ldcg(z + slot); }
-            else if (any_over) { slot = cs[warp][i]; v = cz[warp][i]; }
-            else { slot = cs[warp][i]; v = cz[warp][i] + zmax; }
+        if (i < nitems) {
+            if (over) {
+                slot = s0 + i;
+                const float v = __ldcg(z + slot);
+                x = v > thr ? v - zmax : -INFINITY;
+            } else {
+                slot = cs[warp][i];
+                x = cz[warp][i];
+            }
         }
-        const double r = (double)v - tau_z;
+        const double r = (double)x - tau;
         const bool keep = r > 0.0;
         const unsigned bal = __ballot_sync(kFull, keep);
         const int nb = __popc(bal);
@@ -711,24 +886,24 @@ __device__ void finish_entmax_cta(const DecodeArgs &a, int b, int h, int hq, int
         }
         __syncwarp();
         for (int k0 = 0; k0 < nb; k0 += RPI * UNRV) {
-            uint4 x[UNRV];
+            uint4 xv[UNRV];
             float p[UNRV];
 #pragma unroll
             for (int u = 0; u < UNRV; ++u) {
                 const int k = k0 + u * RPI + row;
                 p[u] = 0.f;
-                x[u] = make_uint4(0, 0, 0, 0);
+                xv[u] = make_uint4(0, 0, 0, 0);
                 if (k < nb) {
                     p[u] = sp[k];
                     const int br = sr[k];
                     const size_t rowi = ((size_t)(br >> a.Pshift) * H + h) * P + (br & (P - 1));
-                    x[u] = ld_stream16(vc + rowi * D * ESZ + cidx * 16);
+                    xv[u] = ld_stream16(vc + rowi * D * ESZ + cidx * 16);
                 }
             }
 #pragma unroll
             for (int u = 0; u < UNRV; ++u) {
                 float f[EPC];
-                Chunk<DT>::unpack(x[u], f);
+                Chunk<DT>::unpack(xv[u], f);
 #pragma unroll
                 for (int e = 0; e < EPC; ++e) acc[e] = fmaf(p[u], f[e], acc[e]);
             }
@@ -750,7 +925,7 @@ __device__ void finish_entmax_cta(const DecodeArgs &a, int b, int h, int hq, int
         for (int w = 0; w < kNW; ++w) sum += o_w[w][i];
         a.out[bq * D + i] = sum;
     }
-    if (tid == 0) a.stat[bq] = (float)tau_z;
+    if (tid == 0) a.stat[bq] = (float)(tau + (double)zmax);
 }
 
 template <int DT, int D, int G, bool SOFTMAX>
