@@ -571,158 +571,176 @@ struct HistScratch {
     int jstar;
 };
 
-// Exact threshold of a candidate set too large for one warp's sort, in the domain x = z - zmax
-// (candidates in (-1, 0]). F(t) = sum (x - t)_+^p (p = 2 for 1.5-entmax, 1 for sparsemax) is
-// decreasing and tau solves F(tau) = 1 with tau >= -1. Each level bins the candidates in the
-// current range [lo, lo + width) into kHistBins bins holding count, sum and sum of squares of the
-// offset from the bin edge, evaluates F at every edge from suffix sums in fp64, and keeps the
-// last bin whose lower edge has F >= 1: tau lies inside it, everything above it is in the
-// support (it joins the known part) and everything below is not. Once the bracketing bin holds
-// at most kHistExact logits one warp solves exactly over them plus the known part; if after
-// kHistLevels levels it still holds more (ties to within 2^-27), support-refinement rounds from
-// the lower edge (each takes the closed-form tau of the logits above the current tau, which
-// rises monotonically to the exact one) finish the job. `visit(fn)` calls fn(x) for every
-// candidate of the calling warp; every thread of the block must call this.
-template <typename Visit>
-__device__ double cta_hist_tau(Visit &&visit, bool sparsemax, HistScratch &H)
+// The threshold bracket, in the domain x = z - zmax (candidates in (-1, 0]). F(t) = sum
+// (x - t)_+^p (p = 2 for 1.5-entmax, 1 for sparsemax) is decreasing and tau solves F(tau) = 1
+// with tau >= -1. A level bins the candidates of the current range [lo, lo + width) into
+// kHistBins bins holding count, sum and sum of squares of the offset from the bin edge,
+// evaluates F at every edge from suffix sums in fp64, and keeps the last bin whose lower edge has
+// F >= 1: tau lies inside it, everything above it is in the support (it joins the known part
+// `base`) and everything below is not. The top level's range is (-1, 0] (its last bin also takes
+// x = 0); deeper levels split the bracketing bin of the level above, and the one that splits a
+// last bin keeps the closed upper end (the maximum, x = 0, stays in range).
+struct HistRange {
+    double lo, width, bw, inv;
+    bool top;
+    __device__ void set(double lo_, double width_, bool top_)
+    {
+        lo = lo_; width = width_; top = top_;
+        bw = width / kHistBins;
+        inv = kHistBins / width;
+    }
+    __device__ __forceinline__ int bin(double xd) const
+    {
+        if (xd < lo || (!top && xd >= lo + width)) return -1;
+        const int k = (int)((xd - lo) * inv);
+        return k < kHistBins - 1 ? k : kHistBins - 1;
+    }
+};
+
+__device__ __forceinline__ void hist_add(HistScratch &H, const HistRange &R, double xd)
 {
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    double lo = -1.0, width = 1.0;
-    if (tid == 0) H.base[0] = H.base[1] = H.base[2] = 0.0;
-    for (int level = 0;; ++level) {
-        for (int i = tid; i < kHistBins; i += 256) { H.c[i] = 0; H.t1[i] = 0.f; H.t2[i] = 0.f; }
-        if (tid == 0) { H.jstar = -1; H.nlist = 0; }
-        __syncthreads();
-        const double bw = width / kHistBins, inv = kHistBins / width, hi = lo + width;
-        // bin of x in this level's range, or -1 (the top level's last bin also takes x = 0)
-        auto bin_of = [&](double xd) -> int {
-            if (xd < lo || (level > 0 && xd >= hi)) return -1;
-            const int k = (int)((xd - lo) * inv);
-            return k < kHistBins - 1 ? k : kHistBins - 1;
-        };
+    const int k = R.bin(xd);
+    if (k < 0) return;
+    const float u = (float)(xd - (R.lo + k * R.bw));
+    atomicAdd(&H.c[k], 1);
+    atomicAdd(&H.t1[k], u);
+    atomicAdd(&H.t2[k], u * u);
+}
+
+// Zero the bins (block-wide; a __syncthreads must follow before the first hist_add).
+__device__ __forceinline__ void hist_clear(HistScratch &H, bool reset_base)
+{
+    for (int i = threadIdx.x; i < kHistBins; i += 256) { H.c[i] = 0; H.t1[i] = 0.f; H.t2[i] = 0.f; }
+    if (threadIdx.x == 0) {
+        H.jstar = -1;
+        H.nlist = 0;
+        if (reset_base) H.base[0] = H.base[1] = H.base[2] = 0.0;
+    }
+}
+
+// With the bins of range R filled: the bracketing bin j (returned; H.c[j] holds its count), and
+// the bins above j added to H.base. Every thread of the block must call this.
+__device__ int hist_bracket(HistScratch &H, const HistRange &R, bool sparsemax)
+{
+    const int tid = threadIdx.x;
+    __syncthreads();
+    // this thread's bins 2*tid and 2*tid+1 as (count, sum, sum of squares) of x - lo
+    double own[2][3], suf[3];
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        const int k = 2 * tid + r;
+        const double cc = H.c[k], e = k * R.bw, t1 = H.t1[k], t2 = H.t2[k];
+        own[r][0] = cc;
+        own[r][1] = cc * e + t1;
+        own[r][2] = cc * e * e + 2.0 * e * t1 + t2;
+    }
+#pragma unroll
+    for (int i = 0; i < 3; ++i) suf[i] = own[0][i] + own[1][i];
+    block_suffix3(suf, H.wtot);
+    const double n0 = H.base[0], a0 = H.base[1], b0 = H.base[2], lo = R.lo;
+    // F at the edge lo + e from the suffix (C, S1, S2) of the bins at and above it
+    auto F_at = [&](double e, const double (&s)[3]) {
+        const double t = lo + e;
+        if (sparsemax) return (a0 - t * n0) + (s[1] - e * s[0]);
+        return (b0 - 2.0 * t * a0 + t * t * n0) + (s[2] - 2.0 * e * s[1] + e * e * s[0]);
+    };
+    double suf1[3];  // suffix from bin 2*tid+1
+#pragma unroll
+    for (int i = 0; i < 3; ++i) suf1[i] = suf[i] - own[0][i];
+    int jm = -1;
+    if (F_at((2 * tid + 1) * R.bw, suf1) >= 1.0) jm = 2 * tid + 1;
+    else if (F_at(2 * tid * R.bw, suf) >= 1.0) jm = 2 * tid;
+    if (jm >= 0) atomicMax(&H.jstar, jm);
+    __syncthreads();
+    const int j = H.jstar < 0 ? 0 : H.jstar;
+    if (j + 1 < kHistBins && tid == (j + 1) / 2) {
+        const double *s = ((j + 1) & 1) ? suf1 : suf;
+        H.base[0] = n0 + s[0];
+        H.base[1] = a0 + s[1] + s[0] * lo;
+        H.base[2] = b0 + s[2] + 2.0 * lo * s[1] + lo * lo * s[0];
+    }
+    __syncthreads();
+    return j;
+}
+
+// tau once bin j of range R brackets it: with at most kHistExact logits in the bin one warp
+// solves exactly over them plus the known part; with more (only after kHistLevels levels: ties
+// to within 2^-27), support-refinement rounds from the bin's lower edge (each takes the
+// closed-form tau of the known part plus the bin's logits above the current tau, which rises
+// monotonically onto the exact one). `visit(fn)` calls fn(x) for every candidate of the calling
+// warp; every thread of the block must call this.
+template <typename Visit>
+__device__ double hist_solve(Visit &&visit, HistScratch &H, const HistRange &R, int j, bool sparsemax)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int cj = H.c[j];
+    const double flo = R.lo + j * R.bw;
+    const double N0 = H.base[0], A0 = H.base[1], B0 = H.base[2];
+    if (cj <= kHistExact) {
         visit([&](float x) {
             const double xd = x;
-            const int k = bin_of(xd);
-            if (k < 0) return;
-            const float u = (float)(xd - (lo + k * bw));
-            atomicAdd(&H.c[k], 1);
-            atomicAdd(&H.t1[k], u);
-            atomicAdd(&H.t2[k], u * u);
+            if (R.bin(xd) != j) return;
+            const int pos = atomicAdd(&H.nlist, 1);
+            if (pos < kHistExact) H.list[pos] = (float)(xd - flo);
         });
         __syncthreads();
-        // this thread's bins 2*tid and 2*tid+1 as (count, sum, sum of squares) of x - lo
-        double own[2][3], suf[3];
+        if (warp == 0) {
+            const int n = H.nlist < kHistExact ? H.nlist : kHistExact;
+            float y[4];
 #pragma unroll
-        for (int r = 0; r < 2; ++r) {
-            const int k = 2 * tid + r;
-            const double cc = H.c[k], e = k * bw, t1 = H.t1[k], t2 = H.t2[k];
-            own[r][0] = cc;
-            own[r][1] = cc * e + t1;
-            own[r][2] = cc * e * e + 2.0 * e * t1 + t2;
-        }
-#pragma unroll
-        for (int i = 0; i < 3; ++i) suf[i] = own[0][i] + own[1][i];
-        block_suffix3(suf, H.wtot);
-        const double n0 = H.base[0], a0 = H.base[1], b0 = H.base[2];
-        // F at an edge lo + e from the suffix (C, S1, S2) of the bins at and above it
-        auto F_at = [&](double e, const double (&s)[3]) {
-            const double t = lo + e;
-            if (sparsemax) return (a0 - t * n0) + (s[1] - e * s[0]);
-            return (b0 - 2.0 * t * a0 + t * t * n0) + (s[2] - 2.0 * e * s[1] + e * e * s[0]);
-        };
-        double suf1[3];  // suffix from bin 2*tid+1
-#pragma unroll
-        for (int i = 0; i < 3; ++i) suf1[i] = suf[i] - own[0][i];
-        int jm = -1;
-        if (F_at((2 * tid + 1) * bw, suf1) >= 1.0) jm = 2 * tid + 1;
-        else if (F_at(2 * tid * bw, suf) >= 1.0) jm = 2 * tid;
-        if (jm >= 0) atomicMax(&H.jstar, jm);
-        __syncthreads();
-        const int j = H.jstar < 0 ? 0 : H.jstar;
-        const int cj = H.c[j];
-        // the bins above j join the known part of the support
-        if (j + 1 < kHistBins && tid == (j + 1) / 2) {
-            const double *s = ((j + 1) & 1) ? suf1 : suf;
-            H.base[0] = n0 + s[0];
-            H.base[1] = a0 + s[1] + s[0] * lo;
-            H.base[2] = b0 + s[2] + 2.0 * lo * s[1] + lo * lo * s[0];
-        }
-        if (cj <= kHistExact || level == kHistLevels - 1) {
-            // collect the bracketing bin's logits as offsets from its lower edge
-            const double flo = lo + j * bw;
-            visit([&](float x) {
-                const double xd = x;
-                if (bin_of(xd) != j) return;
-                const int pos = atomicAdd(&H.nlist, 1);
-                if (pos < kHistExact) H.list[pos] = (float)(xd - flo);
-            });
-            __syncthreads();
-            const double N0 = H.base[0], A0 = H.base[1], B0 = H.base[2];
-            if (cj <= kHistExact) {
-                double tau = 0.0;
-                if (warp == 0) {
-                    const int n = H.nlist < kHistExact ? H.nlist : kHistExact;
-                    float y[4];
-#pragma unroll
-                    for (int r = 0; r < 4; ++r) {
-                        const int e = r * 32 + lane;
-                        y[r] = e < n ? H.list[e] : -INFINITY;
-                    }
-                    if (n <= 32) {
-                        float y1[1] = {y[0]};
-                        tau = warp_exact_tau_based<1>(y1, n, flo, N0, A0, B0, sparsemax);
-                    } else if (n <= 64) {
-                        float y2[2] = {y[0], y[1]};
-                        tau = warp_exact_tau_based<2>(y2, n, flo, N0, A0, B0, sparsemax);
-                    } else {
-                        tau = warp_exact_tau_based<4>(y, n, flo, N0, A0, B0, sparsemax);
-                    }
-                    if (lane == 0) H.wtot[0][0] = tau;
-                }
-                __syncthreads();
-                tau = H.wtot[0][0];
-                __syncthreads();
-                return tau;
+            for (int r = 0; r < 4; ++r) {
+                const int e = r * 32 + lane;
+                y[r] = e < n ? H.list[e] : -INFINITY;
             }
-            // more than kHistExact logits within 2^-27: refine the support from the lower edge
-            double tau = flo;
-            double prev = -1.0;
-#pragma unroll 1
-            for (int round = 0; round < 16; ++round) {
-                double acc[3] = {0.0, 0.0, 0.0};
-                visit([&](float x) {
-                    const double xd = x;
-                    if (bin_of(xd) == j && xd > tau) { acc[0] += 1.0; acc[1] += xd; acc[2] += xd * xd; }
-                });
-#pragma unroll
-                for (int i = 0; i < 3; ++i) acc[i] = warp_sum(acc[i]);
-                __syncthreads();
-                if (lane == 0) {
-#pragma unroll
-                    for (int i = 0; i < 3; ++i) H.wtot[warp][i] = acc[i];
-                }
-                __syncthreads();
-                double tot[3] = {0.0, 0.0, 0.0};
-#pragma unroll
-                for (int w = 0; w < kNW; ++w)
-#pragma unroll
-                    for (int i = 0; i < 3; ++i) tot[i] += H.wtot[w][i];
-                if (tot[0] == prev) break;
-                prev = tot[0];
-                double t2 = tau;
-                if (N0 + tot[0] > 0.0 &&
-                    closed_form_tau(N0 + tot[0], A0 + tot[1], B0 + tot[2], sparsemax, t2))
-                    tau = fmax(tau, t2);
-                else
-                    break;
+            double tau;
+            if (n <= 32) {
+                float y1[1] = {y[0]};
+                tau = warp_exact_tau_based<1>(y1, n, flo, N0, A0, B0, sparsemax);
+            } else if (n <= 64) {
+                float y2[2] = {y[0], y[1]};
+                tau = warp_exact_tau_based<2>(y2, n, flo, N0, A0, B0, sparsemax);
+            } else {
+                tau = warp_exact_tau_based<4>(y, n, flo, N0, A0, B0, sparsemax);
             }
-            __syncthreads();
-            return tau;
+            if (lane == 0) H.wtot[0][0] = tau;
         }
         __syncthreads();
-        lo = lo + j * bw;
-        width = bw;
+        const double tau = H.wtot[0][0];
+        __syncthreads();
+        return tau;
     }
+    double tau = flo, prev = -1.0;
+#pragma unroll 1
+    for (int round = 0; round < 16; ++round) {
+        double acc[3] = {0.0, 0.0, 0.0};
+        visit([&](float x) {
+            const double xd = x;
+            if (R.bin(xd) == j && xd > tau) { acc[0] += 1.0; acc[1] += xd; acc[2] += xd * xd; }
+        });
+#pragma unroll
+        for (int i = 0; i < 3; ++i) acc[i] = warp_sum(acc[i]);
+        __syncthreads();
+        if (lane == 0) {
+#pragma unroll
+            for (int i = 0; i < 3; ++i) H.wtot[warp][i] = acc[i];
+        }
+        __syncthreads();
+        double tot[3] = {0.0, 0.0, 0.0};
+#pragma unroll
+        for (int w = 0; w < kNW; ++w)
+#pragma unroll
+            for (int i = 0; i < 3; ++i) tot[i] += H.wtot[w][i];
+        if (tot[0] == prev) break;
+        prev = tot[0];
+        double t2 = tau;
+        if (N0 + tot[0] > 0.0 &&
+            closed_form_tau(N0 + tot[0], A0 + tot[1], B0 + tot[2], sparsemax, t2))
+            tau = fmax(tau, t2);
+        else
+            break;
+    }
+    __syncthreads();
+    return tau;
 }
 
 template <int DT, int D>
@@ -732,7 +750,7 @@ __device__ void finish_entmax_cta(const DecodeArgs &a, int b, int h, int hq, int
     constexpr int ESZ = Chunk<DT>::kBytes;
     constexpr int W = D * ESZ / 16;
     constexpr int RPI = 32 / W;
-    constexpr int UNRV = 4;  // V rows in flight per lane group
+    constexpr int UNRV = 8;  // V rows in flight per lane group
     constexpr int UNR = 4;   // float4 logit loads in flight per lane while gathering
     __shared__ float cz[kNW][kCapW];
     __shared__ int cs[kNW][kCapW];
@@ -748,6 +766,7 @@ __device__ void finish_entmax_cta(const DecodeArgs &a, int b, int h, int hq, int
     const float *z = a.logits + bq * (size_t)a.LS;
     const bool sparsemax = a.alpha == 2.0f;
 
+    hist_clear(hist, true);
     float zmax = -INFINITY;
     for (int ch = tid; ch < nchunks; ch += 256) zmax = fmaxf(zmax, __ldcg(a.part_ml + (bq * a.NC + ch) * 2));
     zmax = warp_max(zmax);
@@ -763,38 +782,49 @@ __device__ void finish_entmax_cta(const DecodeArgs &a, int b, int h, int hq, int
     }
     const float thr = zmax - 1.0f;  // the largest weight is at most 1, so tau >= zmax - 1
 
-    // gather: warp w owns slots [s0, s1), a multiple of 4 wide so rows are read as float4
+    // gather: warp w owns slots [s0, s1), a multiple of 4 wide so rows are read as float4. Every
+    // candidate goes into the top level of the threshold bracket; the first kCapW of each warp
+    // are also listed (x = z - zmax and slot)
+    HistRange R;
+    R.set(-1.0, 1.0, true);
     const int nslots = nsel * P;
     const int per = ((nslots + kNW - 1) / kNW + 3) & ~3;
     const int s0 = min(warp * per, nslots), s1 = min(s0 + per, nslots);
-    int cnt = 0;
-    for (int s = s0; s < s1; s += 128 * UNR) {
-        float4 v[UNR];
+    // candidates are z > thr with x = z - zmax >= clo (clo rises once the top level is bracketed)
+    double clo = -INFINITY;
+    auto gather = [&](bool binning) {
+        int cnt = 0;
+        for (int s = s0; s < s1; s += 128 * UNR) {
+            float4 v[UNR];
 #pragma unroll
-        for (int u = 0; u < UNR; ++u) {
-            const int sl = s + (u * 32 + lane) * 4;
-            v[u] = sl < s1 ? __ldcg(reinterpret_cast<const float4 *>(z + sl))
-                           : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
-        }
+            for (int u = 0; u < UNR; ++u) {
+                const int sl = s + (u * 32 + lane) * 4;
+                v[u] = sl < s1 ? __ldcg(reinterpret_cast<const float4 *>(z + sl))
+                               : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+            }
 #pragma unroll
-        for (int u = 0; u < UNR; ++u) {
-            const float e4[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+            for (int u = 0; u < UNR; ++u) {
+                const float e4[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const bool keep = e4[e] > thr;
-                const unsigned bal = __ballot_sync(kFull, keep);
-                const int pos = cnt + __popc(bal & ((1u << lane) - 1u));
-                if (keep && pos < kCapW) {
-                    cz[warp][pos] = e4[e] - zmax;  // lists hold x = z - zmax
-                    cs[warp][pos] = s + (u * 32 + lane) * 4 + e;
+                for (int e = 0; e < 4; ++e) {
+                    const float x = e4[e] - zmax;
+                    const bool keep = e4[e] > thr && (double)x >= clo;
+                    if (keep && binning) hist_add(hist, R, (double)x);
+                    const unsigned bal = __ballot_sync(kFull, keep);
+                    const int pos = cnt + __popc(bal & ((1u << lane) - 1u));
+                    if (keep && pos < kCapW) {
+                        cz[warp][pos] = x;
+                        cs[warp][pos] = s + (u * 32 + lane) * 4 + e;
+                    }
+                    cnt += __popc(bal);
                 }
-                cnt += __popc(bal);
             }
         }
-    }
+        return cnt;
+    };
+    int cnt = gather(true);
     if (lane == 0) cn[warp] = cnt;
     __syncthreads();
-    const bool over = cnt > kCapW;
     bool any_over = false;
     int total = 0;
 #pragma unroll
@@ -802,6 +832,7 @@ __device__ void finish_entmax_cta(const DecodeArgs &a, int b, int h, int hq, int
         any_over |= cn[w] > kCapW;
         total += cn[w];
     }
+    bool over = cnt > kCapW;
     // this warp's candidates: its list, or its slot range again when the list overflowed
     auto visit_own = [&](auto &&fn) {
         if (!over) {
@@ -809,7 +840,8 @@ __device__ void finish_entmax_cta(const DecodeArgs &a, int b, int h, int hq, int
         } else {
             for (int sl = s0 + lane; sl < s1; sl += 32) {
                 const float v = __ldcg(z + sl);
-                if (v > thr) fn(v - zmax);
+                const float x = v - zmax;
+                if (v > thr && (double)x >= clo) fn(x);
             }
         }
     };
@@ -845,47 +877,90 @@ __device__ void finish_entmax_cta(const DecodeArgs &a, int b, int h, int hq, int
         __syncthreads();
         tau = s_tau;
     } else {
-        tau = cta_hist_tau(visit_own, sparsemax, hist);
+        int j = hist_bracket(hist, R, sparsemax);
+        if (any_over) {
+            // only logits at or above the bracketing bin can be in the support: an overflowed
+            // warp lists those again
+            clo = R.lo + j * R.bw;
+            if (over) {
+                cnt = gather(false);
+                over = cnt > kCapW;
+            }
+        }
+        for (int level = 0;; ++level) {
+            if (hist.c[j] <= kHistExact || level == kHistLevels - 1) {
+                tau = hist_solve(visit_own, hist, R, j, sparsemax);
+                break;
+            }
+            R.set(R.lo + j * R.bw, R.bw, R.top && j == kHistBins - 1);
+            __syncthreads();
+            hist_clear(hist, false);
+            __syncthreads();
+            visit_own([&](float x) { hist_add(hist, R, (double)x); });
+            j = hist_bracket(hist, R, sparsemax);
+        }
     }
 
-    // o = sum over the support of p_i v_i, each warp over its own entries
+    // o = sum over the support of p_i v_i, each warp over its own entries: compact the support
+    // (weight, slot) in place over the gathered list, resolve every slot to its cache row with
+    // all lookups in flight, then stream the V rows UNRV per lane group; a warp whose list
+    // overflowed does this in rounds of at most kCapW entries
     const char *vc = static_cast<const char *>(c.v_cache);
     const int cidx = lane % W, row = lane / W;
     float acc[EPC];
 #pragma unroll
     for (int e = 0; e < EPC; ++e) acc[e] = 0.f;
-    float *sp = cz[warp];  // compacted support weights, in place over the gathered list
-    int *sr = cs[warp];    // and rows as blk * P + t
+    float *sp = cz[warp];  // compacted support weights
+    int *sr = cs[warp];    // and slots, then rows as blk * P + t
     const int nitems = over ? s1 - s0 : cnt;
-    for (int i0 = 0; i0 < nitems; i0 += 32) {
-        const int i = i0 + lane;
-        float x = -INFINITY;
-        int slot = 0;
-        if (i < nitems) {
-            if (over) {
-                slot = s0 + i;
-                const float v = __ldcg(z + slot);
-                x = v > thr ? v - zmax : -INFINITY;
-            } else {
-                slot = cs[warp][i];
-                x = cz[warp][i];
+    const int32_t *sel_row = a.sel_idx + ((size_t)b * H + h) * a.max_sel;
+    const int32_t *pt_row = c.page_table + (size_t)b * c.max_pages;
+    int it0 = 0;
+    do {
+        int ns = 0;
+        while (it0 < nitems && ns <= kCapW - 32) {
+            const int i = it0 + lane;
+            float x = -INFINITY;
+            int slot = 0;
+            if (i < nitems) {
+                if (over) {
+                    slot = s0 + i;
+                    const float v = __ldcg(z + slot);
+                    x = v > thr ? v - zmax : -INFINITY;
+                } else {
+                    slot = cs[warp][i];
+                    x = cz[warp][i];
+                }
+            }
+            const double r = (double)x - tau;
+            const bool keep = r > 0.0;
+            const unsigned bal = __ballot_sync(kFull, keep);
+            __syncwarp();
+            if (keep) {
+                const int pos = ns + __popc(bal & ((1u << lane) - 1u));
+                sp[pos] = (float)(sparsemax ? r : r * r);
+                sr[pos] = slot;
+            }
+            __syncwarp();
+            ns += __popc(bal);
+            it0 += 32;
+        }
+        for (int k0 = 0; k0 < ns; k0 += 128) {
+            int sl[4], jv[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int k = k0 + u * 32 + lane;
+                sl[u] = k < ns ? sr[k] : 0;
+                jv[u] = k < ns ? __ldg(sel_row + (sl[u] >> a.Pshift)) : 0;
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int k = k0 + u * 32 + lane;
+                if (k < ns) sr[k] = __ldg(pt_row + jv[u]) * P + (sl[u] & (P - 1));
             }
         }
-        const double r = (double)x - tau;
-        const bool keep = r > 0.0;
-        const unsigned bal = __ballot_sync(kFull, keep);
-        const int nb = __popc(bal);
         __syncwarp();
-        if (keep) {
-            const int pos = __popc(bal & ((1u << lane) - 1u));
-            const int pi = slot >> a.Pshift, t = slot & (P - 1);
-            const int j = a.sel_idx[((size_t)b * H + h) * a.max_sel + pi];
-            const int blk = c.page_table[(size_t)b * c.max_pages + j];
-            sp[pos] = (float)(sparsemax ? r : r * r);
-            sr[pos] = blk * P + t;
-        }
-        __syncwarp();
-        for (int k0 = 0; k0 < nb; k0 += RPI * UNRV) {
+        for (int k0 = 0; k0 < ns; k0 += RPI * UNRV) {
             uint4 xv[UNRV];
             float p[UNRV];
 #pragma unroll
@@ -893,7 +968,7 @@ __device__ void finish_entmax_cta(const DecodeArgs &a, int b, int h, int hq, int
                 const int k = k0 + u * RPI + row;
                 p[u] = 0.f;
                 xv[u] = make_uint4(0, 0, 0, 0);
-                if (k < nb) {
+                if (k < ns) {
                     p[u] = sp[k];
                     const int br = sr[k];
                     const size_t rowi = ((size_t)(br >> a.Pshift) * H + h) * P + (br & (P - 1));
@@ -909,7 +984,7 @@ __device__ void finish_entmax_cta(const DecodeArgs &a, int b, int h, int hq, int
             }
         }
         __syncwarp();
-    }
+    } while (it0 < nitems);
 #pragma unroll
     for (int o = W; o < 32; o <<= 1)
 #pragma unroll
@@ -929,7 +1004,7 @@ __device__ void finish_entmax_cta(const DecodeArgs &a, int b, int h, int hq, int
 }
 
 template <int DT, int D, int G, bool SOFTMAX>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 4)
 decode_finish_kernel(DecodeArgs a)
 {
     // one CTA per (sequence, query head)

@@ -284,17 +284,32 @@ __device__ __forceinline__ void trunc_moment(float a, float b, float tau, bool s
     }
 }
 
+constexpr int kGaussSmemBytes = 192 * 1024;  // survivor lists of one CTA (all G queries)
+
+// One CTA per (sequence, KV head); the G queries of the group each get 8/G warps. Each warp owns
+// a slice of the pages and a slice of the survivor list in shared memory: (a_j, b_j, n_j) with
+// a = (alpha-1) m, b = (alpha-1) sqrt(v) and n_j the page's token count. When the slice fits, the
+// warp stages its pages' model with all loads in flight; otherwise it reads them from global
+// memory for the maximum and keeps only the pages that survive the first prune (more than the
+// capacity and it walks global memory on every iteration).
+//
+// tau solves F(tau) = sum_j n_j E[(X_j - tau)_+^p] = 1. F is convex and decreasing, so Newton
+// from tau0 = max_j a_j - 1 (where F >= 1) rises monotonically onto the root; the sums are
+// combined over the query's warps each iteration (double-buffered partials, one named barrier).
+// Pages with a + 8 b <= tau contribute below 1e-14 of their count and are pruned every fourth
+// step. The union over the group then lists, in ascending page order, every page with
+// (alpha-1) UB_j > tau_g - delta for some query g.
 template <int G>
 __global__ void __launch_bounds__(256)
 select_gauss_kernel(const float *__restrict__ scores, int H, int max_pages, int P,
                     const int32_t *__restrict__ seq_lens, float alpha, float delta,
                     int32_t *__restrict__ sel_idx, int32_t *__restrict__ sel_count, int max_sel,
-                    float *__restrict__ tau_hat, uint32_t *status)
+                    float *__restrict__ tau_hat, uint32_t *status, int capw)
 {
-    constexpr int NT = 256;
-    constexpr int CAP = 2048 / G;  // survivors kept in shared memory per query
-    __shared__ float s_a[G][CAP], s_b[G][CAP];
-    __shared__ int s_n[G][CAP];
+    constexpr int NT = 256, WPQ = 8 / G;
+    extern __shared__ float gdyn[];
+    __shared__ double s_part[2][G][WPQ][2];
+    __shared__ float s_amax[G][WPQ];
     __shared__ double s_tau[G];
     __shared__ int warp_tot[8];
     pdl_wait();
@@ -304,38 +319,80 @@ select_gauss_kernel(const float *__restrict__ scores, int H, int max_pages, int 
     int len;
     const int n = seq_pages(seq_lens, b, P, max_pages, h == 0 ? status : nullptr, &len);
     const bool sparsemax = alpha == 2.0f;
-    const double am1 = (double)alpha - 1.0;
+    const float am1 = alpha - 1.0f;
 
-    if (warp < G) {
-        const int g = warp, hq = h * G + g;
+    {
+        const int g = warp / WPQ, r = warp % WPQ, hq = h * G + g;
         const float *sc = scores + ((size_t)b * H_q + hq) * 3 * max_pages;
         const float *m = sc + max_pages, *v = sc + 2 * (size_t)max_pages;
-        double amax = -INFINITY;
-        for (int j = lane; j < n; j += 32) amax = fmax(amax, am1 * (double)m[j]);
+        float *sa = gdyn + (size_t)warp * 3 * capw, *sb = sa + capw, *sn = sb + capw;
+        const int per = (n + WPQ - 1) / WPQ;
+        const int p0 = min(r * per, n), p1 = min(p0 + per, n);
+        const bool staged = p1 - p0 <= capw;
+        auto page_n = [&](int j) { return (float)(len - j * P < P ? len - j * P : P); };
+        auto model = [&](int j, float &aj, float &bj) {
+            aj = am1 * __ldcg(m + j);
+            bj = am1 * sqrtf(fmaxf(__ldcg(v + j), 0.f));
+        };
+        float amax = -INFINITY;
+        if (staged) {
+            for (int j0 = p0; j0 < p1; j0 += 128) {
+                float av[4], bv[4];
 #pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) amax = fmax(amax, __shfl_xor_sync(kFull, amax, o));
-        double tau = amax - 1.0;
-        // survivors: pages that can still contribute at tau >= amax - 1
+                for (int u = 0; u < 4; ++u) {
+                    const int j = j0 + u * 32 + lane;
+                    av[u] = -INFINITY; bv[u] = 0.f;
+                    if (j < p1) model(j, av[u], bv[u]);
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int j = j0 + u * 32 + lane;
+                    if (j < p1) {
+                        sa[j - p0] = av[u]; sb[j - p0] = bv[u]; sn[j - p0] = page_n(j);
+                        amax = fmaxf(amax, av[u]);
+                    }
+                }
+            }
+        } else {
+            for (int j0 = p0; j0 < p1; j0 += 256) {
+                float mv[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int j = j0 + u * 32 + lane;
+                    mv[u] = j < p1 ? __ldcg(m + j) : -INFINITY;
+                }
+#pragma unroll
+                for (int u = 0; u < 8; ++u) amax = fmaxf(amax, am1 * mv[u]);
+            }
+        }
+        amax = warp_max(amax);
+        if (lane == 0) s_amax[g][r] = amax;
+        named_sync(1 + g, 32 * WPQ);
+        amax = s_amax[g][0];
+#pragma unroll
+        for (int k = 1; k < WPQ; ++k) amax = fmaxf(amax, s_amax[g][k]);
+        double tau = (double)amax - 1.0;
+
+        // first prune: pages that can still contribute at tau >= amax - 1
         int cnt = 0;
-        for (int j0 = 0; j0 < n; j0 += 32) {
+        for (int j0 = p0; j0 < p1; j0 += 32) {
             const int j = j0 + lane;
-            float aj = 0.f, bj = 0.f;
+            float aj = 0.f, bj = 0.f, nj = 0.f;
             bool keep = false;
-            if (j < n) {
-                aj = (float)(am1 * (double)m[j]);
-                bj = (float)(am1 * sqrt(fmax((double)v[j], 0.0)));
+            if (j < p1) {
+                if (staged) { aj = sa[j - p0]; bj = sb[j - p0]; nj = sn[j - p0]; }
+                else { model(j, aj, bj); nj = page_n(j); }
                 keep = (double)aj + 8.0 * (double)bj > tau;
             }
             const unsigned bal = __ballot_sync(kFull, keep);
             const int pos = cnt + __popc(bal & ((1u << lane) - 1u));
-            if (keep && pos < CAP) {
-                s_a[g][pos] = aj;
-                s_b[g][pos] = bj;
-                s_n[g][pos] = len - j * P < P ? len - j * P : P;
-            }
+            __syncwarp();
+            if (keep && pos < capw) { sa[pos] = aj; sb[pos] = bj; sn[pos] = nj; }
             cnt += __popc(bal);
+            __syncwarp();
         }
-        __syncwarp();
+        const bool over = cnt > capw;
+
         if (n == 0) {
             tau = -INFINITY;
         } else {
@@ -343,46 +400,48 @@ select_gauss_kernel(const float *__restrict__ scores, int H, int max_pages, int 
             for (int it = 0; it < 48; ++it) {
                 float F = 0.f, dF = 0.f;
                 const float tf = (float)tau;
-                if (cnt <= CAP) {
+                if (!over) {
                     for (int i = lane; i < cnt; i += 32) {
                         float E, dE;
-                        trunc_moment(s_a[g][i], s_b[g][i], tf, sparsemax, E, dE);
-                        F = fmaf((float)s_n[g][i], E, F);
-                        dF = fmaf((float)s_n[g][i], dE, dF);
+                        trunc_moment(sa[i], sb[i], tf, sparsemax, E, dE);
+                        F = fmaf(sn[i], E, F);
+                        dF = fmaf(sn[i], dE, dF);
                     }
-                } else {  // too many survivors for shared memory: walk every page
-                    for (int j = lane; j < n; j += 32) {
-                        float E, dE;
-                        const float aj = (float)(am1 * (double)m[j]);
-                        const float bj = (float)(am1 * sqrt(fmax((double)v[j], 0.0)));
+                } else {
+                    for (int j = p0 + lane; j < p1; j += 32) {
+                        float aj, bj, E, dE;
+                        model(j, aj, bj);
                         trunc_moment(aj, bj, tf, sparsemax, E, dE);
-                        const int nj = len - j * P < P ? len - j * P : P;
-                        F = fmaf((float)nj, E, F);
-                        dF = fmaf((float)nj, dE, dF);
+                        F = fmaf(page_n(j), E, F);
+                        dF = fmaf(page_n(j), dE, dF);
                     }
                 }
-                const double Fs = warp_sum((double)F), dFs = warp_sum((double)dF);
+                const double Fw = warp_sum((double)F), dFw = warp_sum((double)dF);
+                if (lane == 0) { s_part[it & 1][g][r][0] = Fw; s_part[it & 1][g][r][1] = dFw; }
+                named_sync(1 + g, 32 * WPQ);
+                double Fs = 0.0, dFs = 0.0;
+#pragma unroll
+                for (int k = 0; k < WPQ; ++k) { Fs += s_part[it & 1][g][k][0]; dFs += s_part[it & 1][g][k][1]; }
                 if (!(dFs < 0.0)) break;
                 const double step = (Fs - 1.0) / -dFs;
                 if (!(step > 1e-7 * fmax(1.0, fabs(tau)))) break;
                 tau += step;
                 // pages with a + 8 b below the (rising) threshold contribute nothing any more
-                if (cnt <= CAP && (it & 3) == 3) {
+                if (!over && (it & 3) == 3) {
                     int kept = 0;
                     for (int i0 = 0; i0 < cnt; i0 += 32) {
                         const int i = i0 + lane;
-                        float ai = 0.f, bi = 0.f;
-                        int ni = 0;
+                        float ai = 0.f, bi = 0.f, ni = 0.f;
                         bool keep = false;
                         if (i < cnt) {
-                            ai = s_a[g][i]; bi = s_b[g][i]; ni = s_n[g][i];
+                            ai = sa[i]; bi = sb[i]; ni = sn[i];
                             keep = (double)ai + 8.0 * (double)bi > tau;
                         }
                         const unsigned bal = __ballot_sync(kFull, keep);
                         __syncwarp();
                         if (keep) {
                             const int pos = kept + __popc(bal & ((1u << lane) - 1u));
-                            s_a[g][pos] = ai; s_b[g][pos] = bi; s_n[g][pos] = ni;
+                            sa[pos] = ai; sb[pos] = bi; sn[pos] = ni;
                         }
                         kept += __popc(bal);
                         __syncwarp();
@@ -391,37 +450,57 @@ select_gauss_kernel(const float *__restrict__ scores, int H, int max_pages, int 
                 }
             }
         }
-        if (lane == 0) {
+        if (r == 0 && lane == 0) {
             s_tau[g] = tau;
             tau_hat[(size_t)b * H_q + hq] = (float)tau;
         }
     }
     __syncthreads();
 
-    // union over the group, ascending page order
-    const int E = (n + NT - 1) / NT;
-    const int j0 = tid * E, j1 = j0 + E < n ? j0 + E : n;
+    // union over the group, ascending page order: warp w owns pages [q0, q1) in 32-page rows;
+    // the first pass counts, the second writes at the warp's offset
+    const float *ub0 = scores + ((size_t)b * H_q + h * G) * 3 * max_pages;
+    double thr[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) thr[g] = s_tau[g] - (double)delta;
+    auto keep_page = [&](int j) {
+        bool keep = false;
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            const float ub = __ldcg(ub0 + (size_t)g * 3 * max_pages + j);
+            keep |= (double)am1 * (double)ub > thr[g];
+        }
+        return keep;
+    };
+    const int per = ((n + 7) / 8 + 31) & ~31;
+    const int q0 = min(warp * per, n), q1 = min(q0 + per, n);
     int mine = 0;
-    for (int j = j0; j < j1; ++j) {
-        bool keep = false;
+    for (int j0 = q0; j0 < q1; j0 += 128) {
+        bool kp[4];
 #pragma unroll
-        for (int g = 0; g < G; ++g) {
-            const float ub = scores[((size_t)b * H_q + h * G + g) * 3 * max_pages + j];
-            keep |= am1 * (double)ub > s_tau[g] - (double)delta;
+        for (int u = 0; u < 4; ++u) {
+            const int j = j0 + u * 32 + lane;
+            kp[u] = j < q1 && keep_page(j);
         }
-        mine += keep;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) mine += __popc(__ballot_sync(kFull, kp[u]));
     }
-    int total;
-    int pos = block_incl_scan<NT>(mine, warp_tot, &total) - mine;
-    int32_t *out = sel_idx + (size_t)bh * max_sel;
-    for (int j = j0; j < j1 && pos < max_sel; ++j) {
-        bool keep = false;
+    if (lane == 0) warp_tot[warp] = mine;
+    __syncthreads();
+    int pos = 0, total = 0;
 #pragma unroll
-        for (int g = 0; g < G; ++g) {
-            const float ub = scores[((size_t)b * H_q + h * G + g) * 3 * max_pages + j];
-            keep |= am1 * (double)ub > s_tau[g] - (double)delta;
-        }
-        if (keep) out[pos++] = j;
+    for (int w = 0; w < 8; ++w) {
+        pos += w < warp ? warp_tot[w] : 0;
+        total += warp_tot[w];
+    }
+    int32_t *out = sel_idx + (size_t)bh * max_sel;
+    for (int j0 = q0; j0 < q1; j0 += 32) {
+        const int j = j0 + lane;
+        const bool keep = j < q1 && keep_page(j);
+        const unsigned bal = __ballot_sync(kFull, keep);
+        const int at = pos + __popc(bal & ((1u << lane) - 1u));
+        if (keep && at < max_sel) out[at] = j;
+        pos += __popc(bal);
     }
     for (int j = total + tid; j < max_sel; j += NT) out[j] = -1;
     if (tid == 0) {
@@ -467,11 +546,25 @@ cudaError_t launch_select_pages(const ekv_cache &c, int H_q, int policy, int top
                                   c.dev_status);
     }
     cudaLaunchConfig_t cfg = pdl_config(grid, dim3(256), st, pdl, attr);
-#define EKV_GSEL(G)                                                                            \
-    cudaLaunchKernelEx(&cfg, select_gauss_kernel<G>, scores, c.num_kv_heads, c.max_pages,      \
-                       c.page_size, c.seq_lens, alpha, delta, sel_idx, sel_count, max_sel,     \
-                       tau_hat, c.dev_status)
-    switch (H_q / c.num_kv_heads) {
+    const int G = H_q / c.num_kv_heads, wpq = 8 / G;
+    // per-warp survivor capacity: a warp's whole page slice when the shared memory allows
+    const int cap_max = kGaussSmemBytes / (8 * 3 * (int)sizeof(float));
+    int capw = (c.max_pages + wpq - 1) / wpq;
+    capw = ((capw < cap_max ? capw : cap_max) + 3) & ~3;
+    cfg.dynamicSmemBytes = (size_t)8 * 3 * sizeof(float) * capw;
+#define EKV_GSEL(GG)                                                                           \
+    [&]() {                                                                                    \
+        static bool attr_set = false;                                                          \
+        if (!attr_set) {                                                                       \
+            cudaFuncSetAttribute(select_gauss_kernel<GG>,                                      \
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kGaussSmemBytes); \
+            attr_set = true;                                                                   \
+        }                                                                                      \
+        return cudaLaunchKernelEx(&cfg, select_gauss_kernel<GG>, scores, c.num_kv_heads,       \
+                                  c.max_pages, c.page_size, c.seq_lens, alpha, delta, sel_idx, \
+                                  sel_count, max_sel, tau_hat, c.dev_status, capw);            \
+    }()
+    switch (G) {
     case 1: return EKV_GSEL(1);
     case 2: return EKV_GSEL(2);
     case 4: return EKV_GSEL(4);

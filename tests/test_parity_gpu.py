@@ -71,6 +71,26 @@ def test_multi_chunk_pages(cuda_device):
             check_head(wl, cache, dec, b, h, attn)
 
 
+LARGE_CASES = [(torch.bfloat16, 2e-3), (torch.float32, 2e-3), (torch.bfloat16, 0.05),
+               (torch.bfloat16, 0.0)]
+
+
+@pytest.mark.parametrize("dtype,q_scale", LARGE_CASES,
+                         ids=["%s-q%g" % (str(t)[6:], s) for t, s in LARGE_CASES])
+def test_entmax_large_candidate_sets(cuda_device, dtype, q_scale):
+    # nearly flat logits put thousands of tokens within 1 of the maximum: the per-warp lists
+    # overflow, the threshold bracket descends several histogram levels, and q = 0 makes every
+    # logit equal (ties in the last bin)
+    wl = make_random(B=2, H_kv=2, G=4, d=128, P=16, lens=(20000, 7777), dtype=dtype,
+                     device="cuda", seed=11, q_scale=q_scale, topk=1250)
+    for attn in [ekv.EKV_ENTMAX15, ekv.EKV_SPARSEMAX]:
+        wl.alpha = 1.5 if attn == ekv.EKV_ENTMAX15 else 2.0
+        cache, dec = run_gpu(wl, attn)
+        assert_status_ok(cache)
+        for b, h in [(0, 0), (0, 1), (1, 1)]:
+            check_head(wl, cache, dec, b, h, attn)
+
+
 # ------------------------------------------------------------------ the five named workloads
 def test_tiny_full_and_support_invariant(cuda_device):
     wl = make("tiny", device="cuda")
