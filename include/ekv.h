@@ -124,6 +124,8 @@ ekv_status ekv_page_meta_update(const ekv_cache *c, const int32_t *new_start,
  *             v_{g,j} = scale^2 * sum_c q_gc^2 var_jc (needs c->meta_mom).
  * Entries for pages j >= ceil(seq_lens[b] / P) are not written. A page whose page-table entry
  * is out of range scores -inf (and m = v = 0) and is flagged.
+ * c->meta_bbox (and c->meta_mom for EKV_SEL_GAUSS) must be 16-byte aligned: metadata rows are
+ * read with 16-byte vector loads (EKV_ERR_INVALID_ARG otherwise).
  */
 ekv_status ekv_score_pages(const ekv_cache *c, const void *q, int32_t num_q_heads, float scale,
                            int32_t policy, float *scores, void *stream);

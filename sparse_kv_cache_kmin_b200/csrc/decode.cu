@@ -396,8 +396,9 @@ __device__ void finish_softmax(const DecodeArgs &a, int b, int hq, int nchunks)
 
 constexpr int kCapW = 512;       // gathered logits per warp kept in shared memory
 constexpr int kHistBins = 512;   // bins per level of the threshold bracket (two per thread)
-constexpr int kHistLevels = 3;   // bracket levels: bin widths 2^-9, 2^-18, 2^-27
-constexpr int kHistExact = 128;  // a bracket bin with at most this many logits is solved exactly
+constexpr int kHistLevels = 4;   // bracket levels before the tie fallback
+constexpr int kHistExact = 128;  // a bracket range with at most this many logits is solved exactly
+constexpr int kActCap = 1024;    // active chunks listed by the finish (more: walk every chunk)
 
 // Bitonic sort, descending, of 32*R values held R per lane (element e = r*32 + lane).
 template <int R>
@@ -562,124 +563,166 @@ __device__ __forceinline__ void block_suffix3(double (&v)[3], double (*wtot)[3])
 }
 
 struct HistScratch {
-    int c[kHistBins];
-    float t1[kHistBins], t2[kHistBins];  // per bin: sum and sum of squares of x - bin edge
-    double base[3];                      // count, sum x, sum x^2 of logits above the range
+    int c[kHistBins];        // logits per bin of the current range
+    double base[3];          // count, sum x, sum x^2 of the logits above the current range
     double wtot[kNW][3];
     float list[kHistExact];
     int nlist;
-    int jstar;
+    int jlo, jhi;
 };
 
 // The threshold bracket, in the domain x = z - zmax (candidates in (-1, 0]). F(t) = sum
 // (x - t)_+^p (p = 2 for 1.5-entmax, 1 for sparsemax) is decreasing and tau solves F(tau) = 1
-// with tau >= -1. A level bins the candidates of the current range [lo, lo + width) into
-// kHistBins bins holding count, sum and sum of squares of the offset from the bin edge,
-// evaluates F at every edge from suffix sums in fp64, and keeps the last bin whose lower edge has
-// F >= 1: tau lies inside it, everything above it is in the support (it joins the known part
-// `base`) and everything below is not. The top level's range is (-1, 0] (its last bin also takes
-// x = 0); deeper levels split the bracketing bin of the level above, and the one that splits a
-// last bin keeps the closed upper end (the maximum, x = 0, stays in range).
+// with tau >= -1. A level counts the candidates of its range [lo, hi) in bins of a power-of-two
+// width (exact binning in fp64). With only counts, F at a bin edge e is bracketed by placing
+// every logit at its bin's lower or upper edge: F_lo(e) <= F(e) <= F_hi(e). The last edge with
+// F_lo >= 1 is a lower bound on tau, the first edge after it with F_hi < 1 an upper bound; the
+// logits above the upper bound are in the support and join the known part `base` (exact sums),
+// those below the lower bound are out, and the bins between form the next range. The top
+// level's range is (-1, 0] (its last bin also takes x = 0); a range that reaches the top of a
+// closed range stays closed, so the maximum never drops out.
 struct HistRange {
-    double lo, width, bw, inv;
-    bool top;
-    __device__ void set(double lo_, double width_, bool top_)
+    double lo, hi, bw, inv;
+    int nb;     // bins in use
+    bool top;   // closed at hi
+    __device__ void set(double lo_, double hi_, double bw_, bool top_)
     {
-        lo = lo_; width = width_; top = top_;
-        bw = width / kHistBins;
-        inv = kHistBins / width;
+        lo = lo_; hi = hi_; bw = bw_; inv = 1.0 / bw_; top = top_;
+        nb = (int)ceil((hi - lo) * inv);
+        nb = nb < 1 ? 1 : (nb > kHistBins ? kHistBins : nb);
     }
     __device__ __forceinline__ int bin(double xd) const
     {
-        if (xd < lo || (!top && xd >= lo + width)) return -1;
+        if (xd < lo || (!top && xd >= hi)) return -1;
         const int k = (int)((xd - lo) * inv);
-        return k < kHistBins - 1 ? k : kHistBins - 1;
+        return k < nb - 1 ? k : nb - 1;
     }
 };
 
-__device__ __forceinline__ void hist_add(HistScratch &H, const HistRange &R, double xd)
+__device__ __forceinline__ void hist_count(HistScratch &H, const HistRange &R, double xd)
 {
     const int k = R.bin(xd);
-    if (k < 0) return;
-    const float u = (float)(xd - (R.lo + k * R.bw));
-    atomicAdd(&H.c[k], 1);
-    atomicAdd(&H.t1[k], u);
-    atomicAdd(&H.t2[k], u * u);
+    if (k >= 0) atomicAdd(&H.c[k], 1);
 }
 
-// Zero the bins (block-wide; a __syncthreads must follow before the first hist_add).
+// Zero the bins (block-wide; a __syncthreads must follow before the first hist_count).
 __device__ __forceinline__ void hist_clear(HistScratch &H, bool reset_base)
 {
-    for (int i = threadIdx.x; i < kHistBins; i += 256) { H.c[i] = 0; H.t1[i] = 0.f; H.t2[i] = 0.f; }
+    for (int i = threadIdx.x; i < kHistBins; i += 256) H.c[i] = 0;
     if (threadIdx.x == 0) {
-        H.jstar = -1;
+        H.jlo = 0;
+        H.jhi = 0;
         H.nlist = 0;
         if (reset_base) H.base[0] = H.base[1] = H.base[2] = 0.0;
     }
 }
 
-// With the bins of range R filled: the bracketing bin j (returned; H.c[j] holds its count), and
-// the bins above j added to H.base. Every thread of the block must call this.
-__device__ int hist_bracket(HistScratch &H, const HistRange &R, bool sparsemax)
+// Block-wide sum of three doubles per thread (every thread gets the total).
+__device__ __forceinline__ void block_sum3(double (&v)[3], double (*wtot)[3])
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int i = 0; i < 3; ++i) v[i] = warp_sum(v[i]);
+    __syncthreads();
+    if (lane == 0) {
+#pragma unroll
+        for (int i = 0; i < 3; ++i) wtot[warp][i] = v[i];
+    }
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < 3; ++i) {
+        double s = 0.0;
+#pragma unroll
+        for (int w = 0; w < kNW; ++w) s += wtot[w][i];
+        v[i] = s;
+    }
+    __syncthreads();
+}
+
+// With the bins of range R counted: the bracketing bins [jlo, jhi) into H.jlo, H.jhi. Every
+// thread of the block must call this.
+__device__ void hist_bracket(HistScratch &H, const HistRange &R, bool sparsemax)
 {
     const int tid = threadIdx.x;
     __syncthreads();
-    // this thread's bins 2*tid and 2*tid+1 as (count, sum, sum of squares) of x - lo
+    // suffix sums from bin 2*tid of (count, count*k, count*k^2)
     double own[2][3], suf[3];
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
         const int k = 2 * tid + r;
-        const double cc = H.c[k], e = k * R.bw, t1 = H.t1[k], t2 = H.t2[k];
+        const double cc = k < R.nb ? (double)H.c[k] : 0.0;
         own[r][0] = cc;
-        own[r][1] = cc * e + t1;
-        own[r][2] = cc * e * e + 2.0 * e * t1 + t2;
+        own[r][1] = cc * k;
+        own[r][2] = cc * k * k;
     }
 #pragma unroll
     for (int i = 0; i < 3; ++i) suf[i] = own[0][i] + own[1][i];
     block_suffix3(suf, H.wtot);
-    const double n0 = H.base[0], a0 = H.base[1], b0 = H.base[2], lo = R.lo;
-    // F at the edge lo + e from the suffix (C, S1, S2) of the bins at and above it
-    auto F_at = [&](double e, const double (&s)[3]) {
-        const double t = lo + e;
-        if (sparsemax) return (a0 - t * n0) + (s[1] - e * s[0]);
-        return (b0 - 2.0 * t * a0 + t * t * n0) + (s[2] - 2.0 * e * s[1] + e * e * s[0]);
+    const double n0 = H.base[0], a0 = H.base[1], b0 = H.base[2], bw = R.bw;
+    // F at edge j with every logit of bin k >= j placed at edge k + off (off = 0 or 1)
+    auto F_edge = [&](int j, const double (&s)[3], int off) {
+        const double e = R.lo + j * bw;
+        const double C = s[0], K1 = s[1] + off * s[0], K2 = s[2] + 2.0 * off * s[1] + off * s[0];
+        if (sparsemax) return (a0 - e * n0) + bw * (K1 - j * C);
+        return (b0 - 2.0 * e * a0 + e * e * n0) + bw * bw * (K2 - 2.0 * j * K1 + (double)j * j * C);
     };
     double suf1[3];  // suffix from bin 2*tid+1
 #pragma unroll
     for (int i = 0; i < 3; ++i) suf1[i] = suf[i] - own[0][i];
-    int jm = -1;
-    if (F_at((2 * tid + 1) * R.bw, suf1) >= 1.0) jm = 2 * tid + 1;
-    else if (F_at(2 * tid * R.bw, suf) >= 1.0) jm = 2 * tid;
-    if (jm >= 0) atomicMax(&H.jstar, jm);
+    const int j0 = 2 * tid, j1 = 2 * tid + 1;
+    int lo_m = -1, hi_m = -1;
+    if (j1 < R.nb && F_edge(j1, suf1, 0) >= 1.0) lo_m = j1;
+    else if (j0 < R.nb && F_edge(j0, suf, 0) >= 1.0) lo_m = j0;
+    if (j1 < R.nb && F_edge(j1, suf1, 1) >= 1.0) hi_m = j1;
+    else if (j0 < R.nb && F_edge(j0, suf, 1) >= 1.0) hi_m = j0;
+    if (lo_m >= 0) atomicMax(&H.jlo, lo_m);
+    if (hi_m >= 0) atomicMax(&H.jhi, hi_m + 1);
     __syncthreads();
-    const int j = H.jstar < 0 ? 0 : H.jstar;
-    if (j + 1 < kHistBins && tid == (j + 1) / 2) {
-        const double *s = ((j + 1) & 1) ? suf1 : suf;
-        H.base[0] = n0 + s[0];
-        H.base[1] = a0 + s[1] + s[0] * lo;
-        H.base[2] = b0 + s[2] + 2.0 * lo * s[1] + lo * lo * s[0];
-    }
+    const int jlo = H.jlo, jhi = max(H.jhi, jlo + 1);
     __syncthreads();
-    return j;
+    if (tid == 0) H.jhi = jhi;
+    __syncthreads();
 }
 
-// tau once bin j of range R brackets it: with at most kHistExact logits in the bin one warp
-// solves exactly over them plus the known part; with more (only after kHistLevels levels: ties
-// to within 2^-27), support-refinement rounds from the bin's lower edge (each takes the
-// closed-form tau of the known part plus the bin's logits above the current tau, which rises
-// monotonically onto the exact one). `visit(fn)` calls fn(x) for every candidate of the calling
-// warp; every thread of the block must call this.
+// Add the logits of range R at and above bin jhi to H.base (exact fp64 sums). `visit(fn)` calls
+// fn(x) for every candidate of the calling warp; every thread of the block must call this.
 template <typename Visit>
-__device__ double hist_solve(Visit &&visit, HistScratch &H, const HistRange &R, int j, bool sparsemax)
+__device__ void hist_add_base(Visit &&visit, HistScratch &H, const HistRange &R, int jhi)
 {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int cj = H.c[j];
-    const double flo = R.lo + j * R.bw;
-    const double N0 = H.base[0], A0 = H.base[1], B0 = H.base[2];
-    if (cj <= kHistExact) {
+    double acc[3] = {0.0, 0.0, 0.0};
+    if (jhi < R.nb) {
         visit([&](float x) {
             const double xd = x;
-            if (R.bin(xd) != j) return;
+            if (R.bin(xd) >= jhi) { acc[0] += 1.0; acc[1] += xd; acc[2] += xd * xd; }
+        });
+    }
+    block_sum3(acc, H.wtot);
+    if (threadIdx.x == 0) {
+        H.base[0] += acc[0];
+        H.base[1] += acc[1];
+        H.base[2] += acc[2];
+    }
+    __syncthreads();
+}
+
+// tau once range R (its logits counted in H.c) brackets it: with at most kHistExact logits in
+// the range one warp solves exactly over them plus the known part; with more (ties to within
+// the last level's bin width), support-refinement rounds from the range's lower edge (each takes
+// the closed-form tau of the known part plus the range's logits above the current tau, which
+// rises monotonically onto the exact one). Every thread of the block must call this.
+template <typename Visit>
+__device__ double hist_solve(Visit &&visit, HistScratch &H, const HistRange &R, int cnt_range,
+                             bool sparsemax)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const double flo = R.lo;
+    const double N0 = H.base[0], A0 = H.base[1], B0 = H.base[2];
+    if (cnt_range <= kHistExact) {
+        if (threadIdx.x == 0) H.nlist = 0;
+        __syncthreads();
+        visit([&](float x) {
+            const double xd = x;
+            if (R.bin(xd) < 0) return;
             const int pos = atomicAdd(&H.nlist, 1);
             if (pos < kHistExact) H.list[pos] = (float)(xd - flo);
         });
@@ -715,31 +758,18 @@ __device__ double hist_solve(Visit &&visit, HistScratch &H, const HistRange &R, 
         double acc[3] = {0.0, 0.0, 0.0};
         visit([&](float x) {
             const double xd = x;
-            if (R.bin(xd) == j && xd > tau) { acc[0] += 1.0; acc[1] += xd; acc[2] += xd * xd; }
+            if (R.bin(xd) >= 0 && xd > tau) { acc[0] += 1.0; acc[1] += xd; acc[2] += xd * xd; }
         });
-#pragma unroll
-        for (int i = 0; i < 3; ++i) acc[i] = warp_sum(acc[i]);
-        __syncthreads();
-        if (lane == 0) {
-#pragma unroll
-            for (int i = 0; i < 3; ++i) H.wtot[warp][i] = acc[i];
-        }
-        __syncthreads();
-        double tot[3] = {0.0, 0.0, 0.0};
-#pragma unroll
-        for (int w = 0; w < kNW; ++w)
-#pragma unroll
-            for (int i = 0; i < 3; ++i) tot[i] += H.wtot[w][i];
-        if (tot[0] == prev) break;
-        prev = tot[0];
+        block_sum3(acc, H.wtot);
+        if (acc[0] == prev) break;
+        prev = acc[0];
         double t2 = tau;
-        if (N0 + tot[0] > 0.0 &&
-            closed_form_tau(N0 + tot[0], A0 + tot[1], B0 + tot[2], sparsemax, t2))
+        if (N0 + acc[0] > 0.0 &&
+            closed_form_tau(N0 + acc[0], A0 + acc[1], B0 + acc[2], sparsemax, t2))
             tau = fmax(tau, t2);
         else
             break;
     }
-    __syncthreads();
     return tau;
 }
 
@@ -759,6 +789,7 @@ __device__ void finish_entmax_cta(const DecodeArgs &a, int b, int h, int hq, int
     __shared__ double s_tau;
     __shared__ float o_w[kNW][D];
     __shared__ HistScratch hist;
+    __shared__ int act[kActCap];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const ekv_cache &c = a.c;
     const int P = c.page_size, H = c.num_kv_heads;
@@ -767,8 +798,9 @@ __device__ void finish_entmax_cta(const DecodeArgs &a, int b, int h, int hq, int
     const bool sparsemax = a.alpha == 2.0f;
 
     hist_clear(hist, true);
+    const float *ml = a.part_ml + bq * a.NC * 2;
     float zmax = -INFINITY;
-    for (int ch = tid; ch < nchunks; ch += 256) zmax = fmaxf(zmax, __ldcg(a.part_ml + (bq * a.NC + ch) * 2));
+    for (int ch = tid; ch < nchunks; ch += 256) zmax = fmaxf(zmax, __ldcg(ml + 2 * ch));
     zmax = warp_max(zmax);
     if (lane == 0) red[warp] = zmax;
     __syncthreads();
@@ -782,25 +814,45 @@ __device__ void finish_entmax_cta(const DecodeArgs &a, int b, int h, int hq, int
     }
     const float thr = zmax - 1.0f;  // the largest weight is at most 1, so tau >= zmax - 1
 
-    // gather: warp w owns slots [s0, s1), a multiple of 4 wide so rows are read as float4. Every
-    // candidate goes into the top level of the threshold bracket; the first kCapW of each warp
-    // are also listed (x = z - zmax and slot)
-    HistRange R;
-    R.set(-1.0, 1.0, true);
-    const int nslots = nsel * P;
-    const int per = ((nslots + kNW - 1) / kNW + 3) & ~3;
-    const int s0 = min(warp * per, nslots), s1 = min(s0 + per, nslots);
+    // active chunks: those whose maximum exceeds zmax - 1 (no other chunk holds a candidate),
+    // listed in order; with more than kActCap of them every chunk is walked
+    int nact = 0;
+    for (int ch0 = 0; ch0 < nchunks; ch0 += 256) {
+        const int ch = ch0 + tid;
+        const int keep = ch < nchunks && __ldcg(ml + 2 * ch) > thr;
+        int tot;
+        const int pos = nact + block_incl_scan<256>(keep, cn, &tot) - keep;
+        if (keep && pos < kActCap) act[pos] = ch;
+        nact += tot;
+    }
+    const bool dense = nact > kActCap;
+    if (dense) nact = nchunks;
+    __syncthreads();
+
+    // gather: the active chunks form a virtual run of nact * CT slots; warp w owns a contiguous
+    // range of its float4 groups [f0w, f1w). Candidates (x = z - zmax and the slot) are listed,
+    // the first kCapW of each warp
+    const int CT = a.CP * P, CT4 = CT / 4;
+    const int nf4 = nact * CT4;
+    const int perf = (nf4 + kNW - 1) / kNW;
+    const int f0w = min(warp * perf, nf4), f1w = min(f0w + perf, nf4);
+    auto slot_of = [&](int f) {  // first slot of virtual float4 group f
+        const int i = f / CT4;
+        return (dense ? i : act[i]) * CT + (f - i * CT4) * 4;
+    };
     // candidates are z > thr with x = z - zmax >= clo (clo rises once the top level is bracketed)
     double clo = -INFINITY;
-    auto gather = [&](bool binning) {
+    auto gather = [&]() {
         int cnt = 0;
-        for (int s = s0; s < s1; s += 128 * UNR) {
+        for (int f = f0w; f < f1w; f += 32 * UNR) {
             float4 v[UNR];
+            int sl[UNR];
 #pragma unroll
             for (int u = 0; u < UNR; ++u) {
-                const int sl = s + (u * 32 + lane) * 4;
-                v[u] = sl < s1 ? __ldcg(reinterpret_cast<const float4 *>(z + sl))
-                               : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+                const int fu = f + u * 32 + lane;
+                sl[u] = fu < f1w ? slot_of(fu) : 0;
+                v[u] = fu < f1w ? __ldcg(reinterpret_cast<const float4 *>(z + sl[u]))
+                                : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
             }
 #pragma unroll
             for (int u = 0; u < UNR; ++u) {
@@ -809,12 +861,11 @@ __device__ void finish_entmax_cta(const DecodeArgs &a, int b, int h, int hq, int
                 for (int e = 0; e < 4; ++e) {
                     const float x = e4[e] - zmax;
                     const bool keep = e4[e] > thr && (double)x >= clo;
-                    if (keep && binning) hist_add(hist, R, (double)x);
                     const unsigned bal = __ballot_sync(kFull, keep);
                     const int pos = cnt + __popc(bal & ((1u << lane) - 1u));
                     if (keep && pos < kCapW) {
                         cz[warp][pos] = x;
-                        cs[warp][pos] = s + (u * 32 + lane) * 4 + e;
+                        cs[warp][pos] = sl[u] + e;
                     }
                     cnt += __popc(bal);
                 }
@@ -822,7 +873,8 @@ __device__ void finish_entmax_cta(const DecodeArgs &a, int b, int h, int hq, int
         }
         return cnt;
     };
-    int cnt = gather(true);
+    int cnt = gather();
+    __syncthreads();
     if (lane == 0) cn[warp] = cnt;
     __syncthreads();
     bool any_over = false;
@@ -833,18 +885,21 @@ __device__ void finish_entmax_cta(const DecodeArgs &a, int b, int h, int hq, int
         total += cn[w];
     }
     bool over = cnt > kCapW;
-    // this warp's candidates: its list, or its slot range again when the list overflowed
+    // this warp's candidates: its list, or its range of the active chunks again when the list
+    // overflowed
     auto visit_own = [&](auto &&fn) {
         if (!over) {
             for (int i = lane; i < cnt; i += 32) fn(cz[warp][i]);
         } else {
-            for (int sl = s0 + lane; sl < s1; sl += 32) {
-                const float v = __ldcg(z + sl);
+            for (int i = lane; i < (f1w - f0w) * 4; i += 32) {
+                const float v = __ldcg(z + slot_of(f0w + i / 4) + (i & 3));
                 const float x = v - zmax;
                 if (v > thr && (double)x >= clo) fn(x);
             }
         }
     };
+    HistRange R;
+    R.set(-1.0, 0.0, 1.0 / kHistBins, true);
 
     double tau;  // in the shifted domain x = z - zmax
     if (!any_over && total <= 128) {
@@ -877,27 +932,35 @@ __device__ void finish_entmax_cta(const DecodeArgs &a, int b, int h, int hq, int
         __syncthreads();
         tau = s_tau;
     } else {
-        int j = hist_bracket(hist, R, sparsemax);
-        if (any_over) {
-            // only logits at or above the bracketing bin can be in the support: an overflowed
-            // warp lists those again
-            clo = R.lo + j * R.bw;
-            if (over) {
-                cnt = gather(false);
-                over = cnt > kCapW;
-            }
-        }
+        visit_own([&](float x) { hist_count(hist, R, (double)x); });
         for (int level = 0;; ++level) {
-            if (hist.c[j] <= kHistExact || level == kHistLevels - 1) {
-                tau = hist_solve(visit_own, hist, R, j, sparsemax);
+            hist_bracket(hist, R, sparsemax);
+            const int jlo = hist.jlo, jhi = hist.jhi;
+            int cr = 0;
+            for (int k = jlo; k < jhi; ++k) cr += hist.c[k];
+            const double nlo = R.lo + jlo * R.bw, nhi = R.lo + jhi * R.bw;
+            const bool ntop = R.top && jhi >= R.nb;
+            // bins of the next range: the power-of-two width that covers it in kHistBins
+            double nbw = R.bw;
+            while (nbw * kHistBins > (jhi - jlo) * R.bw * 2.0 && nbw > 0x1p-60) nbw *= 0.5;
+            if (level == 0 && any_over) {
+                // only logits at or above the lower bound can be in the support: an overflowed
+                // warp lists those again
+                clo = nlo;
+                if (over) {
+                    cnt = gather();
+                    over = cnt > kCapW;
+                }
+            }
+            hist_add_base(visit_own, hist, R, jhi);
+            R.set(nlo, nhi, nbw, ntop);
+            if (cr <= kHistExact || level == kHistLevels - 1) {
+                tau = hist_solve(visit_own, hist, R, cr, sparsemax);
                 break;
             }
-            R.set(R.lo + j * R.bw, R.bw, R.top && j == kHistBins - 1);
-            __syncthreads();
             hist_clear(hist, false);
             __syncthreads();
-            visit_own([&](float x) { hist_add(hist, R, (double)x); });
-            j = hist_bracket(hist, R, sparsemax);
+            visit_own([&](float x) { hist_count(hist, R, (double)x); });
         }
     }
 
@@ -912,7 +975,7 @@ __device__ void finish_entmax_cta(const DecodeArgs &a, int b, int h, int hq, int
     for (int e = 0; e < EPC; ++e) acc[e] = 0.f;
     float *sp = cz[warp];  // compacted support weights
     int *sr = cs[warp];    // and slots, then rows as blk * P + t
-    const int nitems = over ? s1 - s0 : cnt;
+    const int nitems = over ? (f1w - f0w) * 4 : cnt;
     const int32_t *sel_row = a.sel_idx + ((size_t)b * H + h) * a.max_sel;
     const int32_t *pt_row = c.page_table + (size_t)b * c.max_pages;
     int it0 = 0;
@@ -924,7 +987,7 @@ __device__ void finish_entmax_cta(const DecodeArgs &a, int b, int h, int hq, int
             int slot = 0;
             if (i < nitems) {
                 if (over) {
-                    slot = s0 + i;
+                    slot = slot_of(f0w + i / 4) + (i & 3);
                     const float v = __ldcg(z + slot);
                     x = v > thr ? v - zmax : -INFINITY;
                 } else {

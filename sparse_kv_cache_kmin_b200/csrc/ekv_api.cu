@@ -109,6 +109,8 @@ ekv_status ekv_score_pages(const ekv_cache *c, const void *q, int32_t num_q_head
     if (!q || !scores || !(scale > 0.0f) || !std::isfinite(scale)) return EKV_ERR_INVALID_ARG;
     if (policy != EKV_SEL_TOPK && policy != EKV_SEL_GAUSS) return EKV_ERR_UNSUPPORTED;
     if (policy == EKV_SEL_GAUSS && !c->meta_mom) return EKV_ERR_INVALID_ARG;
+    if ((uintptr_t)c->meta_bbox & 15u) return EKV_ERR_INVALID_ARG;
+    if (policy == EKV_SEL_GAUSS && ((uintptr_t)c->meta_mom & 15u)) return EKV_ERR_INVALID_ARG;
     return cuda_status(launch_score_pages(*c, q, num_q_heads, scale, policy, scores,
                                           static_cast<cudaStream_t>(stream), use_pdl()));
 }

@@ -82,7 +82,7 @@ def fake_cache(**over):
 @pytest.mark.parametrize("over,status", [
     ({"head_dim": 96}, 2), ({"page_size": 8}, 2), ({"dtype": 7}, 2),
     ({"num_kv_heads": 0}, 1), ({"k_cache": None}, 1), ({"dev_status": None}, 1),
-    ({"batch": 9000}, 2),
+    ({"batch": 9000}, 2), ({"meta_bbox": 0x1008}, 1),
 ])
 def test_score_validation(lib, over, status):
     c = fake_cache(**over)
@@ -97,6 +97,8 @@ def test_head_count_and_policy_validation(lib):
     assert lib.ekv_score_pages(ctypes.byref(c), 0x1000, 32, 1.0, 5, 0x1000, None) == 2   # policy
     c2 = fake_cache(meta_mom=None)
     assert lib.ekv_score_pages(ctypes.byref(c2), 0x1000, 32, 1.0, 1, 0x1000, None) == 1  # gauss w/o moments
+    c3 = fake_cache(meta_mom=0x1004)
+    assert lib.ekv_score_pages(ctypes.byref(c3), 0x1000, 32, 1.0, 1, 0x1000, None) == 1  # misaligned moments
 
 
 def test_select_validation(lib):
