@@ -45,6 +45,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch (smaller cases for profiler captures)")
+    ap.add_argument("--no-full-cache", action="store_true",
+                    help="skip the full-cache decode (every page selected) timed for comparison")
     return ap.parse_args()
 
 
@@ -247,6 +249,46 @@ def oracle_sample(wl, attn, budget_s, max_heads=None):
     return per_step, desc
 
 
+
+# ----------------------------------------------------------------------------- full-cache decode
+def full_cache_time(ekv, cache, wl, attn, steps, flush, stream):
+    """The same attention over every page of every sequence (no scoring, no selection): one
+    ekv_sparse_decode call with the identity selection, captured in a graph and timed like the
+    sparse step. Returns ms per step."""
+    B, H, P = wl.batch, wl.num_kv_heads, wl.page_size
+    dev = wl.k_cache.device
+    n_pages = ((wl.seq_lens.long() + P - 1) // P).to(torch.int32)
+    mp = int(wl.page_table.shape[1])
+    sel = torch.arange(mp, dtype=torch.int32, device=dev).expand(B, H, mp).contiguous()
+    sel = torch.where(sel < n_pages.view(B, 1, 1), sel, torch.full_like(sel, -1))
+    cnt = n_pages.view(B, 1).expand(B, H).contiguous()
+    out = torch.empty((B, wl.num_q_heads, wl.head_dim), dtype=torch.float32, device=dev)
+    stat = torch.empty((B, wl.num_q_heads), dtype=torch.float32, device=dev)
+    ws = torch.empty(ekv.ekv_decode_workspace_bytes(cache, wl.num_q_heads, mp), dtype=torch.uint8,
+                     device=dev)
+
+    def call():
+        ekv.ekv_sparse_decode(cache, wl.q, wl.num_q_heads, wl.scale, attn, sel, cnt, mp, out,
+                              stat, ws)
+    call()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        call()
+    for _ in range(3):
+        flush.fill_(1)
+        g.replay()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    for i in range(steps):
+        flush.fill_(i & 0xff)
+        ev[i][0].record(stream)
+        g.replay()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    del g
+    return statistics.mean(a.elapsed_time(b) for a, b in ev)
+
 # ----------------------------------------------------------------------------- main
 def main():
     args = parse()
@@ -394,6 +436,13 @@ def main():
     e2e_s = replicas.max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e_ev) / 1e3, device=dev)
     d2h = out_host.numel() * 4 + stat_host.numel() * 4
 
+    full_ms = None
+    if not args.no_full_cache and world == 1:
+        full_ms = full_cache_time(ekv, cache, wl, attn, min(args.steps, 20), flush, stream)
+        st, bits = ekv.ekv_device_status(cache)
+        if st != ekv.EKV_OK:
+            raise RuntimeError("device status 0x%x after the full-cache decode" % bits)
+
     if rank != 0:
         if pg:
             pg.barrier()
@@ -439,6 +488,10 @@ def main():
                      "algorithmic_bytes_per_launch": by["score"]},
         "decode_kernel": {"achieved_GBps": by["decode"] / decode_s / 1e9,
                           "frac": by["decode"] / decode_s / 1e9 / peak},
+        "full_cache": None if full_ms is None else {
+            "what": "the same attention over every page (no scoring, no selection) on this GPU",
+            "ms_per_step": full_ms, "steps_per_s": 1e3 / full_ms,
+            "sparse_speedup": full_ms / ms},
         "e2e": {"value": replicas.job_rate(args.steps, world, e2e_s), "unit": "steps/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * args.steps,

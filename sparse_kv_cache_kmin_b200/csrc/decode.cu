@@ -135,6 +135,7 @@ decode_chunk_kernel(DecodeArgs a)
                         nt = len - j * P < P ? len - j * P : P;
                     }
                 }
+                if (!SOFTMAX) a.sel_blk[(size_t)bh * a.max_sel + i] = nt > 0 ? blk : -1;
             }
         };
         advance();
@@ -479,6 +480,19 @@ __device__ __forceinline__ double warp_exact_tau(float (&v)[R], int cnt, bool sp
     return (double)best_t;  // element 0 is always valid: tau(1) = x_(1) - 1
 }
 
+// Whether the closed-form threshold of a support with n members, sum s1 and sum of squares s2
+// is real and at most x (the support's smallest member), without a division or a square root:
+// sparsemax: (s1 - 1) / n <= x  <=>  s1 - 1 <= n x; 1.5-entmax: with n^2 disc = n - n s2 + s1^2,
+// s1 / n - sqrt(disc) <= x  <=>  s1 - n x <= 0 or (s1 - n x)^2 <= n^2 disc.
+__device__ __forceinline__ bool closed_form_ok(double n, double s1, double s2, double x, bool sparsemax)
+{
+    if (sparsemax) return s1 - 1.0 <= n * x;
+    const double d2 = n - n * s2 + s1 * s1;
+    if (d2 < 0.0) return false;
+    const double u = s1 - n * x;
+    return u <= 0.0 || u * u <= d2;
+}
+
 // Closed-form threshold of a support with n members, sum s1 and sum of squares s2 (x space):
 // sparsemax sum (x - tau) = 1; 1.5-entmax sum (x - tau)^2 = 1 (smaller root). Returns false when
 // the quadratic has no real root (the support is too wide).
@@ -505,9 +519,8 @@ __device__ double warp_exact_tau_based(float (&y)[R], int cnt, double lo, double
 {
     const int lane = threadIdx.x & 31;
     warp_sort_desc<R>(y);
-    double best = 0.0;
-    bool found = false;
-    if (n0 > 0.0) found = closed_form_tau(n0, a0, b0, sparsemax, best) || sparsemax;
+    int bk = 0;  // candidates in the support (0: the known part alone)
+    double bx = 0.0, bxx = 0.0;
     float carry1 = 0.f, carry2 = 0.f;
 #pragma unroll
     for (int r = 0; r < R; ++r) {
@@ -527,16 +540,19 @@ __device__ double warp_exact_tau_based(float (&y)[R], int cnt, double lo, double
         const double k = (double)(e + 1);
         const double sx = k * lo + (double)s1;
         const double sxx = k * lo * lo + 2.0 * lo * (double)s1 + (double)s2;
-        double tk = 0.0;
-        const bool real = closed_form_tau(n0 + k, a0 + sx, b0 + sxx, sparsemax, tk);
-        const bool ok = in && real && tk <= lo + (double)yd;
+        const bool ok = in && closed_form_ok(n0 + k, a0 + sx, b0 + sxx, lo + (double)yd, sparsemax);
         const unsigned bal = __ballot_sync(kFull, ok);
-        if (bal) {
-            best = __shfl_sync(kFull, tk, 31 - __clz(bal));  // later rows win
-            found = true;
+        if (bal) {  // later rows win
+            const int src = 31 - __clz(bal);
+            bk = r * 32 + src + 1;
+            bx = __shfl_sync(kFull, sx, src);
+            bxx = __shfl_sync(kFull, sxx, src);
         }
     }
-    return found ? best : lo;
+    if (n0 + bk == 0.0) return lo;
+    double tau = lo;
+    closed_form_tau(n0 + bk, a0 + bx, b0 + bxx, sparsemax, tau);
+    return tau;
 }
 
 // Block-wide suffix sums (inclusive, from the highest thread down) of three doubles.
@@ -707,9 +723,8 @@ __device__ void hist_add_base(Visit &&visit, HistScratch &H, const HistRange &R,
 
 // tau once range R (its logits counted in H.c) brackets it: with at most kHistExact logits in
 // the range one warp solves exactly over them plus the known part; with more (ties to within
-// the last level's bin width), support-refinement rounds from the range's lower edge (each takes
-// the closed-form tau of the known part plus the range's logits above the current tau, which
-// rises monotonically onto the exact one). Every thread of the block must call this.
+// the last level's bin width) the range is taken whole or not at all. Every thread of the
+// block must call this.
 template <typename Visit>
 __device__ double hist_solve(Visit &&visit, HistScratch &H, const HistRange &R, int cnt_range,
                              bool sparsemax)
@@ -752,24 +767,29 @@ __device__ double hist_solve(Visit &&visit, HistScratch &H, const HistRange &R, 
         __syncthreads();
         return tau;
     }
-    double tau = flo, prev = -1.0;
-#pragma unroll 1
-    for (int round = 0; round < 16; ++round) {
-        double acc[3] = {0.0, 0.0, 0.0};
-        visit([&](float x) {
-            const double xd = x;
-            if (R.bin(xd) >= 0 && xd > tau) { acc[0] += 1.0; acc[1] += xd; acc[2] += xd * xd; }
-        });
-        block_sum3(acc, H.wtot);
-        if (acc[0] == prev) break;
-        prev = acc[0];
-        double t2 = tau;
-        if (N0 + acc[0] > 0.0 &&
-            closed_form_tau(N0 + acc[0], A0 + acc[1], B0 + acc[2], sparsemax, t2))
-            tau = fmax(tau, t2);
-        else
-            break;
-    }
+    // more than kHistExact logits within the last level's bin width: ties at the resolution of
+    // the logits. Equal logits are in the support together or not at all, so the range joins
+    // the support as a block if the closed form over the known part plus the whole range falls
+    // below the range, and stays out otherwise.
+    double acc[3] = {0.0, 0.0, 0.0};
+    double rmin = INFINITY;
+    visit([&](float x) {
+        const double xd = x;
+        if (R.bin(xd) >= 0) { acc[0] += 1.0; acc[1] += xd; acc[2] += xd * xd; rmin = fmin(rmin, xd); }
+    });
+    rmin = -warp_max((float)-rmin);
+    block_sum3(acc, H.wtot);
+    if (lane == 0) H.list[warp] = (float)rmin;
+    __syncthreads();
+    float lo_r = H.list[0];
+#pragma unroll
+    for (int w = 1; w < kNW; ++w) lo_r = fminf(lo_r, H.list[w]);
+    __syncthreads();
+    double tau = flo;
+    if (closed_form_tau(N0 + acc[0], A0 + acc[1], B0 + acc[2], sparsemax, tau) && tau < (double)lo_r)
+        return tau;
+    tau = flo;
+    if (N0 > 0.0) closed_form_tau(N0, A0, B0, sparsemax, tau);
     return tau;
 }
 
@@ -799,8 +819,14 @@ __device__ void finish_entmax_cta(const DecodeArgs &a, int b, int h, int hq, int
 
     hist_clear(hist, true);
     const float *ml = a.part_ml + bq * a.NC * 2;
-    float zmax = -INFINITY;
-    for (int ch = tid; ch < nchunks; ch += 256) zmax = fmaxf(zmax, __ldcg(ml + 2 * ch));
+    float zmax = -INFINITY, mv[4];  // chunk maxima; the first 1024 stay in registers
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+        const int ch = tid + 256 * r;
+        mv[r] = ch < nchunks ? __ldcg(ml + 2 * ch) : -INFINITY;
+        zmax = fmaxf(zmax, mv[r]);
+    }
+    for (int ch = tid + 1024; ch < nchunks; ch += 256) zmax = fmaxf(zmax, __ldcg(ml + 2 * ch));
     zmax = warp_max(zmax);
     if (lane == 0) red[warp] = zmax;
     __syncthreads();
@@ -814,12 +840,47 @@ __device__ void finish_entmax_cta(const DecodeArgs &a, int b, int h, int hq, int
     }
     const float thr = zmax - 1.0f;  // the largest weight is at most 1, so tau >= zmax - 1
 
-    // active chunks: those whose maximum exceeds zmax - 1 (no other chunk holds a candidate),
-    // listed in order; with more than kActCap of them every chunk is walked
+    // A lower bound on tau from the chunk maxima: they are logits, and the exact threshold of
+    // any subset of the logits is at most that of all of them. Each warp solves exactly over the
+    // maxima it holds (32, or 128 when there are more than 256 chunks); no logit at or below the
+    // largest bound can carry weight. Candidates are z > thr with x = z - zmax >= clo.
+    double clo = -INFINITY;
+    {
+        float lbw = -INFINITY;
+        if (nchunks <= 256) {
+            float v1[1] = {mv[0] - zmax};
+            const int nv = __popc(__ballot_sync(kFull, mv[0] > thr));
+            if (nv > 1) lbw = (float)warp_exact_tau<1>(v1, nv, sparsemax);
+        } else {
+            float v4[4];
+            int nv = 0;
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                v4[r] = mv[r] - zmax;
+                nv += __popc(__ballot_sync(kFull, mv[r] > thr));
+            }
+            if (nv > 1) lbw = (float)warp_exact_tau<4>(v4, nv, sparsemax);
+        }
+        __syncthreads();  // every warp has read zmax from red[]
+        if (lane == 0) red[warp] = lbw;
+        __syncthreads();
+        float lb = red[0];
+#pragma unroll
+        for (int w = 1; w < kNW; ++w) lb = fmaxf(lb, red[w]);
+        // lowered a little so that the fp32 rounding of the bound never drops a support member
+        clo = (double)lb - 1e-6 * fmax(1.0, fabs((double)lb));
+        __syncthreads();
+    }
+
+    // active chunks: those whose maximum is a candidate (no other chunk holds one), listed in
+    // order; with more than kActCap of them every chunk is walked
     int nact = 0;
     for (int ch0 = 0; ch0 < nchunks; ch0 += 256) {
         const int ch = ch0 + tid;
-        const int keep = ch < nchunks && __ldcg(ml + 2 * ch) > thr;
+        const int r = ch0 >> 8;
+        const float m = r == 0 ? mv[0] : (r == 1 ? mv[1] : (r == 2 ? mv[2] : (r == 3 ? mv[3]
+                      : (ch < nchunks ? __ldcg(ml + 2 * ch) : -INFINITY))));
+        const int keep = m > thr && (double)(m - zmax) >= clo;
         int tot;
         const int pos = nact + block_incl_scan<256>(keep, cn, &tot) - keep;
         if (keep && pos < kActCap) act[pos] = ch;
@@ -840,8 +901,7 @@ __device__ void finish_entmax_cta(const DecodeArgs &a, int b, int h, int hq, int
         const int i = f / CT4;
         return (dense ? i : act[i]) * CT + (f - i * CT4) * 4;
     };
-    // candidates are z > thr with x = z - zmax >= clo (clo rises once the top level is bracketed)
-    double clo = -INFINITY;
+    // (clo rises again once the top level of the threshold bracket is bracketed)
     auto gather = [&]() {
         int cnt = 0;
         for (int f = f0w; f < f1w; f += 32 * UNR) {
@@ -903,29 +963,31 @@ __device__ void finish_entmax_cta(const DecodeArgs &a, int b, int h, int hq, int
 
     double tau;  // in the shifted domain x = z - zmax
     if (!any_over && total <= 128) {
-        // one warp sorts every candidate: element e = r * 32 + lane is the e-th in warp order
+        // one warp sorts every candidate (no block barrier on this path): element e = r * 32 +
+        // lane is the e-th in warp order
         if (warp == 0) {
-            float x[4];
-#pragma unroll
-            for (int r = 0; r < 4; ++r) {
-                const int e = r * 32 + lane;
-                x[r] = -INFINITY;
+            auto load = [&](int e) {
                 int base = 0;
+                float x = -INFINITY;
 #pragma unroll
                 for (int w = 0; w < kNW; ++w) {
-                    if (e >= base && e < base + cn[w]) x[r] = cz[w][e - base];
+                    if (e >= base && e < base + cn[w]) x = cz[w][e - base];
                     base += cn[w];
                 }
-            }
+                return x;
+            };
             double t;
             if (total <= 32) {
-                float x1[1] = {x[0]};
+                float x1[1] = {load(lane)};
                 t = warp_exact_tau<1>(x1, total, sparsemax);
             } else if (total <= 64) {
-                float x2[2] = {x[0], x[1]};
+                float x2[2] = {load(lane), load(32 + lane)};
                 t = warp_exact_tau<2>(x2, total, sparsemax);
             } else {
-                t = warp_exact_tau<4>(x, total, sparsemax);
+                float x4[4];
+#pragma unroll
+                for (int r = 0; r < 4; ++r) x4[r] = load(r * 32 + lane);
+                t = warp_exact_tau<4>(x4, total, sparsemax);
             }
             if (lane == 0) s_tau = t;
         }
@@ -965,9 +1027,10 @@ __device__ void finish_entmax_cta(const DecodeArgs &a, int b, int h, int hq, int
     }
 
     // o = sum over the support of p_i v_i, each warp over its own entries: compact the support
-    // (weight, slot) in place over the gathered list, resolve every slot to its cache row with
-    // all lookups in flight, then stream the V rows UNRV per lane group; a warp whose list
-    // overflowed does this in rounds of at most kCapW entries
+    // (weight, slot) in place over the gathered list, resolve every slot to its cache row (the
+    // chunk kernel recorded the block of every selected page) with all lookups in flight, then
+    // stream the V rows UNRV per lane group; a warp whose list overflowed does this in rounds of
+    // at most kCapW entries
     const char *vc = static_cast<const char *>(c.v_cache);
     const int cidx = lane % W, row = lane / W;
     float acc[EPC];
@@ -976,8 +1039,7 @@ __device__ void finish_entmax_cta(const DecodeArgs &a, int b, int h, int hq, int
     float *sp = cz[warp];  // compacted support weights
     int *sr = cs[warp];    // and slots, then rows as blk * P + t
     const int nitems = over ? (f1w - f0w) * 4 : cnt;
-    const int32_t *sel_row = a.sel_idx + ((size_t)b * H + h) * a.max_sel;
-    const int32_t *pt_row = c.page_table + (size_t)b * c.max_pages;
+    const int32_t *blk_row = a.sel_blk + ((size_t)b * H + h) * a.max_sel;
     int it0 = 0;
     do {
         int ns = 0;
@@ -1009,17 +1071,17 @@ __device__ void finish_entmax_cta(const DecodeArgs &a, int b, int h, int hq, int
             it0 += 32;
         }
         for (int k0 = 0; k0 < ns; k0 += 128) {
-            int sl[4], jv[4];
+            int sl[4], bv[4];
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
                 const int k = k0 + u * 32 + lane;
                 sl[u] = k < ns ? sr[k] : 0;
-                jv[u] = k < ns ? __ldg(sel_row + (sl[u] >> a.Pshift)) : 0;
+                bv[u] = k < ns ? __ldcg(blk_row + (sl[u] >> a.Pshift)) : 0;
             }
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
                 const int k = k0 + u * 32 + lane;
-                if (k < ns) sr[k] = __ldg(pt_row + jv[u]) * P + (sl[u] & (P - 1));
+                if (k < ns) sr[k] = bv[u] * P + (sl[u] & (P - 1));
             }
         }
         __syncwarp();
@@ -1067,7 +1129,7 @@ __device__ void finish_entmax_cta(const DecodeArgs &a, int b, int h, int hq, int
 }
 
 template <int DT, int D, int G, bool SOFTMAX>
-__global__ void __launch_bounds__(256, 4)
+__global__ void __launch_bounds__(256, 3)
 decode_finish_kernel(DecodeArgs a)
 {
     // one CTA per (sequence, query head)
@@ -1093,9 +1155,11 @@ decode_finish_kernel(DecodeArgs a)
 static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 // Workspace layout of one attention mode: [B*H_q][NC][2] chunk (m, l) | [B*H_q][NC][D] chunk
-// sums (softmax) | [B*H_q][NC*CP*P] logits (entmax), each 256-byte aligned.
-static size_t mode_layout(int batch, int H_q, int D, int P, int dtype, int max_sel, bool softmax,
-                          size_t *off_o, size_t *off_logits, int *CP, int *NC)
+// sums (softmax) | [B*H_q][NC*CP*P] logits (entmax) | [B*H_kv][max_sel] cache block of every
+// selected page (entmax), each 256-byte aligned.
+static size_t mode_layout(int batch, int H_q, int H, int D, int P, int dtype, int max_sel,
+                          bool softmax, size_t *off_o, size_t *off_logits, size_t *off_blk,
+                          int *CP, int *NC)
 {
     const int rb = D * (dtype == EKV_BF16 ? 2 : 4);
     // bf16 entmax chunks are one 128-token tensor-core tile
@@ -1107,16 +1171,21 @@ static size_t mode_layout(int batch, int H_q, int D, int P, int dtype, int max_s
     off += align256(BQ * nc * D * sizeof(float));
     if (off_logits) *off_logits = off;
     off += align256(BQ * (size_t)nc * cp * P * sizeof(float));
+    if (off_blk) *off_blk = off;
+    off += align256((size_t)batch * H * max_sel * sizeof(int32_t));
     if (CP) *CP = cp;
     if (NC) *NC = nc;
     return off;
 }
 
 // Bytes that cover every attention mode.
-size_t decode_workspace_bytes_all_modes(int batch, int H_q, int D, int P, int dtype, int max_sel)
+size_t decode_workspace_bytes_all_modes(int batch, int H_q, int H, int D, int P, int dtype,
+                                        int max_sel)
 {
-    const size_t a = mode_layout(batch, H_q, D, P, dtype, max_sel, true, nullptr, nullptr, nullptr, nullptr);
-    const size_t b = mode_layout(batch, H_q, D, P, dtype, max_sel, false, nullptr, nullptr, nullptr, nullptr);
+    const size_t a = mode_layout(batch, H_q, H, D, P, dtype, max_sel, true, nullptr, nullptr,
+                                 nullptr, nullptr, nullptr);
+    const size_t b = mode_layout(batch, H_q, H, D, P, dtype, max_sel, false, nullptr, nullptr,
+                                 nullptr, nullptr, nullptr);
     return a > b ? a : b;
 }
 
@@ -1191,9 +1260,9 @@ cudaError_t launch_sparse_decode(const ekv_cache &c, const void *q, int H_q, flo
                                  bool pdl)
 {
     DecodeArgs a;
-    size_t off_o, off_logits;
-    mode_layout(c.batch, H_q, c.head_dim, c.page_size, c.dtype, max_sel, attn == EKV_SOFTMAX,
-                &off_o, &off_logits, &a.CP, &a.NC);
+    size_t off_o, off_logits, off_blk;
+    mode_layout(c.batch, H_q, c.num_kv_heads, c.head_dim, c.page_size, c.dtype, max_sel,
+                attn == EKV_SOFTMAX, &off_o, &off_logits, &off_blk, &a.CP, &a.NC);
     a.LS = a.NC * a.CP * c.page_size;
     a.Pshift = c.page_size == 16 ? 4 : (c.page_size == 32 ? 5 : 6);
     a.c = c;
@@ -1207,6 +1276,7 @@ cudaError_t launch_sparse_decode(const ekv_cache &c, const void *q, int H_q, flo
     a.part_ml = static_cast<float *>(ws);
     a.part_o = reinterpret_cast<float *>(static_cast<char *>(ws) + off_o);
     a.logits = reinterpret_cast<float *>(static_cast<char *>(ws) + off_logits);
+    a.sel_blk = reinterpret_cast<int32_t *>(static_cast<char *>(ws) + off_blk);
     a.out = out;
     a.stat = stat;
     const bool softmax = attn == EKV_SOFTMAX;

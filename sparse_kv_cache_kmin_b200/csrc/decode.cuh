@@ -22,6 +22,7 @@ struct DecodeArgs {
     float *part_ml; // [B * H_q][NC][2]   softmax (m, l); entmax (max z, unused)
     float *part_o;  // [B * H_q][NC][D]   softmax sum p v
     float *logits;  // [B * H_q][LS]       entmax z
+    int32_t *sel_blk;  // [B * H_kv][max_sel] entmax: cache block of selected page i (-1: none)
     float *out;
     float *stat;
 };

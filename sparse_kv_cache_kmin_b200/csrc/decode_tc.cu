@@ -150,6 +150,7 @@ decode_chunk_tc_kernel(const __grid_constant__ CUtensorMap kmap,
                             nt = len - j * P < P ? len - j * P : P;
                         }
                     }
+                    a.sel_blk[(size_t)bh * a.max_sel + i] = nt > 0 ? blk : -1;  // for the finish
                 }
             }
             // 3. one record per chunk (an end mark when there are none left)

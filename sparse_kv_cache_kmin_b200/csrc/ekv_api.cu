@@ -23,7 +23,8 @@ cudaError_t launch_sparse_decode(const ekv_cache &c, const void *q, int H_q, flo
                                  int attn, const int32_t *sel_idx, const int32_t *sel_count,
                                  int max_sel, float *out, float *stat, void *ws, cudaStream_t st,
                                  bool pdl);
-size_t decode_workspace_bytes_all_modes(int batch, int H_q, int D, int P, int dtype, int max_sel);
+size_t decode_workspace_bytes_all_modes(int batch, int H_q, int H, int D, int P, int dtype,
+                                        int max_sel);
 
 int persistent_grid_size(const void *kernel, int threads, size_t smem)
 {
@@ -143,8 +144,8 @@ size_t ekv_decode_workspace_bytes(const ekv_cache *c, int32_t num_q_heads, int32
 {
     if (check_cache(c, false) != EKV_OK || check_heads(c, num_q_heads) != EKV_OK || max_sel < 1)
         return 0;
-    return decode_workspace_bytes_all_modes(c->batch, num_q_heads, c->head_dim, c->page_size,
-                                            c->dtype, max_sel);
+    return decode_workspace_bytes_all_modes(c->batch, num_q_heads, c->num_kv_heads, c->head_dim,
+                                            c->page_size, c->dtype, max_sel);
 }
 
 ekv_status ekv_sparse_decode(const ekv_cache *c, const void *q, int32_t num_q_heads,

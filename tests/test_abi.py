@@ -115,8 +115,9 @@ def test_decode_validation_and_workspace(lib):
     P = 0x1000
     need = lib.ekv_decode_workspace_bytes(ctypes.byref(c), 32, 256)
     assert need > 0
-    # [B*H_q][NC][2] + [B*H_q][NC][D] + [B*H_q][NC*CP*P] floats, each 256-byte aligned
-    assert need >= 4 * 32 * 256 * 16 * 4
+    # [B*H_q][NC][2] + [B*H_q][NC][D] + [B*H_q][NC*CP*P] floats + [B*H_kv][max_sel] ints,
+    # each 256-byte aligned
+    assert need >= 4 * 32 * 256 * 16 * 4 + 4 * 8 * 256 * 4
     assert lib.ekv_decode_workspace_bytes(ctypes.byref(c), 30, 256) == 0
     assert lib.ekv_sparse_decode(ctypes.byref(c), P, 32, 1.0, 1, P, P, 256, P, P, P, need - 1, None) == 3
     assert lib.ekv_sparse_decode(ctypes.byref(c), P, 32, 1.0, 1, P, P, 256, P, P, None, need, None) == 3
