@@ -1162,8 +1162,10 @@ static size_t mode_layout(int batch, int H_q, int H, int D, int P, int dtype, in
                           int *CP, int *NC)
 {
     const int rb = D * (dtype == EKV_BF16 ? 2 : 4);
-    // bf16 entmax chunks are one 128-token tensor-core tile
-    const int cp = (dtype == EKV_BF16 && !softmax) ? 128 / P : chunk_tokens(rb, P, softmax) / P;
+    // bf16 chunks served by the tensor-core kernels are one 128-token tile (entmax; softmax at
+    // d = 128)
+    const bool tc = dtype == EKV_BF16 && (!softmax || D == 128);
+    const int cp = tc ? 128 / P : chunk_tokens(rb, P, softmax) / P;
     const int nc = (max_sel + cp - 1) / cp;
     const size_t BQ = (size_t)batch * H_q;
     size_t off = align256(BQ * nc * 2 * sizeof(float));
@@ -1216,6 +1218,7 @@ static cudaError_t launch_chunk(const DecodeArgs &a, cudaLaunchConfig_t cfg)
 
 bool tc_chunk_supported(const ekv_cache &c, int H_q, bool softmax);
 cudaError_t launch_chunk_tc(const DecodeArgs &a, int G, cudaLaunchConfig_t cfg);
+cudaError_t launch_softmax_tc(const DecodeArgs &a, int G, cudaLaunchConfig_t cfg);
 
 template <int DT, int D, int G>
 static cudaError_t launch_decode_t(const DecodeArgs &a, bool softmax, cudaStream_t st, bool pdl)
@@ -1228,12 +1231,11 @@ static cudaError_t launch_decode_t(const DecodeArgs &a, bool softmax, cudaStream
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
     cudaError_t e;
+    const bool tc = DT == EKV_BF16 && tc_chunk_supported(a.c, a.H_q, softmax);
     if (softmax)
-        e = launch_chunk<DT, D, G, true>(a, cfg);
-    else if (DT == EKV_BF16 && tc_chunk_supported(a.c, a.H_q, false))
-        e = launch_chunk_tc(a, G, cfg);
+        e = tc ? launch_softmax_tc(a, G, cfg) : launch_chunk<DT, D, G, true>(a, cfg);
     else
-        e = launch_chunk<DT, D, G, false>(a, cfg);
+        e = tc ? launch_chunk_tc(a, G, cfg) : launch_chunk<DT, D, G, false>(a, cfg);
     if (e != cudaSuccess) return e;
     cfg.blockDim = dim3(256);
     cfg.dynamicSmemBytes = 0;

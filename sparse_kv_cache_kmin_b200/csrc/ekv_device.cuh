@@ -314,4 +314,18 @@ __device__ __forceinline__ void named_sync(int id, int threads)
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
+// Named barrier that also ANDs a flag over the participating threads: every thread gets the
+// same answer, so a group of warps leaves a loop together or not at all.
+__device__ __forceinline__ bool named_sync_and(int id, int threads, bool v)
+{
+    uint32_t r;
+    asm volatile(
+        "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.and.pred q, %2, %3, p;\n"
+        " selp.u32 %0, 1, 0, q;\n}"
+        : "=r"(r)
+        : "r"((uint32_t)v), "r"(id), "r"(threads)
+        : "memory");
+    return r != 0;
+}
+
 }  // namespace ekv

@@ -35,12 +35,28 @@ __device__ __forceinline__ uint64_t sw128_kmajor_desc(const void *smem_ptr)
            (2ull << 61);
 }
 
+// ---- descriptor of an MN-major operand in the 128-byte swizzled layout: each 128-byte row
+// holds 64 consecutive bf16 of M (or N) for one K index, 8 K rows form a 1024-byte swizzle atom;
+// atoms along K are 1024 bytes apart (stride byte offset) and 64-element blocks along M are
+// `lbo_bytes` apart (leading byte offset).
+__device__ __forceinline__ uint64_t sw128_mnmajor_desc(const void *smem_ptr, uint32_t lbo_bytes)
+{
+    const uint64_t addr = smem_addr(smem_ptr);
+    return ((addr >> 4) & 0x3FFFull) | ((uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16) |
+           ((1024ull >> 4) << 32) | (1ull << 46) | (2ull << 61);
+}
+
 // ---- instruction descriptor of tcgen05.mma.kind::f16: bf16 A and B (K-major), fp32 D,
 // M x N tile: D format (bits 4-5) = 1 (f32), A format (7-9) = 1 (bf16), B format (10-12) = 1,
 // N >> 3 (17-22), M >> 4 (24-28).
 __host__ __device__ constexpr uint32_t mma_idesc_bf16_f32(int M, int N)
 {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+// the same with A MN-major (bit 15)
+__host__ __device__ constexpr uint32_t mma_idesc_bf16_f32_amn(int M, int N)
+{
+    return mma_idesc_bf16_f32(M, N) | (1u << 15);
 }
 
 // D[tmem] (+)= A[smem] * B[smem]^T, issued by one thread
