@@ -709,7 +709,13 @@ static cudaError_t launch_tc_t(const DecodeArgs &a, cudaLaunchConfig_t cfg)
     cfg.blockDim = dim3(kTcThreads);
     cfg.dynamicSmemBytes = L::SMEM;
     const long long items = (long long)c.batch * c.num_kv_heads * a.NC;
-    const long long grid = persistent_grid_size((const void *)k, kTcThreads, L::SMEM);
+    // two CTAs per SM fit (2 x (L::SMEM + static + reserved) is below the 228 KiB of an SM);
+    // the occupancy query reports one, so size the grid from the SM count directly. CTAs never
+    // wait on one another, so an over-full grid would only queue.
+    int sms = 148, dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const long long grid = 2ll * sms;
     cfg.gridDim = dim3((unsigned)(items < grid ? items : grid));
     return cudaLaunchKernelEx(&cfg, k, kmap, qmap, a);
 }
