@@ -29,6 +29,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "sparse decode steps/s at 128K ctx; achieved HBM GB/s vs ~8 TB/s peak"
 ATTN_NAME = {0: "softmax", 1: "entmax1.5", 2: "sparsemax"}
+POLICY_NAME = {0: "topk", 1: "gauss", 2: "gauss_max"}
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -47,6 +48,9 @@ def parse():
                     help="override the workload's batch (smaller cases for profiler captures)")
     ap.add_argument("--no-full-cache", action="store_true",
                     help="skip the full-cache decode (every page selected) timed for comparison")
+    ap.add_argument("--policy", default=None, choices=["topk", "gauss", "gauss_max"],
+                    help="selection policy (default: the workload's); gauss_max is the estimated-"
+                         "maximum reading of the Gaussian rule")
     return ap.parse_args()
 
 
@@ -64,7 +68,7 @@ def step_bytes(wl, dec, attn):
     lens = wl.seq_lens.long().cpu()
     n_pages = (lens + P - 1) // P
     total_pages = int(n_pages.sum())
-    meta_row = 2 * d * esz + (2 * d * 4 if wl.policy == 1 else 0)
+    meta_row = 2 * d * esz + (2 * d * 4 if wl.policy != 0 else 0)
     meta = total_pages * H * meta_row
     ptab = total_pages * 4
     qb = wl.q.numel() * wl.q.element_size()
@@ -235,8 +239,7 @@ def oracle_sample(wl, attn, budget_s, max_heads=None):
         meta = O.page_meta_head(hc.k, hc.pt, hc.L, h)  # built at prefill, not part of a step
         t0 = time.perf_counter()
         O.decode_step_head(hc.k, hc.v, hc.pt, hc.L, h, hc.q[h], wl.scale, mode,
-                           "topk" if wl.policy == 0 else "gauss", wl.topk, wl.alpha, wl.delta,
-                           meta=meta)
+                           POLICY_NAME[wl.policy], wl.topk, wl.alpha, wl.delta, meta=meta)
         if wl.append is not None:  # the step also rebuilds the appended page's metadata
             O.page_meta_head(hc.k[-1:], np.zeros(1, np.int32), hc.L - (hc.np - 1) * wl.page_size, h)
         spent += time.perf_counter() - t0
@@ -287,7 +290,49 @@ def full_cache_time(ekv, cache, wl, attn, steps, flush, stream):
         ev[i][1].record(stream)
     torch.cuda.synchronize()
     del g
-    return statistics.mean(a.elapsed_time(b) for a, b in ev)
+    return statistics.mean(a.elapsed_time(b) for a, b in ev), out, stat
+
+
+def selection_quality(wl, dec, attn, stat_full):
+    """How much of the full-cache attention the selection keeps, per query: the dropped mass
+    delta = sum of full-cache weights on tokens outside the selected pages (the quantity of the
+    2 B delta error bound) and, for entmax, the recall of the full-cache support. Computed with
+    torch on the GPU from the cache and the full-cache stat, outside every timed region."""
+    P, H = wl.page_size, wl.num_kv_heads
+    G = wl.num_q_heads // H
+    alpha = {1: 1.5, 2: 2.0}.get(attn)
+    deltas, recalls = [], []
+    for b in range(wl.batch):
+        L = int(wl.seq_lens[b])
+        n = (L + P - 1) // P
+        blk = wl.page_table[b, :n].long()
+        valid = (torch.arange(n, device=blk.device)[:, None] * P
+                 + torch.arange(P, device=blk.device)[None, :]) < L
+        for h in range(H):
+            kk = wl.k_cache[blk, h].float()                          # [n, P, d]
+            q = wl.q[b, h * G:(h + 1) * G].float()                   # [G, d]
+            s = wl.scale * torch.einsum("npd,gd->gnp", kk, q)
+            st = stat_full[b, h * G:(h + 1) * G].float()[:, None, None]
+            if alpha is None:
+                p = torch.exp(s - st)
+            else:
+                p = torch.clamp((alpha - 1.0) * s - st, min=0.0) ** (1.0 / (alpha - 1.0))
+            p = p * valid
+            kept = torch.zeros(n, dtype=torch.bool, device=p.device)
+            cnt = int(dec.sel_count[b, h])
+            kept[dec.sel_idx[b, h, :cnt].long()] = True
+            deltas += (p * (~kept)[None, :, None]).sum((1, 2)).tolist()
+            if alpha is not None:
+                sup = p > 0
+                recalls += ((sup & kept[None, :, None]).sum((1, 2)).float()
+                            / sup.sum((1, 2)).clamp(min=1).float()).tolist()
+    out = {"dropped_mass_mean": statistics.mean(deltas), "dropped_mass_max": max(deltas),
+           "kept_pages_mean": float(dec.sel_count.float().mean()),
+           "pages_mean": float(((wl.seq_lens.float() + P - 1) // P).mean())}
+    if recalls:
+        out["support_recall_mean"] = statistics.mean(recalls)
+        out["support_recall_min"] = min(recalls)
+    return out
 
 # ----------------------------------------------------------------------------- main
 def main():
@@ -317,11 +362,15 @@ def main():
     kw = {"B": args.batch} if args.batch else {}
     wl = make(args.workload, device=dev, seed=replicas.workload_seed(args.workload, rank), **kw)
     attn = wl.attn_modes[0] if args.attn is None else args.attn
+    if args.policy is not None:
+        wl.policy = {v: k for k, v in POLICY_NAME.items()}[args.policy]
+        if wl.policy == 0 and not wl.topk:
+            raise SystemExit("--policy topk needs a workload with a top-k budget")
     nb, H, P, d = wl.k_cache.shape
     cache = ekv.PagedKVCache(
         k_cache=wl.k_cache, v_cache=wl.v_cache,
         meta_bbox=torch.empty((nb, H, 2, d), dtype=wl.k_cache.dtype, device=dev),
-        meta_mom=torch.empty((nb, H, 2, d), dtype=torch.float32, device=dev) if wl.policy == 1 else None,
+        meta_mom=torch.empty((nb, H, 2, d), dtype=torch.float32, device=dev) if wl.policy != 0 else None,
         page_table=wl.page_table, seq_lens=wl.seq_lens,
         dev_status=torch.zeros(1, dtype=torch.int32, device=dev))
     B = wl.batch
@@ -436,9 +485,11 @@ def main():
     e2e_s = replicas.max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e_ev) / 1e3, device=dev)
     d2h = out_host.numel() * 4 + stat_host.numel() * 4
 
-    full_ms = None
+    full_ms, quality = None, None
     if not args.no_full_cache and world == 1:
-        full_ms = full_cache_time(ekv, cache, wl, attn, min(args.steps, 20), flush, stream)
+        full_ms, _, stat_full = full_cache_time(ekv, cache, wl, attn, min(args.steps, 20), flush,
+                                                stream)
+        quality = selection_quality(wl, dec, attn, stat_full)
         st, bits = ekv.ekv_device_status(cache)
         if st != ekv.EKV_OK:
             raise RuntimeError("device status 0x%x after the full-cache decode" % bits)
@@ -472,7 +523,7 @@ def main():
         "data": "synthetic (seeded; rank r decodes its own batch)",
         "config": {"workload": wl.name, "batch_per_gpu": B, "ctx": int(wl.seq_lens.max()),
                    "q_heads": wl.num_q_heads, "kv_heads": H, "head_dim": d, "page": P,
-                   "policy": "top-k %d" % wl.topk if wl.policy == 0 else "gaussian delta %g" % wl.delta,
+                   "policy": "top-k %d" % wl.topk if wl.policy == 0 else "%s delta %g" % (POLICY_NAME[wl.policy], wl.delta),
                    "attn": ATTN_NAME[attn], "l2": "flushed before every step (256 MiB write, outside the timed events)",
                    "parallelism": "replicas x%d, no collective" % world},
         "hbm": {"required_bytes_per_step": by["required_step"],
@@ -492,6 +543,7 @@ def main():
             "what": "the same attention over every page (no scoring, no selection) on this GPU",
             "ms_per_step": full_ms, "steps_per_s": 1e3 / full_ms,
             "sparse_speedup": full_ms / ms},
+        "selection_quality": quality,
         "e2e": {"value": replicas.job_rate(args.steps, world, e2e_s), "unit": "steps/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * args.steps,
@@ -513,6 +565,8 @@ def reference_arm(args, rank, world, make):
     from sparse_kv_cache_kmin_b200 import replicas
     wl = make(args.workload, device=dev, seed=replicas.workload_seed(args.workload, 0))
     attn = wl.attn_modes[0] if args.attn is None else args.attn
+    if args.policy is not None:
+        wl.policy = {v: k for k, v in POLICY_NAME.items()}[args.policy]
     n_steps = max(args.warmup, 3) + args.steps
     budget = max(2.0, 150.0 / n_steps)  # the whole run stays within a few minutes
     times = []

@@ -55,7 +55,7 @@ typedef enum { EKV_F32 = 0, EKV_BF16 = 1 } ekv_dtype;
 typedef enum { EKV_SOFTMAX = 0, EKV_ENTMAX15 = 1, EKV_SPARSEMAX = 2 } ekv_attn;
 
 /* candidate selection policy (§2.B) */
-typedef enum { EKV_SEL_TOPK = 0, EKV_SEL_GAUSS = 1 } ekv_policy;
+typedef enum { EKV_SEL_TOPK = 0, EKV_SEL_GAUSS = 1, EKV_SEL_GAUSS_MAX = 2 } ekv_policy;
 
 /* bits OR-ed into *dev_status by kernels that meet bad input */
 #define EKV_DEV_BAD_BLOCK 0x1u    /* page-table entry outside [0, num_blocks)            */
@@ -73,7 +73,7 @@ typedef enum { EKV_SEL_TOPK = 0, EKV_SEL_GAUSS = 1 } ekv_policy;
  *   meta_bbox         [num_blocks][H_kv][2][d] in `dtype`: row 0 kmin, row 1 kmax of the
  *                     page's valid keys (exact: min/max of stored values).
  *   meta_mom          [num_blocks][H_kv][2][d] fp32: row 0 mean, row 1 population variance of
- *                     the page's valid keys. NULL is allowed unless EKV_SEL_GAUSS is used.
+ *                     the page's valid keys. NULL is allowed unless a Gaussian policy is used.
  *   page_table        [batch][max_pages] int32: logical page j of sequence b is block
  *                     page_table[b * max_pages + j].
  *   seq_lens          [batch] int32: tokens in each sequence.
@@ -119,12 +119,12 @@ ekv_status ekv_page_meta_update(const ekv_cache *c, const int32_t *new_start,
  *   scale   logit scale (> 0): s = scale * q.k.
  *   policy  EKV_SEL_TOPK: scores is [batch][H_kv][max_pages] fp32 and holds the group bound
  *             S_j = sum_{g in group} UB_{g,j},  UB_{g,j} = scale * sum_c max(q_gc kmin_jc, q_gc kmax_jc).
- *           EKV_SEL_GAUSS: scores is [batch][num_q_heads][3][max_pages] fp32 and holds, per
+ *           EKV_SEL_GAUSS, EKV_SEL_GAUSS_MAX: scores is [batch][num_q_heads][3][max_pages] fp32 and holds, per
  *             query, UB_{g,j}, m_{g,j} = scale * q_g.mean_j and
  *             v_{g,j} = scale^2 * sum_c q_gc^2 var_jc (needs c->meta_mom).
  * Entries for pages j >= ceil(seq_lens[b] / P) are not written. A page whose page-table entry
  * is out of range scores -inf (and m = v = 0) and is flagged.
- * c->meta_bbox (and c->meta_mom for EKV_SEL_GAUSS) must be 16-byte aligned: metadata rows are
+ * c->meta_bbox (and c->meta_mom for the Gaussian policies) must be 16-byte aligned: metadata rows are
  * read with 16-byte vector loads (EKV_ERR_INVALID_ARG otherwise).
  */
 ekv_status ekv_score_pages(const ekv_cache *c, const void *q, int32_t num_q_heads, float scale,
@@ -141,6 +141,10 @@ ekv_status ekv_score_pages(const ekv_cache *c, const void *q, int32_t num_q_head
  *     the group has (alpha-1) * UB_{g,j} > tau_hat_g - delta. tau_hat: [batch][num_q_heads]
  *     fp32 output (-inf for an empty sequence). More than max_sel kept pages: the first
  *     max_sel (ascending) are emitted, sel_count holds max_sel, EKV_DEV_SEL_OVERFLOW is set.
+ *   EKV_SEL_GAUSS_MAX: the same tau_hat, with the second reading of §2.B.2's "estimated
+ *     maximum score": page j is kept iff some query g has (alpha-1) * est_{g,j} >
+ *     tau_hat_g - delta, est = min(UB_{g,j}, m_{g,j} + sqrt(2 ln n_j) * sqrt(v_{g,j})) -- the
+ *     Gaussian estimate of the page's largest score, capped by the bound (fp64 decision).
  *   scores     as written by ekv_score_pages with the same policy.
  *   sel_idx    [batch][H_kv][max_sel] int32 output: logical page indices, ascending, then -1.
  *   sel_count  [batch][H_kv] int32 output.

@@ -55,6 +55,10 @@ def _load():
     lib.ora_gauss_tau.restype = c_double
     lib.ora_gauss_select.argtypes = [_dp, _dp, c_int, c_int, c_double, c_double, _ip]
     lib.ora_gauss_select.restype = c_int
+    lib.ora_est_max.argtypes = [c_double, c_double, c_double, c_int]
+    lib.ora_est_max.restype = c_double
+    lib.ora_gauss_select_est.argtypes = [_dp, _dp, _dp, _ip, _dp, c_int, c_int, c_double, c_double, _ip]
+    lib.ora_gauss_select_est.restype = c_int
     lib.ora_entmax_tau.argtypes = [_dp, c_int, c_double]
     lib.ora_entmax_tau.restype = c_double
     lib.ora_attend_head.argtypes = [vp, vp, c_int, c_int, c_int, c_int, c_int, _ip, c_int, c_int,
@@ -167,6 +171,24 @@ def gauss_select(ub, tau_hat, alpha: float, delta: float) -> np.ndarray:
     return out[:cnt].copy()
 
 
+def est_max(ub: float, m: float, v: float, n: int) -> float:
+    return _load().ora_est_max(float(ub), float(m), float(v), int(n))
+
+
+def gauss_select_est(ub, m, v, cnt, tau_hat, alpha: float, delta: float) -> np.ndarray:
+    """The Gaussian rule with the capped Gaussian estimate of each page's maximum."""
+    ub, up = _d(np.atleast_2d(ub))
+    m, mp = _d(np.atleast_2d(m))
+    v, vp_ = _d(np.atleast_2d(v))
+    cnt, cp = _i(cnt)
+    tau_hat, tp = _d(np.atleast_1d(tau_hat))
+    G, n = ub.shape
+    out = np.zeros(max(n, 1), dtype=np.int32)
+    k = _load().ora_gauss_select_est(up, mp, vp_, cp, tp, G, n, float(alpha), float(delta),
+                                     out.ctypes.data_as(_ip))
+    return out[:k].copy()
+
+
 # ----------------------------------------------------------------------------- §2.C attention
 def entmax_tau(z, alpha: float) -> float:
     z, zp = _d(np.atleast_1d(z))
@@ -221,7 +243,7 @@ def decode_step_head(k_cache, v_cache, pt_row, seq_len, h, q_group, scale, mode,
                      topk_k=0, alpha=1.5, delta=0.0, meta=None):
     """One full decode step (score -> select -> attend) for one (sequence, KV head).
 
-    policy: "topk" or "gauss". `meta` is (kmin, kmax, mean, var) for this (sequence, head);
+    policy: "topk", "gauss" or "gauss_max". `meta` is (kmin, kmax, mean, var) for this (sequence, head);
     computed from scratch here when None. Returns a dict with every intermediate."""
     if meta is None:
         meta = page_meta_head(k_cache, pt_row, seq_len, h)
@@ -234,7 +256,10 @@ def decode_step_head(k_cache, v_cache, pt_row, seq_len, h, q_group, scale, mode,
         m, v = gauss_stats_head(q_group, scale, mean, var)
         cnt = page_counts(seq_len, k_cache.shape[2])
         tau_hat = np.array([gauss_tau(m[g], v[g], cnt, alpha) for g in range(m.shape[0])])
-        sel = gauss_select(ub, tau_hat, alpha, delta)
+        if policy == "gauss_max":
+            sel = gauss_select_est(ub, m, v, cnt, tau_hat, alpha, delta)
+        else:
+            sel = gauss_select(ub, tau_hat, alpha, delta)
         res.update(m=m, v=v, tau_hat=tau_hat)
     out, stat, _ = attend_head(k_cache, v_cache, pt_row, seq_len, h, q_group, scale, mode, sel)
     res.update(sel=sel, out=out, stat=stat)

@@ -24,7 +24,9 @@
  *     in the z = (alpha-1) s domain as p_i = [z_i - tau]_+^(1/(alpha-1));
  *   - a GQA group of G query heads shares one KV head; the top-k page score is the sum of the
  *     G per-query bounds; the Gaussian policy solves tau-hat per query and keeps the union;
- *   - the "estimated maximum score" of §2.B.2 is the bounding-box bound itself;
+ *   - the "estimated maximum score" of §2.B.2 is the bounding-box bound itself; a second
+ *     reading, the Gaussian estimate of a page's maximum capped by that bound,
+ *     min(UB, m + sqrt(2 ln n_j) sqrt(v)), is offered beside it (ora_gauss_select_est);
  *   - the margin is in the z domain: keep page j iff (alpha-1)*UB > tau-hat - Delta;
  *   - page variance is per coordinate and population (divide by the count n);
  *   - the approximate normalisation equation replaces each page's n_j token scores by n_j
@@ -283,6 +285,37 @@ int ora_gauss_select(const double *ub, const double *tau_hat, int G, int n_pages
             sel[cnt++] = j;
     }
     return cnt;
+}
+
+/* Second reading of the "estimated maximum score" (§2.B.2): a page's n token scores are modelled
+ * as n draws from N(m, v); the expected largest of n standard normal draws is at most
+ * sqrt(2 ln n), so m + sqrt(2 ln n) sqrt(v) estimates the page maximum. The bounding-box bound
+ * holds exactly, so the estimate is capped by it. One token: the estimate is m (v = 0). */
+double ora_est_max(double ub, double m, double v, int n)
+{
+    const double z = n > 1 ? sqrt(2.0 * log((double)n)) : 0.0;
+    const double e = m + z * sqrt(v > 0.0 ? v : 0.0);
+    return e < ub ? e : ub;
+}
+
+/* Keep page j iff some query g has (alpha-1) * est_{g,j} > tau_hat_g - delta, with est the
+ * capped Gaussian estimate above. ub, m, v: [G][n_pages]; cnt: the pages' token counts. */
+int ora_gauss_select_est(const double *ub, const double *m, const double *v, const int32_t *cnt,
+                         const double *tau_hat, int G, int n_pages, double alpha, double delta,
+                         int32_t *sel)
+{
+    int kept = 0;
+    for (int j = 0; j < n_pages; ++j) {
+        int keep = 0;
+        for (int g = 0; g < G; ++g) {
+            const size_t i = (size_t)g * n_pages + j;
+            if ((alpha - 1.0) * ora_est_max(ub[i], m[i], v[i], cnt[j]) > tau_hat[g] - delta)
+                keep = 1;
+        }
+        if (keep)
+            sel[kept++] = j;
+    }
+    return kept;
 }
 
 /* ---------------------------------------------------------------------------------------

@@ -8,7 +8,7 @@ script (``build``). Nothing falls back to a CPU path: without the library, calls
 from .ekv import (ALPHA, EKV_BF16, EKV_DEV_BAD_BLOCK, EKV_DEV_BAD_LEN, EKV_DEV_BAD_RANGE,
                   EKV_DEV_BAD_SEL, EKV_DEV_SEL_OVERFLOW, EKV_ENTMAX15, EKV_ERR_CUDA,
                   EKV_ERR_DEVICE, EKV_ERR_INVALID_ARG, EKV_ERR_UNSUPPORTED, EKV_ERR_WORKSPACE,
-                  EKV_F32, EKV_OK, EKV_SEL_GAUSS, EKV_SEL_TOPK, EKV_SOFTMAX, EKV_SPARSEMAX,
+                  EKV_F32, EKV_OK, EKV_SEL_GAUSS, EKV_SEL_GAUSS_MAX, EKV_SEL_TOPK, EKV_SOFTMAX, EKV_SPARSEMAX,
                   EkvError, PagedKVCache, ekv_clear_device_status, ekv_decode_workspace_bytes,
                   ekv_device_status, ekv_page_meta_update, ekv_score_pages, ekv_select_pages,
                   ekv_sparse_decode, load_library)

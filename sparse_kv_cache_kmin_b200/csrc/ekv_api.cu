@@ -108,10 +108,12 @@ ekv_status ekv_score_pages(const ekv_cache *c, const void *q, int32_t num_q_head
     if (s != EKV_OK) return s;
     if ((s = check_heads(c, num_q_heads)) != EKV_OK) return s;
     if (!q || !scores || !(scale > 0.0f) || !std::isfinite(scale)) return EKV_ERR_INVALID_ARG;
-    if (policy != EKV_SEL_TOPK && policy != EKV_SEL_GAUSS) return EKV_ERR_UNSUPPORTED;
-    if (policy == EKV_SEL_GAUSS && !c->meta_mom) return EKV_ERR_INVALID_ARG;
+    if (policy != EKV_SEL_TOPK && policy != EKV_SEL_GAUSS && policy != EKV_SEL_GAUSS_MAX)
+        return EKV_ERR_UNSUPPORTED;
+    const bool gauss = policy != EKV_SEL_TOPK;
+    if (gauss && !c->meta_mom) return EKV_ERR_INVALID_ARG;
     if ((uintptr_t)c->meta_bbox & 15u) return EKV_ERR_INVALID_ARG;
-    if (policy == EKV_SEL_GAUSS && ((uintptr_t)c->meta_mom & 15u)) return EKV_ERR_INVALID_ARG;
+    if (gauss && ((uintptr_t)c->meta_mom & 15u)) return EKV_ERR_INVALID_ARG;
     return cuda_status(launch_score_pages(*c, q, num_q_heads, scale, policy, scores,
                                           static_cast<cudaStream_t>(stream), use_pdl()));
 }
@@ -129,7 +131,7 @@ ekv_status ekv_select_pages(const ekv_cache *c, int32_t num_q_heads, int32_t pol
         if (topk < 1) return EKV_ERR_INVALID_ARG;
         const int need = topk < c->max_pages ? topk : c->max_pages;
         if (max_sel < need) return EKV_ERR_INVALID_ARG;
-    } else if (policy == EKV_SEL_GAUSS) {
+    } else if (policy == EKV_SEL_GAUSS || policy == EKV_SEL_GAUSS_MAX) {
         if (alpha != 1.5f && alpha != 2.0f) return EKV_ERR_UNSUPPORTED;
         if (!tau_hat || !std::isfinite(delta)) return EKV_ERR_INVALID_ARG;
     } else {

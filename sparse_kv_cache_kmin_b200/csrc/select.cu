@@ -304,7 +304,7 @@ __global__ void __launch_bounds__(256)
 select_gauss_kernel(const float *__restrict__ scores, int H, int max_pages, int P,
                     const int32_t *__restrict__ seq_lens, float alpha, float delta,
                     int32_t *__restrict__ sel_idx, int32_t *__restrict__ sel_count, int max_sel,
-                    float *__restrict__ tau_hat, uint32_t *status, int capw)
+                    float *__restrict__ tau_hat, uint32_t *status, int capw, bool est_max)
 {
     constexpr int NT = 256, WPQ = 8 / G;
     extern __shared__ float gdyn[];
@@ -458,17 +458,30 @@ select_gauss_kernel(const float *__restrict__ scores, int H, int max_pages, int 
     __syncthreads();
 
     // union over the group, ascending page order: warp w owns pages [q0, q1) in 32-page rows;
-    // the first pass counts, the second writes at the warp's offset
+    // the first pass counts, the second writes at the warp's offset. The page statistic is the
+    // bound UB, or (est_max) the Gaussian estimate of the page maximum capped by the bound,
+    // min(UB, m + sqrt(2 ln n) sqrt(v)), decided in fp64.
     const float *ub0 = scores + ((size_t)b * H_q + h * G) * 3 * max_pages;
     double thr[G];
 #pragma unroll
     for (int g = 0; g < G; ++g) thr[g] = s_tau[g] - (double)delta;
     auto keep_page = [&](int j) {
         bool keep = false;
+        double zn = 0.0;
+        if (est_max) {
+            const int nj = len - j * P < P ? len - j * P : P;
+            zn = nj > 1 ? sqrt(2.0 * log((double)nj)) : 0.0;
+        }
 #pragma unroll
         for (int g = 0; g < G; ++g) {
-            const float ub = __ldcg(ub0 + (size_t)g * 3 * max_pages + j);
-            keep |= (double)am1 * (double)ub > thr[g];
+            const float *row = ub0 + (size_t)g * 3 * max_pages + j;
+            double x = (double)__ldcg(row);
+            if (est_max) {
+                const double e = (double)__ldcg(row + max_pages) +
+                                 zn * sqrt(fmax((double)__ldcg(row + 2 * (size_t)max_pages), 0.0));
+                x = e < x ? e : x;
+            }
+            keep |= (double)am1 * x > thr[g];
         }
         return keep;
     };
@@ -562,7 +575,8 @@ cudaError_t launch_select_pages(const ekv_cache &c, int H_q, int policy, int top
         }                                                                                      \
         return cudaLaunchKernelEx(&cfg, select_gauss_kernel<GG>, scores, c.num_kv_heads,       \
                                   c.max_pages, c.page_size, c.seq_lens, alpha, delta, sel_idx, \
-                                  sel_count, max_sel, tau_hat, c.dev_status, capw);            \
+                                  sel_count, max_sel, tau_hat, c.dev_status, capw,             \
+                                  policy == EKV_SEL_GAUSS_MAX);                                \
     }()
     switch (G) {
     case 1: return EKV_GSEL(1);

@@ -25,7 +25,7 @@ from .build import LIB_PATH
 EKV_OK, EKV_ERR_INVALID_ARG, EKV_ERR_UNSUPPORTED, EKV_ERR_WORKSPACE, EKV_ERR_CUDA, EKV_ERR_DEVICE = range(6)
 EKV_F32, EKV_BF16 = 0, 1
 EKV_SOFTMAX, EKV_ENTMAX15, EKV_SPARSEMAX = 0, 1, 2
-EKV_SEL_TOPK, EKV_SEL_GAUSS = 0, 1
+EKV_SEL_TOPK, EKV_SEL_GAUSS, EKV_SEL_GAUSS_MAX = 0, 1, 2
 EKV_DEV_BAD_BLOCK, EKV_DEV_BAD_LEN, EKV_DEV_BAD_SEL, EKV_DEV_SEL_OVERFLOW, EKV_DEV_BAD_RANGE = \
     0x1, 0x2, 0x4, 0x8, 0x10
 EKV_DEV_TIMEOUT = 0x20

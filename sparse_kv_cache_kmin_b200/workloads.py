@@ -34,7 +34,7 @@ import numpy as np
 import torch
 
 SOFTMAX, ENTMAX15, SPARSEMAX = 0, 1, 2  # attention modes (values of ekv_attn)
-TOPK, GAUSS = 0, 1                      # selection policies (values of ekv_policy)
+TOPK, GAUSS, GAUSS_MAX = 0, 1, 2        # selection policies (values of ekv_policy)
 
 
 @dataclass

@@ -21,7 +21,7 @@ import torch
 import oracle as O
 from sparse_kv_cache_kmin_b200 import ekv
 from sparse_kv_cache_kmin_b200.decoder import SparseDecoder
-from sparse_kv_cache_kmin_b200.workloads import GAUSS, TOPK
+from sparse_kv_cache_kmin_b200.workloads import GAUSS, GAUSS_MAX, TOPK
 
 U = 2.0 ** -24
 MODE = {ekv.EKV_SOFTMAX: O.SOFTMAX, ekv.EKV_ENTMAX15: O.ENTMAX15, ekv.EKV_SPARSEMAX: O.SPARSEMAX}
@@ -40,7 +40,7 @@ def widen(t: torch.Tensor) -> np.ndarray:
 
 
 def make_cache(wl, gaussian=None):
-    gaussian = wl.policy == GAUSS if gaussian is None else gaussian
+    gaussian = wl.policy in (GAUSS, GAUSS_MAX) if gaussian is None else gaussian
     nb, H, P, d = wl.k_cache.shape
     dev = wl.k_cache.device
     return ekv.PagedKVCache(
@@ -182,13 +182,21 @@ def check_head(wl, cache, dec, b, h, attn, hc=None, check_scores=True):
         tau_o = np.array([O.gauss_tau(m[g], v[g], cnt, wl.alpha) for g in range(G)])
         tau_g = dec.tau_hat[b, h * G:(h + 1) * G].double().cpu().numpy()
         assert np.all(np.abs(tau_g - tau_o) <= 1e-4 * np.maximum(1, np.abs(tau_o))), (tau_g, tau_o)
-        # the GPU's decision on its own UB and tau-hat is the oracle's rule, exactly
-        same = O.gauss_select(sc[:, 0], tau_g.astype(np.float32).astype(np.float64), wl.alpha, wl.delta)
+        # the GPU's decision on its own statistics and tau-hat is the oracle's rule, exactly
+        tau_gf = tau_g.astype(np.float32).astype(np.float64)
+        if wl.policy == GAUSS_MAX:
+            same = O.gauss_select_est(sc[:, 0], sc[:, 1], sc[:, 2], cnt, tau_gf, wl.alpha, wl.delta)
+            ref = O.gauss_select_est(ub, m, v, cnt, tau_o, wl.alpha, wl.delta)
+            stat_o = np.array([[O.est_max(ub[g, j], m[g, j], v[g, j], cnt[j]) for j in range(ub.shape[1])]
+                               for g in range(G)])
+        else:
+            same = O.gauss_select(sc[:, 0], tau_gf, wl.alpha, wl.delta)
+            ref = O.gauss_select(ub, tau_o, wl.alpha, wl.delta)
+            stat_o = ub
         np.testing.assert_array_equal(sel_gpu, same)
-        ref = O.gauss_select(ub, tau_o, wl.alpha, wl.delta)
         diff = np.setxor1d(sel_gpu, ref)
         if len(diff):
-            margin = ((wl.alpha - 1) * ub[:, diff] - (tau_o[:, None] - wl.delta)).max(0)
+            margin = ((wl.alpha - 1) * stat_o[:, diff] - (tau_o[:, None] - wl.delta)).max(0)
             assert np.all(np.abs(margin) <= 1e-4 * max(1.0, np.abs(tau_o).max())), margin
         info["sel_diff"] = len(diff)
         info["kept"] = n_sel

@@ -28,7 +28,10 @@ MUTANTS = {
                                   "return a > b ? -1 : (a < b);\n}\n\nstatic int cmp_int_asc"),
     "gauss_v_not_squared": ("b += qc * qc * var[(size_t)j * d + c];",
                             "b += qc * var[(size_t)j * d + c];"),
-    "gauss_select_not_strict": ("> tau_hat[g] - delta)", ">= tau_hat[g] - delta)"),
+    "gauss_select_not_strict": ("ub[(size_t)g * n_pages + j] > tau_hat[g] - delta)",
+                                "ub[(size_t)g * n_pages + j] >= tau_hat[g] - delta)"),
+    "est_max_uncapped": ("return e < ub ? e : ub;", "return e;"),
+    "est_max_wrong_quantile": ("sqrt(2.0 * log((double)n))", "sqrt(log((double)n))"),
     "softmax_stat_drops_max": ("stat[g] = mx + log(l);", "stat[g] = log(l);"),
     "attention_reads_invalid_tokens": (
         "n_tok += seq_len - j * P < P ? seq_len - j * P : P;", "n_tok += P;"),

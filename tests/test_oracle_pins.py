@@ -357,6 +357,55 @@ def test_gauss_select_rule():
     np.testing.assert_array_equal(O.gauss_select(ub, np.array([2.0, 1.0]), 2.0, 0.0), [2, 3])
 
 
+def test_est_max_bounds_the_expected_page_maximum():
+    # second reading of the "estimated maximum" (EntmaxKV §2.B): for n iid N(m, v) token scores
+    # the expected maximum lies below m + sqrt(2 ln n) sqrt(v) (the classical bound on the
+    # expected maximum of n standard normals) and not far below it; the bbox cap is exact
+    rng = np.random.default_rng(21)
+    for n, m, sd in [(16, 0.3, 1.0), (64, -1.0, 0.5), (2, 2.0, 2.0)]:
+        draws = m + sd * rng.standard_normal((40000, n))
+        mc = draws.max(axis=1).mean()
+        est = O.est_max(np.inf, m, sd * sd, n)
+        assert mc <= est + 0.01 * sd
+        assert est - mc <= 0.8 * sd
+    assert O.est_max(1.5, 1.0, 4.0, 16) == 1.5           # capped by the bound
+    assert O.est_max(9.0, 1.0, 0.0, 16) == 1.0           # zero variance: the common score
+
+
+def test_est_max_of_a_one_token_page_is_its_score():
+    rng = np.random.default_rng(22)
+    k = rng.standard_normal((3, 1, 4, 8)).astype(np.float32)
+    pt = np.array([2, 0], dtype=np.int32)
+    q = rng.standard_normal((1, 8))
+    kmin, kmax, mean, var = O.page_meta_head(k, pt, 5, 0)   # the second page holds one token
+    ub, _ = O.score_head(q, 1.0, kmin, kmax)
+    m, v = O.gauss_stats_head(q, 1.0, mean, var)
+    s_tok = float(q[0] @ k[0, 0, 0].astype(np.float64))
+    assert abs(O.est_max(ub[0, 1], m[0, 1], v[0, 1], 1) - s_tok) < 1e-12
+
+
+def test_gauss_select_est_rule_and_subset():
+    # hand-worked: alpha 2 (factor 1), delta 0.1, tau_hat 1.0 -> keep iff est > 0.9
+    ub = np.array([[2.0, 2.0, 0.5, 2.0]])
+    m = np.array([[0.5, 0.95, 0.4, 0.1]])
+    v = np.array([[0.0, 0.0, 1.0, 0.04]])
+    cnt = np.array([16, 16, 16, 1], dtype=np.int32)
+    # est: 0.5 | 0.95 | min(0.5, 0.4 + 2.355) = 0.5 | 0.1 (one token) -> only page 1
+    np.testing.assert_array_equal(O.gauss_select_est(ub, m, v, cnt, np.array([1.0]), 2.0, 0.1), [1])
+    # est <= UB, so the estimate keeps a subset of what the bound keeps
+    rng = np.random.default_rng(23)
+    G, n = 4, 300
+    ub = rng.normal(3, 1, (G, n))
+    m = ub - rng.uniform(0, 3, (G, n))
+    v = rng.uniform(0, 1, (G, n))
+    cnt = rng.integers(1, 33, n).astype(np.int32)
+    tau = rng.normal(2, 0.5, G)
+    for alpha in (1.5, 2.0):
+        a = set(O.gauss_select_est(ub, m, v, cnt, tau, alpha, 0.1).tolist())
+        b = set(O.gauss_select(ub, tau, alpha, 0.1).tolist())
+        assert a <= b and len(a) < len(b)
+
+
 # ----------------------------------------------------------------------------- §2.C / §3 attention
 def make_seq(rng, P=8, d=16, H_kv=2, L=61, nb=20, dist_scale=1.0):
     k = (rng.standard_normal((nb, H_kv, P, d)) * dist_scale).astype(np.float32)

@@ -10,7 +10,7 @@ import torch
 
 import oracle as O
 from sparse_kv_cache_kmin_b200 import ekv
-from sparse_kv_cache_kmin_b200.workloads import GAUSS, TOPK, make, make_random
+from sparse_kv_cache_kmin_b200.workloads import GAUSS, GAUSS_MAX, TOPK, make, make_random
 from parity_utils import HostCopy, check_head, close, make_cache, prefill_metadata, run_gpu, widen
 
 pytestmark = pytest.mark.gpu
@@ -58,6 +58,37 @@ def test_gauss_small_ragged(cuda_device, dtype, d, P, G, attn):
     for b in range(wl.batch):
         for h in range(wl.num_kv_heads):
             check_head(wl, cache, dec, b, h, attn)
+
+
+GAUSS_MAX_CASES = list(itertools.product([torch.float32, torch.bfloat16], [128], [16, 32], [1, 4],
+                                         [ekv.EKV_ENTMAX15, ekv.EKV_SPARSEMAX]))
+
+
+@pytest.mark.parametrize("dtype,d,P,G,attn", GAUSS_MAX_CASES,
+                         ids=["%s-d%d-P%d-G%d-a%d" % (str(t)[6:], d, P, G, a) for t, d, P, G, a in GAUSS_MAX_CASES])
+def test_gauss_estimated_max_small_ragged(cuda_device, dtype, d, P, G, attn):
+    # the second reading of the estimated page maximum: min(UB, m + sqrt(2 ln n) sqrt(v))
+    lens = (3000 + 5, 700, 64 * 3 + 1)
+    alpha = 1.5 if attn == ekv.EKV_ENTMAX15 else 2.0
+    wl = make_random(B=3, H_kv=2, G=G, d=d, P=P, lens=lens, dtype=dtype, device="cuda",
+                     seed=200 + d + P + G, kv_scale=1.0, q_scale=0.6, policy=GAUSS_MAX,
+                     alpha=alpha, delta=0.1)
+    cache, dec = run_gpu(wl, attn)
+    assert_status_ok(cache)
+    for b in range(wl.batch):
+        for h in range(wl.num_kv_heads):
+            check_head(wl, cache, dec, b, h, attn)
+
+
+def test_gauss_estimated_max_on_the_gauss_workload(cuda_device):
+    wl = make("gauss", device="cuda")
+    wl.policy = GAUSS_MAX
+    cache = make_cache(wl)
+    prefill_metadata(cache, wl)
+    _, dec = run_gpu(wl, ekv.EKV_ENTMAX15, cache=cache)
+    assert_status_ok(cache)
+    for b, h in [(0, 0), (9, 4), (15, 7)]:
+        check_head(wl, cache, dec, b, h, ekv.EKV_ENTMAX15)
 
 
 def test_multi_chunk_pages(cuda_device):
