@@ -958,6 +958,23 @@ __device__ void finish_entmax_cta(const DecodeArgs &a, int b, int h, int hq, int
             }
         }
     };
+    // Resolve the listed candidates' cache rows now (the chunk kernel recorded each selected
+    // page's block) and start their V rows towards L2: the support is among them, so its rows
+    // are on their way while tau is solved. A list refilled later holds slots again.
+    const char *vc = static_cast<const char *>(c.v_cache);
+    const int32_t *blk_row = a.sel_blk + ((size_t)b * H + h) * a.max_sel;
+    bool rows_listed = false;
+    if (!over) {
+        for (int i = lane; i < cnt; i += 32) {
+            const int slot = cs[warp][i], t = slot & (P - 1);
+            const int blk = __ldcg(blk_row + (slot >> a.Pshift));
+            cs[warp][i] = blk * P + t;
+            const char *vrow = vc + (((size_t)blk * H + h) * P + t) * D * ESZ;
+#pragma unroll
+            for (int off = 0; off < D * ESZ; off += 128) prefetch_l2(vrow + off);
+        }
+        rows_listed = true;
+    }
     HistRange R;
     R.set(-1.0, 0.0, 1.0 / kHistBins, true);
 
@@ -1012,6 +1029,7 @@ __device__ void finish_entmax_cta(const DecodeArgs &a, int b, int h, int hq, int
                 if (over) {
                     cnt = gather();
                     over = cnt > kCapW;
+                    rows_listed = false;  // the new list holds slots
                 }
             }
             hist_add_base(visit_own, hist, R, jhi);
@@ -1027,11 +1045,9 @@ __device__ void finish_entmax_cta(const DecodeArgs &a, int b, int h, int hq, int
     }
 
     // o = sum over the support of p_i v_i, each warp over its own entries: compact the support
-    // (weight, slot) in place over the gathered list, resolve every slot to its cache row (the
-    // chunk kernel recorded the block of every selected page) with all lookups in flight, then
-    // stream the V rows UNRV per lane group; a warp whose list overflowed does this in rounds of
-    // at most kCapW entries
-    const char *vc = static_cast<const char *>(c.v_cache);
+    // (weight, row) in place over the gathered list -- rows resolved above, or slots resolved
+    // here with all lookups in flight -- then stream the V rows UNRV per lane group; a warp whose
+    // list overflowed does this in rounds of at most kCapW entries
     const int cidx = lane % W, row = lane / W;
     float acc[EPC];
 #pragma unroll
@@ -1039,7 +1055,6 @@ __device__ void finish_entmax_cta(const DecodeArgs &a, int b, int h, int hq, int
     float *sp = cz[warp];  // compacted support weights
     int *sr = cs[warp];    // and slots, then rows as blk * P + t
     const int nitems = over ? (f1w - f0w) * 4 : cnt;
-    const int32_t *blk_row = a.sel_blk + ((size_t)b * H + h) * a.max_sel;
     int it0 = 0;
     do {
         int ns = 0;
@@ -1070,7 +1085,7 @@ __device__ void finish_entmax_cta(const DecodeArgs &a, int b, int h, int hq, int
             ns += __popc(bal);
             it0 += 32;
         }
-        for (int k0 = 0; k0 < ns; k0 += 128) {
+        for (int k0 = rows_listed ? ns : 0; k0 < ns; k0 += 128) {
             int sl[4], bv[4];
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
