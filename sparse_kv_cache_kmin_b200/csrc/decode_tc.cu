@@ -527,22 +527,34 @@ decode_softmax_tc_kernel(const __grid_constant__ CUtensorMap kmap,
                     for (int k = 0;; ++k) {
                         const int s = k % S, s1 = (k + 1) % S;
                         const uint32_t ph = (k / S) & 1, ph1 = ((k + 1) / S) & 1;
-                        // the next chunk's scores while this chunk's softmax runs
-                        if (!mbar_wait_bounded(&bar_full[s1], ph1)) { ok = false; break; }
-                        tc_fence_after_sync();
-                        const bool next_end = item_s[s1] < 0;
-                        if (next_end) {
-                            mbar_arrive(&bar_sdone[s1]);
-                        } else {
-                            mma_s(s1);
-                            tc_commit(&bar_sdone[s1]);
+                        // two independent issues: the next chunk's scores (once its tiles have
+                        // landed) and this chunk's O (once its P is written and the columns are
+                        // free), whichever is ready first -- neither waits on the other
+                        bool next_done = false, next_end = false, o_done = false;
+                        const uint64_t t0 = global_ns();
+                        while (!(next_done && o_done)) {
+                            if (!next_done && mbar_try_wait(&bar_full[s1], ph1)) {
+                                tc_fence_after_sync();
+                                next_end = item_s[s1] < 0;
+                                if (next_end) {
+                                    mbar_arrive(&bar_sdone[s1]);  // pass the end mark on
+                                } else {
+                                    mma_s(s1);
+                                    tc_commit(&bar_sdone[s1]);
+                                }
+                                next_done = true;
+                            }
+                            if (!o_done && mbar_try_wait(&bar_pready[s], ph) &&
+                                (k < S || mbar_try_wait(&bar_ofree[s], ph ^ 1))) {
+                                tc_fence_after_sync();
+                                mma_o(s);
+                                tc_commit(&bar_odone[s]);
+                                tc_commit(&bar_empty[s]);  // K, V and P of this stage are free
+                                o_done = true;
+                            }
+                            if (global_ns() - t0 > 2000000000ull) break;
                         }
-                        if (!mbar_wait_bounded(&bar_pready[s], ph)) { ok = false; break; }
-                        if (k >= S && !mbar_wait_bounded(&bar_ofree[s], ph ^ 1)) { ok = false; break; }
-                        tc_fence_after_sync();
-                        mma_o(s);
-                        tc_commit(&bar_odone[s]);
-                        tc_commit(&bar_empty[s]);  // K, V and P of this stage are free
+                        if (!(next_done && o_done)) { ok = false; break; }
                         if (next_end) break;
                     }
                 }

@@ -336,16 +336,16 @@ select_gauss_kernel(const float *__restrict__ scores, int H, int max_pages, int 
         };
         float amax = -INFINITY;
         if (staged) {
-            for (int j0 = p0; j0 < p1; j0 += 128) {
-                float av[4], bv[4];
+            for (int j0 = p0; j0 < p1; j0 += 256) {
+                float av[8], bv[8];
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
+                for (int u = 0; u < 8; ++u) {
                     const int j = j0 + u * 32 + lane;
                     av[u] = -INFINITY; bv[u] = 0.f;
                     if (j < p1) model(j, av[u], bv[u]);
                 }
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
+                for (int u = 0; u < 8; ++u) {
                     const int j = j0 + u * 32 + lane;
                     if (j < p1) {
                         sa[j - p0] = av[u]; sb[j - p0] = bv[u]; sn[j - p0] = page_n(j);
