@@ -29,6 +29,34 @@ constexpr int kSelThreads = 1024;
 constexpr int kSmemKeys = 16384;  // keys staged in shared memory (larger n reads them from L2)
 constexpr int kBoundaryMax = 256; // boundary-bin entries resolved by rank counting
 
+// The bin holding the k-th largest key: counts in descending bin order (thread t owns bins
+// nb-1-BPT*t ... nb-BPT-BPT*t), a block scan, and the one thread whose bins cross k writes the
+// bin and the count of keys in the bins above it. Ends with a barrier.
+template <int NT, int BPT>
+__device__ __forceinline__ void find_bin_from_top(const int *hist, int nb, int k, int *warp_tot,
+                                                  int *s_bin, int *s_above)
+{
+    const int tid = threadIdx.x;
+    int cnt[BPT], sum = 0;
+#pragma unroll
+    for (int r = 0; r < BPT; ++r) {
+        const int bin = nb - 1 - BPT * tid - r;
+        cnt[r] = bin >= 0 ? hist[bin] : 0;
+        sum += cnt[r];
+    }
+    const int incl = block_incl_scan<NT>(sum, warp_tot, nullptr);
+    int run = incl - sum;
+#pragma unroll
+    for (int r = 0; r < BPT; ++r) {
+        if (cnt[r] > 0 && run < k && k <= run + cnt[r]) {
+            *s_bin = nb - 1 - BPT * tid - r;
+            *s_above = run;
+        }
+        run += cnt[r];
+    }
+    __syncthreads();
+}
+
 // Exact radix select on the order-preserving keys (11 + 11 + 10 bits) and emission of the
 // kept pages in ascending order. `key(j)` returns the key of page j.
 template <class KeyFn>
@@ -56,13 +84,7 @@ __device__ void radix_select_emit(int n, int kk, KeyFn key, int *hist, int *warp
             if (bin >= 0 && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
         }
         __syncthreads();
-        const int b0 = nb - 1 - 2 * tid, b1 = nb - 2 - 2 * tid;
-        const int c0 = b0 >= 0 ? hist[b0] : 0, c1 = b1 >= 0 ? hist[b1] : 0;
-        const int incl = block_incl_scan<NT>(c0 + c1, warp_tot, nullptr);
-        const int excl = incl - c0 - c1;
-        if (c0 > 0 && excl < remaining && remaining <= excl + c0) { *s_bin = b0; *s_above = excl; }
-        if (c1 > 0 && excl + c0 < remaining && remaining <= incl) { *s_bin = b1; *s_above = excl + c0; }
-        __syncthreads();
+        find_bin_from_top<NT, 2048 / NT>(hist, nb, remaining, warp_tot, s_bin, s_above);
         remaining -= *s_above;
         prefix |= (uint32_t)*s_bin << shift;
         mask |= (uint32_t)(nb - 1) << shift;
@@ -75,7 +97,7 @@ __device__ void radix_select_emit(int n, int kk, KeyFn key, int *hist, int *warp
     // emission in page order: warp w owns a contiguous page range; ties at T are kept while
     // their rank among all ties (in page order) is below `remaining`
     const int warp = tid >> 5;
-    const int per = (n + 31) / 32;
+    const int per = (n + NT / 32 - 1) / (NT / 32);
     const int j0 = warp * per, j1 = j0 + per < n ? j0 + per : n;
     int n_above = 0, n_tie = 0;
     for (int j = j0 + lane; j - lane < j1; j += 32) {
@@ -201,13 +223,7 @@ select_topk_kernel(const float *__restrict__ scores, int H, int max_pages, int P
     for (int j = tid; j < n; j += NT) atomicAdd(&hist[bin_of(keys[j])], 1);
     __syncthreads();
     // counts in descending bin order: thread t owns bins NB-1-2t and NB-2-2t
-    const int b0 = NB - 1 - 2 * tid, b1 = NB - 2 - 2 * tid;
-    const int c0 = b0 >= 0 ? hist[b0] : 0, c1 = b1 >= 0 ? hist[b1] : 0;
-    const int incl = block_incl_scan<NT>(c0 + c1, warp_tot, nullptr);
-    const int excl = incl - c0 - c1;
-    if (c0 > 0 && excl < kk && kk <= excl + c0) { s_bin = b0; s_above = excl; }
-    if (c1 > 0 && excl + c0 < kk && kk <= incl) { s_bin = b1; s_above = excl + c0; }
-    __syncthreads();
+    find_bin_from_top<NT, NB / NT>(hist, NB, kk, warp_tot, &s_bin, &s_above);
     const int B = s_bin, r = kk - s_above, cB = hist[B];
 
     if (cB > kBoundaryMax) {  // heavy ties around the k-th key
@@ -230,7 +246,7 @@ select_topk_kernel(const float *__restrict__ scores, int H, int max_pages, int P
         }
         __syncthreads();
         // emission in page order: warp w owns a contiguous page range
-        const int per = (n + 31) / 32;
+        const int per = (n + NT / 32 - 1) / (NT / 32);
         const int j0 = warp * per, j1 = j0 + per < n ? j0 + per : n;
         auto kept = [&](int j) {
             const int bb = bin_of(keys[j]);
@@ -545,7 +561,7 @@ cudaError_t launch_select_pages(const ekv_cache &c, int H_q, int policy, int top
     cudaLaunchAttribute attr[1];
     const dim3 grid(c.num_kv_heads, c.batch);
     if (policy == EKV_SEL_TOPK) {
-        cudaLaunchConfig_t cfg = pdl_config(grid, dim3(1024), st, pdl, attr);
+        cudaLaunchConfig_t cfg = pdl_config(grid, dim3(kSelThreads), st, pdl, attr);
         const int keys = c.max_pages < kSmemKeys ? c.max_pages : kSmemKeys;
         cfg.dynamicSmemBytes = sizeof(uint32_t) * keys;
         static bool attr_set = false;
