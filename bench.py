@@ -463,22 +463,26 @@ def main():
     h2d = q_host.numel() * q_host.element_size()
     app_host = None
     if wl.append is not None:
-        last = wl.page_table[0].long()[(wl.append[0]) // P]
+        last = int(wl.page_table[0, wl.append[0] // P])  # a host index: no sync in the graph
         app_host = (wl.k_cache[last].cpu().pin_memory(), wl.v_cache[last].cpu().pin_memory(), last)
         h2d += 2 * app_host[0].numel() * app_host[0].element_size()
     e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(args.steps)]
+
+    def host_pre():
+        # the appended page's K and V rows arrive from the host, then its metadata is refreshed
+        if app_host is not None:
+            wl.k_cache[app_host[2]].copy_(app_host[0], non_blocking=True)
+            wl.v_cache[app_host[2]].copy_(app_host[1], non_blocking=True)
+        if pre is not None:
+            pre()
+    # one graph per host-to-host step: query in, step, outputs out
+    graph_e2e = dec.capture_host(wl.q, q_host, out_host, stat_host, pre_step=host_pre)
     for i in range(args.steps + 3):
         flush.fill_(1)
         if i >= 3:
             e2e_ev[i - 3][0].record(stream)
-        if app_host is not None:
-            wl.k_cache[app_host[2]].copy_(app_host[0], non_blocking=True)
-            wl.v_cache[app_host[2]].copy_(app_host[1], non_blocking=True)
-        wl.q.copy_(q_host, non_blocking=True)  # the graph reads q from this buffer
-        graph.replay()
-        out_host.copy_(dec.out, non_blocking=True)
-        stat_host.copy_(dec.stat, non_blocking=True)
+        graph_e2e.replay()
         if i >= 3:
             e2e_ev[i - 3][1].record(stream)
         stream.synchronize()

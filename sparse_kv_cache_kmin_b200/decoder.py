@@ -55,6 +55,21 @@ class SparseDecoder:
             self.step(q_static)
         return g
 
+    def capture_host(self, q_dev: torch.Tensor, q_host: torch.Tensor, out_host: torch.Tensor,
+                     stat_host: torch.Tensor, pre_step=None) -> torch.cuda.CUDAGraph:
+        """Capture a whole host-to-host step in one CUDA graph: the query copied from pinned
+        host memory into `q_dev`, the decode step, and the outputs copied back into pinned host
+        buffers. Replay, then synchronise the stream, to run one step."""
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            if pre_step is not None:
+                pre_step()
+            q_dev.copy_(q_host, non_blocking=True)
+            self.step(q_dev)
+            out_host.copy_(self.out, non_blocking=True)
+            stat_host.copy_(self.stat, non_blocking=True)
+        return g
+
     def step(self, q: torch.Tensor, stream=None):
         c = self.cache
         ekv.ekv_score_pages(c, q, self.num_q_heads, self.scale, self.policy, self.scores, stream)
