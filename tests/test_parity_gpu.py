@@ -181,6 +181,24 @@ def test_named_workload_sampled_heads(cuda_device, name, heads):
             check_head(wl, cache, dec, b, h, attn, hc=hc)
 
 
+def test_host_to_host_graph_matches_the_eager_step(cuda_device):
+    # the end-to-end path: one graph copies the query in, runs the step, copies outputs out
+    wl = make_random(B=2, H_kv=2, G=4, d=128, P=16, lens=(3000, 1111), dtype=torch.bfloat16,
+                     device="cuda", seed=31, topk=40)
+    cache, dec = run_gpu(wl, ekv.EKV_ENTMAX15)
+    out_ref, stat_ref = dec.out.clone(), dec.stat.clone()
+    q_dev = torch.empty_like(wl.q)
+    q_host = wl.q.cpu().pin_memory()
+    out_host = torch.empty(dec.out.shape, dtype=dec.out.dtype).pin_memory()
+    stat_host = torch.empty(dec.stat.shape, dtype=dec.stat.dtype).pin_memory()
+    g = dec.capture_host(q_dev, q_host, out_host, stat_host)
+    for _ in range(2):
+        g.replay()
+        torch.cuda.synchronize()
+    assert_status_ok(cache)
+    assert torch.equal(out_host, out_ref.cpu()) and torch.equal(stat_host, stat_ref.cpu())
+
+
 # ------------------------------------------------------------------ edge cases
 def test_edge_lengths_and_budgets(cuda_device):
     # empty sequence, one token, exactly one page, k >= n_pages
