@@ -1234,6 +1234,8 @@ static cudaError_t launch_chunk(const DecodeArgs &a, cudaLaunchConfig_t cfg)
 bool tc_chunk_supported(const ekv_cache &c, int H_q, bool softmax);
 cudaError_t launch_chunk_tc(const DecodeArgs &a, int G, cudaLaunchConfig_t cfg);
 cudaError_t launch_softmax_tc(const DecodeArgs &a, int G, cudaLaunchConfig_t cfg);
+bool direct_logits_supported(const ekv_cache &c, int H_q);
+cudaError_t launch_logits_direct(const DecodeArgs &a, int G, cudaLaunchConfig_t cfg, bool *launched);
 
 template <int DT, int D, int G>
 static cudaError_t launch_decode_t(const DecodeArgs &a, bool softmax, cudaStream_t st, bool pdl)
@@ -1245,11 +1247,14 @@ static cudaError_t launch_decode_t(const DecodeArgs &a, bool softmax, cudaStream
     cfg.stream = st;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    cudaError_t e;
+    cudaError_t e = cudaSuccess;
     const bool tc = DT == EKV_BF16 && tc_chunk_supported(a.c, a.H_q, softmax);
+    bool direct = false;
+    if (!softmax && tc && direct_logits_supported(a.c, a.H_q)) e = launch_logits_direct(a, G, cfg, &direct);
+    if (e != cudaSuccess) return e;
     if (softmax)
         e = tc ? launch_softmax_tc(a, G, cfg) : launch_chunk<DT, D, G, true>(a, cfg);
-    else
+    else if (!direct)
         e = tc ? launch_chunk_tc(a, G, cfg) : launch_chunk<DT, D, G, false>(a, cfg);
     if (e != cudaSuccess) return e;
     cfg.blockDim = dim3(256);
