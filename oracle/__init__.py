@@ -64,6 +64,9 @@ def _load():
     lib.ora_attend_head.argtypes = [vp, vp, c_int, c_int, c_int, c_int, c_int, _ip, c_int, c_int,
                                     _dp, c_int, c_double, c_int, _ip, c_int, _dp, _dp, _dp]
     lib.ora_attend_head.restype = c_int
+    lib.ora_moment_corrected_head.argtypes = [vp, vp, c_int, c_int, c_int, c_int, c_int, _ip, c_int,
+                                              c_int, _dp, c_int, c_double, _ip, c_int, _dp, _dp]
+    lib.ora_moment_corrected_head.restype = c_int
     _lib = lib
     return lib
 
@@ -230,6 +233,32 @@ def attend_head(k_cache, v_cache, pt_row, seq_len: int, h: int, q, scale: float,
         raise ValueError("selected page or page-table entry out of range")
     weights = w[:G * rc].reshape(G, rc) if w is not None else None
     return out, stat, weights
+
+
+def moment_corrected_head(k_cache, v_cache, pt_row, seq_len: int, h: int, q, scale: float, sel):
+    """Softmax over the selected pages, corrected for the skipped ones from their moments
+    (MomentKV technical summary, Methodology §1, §2, §4; see ``ora_moment_corrected_head``).
+
+    Returns (out [G, d], stat [G] = log of the estimated partition sum, n_e evicted tokens)."""
+    nb, H_kv, P, d = k_cache.shape
+    k_cache = np.ascontiguousarray(k_cache)
+    v_cache = np.ascontiguousarray(v_cache)
+    dt = _cache_dtype(k_cache)
+    if _cache_dtype(v_cache) != dt:
+        raise TypeError("K and V caches must share a dtype")
+    q, qp = _d(np.atleast_2d(q))
+    G = q.shape[0]
+    pt, ptp = _i(pt_row)
+    sel, sp = _i(np.asarray(sel, dtype=np.int32).reshape(-1))
+    out = np.zeros((G, d))
+    stat = np.zeros(G)
+    rc = _load().ora_moment_corrected_head(k_cache.ctypes.data, v_cache.ctypes.data, dt, nb, H_kv,
+                                           P, d, ptp, int(seq_len), int(h), qp, G, float(scale),
+                                           sp, len(sel), out.ctypes.data_as(_dp),
+                                           stat.ctypes.data_as(_dp))
+    if rc < 0:
+        raise ValueError("selected page or page-table entry out of range")
+    return out, stat, rc
 
 
 def page_counts(seq_len: int, P: int) -> np.ndarray:

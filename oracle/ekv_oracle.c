@@ -18,6 +18,9 @@
  *          safety margin Delta;
  *   §2.C   exact alpha-entmax attention over the selected pages only (softmax for the
  *          comparison the summary draws in §1 and §3).
+ * And, for softmax over a page selection, the moment correction for the skipped tokens of the
+ * MomentKV technical summary (gist.science), Methodology §1, §2, §4 (ora_moment_corrected_head,
+ * with its readings at the function).
  * Readings of points the summary leaves open (all stated again in the design notes):
  *   - logits are s = scale * q.k, with scale an argument;
  *   - alpha-entmax: p_i = [(alpha-1) z_i - tau]_+^(1/(alpha-1)) with sum p = 1, written here
@@ -454,4 +457,108 @@ int ora_attend_head(const void *k_cache, const void *v_cache, int dtype, int num
     free(s);
     free(p);
     return n_tok;
+}
+
+/*
+ * Moment-corrected sparse softmax ("MomentKV", technical summary on gist.science,
+ * Methodology §1, §2 and §4), read for a paged cache that keeps every token but skips the
+ * pages a decode step did not select:
+ *   - the evicted set E of the step is every valid token of the sequence outside the selected
+ *     pages; its statistics are taken from E's rows directly: n_e, the key mean kbar, the value
+ *     mean vbar and the centred value-key cross moment St = sum_E (v - vbar)(k - kbar)^T;
+ *   - first-order estimate of the softmax output over E (logits s = scale q.k expanded around
+ *     scale q.kbar, §2): fE = vbar + (scale / n_e) St q -- the summary's 1/(n_e sqrt(d)) is this
+ *     factor at scale = 1/sqrt(d);
+ *   - Jensen lower bound on E's partition sum (§4): ZE = n_e exp(scale q.kbar);
+ *   - with fR, ZR the plain softmax output and partition sum over the selected pages:
+ *     out = wR fR + (1 - wR) fE, wR = ZR / (ZR + ZE), stat = log(ZR + ZE).
+ * Returns n_e, or -1 when a selected page or page-table entry is out of range.
+ */
+int ora_moment_corrected_head(const void *k_cache, const void *v_cache, int dtype, int num_blocks,
+                              int H_kv, int P, int d, const int32_t *pt_row, int seq_len, int h,
+                              const double *q, int G, double scale, const int32_t *sel, int n_sel,
+                              double *out, double *stat)
+{
+    if (ora_attend_head(k_cache, v_cache, dtype, num_blocks, H_kv, P, d, pt_row, seq_len, h, q, G,
+                        scale, ORA_SOFTMAX, sel, n_sel, out, stat, NULL) < 0)
+        return -1;
+    const int n_pages = pages_of(seq_len, P);
+    char *kept = (char *)calloc((size_t)(n_pages > 0 ? n_pages : 1), 1);
+    for (int i = 0; i < n_sel; ++i)
+        kept[sel[i]] = 1;
+    int n_e = 0;
+    for (int j = 0; j < n_pages; ++j) {
+        if (kept[j]) continue;
+        if (pt_row[j] < 0 || pt_row[j] >= num_blocks) {
+            free(kept);
+            return -1;
+        }
+        n_e += seq_len - j * P < P ? seq_len - j * P : P;
+    }
+    if (n_e == 0) {
+        free(kept);
+        return 0;
+    }
+    double *kbar = (double *)calloc((size_t)d, sizeof(double));
+    double *vbar = (double *)calloc((size_t)d, sizeof(double));
+    double *St = (double *)calloc((size_t)d * d, sizeof(double));
+    double *dv = (double *)malloc(sizeof(double) * (size_t)d);
+    double *dk = (double *)malloc(sizeof(double) * (size_t)d);
+    double *fE = (double *)malloc(sizeof(double) * (size_t)d);
+    for (int j = 0; j < n_pages; ++j) {
+        if (kept[j]) continue;
+        const int n = seq_len - j * P < P ? seq_len - j * P : P;
+        for (int t = 0; t < n; ++t)
+            for (int c = 0; c < d; ++c) {
+                kbar[c] += elem(k_cache, dtype, cache_off(pt_row[j], h, t, c, H_kv, P, d));
+                vbar[c] += elem(v_cache, dtype, cache_off(pt_row[j], h, t, c, H_kv, P, d));
+            }
+    }
+    for (int c = 0; c < d; ++c) {
+        kbar[c] /= n_e;
+        vbar[c] /= n_e;
+    }
+    for (int j = 0; j < n_pages; ++j) {
+        if (kept[j]) continue;
+        const int n = seq_len - j * P < P ? seq_len - j * P : P;
+        for (int t = 0; t < n; ++t) {
+            for (int c = 0; c < d; ++c) {
+                dk[c] = elem(k_cache, dtype, cache_off(pt_row[j], h, t, c, H_kv, P, d)) - kbar[c];
+                dv[c] = elem(v_cache, dtype, cache_off(pt_row[j], h, t, c, H_kv, P, d)) - vbar[c];
+            }
+            for (int a = 0; a < d; ++a)
+                for (int c = 0; c < d; ++c)
+                    St[(size_t)a * d + c] += dv[a] * dk[c];
+        }
+    }
+    for (int g = 0; g < G; ++g) {
+        const double *qg = q + (size_t)g * d;
+        double *og = out + (size_t)g * d;
+        double sbar = 0.0;
+        for (int c = 0; c < d; ++c)
+            sbar += qg[c] * kbar[c];
+        sbar *= scale;
+        for (int a = 0; a < d; ++a) {
+            double acc = 0.0;
+            for (int c = 0; c < d; ++c)
+                acc += St[(size_t)a * d + c] * qg[c];
+            fE[a] = vbar[a] + scale / n_e * acc;
+        }
+        const double logZR = stat[g];  /* -inf when no token is selected */
+        const double logZE = log((double)n_e) + sbar;
+        const double mx = logZR > logZE ? logZR : logZE;
+        const double zr = exp(logZR - mx), ze = exp(logZE - mx);
+        const double wR = zr / (zr + ze);
+        for (int a = 0; a < d; ++a)
+            og[a] = wR * og[a] + (1.0 - wR) * fE[a];
+        stat[g] = mx + log(zr + ze);
+    }
+    free(kept);
+    free(kbar);
+    free(vbar);
+    free(St);
+    free(dv);
+    free(dk);
+    free(fE);
+    return n_e;
 }

@@ -33,6 +33,18 @@ MUTANTS = {
     "est_max_uncapped": ("return e < ub ? e : ub;", "return e;"),
     "est_max_wrong_quantile": ("sqrt(2.0 * log((double)n))", "sqrt(log((double)n))"),
     "softmax_stat_drops_max": ("stat[g] = mx + log(l);", "stat[g] = log(l);"),
+    "moment_drops_cross_moment_term": ("fE[a] = vbar[a] + scale / n_e * acc;", "fE[a] = vbar[a];"),
+    "moment_cross_moment_uncentred": (
+        "cache_off(pt_row[j], h, t, c, H_kv, P, d)) - kbar[c];\n"
+        "                dv[c] = elem(v_cache, dtype, cache_off(pt_row[j], h, t, c, H_kv, P, d)) - vbar[c];",
+        "cache_off(pt_row[j], h, t, c, H_kv, P, d));\n"
+        "                dv[c] = elem(v_cache, dtype, cache_off(pt_row[j], h, t, c, H_kv, P, d));"),
+    "moment_cross_moment_without_scale": ("fE[a] = vbar[a] + scale / n_e * acc;",
+                                          "fE[a] = vbar[a] + acc / n_e;"),
+    "moment_jensen_drops_count": ("const double logZE = log((double)n_e) + sbar;",
+                                  "const double logZE = sbar;"),
+    "moment_mix_weights_swapped": ("og[a] = wR * og[a] + (1.0 - wR) * fE[a];",
+                                   "og[a] = (1.0 - wR) * og[a] + wR * fE[a];"),
     "attention_reads_invalid_tokens": (
         "n_tok += seq_len - j * P < P ? seq_len - j * P : P;", "n_tok += P;"),
 }

@@ -551,3 +551,82 @@ def test_partial_last_page_only_reads_valid_tokens():
     m2 = O.page_meta_head(k2, pt, 61, 0)
     for x, y in zip(m1, m2):
         np.testing.assert_array_equal(x, y)
+
+
+# ----------------------------------------------------------------------------- MomentKV correction
+# MomentKV technical summary (gist.science), Methodology §1 (compact moments of the evicted
+# set), §2 (first-order estimate of the evicted output), §4 (Jensen-weighted mix).
+def test_moment_correction_golden_fixture():
+    g = parse_golden("moment_correction_example.txt")
+    k = np.zeros((2, 1, 2, 2), dtype=np.float32)
+    v = np.zeros((2, 1, 2, 2), dtype=np.float32)
+    k[0, 0], v[0, 0] = g["keys_page0"], g["vals_page0"]
+    k[1, 0], v[1, 0] = g["keys_page1"], g["vals_page1"]
+    out, stat, n_e = O.moment_corrected_head(k, v, np.array([0, 1], np.int32), 4, 0,
+                                             g["q"][None, :], float(g["scale"][0]), [0])
+    assert n_e == int(g["n_e"][0])
+    e = math.e
+    zr, ze = math.exp(0.5) + e, int(g["n_e"][0]) * math.exp(float(g["sbar"][0]))
+    ref = (math.exp(0.5) * np.array([1.0, 1.0]) + e * np.array([-1.0, 3.0]) + ze * g["fE"]) / (zr + ze)
+    np.testing.assert_allclose(out[0], ref, rtol=0, atol=1e-14)
+    np.testing.assert_allclose(out[0], [(math.exp(0.5) + 2 * e) / (math.exp(0.5) + 3 * e),
+                                        (math.exp(0.5) + 5 * e) / (math.exp(0.5) + 3 * e)],
+                               rtol=0, atol=1e-14)
+    assert abs(stat[0] - math.log(zr + ze)) < 1e-14
+
+
+@pytest.mark.parametrize("sel", [[1, 4], [], [0, 2, 5, 7]])
+def test_moment_correction_exact_when_skipped_keys_coincide(sel):
+    # All skipped tokens share one key: their softmax is uniform (output = their mean value) and
+    # Jensen's bound on their partition sum is an equality, so the corrected output is the
+    # full-cache softmax.
+    rng = np.random.default_rng(31)
+    L, P, d, h, scale = 61, 8, 16, 1, 0.4
+    k, v, pt = make_seq(rng, P=P, d=d, L=L)
+    common = rng.standard_normal(d).astype(np.float32)
+    for j in range(O.pages_of(L, P)):
+        if j not in sel:
+            k[pt[j], h] = common
+    q = rng.standard_normal((3, d))
+    out, stat, n_e = O.moment_corrected_head(k, v, pt, L, h, q, scale, sel)
+    full, fstat, _ = O.attend_head(k, v, pt, L, h, q, scale, O.SOFTMAX, np.arange(O.pages_of(L, P)))
+    assert n_e == L - sum(min(P, L - j * P) for j in sel)
+    np.testing.assert_allclose(out, full, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(stat, fstat, rtol=0, atol=1e-12)
+
+
+def test_moment_correction_error_is_second_order_in_the_logit_scale():
+    # For logits scale * q.k with small scale, expanding the skipped tokens' softmax to first
+    # order leaves an O(scale^2) error in the output and in the partition sum, while dropping
+    # the skipped tokens (plain renormalisation) leaves an O(1) error.
+    rng = np.random.default_rng(32)
+    L, P, d, h = 61, 8, 16, 0
+    k, v, pt = make_seq(rng, P=P, d=d, L=L)
+    q = rng.standard_normal((2, d))
+    sel = [1, 3, 6]
+    allp = np.arange(O.pages_of(L, P))
+    errs, stat_errs, plain = [], [], []
+    for scale in (0.04, 0.02, 0.01):
+        out, stat, _ = O.moment_corrected_head(k, v, pt, L, h, q, scale, sel)
+        full, fstat, _ = O.attend_head(k, v, pt, L, h, q, scale, O.SOFTMAX, allp)
+        sparse, _, _ = O.attend_head(k, v, pt, L, h, q, scale, O.SOFTMAX, sel)
+        errs.append(np.abs(out - full).max())
+        stat_errs.append(np.abs(stat - fstat).max())
+        plain.append(np.abs(sparse - full).max())
+    for e in (errs, stat_errs):
+        for a, b in zip(e, e[1:]):
+            assert 3.4 < a / b < 4.6, e
+    assert errs[-1] < 1e-2 * plain[-1]
+
+
+def test_moment_correction_without_skipped_tokens_is_the_plain_softmax():
+    rng = np.random.default_rng(33)
+    L, P = 61, 8
+    k, v, pt = make_seq(rng, P=P, L=L)
+    q = rng.standard_normal((2, 16))
+    allp = np.arange(O.pages_of(L, P))
+    out, stat, n_e = O.moment_corrected_head(k, v, pt, L, 0, q, 0.7, allp)
+    ref, rstat, _ = O.attend_head(k, v, pt, L, 0, q, 0.7, O.SOFTMAX, allp)
+    assert n_e == 0
+    np.testing.assert_array_equal(out, ref)
+    np.testing.assert_array_equal(stat, rstat)
