@@ -67,6 +67,13 @@ def _load():
     lib.ora_moment_corrected_head.argtypes = [vp, vp, c_int, c_int, c_int, c_int, c_int, _ip, c_int,
                                               c_int, _dp, c_int, c_double, _ip, c_int, _dp, _dp]
     lib.ora_moment_corrected_head.restype = c_int
+    lib.ora_token_topk_head.argtypes = [vp, c_int, c_int, c_int, c_int, c_int, _ip, c_int, c_int,
+                                        _dp, c_int, c_double, _ip, c_int, c_int, _ip, _ip]
+    lib.ora_token_topk_head.restype = c_int
+    lib.ora_attend_tokens_head.argtypes = [vp, vp, c_int, c_int, c_int, c_int, c_int, _ip, c_int,
+                                           c_int, _dp, c_int, c_double, c_int, _ip, _ip, c_int,
+                                           _dp, _dp]
+    lib.ora_attend_tokens_head.restype = c_int
     _lib = lib
     return lib
 
@@ -259,6 +266,57 @@ def moment_corrected_head(k_cache, v_cache, pt_row, seq_len: int, h: int, q, sca
     if rc < 0:
         raise ValueError("selected page or page-table entry out of range")
     return out, stat, rc
+
+
+def token_topk_head(k_cache, pt_row, seq_len: int, h: int, q, scale: float, sel, T: int):
+    """Token-level selection inside the selected pages for one KV head (JSSA abstract; see
+    ``ora_token_topk_head``): the T candidate tokens with the largest group score
+    sum_g scale * q_g . k, ties to the earlier candidate, in candidate order.
+
+    Returns (pages [n] int32, positions [n] int32)."""
+    nb, H_kv, P, d = k_cache.shape
+    k_cache = np.ascontiguousarray(k_cache)
+    q, qp = _d(np.atleast_2d(q))
+    pt, ptp = _i(pt_row)
+    sel, sp = _i(np.asarray(sel, dtype=np.int32).reshape(-1))
+    cap = max(1, len(sel) * P)
+    pages = np.zeros(cap, dtype=np.int32)
+    pos = np.zeros(cap, dtype=np.int32)
+    rc = _load().ora_token_topk_head(k_cache.ctypes.data, _cache_dtype(k_cache), nb, H_kv, P, d,
+                                     ptp, int(seq_len), int(h), qp, q.shape[0], float(scale), sp,
+                                     len(sel), int(T), pages.ctypes.data_as(_ip),
+                                     pos.ctypes.data_as(_ip))
+    if rc < 0:
+        raise ValueError("selected page or page-table entry out of range")
+    return pages[:rc].copy(), pos[:rc].copy()
+
+
+def attend_tokens_head(k_cache, v_cache, pt_row, seq_len: int, h: int, q, scale: float,
+                       mode: int, tok_pages, tok_pos):
+    """Attention of the G queries over an explicit (logical page, position) token list, read
+    through the page table. Returns (out [G, d], stat [G])."""
+    nb, H_kv, P, d = k_cache.shape
+    k_cache = np.ascontiguousarray(k_cache)
+    v_cache = np.ascontiguousarray(v_cache)
+    dt = _cache_dtype(k_cache)
+    if _cache_dtype(v_cache) != dt:
+        raise TypeError("K and V caches must share a dtype")
+    q, qp = _d(np.atleast_2d(q))
+    G = q.shape[0]
+    pt, ptp = _i(pt_row)
+    tp, tpp = _i(np.asarray(tok_pages, dtype=np.int32).reshape(-1))
+    tt, ttp = _i(np.asarray(tok_pos, dtype=np.int32).reshape(-1))
+    if len(tp) != len(tt):
+        raise ValueError("token pages and positions differ in length")
+    out = np.zeros((G, d))
+    stat = np.zeros(G)
+    rc = _load().ora_attend_tokens_head(k_cache.ctypes.data, v_cache.ctypes.data, dt, nb, H_kv, P,
+                                        d, ptp, int(seq_len), int(h), qp, G, float(scale),
+                                        int(mode), tpp, ttp, len(tp), out.ctypes.data_as(_dp),
+                                        stat.ctypes.data_as(_dp))
+    if rc < 0:
+        raise ValueError("token page, position or page-table entry out of range")
+    return out, stat
 
 
 def page_counts(seq_len: int, P: int) -> np.ndarray:

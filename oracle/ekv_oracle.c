@@ -19,8 +19,10 @@
  *   §2.C   exact alpha-entmax attention over the selected pages only (softmax for the
  *          comparison the summary draws in §1 and §3).
  * And, for softmax over a page selection, the moment correction for the skipped tokens of the
- * MomentKV technical summary (gist.science), Methodology §1, §2, §4 (ora_moment_corrected_head,
- * with its readings at the function).
+ * MomentKV technical summary (gist.science), Methodology §1, §2, §4 (ora_moment_corrected_head);
+ * token-level selection inside the selected pages with indexed attention, after the JSSA
+ * abstract (ai.info) (ora_token_topk_head, ora_attend_tokens_head). Their readings are stated
+ * at the functions.
  * Readings of points the summary leaves open (all stated again in the design notes):
  *   - logits are s = scale * q.k, with scale an argument;
  *   - alpha-entmax: p_i = [(alpha-1) z_i - tau]_+^(1/(alpha-1)) with sum p = 1, written here
@@ -370,44 +372,20 @@ double ora_entmax_tau(const double *z, int n, double alpha)
 }
 
 /* ---------------------------------------------------------------------------------------
- * §2.C attention for the G query heads of one KV head over the selected pages of one
- * sequence. Tokens are visited page by page in the order of `sel` (ascending logical page
- * index), then by position in the page; only t < seq_len exist.
+ * §2.C attention for the G query heads of one KV head over a list of token rows (cache block,
+ * position), visited in list order.
  *   s_i = scale * q_g . k_i
  *   softmax:  p_i = exp(s_i - max s) / sum,       stat = log sum_i exp(s_i)
  *   entmax:   z_i = (alpha-1) s_i, tau exact,     p_i = [z_i - tau]_+^(1/(alpha-1)), stat = tau
  *   o_g = sum_i p_i v_i
- * q: [G][d]; out: [G][d]; stat: [G]; weights (optional): [G][n_tok] in visiting order.
- * An empty selection gives o = 0 and stat = -inf. Returns the token count, or -1 on a bad
- * page index or page-table entry.
+ * q: [G][d]; out: [G][d]; stat: [G]; weights (optional): [G][n_tok] in list order.
  * ------------------------------------------------------------------------------------- */
-int ora_attend_head(const void *k_cache, const void *v_cache, int dtype, int num_blocks,
-                    int H_kv, int P, int d, const int32_t *pt_row, int seq_len, int h,
-                    const double *q, int G, double scale, int mode,
-                    const int32_t *sel, int n_sel, double *out, double *stat, double *weights)
+static void attend_rows(const void *k_cache, const void *v_cache, int dtype, int H_kv, int P,
+                        int d, const int *blk, const int *pos, int n_tok, int h, const double *q,
+                        int G, double scale, int mode, double *out, double *stat, double *weights)
 {
-    int n_pages = pages_of(seq_len, P);
-    int n_tok = 0;
-    for (int i = 0; i < n_sel; ++i) {
-        int j = sel[i];
-        if (j < 0 || j >= n_pages || pt_row[j] < 0 || pt_row[j] >= num_blocks)
-            return -1;
-        n_tok += seq_len - j * P < P ? seq_len - j * P : P;
-    }
-    int *blk = (int *)malloc(sizeof(int) * (size_t)(n_tok > 0 ? n_tok : 1));
-    int *pos = (int *)malloc(sizeof(int) * (size_t)(n_tok > 0 ? n_tok : 1));
     double *s = (double *)malloc(sizeof(double) * (size_t)(n_tok > 0 ? n_tok : 1));
     double *p = (double *)malloc(sizeof(double) * (size_t)(n_tok > 0 ? n_tok : 1));
-    int t_all = 0;
-    for (int i = 0; i < n_sel; ++i) {
-        int j = sel[i];
-        int n = seq_len - j * P < P ? seq_len - j * P : P;
-        for (int t = 0; t < n; ++t) {
-            blk[t_all] = pt_row[j];
-            pos[t_all] = t;
-            ++t_all;
-        }
-    }
     double alpha = mode == ORA_ENTMAX15 ? 1.5 : 2.0;
     for (int g = 0; g < G; ++g) {
         const double *qg = q + (size_t)g * d;
@@ -452,10 +430,136 @@ int ora_attend_head(const void *k_cache, const void *v_cache, int dtype, int num
                 og[c] += p[i] * elem(v_cache, dtype, cache_off(blk[i], h, pos[i], c, H_kv, P, d));
         }
     }
-    free(blk);
-    free(pos);
     free(s);
     free(p);
+}
+
+/* Attention over the selected pages of one sequence: tokens page by page in the order of `sel`
+ * (ascending logical page index), then by position; only t < seq_len exist. Returns the token
+ * count, or -1 when a selected page or its page-table entry is out of range. */
+int ora_attend_head(const void *k_cache, const void *v_cache, int dtype, int num_blocks,
+                    int H_kv, int P, int d, const int32_t *pt_row, int seq_len, int h,
+                    const double *q, int G, double scale, int mode,
+                    const int32_t *sel, int n_sel, double *out, double *stat, double *weights)
+{
+    int n_pages = pages_of(seq_len, P);
+    int n_tok = 0;
+    for (int i = 0; i < n_sel; ++i) {
+        int j = sel[i];
+        if (j < 0 || j >= n_pages || pt_row[j] < 0 || pt_row[j] >= num_blocks)
+            return -1;
+        n_tok += seq_len - j * P < P ? seq_len - j * P : P;
+    }
+    int *blk = (int *)malloc(sizeof(int) * (size_t)(n_tok > 0 ? n_tok : 1));
+    int *pos = (int *)malloc(sizeof(int) * (size_t)(n_tok > 0 ? n_tok : 1));
+    int t_all = 0;
+    for (int i = 0; i < n_sel; ++i) {
+        int j = sel[i];
+        int n = seq_len - j * P < P ? seq_len - j * P : P;
+        for (int t = 0; t < n; ++t) {
+            blk[t_all] = pt_row[j];
+            pos[t_all] = t;
+            ++t_all;
+        }
+    }
+    attend_rows(k_cache, v_cache, dtype, H_kv, P, d, blk, pos, n_tok, h, q, G, scale, mode, out,
+                stat, weights);
+    free(blk);
+    free(pos);
+    return n_tok;
+}
+
+/* ---------------------------------------------------------------------------------------
+ * Token-level selection inside the selected pages, one selection per KV head (JSSA, "Joint
+ * Subspace Sparse Attention for efficient long-context decoding", abstract on ai.info:
+ * token-granular selection and an attention kernel indexed into the standard GQA cache
+ * layout, with distinct selections per KV head). Readings:
+ *   - a candidate token's score for KV head h is the sum over the G query heads of the group of
+ *     scale * q_g . k, taken in the full key space (JSSA scores in a low-dimensional subspace
+ *     fitted to data; with no data the subspace is the whole space, the full-rank limit);
+ *   - candidates are the valid tokens of the selected pages, numbered in visiting order (page
+ *     order of `sel`, then position); the T best by (score descending, number ascending) are
+ *     kept and emitted in candidate order as (logical page, position) pairs.
+ * Returns min(T, candidates), or -1 when a selected page or its page-table entry is out of
+ * range.
+ * ------------------------------------------------------------------------------------- */
+int ora_token_topk_head(const void *k_cache, int dtype, int num_blocks, int H_kv, int P, int d,
+                        const int32_t *pt_row, int seq_len, int h, const double *q, int G,
+                        double scale, const int32_t *sel, int n_sel, int T, int32_t *tok_page,
+                        int32_t *tok_pos)
+{
+    int n_pages = pages_of(seq_len, P);
+    int n_cand = 0;
+    for (int i = 0; i < n_sel; ++i) {
+        int j = sel[i];
+        if (j < 0 || j >= n_pages || pt_row[j] < 0 || pt_row[j] >= num_blocks)
+            return -1;
+        n_cand += seq_len - j * P < P ? seq_len - j * P : P;
+    }
+    if (n_cand == 0 || T <= 0)
+        return 0;
+    int32_t *cpage = (int32_t *)malloc(sizeof(int32_t) * (size_t)n_cand);
+    int32_t *cpos = (int32_t *)malloc(sizeof(int32_t) * (size_t)n_cand);
+    double *score = (double *)malloc(sizeof(double) * (size_t)n_cand);
+    int32_t *kept = (int32_t *)malloc(sizeof(int32_t) * (size_t)n_cand);
+    int m = 0;
+    for (int i = 0; i < n_sel; ++i) {
+        int j = sel[i];
+        int n = seq_len - j * P < P ? seq_len - j * P : P;
+        for (int t = 0; t < n; ++t) {
+            double acc = 0.0;
+            for (int g = 0; g < G; ++g) {
+                double sg = 0.0;
+                for (int c = 0; c < d; ++c)
+                    sg += q[(size_t)g * d + c] * elem(k_cache, dtype, cache_off(pt_row[j], h, t, c, H_kv, P, d));
+                acc += scale * sg;
+            }
+            cpage[m] = j;
+            cpos[m] = t;
+            score[m] = acc;
+            ++m;
+        }
+    }
+    int cnt = ora_topk(score, n_cand, T, kept);  /* candidate numbers, ascending */
+    for (int i = 0; i < cnt; ++i) {
+        tok_page[i] = cpage[kept[i]];
+        tok_pos[i] = cpos[kept[i]];
+    }
+    free(cpage);
+    free(cpos);
+    free(score);
+    free(kept);
+    return cnt;
+}
+
+/* Attention of the G queries over an explicit list of (logical page, position) tokens of one
+ * sequence, read in place through the page table: the indexed attention of the token-level
+ * selection above, with the arithmetic of ora_attend_head. Returns the token count, or -1 when a
+ * page, a position or a page-table entry is out of range. */
+int ora_attend_tokens_head(const void *k_cache, const void *v_cache, int dtype, int num_blocks,
+                           int H_kv, int P, int d, const int32_t *pt_row, int seq_len, int h,
+                           const double *q, int G, double scale, int mode,
+                           const int32_t *tok_page, const int32_t *tok_pos, int n_tok,
+                           double *out, double *stat)
+{
+    int n_pages = pages_of(seq_len, P);
+    int *blk = (int *)malloc(sizeof(int) * (size_t)(n_tok > 0 ? n_tok : 1));
+    int *pos = (int *)malloc(sizeof(int) * (size_t)(n_tok > 0 ? n_tok : 1));
+    for (int i = 0; i < n_tok; ++i) {
+        int j = tok_page[i], t = tok_pos[i];
+        if (j < 0 || j >= n_pages || pt_row[j] < 0 || pt_row[j] >= num_blocks || t < 0 ||
+            t >= P || j * P + t >= seq_len) {
+            free(blk);
+            free(pos);
+            return -1;
+        }
+        blk[i] = pt_row[j];
+        pos[i] = t;
+    }
+    attend_rows(k_cache, v_cache, dtype, H_kv, P, d, blk, pos, n_tok, h, q, G, scale, mode, out,
+                stat, NULL);
+    free(blk);
+    free(pos);
     return n_tok;
 }
 

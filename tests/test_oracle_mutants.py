@@ -45,6 +45,13 @@ MUTANTS = {
                                   "const double logZE = sbar;"),
     "moment_mix_weights_swapped": ("og[a] = wR * og[a] + (1.0 - wR) * fE[a];",
                                    "og[a] = (1.0 - wR) * og[a] + wR * fE[a];"),
+    "token_score_first_query_only": ("            for (int g = 0; g < G; ++g) {\n                double sg = 0.0;",
+                                     "            for (int g = 0; g < 1; ++g) {\n                double sg = 0.0;"),
+    "token_candidates_past_the_sequence_end": (
+        "        int n = seq_len - j * P < P ? seq_len - j * P : P;\n        for (int t = 0; t < n; ++t) {\n            double acc",
+        "        int n = P;\n        for (int t = 0; t < n; ++t) {\n            double acc"),
+    "token_attention_ignores_position": ("        blk[i] = pt_row[j];\n        pos[i] = t;",
+                                         "        blk[i] = pt_row[j];\n        pos[i] = 0;"),
     "attention_reads_invalid_tokens": (
         "n_tok += seq_len - j * P < P ? seq_len - j * P : P;", "n_tok += P;"),
 }

@@ -630,3 +630,105 @@ def test_moment_correction_without_skipped_tokens_is_the_plain_softmax():
     assert n_e == 0
     np.testing.assert_array_equal(out, ref)
     np.testing.assert_array_equal(stat, rstat)
+
+
+# ----------------------------------------------------------------------------- token-level selection
+# JSSA abstract (ai.info): token-granular selection, one selection per KV head, attention indexed
+# into the standard GQA cache layout.
+def candidate_rows(cache, pt, L, h, sel):
+    P = cache.shape[2]
+    idx = [(j, t) for j in sel for t in range(min(P, L - j * P))]
+    rows = np.array([cache[pt[j], h, t] for j, t in idx], dtype=np.float64)
+    return idx, rows
+
+
+@pytest.mark.parametrize("T", [1, 5, 17, 1000])
+def test_token_topk_matches_library_sort(T):
+    rng = np.random.default_rng(41)
+    L, P, d, h, scale = 61, 8, 16, 1, 0.3
+    k, v, pt = make_seq(rng, P=P, d=d, L=L)
+    q = rng.standard_normal((3, d))
+    sel = [0, 2, 5, 7]  # page 7 holds the five valid tokens of the partial last page
+    pages, pos = O.token_topk_head(k, pt, L, h, q, scale, sel, T)
+    idx, K = candidate_rows(k, pt, L, h, sel)
+    score = (scale * (q @ K.T)).sum(axis=0)
+    order = np.lexsort((np.arange(len(idx)), -score))  # score descending, earlier first on ties
+    keep = np.sort(order[:T])
+    assert list(zip(pages.tolist(), pos.tolist())) == [idx[i] for i in keep]
+
+
+def test_token_topk_ties_prefer_earlier_candidates():
+    rng = np.random.default_rng(42)
+    L, P, d = 61, 8, 16
+    k, v, pt = make_seq(rng, P=P, d=d, L=L)
+    k[:, 0] = 0.5  # every key of head 0 equal: every candidate ties
+    pages, pos = O.token_topk_head(k, pt, L, 0, rng.standard_normal((2, d)), 1.0, [3, 1, 6], 11)
+    assert pages.tolist() == [3] * 8 + [1] * 3 and pos.tolist() == list(range(8)) + [0, 1, 2]
+
+
+@pytest.mark.parametrize("mode", [O.SOFTMAX, O.ENTMAX15, O.SPARSEMAX])
+def test_attention_over_every_candidate_is_the_page_attention(mode):
+    rng = np.random.default_rng(43)
+    L, P, d, h = 61, 8, 16, 0
+    k, v, pt = make_seq(rng, P=P, d=d, L=L, dist_scale=2.0)
+    q = rng.standard_normal((4, d))
+    sel = [1, 4, 7]
+    pages, pos = O.token_topk_head(k, pt, L, h, q, 0.5, sel, 10 ** 6)
+    out, stat = O.attend_tokens_head(k, v, pt, L, h, q, 0.5, mode, pages, pos)
+    ref, rstat, _ = O.attend_head(k, v, pt, L, h, q, 0.5, mode, sel)
+    np.testing.assert_array_equal(out, ref)
+    np.testing.assert_array_equal(stat, rstat)
+
+
+@pytest.mark.parametrize("mode", [O.SOFTMAX, O.ENTMAX15, O.SPARSEMAX])
+def test_attention_over_one_token_is_its_value(mode):
+    # one token: softmax weight 1 with log-partition = its logit; entmax tau = z - 1, weight 1
+    rng = np.random.default_rng(44)
+    k, v, pt = make_seq(rng, P=8, d=16, L=61)
+    q = rng.standard_normal((2, 16))
+    out, stat = O.attend_tokens_head(k, v, pt, 61, 1, q, 0.7, mode, [6], [3])
+    row_k, row_v = k[pt[6], 1, 3].astype(np.float64), v[pt[6], 1, 3].astype(np.float64)
+    np.testing.assert_allclose(out, np.tile(row_v, (2, 1)), rtol=0, atol=1e-15)
+    s = 0.7 * q @ row_k
+    want = s if mode == O.SOFTMAX else (O.ALPHA_OF_MODE[mode] - 1.0) * s - 1.0
+    np.testing.assert_allclose(stat, want, rtol=0, atol=1e-13)
+
+
+@pytest.mark.parametrize("mode", [O.ENTMAX15, O.SPARSEMAX])
+def test_token_selection_holding_the_support_gives_the_page_output(mode):
+    # EntmaxKV §3 at token granularity: entmax over any superset of its support has the same
+    # threshold and output, because the extra tokens sit at or below tau.
+    rng = np.random.default_rng(45)
+    L, P, d, h, scale = 61, 8, 16, 1, 0.8
+    k, v, pt = make_seq(rng, P=P, d=d, L=L, dist_scale=3.0)
+    q = rng.standard_normal((2, d))
+    sel = list(range(O.pages_of(L, P)))
+    ref, rstat, w = O.attend_head(k, v, pt, L, h, q, scale, mode, sel, want_weights=True)
+    idx, _ = candidate_rows(k, pt, L, h, sel)
+    support = {idx[i] for i in np.nonzero((w > 0).any(axis=0))[0]}
+    assert 0 < len(support) < len(idx) // 2
+    for T in range(1, len(idx) + 1):
+        pages, pos = O.token_topk_head(k, pt, L, h, q, scale, sel, T)
+        if support <= set(zip(pages.tolist(), pos.tolist())):
+            break
+    assert T < len(idx)
+    out, stat = O.attend_tokens_head(k, v, pt, L, h, q, scale, mode, pages, pos)
+    np.testing.assert_allclose(out, ref, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(stat, rstat, rtol=0, atol=1e-12)
+
+
+def test_indexed_attention_reads_only_the_listed_rows():
+    rng = np.random.default_rng(46)
+    L, P, d = 61, 8, 16
+    k, v, pt = make_seq(rng, P=P, d=d, L=L)
+    q = rng.standard_normal((2, d))
+    pages, pos = [0, 0, 3, 7], [1, 6, 2, 4]
+    a = O.attend_tokens_head(k, v, pt, L, 0, q, 1.0, O.SOFTMAX, pages, pos)
+    k2, v2 = np.full_like(k, 1e6), np.full_like(v, 1e6)
+    for j, t in zip(pages, pos):
+        k2[pt[j], 0, t], v2[pt[j], 0, t] = k[pt[j], 0, t], v[pt[j], 0, t]
+    b = O.attend_tokens_head(k2, v2, pt, L, 0, q, 1.0, O.SOFTMAX, pages, pos)
+    np.testing.assert_array_equal(a[0], b[0])
+    np.testing.assert_array_equal(a[1], b[1])
+    with pytest.raises(ValueError):  # position 5 of page 7 is past the sequence end (61 tokens)
+        O.attend_tokens_head(k, v, pt, L, 0, q, 1.0, O.SOFTMAX, [7], [5])
