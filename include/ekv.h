@@ -204,6 +204,60 @@ ekv_status ekv_sparse_decode_noalloc(const ekv_cache *c, const void *q, int32_t 
  * (0 on invalid arguments). */
 size_t ekv_decode_workspace_bytes(const ekv_cache *c, int32_t num_q_heads, int32_t max_sel);
 
+/*
+ * Moment correction of a softmax decode for the pages it skips (MomentKV technical summary,
+ * gist.science, Methodology §1, §2, §4). (Not part of the EntmaxKV method: entmax gives the
+ * skipped tokens exact zeros wherever the support is kept; this is the softmax remedy.)
+ * The cache keeps every token and a decode step skips the pages it did not select: those tokens
+ * form the evicted set E of that step.
+ *
+ * Running moments: per (sequence, KV head), sums over every token appended so far, one fp32
+ * record of EKV_MOMENT_FLOATS(d) floats:
+ *   [0] n (token count)   [1..3] 0   [4, 4+d) sum k   [4+d, 4+2d) sum v
+ *   [4+2d, 4+2d+d*d) sum v k^T, row a = value coordinate, column c = key coordinate.
+ * moments: [batch][H_kv] records, ekv_moment_bytes(c) bytes, zero-filled by the caller before
+ * the first update.
+ */
+#define EKV_MOMENT_FLOATS(d) (4 + 2 * (d) + (d) * (d))
+
+/* Bytes of the running-moment records of this cache geometry (0 on invalid arguments). */
+size_t ekv_moment_bytes(const ekv_cache *c);
+
+/*
+ * Add the tokens [new_start[b], new_start[b] + new_count[b]) of every sequence b to its running
+ * moments (every KV head). Each token must be added once: prefill with new_start = 0,
+ * new_count = seq_lens, then each appended range. Arguments and range checks are those of
+ * ekv_page_meta_update (a range outside [0, seq_lens[b]] or longer than max_new is clamped and
+ * flagged EKV_DEV_BAD_RANGE; a bad page-table entry is skipped and flagged). Needs c->v_cache.
+ */
+ekv_status ekv_moment_update(const ekv_cache *c, float *moments, const int32_t *new_start,
+                             const int32_t *new_count, int32_t max_new, void *stream);
+
+/* Scratch bytes ekv_sparse_decode_moment needs (0 on invalid arguments). */
+size_t ekv_moment_decode_workspace_bytes(const ekv_cache *c, int32_t num_q_heads,
+                                         int32_t max_sel);
+
+/*
+ * ekv_sparse_decode with attn = EKV_SOFTMAX, then corrected for the skipped tokens E of each
+ * (sequence, KV head), per query head (logits s = scale q.k):
+ *   n_e = |E|, kbar, vbar = the mean key and value over E,
+ *   fE = vbar + (scale / n_e) sum_E (v - vbar)(k - kbar)^T q     (first-order estimate of E's
+ *        softmax output around the mean logit scale q.kbar),
+ *   ZE = n_e exp(scale q.kbar)                                    (Jensen lower bound on E's
+ *        partition sum),
+ *   out = wR fR + (1 - wR) fE,  wR = ZR / (ZR + ZE),  stat = log(ZR + ZE),
+ * with fR, log ZR the softmax output and stat over the selected pages. E's sums are the running
+ * moments less the sums over the selected tokens, which this call re-reads. With nothing
+ * skipped (n_e = 0) the result is the plain softmax. Arguments are those of
+ * ekv_sparse_decode, plus `moments` (as kept by ekv_moment_update for exactly the tokens
+ * [0, seq_lens[b]) of each sequence); ws holds at least
+ * ekv_moment_decode_workspace_bytes(c, num_q_heads, max_sel) bytes under the same rules.
+ */
+ekv_status ekv_sparse_decode_moment(const ekv_cache *c, const float *moments, const void *q,
+                                    int32_t num_q_heads, float scale, const int32_t *sel_idx,
+                                    const int32_t *sel_count, int32_t max_sel, float *out,
+                                    float *stat, void *ws, size_t ws_bytes, void *stream);
+
 /* Synchronise `stream`, copy *c->dev_status to *bits (host pointer, may be NULL) and return
  * EKV_ERR_DEVICE if any bit is set, else EKV_OK (EKV_ERR_CUDA if the copy fails). */
 ekv_status ekv_device_status(const ekv_cache *c, uint32_t *bits, void *stream);

@@ -67,6 +67,9 @@ def _load():
     lib.ora_moment_corrected_head.argtypes = [vp, vp, c_int, c_int, c_int, c_int, c_int, _ip, c_int,
                                               c_int, _dp, c_int, c_double, _ip, c_int, _dp, _dp]
     lib.ora_moment_corrected_head.restype = c_int
+    lib.ora_moment_sums_head.argtypes = [vp, vp, c_int, c_int, c_int, c_int, c_int, _ip, c_int,
+                                         c_int, _ip, c_int, _dp, _dp, _dp]
+    lib.ora_moment_sums_head.restype = c_int
     lib.ora_token_topk_head.argtypes = [vp, c_int, c_int, c_int, c_int, c_int, _ip, c_int, c_int,
                                         _dp, c_int, c_double, _ip, c_int, c_int, _ip, _ip]
     lib.ora_token_topk_head.restype = c_int
@@ -266,6 +269,30 @@ def moment_corrected_head(k_cache, v_cache, pt_row, seq_len: int, h: int, q, sca
     if rc < 0:
         raise ValueError("selected page or page-table entry out of range")
     return out, stat, rc
+
+
+def moment_sums_head(k_cache, v_cache, pt_row, seq_len: int, h: int, pages=None):
+    """Count, key sum, value sum and value-key outer-product sum S[a][c] = sum v_a k_c over the
+    valid tokens of the listed logical pages (all pages when None) of one (sequence, KV head)
+    (MomentKV technical summary, Methodology §1). Returns (n, sk [d], sv [d], S [d, d])."""
+    nb, H_kv, P, d = k_cache.shape
+    k_cache = np.ascontiguousarray(k_cache)
+    v_cache = np.ascontiguousarray(v_cache)
+    dt = _cache_dtype(k_cache)
+    if _cache_dtype(v_cache) != dt:
+        raise TypeError("K and V caches must share a dtype")
+    if pages is None:
+        pages = np.arange(pages_of(seq_len, P))
+    pt, ptp = _i(pt_row)
+    pg, pgp = _i(np.asarray(pages, dtype=np.int32).reshape(-1))
+    sk, sv, S = np.zeros(d), np.zeros(d), np.zeros((d, d))
+    n = _load().ora_moment_sums_head(k_cache.ctypes.data, v_cache.ctypes.data, dt, nb, H_kv, P, d,
+                                     ptp, int(seq_len), int(h), pgp, len(pg),
+                                     sk.ctypes.data_as(_dp), sv.ctypes.data_as(_dp),
+                                     S.ctypes.data_as(_dp))
+    if n < 0:
+        raise ValueError("page or page-table entry out of range")
+    return n, sk, sv, S
 
 
 def token_topk_head(k_cache, pt_row, seq_len: int, h: int, q, scale: float, sel, T: int):

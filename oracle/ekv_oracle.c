@@ -666,3 +666,37 @@ int ora_moment_corrected_head(const void *k_cache, const void *v_cache, int dtyp
     free(fE);
     return n_e;
 }
+
+/* Moment sums of one (sequence, KV head) over the valid tokens of the listed logical pages
+ * (MomentKV technical summary, Methodology §1: count, key sum, value sum and value-key
+ * outer-product sum): n, sk [d], sv [d], S [d][d] with S[a][c] = sum v_a k_c.
+ * Returns n, or -1 when a page or page-table entry is out of range. */
+int ora_moment_sums_head(const void *k_cache, const void *v_cache, int dtype, int num_blocks,
+                         int H_kv, int P, int d, const int32_t *pt_row, int seq_len, int h,
+                         const int32_t *pages, int n_list, double *sk, double *sv, double *S)
+{
+    const int n_pages = pages_of(seq_len, P);
+    for (int c = 0; c < d; ++c)
+        sk[c] = sv[c] = 0.0;
+    for (size_t i = 0; i < (size_t)d * d; ++i)
+        S[i] = 0.0;
+    int n = 0;
+    for (int i = 0; i < n_list; ++i) {
+        const int j = pages[i];
+        if (j < 0 || j >= n_pages || pt_row[j] < 0 || pt_row[j] >= num_blocks)
+            return -1;
+        const int cnt = seq_len - j * P < P ? seq_len - j * P : P;
+        for (int t = 0; t < cnt; ++t) {
+            for (int a = 0; a < d; ++a) {
+                const double va = elem(v_cache, dtype, cache_off(pt_row[j], h, t, a, H_kv, P, d));
+                sv[a] += va;
+                for (int c = 0; c < d; ++c)
+                    S[(size_t)a * d + c] += va * elem(k_cache, dtype, cache_off(pt_row[j], h, t, c, H_kv, P, d));
+            }
+            for (int c = 0; c < d; ++c)
+                sk[c] += elem(k_cache, dtype, cache_off(pt_row[j], h, t, c, H_kv, P, d));
+            ++n;
+        }
+    }
+    return n;
+}

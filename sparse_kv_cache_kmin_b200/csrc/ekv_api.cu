@@ -25,6 +25,13 @@ cudaError_t launch_sparse_decode(const ekv_cache &c, const void *q, int H_q, flo
                                  bool pdl);
 size_t decode_workspace_bytes_all_modes(int batch, int H_q, int H, int D, int P, int dtype,
                                         int max_sel);
+cudaError_t launch_moment_update(const ekv_cache &c, float *moments, const int32_t *new_start,
+                                 const int32_t *new_count, int max_new, cudaStream_t st);
+cudaError_t launch_moment_pass(const ekv_cache &c, const float *moments, const void *q, int H_q,
+                               float scale, const int32_t *sel_idx, const int32_t *sel_count,
+                               int max_sel, float *ret, float *out, float *stat, cudaStream_t st,
+                               bool after_decode);
+size_t moment_retained_bytes(int batch, int H_kv, int D, int G);
 
 int persistent_grid_size(const void *kernel, int threads, size_t smem)
 {
@@ -171,6 +178,63 @@ ekv_status ekv_sparse_decode(const ekv_cache *c, const void *q, int32_t num_q_he
     return cuda_status(launch_sparse_decode(*c, q, num_q_heads, scale, attn, sel_idx, sel_count,
                                             max_sel, out, stat, ws,
                                             static_cast<cudaStream_t>(stream), use_pdl()));
+}
+
+size_t ekv_moment_bytes(const ekv_cache *c)
+{
+    if (check_cache(c, true) != EKV_OK) return 0;
+    return (size_t)c->batch * c->num_kv_heads * EKV_MOMENT_FLOATS((size_t)c->head_dim) * sizeof(float);
+}
+
+ekv_status ekv_moment_update(const ekv_cache *c, float *moments, const int32_t *new_start,
+                             const int32_t *new_count, int32_t max_new, void *stream)
+{
+    ekv_status s = check_cache(c, true);
+    if (s != EKV_OK) return s;
+    if (!moments || !new_start || !new_count || max_new < 0) return EKV_ERR_INVALID_ARG;
+    if ((long long)max_new > (long long)c->max_pages * c->page_size) return EKV_ERR_INVALID_ARG;
+    return cuda_status(launch_moment_update(*c, moments, new_start, new_count, max_new,
+                                            static_cast<cudaStream_t>(stream)));
+}
+
+// The decode workspace, then (256-byte aligned) the sums over the selected tokens.
+static size_t moment_ret_offset(size_t decode_bytes) { return (decode_bytes + 255) & ~(size_t)255; }
+
+size_t ekv_moment_decode_workspace_bytes(const ekv_cache *c, int32_t num_q_heads, int32_t max_sel)
+{
+    const size_t base = ekv_decode_workspace_bytes(c, num_q_heads, max_sel);
+    if (!base) return 0;
+    return moment_ret_offset(base) + moment_retained_bytes(c->batch, c->num_kv_heads, c->head_dim,
+                                                           num_q_heads / c->num_kv_heads);
+}
+
+ekv_status ekv_sparse_decode_moment(const ekv_cache *c, const float *moments, const void *q,
+                                    int32_t num_q_heads, float scale, const int32_t *sel_idx,
+                                    const int32_t *sel_count, int32_t max_sel, float *out,
+                                    float *stat, void *ws, size_t ws_bytes, void *stream)
+{
+    ekv_status s = check_cache(c, true);
+    if (s != EKV_OK) return s;
+    if ((s = check_heads(c, num_q_heads)) != EKV_OK) return s;
+    if (!moments || !q || !sel_idx || !sel_count || !out || !stat || max_sel < 1 ||
+        !(scale > 0.0f) || !std::isfinite(scale))
+        return EKV_ERR_INVALID_ARG;
+    if (((uintptr_t)q | (uintptr_t)c->k_cache | (uintptr_t)c->v_cache) & 15u)
+        return EKV_ERR_INVALID_ARG;
+    if (!ws || ws_bytes < ekv_moment_decode_workspace_bytes(c, num_q_heads, max_sel))
+        return EKV_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    float *ret = reinterpret_cast<float *>(
+        static_cast<char *>(ws) + moment_ret_offset(ekv_decode_workspace_bytes(c, num_q_heads, max_sel)));
+    cudaError_t e = launch_moment_pass(*c, moments, q, num_q_heads, scale, sel_idx, sel_count,
+                                       max_sel, ret, out, stat, st, false);
+    if (e == cudaSuccess)
+        e = launch_sparse_decode(*c, q, num_q_heads, scale, EKV_SOFTMAX, sel_idx, sel_count,
+                                 max_sel, out, stat, ws, st, use_pdl());
+    if (e == cudaSuccess)
+        e = launch_moment_pass(*c, moments, q, num_q_heads, scale, sel_idx, sel_count, max_sel,
+                               ret, out, stat, st, true);
+    return cuda_status(e);
 }
 
 ekv_status ekv_device_status(const ekv_cache *c, uint32_t *bits, void *stream)

@@ -279,3 +279,51 @@ def ekv_sparse_decode_noalloc(cache: PagedKVCache, q: torch.Tensor, num_q_heads:
     _check(fn(ctypes.byref(c), _ptr(q), int(num_q_heads), float(scale), int(attn), _ptr(sel_idx),
               _ptr(sel_count), int(max_sel), _ptr(out), _ptr(stat), _stream(stream)),
            "ekv_sparse_decode_noalloc")
+
+
+def _moment_fn(name, args, res=ctypes.c_int):
+    fn = getattr(load_library(), name)
+    if fn.argtypes is None:
+        fn.argtypes, fn.restype = args, res
+    return fn
+
+
+def ekv_moment_bytes(cache: PagedKVCache) -> int:
+    """Bytes of the running-moment records [batch][H_kv][EKV_MOMENT_FLOATS(d)] fp32."""
+    fn = _moment_fn("ekv_moment_bytes", [ctypes.POINTER(EkvCacheStruct)], ctypes.c_size_t)
+    c = cache.struct()
+    return int(fn(ctypes.byref(c)))
+
+
+def ekv_moment_update(cache: PagedKVCache, moments: torch.Tensor, new_start: torch.Tensor,
+                      new_count: torch.Tensor, max_new: int, stream=None):
+    """Add the token ranges [new_start[b], new_start[b] + new_count[b]) to the running moments
+    (a zero-filled float32 tensor of ekv_moment_bytes bytes before the first update)."""
+    P, I32 = ctypes.c_void_p, ctypes.c_int32
+    fn = _moment_fn("ekv_moment_update", [ctypes.POINTER(EkvCacheStruct), P, P, P, I32, P])
+    c = cache.struct()
+    _check(fn(ctypes.byref(c), _ptr(moments), _ptr(new_start), _ptr(new_count), int(max_new),
+              _stream(stream)), "ekv_moment_update")
+
+
+def ekv_moment_decode_workspace_bytes(cache: PagedKVCache, num_q_heads: int, max_sel: int) -> int:
+    fn = _moment_fn("ekv_moment_decode_workspace_bytes",
+                    [ctypes.POINTER(EkvCacheStruct), ctypes.c_int32, ctypes.c_int32],
+                    ctypes.c_size_t)
+    c = cache.struct()
+    return int(fn(ctypes.byref(c), int(num_q_heads), int(max_sel)))
+
+
+def ekv_sparse_decode_moment(cache: PagedKVCache, moments: torch.Tensor, q: torch.Tensor,
+                             num_q_heads: int, scale: float, sel_idx: torch.Tensor,
+                             sel_count: torch.Tensor, max_sel: int, out: torch.Tensor,
+                             stat: torch.Tensor, ws: torch.Tensor, stream=None):
+    """Softmax over the selected pages, corrected for the skipped tokens from the running
+    moments (see include/ekv.h)."""
+    P, I32, F, U64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float, ctypes.c_size_t
+    fn = _moment_fn("ekv_sparse_decode_moment",
+                    [ctypes.POINTER(EkvCacheStruct), P, P, I32, F, P, P, I32, P, P, P, U64, P])
+    c = cache.struct()
+    _check(fn(ctypes.byref(c), _ptr(moments), _ptr(q), int(num_q_heads), float(scale),
+              _ptr(sel_idx), _ptr(sel_count), int(max_sel), _ptr(out), _ptr(stat), _ptr(ws),
+              ws.numel() * ws.element_size(), _stream(stream)), "ekv_sparse_decode_moment")

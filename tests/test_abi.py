@@ -149,3 +149,34 @@ def test_product_path_does_not_import_the_oracle():
                 text = open(os.path.join(dirpath, f)).read()
                 assert not re.search(r"^\s*(from|import)\s+oracle\b", text, re.M), f
                 assert "ekv_oracle" not in text, f
+
+
+def test_moment_entry_points_validation(lib):
+    from sparse_kv_cache_kmin_b200.ekv import load_library
+    import ctypes as C
+    P = 0x1000
+    lib = load_library()
+    cp = C.POINTER(type(fake_cache()))
+    lib.ekv_moment_bytes.argtypes, lib.ekv_moment_bytes.restype = [cp], C.c_size_t
+    lib.ekv_moment_decode_workspace_bytes.argtypes = [cp, C.c_int32, C.c_int32]
+    lib.ekv_moment_decode_workspace_bytes.restype = C.c_size_t
+    lib.ekv_moment_update.argtypes = [cp, C.c_void_p, C.c_void_p, C.c_void_p, C.c_int32, C.c_void_p]
+    lib.ekv_sparse_decode_moment.argtypes = [cp, C.c_void_p, C.c_void_p, C.c_int32, C.c_float,
+                                             C.c_void_p, C.c_void_p, C.c_int32, C.c_void_p,
+                                             C.c_void_p, C.c_void_p, C.c_size_t, C.c_void_p]
+    c = fake_cache()
+    # [batch][H_kv] records of 4 + 2d + d*d floats
+    assert lib.ekv_moment_bytes(C.byref(c)) == 4 * 8 * (4 + 2 * 128 + 128 * 128) * 4
+    assert lib.ekv_moment_bytes(C.byref(fake_cache(v_cache=None))) == 0
+    base = lib.ekv_decode_workspace_bytes(C.byref(c), 32, 256)
+    need = lib.ekv_moment_decode_workspace_bytes(C.byref(c), 32, 256)
+    # the decode workspace, then [batch][H_kv] records of 4 + 2d + G*d floats
+    assert need >= base + 4 * 8 * (4 + 2 * 128 + 4 * 128) * 4
+    assert lib.ekv_moment_decode_workspace_bytes(C.byref(c), 30, 256) == 0
+    assert lib.ekv_moment_update(C.byref(c), None, P, P, 16, None) == 1
+    assert lib.ekv_moment_update(C.byref(c), P, P, P, -1, None) == 1
+    assert lib.ekv_moment_update(C.byref(c), P, P, P, 256 * 16 + 1, None) == 1
+    assert lib.ekv_sparse_decode_moment(C.byref(c), None, P, 32, 1.0, P, P, 256, P, P, P, need, None) == 1
+    assert lib.ekv_sparse_decode_moment(C.byref(c), P, P, 32, 1.0, P, P, 256, P, P, P, need - 1, None) == 3
+    assert lib.ekv_sparse_decode_moment(C.byref(c), P, P, 30, 1.0, P, P, 256, P, P, P, need, None) == 1
+    assert lib.ekv_sparse_decode_moment(C.byref(c), P, P, 32, 0.0, P, P, 256, P, P, P, need, None) == 1

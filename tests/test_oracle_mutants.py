@@ -52,6 +52,8 @@ MUTANTS = {
         "        int n = P;\n        for (int t = 0; t < n; ++t) {\n            double acc"),
     "token_attention_ignores_position": ("        blk[i] = pt_row[j];\n        pos[i] = t;",
                                          "        blk[i] = pt_row[j];\n        pos[i] = 0;"),
+    "moment_sums_transposed": ("                    S[(size_t)a * d + c] += va * elem(",
+                               "                    S[(size_t)c * d + a] += va * elem("),
     "attention_reads_invalid_tokens": (
         "n_tok += seq_len - j * P < P ? seq_len - j * P : P;", "n_tok += P;"),
 }

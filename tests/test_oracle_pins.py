@@ -732,3 +732,27 @@ def test_indexed_attention_reads_only_the_listed_rows():
     np.testing.assert_array_equal(a[1], b[1])
     with pytest.raises(ValueError):  # position 5 of page 7 is past the sequence end (61 tokens)
         O.attend_tokens_head(k, v, pt, L, 0, q, 1.0, O.SOFTMAX, [7], [5])
+
+
+def test_moment_sums_golden_fixture_and_additivity():
+    g = parse_golden("moment_correction_example.txt")
+    k = np.zeros((2, 1, 2, 2), dtype=np.float32)
+    v = np.zeros((2, 1, 2, 2), dtype=np.float32)
+    k[0, 0], v[0, 0] = g["keys_page0"], g["vals_page0"]
+    k[1, 0], v[1, 0] = g["keys_page1"], g["vals_page1"]
+    pt = np.array([0, 1], np.int32)
+    n, sk, sv, S = O.moment_sums_head(k, v, pt, 4, 0, [1])
+    assert n == 2
+    np.testing.assert_array_equal(sk, g["sums_page1_k"])
+    np.testing.assert_array_equal(sv, g["sums_page1_v"])
+    np.testing.assert_array_equal(S, g["sums_page1_vk"])
+    # sums over disjoint page sets add up (the running sums less the selected ones are the
+    # skipped ones), checked on a random paged sequence with a partial last page
+    rng = np.random.default_rng(47)
+    k, v, pt = make_seq(rng, P=8, d=16, L=61)
+    whole = O.moment_sums_head(k, v, pt, 61, 1)
+    a = O.moment_sums_head(k, v, pt, 61, 1, [0, 3, 7])
+    b = O.moment_sums_head(k, v, pt, 61, 1, [1, 2, 4, 5, 6])
+    assert whole[0] == 61 and a[0] + b[0] == 61
+    for x, y, z in zip(whole[1:], a[1:], b[1:]):
+        np.testing.assert_allclose(x, y + z, rtol=0, atol=1e-12)
