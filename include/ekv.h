@@ -258,6 +258,44 @@ ekv_status ekv_sparse_decode_moment(const ekv_cache *c, const float *moments, co
                                     const int32_t *sel_count, int32_t max_sel, float *out,
                                     float *stat, void *ws, size_t ws_bytes, void *stream);
 
+/*
+ * Token-level selection inside the selected pages, with attention indexed into the cache
+ * (after the JSSA abstract on ai.info: token-granular selection, one selection per KV head,
+ * attention on the standard GQA cache layout with no gather copy). Not part of EntmaxKV:
+ * a finer granularity applied after its page selection.
+ *   Candidates of (sequence b, KV head h): the valid tokens of the pages in
+ *   sel_idx[b][h][0 .. sel_count), in that order and then by position. A candidate's score is
+ *   the group sum sum_g scale * q_g . k over the G query heads of h (the full key space).
+ *   The T best, ties to the earlier candidate, are kept in candidate order.
+ */
+#define EKV_MAX_TOKENS 32768 /* largest T */
+
+/* Scratch bytes of ekv_select_tokens: one fp32 score per candidate slot,
+ * batch * H_kv * max_sel * P * 4 (0 on invalid arguments). */
+size_t ekv_token_workspace_bytes(const ekv_cache *c, int32_t max_sel);
+
+/*
+ *   tok_page, tok_pos  [batch][H_kv][T] int32 outputs: logical page and position of each kept
+ *                      token, -1 padded.   tok_count [batch][H_kv] int32 output.
+ *   T in [1, EKV_MAX_TOKENS] (EKV_ERR_UNSUPPORTED above, EKV_ERR_INVALID_ARG below);
+ *   other arguments as in ekv_score_pages / ekv_sparse_decode.
+ */
+ekv_status ekv_select_tokens(const ekv_cache *c, const void *q, int32_t num_q_heads, float scale,
+                             const int32_t *sel_idx, const int32_t *sel_count, int32_t max_sel,
+                             int32_t T, int32_t *tok_page, int32_t *tok_pos, int32_t *tok_count,
+                             void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Attention of every query head over the tokens ekv_select_tokens kept for its KV head, their K
+ * and V rows read in place through the page table: softmax (stat = log-partition) or exact
+ * alpha-entmax (stat = tau), as in ekv_sparse_decode; no kept token gives out = 0,
+ * stat = -inf. A listed token outside its sequence is skipped and flagged EKV_DEV_BAD_SEL.
+ */
+ekv_status ekv_sparse_decode_tokens(const ekv_cache *c, const void *q, int32_t num_q_heads,
+                                    float scale, int32_t attn, const int32_t *tok_page,
+                                    const int32_t *tok_pos, const int32_t *tok_count, int32_t T,
+                                    float *out, float *stat, void *stream);
+
 /* Synchronise `stream`, copy *c->dev_status to *bits (host pointer, may be NULL) and return
  * EKV_ERR_DEVICE if any bit is set, else EKV_OK (EKV_ERR_CUDA if the copy fails). */
 ekv_status ekv_device_status(const ekv_cache *c, uint32_t *bits, void *stream);

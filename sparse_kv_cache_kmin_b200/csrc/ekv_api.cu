@@ -32,6 +32,16 @@ cudaError_t launch_moment_pass(const ekv_cache &c, const float *moments, const v
                                int max_sel, float *ret, float *out, float *stat, cudaStream_t st,
                                bool after_decode);
 size_t moment_retained_bytes(int batch, int H_kv, int D, int G);
+cudaError_t launch_token_scores(const ekv_cache &c, const void *q, int H_q, float scale,
+                                const int32_t *sel_idx, const int32_t *sel_count, int max_sel,
+                                float *tscores, cudaStream_t st);
+cudaError_t launch_select_tokens(const ekv_cache &c, const float *tscores, const int32_t *sel_idx,
+                                 const int32_t *sel_count, int max_sel, int T, int32_t *tok_page,
+                                 int32_t *tok_pos, int32_t *tok_count, cudaStream_t st);
+cudaError_t launch_token_attend(const ekv_cache &c, const void *q, int H_q, float scale, int attn,
+                                const int32_t *tok_page, const int32_t *tok_pos,
+                                const int32_t *tok_count, int T, float *out, float *stat,
+                                cudaStream_t st);
 
 int persistent_grid_size(const void *kernel, int threads, size_t smem)
 {
@@ -235,6 +245,54 @@ ekv_status ekv_sparse_decode_moment(const ekv_cache *c, const float *moments, co
         e = launch_moment_pass(*c, moments, q, num_q_heads, scale, sel_idx, sel_count, max_sel,
                                ret, out, stat, st, true);
     return cuda_status(e);
+}
+
+size_t ekv_token_workspace_bytes(const ekv_cache *c, int32_t max_sel)
+{
+    if (check_cache(c, false) != EKV_OK || max_sel < 1) return 0;
+    return (size_t)c->batch * c->num_kv_heads * max_sel * c->page_size * sizeof(float);
+}
+
+ekv_status ekv_select_tokens(const ekv_cache *c, const void *q, int32_t num_q_heads, float scale,
+                             const int32_t *sel_idx, const int32_t *sel_count, int32_t max_sel,
+                             int32_t T, int32_t *tok_page, int32_t *tok_pos, int32_t *tok_count,
+                             void *ws, size_t ws_bytes, void *stream)
+{
+    ekv_status s = check_cache(c, false);
+    if (s != EKV_OK) return s;
+    if ((s = check_heads(c, num_q_heads)) != EKV_OK) return s;
+    if (!q || !sel_idx || !sel_count || !tok_page || !tok_pos || !tok_count || max_sel < 1 ||
+        T < 1 || !(scale > 0.0f) || !std::isfinite(scale))
+        return EKV_ERR_INVALID_ARG;
+    if (T > EKV_MAX_TOKENS) return EKV_ERR_UNSUPPORTED;
+    if (!ws || ws_bytes < ekv_token_workspace_bytes(c, max_sel)) return EKV_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    float *tscores = static_cast<float *>(ws);
+    cudaError_t e = launch_token_scores(*c, q, num_q_heads, scale, sel_idx, sel_count, max_sel,
+                                        tscores, st);
+    if (e == cudaSuccess)
+        e = launch_select_tokens(*c, tscores, sel_idx, sel_count, max_sel, T, tok_page, tok_pos,
+                                 tok_count, st);
+    return cuda_status(e);
+}
+
+ekv_status ekv_sparse_decode_tokens(const ekv_cache *c, const void *q, int32_t num_q_heads,
+                                    float scale, int32_t attn, const int32_t *tok_page,
+                                    const int32_t *tok_pos, const int32_t *tok_count, int32_t T,
+                                    float *out, float *stat, void *stream)
+{
+    ekv_status s = check_cache(c, true);
+    if (s != EKV_OK) return s;
+    if ((s = check_heads(c, num_q_heads)) != EKV_OK) return s;
+    if (attn != EKV_SOFTMAX && attn != EKV_ENTMAX15 && attn != EKV_SPARSEMAX)
+        return EKV_ERR_UNSUPPORTED;
+    if (!q || !tok_page || !tok_pos || !tok_count || !out || !stat || T < 1 || !(scale > 0.0f) ||
+        !std::isfinite(scale))
+        return EKV_ERR_INVALID_ARG;
+    if (T > EKV_MAX_TOKENS) return EKV_ERR_UNSUPPORTED;
+    return cuda_status(launch_token_attend(*c, q, num_q_heads, scale, attn, tok_page, tok_pos,
+                                           tok_count, T, out, stat,
+                                           static_cast<cudaStream_t>(stream)));
 }
 
 ekv_status ekv_device_status(const ekv_cache *c, uint32_t *bits, void *stream)

@@ -604,3 +604,85 @@ cudaError_t launch_select_pages(const ekv_cache &c, int H_q, int policy, int top
 }
 
 }  // namespace ekv
+
+namespace ekv {
+
+// Token-level top-T inside the selected pages, one 1024-thread CTA per (sequence, KV head).
+// The candidate scores sit at slot i * P + t (selected page i, position t; -inf past a page's
+// valid tokens); the exact radix select above keeps the T largest, ties to the lower slot, in
+// slot order -- which is the candidate order (selection order, then position). Emits
+// (logical page, position) pairs, -1 padded to T, and the count.
+__global__ void __launch_bounds__(kSelThreads)
+select_tokens_kernel(const float *__restrict__ tscores, int H, int P, const int32_t *__restrict__ seq_lens,
+                     int max_pages, const int32_t *__restrict__ sel_idx,
+                     const int32_t *__restrict__ sel_count, int max_sel, int T,
+                     int32_t *__restrict__ tok_page, int32_t *__restrict__ tok_pos,
+                     int32_t *__restrict__ tok_count)
+{
+    constexpr int NT = kSelThreads;
+    __shared__ int hist[2048];
+    __shared__ int warp_tot[32];
+    __shared__ int s_bin, s_above;
+    pdl_wait();
+    const int tid = threadIdx.x;
+    const int bh = blockIdx.x, b = bh / H;
+    int ns = sel_count[bh];
+    ns = ns < 0 ? 0 : (ns > max_sel ? max_sel : ns);
+    int len;
+    const int np = seq_pages(seq_lens, b, P, max_pages, nullptr, &len);
+    const int32_t *sel = sel_idx + (size_t)bh * max_sel;
+    // valid candidates: the tokens of the selected pages that exist
+    int mine = 0;
+    for (int i = tid; i < ns; i += NT) {
+        const int j = sel[i];
+        if (j >= 0 && j < np) mine += len - j * P < P ? len - j * P : P;
+    }
+    int n_valid;
+    block_incl_scan<NT>(mine, warp_tot, &n_valid);
+    const int n = ns * P;
+    const float *S = tscores + (size_t)bh * max_sel * P;
+    int32_t *pg = tok_page + (size_t)bh * T, *ps = tok_pos + (size_t)bh * T;
+    int kk = T < n_valid ? T : n_valid;
+    if (kk > 0) {
+        if (kk == n_valid) {  // every valid candidate is kept: emit them in slot order
+            int pos = 0;
+            for (int j0 = 0; j0 < n; j0 += NT) {
+                const int j = j0 + tid;
+                const bool keep = j < n && __ldcg(S + j) > -INFINITY;
+                int tot;
+                const int incl = block_incl_scan<NT>(keep ? 1 : 0, warp_tot, &tot);
+                if (keep && pos + incl - 1 < T) ps[pos + incl - 1] = j;
+                pos += tot;
+            }
+            kk = pos < kk ? pos : kk;  // a non-finite score is not a candidate
+        } else {
+            radix_select_emit(n, kk, [&](int j) { return order_key(__ldcg(S + j)); }, hist, warp_tot,
+                              &s_bin, &s_above, ps);
+        }
+    }
+    __syncthreads();
+    for (int k = tid; k < T; k += NT) {
+        const int slot = k < kk ? ps[k] : -1;
+        if (slot >= 0 && slot < n) {
+            pg[k] = sel[slot / P];
+            ps[k] = slot % P;
+        } else {
+            pg[k] = -1;
+            ps[k] = -1;
+        }
+    }
+    if (tid == 0) tok_count[bh] = kk;
+    pdl_trigger();
+}
+
+cudaError_t launch_select_tokens(const ekv_cache &c, const float *tscores, const int32_t *sel_idx,
+                                 const int32_t *sel_count, int max_sel, int T, int32_t *tok_page,
+                                 int32_t *tok_pos, int32_t *tok_count, cudaStream_t st)
+{
+    select_tokens_kernel<<<c.batch * c.num_kv_heads, kSelThreads, 0, st>>>(
+        tscores, c.num_kv_heads, c.page_size, c.seq_lens, c.max_pages, sel_idx, sel_count, max_sel,
+        T, tok_page, tok_pos, tok_count);
+    return cudaGetLastError();
+}
+
+}  // namespace ekv

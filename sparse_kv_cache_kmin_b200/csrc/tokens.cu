@@ -1,0 +1,285 @@
+// tokens.cu -- token-level selection inside the selected pages and attention indexed into the
+// paged cache (after the JSSA abstract on ai.info: token-granular selection, one selection per
+// KV head, an indexed attention kernel on the standard GQA cache layout with no gather copy).
+//
+// Step 1 (token_score_kernel): the group score of every candidate token -- the valid tokens of
+// the selected pages -- for its KV head, sum_g scale q_g . k = scale (sum_g q_g) . k, in the
+// full key space (JSSA fits a low-dimensional scoring subspace to data; with no data the
+// subspace is the whole space). Candidate slot i * P + t holds page i of the selection,
+// position t; slots past a page's valid tokens hold -inf.
+// Step 2 (select_tokens_kernel, select.cu): the T best slots, ties to the lower slot.
+// Step 3 (token_attend_kernel): per query head, softmax or exact alpha-entmax over the kept
+// tokens, whose K and V rows are read in place through the page table.
+#include "decode.cuh"
+
+namespace ekv {
+
+// One CTA per (8 selected pages, sequence x KV head). The group query sum Q = sum_g q_g is in
+// shared memory; a warp scores one token row at a time (lane l reads elements l, l + 32, ...).
+template <int DT, int D, int G>
+__global__ void __launch_bounds__(256)
+token_score_kernel(ekv_cache c, const void *__restrict__ q, int H_q, float scale,
+                   const int32_t *__restrict__ sel_idx, const int32_t *__restrict__ sel_count,
+                   int max_sel, float *__restrict__ tscores)
+{
+    constexpr int PPC = 8;
+    __shared__ float qsum[D];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int bh = blockIdx.y, b = bh / c.num_kv_heads, h = bh % c.num_kv_heads;
+    const int P = c.page_size;
+    pdl_wait();
+    int ns = sel_count[bh];
+    ns = ns < 0 ? 0 : (ns > max_sel ? max_sel : ns);
+    const int i0 = blockIdx.x * PPC;
+    if (i0 >= ns) return;
+    int len;
+    const int np = seq_pages(c.seq_lens, b, P, c.max_pages, nullptr, &len);
+    for (int e = tid; e < D; e += 256) {
+        float s = 0.f;
+#pragma unroll
+        for (int g = 0; g < G; ++g) s += load_elem<DT>(q, ((size_t)b * H_q + (size_t)h * G + g) * D + e);
+        qsum[e] = s;
+    }
+    __syncthreads();
+    float *out = tscores + (size_t)bh * max_sel * P;
+    const int i1 = i0 + PPC < ns ? i0 + PPC : ns;
+    for (int r = warp; r < (i1 - i0) * P; r += 8) {
+        const int i = i0 + r / P, t = r % P;
+        const int j = sel_idx[(size_t)bh * max_sel + i];
+        int blk = -1;
+        if (j >= 0 && j < np && j * P + t < len) {
+            blk = c.page_table[(size_t)b * c.max_pages + j];
+            if (blk >= c.num_blocks) blk = -1;
+        }
+        float acc = 0.f;
+        if (blk >= 0) {
+            const size_t row = ((size_t)blk * c.num_kv_heads + h) * P + t;
+            for (int e = lane; e < D; e += 32) acc = fmaf(qsum[e], load_elem<DT>(c.k_cache, row * D + e), acc);
+            acc = warp_sum(acc);
+        }
+        if (lane == 0) out[(size_t)i * P + t] = blk >= 0 ? scale * acc : -INFINITY;
+    }
+    pdl_trigger();
+}
+
+// One CTA per (sequence, query head), the kept tokens' logits in shared memory.
+//   softmax: p = exp(s - max) / sum, stat = log sum exp(s);
+//   entmax:  z = (alpha - 1) s; tau by bisection on f(tau) = sum [z - tau]_+^(1/(alpha-1)) - 1
+//            over [max z - 1, max z] in fp64, then recomputed in closed form over the support
+//            {z > tau} (sparsemax: (sum_S z - 1) / |S|; 1.5-entmax: mean_S - sqrt((1 -
+//            sum_S (z - mean_S)^2) / |S|)); p = [z - tau]_+^(1/(alpha-1)), stat = tau.
+//   out = sum_i p_i v_i, reading only rows with p_i > 0.
+template <int DT, int D, int G>
+__global__ void __launch_bounds__(256)
+token_attend_kernel(ekv_cache c, const void *__restrict__ q, int H_q, float scale, int attn,
+                    const int32_t *__restrict__ tok_page, const int32_t *__restrict__ tok_pos,
+                    const int32_t *__restrict__ tok_count, int T, float *__restrict__ out,
+                    float *__restrict__ stat)
+{
+    extern __shared__ float zs[];   // [T] logits, then weights
+    __shared__ float qs[D];
+    __shared__ double dred[8];
+    __shared__ float fred[8];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int hq = blockIdx.x, b = blockIdx.y, h = hq / G;
+    const int bh = b * c.num_kv_heads + h;
+    const size_t bq = (size_t)b * H_q + hq;
+    const int P = c.page_size;
+    pdl_wait();
+    int n = tok_count[bh];
+    n = n < 0 ? 0 : (n > T ? T : n);
+    if (n == 0) {
+        for (int a = tid; a < D; a += 256) out[bq * D + a] = 0.f;
+        if (tid == 0) stat[bq] = -INFINITY;
+        return;
+    }
+    int len;
+    const int np = seq_pages(c.seq_lens, b, P, c.max_pages, nullptr, &len);
+    for (int e = tid; e < D; e += 256) qs[e] = load_elem<DT>(q, bq * D + e);
+    __syncthreads();
+    const int32_t *pg = tok_page + (size_t)bh * T, *ps = tok_pos + (size_t)bh * T;
+    auto row_of = [&](int i) -> long long {
+        const int j = pg[i], t = ps[i];
+        if (j < 0 || j >= np || t < 0 || t >= P || j * P + t >= len) return -1;
+        const int blk = c.page_table[(size_t)b * c.max_pages + j];
+        if (blk < 0 || blk >= c.num_blocks) return -1;
+        return ((long long)blk * c.num_kv_heads + h) * P + t;
+    };
+    const float alpha = attn == EKV_SOFTMAX ? 1.f : (attn == EKV_ENTMAX15 ? 1.5f : 2.f);
+    for (int i = warp; i < n; i += 8) {
+        const long long row = row_of(i);
+        float acc = 0.f;
+        if (row >= 0) {
+            for (int e = lane; e < D; e += 32) acc = fmaf(qs[e], load_elem<DT>(c.k_cache, (size_t)row * D + e), acc);
+            acc = warp_sum(acc);
+        }
+        if (lane == 0) {
+            if (row < 0) flag(c.dev_status, EKV_DEV_BAD_SEL);
+            zs[i] = row >= 0 ? scale * acc * (attn == EKV_SOFTMAX ? 1.f : alpha - 1.f) : -INFINITY;
+        }
+    }
+    __syncthreads();
+    auto block_max = [&](float v) {
+        v = warp_max(v);
+        if (lane == 0) fred[warp] = v;
+        __syncthreads();
+        float m = fred[0];
+#pragma unroll
+        for (int w = 1; w < 8; ++w) m = fmaxf(m, fred[w]);
+        __syncthreads();
+        return m;
+    };
+    auto block_dsum = [&](double v) {
+        v = warp_sum(v);
+        if (lane == 0) dred[warp] = v;
+        __syncthreads();
+        double s = 0.0;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) s += dred[w];
+        __syncthreads();
+        return s;
+    };
+    float mx = -INFINITY;
+    for (int i = tid; i < n; i += 256) mx = fmaxf(mx, zs[i]);
+    mx = block_max(mx);
+    float st;
+    if (attn == EKV_SOFTMAX) {
+        double l = 0.0;
+        for (int i = tid; i < n; i += 256) {
+            const float p = zs[i] == -INFINITY ? 0.f : expf(zs[i] - mx);
+            zs[i] = p;
+            l += p;
+        }
+        l = block_dsum(l);
+        const float inv = (float)(1.0 / l);
+        for (int i = tid; i < n; i += 256) zs[i] *= inv;
+        st = mx + (float)log(l);
+    } else {
+        const bool sparse = attn == EKV_SPARSEMAX;
+        double lo = (double)mx - 1.0, hi = (double)mx;  // f(lo) >= 0 > f(hi)
+        for (int it = 0; it < 60; ++it) {
+            const double mid = 0.5 * (lo + hi);
+            double f = 0.0;
+            for (int i = tid; i < n; i += 256) {
+                const double r = (double)zs[i] - mid;
+                if (r > 0.0) f += sparse ? r : r * r;
+            }
+            f = block_dsum(f);
+            if (f >= 1.0) lo = mid; else hi = mid;
+        }
+        // closed form over the support {z > lo}
+        double s1 = 0.0, s2 = 0.0, k = 0.0;
+        for (int i = tid; i < n; i += 256) {
+            if ((double)zs[i] > lo) { s1 += zs[i]; s2 += (double)zs[i] * zs[i]; k += 1.0; }
+        }
+        s1 = block_dsum(s1);
+        s2 = block_dsum(s2);
+        k = block_dsum(k);
+        double tau;
+        if (sparse) {
+            tau = (s1 - 1.0) / k;
+        } else {
+            const double mean = s1 / k, ss = s2 - k * mean * mean;
+            const double disc = (1.0 - ss) / k;
+            tau = mean - sqrt(disc > 0.0 ? disc : 0.0);
+        }
+        for (int i = tid; i < n; i += 256) {
+            const double r = (double)zs[i] - tau;
+            zs[i] = r > 0.0 ? (float)(sparse ? r : r * r) : 0.f;
+        }
+        st = (float)tau;
+    }
+    __syncthreads();
+    for (int a = tid; a < D; a += 256) {
+        float acc = 0.f;
+        for (int i = 0; i < n; ++i) {
+            const float p = zs[i];
+            if (p == 0.f) continue;
+            const long long row = row_of(i);
+            if (row >= 0) acc = fmaf(p, load_elem<DT>(c.v_cache, (size_t)row * D + a), acc);
+        }
+        out[bq * D + a] = acc;
+    }
+    if (tid == 0) stat[bq] = st;
+}
+
+template <int DT, int D, int G>
+static cudaError_t launch_tokens_t(const ekv_cache &c, const void *q, int H_q, float scale,
+                                   const int32_t *sel_idx, const int32_t *sel_count, int max_sel,
+                                   float *tscores, cudaStream_t st)
+{
+    const dim3 grid((max_sel + 7) / 8, c.batch * c.num_kv_heads);
+    token_score_kernel<DT, D, G><<<grid, 256, 0, st>>>(c, q, H_q, scale, sel_idx, sel_count, max_sel, tscores);
+    return cudaGetLastError();
+}
+
+template <int DT, int D, int G>
+static cudaError_t launch_attend_t(const ekv_cache &c, const void *q, int H_q, float scale, int attn,
+                                   const int32_t *tok_page, const int32_t *tok_pos,
+                                   const int32_t *tok_count, int T, float *out, float *stat,
+                                   cudaStream_t st)
+{
+    auto k = token_attend_kernel<DT, D, G>;
+    const size_t smem = sizeof(float) * (size_t)T;
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    k<<<dim3(H_q, c.batch), 256, smem, st>>>(c, q, H_q, scale, attn, tok_page, tok_pos, tok_count, T, out, stat);
+    return cudaGetLastError();
+}
+
+#define EKV_TOKEN_DISPATCH(FN, ...)                                                               \
+    do {                                                                                          \
+        const int G = H_q / c.num_kv_heads;                                                       \
+        if (c.dtype == EKV_BF16) {                                                                \
+            if (c.head_dim == 128) {                                                              \
+                switch (G) {                                                                      \
+                case 1: return FN<EKV_BF16, 128, 1>(__VA_ARGS__);                                 \
+                case 2: return FN<EKV_BF16, 128, 2>(__VA_ARGS__);                                 \
+                case 4: return FN<EKV_BF16, 128, 4>(__VA_ARGS__);                                 \
+                default: return FN<EKV_BF16, 128, 8>(__VA_ARGS__);                                \
+                }                                                                                 \
+            }                                                                                     \
+            switch (G) {                                                                          \
+            case 1: return FN<EKV_BF16, 64, 1>(__VA_ARGS__);                                      \
+            case 2: return FN<EKV_BF16, 64, 2>(__VA_ARGS__);                                      \
+            case 4: return FN<EKV_BF16, 64, 4>(__VA_ARGS__);                                      \
+            default: return FN<EKV_BF16, 64, 8>(__VA_ARGS__);                                     \
+            }                                                                                     \
+        }                                                                                         \
+        if (c.head_dim == 128) {                                                                  \
+            switch (G) {                                                                          \
+            case 1: return FN<EKV_F32, 128, 1>(__VA_ARGS__);                                      \
+            case 2: return FN<EKV_F32, 128, 2>(__VA_ARGS__);                                      \
+            case 4: return FN<EKV_F32, 128, 4>(__VA_ARGS__);                                      \
+            default: return FN<EKV_F32, 128, 8>(__VA_ARGS__);                                     \
+            }                                                                                     \
+        }                                                                                         \
+        switch (G) {                                                                              \
+        case 1: return FN<EKV_F32, 64, 1>(__VA_ARGS__);                                           \
+        case 2: return FN<EKV_F32, 64, 2>(__VA_ARGS__);                                           \
+        case 4: return FN<EKV_F32, 64, 4>(__VA_ARGS__);                                           \
+        default: return FN<EKV_F32, 64, 8>(__VA_ARGS__);                                          \
+        }                                                                                         \
+    } while (0)
+
+cudaError_t launch_token_scores(const ekv_cache &c, const void *q, int H_q, float scale,
+                                const int32_t *sel_idx, const int32_t *sel_count, int max_sel,
+                                float *tscores, cudaStream_t st)
+{
+    EKV_TOKEN_DISPATCH(launch_tokens_t, c, q, H_q, scale, sel_idx, sel_count, max_sel, tscores, st);
+}
+
+cudaError_t launch_token_attend(const ekv_cache &c, const void *q, int H_q, float scale, int attn,
+                                const int32_t *tok_page, const int32_t *tok_pos,
+                                const int32_t *tok_count, int T, float *out, float *stat,
+                                cudaStream_t st)
+{
+    EKV_TOKEN_DISPATCH(launch_attend_t, c, q, H_q, scale, attn, tok_page, tok_pos, tok_count, T,
+                       out, stat, st);
+}
+
+#undef EKV_TOKEN_DISPATCH
+
+}  // namespace ekv

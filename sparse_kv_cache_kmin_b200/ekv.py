@@ -282,6 +282,7 @@ def ekv_sparse_decode_noalloc(cache: PagedKVCache, q: torch.Tensor, num_q_heads:
 
 
 def _moment_fn(name, args, res=ctypes.c_int):
+    """An entry point beyond the four calls, its signature set on first use."""
     fn = getattr(load_library(), name)
     if fn.argtypes is None:
         fn.argtypes, fn.restype = args, res
@@ -327,3 +328,39 @@ def ekv_sparse_decode_moment(cache: PagedKVCache, moments: torch.Tensor, q: torc
     _check(fn(ctypes.byref(c), _ptr(moments), _ptr(q), int(num_q_heads), float(scale),
               _ptr(sel_idx), _ptr(sel_count), int(max_sel), _ptr(out), _ptr(stat), _ptr(ws),
               ws.numel() * ws.element_size(), _stream(stream)), "ekv_sparse_decode_moment")
+
+
+def ekv_token_workspace_bytes(cache: PagedKVCache, max_sel: int) -> int:
+    fn = _moment_fn("ekv_token_workspace_bytes", [ctypes.POINTER(EkvCacheStruct), ctypes.c_int32],
+                    ctypes.c_size_t)
+    c = cache.struct()
+    return int(fn(ctypes.byref(c), int(max_sel)))
+
+
+def ekv_select_tokens(cache: PagedKVCache, q: torch.Tensor, num_q_heads: int, scale: float,
+                      sel_idx: torch.Tensor, sel_count: torch.Tensor, max_sel: int, T: int,
+                      tok_page: torch.Tensor, tok_pos: torch.Tensor, tok_count: torch.Tensor,
+                      ws: torch.Tensor, stream=None):
+    """Token-level top-T inside the selected pages, per KV head (see include/ekv.h)."""
+    P, I32, F, U64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float, ctypes.c_size_t
+    fn = _moment_fn("ekv_select_tokens", [ctypes.POINTER(EkvCacheStruct), P, I32, F, P, P, I32,
+                                          I32, P, P, P, P, U64, P])
+    c = cache.struct()
+    _check(fn(ctypes.byref(c), _ptr(q), int(num_q_heads), float(scale), _ptr(sel_idx),
+              _ptr(sel_count), int(max_sel), int(T), _ptr(tok_page), _ptr(tok_pos),
+              _ptr(tok_count), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "ekv_select_tokens")
+
+
+def ekv_sparse_decode_tokens(cache: PagedKVCache, q: torch.Tensor, num_q_heads: int,
+                             scale: float, attn: int, tok_page: torch.Tensor,
+                             tok_pos: torch.Tensor, tok_count: torch.Tensor, T: int,
+                             out: torch.Tensor, stat: torch.Tensor, stream=None):
+    """Attention over the kept tokens, read in place through the page table."""
+    P, I32, F = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float
+    fn = _moment_fn("ekv_sparse_decode_tokens", [ctypes.POINTER(EkvCacheStruct), P, I32, F, I32,
+                                                 P, P, P, I32, P, P, P])
+    c = cache.struct()
+    _check(fn(ctypes.byref(c), _ptr(q), int(num_q_heads), float(scale), int(attn),
+              _ptr(tok_page), _ptr(tok_pos), _ptr(tok_count), int(T), _ptr(out), _ptr(stat),
+              _stream(stream)), "ekv_sparse_decode_tokens")

@@ -180,3 +180,30 @@ def test_moment_entry_points_validation(lib):
     assert lib.ekv_sparse_decode_moment(C.byref(c), P, P, 32, 1.0, P, P, 256, P, P, P, need - 1, None) == 3
     assert lib.ekv_sparse_decode_moment(C.byref(c), P, P, 30, 1.0, P, P, 256, P, P, P, need, None) == 1
     assert lib.ekv_sparse_decode_moment(C.byref(c), P, P, 32, 0.0, P, P, 256, P, P, P, need, None) == 1
+
+
+def test_token_entry_points_validation(lib):
+    from sparse_kv_cache_kmin_b200.ekv import load_library
+    import ctypes as C
+    P = 0x1000
+    lib = load_library()
+    cp = C.POINTER(type(fake_cache()))
+    vp, i32, f32 = C.c_void_p, C.c_int32, C.c_float
+    lib.ekv_token_workspace_bytes.argtypes = [cp, i32]
+    lib.ekv_token_workspace_bytes.restype = C.c_size_t
+    lib.ekv_select_tokens.argtypes = [cp, vp, i32, f32, vp, vp, i32, i32, vp, vp, vp, vp, C.c_size_t, vp]
+    lib.ekv_sparse_decode_tokens.argtypes = [cp, vp, i32, f32, i32, vp, vp, vp, i32, vp, vp, vp]
+    c = fake_cache()
+    need = lib.ekv_token_workspace_bytes(C.byref(c), 256)
+    assert need == 4 * 8 * 256 * 16 * 4  # one fp32 score per candidate slot
+    assert lib.ekv_token_workspace_bytes(C.byref(c), 0) == 0
+    sel = lambda T, ws=need: lib.ekv_select_tokens(C.byref(c), P, 32, 1.0, P, P, 256, T, P, P, P, P, ws, None)
+    assert sel(0) == 1
+    assert sel(32769) == 2
+    assert sel(512, need - 1) == 3
+    dec = lambda attn, T: lib.ekv_sparse_decode_tokens(C.byref(c), P, 32, 1.0, attn, P, P, P, T, P, P, None)
+    assert dec(7, 64) == 2
+    assert dec(1, 0) == 1
+    assert dec(1, 32769) == 2
+    c2 = fake_cache(v_cache=None)
+    assert lib.ekv_sparse_decode_tokens(C.byref(c2), P, 32, 1.0, 1, P, P, P, 64, P, P, None) == 1
