@@ -142,6 +142,11 @@ token_attend_kernel(ekv_cache c, const void *__restrict__ q, int H_q, float scal
     float mx = -INFINITY;
     for (int i = tid; i < n; i += 256) mx = fmaxf(mx, zs[i]);
     mx = block_max(mx);
+    if (mx == -INFINITY) {  // every listed token was out of range (flagged above)
+        for (int a = tid; a < D; a += 256) out[bq * D + a] = 0.f;
+        if (tid == 0) stat[bq] = -INFINITY;
+        return;
+    }
     float st;
     if (attn == EKV_SOFTMAX) {
         double l = 0.0;
