@@ -161,7 +161,7 @@ token_attend_kernel(ekv_cache c, const void *__restrict__ q, int H_q, float scal
         st = mx + (float)log(l);
     } else {
         const bool sparse = attn == EKV_SPARSEMAX;
-        double lo = (double)mx - 1.0, hi = (double)mx;  // f(lo) >= 0 > f(hi)
+        double lo = (double)mx - 1.0, hi = (double)mx;  // the sum is >= 1 at lo and 0 at hi
         for (int it = 0; it < 60; ++it) {
             const double mid = 0.5 * (lo + hi);
             double f = 0.0;
