@@ -54,6 +54,11 @@ MUTANTS = {
                                          "        blk[i] = pt_row[j];\n        pos[i] = 0;"),
     "moment_sums_transposed": ("                    S[(size_t)a * d + c] += va * elem(",
                                "                    S[(size_t)c * d + a] += va * elem("),
+    "bound_drops_scale": ("            acc *= scale;\n", "            (void)scale;\n"),
+    "gauss_mean_drops_scale": ("m[(size_t)g * n_pages + j] = scale * a;", "m[(size_t)g * n_pages + j] = a;"),
+    "gauss_variance_scale_not_squared": ("v[(size_t)g * n_pages + j] = scale * scale * b;",
+                                         "v[(size_t)g * n_pages + j] = scale * b;"),
+    "topk_keeps_one_page_too_many": ("int cnt = k < n ? k : n;", "int cnt = k < n ? k + 1 : n;"),
     "attention_reads_invalid_tokens": (
         "n_tok += seq_len - j * P < P ? seq_len - j * P : P;", "n_tok += P;"),
 }

@@ -176,9 +176,11 @@ def test_bound_sign_split_closed_form():
     np.testing.assert_allclose(ub[0], kmin @ -qp[0], rtol=1e-14)
 
 
-def test_gauss_stats_are_mean_and_variance_of_the_scores():
-    # m = q.mean and v = sum_c q_c^2 var_c are the exact mean and variance of q.k over a
-    # page whose coordinates are independent: check on an outer-product page where they are.
+@pytest.mark.parametrize("scale", [1.0, 0.37])
+def test_gauss_stats_are_mean_and_variance_of_the_scores(scale):
+    # m = scale q.mean and v = scale^2 sum_c q_c^2 var_c are the exact mean and variance of the
+    # scores scale q.k over a page whose coordinates are independent: check on an outer-product
+    # page where they are.
     rng = np.random.default_rng(6)
     d = 3
     vals = [rng.standard_normal(2) for _ in range(d)]
@@ -187,8 +189,8 @@ def test_gauss_stats_are_mean_and_variance_of_the_scores():
     k = page_cache_from_keys(keys.astype(np.float32))
     _, _, mean, var = O.page_meta_head(k, [0], len(keys), 0)
     q = rng.standard_normal((2, d))
-    m, v = O.gauss_stats_head(q, 1.0, mean, var)
-    s = q @ k[0, 0].astype(np.float64).T
+    m, v = O.gauss_stats_head(q, scale, mean, var)
+    s = scale * (q @ k[0, 0].astype(np.float64).T)
     np.testing.assert_allclose(m[:, 0], s.mean(1), atol=1e-13)
     np.testing.assert_allclose(v[:, 0], s.var(1), atol=1e-13)
 
