@@ -59,6 +59,23 @@ MUTANTS = {
     "gauss_variance_scale_not_squared": ("v[(size_t)g * n_pages + j] = scale * scale * b;",
                                          "v[(size_t)g * n_pages + j] = scale * b;"),
     "topk_keeps_one_page_too_many": ("int cnt = k < n ? k : n;", "int cnt = k < n ? k + 1 : n;"),
+    "meta_max_takes_min": ("                if (x > hi) hi = x;", "                if (x < hi) hi = x;"),
+    "meta_mean_divides_by_page_size": ("            double mu = sum / n;", "            double mu = sum / P;"),
+    "gauss_F_ignores_token_counts": ("F += (double)cnt[j] * ora_trunc_moment(a, b, tau, alpha);",
+                                     "F += ora_trunc_moment(a, b, tau, alpha); (void)cnt;"),
+    "gauss_F_drops_alpha_factor_on_b": ("        double b = (alpha - 1.0) * sqrt(v[j] > 0.0 ? v[j] : 0.0);\n        F +=",
+                                        "        double b = sqrt(v[j] > 0.0 ? v[j] : 0.0);\n        F +="),
+    "gauss_tau_bisects_the_wrong_way": ("            lo = mid;\n        else\n            hi = mid;",
+                                        "            hi = mid;\n        else\n            lo = mid;"),
+    "gauss_select_needs_every_query": (
+        "        int keep = 0;\n        for (int g = 0; g < G; ++g)\n            if ((alpha - 1.0) * ub[(size_t)g * n_pages + j] > tau_hat[g] - delta)\n                keep = 1;",
+        "        int keep = 1;\n        for (int g = 0; g < G; ++g)\n            if (!((alpha - 1.0) * ub[(size_t)g * n_pages + j] > tau_hat[g] - delta))\n                keep = 0;"),
+    "gauss_select_margin_sign": ("ub[(size_t)g * n_pages + j] > tau_hat[g] - delta)\n                keep = 1;",
+                                 "ub[(size_t)g * n_pages + j] > tau_hat[g] + delta)\n                keep = 1;"),
+    "entmax15_weights_not_squared": ("p[i] = r > 0.0 ? (alpha == 2.0 ? r : r * r) : 0.0;",
+                                     "p[i] = r > 0.0 ? r : 0.0;"),
+    "softmax_not_normalised": ("            for (int i = 0; i < n_tok; ++i)\n                p[i] /= l;\n",
+                               "            (void)0;\n"),
     "attention_reads_invalid_tokens": (
         "n_tok += seq_len - j * P < P ? seq_len - j * P : P;", "n_tok += P;"),
 }
