@@ -2,21 +2,28 @@
 """Benchmark of one sparse decode step (page scores -> page selection -> sparse attention,
 plus the page-metadata refresh when the workload appends a page) on B200.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload needle128k] [--impl ours|reference]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload needle128k]
+                  [--variant pages|tokens|moment] [--impl ours|reference]
 
 One process per GPU (torchrun for N > 1). Every rank decodes its own seeded batch (weak
 scaling, no collective on the data path); the timed region is bracketed by a barrier and a
 device synchronise, and the whole-job rate uses the slowest rank's device time. L2 is flushed
 (a 256 MiB write, outside the timed events) before every timed step. Rank 0 prints one JSON
-line. `--impl reference` times the CPU oracle on a bounded sample of the same workload.
+line. `--impl reference` times the CPU oracle on the same workload.
+
+Variants (what one step runs after scoring and top-k page selection):
+  pages    exact attention over the selected pages (the method's decode)
+  tokens   the T best tokens of the selected pages per KV head, then attention over those
+  moment   softmax over the selected pages corrected for the skipped ones from running moments
 """
 from __future__ import annotations
 
 import argparse
+import concurrent.futures as cf
 import hashlib
 import json
-import math
 import os
+import platform
 import statistics
 import subprocess
 import sys
@@ -32,6 +39,7 @@ METRIC = "sparse decode steps/s at 128K ctx; achieved HBM GB/s vs ~8 TB/s peak"
 ATTN_NAME = {0: "softmax", 1: "entmax1.5", 2: "sparsemax"}
 POLICY_NAME = {0: "topk", 1: "gauss", 2: "gauss_max"}
 FALLBACK_HBM_GBS = 6650.0
+TARGET_FRAC = 0.70  # the 128K step's required bytes at >= 70% of the HBM roofline
 
 
 def parse():
@@ -41,6 +49,10 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="needle128k",
                     choices=["tiny", "gqa32k", "needle128k", "gauss", "long1m"])
+    ap.add_argument("--variant", default="pages", choices=["pages", "tokens", "moment"])
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="tokens kept per KV head by the tokens variant (default: a quarter of "
+                         "the selected pages' tokens)")
     ap.add_argument("--attn", type=int, default=None, help="attention mode (default: workload's first)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-sample-seconds", type=float, default=12.0)
@@ -55,58 +67,108 @@ def parse():
     return ap.parse_args()
 
 
+def setup_workload(args, make, rank, device):
+    from sparse_kv_cache_kmin_b200 import replicas
+    kw = {"B": args.batch} if args.batch else {}
+    wl = make(args.workload, device=device, seed=replicas.workload_seed(args.workload, rank), **kw)
+    attn = wl.attn_modes[0] if args.attn is None else args.attn
+    if args.variant == "moment":
+        attn = 0  # the moment correction is a softmax remedy
+    if args.policy is not None:
+        wl.policy = {v: k for k, v in POLICY_NAME.items()}[args.policy]
+        if wl.policy == 0 and not wl.topk:
+            raise SystemExit("--policy topk needs a workload with a top-k budget")
+    if args.variant != "pages" and wl.policy != 0:
+        raise SystemExit("the tokens and moment variants run after top-k page selection")
+    T = None
+    if args.variant == "tokens":
+        T = args.tokens or max(1, wl.topk * wl.page_size // 4)
+    return wl, attn, T
+
+
+def config_of(wl, attn, variant, T, world):
+    """The workload a line measures; the same dict in both arms."""
+    cfg = {"workload": wl.name, "batch_per_gpu": wl.batch, "ctx": int(wl.seq_lens.max()),
+           "q_heads": wl.num_q_heads, "kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim,
+           "page": wl.page_size,
+           "policy": "top-k %d" % wl.topk if wl.policy == 0 else "%s delta %g" % (POLICY_NAME[wl.policy], wl.delta),
+           "attn": ATTN_NAME[attn], "variant": variant,
+           "l2": "flushed before every step (256 MiB write, outside the timed events)",
+           "parallelism": "replicas x%d, no collective" % world}
+    if T is not None:
+        cfg["tokens_per_kv_head"] = T
+    return cfg
+
+
 # ----------------------------------------------------------------------------- byte accounting
-def step_bytes(wl, dec, attn):
+def selected_tokens(wl, dec):
+    P = wl.page_size
+    lens = wl.seq_lens.long().cpu()
+    sel = dec.sel_idx.long().cpu()
+    cnt = dec.sel_count.long().cpu()
+    n = 0
+    for b in range(wl.batch):
+        L = int(lens[b])
+        for h in range(wl.num_kv_heads):
+            j = sel[b, h, :int(cnt[b, h])]
+            n += int(torch.clamp(L - j * P, 0, P).sum())
+    return n
+
+
+def step_bytes(wl, dec, attn, variant, extra):
     """Required bytes of one step and of each call (what the computation must touch once).
 
-    metadata rows of every existing page (bbox, plus moments for the Gaussian policy), the
-    page-table rows, q, the K rows of the selected pages' valid tokens, the V rows that carry
-    weight (softmax: all selected tokens; entmax: the tokens in the support of some query of
-    the group -- the rest provably have zero weight and are not read), the outputs; the
-    appended page when the workload appends one."""
+    Every variant: the metadata rows of every existing page (bbox, plus moments for the
+    Gaussian policy), the page-table rows, q and the outputs; the appended page when the
+    workload appends one. Then
+      pages    the K rows of the selected pages' valid tokens and the V rows that carry weight
+               (softmax: all of them; entmax: the tokens in the support of some query of the
+               group -- the rest provably have zero weight and are not read);
+      tokens   the K rows of the selected pages' valid tokens (token scores) and the K and V
+               rows of the kept tokens;
+      moment   the K and V rows of the selected pages' valid tokens and the running-moment
+               records."""
     P, d, H = wl.page_size, wl.head_dim, wl.num_kv_heads
     esz = wl.k_cache.element_size()
     lens = wl.seq_lens.long().cpu()
-    n_pages = (lens + P - 1) // P
-    total_pages = int(n_pages.sum())
+    total_pages = int(((lens + P - 1) // P).sum())
     meta_row = 2 * d * esz + (2 * d * 4 if wl.policy != 0 else 0)
     meta = total_pages * H * meta_row
     ptab = total_pages * 4
     qb = wl.q.numel() * wl.q.element_size()
     scores_out = total_pages * H * 4 if wl.policy == 0 else total_pages * wl.num_q_heads * 12
-    # selected tokens (valid ones) from the device selection
-    sel = dec.sel_idx.long().cpu()
-    cnt = dec.sel_count.long().cpu()
-    sel_tok = 0
-    for b in range(wl.batch):
-        L = int(lens[b])
-        for h in range(H):
-            j = sel[b, h, :int(cnt[b, h])]
-            sel_tok += int(torch.clamp(L - j * P, 0, P).sum())
-    k_bytes = sel_tok * d * esz
-    if attn == 0:
-        v_rows = sel_tok
-    else:
-        v_rows = support_rows(wl, dec, attn)
-    v_bytes = v_rows * d * esz
-    out_b = dec.out.numel() * 4 + dec.stat.numel() * 4
+    sel_tok = selected_tokens(wl, dec)
+    row = d * esz
+    out_b = wl.batch * wl.num_q_heads * (d + 1) * 4
     append_b = 0
     if wl.append is not None:
         append_b = wl.batch * H * wl.append[1] * d * esz + wl.batch * H * meta_row
-    return {
-        "score": meta + ptab + qb + scores_out,
-        "select": scores_out + dec.sel_idx.numel() * 4,
-        "decode": k_bytes + v_bytes + qb + out_b + ptab,
-        "required_step": meta + ptab + qb + k_bytes + v_bytes + out_b + append_b,
-        "required_step_all_v": meta + ptab + qb + 2 * k_bytes + out_b + append_b,
-        "selected_tokens": sel_tok, "support_rows": v_rows, "meta_bytes": meta,
-    }
+    by = {"score": meta + ptab + qb + scores_out, "select": scores_out + dec.sel_idx.numel() * 4,
+          "selected_tokens": sel_tok, "meta_bytes": meta}
+    if variant == "pages":
+        v_rows = sel_tok if attn == 0 else support_rows(wl, dec, attn)
+        by["decode"] = sel_tok * row + v_rows * row + qb + out_b + ptab
+        body, body_all_v = sel_tok * row + v_rows * row, 2 * sel_tok * row
+        by["support_rows"] = v_rows
+    elif variant == "tokens":
+        kept = int(extra["tok_count"].long().sum())
+        by["select_tokens"] = sel_tok * row + qb + kept * 8
+        by["decode_tokens"] = 2 * kept * row + qb + out_b + kept * 8
+        body = body_all_v = sel_tok * row + 2 * kept * row
+        by["kept_tokens"] = kept
+    else:
+        mom = extra["moments"].numel() * 4
+        by["decode_moment"] = 2 * sel_tok * row + mom + qb + out_b + ptab
+        body = body_all_v = 2 * sel_tok * row + mom
+    by["required_step"] = meta + ptab + qb + body + out_b + append_b
+    by["required_step_all_v"] = meta + ptab + qb + body_all_v + out_b + append_b
+    return by
 
 
 def support_rows(wl, dec, attn):
     """V rows with non-zero weight for some query of the group: z > tau, recomputed on the
     device from the stored threshold (stat) with torch -- accounting only."""
-    P, d, H = wl.page_size, wl.head_dim, wl.num_kv_heads
+    P, H = wl.page_size, wl.num_kv_heads
     G = wl.num_q_heads // H
     alpha = 1.5 if attn == 1 else 2.0
     rows = 0
@@ -218,47 +280,199 @@ def ncu_traffic(kernel_file, summary_name, units):
 
 
 # ----------------------------------------------------------------------------- oracle timing
-def oracle_sample(wl, attn, budget_s, max_heads=None):
-    """Time the CPU oracle's decode step on (sequence, KV head) problems of the workload until
-    `budget_s` of CPU time is spent; returns (seconds per full step, description)."""
-    import numpy as np
-    import oracle as O
-    sys.path.insert(0, os.path.join(ROOT, "tests"))
-    from parity_utils import HostCopy
-    H = wl.num_kv_heads
-    G = wl.num_q_heads // H
-    mode = {0: O.SOFTMAX, 1: O.ENTMAX15, 2: O.SPARSEMAX}[attn]
-    order = [(b, h) for b in range(wl.batch) for h in range(H)]
-    rng = np.random.default_rng(0)
-    rng.shuffle(order)
-    if max_heads:
-        order = order[:max_heads]
-    spent, done, hcs = 0.0, 0, {}
-    for b, h in order:
-        hc = hcs.get(b) or HostCopy(wl, b)
-        hcs = {b: hc}
-        meta = O.page_meta_head(hc.k, hc.pt, hc.L, h)  # built at prefill, not part of a step
-        t0 = time.perf_counter()
-        O.decode_step_head(hc.k, hc.v, hc.pt, hc.L, h, hc.q[h], wl.scale, mode,
-                           POLICY_NAME[wl.policy], wl.topk, wl.alpha, wl.delta, meta=meta)
+def cpu_model():
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return platform.processor() or "unknown"
+
+
+class OracleStep:
+    """The CPU oracle's decode step, one (sequence, KV head) problem at a time, on host copies
+    of the workload (taken once, outside every timed region). Problems are independent, and
+    the oracle's C routines release the GIL, so a thread pool runs them on all host cores."""
+
+    def __init__(self, wl, attn, variant, T):
+        import numpy as np
+        import oracle as O
+        sys.path.insert(0, os.path.join(ROOT, "tests"))
+        from parity_utils import HostCopy
+        self.O, self.np = O, np
+        self.wl, self.variant, self.T = wl, variant, T
+        self.mode = {0: O.SOFTMAX, 1: O.ENTMAX15, 2: O.SPARSEMAX}[attn]
+        self.H = wl.num_kv_heads
+        self.problems = [(b, h) for b in range(wl.batch) for h in range(self.H)]
+        self.hc = {b: HostCopy(wl, b) for b in range(wl.batch)}
+        # page metadata is built at prefill, not in a step
+        self.meta = {(b, h): O.page_meta_head(self.hc[b].k, self.hc[b].pt, self.hc[b].L, h)
+                     for (b, h) in self.problems}
+
+    def run(self, b, h):
+        O, wl, hc = self.O, self.wl, self.hc[b]
+        meta = self.meta[(b, h)]
+        q = hc.q[h]
+        if self.variant == "pages":
+            O.decode_step_head(hc.k, hc.v, hc.pt, hc.L, h, q, wl.scale, self.mode,
+                               POLICY_NAME[wl.policy], wl.topk, wl.alpha, wl.delta, meta=meta)
+        else:
+            _, S = O.score_head(q, wl.scale, meta[0], meta[1])
+            sel = O.topk(S, wl.topk)
+            if self.variant == "tokens":
+                pages, pos = O.token_topk_head(hc.k, hc.pt, hc.L, h, q, wl.scale, sel, self.T)
+                O.attend_tokens_head(hc.k, hc.v, hc.pt, hc.L, h, q, wl.scale, self.mode, pages, pos)
+            else:
+                O.moment_corrected_head(hc.k, hc.v, hc.pt, hc.L, h, q, wl.scale, sel)
         if wl.append is not None:  # the step also rebuilds the appended page's metadata
-            O.page_meta_head(hc.k[-1:], np.zeros(1, np.int32), hc.L - (hc.np - 1) * wl.page_size, h)
-        spent += time.perf_counter() - t0
-        done += 1
-        if spent >= budget_s:
-            break
-    per_step = spent / done * len([(b, h) for b in range(wl.batch) for h in range(H)])
-    desc = ("%d of %d (sequence, KV head) decode problems (score all pages, select, attend), "
-            "timed single-threaded and scaled to the full step" % (done, wl.batch * H))
-    return per_step, desc
+            O.page_meta_head(hc.k[-1:], self.np.zeros(1, self.np.int32),
+                             hc.L - (hc.np - 1) * wl.page_size, h)
+
+    def single_thread(self, budget_s, seed=0):
+        """Seconds per full step, single-threaded, from as many problems as `budget_s` allows."""
+        order = list(self.problems)
+        self.np.random.default_rng(seed).shuffle(order)
+        spent, done = 0.0, 0
+        for b, h in order:
+            t0 = time.perf_counter()
+            self.run(b, h)
+            spent += time.perf_counter() - t0
+            done += 1
+            if spent >= budget_s:
+                break
+        return spent / done * len(self.problems), done
+
+    def all_cores(self, threads, budget_s, per_problem_s):
+        """Seconds per full step with every problem on a pool of `threads` threads (wall time);
+        when the whole step would overrun `budget_s`, a whole number of rounds of `threads`
+        problems is timed and scaled."""
+        n = len(self.problems)
+        rounds_fit = max(1, int(budget_s / max(per_problem_s, 1e-9)))
+        m = min(n, threads * rounds_fit)
+        work = self.problems[:m]
+        with cf.ThreadPoolExecutor(max_workers=threads) as ex:
+            t0 = time.perf_counter()
+            list(ex.map(lambda p: self.run(*p), work))
+            wall = time.perf_counter() - t0
+        return wall * n / m, m
 
 
+def cpu_baseline(wl, attn, variant, T, budget_s):
+    st = OracleStep(wl, attn, variant, T)
+    n = len(st.problems)
+    single, done1 = st.single_thread(budget_s / 2)
+    threads = os.cpu_count() or 1
+    per_problem = single / n
+    multi, done_m = st.all_cores(threads, budget_s / 2, per_problem)
+    return {"value": 1.0 / multi, "unit": "steps/s", "cores": threads, "kind": "oracle",
+            "cpu_model": cpu_model(), "nproc": threads,
+            "sample": "%d of %d (sequence, KV head) decode problems of the step on a pool of %d "
+                      "threads (the oracle's C routines release the GIL), wall time scaled to "
+                      "the full step" % (done_m, n, threads),
+            "single_thread": {"value": 1.0 / single, "unit": "steps/s", "cores": 1,
+                              "sample": "%d of %d problems, scaled to the full step" % (done1, n)}}
 
-# ----------------------------------------------------------------------------- full-cache decode
+
+# ----------------------------------------------------------------------------- the step on the GPU
+class Step:
+    """The public calls of one decode step of a variant, as (name, fn) pairs, with the buffers
+    they write. Every call goes through the C ABI binding; nothing here computes."""
+
+    def __init__(self, ekv, SparseDecoder, cache, wl, attn, variant, T):
+        self.wl, self.variant, self.T = wl, variant, T
+        dev = wl.k_cache.device
+        B, H = wl.batch, wl.num_kv_heads
+        self.dec = dec = SparseDecoder(cache, wl.num_q_heads, wl.policy, attn, topk=wl.topk,
+                                       alpha=wl.alpha, delta=wl.delta, scale=wl.scale)
+        self.extra = {}
+        calls = []
+        if wl.append is not None:
+            ap_start = torch.full((B,), wl.append[0], dtype=torch.int32, device=dev)
+            ap_count = torch.full((B,), wl.append[1], dtype=torch.int32, device=dev)
+            calls.append(("meta", lambda: ekv.ekv_page_meta_update(cache, ap_start, ap_count,
+                                                                   wl.append[1])))
+        q = wl.q
+        calls.append(("score", lambda: ekv.ekv_score_pages(cache, q, wl.num_q_heads, wl.scale,
+                                                           wl.policy, dec.scores)))
+        calls.append(("select", lambda: ekv.ekv_select_pages(
+            cache, wl.num_q_heads, wl.policy, wl.topk, wl.alpha, wl.delta, dec.scores,
+            dec.sel_idx, dec.sel_count, dec.max_sel, dec.tau_hat)))
+        self.out, self.stat = dec.out, dec.stat
+        if variant == "pages":
+            calls.append(("decode", lambda: ekv.ekv_sparse_decode(
+                cache, q, wl.num_q_heads, wl.scale, attn, dec.sel_idx, dec.sel_count,
+                dec.max_sel, dec.out, dec.stat, dec.ws)))
+            self.kernels = {"meta": 1, "score": 1, "select": 1, "decode": 2}
+        elif variant == "tokens":
+            tws = torch.empty(ekv.ekv_token_workspace_bytes(cache, dec.max_sel), dtype=torch.uint8,
+                              device=dev)
+            tp = torch.empty((B, H, T), dtype=torch.int32, device=dev)
+            tt = torch.empty_like(tp)
+            tc = torch.empty((B, H), dtype=torch.int32, device=dev)
+            self.extra.update(tok_page=tp, tok_pos=tt, tok_count=tc)
+            calls.append(("select_tokens", lambda: ekv.ekv_select_tokens(
+                cache, q, wl.num_q_heads, wl.scale, dec.sel_idx, dec.sel_count, dec.max_sel, T,
+                tp, tt, tc, tws)))
+            calls.append(("decode_tokens", lambda: ekv.ekv_sparse_decode_tokens(
+                cache, q, wl.num_q_heads, wl.scale, attn, tp, tt, tc, T, dec.out, dec.stat)))
+            self.kernels = {"score": 1, "select": 1, "select_tokens": 2, "decode_tokens": 1}
+        else:
+            moments = torch.zeros(ekv.ekv_moment_bytes(cache) // 4, dtype=torch.float32, device=dev)
+            ekv.ekv_moment_update(cache, moments, torch.zeros(B, dtype=torch.int32, device=dev),
+                                  wl.seq_lens, int(wl.seq_lens.max()))
+            mws = torch.empty(ekv.ekv_moment_decode_workspace_bytes(cache, wl.num_q_heads,
+                                                                    dec.max_sel),
+                              dtype=torch.uint8, device=dev)
+            self.extra.update(moments=moments)
+            calls.append(("decode_moment", lambda: ekv.ekv_sparse_decode_moment(
+                cache, moments, q, wl.num_q_heads, wl.scale, dec.sel_idx, dec.sel_count,
+                dec.max_sel, dec.out, dec.stat, mws)))
+            self.kernels = {"score": 1, "select": 1, "decode_moment": 4}
+        self.calls = calls
+
+    def launches(self):
+        return sum(self.kernels.get(name, 1) for name, _ in self.calls)
+
+    def run(self):
+        for _, fn in self.calls:
+            fn()
+
+    def graph(self):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            self.run()
+        return g
+
+    def graph_with_events(self):
+        """The same calls with an event node around each (per-call durations)."""
+        ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(self.calls) + 1)]
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            ev[0].record()
+            for i, (_, fn) in enumerate(self.calls):
+                fn()
+                ev[i + 1].record()
+        return g, ev
+
+    def graph_host(self, q_host, out_host, stat_host, host_pre=None):
+        """A whole host-to-host step: the query copied in from pinned host memory, the calls,
+        the outputs copied back to pinned host buffers."""
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            if host_pre is not None:
+                host_pre()
+            self.wl.q.copy_(q_host, non_blocking=True)
+            self.run()
+            out_host.copy_(self.out, non_blocking=True)
+            stat_host.copy_(self.stat, non_blocking=True)
+        return g
+
+
 def full_cache_time(ekv, cache, wl, attn, steps, flush, stream):
     """The same attention over every page of every sequence (no scoring, no selection): one
     ekv_sparse_decode call with the identity selection, captured in a graph and timed like the
-    sparse step. Returns ms per step."""
+    sparse step. Returns (ms per step, out, stat)."""
     B, H, P = wl.batch, wl.num_kv_heads, wl.page_size
     dev = wl.k_cache.device
     n_pages = ((wl.seq_lens.long() + P - 1) // P).to(torch.int32)
@@ -291,49 +505,34 @@ def full_cache_time(ekv, cache, wl, attn, steps, flush, stream):
         ev[i][1].record(stream)
     torch.cuda.synchronize()
     del g
-    return statistics.mean(a.elapsed_time(b) for a, b in ev), out, stat
+    return statistics.median(a.elapsed_time(b) for a, b in ev), out, stat
 
 
-def selection_quality(wl, dec, attn, stat_full):
-    """How much of the full-cache attention the selection keeps, per query: the dropped mass
-    delta = sum of full-cache weights on tokens outside the selected pages (the quantity of the
-    2 B delta error bound) and, for entmax, the recall of the full-cache support. Computed with
-    torch on the GPU from the cache and the full-cache stat, outside every timed region."""
-    P, H = wl.page_size, wl.num_kv_heads
-    G = wl.num_q_heads // H
-    alpha = {1: 1.5, 2: 2.0}.get(attn)
-    deltas, recalls = [], []
-    for b in range(wl.batch):
-        L = int(wl.seq_lens[b])
-        n = (L + P - 1) // P
-        blk = wl.page_table[b, :n].long()
-        valid = (torch.arange(n, device=blk.device)[:, None] * P
-                 + torch.arange(P, device=blk.device)[None, :]) < L
-        for h in range(H):
-            kk = wl.k_cache[blk, h].float()                          # [n, P, d]
-            q = wl.q[b, h * G:(h + 1) * G].float()                   # [G, d]
-            s = wl.scale * torch.einsum("npd,gd->gnp", kk, q)
-            st = stat_full[b, h * G:(h + 1) * G].float()[:, None, None]
-            if alpha is None:
-                p = torch.exp(s - st)
-            else:
-                p = torch.clamp((alpha - 1.0) * s - st, min=0.0) ** (1.0 / (alpha - 1.0))
-            p = p * valid
-            kept = torch.zeros(n, dtype=torch.bool, device=p.device)
-            cnt = int(dec.sel_count[b, h])
-            kept[dec.sel_idx[b, h, :cnt].long()] = True
-            deltas += (p * (~kept)[None, :, None]).sum((1, 2)).tolist()
-            if alpha is not None:
-                sup = p > 0
-                recalls += ((sup & kept[None, :, None]).sum((1, 2)).float()
-                            / sup.sum((1, 2)).clamp(min=1).float()).tolist()
-    out = {"dropped_mass_mean": statistics.mean(deltas), "dropped_mass_max": max(deltas),
+def selection_quality(ekv, cache, wl, dec, attn, stat_full):
+    """How much of the full-cache attention the page selection keeps, per query, from the
+    library's ekv_selection_quality kernel (outside every timed region): the dropped mass delta
+    (the quantity of the 2 B delta error bound) and, for entmax, the recall of the full-cache
+    support."""
+    dev = wl.k_cache.device
+    dropped = torch.empty((wl.batch, wl.num_q_heads), dtype=torch.float64, device=dev)
+    support = torch.empty((wl.batch, wl.num_q_heads, 2), dtype=torch.int32, device=dev)
+    ekv.ekv_selection_quality(cache, wl.q, wl.num_q_heads, wl.scale, attn, stat_full, dec.sel_idx,
+                              dec.sel_count, dec.max_sel, dropped, support)
+    torch.cuda.synchronize()
+    dl = dropped.flatten().tolist()
+    P = wl.page_size
+    out = {"dropped_mass_mean": statistics.mean(dl), "dropped_mass_max": max(dl),
            "kept_pages_mean": float(dec.sel_count.float().mean()),
-           "pages_mean": float(((wl.seq_lens.float() + P - 1) // P).mean())}
-    if recalls:
-        out["support_recall_mean"] = statistics.mean(recalls)
-        out["support_recall_min"] = min(recalls)
+           "pages_mean": float(((wl.seq_lens.float() + P - 1) // P).mean()),
+           "how": "ekv_selection_quality on the full-cache stat of this GPU"}
+    if attn != 0:
+        sup = support.double()
+        rec = (sup[..., 1] / sup[..., 0].clamp(min=1)).flatten().tolist()
+        out["support_recall_mean"] = statistics.mean(rec)
+        out["support_recall_min"] = min(rec)
+        out["support_size_mean"] = float(sup[..., 0].mean())
     return out
+
 
 # ----------------------------------------------------------------------------- main
 def main():
@@ -346,7 +545,6 @@ def main():
     if args.impl == "reference":
         return reference_arm(args, rank, world, make)
 
-    import sparse_kv_cache_kmin_b200 as ekvpkg
     from sparse_kv_cache_kmin_b200 import ekv
     from sparse_kv_cache_kmin_b200.decoder import SparseDecoder
 
@@ -360,13 +558,7 @@ def main():
                                 device_id=dev)
         pg = dist
 
-    kw = {"B": args.batch} if args.batch else {}
-    wl = make(args.workload, device=dev, seed=replicas.workload_seed(args.workload, rank), **kw)
-    attn = wl.attn_modes[0] if args.attn is None else args.attn
-    if args.policy is not None:
-        wl.policy = {v: k for k, v in POLICY_NAME.items()}[args.policy]
-        if wl.policy == 0 and not wl.topk:
-            raise SystemExit("--policy topk needs a workload with a top-k budget")
+    wl, attn, T = setup_workload(args, make, rank, dev)
     nb, H, P, d = wl.k_cache.shape
     cache = ekv.PagedKVCache(
         k_cache=wl.k_cache, v_cache=wl.v_cache,
@@ -377,49 +569,21 @@ def main():
     B = wl.batch
     ekv.ekv_page_meta_update(cache, torch.zeros(B, dtype=torch.int32, device=dev), wl.seq_lens,
                              int(wl.seq_lens.max()))
-    dec = SparseDecoder(cache, wl.num_q_heads, wl.policy, attn, topk=wl.topk, alpha=wl.alpha,
-                        delta=wl.delta, scale=wl.scale)
-    if wl.append is not None:
-        ap_start = torch.full((B,), wl.append[0], dtype=torch.int32, device=dev)
-        ap_count = torch.full((B,), wl.append[1], dtype=torch.int32, device=dev)
+    step = Step(ekv, SparseDecoder, cache, wl, attn, args.variant, T)
+    dec = step.dec
     stream = torch.cuda.current_stream()
-
-    def step(q):
-        if wl.append is not None:
-            ekv.ekv_page_meta_update(cache, ap_start, ap_count, wl.append[1])
-        return dec.step(q)
-
-    launches_per_step = 4 + (1 if wl.append is not None else 0)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-    pre = None
-    if wl.append is not None:
-        def pre():
-            ekv.ekv_page_meta_update(cache, ap_start, ap_count, wl.append[1])
 
     # eager steps first: one-time set-up (kernel attributes, occupancy queries) stays outside
     # the graph captures
     for _ in range(2):
         flush.fill_(1)
-        step(wl.q)
+        step.run()
     torch.cuda.synchronize()
-    # graph A: the step as one launch (the timed loop); graph B: the same calls with an
-    # event node between them (per-call durations)
-    graph = dec.capture(wl.q, pre_step=pre)
-    evb = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(5)]
-    graph_b = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph_b):
-        evb[0].record()
-        if pre is not None:
-            pre()
-        evb[1].record()
-        ekv.ekv_score_pages(cache, wl.q, wl.num_q_heads, wl.scale, wl.policy, dec.scores)
-        evb[2].record()
-        ekv.ekv_select_pages(cache, wl.num_q_heads, wl.policy, wl.topk, wl.alpha, wl.delta,
-                             dec.scores, dec.sel_idx, dec.sel_count, dec.max_sel, dec.tau_hat)
-        evb[3].record()
-        ekv.ekv_sparse_decode(cache, wl.q, wl.num_q_heads, wl.scale, attn, dec.sel_idx,
-                              dec.sel_count, dec.max_sel, dec.out, dec.stat, dec.ws)
-        evb[4].record()
+    # graph A: the step as one launch (the timed loop); graph B: the same calls with an event
+    # node between them (per-call durations)
+    graph = step.graph()
+    graph_b, evb = step.graph_with_events()
 
     for _ in range(max(args.warmup, 3)):
         flush.fill_(1)
@@ -445,40 +609,40 @@ def main():
             pg.barrier()
         step_ms = [a.elapsed_time(b) for a, b in ev]
         # per-call durations over K more steps of graph B (same work, event nodes between calls)
-        part_ms = {"meta": [], "score": [], "select": [], "decode": []}
+        names = [n for n, _ in step.calls]
+        part_ms = {n: [] for n in names}
         for i in range(args.steps):
             flush.fill_(i & 0xff)
             graph_b.replay()
             torch.cuda.synchronize()
-            for k, j in [("meta", 0), ("score", 1), ("select", 2), ("decode", 3)]:
-                part_ms[k].append(evb[j].elapsed_time(evb[j + 1]))
+            for j, n in enumerate(names):
+                part_ms[n].append(evb[j].elapsed_time(evb[j + 1]))
     total_s = replicas.max_over_ranks(sum(step_ms) / 1e3, device=dev)
+    median_ms = replicas.max_over_ranks(statistics.median(step_ms), device=dev)
     st, bits = ekv.ekv_device_status(cache)
     if st != ekv.EKV_OK:
         raise RuntimeError("device status 0x%x after timing" % bits)
 
     # ---- end to end through the public API with host buffers (pinned), copies inside
     q_host = wl.q.cpu().pin_memory()
-    out_host = torch.empty(dec.out.shape, dtype=dec.out.dtype).pin_memory()
-    stat_host = torch.empty(dec.stat.shape, dtype=dec.stat.dtype).pin_memory()
+    out_host = torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory()
+    stat_host = torch.empty(step.stat.shape, dtype=step.stat.dtype).pin_memory()
     h2d = q_host.numel() * q_host.element_size()
     app_host = None
     if wl.append is not None:
         last = int(wl.page_table[0, wl.append[0] // P])  # a host index: no sync in the graph
         app_host = (wl.k_cache[last].cpu().pin_memory(), wl.v_cache[last].cpu().pin_memory(), last)
         h2d += 2 * app_host[0].numel() * app_host[0].element_size()
-    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(args.steps)]
 
     def host_pre():
-        # the appended page's K and V rows arrive from the host, then its metadata is refreshed
+        # the appended page's K and V rows arrive from the host (its metadata refresh is the
+        # step's first call)
         if app_host is not None:
             wl.k_cache[app_host[2]].copy_(app_host[0], non_blocking=True)
             wl.v_cache[app_host[2]].copy_(app_host[1], non_blocking=True)
-        if pre is not None:
-            pre()
-    # one graph per host-to-host step: query in, step, outputs out
-    graph_e2e = dec.capture_host(wl.q, q_host, out_host, stat_host, pre_step=host_pre)
+    graph_e2e = step.graph_host(q_host, out_host, stat_host, host_pre=host_pre)
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
     for i in range(args.steps + 3):
         flush.fill_(1)
         if i >= 3:
@@ -494,7 +658,7 @@ def main():
     if not args.no_full_cache and world == 1:
         full_ms, _, stat_full = full_cache_time(ekv, cache, wl, attn, min(args.steps, 20), flush,
                                                 stream)
-        quality = selection_quality(wl, dec, attn, stat_full)
+        quality = selection_quality(ekv, cache, wl, dec, attn, stat_full)
         st, bits = ekv.ekv_device_status(cache)
         if st != ekv.EKV_OK:
             raise RuntimeError("device status 0x%x after the full-cache decode" % bits)
@@ -505,53 +669,57 @@ def main():
             pg.destroy_process_group()
         return
 
-    by = step_bytes(wl, dec, attn)
+    by = step_bytes(wl, dec, attn, args.variant, step.extra)
     peak, peak_kind = measured_peak()
-    score_s = statistics.mean(part_ms["score"]) / 1e3
-    decode_s = statistics.mean(part_ms["decode"]) / 1e3
-    total_pages = int(((wl.seq_lens.long() + P - 1) // P).sum())
-    traffic = ncu_traffic("score.cu", "score_pages_needle128k.md", total_pages * H) \
-        if args.workload == "needle128k" else None
-    achieved = by["score"] / score_s / 1e9
+    call_us = {k: statistics.median(v) * 1e3 for k, v in part_ms.items()}
     value = replicas.job_rate(args.steps, world, total_s)
     ms = total_s / args.steps * 1e3
+    if args.variant == "pages":
+        total_pages = int(((wl.seq_lens.long() + P - 1) // P).sum())
+        traffic = ncu_traffic("score.cu", "score_pages_needle128k.md", total_pages * H) \
+            if args.workload == "needle128k" else None
+        dom = "score"
+    else:
+        traffic = None
+        dom = max((n for n in call_us if n in by), key=lambda n: call_us[n])
+    achieved = by[dom] / (call_us[dom] / 1e6) / 1e9
+    frac_step = by["required_step"] / (ms / 1e3) / 1e9 / peak
     cpu = None
     if not args.no_cpu_baseline and world == 1:
-        per_step, desc = oracle_sample(wl, attn, args.cpu_sample_seconds)
-        cpu = {"value": 1.0 / per_step, "unit": "steps/s", "cores": 1, "kind": "oracle",
-               "sample": desc}
+        cpu = cpu_baseline(wl, attn, args.variant, T, args.cpu_sample_seconds)
     line = {
         "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world,
         "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": ms,
+        "ms_per_step_median": median_ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype":
             "bf16" if wl.k_cache.dtype == torch.bfloat16 else "f32",
         "data": "synthetic (seeded; rank r decodes its own batch)",
-        "config": {"workload": wl.name, "batch_per_gpu": B, "ctx": int(wl.seq_lens.max()),
-                   "q_heads": wl.num_q_heads, "kv_heads": H, "head_dim": d, "page": P,
-                   "policy": "top-k %d" % wl.topk if wl.policy == 0 else "%s delta %g" % (POLICY_NAME[wl.policy], wl.delta),
-                   "attn": ATTN_NAME[attn], "l2": "flushed before every step (256 MiB write, outside the timed events)",
-                   "parallelism": "replicas x%d, no collective" % world},
+        "config": config_of(wl, attn, args.variant, T, world),
         "hbm": {"required_bytes_per_step": by["required_step"],
                 "achieved_GBps": by["required_step"] / (ms / 1e3) / 1e9,
                 "frac_of_8TBps": by["required_step"] / (ms / 1e3) / 8e12,
-                "frac_of_measured": by["required_step"] / (ms / 1e3) / 1e9 / peak,
+                "frac_of_measured": frac_step,
                 "required_bytes_if_all_v": by["required_step_all_v"],
-                "selected_tokens": by["selected_tokens"], "v_rows_read": by["support_rows"]},
-        "per_call_us": {k: statistics.mean(v) * 1e3 for k, v in part_ms.items()},
-        "roofline": {"kernel": "score_pages", "bound": "hbm", "achieved": achieved,
-                     "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                "selected_tokens": by["selected_tokens"],
+                **({"v_rows_read": by["support_rows"]} if "support_rows" in by else {}),
+                **({"kept_tokens": by["kept_tokens"]} if "kept_tokens" in by else {})},
+        "target": {"what": "the step's required bytes at >= %.2f of the measured HBM copy "
+                           "bandwidth" % TARGET_FRAC,
+                   "frac": frac_step, "met": frac_step >= TARGET_FRAC},
+        "per_call_us": call_us,
+        "roofline": {"kernel": {"score": "score_pages"}.get(dom, dom), "bound": "hbm",
+                     "achieved": achieved, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic,
-                     "algorithmic_bytes_per_launch": by["score"]},
-        "decode_kernel": {"achieved_GBps": by["decode"] / decode_s / 1e9,
-                          "frac": by["decode"] / decode_s / 1e9 / peak},
+                     "algorithmic_bytes_per_launch": by[dom]},
+        "call_fracs": {n: by[n] / (call_us[n] / 1e6) / 1e9 / peak for n in call_us if n in by},
         "full_cache": None if full_ms is None else {
             "what": "the same attention over every page (no scoring, no selection) on this GPU",
             "ms_per_step": full_ms, "steps_per_s": 1e3 / full_ms,
-            "sparse_speedup": full_ms / ms},
+            "sparse_speedup": full_ms / median_ms},
         "selection_quality": quality,
         "e2e": {"value": replicas.job_rate(args.steps, world, e2e_s), "unit": "steps/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": launches_per_step * args.steps,
+        "gpu_launches": step.launches() * args.steps,
         "launch": "one CUDA graph per step (programmatic dependent launch between its kernels)",
         "clocks": clocks.summary(),
         "cpu_baseline": cpu,
@@ -563,35 +731,36 @@ def main():
 
 
 def reference_arm(args, rank, world, make):
-    """The CPU oracle as it stands, on the host cores, same workload/metric/unit; rank 0 only."""
+    """The CPU oracle as it stands, on all host cores, same workload/metric/unit; rank 0 only."""
     if rank != 0:
         return
     dev = "cuda" if torch.cuda.is_available() else "cpu"
-    from sparse_kv_cache_kmin_b200 import replicas
-    wl = make(args.workload, device=dev, seed=replicas.workload_seed(args.workload, 0))
-    attn = wl.attn_modes[0] if args.attn is None else args.attn
-    if args.policy is not None:
-        wl.policy = {v: k for k, v in POLICY_NAME.items()}[args.policy]
+    wl, attn, T = setup_workload(args, make, 0, dev)
+    st = OracleStep(wl, attn, args.variant, T)
+    threads = os.cpu_count() or 1
+    single, _ = st.single_thread(2.0)
     n_steps = max(args.warmup, 3) + args.steps
-    budget = max(2.0, 150.0 / n_steps)  # the whole run stays within a few minutes
-    times = []
-    desc = ""
+    budget = max(1.0, 150.0 / n_steps)  # the whole run stays within a few minutes
+    times, done = [], 0
     for i in range(n_steps):
-        per_step, desc = oracle_sample(wl, attn, budget, max_heads=None)
+        per_step, done = st.all_cores(threads, budget, single / len(st.problems))
         if i >= max(args.warmup, 3):
             times.append(per_step)
     value = 1.0 / statistics.mean(times)
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world,
         "steps": args.steps, "warmup": max(args.warmup, 3),
-        "ms_per_step": statistics.mean(times) * 1e3, "higher_is_better": True,
+        "ms_per_step": statistics.mean(times) * 1e3,
+        "ms_per_step_median": statistics.median(times) * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic (seeded)",
-        "config": {"workload": wl.name, "batch_per_gpu": wl.batch, "ctx": int(wl.seq_lens.max()),
-                   "q_heads": wl.num_q_heads, "kv_heads": wl.num_kv_heads,
-                   "head_dim": wl.head_dim, "page": wl.page_size, "attn": ATTN_NAME[attn]},
-        "cpu_baseline": {"value": value, "unit": "steps/s", "cores": 1, "kind": "oracle",
-                         "sample": desc + "; each step a fresh bounded sample"},
+        "config": config_of(wl, attn, args.variant, T, world),
+        "cpu_baseline": {"value": value, "unit": "steps/s", "cores": threads, "kind": "oracle",
+                         "cpu_model": cpu_model(), "nproc": threads,
+                         "sample": "%d of %d (sequence, KV head) problems per step on a pool of "
+                                   "%d threads, wall time scaled to the full step; each step a "
+                                   "fresh timing" % (done, len(st.problems), threads),
+                         "single_thread": {"value": 1.0 / single, "unit": "steps/s", "cores": 1}},
         "e2e": {"value": value, "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)

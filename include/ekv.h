@@ -145,7 +145,8 @@ ekv_status ekv_score_pages(const ekv_cache *c, const void *q, int32_t num_q_head
  *     maximum score": page j is kept iff some query g has (alpha-1) * est_{g,j} >
  *     tau_hat_g - delta, est = min(UB_{g,j}, m_{g,j} + sqrt(2 ln n_j) * sqrt(v_{g,j})) -- the
  *     Gaussian estimate of the page's largest score, capped by the bound (fp64 decision).
- *   scores     as written by ekv_score_pages with the same policy.
+ *   scores     as written by ekv_score_pages with the same policy; 16-byte aligned (rows are
+ *              read as float4), else EKV_ERR_INVALID_ARG.
  *   sel_idx    [batch][H_kv][max_sel] int32 output: logical page indices, ascending, then -1.
  *   sel_count  [batch][H_kv] int32 output.
  */
@@ -167,8 +168,9 @@ ekv_status ekv_select_pages(const ekv_cache *c, int32_t num_q_heads, int32_t pol
  *              EKV_ERR_INVALID_ARG.
  *   out        [batch][num_q_heads][d] fp32.   stat [batch][num_q_heads] fp32.
  *   ws         scratch of at least ekv_decode_workspace_bytes(c, num_q_heads, max_sel)
- *              bytes. It must be zero-filled once before its first use; every call leaves
- *              it ready for the next. Calls that share one ws must not overlap on the GPU.
+ *              bytes, 16-byte aligned (EKV_ERR_INVALID_ARG otherwise). Its contents need no
+ *              initialisation: every word a call reads was written earlier in the same call.
+ *              Calls that share one ws must not overlap on the GPU.
  */
 ekv_status ekv_sparse_decode(const ekv_cache *c, const void *q, int32_t num_q_heads,
                              float scale, int32_t attn, const int32_t *sel_idx,
@@ -251,7 +253,8 @@ size_t ekv_moment_decode_workspace_bytes(const ekv_cache *c, int32_t num_q_heads
  * skipped (n_e = 0) the result is the plain softmax. Arguments are those of
  * ekv_sparse_decode, plus `moments` (as kept by ekv_moment_update for exactly the tokens
  * [0, seq_lens[b]) of each sequence); ws holds at least
- * ekv_moment_decode_workspace_bytes(c, num_q_heads, max_sel) bytes under the same rules.
+ * ekv_moment_decode_workspace_bytes(c, num_q_heads, max_sel) bytes under the same rules
+ * (16-byte aligned, no initialisation needed).
  */
 ekv_status ekv_sparse_decode_moment(const ekv_cache *c, const float *moments, const void *q,
                                     int32_t num_q_heads, float scale, const int32_t *sel_idx,
@@ -271,7 +274,8 @@ ekv_status ekv_sparse_decode_moment(const ekv_cache *c, const float *moments, co
 #define EKV_MAX_TOKENS 32768 /* largest T */
 
 /* Scratch bytes of ekv_select_tokens: one fp32 score per candidate slot,
- * batch * H_kv * max_sel * P * 4 (0 on invalid arguments). */
+ * batch * H_kv * max_sel * P * 4 (0 on invalid arguments). The scratch must be 16-byte
+ * aligned and needs no initialisation. */
 size_t ekv_token_workspace_bytes(const ekv_cache *c, int32_t max_sel);
 
 /*
@@ -295,6 +299,29 @@ ekv_status ekv_sparse_decode_tokens(const ekv_cache *c, const void *q, int32_t n
                                     float scale, int32_t attn, const int32_t *tok_page,
                                     const int32_t *tok_pos, const int32_t *tok_count, int32_t T,
                                     float *out, float *stat, void *stream);
+
+/*
+ * How much of the full-cache attention a page selection keeps: a diagnostic beside the decode
+ * (EntmaxKV summary §3: attending over a subset moves the output by at most 2 B delta, delta the
+ * full-cache weight outside the subset; §3-§4: support recovery). It reads every key of every
+ * sequence, so it costs a full-cache pass. For each query head, over every valid token i:
+ *   p_i        the full-cache weight that stat_full defines: softmax exp(s_i - stat),
+ *              entmax [(alpha-1) s_i - stat]_+^(1/(alpha-1)), s = scale q.k_i.
+ *   dropped    [batch][num_q_heads] fp64 output: sum of p_i over tokens of pages outside
+ *              sel_idx[b][h][0 .. sel_count) -- delta.
+ *   support    [batch][num_q_heads][2] int32 output: the support size (entmax: tokens with
+ *              (alpha-1) s_i > stat; softmax: every valid token) and how many of those lie in
+ *              the selected pages (support recall = support[1] / support[0]).
+ *   stat_full  [batch][num_q_heads] fp32: the full-cache statistic, e.g. the stat of
+ *              ekv_sparse_decode called with every page of every sequence selected.
+ * Both outputs are overwritten (zeroed on `stream`, then accumulated). A bad page-table entry is
+ * skipped and flagged EKV_DEV_BAD_BLOCK. Other arguments as in ekv_sparse_decode.
+ */
+ekv_status ekv_selection_quality(const ekv_cache *c, const void *q, int32_t num_q_heads,
+                                 float scale, int32_t attn, const float *stat_full,
+                                 const int32_t *sel_idx, const int32_t *sel_count,
+                                 int32_t max_sel, double *dropped, int32_t *support,
+                                 void *stream);
 
 /* Synchronise `stream`, copy *c->dev_status to *bits (host pointer, may be NULL) and return
  * EKV_ERR_DEVICE if any bit is set, else EKV_OK (EKV_ERR_CUDA if the copy fails). */

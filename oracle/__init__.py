@@ -77,6 +77,10 @@ def _load():
                                            c_int, _dp, c_int, c_double, c_int, _ip, _ip, c_int,
                                            _dp, _dp]
     lib.ora_attend_tokens_head.restype = c_int
+    lib.ora_selection_quality_head.argtypes = [vp, vp, c_int, c_int, c_int, c_int, c_int, _ip,
+                                               c_int, c_int, _dp, c_int, c_double, c_int, _dp,
+                                               _ip, c_int, _dp, _ip, _ip]
+    lib.ora_selection_quality_head.restype = c_int
     _lib = lib
     return lib
 
@@ -243,6 +247,37 @@ def attend_head(k_cache, v_cache, pt_row, seq_len: int, h: int, q, scale: float,
         raise ValueError("selected page or page-table entry out of range")
     weights = w[:G * rc].reshape(G, rc) if w is not None else None
     return out, stat, weights
+
+
+def selection_quality_head(k_cache, v_cache, pt_row, seq_len: int, h: int, q, scale: float,
+                           mode: int, sel, stat=None):
+    """How much of the full-cache attention the selected pages keep, per query of KV head h
+    (EntmaxKV summary §3-§4; see ``ora_selection_quality_head``).
+
+    Returns (dropped [G]: full-cache weight outside the selected pages, n_sup [G]: support size
+    (entmax) or valid tokens (softmax), n_kept [G]: those inside the selected pages). With
+    ``stat`` ([G] full-cache log-partition or tau) the weights are the ones it defines;
+    without, the oracle's own full-cache attention."""
+    nb, H_kv, P, d = k_cache.shape
+    k_cache = np.ascontiguousarray(k_cache)
+    v_cache = np.ascontiguousarray(v_cache)
+    dt = _cache_dtype(k_cache)
+    q, qp = _d(np.atleast_2d(q))
+    G = q.shape[0]
+    pt, ptp = _i(pt_row)
+    sel, sp = _i(np.asarray(sel, dtype=np.int32).reshape(-1))
+    st, stp = (None, None) if stat is None else _d(np.asarray(stat, dtype=np.float64).reshape(G))
+    dropped = np.zeros(G)
+    n_sup = np.zeros(G, np.int32)
+    n_kept = np.zeros(G, np.int32)
+    rc = _load().ora_selection_quality_head(k_cache.ctypes.data, v_cache.ctypes.data, dt, nb, H_kv,
+                                            P, d, ptp, int(seq_len), int(h), qp, G, float(scale),
+                                            int(mode), stp, sp, len(sel),
+                                            dropped.ctypes.data_as(_dp),
+                                            n_sup.ctypes.data_as(_ip), n_kept.ctypes.data_as(_ip))
+    if rc < 0:
+        raise ValueError("selected page or page-table entry out of range")
+    return dropped, n_sup, n_kept
 
 
 def moment_corrected_head(k_cache, v_cache, pt_row, seq_len: int, h: int, q, scale: float, sel):

@@ -700,3 +700,95 @@ int ora_moment_sums_head(const void *k_cache, const void *v_cache, int dtype, in
     }
     return n;
 }
+
+/* ---------------------------------------------------------------------------------------
+ * How much of the full-cache attention a page selection keeps, per query g of KV head h
+ * (EntmaxKV summary §3: attending over a subset of the tokens moves the output by at most
+ * 2 B delta, delta the full-cache weight outside the subset; §3-§4: whether the kept pages
+ * hold the support of the full-cache entmax). Over every valid token i of the sequence:
+ *   p_i   the full-cache weight. With stat == NULL it is the weight of the attention over all
+ *         pages (attend_rows over every token, in page order). With stat given ([G], the
+ *         full-cache log-partition for softmax, the threshold tau for entmax) it is the
+ *         weight that statistic defines: exp(s_i - stat_g), or [z_i - stat_g]_+^(1/(alpha-1))
+ *         with z = (alpha-1) s.
+ *   dropped[g]  sum of p_i over the tokens of pages outside `sel` (delta)
+ *   n_sup[g]    entmax: tokens with p_i > 0 (the support); softmax: every valid token
+ *   n_kept[g]   those of the n_sup[g] tokens that lie in a page of `sel`
+ * Returns the sequence's token count, or -1 when a selected page or a page-table entry is out
+ * of range.
+ * ------------------------------------------------------------------------------------- */
+int ora_selection_quality_head(const void *k_cache, const void *v_cache, int dtype,
+                               int num_blocks, int H_kv, int P, int d, const int32_t *pt_row,
+                               int seq_len, int h, const double *q, int G, double scale,
+                               int mode, const double *stat, const int32_t *sel, int n_sel,
+                               double *dropped, int32_t *n_sup, int32_t *n_kept)
+{
+    int n_pages = pages_of(seq_len, P);
+    for (int j = 0; j < n_pages; ++j)
+        if (pt_row[j] < 0 || pt_row[j] >= num_blocks)
+            return -1;
+    char *kept = (char *)calloc((size_t)(n_pages > 0 ? n_pages : 1), 1);
+    for (int i = 0; i < n_sel; ++i) {
+        if (sel[i] < 0 || sel[i] >= n_pages) {
+            free(kept);
+            return -1;
+        }
+        kept[sel[i]] = 1;
+    }
+    int n_tok = seq_len > 0 ? seq_len : 0;
+    size_t nb = (size_t)(n_tok > 0 ? n_tok : 1);
+    int *blk = (int *)malloc(sizeof(int) * nb);
+    int *pos = (int *)malloc(sizeof(int) * nb);
+    char *in_sel = (char *)malloc(nb);
+    for (int i = 0; i < n_tok; ++i) {
+        blk[i] = pt_row[i / P];
+        pos[i] = i % P;
+        in_sel[i] = kept[i / P];
+    }
+    double *w = (double *)malloc(sizeof(double) * nb * (size_t)G);
+    if (!stat) {
+        double *out = (double *)malloc(sizeof(double) * (size_t)G * d);
+        double *st = (double *)malloc(sizeof(double) * (size_t)G);
+        attend_rows(k_cache, v_cache, dtype, H_kv, P, d, blk, pos, n_tok, h, q, G, scale, mode,
+                    out, st, w);
+        free(out);
+        free(st);
+    } else {
+        double alpha = mode == ORA_ENTMAX15 ? 1.5 : 2.0;
+        for (int g = 0; g < G; ++g)
+            for (int i = 0; i < n_tok; ++i) {
+                double acc = 0.0;
+                for (int c = 0; c < d; ++c)
+                    acc += q[(size_t)g * d + c] *
+                           elem(k_cache, dtype, cache_off(blk[i], h, pos[i], c, H_kv, P, d));
+                double s = scale * acc, p;
+                if (mode == ORA_SOFTMAX) {
+                    p = exp(s - stat[g]);
+                } else {
+                    double r = (alpha - 1.0) * s - stat[g];
+                    p = r > 0.0 ? (alpha == 2.0 ? r : r * r) : 0.0;
+                }
+                w[(size_t)g * n_tok + i] = p;
+            }
+    }
+    for (int g = 0; g < G; ++g) {
+        double dsum = 0.0;
+        int ns = 0, nk = 0;
+        for (int i = 0; i < n_tok; ++i) {
+            double p = w[(size_t)g * n_tok + i];
+            if (!in_sel[i]) dsum += p;
+            int member = mode == ORA_SOFTMAX ? 1 : p > 0.0;
+            ns += member;
+            nk += member && in_sel[i];
+        }
+        dropped[g] = dsum;
+        n_sup[g] = ns;
+        n_kept[g] = nk;
+    }
+    free(w);
+    free(in_sel);
+    free(pos);
+    free(blk);
+    free(kept);
+    return n_tok;
+}

@@ -71,7 +71,8 @@ extern "C" ekv_status ekv_sparse_decode_noalloc(const ekv_cache *c, const void *
     // Nothing in the scratch has to start at zero: every word a call reads was written
     // earlier in the same call.
     return ekv::launch_sparse_decode(*c, q, num_q_heads, scale, attn, sel_idx, sel_count, max_sel,
-                                     out, stat, ws, static_cast<cudaStream_t>(stream), true) ==
+                                     out, stat, ws, static_cast<cudaStream_t>(stream),
+                                     ekv::use_pdl()) ==
                    cudaSuccess
                ? EKV_OK
                : EKV_ERR_CUDA;

@@ -43,6 +43,11 @@ cudaError_t launch_token_attend(const ekv_cache &c, const void *q, int H_q, floa
                                 const int32_t *tok_count, int T, float *out, float *stat,
                                 cudaStream_t st);
 
+cudaError_t launch_selection_quality(const ekv_cache &c, const void *q, int H_q, float scale,
+                                     int attn, const float *stat_full, const int32_t *sel_idx,
+                                     const int32_t *sel_count, int max_sel, double *dropped,
+                                     int32_t *support, cudaStream_t st);
+
 int persistent_grid_size(const void *kernel, int threads, size_t smem)
 {
     static std::mutex mu;
@@ -64,7 +69,7 @@ int persistent_grid_size(const void *kernel, int threads, size_t smem)
 }
 
 // Programmatic dependent launch between consecutive libekv kernels (EKV_PDL=0 turns it off).
-static bool use_pdl()
+bool use_pdl()
 {
     static const bool on = [] {
         const char *e = std::getenv("EKV_PDL");
@@ -144,6 +149,7 @@ ekv_status ekv_select_pages(const ekv_cache *c, int32_t num_q_heads, int32_t pol
     if (s != EKV_OK) return s;
     if ((s = check_heads(c, num_q_heads)) != EKV_OK) return s;
     if (!scores || !sel_idx || !sel_count || max_sel < 1) return EKV_ERR_INVALID_ARG;
+    if ((uintptr_t)scores & 15u) return EKV_ERR_INVALID_ARG;  // score rows are read as float4
     if (policy == EKV_SEL_TOPK) {
         if (topk < 1) return EKV_ERR_INVALID_ARG;
         const int need = topk < c->max_pages ? topk : c->max_pages;
@@ -185,6 +191,7 @@ ekv_status ekv_sparse_decode(const ekv_cache *c, const void *q, int32_t num_q_he
         return EKV_ERR_INVALID_ARG;
     if (!ws || ws_bytes < ekv_decode_workspace_bytes(c, num_q_heads, max_sel))
         return EKV_ERR_WORKSPACE;
+    if ((uintptr_t)ws & 15u) return EKV_ERR_INVALID_ARG;  // logits are read back as float4
     return cuda_status(launch_sparse_decode(*c, q, num_q_heads, scale, attn, sel_idx, sel_count,
                                             max_sel, out, stat, ws,
                                             static_cast<cudaStream_t>(stream), use_pdl()));
@@ -233,6 +240,7 @@ ekv_status ekv_sparse_decode_moment(const ekv_cache *c, const float *moments, co
         return EKV_ERR_INVALID_ARG;
     if (!ws || ws_bytes < ekv_moment_decode_workspace_bytes(c, num_q_heads, max_sel))
         return EKV_ERR_WORKSPACE;
+    if ((uintptr_t)ws & 15u) return EKV_ERR_INVALID_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     float *ret = reinterpret_cast<float *>(
         static_cast<char *>(ws) + moment_ret_offset(ekv_decode_workspace_bytes(c, num_q_heads, max_sel)));
@@ -266,6 +274,7 @@ ekv_status ekv_select_tokens(const ekv_cache *c, const void *q, int32_t num_q_he
         return EKV_ERR_INVALID_ARG;
     if (T > EKV_MAX_TOKENS) return EKV_ERR_UNSUPPORTED;
     if (!ws || ws_bytes < ekv_token_workspace_bytes(c, max_sel)) return EKV_ERR_WORKSPACE;
+    if ((uintptr_t)ws & 15u) return EKV_ERR_INVALID_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     float *tscores = static_cast<float *>(ws);
     cudaError_t e = launch_token_scores(*c, q, num_q_heads, scale, sel_idx, sel_count, max_sel,
@@ -293,6 +302,24 @@ ekv_status ekv_sparse_decode_tokens(const ekv_cache *c, const void *q, int32_t n
     return cuda_status(launch_token_attend(*c, q, num_q_heads, scale, attn, tok_page, tok_pos,
                                            tok_count, T, out, stat,
                                            static_cast<cudaStream_t>(stream)));
+}
+
+ekv_status ekv_selection_quality(const ekv_cache *c, const void *q, int32_t num_q_heads,
+                                 float scale, int32_t attn, const float *stat_full,
+                                 const int32_t *sel_idx, const int32_t *sel_count,
+                                 int32_t max_sel, double *dropped, int32_t *support, void *stream)
+{
+    ekv_status s = check_cache(c, false);
+    if (s != EKV_OK) return s;
+    if ((s = check_heads(c, num_q_heads)) != EKV_OK) return s;
+    if (attn != EKV_SOFTMAX && attn != EKV_ENTMAX15 && attn != EKV_SPARSEMAX)
+        return EKV_ERR_UNSUPPORTED;
+    if (!q || !stat_full || !sel_idx || !sel_count || !dropped || !support || max_sel < 1 ||
+        !(scale > 0.0f) || !std::isfinite(scale))
+        return EKV_ERR_INVALID_ARG;
+    return cuda_status(launch_selection_quality(*c, q, num_q_heads, scale, attn, stat_full,
+                                                sel_idx, sel_count, max_sel, dropped, support,
+                                                static_cast<cudaStream_t>(stream)));
 }
 
 ekv_status ekv_device_status(const ekv_cache *c, uint32_t *bits, void *stream)

@@ -242,6 +242,10 @@ __device__ __forceinline__ void load_vec_nc(const void *p, float (&f)[VEC])
 // (kernel, device, dynamic shared memory).
 int persistent_grid_size(const void *kernel, int threads, size_t smem);
 
+// Whether consecutive libekv kernels use programmatic dependent launch (environment variable
+// EKV_PDL=0 turns it off for every entry point).
+bool use_pdl();
+
 }  // namespace ekv
 
 namespace ekv {

@@ -300,6 +300,29 @@ __device__ __forceinline__ void trunc_moment(float a, float b, float tau, bool s
     }
 }
 
+// The same moments in fp64, for the final Newton steps.
+__device__ __forceinline__ void trunc_moment_d(double a, double b, double tau, bool sparsemax,
+                                               double &E, double &dE)
+{
+    const double r = a - tau;
+    if (b <= 0.0) {
+        const double rp = r > 0.0 ? r : 0.0;
+        E = sparsemax ? rp : rp * rp;
+        dE = sparsemax ? (r > 0.0 ? -1.0 : 0.0) : -2.0 * rp;
+        return;
+    }
+    const double u = r / b;
+    const double Phi = 0.5 * erfc(-u * 0.70710678118654752440);
+    const double phi = 0.39894228040143267794 * exp(-0.5 * u * u);
+    if (sparsemax) {
+        E = r * Phi + b * phi;
+        dE = -Phi;
+    } else {
+        E = (r * r + b * b) * Phi + r * b * phi;
+        dE = -2.0 * (r * Phi + b * phi);
+    }
+}
+
 constexpr int kGaussSmemBytes = 192 * 1024;  // survivor lists of one CTA (all G queries)
 
 // One CTA per (sequence, KV head); the G queries of the group each get 8/G warps. Each warp owns
@@ -313,7 +336,8 @@ constexpr int kGaussSmemBytes = 192 * 1024;  // survivor lists of one CTA (all G
 // from tau0 = max_j a_j - 1 (where F >= 1) rises monotonically onto the root; the sums are
 // combined over the query's warps each iteration (double-buffered partials, one named barrier).
 // Pages with a + 8 b <= tau contribute below 1e-14 of their count and are pruned every fourth
-// step. The union over the group then lists, in ascending page order, every page with
+// step. The fp32 iterates stop within about 1e-7 of the root; a few Newton steps with fp64
+// moments finish it. The union over the group then lists, in ascending page order, every page with
 // (alpha-1) UB_j > tau_g - delta for some query g.
 template <int G>
 __global__ void __launch_bounds__(256)
@@ -409,6 +433,18 @@ select_gauss_kernel(const float *__restrict__ scores, int H, int max_pages, int 
         }
         const bool over = cnt > capw;
 
+        int ph = 0;  // parity of the partial-sum buffer of the next combine
+        // Combine a warp's partial F, F' over the query's warps (double-buffered partials, one
+        // named barrier); every warp of the query gets the same sums.
+        auto combine = [&](double Fw, double dFw, double &Fs, double &dFs) {
+            if (lane == 0) { s_part[ph & 1][g][r][0] = Fw; s_part[ph & 1][g][r][1] = dFw; }
+            named_sync(1 + g, 32 * WPQ);
+            Fs = 0.0;
+            dFs = 0.0;
+#pragma unroll
+            for (int k = 0; k < WPQ; ++k) { Fs += s_part[ph & 1][g][k][0]; dFs += s_part[ph & 1][g][k][1]; }
+            ++ph;
+        };
         if (n == 0) {
             tau = -INFINITY;
         } else {
@@ -432,12 +468,8 @@ select_gauss_kernel(const float *__restrict__ scores, int H, int max_pages, int 
                         dF = fmaf(page_n(j), dE, dF);
                     }
                 }
-                const double Fw = warp_sum((double)F), dFw = warp_sum((double)dF);
-                if (lane == 0) { s_part[it & 1][g][r][0] = Fw; s_part[it & 1][g][r][1] = dFw; }
-                named_sync(1 + g, 32 * WPQ);
-                double Fs = 0.0, dFs = 0.0;
-#pragma unroll
-                for (int k = 0; k < WPQ; ++k) { Fs += s_part[it & 1][g][k][0]; dFs += s_part[it & 1][g][k][1]; }
+                double Fs, dFs;
+                combine(warp_sum((double)F), warp_sum((double)dF), Fs, dFs);
                 if (!(dFs < 0.0)) break;
                 const double step = (Fs - 1.0) / -dFs;
                 if (!(step > 1e-7 * fmax(1.0, fabs(tau)))) break;
@@ -464,6 +496,37 @@ select_gauss_kernel(const float *__restrict__ scores, int H, int max_pages, int 
                     }
                     cnt = kept;
                 }
+            }
+            // fp64 finish: the fp32 moments above carry about 1e-7 relative error, which bounds
+            // how close the fp32 iterates get to the root. Newton steps on double-precision
+            // moments over the same survivors (pruned pages add below 1e-14 of their count)
+            // take the root to fp64 accuracy; each step squares the error.
+#pragma unroll 1
+            for (int it = 0; it < 4; ++it) {
+                double F = 0.0, dF = 0.0;
+                if (!over) {
+                    for (int i = lane; i < cnt; i += 32) {
+                        double E, dE;
+                        trunc_moment_d(sa[i], sb[i], tau, sparsemax, E, dE);
+                        F = fma((double)sn[i], E, F);
+                        dF = fma((double)sn[i], dE, dF);
+                    }
+                } else {
+                    for (int j = p0 + lane; j < p1; j += 32) {
+                        float aj, bj;
+                        double E, dE;
+                        model(j, aj, bj);
+                        trunc_moment_d(aj, bj, tau, sparsemax, E, dE);
+                        F = fma((double)page_n(j), E, F);
+                        dF = fma((double)page_n(j), dE, dF);
+                    }
+                }
+                double Fs, dFs;
+                combine(warp_sum(F), warp_sum(dF), Fs, dFs);
+                if (!(dFs < 0.0)) break;
+                const double step = (Fs - 1.0) / -dFs;
+                tau += step;
+                if (!(fabs(step) > 1e-13 * fmax(1.0, fabs(tau)))) break;
             }
         }
         if (r == 0 && lane == 0) {

@@ -47,9 +47,14 @@ token_score_kernel(ekv_cache c, const void *__restrict__ q, int H_q, float scale
         const int i = i0 + r / P, t = r % P;
         const int j = sel_idx[(size_t)bh * max_sel + i];
         int blk = -1;
-        if (j >= 0 && j < np && j * P + t < len) {
+        if (j < 0 || j >= np) {
+            if (t == 0 && lane == 0) flag(c.dev_status, EKV_DEV_BAD_SEL);
+        } else if (j * P + t < len) {
             blk = c.page_table[(size_t)b * c.max_pages + j];
-            if (blk >= c.num_blocks) blk = -1;
+            if (blk < 0 || blk >= c.num_blocks) {
+                if (lane == 0) flag(c.dev_status, EKV_DEV_BAD_BLOCK);
+                blk = -1;
+            }
         }
         float acc = 0.f;
         if (blk >= 0) {

@@ -364,3 +364,19 @@ def ekv_sparse_decode_tokens(cache: PagedKVCache, q: torch.Tensor, num_q_heads: 
     _check(fn(ctypes.byref(c), _ptr(q), int(num_q_heads), float(scale), int(attn),
               _ptr(tok_page), _ptr(tok_pos), _ptr(tok_count), int(T), _ptr(out), _ptr(stat),
               _stream(stream)), "ekv_sparse_decode_tokens")
+
+
+def ekv_selection_quality(cache: PagedKVCache, q: torch.Tensor, num_q_heads: int, scale: float,
+                          attn: int, stat_full: torch.Tensor, sel_idx: torch.Tensor,
+                          sel_count: torch.Tensor, max_sel: int, dropped: torch.Tensor,
+                          support: torch.Tensor, stream=None):
+    """Full-cache weight outside the selected pages (dropped [B, H_q] float64) and the support
+    counts (support [B, H_q, 2] int32: size, inside the selection) for the full-cache statistic
+    stat_full [B, H_q] (see include/ekv.h)."""
+    P, I32, F = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float
+    fn = _moment_fn("ekv_selection_quality", [ctypes.POINTER(EkvCacheStruct), P, I32, F, I32, P,
+                                              P, P, I32, P, P, P])
+    c = cache.struct()
+    _check(fn(ctypes.byref(c), _ptr(q), int(num_q_heads), float(scale), int(attn),
+              _ptr(stat_full), _ptr(sel_idx), _ptr(sel_count), int(max_sel), _ptr(dropped),
+              _ptr(support), _stream(stream)), "ekv_selection_quality")

@@ -8,12 +8,22 @@ Tolerances (derived from the arithmetic; u = 2^-24 is the fp32 unit roundoff):
   top-k group bound          S = scale (Q+ . kmax + Q- . kmin) in fp32 with Q+- summed over G:
                              |err| <= 2 (2d + G + 1) u T,  T = scale sum_c |Q+_c||kmax_c| + |Q-_c||kmin_c|
   Gaussian UB, m, v          |err| <= 2 (2d + 2) u times the sum of the magnitudes of the terms
-  selection                  bit-exact on the GPU's own scores; against the oracle's float64
+  top-k selection            bit-exact on the GPU's own scores; against the oracle's float64
                              scores, pages in the symmetric difference must be ties within 1e-6
-                             of the k-th score (relative), the Gaussian threshold likewise
+                             of the k-th score (relative)
+  Gaussian tau-hat           on the GPU's own m, v: within 1e-6 max(1, |tau|) of the oracle's
+                             tau-hat on those statistics (the solver). On the oracle's own m, v:
+                             that, plus twice the first-order propagation of the m, v bounds
+                             above: |d tau| <= sum_j n_j (E_a |da_j| + E_b |db_j|) / sum_j n_j E_a,
+                             E_a, E_b the derivatives of the truncated moment in a and b
+  Gaussian selection         bit-exact on the GPU's own statistics and tau-hat; against the
+                             oracle's, a page in the symmetric difference must lie within
+                             (alpha-1) |d stat| + |d tau| + 1e-6 max(1, |tau|) of the threshold
   attention output / stat    fp32 inputs: 1e-5 absolute; bf16 inputs: 2e-2 relative + 5e-3 absolute
 """
 from __future__ import annotations
+
+import math
 
 import numpy as np
 import torch
@@ -135,6 +145,34 @@ def check_topk_selection(sel_gpu, scores_gpu, S_oracle, k):
     return len(diff)
 
 
+def tau_sensitivity(m, v, cnt, alpha, tau, dm, dv):
+    """First-order bound on how far the root of sum_j n_j E_j(tau) = 1 moves when each page's
+    m, v move by at most dm, dv: E_j(tau) = E[(X - tau)_+^p], X ~ N(a, b^2), a = (alpha-1) m,
+    b = (alpha-1) sqrt(v). Derivatives (u = (a - tau) / b):
+      p = 1: dE/da = Phi(u),              dE/db = phi(u)
+      p = 2: dE/da = 2 (r Phi + b phi),   dE/db = 2 b Phi(u)     (r = a - tau)
+    and dE/dtau = -dE/da, so |d tau| <= sum n (E_a |da| + E_b |db|) / sum n E_a."""
+    from scipy import special
+    am1 = alpha - 1.0
+    a = am1 * m
+    b = am1 * np.sqrt(np.maximum(v, 0.0))
+    r = a - tau
+    with np.errstate(divide="ignore", invalid="ignore"):
+        u = np.where(b > 0, r / np.where(b > 0, b, 1.0), np.sign(r) * np.inf)
+    Phi = special.ndtr(u)
+    phi = np.where(np.isfinite(u), np.exp(-0.5 * np.where(np.isfinite(u), u, 0.0) ** 2), 0.0) \
+        / math.sqrt(2 * math.pi)
+    if alpha == 2.0:
+        Ea, Eb = Phi, phi
+    else:
+        Ea, Eb = 2 * (np.maximum(r, 0) * (b == 0) + (r * Phi + b * phi) * (b > 0)), 2 * b * Phi
+    da = am1 * dm
+    with np.errstate(divide="ignore", invalid="ignore"):
+        db = am1 * np.minimum(np.sqrt(dv), np.where(v > 0, dv / (2 * np.sqrt(np.maximum(v, 1e-300))), np.inf))
+    den = np.sum(cnt * Ea)
+    return np.sum(cnt * (Ea * da + Eb * db)) / den if den > 0 else np.inf
+
+
 def close(a, b, dtype_bf16):
     if dtype_bf16:
         np.testing.assert_allclose(a, b, rtol=2e-2, atol=5e-3)
@@ -165,23 +203,34 @@ def check_head(wl, cache, dec, b, h, attn, hc=None, check_scores=True):
     else:
         m, v = O.gauss_stats_head(qg, wl.scale, mean, var)
         sc = dec.scores[b, h * G:(h + 1) * G, :, :hc.np].double().cpu().numpy()  # [G, 3, np]
+        d = qg.shape[1]
+        Tu = wl.scale * (np.abs(qg) @ np.maximum(np.abs(kmin), np.abs(kmax)).T)
+        Tm = wl.scale * (np.abs(qg) @ np.abs(mean).T)
+        Tv = wl.scale ** 2 * ((qg * qg) @ np.abs(var).T)
+        f = 2 * (2 * d + 2) * U
+        # m and v also carry the fp32 rounding of the page mean / variance they read
+        P = wl.page_size
+        kabs = np.maximum(np.abs(kmin), np.abs(kmax))
+        Tk2 = wl.scale ** 2 * ((qg * qg) @ (kabs * kabs).T)
+        tol_u = f * Tu + 1e-30
+        tol_m = f * Tm + 4 * P * U * Tu + 1e-30
+        tol_v = f * Tv + 24 * P * U * Tk2 + 1e-30
         if check_scores:
-            d = qg.shape[1]
-            Tu = wl.scale * (np.abs(qg) @ np.maximum(np.abs(kmin), np.abs(kmax)).T)
-            Tm = wl.scale * (np.abs(qg) @ np.abs(mean).T)
-            Tv = wl.scale ** 2 * ((qg * qg) @ np.abs(var).T)
-            f = 2 * (2 * d + 2) * U
-            # m and v also carry the fp32 rounding of the page mean / variance they read
-            P = wl.page_size
-            kabs = np.maximum(np.abs(kmin), np.abs(kmax))
-            Tk2 = wl.scale ** 2 * ((qg * qg) @ (kabs * kabs).T)
-            assert np.all(np.abs(sc[:, 0] - ub) <= f * Tu + 1e-30)
-            assert np.all(np.abs(sc[:, 1] - m) <= f * Tm + 4 * P * U * Tu + 1e-30)
-            assert np.all(np.abs(sc[:, 2] - v) <= f * Tv + 24 * P * U * Tk2 + 1e-30)
+            assert np.all(np.abs(sc[:, 0] - ub) <= tol_u)
+            assert np.all(np.abs(sc[:, 1] - m) <= tol_m)
+            assert np.all(np.abs(sc[:, 2] - v) <= tol_v)
         cnt = O.page_counts(hc.L, wl.page_size)
         tau_o = np.array([O.gauss_tau(m[g], v[g], cnt, wl.alpha) for g in range(G)])
         tau_g = dec.tau_hat[b, h * G:(h + 1) * G].double().cpu().numpy()
-        assert np.all(np.abs(tau_g - tau_o) <= 1e-4 * np.maximum(1, np.abs(tau_o))), (tau_g, tau_o)
+        # the solver: the oracle's tau-hat on the GPU's own statistics (float64 of its floats)
+        tau_same = np.array([O.gauss_tau(sc[g, 1], sc[g, 2], cnt, wl.alpha) for g in range(G)])
+        assert np.all(np.abs(tau_g - tau_same) <= 1e-6 * np.maximum(1, np.abs(tau_same))), \
+            (tau_g, tau_same)
+        # end to end: plus the propagated error of the GPU's fp32 statistics
+        tol_tau = np.array([1e-6 * max(1.0, abs(tau_o[g])) +
+                            2 * tau_sensitivity(m[g], v[g], cnt, wl.alpha, tau_o[g], tol_m[g], tol_v[g])
+                            for g in range(G)])
+        assert np.all(np.abs(tau_g - tau_o) <= tol_tau), (tau_g, tau_o, tol_tau)
         # the GPU's decision on its own statistics and tau-hat is the oracle's rule, exactly
         tau_gf = tau_g.astype(np.float32).astype(np.float64)
         if wl.policy == GAUSS_MAX:
@@ -189,15 +238,22 @@ def check_head(wl, cache, dec, b, h, attn, hc=None, check_scores=True):
             ref = O.gauss_select_est(ub, m, v, cnt, tau_o, wl.alpha, wl.delta)
             stat_o = np.array([[O.est_max(ub[g, j], m[g, j], v[g, j], cnt[j]) for j in range(ub.shape[1])]
                                for g in range(G)])
+            zn = np.sqrt(2 * np.log(np.maximum(cnt, 1)))
+            tol_stat = np.maximum(tol_u, tol_m + zn[None, :] * np.sqrt(tol_v))
         else:
             same = O.gauss_select(sc[:, 0], tau_gf, wl.alpha, wl.delta)
             ref = O.gauss_select(ub, tau_o, wl.alpha, wl.delta)
             stat_o = ub
+            tol_stat = tol_u
         np.testing.assert_array_equal(sel_gpu, same)
         diff = np.setxor1d(sel_gpu, ref)
         if len(diff):
-            margin = ((wl.alpha - 1) * stat_o[:, diff] - (tau_o[:, None] - wl.delta)).max(0)
-            assert np.all(np.abs(margin) <= 1e-4 * max(1.0, np.abs(tau_o).max())), margin
+            # a page decided differently must lie, for the query whose decision flips, within the
+            # statistic's and tau-hat's error of the threshold
+            margin = (wl.alpha - 1) * stat_o[:, diff] - (tau_o[:, None] - wl.delta)
+            tol = (wl.alpha - 1) * tol_stat[:, diff] + tol_tau[:, None] + \
+                1e-6 * np.maximum(1, np.abs(tau_o))[:, None]
+            assert np.all((np.abs(margin) <= tol).any(0)), (diff, margin, tol)
         info["sel_diff"] = len(diff)
         info["kept"] = n_sel
     out_o, stat_o, _ = O.attend_head(hc.k, hc.v, hc.pt, hc.L, h, qg, wl.scale, MODE[attn], sel_gpu)

@@ -207,3 +207,37 @@ def test_token_entry_points_validation(lib):
     assert dec(1, 32769) == 2
     c2 = fake_cache(v_cache=None)
     assert lib.ekv_sparse_decode_tokens(C.byref(c2), P, 32, 1.0, 1, P, P, P, 64, P, P, None) == 1
+
+
+def test_misaligned_scores_and_workspaces_are_refused_before_any_launch(lib):
+    # select reads score rows as float4 and the decode reads logits back from its workspace as
+    # float4: a pointer 4 or 8 bytes off a 16-byte boundary (a tensor slice, say) is refused on
+    # the host with EKV_ERR_INVALID_ARG; the placeholder pointers are never dereferenced
+    import ctypes as C
+    from sparse_kv_cache_kmin_b200.ekv import load_library
+    lib = load_library()
+    cp = C.POINTER(type(fake_cache()))
+    vp, i32, f32 = C.c_void_p, C.c_int32, C.c_float
+    c = fake_cache()
+    P = 0x1000
+    for off in (4, 8):
+        assert lib.ekv_select_pages(C.byref(c), 32, 0, 64, 1.5, 0.1, P + off, P, P, 64, None, None) == 1
+        assert lib.ekv_select_pages(C.byref(c), 32, 1, 0, 1.5, 0.1, P + off, P, P, 64, P, None) == 1
+    need = lib.ekv_decode_workspace_bytes(C.byref(c), 32, 256)
+    for off in (4, 8):
+        assert lib.ekv_sparse_decode(C.byref(c), P, 32, 1.0, 1, P, P, 256, P, P, P + off, need + 16,
+                                     None) == 1
+    lib.ekv_moment_decode_workspace_bytes.argtypes = [cp, i32, i32]
+    lib.ekv_moment_decode_workspace_bytes.restype = C.c_size_t
+    lib.ekv_sparse_decode_moment.argtypes = [cp, vp, vp, i32, f32, vp, vp, i32, vp, vp, vp,
+                                             C.c_size_t, vp]
+    mneed = lib.ekv_moment_decode_workspace_bytes(C.byref(c), 32, 256)
+    assert lib.ekv_sparse_decode_moment(C.byref(c), P, P, 32, 1.0, P, P, 256, P, P, P + 4,
+                                        mneed + 16, None) == 1
+    lib.ekv_token_workspace_bytes.argtypes = [cp, i32]
+    lib.ekv_token_workspace_bytes.restype = C.c_size_t
+    lib.ekv_select_tokens.argtypes = [cp, vp, i32, f32, vp, vp, i32, i32, vp, vp, vp, vp,
+                                      C.c_size_t, vp]
+    tneed = lib.ekv_token_workspace_bytes(C.byref(c), 256)
+    assert lib.ekv_select_tokens(C.byref(c), P, 32, 1.0, P, P, 256, 512, P, P, P, P + 8,
+                                 tneed + 16, None) == 1

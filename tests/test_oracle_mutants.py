@@ -78,6 +78,10 @@ MUTANTS = {
                                "            (void)0;\n"),
     "attention_reads_invalid_tokens": (
         "n_tok += seq_len - j * P < P ? seq_len - j * P : P;", "n_tok += P;"),
+    "quality_sums_the_kept_mass": ("            if (!in_sel[i]) dsum += p;", "            if (in_sel[i]) dsum += p;"),
+    "quality_given_stat_ignored": ("                    p = exp(s - stat[g]);", "                    p = exp(s);"),
+    "quality_counts_every_token_as_support": ("            int member = mode == ORA_SOFTMAX ? 1 : p > 0.0;",
+                                              "            int member = 1;"),
 }
 
 

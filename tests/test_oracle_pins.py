@@ -758,3 +758,98 @@ def test_moment_sums_golden_fixture_and_additivity():
     assert whole[0] == 61 and a[0] + b[0] == 61
     for x, y, z in zip(whole[1:], a[1:], b[1:]):
         np.testing.assert_allclose(x, y + z, rtol=0, atol=1e-12)
+
+
+# ----------------------------------------------------------------------------- §3 selection quality
+def dense_full_cache_weights(k, pt, L, h, qg, scale, mode):
+    """Full-cache weights of one query from a dense evaluation: scipy softmax, or entmax with
+    tau from brentq on its normalisation equation; also the support mask and min |z - tau|."""
+    s = scale * dense_tokens(k, pt, L, h) @ qg
+    if mode == O.SOFTMAX:
+        return special.softmax(s), np.ones(len(s), bool), np.inf
+    alpha = O.ALPHA_OF_MODE[mode]
+    pw = 1.0 / (alpha - 1.0)
+    z = (alpha - 1.0) * s
+    tau = optimize.brentq(lambda t: np.sum(np.maximum(z - t, 0) ** pw) - 1.0, z.max() - 1,
+                          z.max(), xtol=1e-15, rtol=1e-15)
+    return np.maximum(z - tau, 0) ** pw, z > tau, np.abs(z - tau).min()
+
+
+@pytest.mark.parametrize("mode", [O.SOFTMAX, O.ENTMAX15, O.SPARSEMAX])
+def test_selection_quality_against_dense_weights(mode):
+    # delta = the full-cache weight outside the kept pages, and the support counts, against a
+    # dense scipy evaluation of the full-cache weights
+    rng = np.random.default_rng(40)
+    for trial in range(8):
+        L = int(rng.integers(9, 140))
+        k, v, pt = make_seq(rng, L=L, nb=20, dist_scale=2.0)
+        n = O.pages_of(L, 8)
+        q = rng.standard_normal((3, 16))
+        keep = np.sort(rng.choice(n, size=int(rng.integers(0, n + 1)), replace=False)).astype(np.int32)
+        dropped, n_sup, n_kept = O.selection_quality_head(k, v, pt, L, 1, q, 0.6, mode, keep)
+        in_sel = np.isin(np.arange(L) // 8, keep)
+        for g in range(3):
+            p, sup, gap = dense_full_cache_weights(k, pt, L, 1, q[g], 0.6, mode)
+            assert gap > 1e-9  # no token sits on the threshold
+            assert abs(dropped[g] - p[~in_sel].sum()) <= 1e-12
+            assert n_sup[g] == sup.sum() and n_kept[g] == (sup & in_sel).sum()
+
+
+@pytest.mark.parametrize("mode", [O.SOFTMAX, O.ENTMAX15, O.SPARSEMAX])
+def test_selection_quality_extremes_and_complement(mode):
+    # every page kept drops nothing and keeps the whole support; no page kept drops all the
+    # mass; a selection and its complement drop masses that add up to one
+    rng = np.random.default_rng(41)
+    L = 77
+    k, v, pt = make_seq(rng, L=L, nb=20, dist_scale=2.0)
+    n = O.pages_of(L, 8)
+    q = rng.standard_normal((2, 16))
+    d_all, s_all, k_all = O.selection_quality_head(k, v, pt, L, 0, q, 0.8, mode, np.arange(n))
+    assert np.all(d_all == 0) and np.array_equal(s_all, k_all) and np.all(s_all > 0)
+    d_none, s_none, k_none = O.selection_quality_head(k, v, pt, L, 0, q, 0.8, mode, [])
+    np.testing.assert_allclose(d_none, 1.0, atol=1e-12)
+    assert np.all(k_none == 0) and np.array_equal(s_none, s_all)
+    a = np.array([0, 3, 4, 9], np.int32)
+    c = np.setdiff1d(np.arange(n), a).astype(np.int32)
+    d_a, _, k_a = O.selection_quality_head(k, v, pt, L, 0, q, 0.8, mode, a)
+    d_c, _, k_c = O.selection_quality_head(k, v, pt, L, 0, q, 0.8, mode, c)
+    np.testing.assert_allclose(d_a + d_c, 1.0, atol=1e-12)
+    np.testing.assert_array_equal(k_a + k_c, s_all)
+
+
+@pytest.mark.parametrize("mode", [O.SOFTMAX, O.ENTMAX15, O.SPARSEMAX])
+def test_selection_quality_given_stat_reproduces_the_full_cache_weights(mode):
+    # the full-cache statistic (log-partition or tau) of the attention over every page defines
+    # the same weights as that attention; a statistic shifted by 0.05 changes delta
+    rng = np.random.default_rng(42)
+    L = 100
+    k, v, pt = make_seq(rng, L=L, nb=20, dist_scale=2.0)
+    n = O.pages_of(L, 8)
+    q = rng.standard_normal((2, 16))
+    _, stat, _ = O.attend_head(k, v, pt, L, 1, q, 0.7, mode, np.arange(n))
+    keep = np.array([1, 2, 7, 11], np.int32)
+    own = O.selection_quality_head(k, v, pt, L, 1, q, 0.7, mode, keep)
+    given = O.selection_quality_head(k, v, pt, L, 1, q, 0.7, mode, keep, stat=stat)
+    np.testing.assert_allclose(given[0], own[0], atol=1e-12)
+    np.testing.assert_array_equal(given[1], own[1])
+    np.testing.assert_array_equal(given[2], own[2])
+    moved = O.selection_quality_head(k, v, pt, L, 1, q, 0.7, mode, keep, stat=stat + 0.05)
+    assert np.all(np.abs(moved[0] - own[0]) > 1e-6)
+
+
+@pytest.mark.parametrize("mode", [O.SOFTMAX, O.ENTMAX15, O.SPARSEMAX])
+def test_selection_quality_delta_bounds_the_output_error(mode):
+    # §3 with this function's delta: ||o_selected - o_full|| <= 2 B delta, B = max ||v_i||
+    rng = np.random.default_rng(43)
+    for trial in range(10):
+        L = int(rng.integers(9, 120))
+        k, v, pt = make_seq(rng, L=L, nb=16, dist_scale=float(rng.choice([0.5, 2.0])))
+        n = O.pages_of(L, 8)
+        q = rng.standard_normal((2, 16))
+        full, _, _ = O.attend_head(k, v, pt, L, 0, q, 0.5, mode, np.arange(n))
+        keep = np.sort(rng.choice(n, size=int(rng.integers(1, n + 1)), replace=False)).astype(np.int32)
+        out, _, _ = O.attend_head(k, v, pt, L, 0, q, 0.5, mode, keep)
+        dropped, _, _ = O.selection_quality_head(k, v, pt, L, 0, q, 0.5, mode, keep)
+        B = np.linalg.norm(dense_tokens(v, pt, L, 0), axis=1).max()
+        for g in range(2):
+            assert np.linalg.norm(out[g] - full[g]) <= 2 * B * dropped[g] + 1e-12

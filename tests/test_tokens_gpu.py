@@ -69,3 +69,34 @@ def test_token_selection_and_attention_small_ragged(cuda_device, dtype, d, P, G,
                                               MODE[attn], gp, gt)
             close(out[b, h * G:(h + 1) * G].double().cpu().numpy(), ref, bf16)
             close(stat[b, h * G:(h + 1) * G].double().cpu().numpy(), rstat, bf16)
+
+
+def test_bad_page_table_entry_is_flagged_by_token_selection(cuda_device):
+    # a selected page whose page-table entry is out of range: its tokens score -inf (never
+    # kept) and EKV_DEV_BAD_BLOCK is raised; a selected page outside the sequence raises
+    # EKV_DEV_BAD_SEL
+    wl = make_random(B=1, H_kv=2, G=2, d=64, P=16, lens=(200,), dtype=torch.float32,
+                     device="cuda", seed=31, topk=4)
+    cache, dec = run_gpu(wl, ekv.EKV_SOFTMAX)
+    assert ekv.ekv_device_status(cache)[0] == ekv.EKV_OK
+    wl.page_table[0, 3] = wl.k_cache.shape[0] + 5
+    sel = torch.tensor([[[0, 3, 5, -1], [1, 2, 3, -1]]], dtype=torch.int32, device="cuda")
+    cnt = torch.tensor([[3, 3]], dtype=torch.int32, device="cuda")
+    T = 48
+    ws = torch.empty(ekv.ekv_token_workspace_bytes(cache, 4), dtype=torch.uint8, device="cuda")
+    tp = torch.empty((1, 2, T), dtype=torch.int32, device="cuda")
+    tt = torch.empty_like(tp)
+    tc = torch.empty((1, 2), dtype=torch.int32, device="cuda")
+    ekv.ekv_select_tokens(cache, wl.q, wl.num_q_heads, wl.scale, sel, cnt, 4, T, tp, tt, tc, ws)
+    st, bits = ekv.ekv_device_status(cache)
+    assert st == ekv.EKV_ERR_DEVICE and bits & ekv.EKV_DEV_BAD_BLOCK, hex(bits)
+    # only the two good pages' 32 tokens are candidates, and page 3 is never kept
+    assert tc.tolist() == [[32, 32]]
+    assert 3 not in tp[0, :, :32].unique().tolist()
+    ekv.ekv_clear_device_status(cache)
+    bad = torch.tensor([[[0, 99, -1, -1], [1, -1, -1, -1]]], dtype=torch.int32, device="cuda")
+    ekv.ekv_select_tokens(cache, wl.q, wl.num_q_heads, wl.scale, bad,
+                          torch.tensor([[2, 1]], dtype=torch.int32, device="cuda"), 4, T, tp, tt,
+                          tc, ws)
+    st, bits = ekv.ekv_device_status(cache)
+    assert st == ekv.EKV_ERR_DEVICE and bits & ekv.EKV_DEV_BAD_SEL, hex(bits)
