@@ -143,7 +143,9 @@ def step_bytes(wl, dec, attn, variant, extra):
     append_b = 0
     if wl.append is not None:
         append_b = wl.batch * H * wl.append[1] * d * esz + wl.batch * H * meta_row
-    by = {"score": meta + ptab + qb + scores_out, "select": scores_out + dec.sel_idx.numel() * 4,
+    sel_out = dec.sel_idx.numel() * 4
+    by = {"score": meta + ptab + qb + scores_out, "select": scores_out + sel_out,
+          "score_select": meta + ptab + qb + scores_out + sel_out,
           "selected_tokens": sel_tok, "meta_bytes": meta}
     if variant == "pages":
         v_rows = sel_tok if attn == 0 else support_rows(wl, dec, attn)
@@ -393,17 +395,23 @@ class Step:
             calls.append(("meta", lambda: ekv.ekv_page_meta_update(cache, ap_start, ap_count,
                                                                    wl.append[1])))
         q = wl.q
-        calls.append(("score", lambda: ekv.ekv_score_pages(cache, q, wl.num_q_heads, wl.scale,
-                                                           wl.policy, dec.scores)))
-        calls.append(("select", lambda: ekv.ekv_select_pages(
-            cache, wl.num_q_heads, wl.policy, wl.topk, wl.alpha, wl.delta, dec.scores,
-            dec.sel_idx, dec.sel_count, dec.max_sel, dec.tau_hat)))
+        if wl.policy == 0:
+            # top-k: scores and selection in one launch (one cluster per sequence and KV head)
+            calls.append(("score_select", lambda: ekv.ekv_score_select_pages(
+                cache, q, wl.num_q_heads, wl.scale, wl.topk, dec.scores, dec.sel_idx,
+                dec.sel_count, dec.max_sel)))
+        else:
+            calls.append(("score", lambda: ekv.ekv_score_pages(cache, q, wl.num_q_heads, wl.scale,
+                                                               wl.policy, dec.scores)))
+            calls.append(("select", lambda: ekv.ekv_select_pages(
+                cache, wl.num_q_heads, wl.policy, wl.topk, wl.alpha, wl.delta, dec.scores,
+                dec.sel_idx, dec.sel_count, dec.max_sel, dec.tau_hat)))
         self.out, self.stat = dec.out, dec.stat
         if variant == "pages":
             calls.append(("decode", lambda: ekv.ekv_sparse_decode(
                 cache, q, wl.num_q_heads, wl.scale, attn, dec.sel_idx, dec.sel_count,
                 dec.max_sel, dec.out, dec.stat, dec.ws)))
-            self.kernels = {"meta": 1, "score": 1, "select": 1, "decode": 2}
+            self.kernels = {"meta": 1, "score_select": 1, "score": 1, "select": 1, "decode": 2}
         elif variant == "tokens":
             tws = torch.empty(ekv.ekv_token_workspace_bytes(cache, dec.max_sel), dtype=torch.uint8,
                               device=dev)
@@ -416,7 +424,7 @@ class Step:
                 tp, tt, tc, tws)))
             calls.append(("decode_tokens", lambda: ekv.ekv_sparse_decode_tokens(
                 cache, q, wl.num_q_heads, wl.scale, attn, tp, tt, tc, T, dec.out, dec.stat)))
-            self.kernels = {"score": 1, "select": 1, "select_tokens": 2, "decode_tokens": 1}
+            self.kernels = {"score_select": 1, "select_tokens": 2, "decode_tokens": 1}
         else:
             moments = torch.zeros(ekv.ekv_moment_bytes(cache) // 4, dtype=torch.float32, device=dev)
             ekv.ekv_moment_update(cache, moments, torch.zeros(B, dtype=torch.int32, device=dev),
@@ -428,7 +436,7 @@ class Step:
             calls.append(("decode_moment", lambda: ekv.ekv_sparse_decode_moment(
                 cache, moments, q, wl.num_q_heads, wl.scale, dec.sel_idx, dec.sel_count,
                 dec.max_sel, dec.out, dec.stat, mws)))
-            self.kernels = {"score": 1, "select": 1, "decode_moment": 4}
+            self.kernels = {"score_select": 1, "decode_moment": 4}
         self.calls = calls
 
     def launches(self):
@@ -674,14 +682,11 @@ def main():
     call_us = {k: statistics.median(v) * 1e3 for k, v in part_ms.items()}
     value = replicas.job_rate(args.steps, world, total_s)
     ms = total_s / args.steps * 1e3
-    if args.variant == "pages":
+    dom = max((n for n in call_us if n in by), key=lambda n: call_us[n])
+    traffic = None
+    if dom == "score_select" and args.workload == "needle128k":
         total_pages = int(((wl.seq_lens.long() + P - 1) // P).sum())
-        traffic = ncu_traffic("score.cu", "score_pages_needle128k.md", total_pages * H) \
-            if args.workload == "needle128k" else None
-        dom = "score"
-    else:
-        traffic = None
-        dom = max((n for n in call_us if n in by), key=lambda n: call_us[n])
+        traffic = ncu_traffic("step.cu", "score_select_needle128k.md", total_pages * H)
     achieved = by[dom] / (call_us[dom] / 1e6) / 1e9
     frac_step = by["required_step"] / (ms / 1e3) / 1e9 / peak
     cpu = None
@@ -707,7 +712,8 @@ def main():
                            "bandwidth" % TARGET_FRAC,
                    "frac": frac_step, "met": frac_step >= TARGET_FRAC},
         "per_call_us": call_us,
-        "roofline": {"kernel": {"score": "score_pages"}.get(dom, dom), "bound": "hbm",
+        "roofline": {"kernel": {"score": "score_pages", "score_select": "step_score_select"}.get(dom, dom),
+                     "bound": "hbm",
                      "achieved": achieved, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic,
                      "algorithmic_bytes_per_launch": by[dom]},

@@ -156,6 +156,22 @@ ekv_status ekv_select_pages(const ekv_cache *c, int32_t num_q_heads, int32_t pol
                             float *tau_hat, void *stream);
 
 /*
+ * §2.A and §2.B.1 in one call: the top-k page scores of ekv_score_pages (policy EKV_SEL_TOPK)
+ * and the selection of ekv_select_pages, with the same results bit for bit. One
+ * thread-block cluster per (sequence, KV head) scans the pair's metadata and selects from the
+ * scores in its shared memory, so no kernel waits for the whole grid in between.
+ *   scores     [batch][H_kv][max_pages] fp32 output, 16-byte aligned; may be NULL when every
+ *              (sequence, KV head) fits the cluster kernel (at most 16 CTAs of 8192 pages),
+ *              which is then the only path. A geometry beyond that runs the two standalone
+ *              kernels, which pass the scores through `scores` (NULL: EKV_ERR_INVALID_ARG).
+ *   sel_idx, sel_count, max_sel, topk  as in ekv_select_pages (max_sel >= min(topk, max_pages)).
+ * c->meta_bbox must be 16-byte aligned.
+ */
+ekv_status ekv_score_select_pages(const ekv_cache *c, const void *q, int32_t num_q_heads,
+                                  float scale, int32_t topk, float *scores, int32_t *sel_idx,
+                                  int32_t *sel_count, int32_t max_sel, void *stream);
+
+/*
  * §2.C attention over the selected pages only, read in place from the paged cache (no gather
  * copy). For each query head: s_i = scale * q.k_i over the valid tokens of the pages of its
  * KV head listed in sel_idx[b][h][0 .. min(sel_count, max_sel));

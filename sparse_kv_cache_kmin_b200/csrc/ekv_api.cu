@@ -48,6 +48,11 @@ cudaError_t launch_selection_quality(const ekv_cache &c, const void *q, int H_q,
                                      const int32_t *sel_count, int max_sel, double *dropped,
                                      int32_t *support, cudaStream_t st);
 
+bool step_score_select_supported(const ekv_cache &c);
+cudaError_t launch_step_score_select(const ekv_cache &c, const void *q, int H_q, float scale,
+                                     int topk, float *scores, int32_t *sel_idx, int32_t *sel_count,
+                                     int max_sel, cudaStream_t st, bool pdl);
+
 int persistent_grid_size(const void *kernel, int threads, size_t smem)
 {
     static std::mutex mu;
@@ -163,6 +168,32 @@ ekv_status ekv_select_pages(const ekv_cache *c, int32_t num_q_heads, int32_t pol
     return cuda_status(launch_select_pages(*c, num_q_heads, policy, topk, alpha, delta, scores,
                                            sel_idx, sel_count, max_sel, tau_hat,
                                            static_cast<cudaStream_t>(stream), use_pdl()));
+}
+
+ekv_status ekv_score_select_pages(const ekv_cache *c, const void *q, int32_t num_q_heads,
+                                  float scale, int32_t topk, float *scores, int32_t *sel_idx,
+                                  int32_t *sel_count, int32_t max_sel, void *stream)
+{
+    ekv_status s = check_cache(c, false);
+    if (s != EKV_OK) return s;
+    if ((s = check_heads(c, num_q_heads)) != EKV_OK) return s;
+    if (!q || !sel_idx || !sel_count || max_sel < 1 || topk < 1 || !(scale > 0.0f) ||
+        !std::isfinite(scale))
+        return EKV_ERR_INVALID_ARG;
+    if (max_sel < (topk < c->max_pages ? topk : c->max_pages)) return EKV_ERR_INVALID_ARG;
+    if ((uintptr_t)c->meta_bbox & 15u) return EKV_ERR_INVALID_ARG;
+    if (scores && ((uintptr_t)scores & 15u)) return EKV_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (step_score_select_supported(*c))
+        return cuda_status(launch_step_score_select(*c, q, num_q_heads, scale, topk, scores, sel_idx,
+                                                    sel_count, max_sel, st, use_pdl()));
+    // a geometry the cluster kernel does not hold: the two kernels, scores through global memory
+    if (!scores) return EKV_ERR_INVALID_ARG;
+    cudaError_t e = launch_score_pages(*c, q, num_q_heads, scale, EKV_SEL_TOPK, scores, st, use_pdl());
+    if (e == cudaSuccess)
+        e = launch_select_pages(*c, num_q_heads, EKV_SEL_TOPK, topk, 1.5f, 0.0f, scores, sel_idx,
+                                sel_count, max_sel, nullptr, st, use_pdl());
+    return cuda_status(e);
 }
 
 size_t ekv_decode_workspace_bytes(const ekv_cache *c, int32_t num_q_heads, int32_t max_sel)

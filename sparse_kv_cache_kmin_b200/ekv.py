@@ -380,3 +380,17 @@ def ekv_selection_quality(cache: PagedKVCache, q: torch.Tensor, num_q_heads: int
     _check(fn(ctypes.byref(c), _ptr(q), int(num_q_heads), float(scale), int(attn),
               _ptr(stat_full), _ptr(sel_idx), _ptr(sel_count), int(max_sel), _ptr(dropped),
               _ptr(support), _stream(stream)), "ekv_selection_quality")
+
+
+def ekv_score_select_pages(cache: PagedKVCache, q: torch.Tensor, num_q_heads: int, scale: float,
+                           topk: int, scores: Optional[torch.Tensor], sel_idx: torch.Tensor,
+                           sel_count: torch.Tensor, max_sel: int, stream=None):
+    """Top-k page scores and selection in one call (one cluster per sequence and KV head);
+    the results of ekv_score_pages + ekv_select_pages with the top-k policy, bit for bit."""
+    P, I32, F = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float
+    fn = _moment_fn("ekv_score_select_pages", [ctypes.POINTER(EkvCacheStruct), P, I32, F, I32, P,
+                                               P, P, I32, P])
+    c = cache.struct()
+    _check(fn(ctypes.byref(c), _ptr(q), int(num_q_heads), float(scale), int(topk), _ptr(scores),
+              _ptr(sel_idx), _ptr(sel_count), int(max_sel), _stream(stream)),
+           "ekv_score_select_pages")
