@@ -1,0 +1,41 @@
+// cluster.cuh -- thread-block cluster primitives (sm_90+ PTX): rank and size within the
+// cluster, a cluster-wide barrier, and loads from another CTA's shared memory (DSMEM).
+#pragma once
+
+#include "ekv_device.cuh"
+
+namespace ekv {
+
+__device__ __forceinline__ uint32_t cluster_rank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ uint32_t cluster_size()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+    return r;
+}
+// Barrier over every thread of every CTA of the cluster, ordering all memory accesses before
+// it (shared::cluster and global) before all accesses after it.
+__device__ __forceinline__ void cluster_sync()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// The address of `p` (in this CTA's shared memory) in the shared-memory window of CTA `rank`.
+__device__ __forceinline__ uint32_t dsmem(const void *p, uint32_t rank)
+{
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr(p)), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ int ld_dsmem(uint32_t addr)
+{
+    int v;
+    asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+    return v;
+}
+
+}  // namespace ekv

@@ -19,45 +19,13 @@
 // largest key. The passes stop as soon as that bin is taken whole. Keys equal to the final
 // threshold are taken in ascending page order, across CTAs in rank order. Each CTA then
 // writes its kept pages at its offset of the ascending selection.
-#include "ekv_device.cuh"
+#include "cluster.cuh"
 
 namespace ekv {
 
 constexpr int kStepThreads = 512;      // one CTA per SM; 16 warps x 16 rows in flight per lane
 constexpr int kStepKeyCap = 8192;      // pages per CTA (keys in shared memory)
 constexpr int kStepBins = 2048;
-
-__device__ __forceinline__ uint32_t cluster_rank()
-{
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-__device__ __forceinline__ uint32_t cluster_size()
-{
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
-    return r;
-}
-// Barrier over every thread of every CTA of the cluster, ordering all memory accesses before
-// it (shared::cluster and global) before all accesses after it.
-__device__ __forceinline__ void cluster_sync()
-{
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-// The address of `p` (in this CTA's shared memory) in the shared-memory window of CTA `rank`.
-__device__ __forceinline__ uint32_t dsmem(const void *p, uint32_t rank)
-{
-    uint32_t r;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr(p)), "r"(rank));
-    return r;
-}
-__device__ __forceinline__ int ld_dsmem(uint32_t addr)
-{
-    int v;
-    asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
-    return v;
-}
 
 __device__ __forceinline__ uint32_t score_key(float x)
 {
@@ -69,7 +37,7 @@ __device__ __forceinline__ uint32_t score_key(float x)
 struct StepShared {
     int hist[kStepBins];
     int warp_tot[32];
-    int w_above[32], w_tie[32];
+    int w_above[32], w_tie[32];  // per warp (the first NW entries)
     int s_bin, s_above, s_binc;
     int s_cnt[2];  // this CTA's (keys above the threshold, keys equal to it): read by the cluster
 };
@@ -188,7 +156,7 @@ step_score_select_kernel(ekv_cache c, const void *__restrict__ q, int H_q, float
     __syncthreads();
 
     // ---------------------------------------------------------------- select
-    if (kk == n) {  // every page is kept (also n = 0)
+    if (kk == n) {  // every page is kept (also n = 0); p0 + nl <= n <= max_sel
         for (int i = tid; i < nl; i += NT) out[p0 + i] = p0 + i;
         if (rank == C - 1)
             for (int i = n + tid; i < max_sel; i += NT) out[i] = -1;
@@ -257,7 +225,7 @@ step_score_select_kernel(ekv_cache c, const void *__restrict__ q, int H_q, float
     if (lane == 0) { sh.w_above[warp] = n_above; sh.w_tie[warp] = n_tie; }
     __syncthreads();
     if (warp == 0) {
-        const int a = sh.w_above[lane], t = sh.w_tie[lane];
+        const int a = lane < NW ? sh.w_above[lane] : 0, t = lane < NW ? sh.w_tie[lane] : 0;
         const int ia = warp_incl_scan(a), it = warp_incl_scan(t);
         sh.w_above[lane] = ia - a;  // above-keys before this warp
         sh.w_tie[lane] = it - t;    // ties before this warp
@@ -281,7 +249,8 @@ step_score_select_kernel(ekv_cache c, const void *__restrict__ q, int H_q, float
         const unsigned tb = __ballot_sync(kFull, cv == 0);
         const bool keep = cv > 0 || (cv == 0 && tie_rank + __popc(tb & ((1u << lane) - 1u)) < my_take);
         const unsigned kb = __ballot_sync(kFull, keep);
-        if (keep) out[pos + __popc(kb & ((1u << lane) - 1u))] = p0 + j;
+        const int at = pos + __popc(kb & ((1u << lane) - 1u));
+        if (keep && at < kk) out[at] = p0 + j;
         pos += __popc(kb);
         tie_rank += __popc(tb);
     }

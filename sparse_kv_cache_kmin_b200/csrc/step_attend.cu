@@ -1,0 +1,556 @@
+// step_attend.cu -- exact alpha-entmax attention over the selected pages with one thread-block
+// cluster per (sequence, KV head) (EntmaxKV technical summary, §2.C: attention over the
+// selected pages only; only the keys of those pages are read, and only the value rows that
+// carry weight).
+//
+// The pages a (sequence, KV head) selected are split over the C CTAs of its cluster. A CTA
+// resolves its pages (selection -> page table), then its 16 warps stream the K rows in 16-row
+// tiles straight into registers (16 loads of 16 bytes in flight per lane, the load structure
+// that reads scattered rows fastest), stage each tile in a per-warp shared-memory buffer with
+// its 16-byte pieces XOR-swizzled by row, and take the logits of all G queries of the KV head
+// with D / 16 warp-level bf16 MMAs (m16n8k16, fp32 accumulation). The logits z = (alpha-1) s
+// stay in shared memory, with the maximum of every tile.
+//
+// The threshold tau solves sum_i [z_i - tau]_+^(1/(alpha-1)) = 1 over all the pair's tokens,
+// which live in the cluster's distributed shared memory:
+//   1. The tile maxima are logits, and the exact threshold of any subset of the logits is at
+//      most tau (adding tokens only raises it). Each CTA reduces its tile maxima to 256 / C
+//      group maxima; one warp per query gathers all 256 (DSMEM) and solves them exactly
+//      (bitonic sort, closed form) for zmax and a lower bound on tau.
+//   2. Every token above the lower bound is a candidate; each CTA lists its own in token order.
+//      With at most 512 candidates in the cluster, one warp per query gathers them and solves
+//      exactly. More (nearly flat logits): an fp64 bisection whose sums are reduced over the
+//      cluster, then the closed form over the support it brackets.
+//   3. Each CTA accumulates p_i v_i over its support tokens (V rows read only for those), in a
+//      fixed order; the CTAs' partial outputs are summed over DSMEM in rank order.
+#include "cluster.cuh"
+#include "warp_entmax.cuh"
+#include "warp_mma.cuh"
+
+namespace ekv {
+
+constexpr int kAttThreads = 512;
+constexpr int kAttWarps = kAttThreads / 32;
+constexpr int kAttStageBytes = 8192;  // per warp: 16 loads of 16 bytes per lane
+constexpr int kAttGroups = 256;       // lower-bound maxima per query over the cluster
+constexpr int kAttCand = 512;         // candidates per query solved by one warp (16 per lane)
+
+struct AttArgs {
+    ekv_cache c;
+    const void *q;
+    int H_q;
+    float qscale;  // scale * (alpha - 1)
+    int sparsemax;
+    const int32_t *sel_idx;
+    const int32_t *sel_count;
+    int max_sel;
+    float *out;
+    float *stat;
+    int ent_cap;   // selected pages per CTA at most
+};
+
+// Small per-CTA state; the group maxima and candidate lists live in dynamic shared memory, on
+// the tile staging buffers (free once the logits are taken).
+template <int D, int G>
+struct AttShared {
+    int ccnt[G];                 // candidates of this CTA (read by the cluster)
+    int wcnt[kAttWarps];
+    float zmax[G];
+    double tlb[G], tau[G];
+    int fast[G];
+    double fpart[2][G];          // bisection partial sums (read by the cluster)
+    double cpart[3];             // closed-form partial sums (read by the cluster)
+    double red[kAttWarps];
+    float opart[kAttWarps][D];
+    float ocat[G][D];            // this CTA's partial output (read by the cluster)
+};
+
+__device__ __forceinline__ float ld_dsmem_f32(uint32_t addr)
+{
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+    return v;
+}
+__device__ __forceinline__ double ld_dsmem_f64(uint32_t addr)
+{
+    double v;
+    asm volatile("ld.shared::cluster.f64 %0, [%1];" : "=d"(v) : "r"(addr) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_shared_v4(void *p, const uint4 &v)
+{
+    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(smem_addr(p)), "r"(v.x), "r"(v.y),
+                 "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+template <int D, int G>
+__global__ void __launch_bounds__(kAttThreads, 1)
+step_attend_kernel(AttArgs a)
+{
+    constexpr int NT = kAttThreads, NW = kAttWarps;
+    constexpr int RB = D * 2;                 // bytes per bf16 row
+    constexpr int W = RB / 16;                // 16-byte pieces per row
+    constexpr int TB = 16 * RB;               // bytes per 16-row tile
+    constexpr int TPL = TB / 512;             // pieces per lane per tile
+    constexpr int TPS = kAttStageBytes / TB;  // tiles per warp step
+    constexpr int KS = D / 16;                // MMA k-steps per tile
+    static_assert(G <= 8, "one n = 8 MMA column block");
+    static_assert(G * (kAttGroups + 2 * kAttCand) * 4 <= kAttWarps * kAttStageBytes,
+                  "the lists fit on the staging buffers");
+    extern __shared__ __align__(128) unsigned char smem[];
+    __shared__ AttShared<D, G> sh;
+
+    const ekv_cache &c = a.c;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const uint32_t rank = cluster_rank(), C = cluster_size();
+    const int H = c.num_kv_heads, P = c.page_size, TPP = P / 16;
+    const int bh = blockIdx.x / (int)C, b = bh / H, h = bh % H;
+    const int ent_cap = a.ent_cap, ntok_cap = ent_cap * P, tile_cap = ent_cap * TPP;
+    unsigned char *stage = smem + (size_t)warp * kAttStageBytes;
+    float *zs = reinterpret_cast<float *>(smem + (size_t)NW * kAttStageBytes);  // [G][ntok_cap]
+    int *ent_blk = reinterpret_cast<int *>(zs + (size_t)G * ntok_cap);        // [ent_cap]
+    int *ent_nt = ent_blk + ent_cap;                                            // [ent_cap]
+    float *tmax = reinterpret_cast<float *>(ent_nt + ent_cap);                  // [G][tile_cap]
+    // after the logits phase, on the staging buffers (read by the cluster):
+    float *gm = reinterpret_cast<float *>(smem);                 // [G][kAttGroups] group maxima
+    float *cx = gm + G * kAttGroups;                             // [G][kAttCand] candidates z - zmax
+    int *ct = reinterpret_cast<int *>(cx + G * kAttCand);        // [G][kAttCand] their tokens
+
+    pdl_wait();
+    int len;
+    const int np = seq_pages(c.seq_lens, b, P, c.max_pages, nullptr, &len);
+    int ns = a.sel_count[bh];
+    ns = ns < 0 ? 0 : (ns > a.max_sel ? a.max_sel : ns);
+    const int e0 = (int)((long long)ns * rank / C), e1 = (int)((long long)ns * (rank + 1) / C);
+    const int ne = e1 - e0, ntiles = ne * TPP, ntok = ne * P;
+    for (int i = tid; i < ne; i += NT) {
+        const int j = a.sel_idx[(size_t)bh * a.max_sel + e0 + i];
+        int blk = -1, nt = 0;
+        if (j < 0 || j >= np) {
+            flag(c.dev_status, EKV_DEV_BAD_SEL);
+        } else {
+            const int bk = c.page_table[(size_t)b * c.max_pages + j];
+            if (bk < 0 || bk >= c.num_blocks) {
+                flag(c.dev_status, EKV_DEV_BAD_BLOCK);
+            } else {
+                blk = bk;
+                nt = len - j * P < P ? len - j * P : P;
+            }
+        }
+        ent_blk[i] = blk;
+        ent_nt[i] = nt;
+    }
+    if (tid < G) sh.ccnt[tid] = 0;
+    // B fragments of the group's queries: column n = lane / 4 is query n (zero past G)
+    uint32_t qb[KS][2];
+    {
+        const int n = lane >> 2;
+        const uint32_t *qr = reinterpret_cast<const uint32_t *>(
+            static_cast<const char *>(a.q) + (((size_t)b * a.H_q + (size_t)h * G + (n < G ? n : 0)) * D) * 2);
+#pragma unroll
+        for (int s = 0; s < KS; ++s) {
+            qb[s][0] = n < G ? __ldg(qr + s * 8 + (lane & 3)) : 0u;
+            qb[s][1] = n < G ? __ldg(qr + s * 8 + 4 + (lane & 3)) : 0u;
+        }
+    }
+    __syncthreads();
+
+    // ---------------------------------------------------------------- logits
+    const char *kc = static_cast<const char *>(c.k_cache);
+    const int lrow = lane & 15, lk = lane >> 4;
+    const int r0 = lane >> 2, n0 = (lane & 3) * 2;
+    for (int t0 = warp * TPS; t0 < ntiles; t0 += NW * TPS) {
+        uint4 x[TPS][TPL];
+        int ntt[TPS];
+#pragma unroll
+        for (int u = 0; u < TPS; ++u) {
+            const int t = t0 + u;
+            const int e = t / TPP, sub = t - e * TPP;
+            const int blk = t < ntiles ? ent_blk[e] : -1;
+            ntt[u] = blk >= 0 ? ent_nt[e] - sub * 16 : 0;
+            const char *g = kc + (((size_t)(blk < 0 ? 0 : blk) * H + h) * P + sub * 16) * RB;
+#pragma unroll
+            for (int k = 0; k < TPL; ++k)
+                x[u][k] = ntt[u] > 0 ? ld_stream16(g + (k * 32 + lane) * 16) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < TPS; ++u)
+#pragma unroll
+            for (int k = 0; k < TPL; ++k) {
+                const int p = k * 32 + lane, row = p / W, pc = p % W;
+                st_shared_v4(stage + u * TB + row * RB + ((pc ^ (row & 7)) << 4), x[u][k]);
+            }
+        __syncwarp();
+#pragma unroll
+        for (int u = 0; u < TPS; ++u) {
+            const int t = t0 + u;
+            if (t >= ntiles) break;  // uniform over the warp
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            const unsigned char *tile = stage + u * TB;
+#pragma unroll
+            for (int s = 0; s < KS; ++s) {
+                uint32_t af[4];
+                const int pc = s * 2 + lk;
+                ldsm_x4(af, tile + lrow * RB + ((pc ^ (lrow & 7)) << 4));
+                mma_bf16_16816(acc, af, qb[s][0], qb[s][1]);
+            }
+            const float z00 = r0 < ntt[u] ? a.qscale * acc[0] : -INFINITY;
+            const float z01 = r0 < ntt[u] ? a.qscale * acc[1] : -INFINITY;
+            const float z10 = r0 + 8 < ntt[u] ? a.qscale * acc[2] : -INFINITY;
+            const float z11 = r0 + 8 < ntt[u] ? a.qscale * acc[3] : -INFINITY;
+            const int tok = t * 16 + r0;
+            float m0 = fmaxf(z00, z10), m1 = fmaxf(z01, z11);
+            if (n0 < G) {
+                zs[(size_t)n0 * ntok_cap + tok] = z00;
+                zs[(size_t)n0 * ntok_cap + tok + 8] = z10;
+            }
+            if (n0 + 1 < G) {
+                zs[(size_t)(n0 + 1) * ntok_cap + tok] = z01;
+                zs[(size_t)(n0 + 1) * ntok_cap + tok + 8] = z11;
+            }
+#pragma unroll
+            for (int o = 4; o < 32; o <<= 1) {
+                m0 = fmaxf(m0, __shfl_xor_sync(kFull, m0, o));
+                m1 = fmaxf(m1, __shfl_xor_sync(kFull, m1, o));
+            }
+            if (lane < 4 && n0 < G) tmax[(size_t)n0 * tile_cap + t] = m0;
+            if (lane < 4 && n0 + 1 < G) tmax[(size_t)(n0 + 1) * tile_cap + t] = m1;
+        }
+        __syncwarp();  // the stage is read before the next tiles overwrite it
+    }
+    __syncthreads();
+
+    // ---------------------------------------------------------------- lower bound on tau
+    const int GM = kAttGroups / (int)C;  // group maxima per CTA
+    for (int i = tid; i < G * GM; i += NT) {
+        const int g = i / GM, k = i - g * GM;
+        const int ta = (int)((long long)ntiles * k / GM), tb = (int)((long long)ntiles * (k + 1) / GM);
+        float m = -INFINITY;
+        for (int t = ta; t < tb; ++t) m = fmaxf(m, tmax[(size_t)g * tile_cap + t]);
+        gm[g * kAttGroups + k] = m;
+    }
+    cluster_sync();
+    if (warp < G) {
+        const int g = warp;
+        float v[kAttGroups / 32];
+        float zm = -INFINITY;
+#pragma unroll
+        for (int r = 0; r < kAttGroups / 32; ++r) {
+            const int idx = r * 32 + lane, cr = idx / GM, k = idx - cr * GM;
+            v[r] = ld_dsmem_f32(dsmem(&gm[g * kAttGroups + k], (uint32_t)cr));
+            zm = fmaxf(zm, v[r]);
+        }
+        zm = warp_max(zm);
+        int cnt = 0;
+#pragma unroll
+        for (int r = 0; r < kAttGroups / 32; ++r) {
+            v[r] = v[r] - zm;  // -inf stays -inf
+            cnt += __popc(__ballot_sync(kFull, v[r] > -INFINITY));
+        }
+        double lb = 0.0;
+        if (zm > -INFINITY) {
+            lb = warp_exact_tau<kAttGroups / 32>(v, cnt, a.sparsemax != 0);
+            // lowered a little so that the fp32 rounding of the bound (prefix sums of up to 256
+            // values) never drops a support member
+            lb -= 1e-5 * fmax(1.0, fabs(lb));
+        }
+        if (lane == 0) {
+            sh.zmax[g] = zm;
+            sh.tlb[g] = lb;
+        }
+    }
+    __syncthreads();
+
+    // ---------------------------------------------------------------- candidates, token order
+    {
+        constexpr int WPQ = NW / G;  // warps per query
+        const int g = warp % G, part = warp / G;
+        const int ta = (int)((long long)ntok * part / WPQ), tb = (int)((long long)ntok * (part + 1) / WPQ);
+        const float zm = sh.zmax[g];
+        const double lb = sh.tlb[g];
+        const float *zg = zs + (size_t)g * ntok_cap;
+        int mine = 0;
+        for (int i = ta + lane; i - lane < tb; i += 32)
+            mine += __popc(__ballot_sync(kFull, i < tb && (double)(zg[i] - zm) > lb));
+        if (lane == 0) sh.wcnt[warp] = mine;
+        __syncthreads();
+        int pos = 0;
+        for (int p = 0; p < part; ++p) pos += sh.wcnt[p * G + g];
+        for (int i = ta + lane; i - lane < tb; i += 32) {
+            const float x = i < tb ? zg[i] - zm : -INFINITY;
+            const bool keep = i < tb && (double)x > lb;
+            const unsigned bal = __ballot_sync(kFull, keep);
+            const int at = pos + __popc(bal & ((1u << lane) - 1u));
+            if (keep && at < kAttCand) {
+                cx[g * kAttCand + at] = x;
+                ct[g * kAttCand + at] = i;
+            }
+            pos += __popc(bal);
+        }
+        if (part == WPQ - 1 && lane == 0) sh.ccnt[g] = pos;
+    }
+    cluster_sync();
+
+    // ---------------------------------------------------------------- exact tau
+    if (warp < G) {
+        const int g = warp;
+        int offs[17];
+        offs[0] = 0;
+        bool fits = true;
+        for (uint32_t cr = 0; cr < C; ++cr) {
+            const int n = ld_dsmem(dsmem(&sh.ccnt[g], cr));
+            fits = fits && n <= kAttCand;
+            offs[cr + 1] = offs[cr] + n;
+        }
+        const int total = offs[C];
+        fits = fits && total <= kAttCand;
+        double tau = 0.0;
+        if (sh.zmax[g] > -INFINITY && fits) {
+            float v[kAttCand / 32];
+#pragma unroll
+            for (int r = 0; r < kAttCand / 32; ++r) {
+                const int idx = r * 32 + lane;
+                v[r] = -INFINITY;
+                if (idx < total) {
+                    uint32_t cr = 0;
+                    while (idx >= offs[cr + 1]) ++cr;
+                    v[r] = ld_dsmem_f32(dsmem(&cx[g * kAttCand + idx - offs[cr]], cr));
+                }
+            }
+            tau = warp_exact_tau<kAttCand / 32>(v, total, a.sparsemax != 0);
+        }
+        if (lane == 0) {
+            sh.tau[g] = tau;
+            sh.fast[g] = sh.zmax[g] == -INFINITY || fits;
+        }
+    }
+    __syncthreads();
+    // Too many candidates for one warp (nearly flat logits): fp64 bisection on
+    // f(t) = sum [x - t]_+^p over the cluster's candidates, then the closed form over the support
+    // it brackets. The decision is the same in every CTA (the same counts were read), so every
+    // CTA takes the same cluster barriers.
+    for (int g = 0; g < G; ++g) {
+        if (sh.fast[g]) continue;
+        const float zm = sh.zmax[g];
+        const float *zg = zs + (size_t)g * ntok_cap;
+        double lo = sh.tlb[g], hi = 0.0;
+        auto cluster_total = [&](double v, double *slot) {  // sum over the cluster, rank order
+            v = warp_sum(v);
+            if (lane == 0) sh.red[warp] = v;
+            __syncthreads();
+            if (tid == 0) {
+                double s = 0.0;
+                for (int w = 0; w < NW; ++w) s += sh.red[w];
+                *slot = s;
+            }
+            cluster_sync();
+            double tot = 0.0;
+            for (uint32_t cr = 0; cr < C; ++cr) tot += ld_dsmem_f64(dsmem(slot, cr));
+            return tot;
+        };
+        for (int it = 0; it < 60; ++it) {
+            const double mid = 0.5 * (lo + hi);
+            double f = 0.0;
+            for (int i = tid; i < ntok; i += NT) {
+                const double r = (double)(zg[i] - zm) - mid;
+                if (r > 0.0) f += a.sparsemax ? r : r * r;
+            }
+            const double F = cluster_total(f, &sh.fpart[it & 1][g]);
+            if (F >= 1.0) lo = mid; else hi = mid;
+        }
+        double s1 = 0.0, s2 = 0.0, k = 0.0;
+        for (int i = tid; i < ntok; i += NT) {
+            const double x = (double)(zg[i] - zm);
+            if (x > lo) { s1 += x; s2 += x * x; k += 1.0; }
+        }
+        s1 = cluster_total(s1, &sh.cpart[0]);
+        s2 = cluster_total(s2, &sh.cpart[1]);
+        k = cluster_total(k, &sh.cpart[2]);
+        double tau = lo;
+        if (k > 0.0) closed_form_tau(k, s1, s2, a.sparsemax != 0, tau);
+        __syncthreads();
+        if (tid == 0) sh.tau[g] = tau;
+        cluster_sync();  // every CTA has read the partial sums before they are reused
+    }
+    __syncthreads();
+
+    // ---------------------------------------------------------------- output
+    {
+        constexpr int WPQ = NW / G;
+        const int g = warp % G, part = warp / G;
+        const float zm = sh.zmax[g];
+        const double tau = sh.tau[g];
+        const int half = lane >> 4, hl = lane & 15;
+        float acc[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+        const char *vc = static_cast<const char *>(c.v_cache);
+        auto add_row = [&](int tl, double r) {
+            const float p = (float)(a.sparsemax ? r : r * r);
+            const int e = tl / P, tok = tl - e * P;
+            const int blk = ent_blk[e];
+            if (hl < W && blk >= 0) {
+                const uint4 v = ld_stream16(vc + (((size_t)blk * H + h) * P + tok) * RB + hl * 16);
+                float f[8];
+                Chunk<EKV_BF16>::unpack(v, f);
+#pragma unroll
+                for (int q8 = 0; q8 < 8; ++q8) acc[q8] = fmaf(p, f[q8], acc[q8]);
+            }
+        };
+        if (zm > -INFINITY) {
+            if (sh.fast[g]) {
+                const int n = sh.ccnt[g];  // this CTA's candidates (<= kAttCand on this path)
+                for (int i = part * 2 + half; i < n; i += WPQ * 2) {
+                    const double r = (double)cx[g * kAttCand + i] - tau;
+                    if (r > 0.0) add_row(ct[g * kAttCand + i], r);
+                }
+            } else {
+                const float *zg = zs + (size_t)g * ntok_cap;
+                for (int i = part * 2 + half; i < ntok; i += WPQ * 2) {
+                    const double r = (double)(zg[i] - zm) - tau;
+                    if (r > 0.0) add_row(i, r);
+                }
+            }
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] += __shfl_xor_sync(kFull, acc[e], 16);
+        if (half == 0 && hl < W) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) sh.opart[warp][hl * 8 + e] = acc[e];
+        }
+        __syncthreads();
+        for (int i = tid; i < G * D; i += NT) {
+            const int gg = i / D, dd = i - gg * D;
+            float s = 0.f;
+            for (int p = 0; p < WPQ; ++p) s += sh.opart[p * G + gg][dd];
+            sh.ocat[gg][dd] = s;
+        }
+    }
+    cluster_sync();
+    // CTA `rank` writes the slice [rank * G * D / C, (rank + 1) * G * D / C) of the outputs
+    {
+        const int o0 = (int)((long long)G * D * rank / C), o1 = (int)((long long)G * D * (rank + 1) / C);
+        const size_t bq0 = (size_t)b * a.H_q + (size_t)h * G;
+        for (int i = o0 + tid; i < o1; i += NT) {
+            const int gg = i / D, dd = i - gg * D;
+            float s = 0.f;
+            for (uint32_t cr = 0; cr < C; ++cr) s += ld_dsmem_f32(dsmem(&sh.ocat[gg][dd], cr));
+            a.out[(bq0 + gg) * D + dd] = s;
+        }
+        if (rank == 0 && tid < G)
+            a.stat[bq0 + tid] = sh.zmax[tid] == -INFINITY ? -INFINITY : (float)((double)sh.zmax[tid] + sh.tau[tid]);
+    }
+    cluster_sync();  // no CTA leaves while another may still read its partial output
+    pdl_trigger();
+}
+
+// Dynamic shared memory of the kernel for `ent_cap` pages per CTA.
+static size_t att_smem_bytes(int ent_cap, int P, int G)
+{
+    const size_t ntok = (size_t)ent_cap * P, tiles = (size_t)ent_cap * (P / 16);
+    return (size_t)kAttWarps * kAttStageBytes + sizeof(float) * G * ntok + 2 * sizeof(int) * ent_cap +
+           sizeof(float) * G * tiles;
+}
+
+constexpr size_t kAttSmemMax = 227 * 1024;
+
+template <int D, int G>
+static cudaError_t launch_attend_t(const AttArgs &a0, cudaStream_t st, bool pdl, bool *launched)
+{
+    auto k = step_attend_kernel<D, G>;
+    const ekv_cache &c = a0.c;
+    *launched = false;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int pairs = c.batch * c.num_kv_heads;
+    const size_t stat_bytes = sizeof(AttShared<D, G>);
+    int C = 1;
+    while (C < 16 && (long long)pairs * C * 2 <= sms) C *= 2;
+    auto smem_for = [&](int Cc) { return att_smem_bytes((a0.max_sel + Cc - 1) / Cc, c.page_size, G); };
+    while (C <= 16 && smem_for(C) + stat_bytes > kAttSmemMax) C *= 2;
+    // not served (the caller takes the chunk kernels): a selection too large for 16 CTAs, or
+    // clusters that would not all be resident at once
+    if (C > 16 || (C > 1 && (long long)pairs * C > sms)) return cudaSuccess;
+    static bool attr_set = false;  // per instantiation
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)(kAttSmemMax - stat_bytes));
+        if (e == cudaSuccess) e = cudaFuncSetAttribute(k, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    AttArgs a = a0;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = C;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(kAttThreads);
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 2 : 1;
+    auto set_c = [&](int Cc) {
+        a.ent_cap = (a0.max_sel + Cc - 1) / Cc;
+        attr[0].val.clusterDim.x = Cc;
+        cfg.gridDim = dim3((unsigned)(pairs * Cc));
+        cfg.dynamicSmemBytes = smem_for(Cc);
+    };
+    set_c(C);
+    // a smaller cluster when the GPU cannot hold every cluster of this size at once
+    for (;;) {
+        int active = 0;
+        if (cudaOccupancyMaxActiveClusters(&active, (const void *)k, &cfg) != cudaSuccess) active = 0;
+        const int Cn = C / 2;
+        if (active >= pairs || Cn < 1 || smem_for(Cn) + stat_bytes > kAttSmemMax) break;
+        C = Cn;
+        set_c(C);
+    }
+    *launched = true;
+    return cudaLaunchKernelEx(&cfg, k, a);
+}
+
+// Launches the cluster attention when it serves the call (bf16, entmax, P a multiple of 16,
+// d in {64, 128}, G <= 8, the selection fits the cluster's shared memory); otherwise launches
+// nothing and leaves *launched false.
+cudaError_t launch_step_attend(const ekv_cache &c, const void *q, int H_q, float scale, int attn,
+                               const int32_t *sel_idx, const int32_t *sel_count, int max_sel,
+                               float *out, float *stat, cudaStream_t st, bool pdl, bool *launched)
+{
+    *launched = false;
+    if (c.dtype != EKV_BF16 || attn == EKV_SOFTMAX || c.page_size % 16 != 0) return cudaSuccess;
+    AttArgs a;
+    a.c = c;
+    a.q = q;
+    a.H_q = H_q;
+    const float alpha = attn == EKV_ENTMAX15 ? 1.5f : 2.0f;
+    a.qscale = scale * (alpha - 1.0f);
+    a.sparsemax = attn == EKV_SPARSEMAX;
+    a.sel_idx = sel_idx;
+    a.sel_count = sel_count;
+    a.max_sel = max_sel;
+    a.out = out;
+    a.stat = stat;
+    a.ent_cap = max_sel;
+    const int G = H_q / c.num_kv_heads;
+    if (c.head_dim == 128) {
+        switch (G) {
+        case 1: return launch_attend_t<128, 1>(a, st, pdl, launched);
+        case 2: return launch_attend_t<128, 2>(a, st, pdl, launched);
+        case 4: return launch_attend_t<128, 4>(a, st, pdl, launched);
+        default: return launch_attend_t<128, 8>(a, st, pdl, launched);
+        }
+    }
+    switch (G) {
+    case 1: return launch_attend_t<64, 1>(a, st, pdl, launched);
+    case 2: return launch_attend_t<64, 2>(a, st, pdl, launched);
+    case 4: return launch_attend_t<64, 4>(a, st, pdl, launched);
+    default: return launch_attend_t<64, 8>(a, st, pdl, launched);
+    }
+}
+
+}  // namespace ekv
