@@ -111,17 +111,25 @@ moment_update_kernel(ekv_cache c, float *__restrict__ moments, const int32_t *__
 
 // Sums over the selected tokens of one (sequence, KV head), eight selected pages per CTA:
 // n_R, sum_R k, sum_R v and u_g = sum_R v (k . q_g) for the G queries, added with atomics to a
-// zeroed [B * H_kv][retained_floats(d, G)] region.
+// zeroed [B * H_kv][retained_floats(d, G)] region. A half-warp takes one token row at a time:
+// lane l of the half reads the 16-byte pieces l of the K and V rows (8 coordinates each), the
+// G dot products k . q_g are summed over the half's lanes, and each lane keeps its coordinates
+// of sum k, sum v and u_g in registers; the CTA adds its partial sums once at the end.
 template <int DT, int D, int G>
 __global__ void __launch_bounds__(256)
 moment_retained_kernel(ekv_cache c, const void *__restrict__ q, int H_q,
                        const int32_t *__restrict__ sel_idx, const int32_t *__restrict__ sel_count,
                        int max_sel, float *__restrict__ ret)
 {
-    constexpr int PPC = 8;  // selected pages per CTA
-    constexpr int SUB = 16; // token rows staged at a time
-    __shared__ float qs[G][D], ks[SUB][D], vs[SUB][D], dots[SUB][G];
-    const int tid = threadIdx.x;
+    constexpr int PPC = 8;                         // selected pages per CTA
+    constexpr int EPC = Chunk<DT>::N;              // coordinates per 16-byte piece
+    constexpr int W = D * Chunk<DT>::kBytes / 16;  // pieces per row
+    constexpr int PPL = (W + 15) / 16;             // pieces per lane of a half-warp
+    __shared__ int s_blk[PPC], s_nt[PPC];
+    __shared__ float red[8][2 * D + G * D];
+    __shared__ int s_cnt[8];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int half = lane >> 4, hl = lane & 15;
     const int bh = blockIdx.y, b = bh / c.num_kv_heads, h = bh % c.num_kv_heads;
     const int P = c.page_size;
     int ns = sel_count[bh];
@@ -130,58 +138,124 @@ moment_retained_kernel(ekv_cache c, const void *__restrict__ q, int H_q,
     if (i0 >= ns) return;
     int len;
     const int np = seq_pages(c.seq_lens, b, P, c.max_pages, nullptr, &len);
-    for (int i = tid; i < G * D; i += 256)
-        qs[i / D][i % D] = load_elem<DT>(q, ((size_t)b * H_q + (size_t)h * G + i / D) * D + i % D);
-    float sk = 0.f, sv = 0.f, u[G];
-#pragma unroll
-    for (int g = 0; g < G; ++g) u[g] = 0.f;
-    int counted = 0;
-    // a page at a time, in groups of SUB token rows (an invalid page or selection counts
-    // nothing; the decode flags it)
-    for (int i = i0; i < i0 + PPC && i < ns; ++i) {
-        const int j = sel_idx[(size_t)bh * max_sel + i];
+    if (tid < PPC) {  // an invalid page or selection counts nothing; the decode flags it
+        const int i = i0 + tid;
         int blk = -1, nt = 0;
-        if (j >= 0 && j < np) {
-            blk = c.page_table[(size_t)b * c.max_pages + j];
-            if (blk >= 0 && blk < c.num_blocks) nt = len - j * P < P ? len - j * P : P;
+        if (i < ns) {
+            const int j = sel_idx[(size_t)bh * max_sel + i];
+            if (j >= 0 && j < np) {
+                blk = c.page_table[(size_t)b * c.max_pages + j];
+                if (blk >= 0 && blk < c.num_blocks) nt = len - j * P < P ? len - j * P : P;
+                else blk = -1;
+            }
         }
-        const size_t row0 = ((size_t)(blk < 0 ? 0 : blk) * c.num_kv_heads + h) * P;
-        for (int r0 = 0; r0 < nt; r0 += SUB) {
-            const int nr = nt - r0 < SUB ? nt - r0 : SUB;
-            __syncthreads();  // the previous rows are no longer read
-            for (int e = tid; e < nr * D; e += 256) {
-                ks[e / D][e % D] = load_elem<DT>(c.k_cache, (row0 + r0) * D + e);
-                vs[e / D][e % D] = load_elem<DT>(c.v_cache, (row0 + r0) * D + e);
-            }
-            __syncthreads();
-            for (int e = tid; e < nr * G; e += 256) {
-                const int t = e / G, g = e % G;
-                float acc = 0.f;
-                for (int cc = 0; cc < D; ++cc) acc = fmaf(qs[g][cc], ks[t][cc], acc);
-                dots[t][g] = acc;
-            }
-            __syncthreads();
-            counted += nr;
-            if (tid < D) {
-                for (int t = 0; t < nr; ++t) {
-                    const float v = vs[t][tid];
-                    sv += v;
+        s_blk[tid] = blk;
+        s_nt[tid] = nt;
+    }
+    // lane hl of a half-warp owns pieces hl + 16 k (k < PPL) of a row: coordinates
+    // [(hl + 16 k) * EPC, (hl + 16 k + 1) * EPC)
+    auto owns = [&](int k) { return hl + 16 * k < W; };
+    float qv[G][PPL][EPC];
 #pragma unroll
-                    for (int g = 0; g < G; ++g) u[g] = fmaf(v, dots[t][g], u[g]);
-                }
-            } else if (tid < 2 * D) {
-                for (int t = 0; t < nr; ++t) sk += ks[t][tid - D];
+    for (int g = 0; g < G; ++g)
+#pragma unroll
+        for (int k = 0; k < PPL; ++k)
+#pragma unroll
+            for (int e = 0; e < EPC; ++e)
+                qv[g][k][e] = owns(k) ? load_elem<DT>(q, ((size_t)b * H_q + (size_t)h * G + g) * D +
+                                                             (hl + 16 * k) * EPC + e)
+                                      : 0.f;
+    float sk[PPL][EPC], sv[PPL][EPC], u[G][PPL][EPC];
+#pragma unroll
+    for (int k = 0; k < PPL; ++k)
+#pragma unroll
+        for (int e = 0; e < EPC; ++e) {
+            sk[k][e] = 0.f;
+            sv[k][e] = 0.f;
+#pragma unroll
+            for (int g = 0; g < G; ++g) u[g][k][e] = 0.f;
+        }
+    int counted = 0;
+    __syncthreads();
+    const char *kc = static_cast<const char *>(c.k_cache), *vc = static_cast<const char *>(c.v_cache);
+    constexpr int RB = D * Chunk<DT>::kBytes;
+    for (int rho = warp * 2 + half; rho < PPC * P; rho += 16) {
+        const int slot = rho / P, t = rho - slot * P;
+        const bool valid = t < s_nt[slot];
+        const size_t row = ((size_t)(valid ? s_blk[slot] : 0) * c.num_kv_heads + h) * P + t;
+        float kf[PPL][EPC], vf[PPL][EPC];
+#pragma unroll
+        for (int k = 0; k < PPL; ++k) {
+            if (valid && owns(k)) {
+                Chunk<DT>::unpack(ld_stream16(kc + row * RB + (hl + 16 * k) * 16), kf[k]);
+                Chunk<DT>::unpack(ld_stream16(vc + row * RB + (hl + 16 * k) * 16), vf[k]);
+            } else {
+#pragma unroll
+                for (int e = 0; e < EPC; ++e) { kf[k][e] = 0.f; vf[k][e] = 0.f; }
+            }
+        }
+        float dot[G];
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            float acc = 0.f;
+#pragma unroll
+            for (int k = 0; k < PPL; ++k)
+#pragma unroll
+                for (int e = 0; e < EPC; ++e) acc = fmaf(qv[g][k][e], kf[k][e], acc);
+#pragma unroll
+            for (int o = 1; o < 16; o <<= 1) acc += __shfl_xor_sync(kFull, acc, o);
+            dot[g] = acc;
+        }
+#pragma unroll
+        for (int k = 0; k < PPL; ++k)
+#pragma unroll
+            for (int e = 0; e < EPC; ++e) {
+                sk[k][e] += kf[k][e];
+                sv[k][e] += vf[k][e];
+#pragma unroll
+                for (int g = 0; g < G; ++g) u[g][k][e] = fmaf(vf[k][e], dot[g], u[g][k][e]);
+            }
+        counted += valid;
+    }
+    // the two half-warps' rows, then the warps
+#pragma unroll
+    for (int k = 0; k < PPL; ++k)
+#pragma unroll
+        for (int e = 0; e < EPC; ++e) {
+            sk[k][e] += __shfl_xor_sync(kFull, sk[k][e], 16);
+            sv[k][e] += __shfl_xor_sync(kFull, sv[k][e], 16);
+#pragma unroll
+            for (int g = 0; g < G; ++g) u[g][k][e] += __shfl_xor_sync(kFull, u[g][k][e], 16);
+        }
+    counted += __shfl_xor_sync(kFull, counted, 16);
+    if (half == 0) {
+#pragma unroll
+        for (int k = 0; k < PPL; ++k) {
+            if (!owns(k)) continue;
+            const int c0 = (hl + 16 * k) * EPC;
+#pragma unroll
+            for (int e = 0; e < EPC; ++e) {
+                red[warp][c0 + e] = sk[k][e];
+                red[warp][D + c0 + e] = sv[k][e];
+#pragma unroll
+                for (int g = 0; g < G; ++g) red[warp][2 * D + g * D + c0 + e] = u[g][k][e];
             }
         }
     }
+    if (lane == 0) s_cnt[warp] = counted;
+    __syncthreads();
     float *r = ret + (size_t)bh * retained_floats(D, G);
-    if (tid == 0) atomicAdd(r, (float)counted);
-    if (tid < D) {
-        atomicAdd(r + 4 + D + tid, sv);
+    for (int i = tid; i < 2 * D + G * D; i += 256) {
+        float sum = 0.f;
 #pragma unroll
-        for (int g = 0; g < G; ++g) atomicAdd(r + 4 + 2 * D + g * D + tid, u[g]);
-    } else if (tid < 2 * D) {
-        atomicAdd(r + 4 + (tid - D), sk);
+        for (int w = 0; w < 8; ++w) sum += red[w][i];
+        atomicAdd(r + 4 + i, sum);
+    }
+    if (tid == 0) {
+        int n = 0;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) n += s_cnt[w];
+        atomicAdd(r, (float)n);
     }
 }
 
@@ -215,13 +289,23 @@ moment_correct_kernel(ekv_cache c, const float *__restrict__ moments, const void
     float qk = 0.f;
 #pragma unroll
     for (int w = 0; w < 8; ++w) qk += red[w];
-    // (sum v k^T) q, one row per warp step: lane l reads coordinates l, l + 32, ...
+    // (sum v k^T) q: warp w takes rows a = w, w + 8, ... (D / 8 of them), lane l coordinates
+    // l, l + 32, ...; every row's loads are issued before any product, so they are in flight
+    // together
     const float *S = rec + 4 + 2 * D;
-    for (int a = warp; a < D; a += 8) {
+    constexpr int RPW = D / 8, CPL = D / 32;
+    float sv[RPW][CPL];
+#pragma unroll
+    for (int i = 0; i < RPW; ++i)
+#pragma unroll
+        for (int k = 0; k < CPL; ++k) sv[i][k] = __ldg(S + (size_t)(warp + 8 * i) * D + lane + 32 * k);
+#pragma unroll
+    for (int i = 0; i < RPW; ++i) {
         float acc = 0.f;
 #pragma unroll
-        for (int cc = lane; cc < D; cc += 32) acc = fmaf(S[(size_t)a * D + cc], qs[cc], acc);
+        for (int k = 0; k < CPL; ++k) acc = fmaf(sv[i][k], qs[lane + 32 * k], acc);
         acc = warp_sum(acc);
+        const int a = warp + 8 * i;
         if (lane == 0) sq[a] = acc - r[4 + 2 * D + g * D + a];  // sum_E v (k.q)
     }
     __syncthreads();

@@ -453,34 +453,40 @@ static size_t att_smem_bytes(int ent_cap, int P, int G)
            sizeof(float) * G * tiles;
 }
 
-constexpr size_t kAttSmemMax = 227 * 1024;
-
 template <int D, int G>
 static cudaError_t launch_attend_t(const AttArgs &a0, cudaStream_t st, bool pdl, bool *launched)
 {
     auto k = step_attend_kernel<D, G>;
     const ekv_cache &c = a0.c;
     *launched = false;
-    int dev = 0, sms = 148;
+    int dev = 0, sms = 148, optin = 0;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    // the kernel's own static shared memory, as compiled, bounds the dynamic part
+    static size_t stat_bytes = 0;  // per instantiation
+    static bool attr_set = false, attr_ok = false;
+    if (!attr_set) {
+        attr_set = true;
+        cudaFuncAttributes fa;
+        if (cudaFuncGetAttributes(&fa, k) == cudaSuccess && (size_t)optin > fa.sharedSizeBytes) {
+            stat_bytes = fa.sharedSizeBytes;
+            attr_ok = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           (int)((size_t)optin - stat_bytes)) == cudaSuccess &&
+                      cudaFuncSetAttribute(k, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess;
+        }
+        if (!attr_ok) cudaGetLastError();  // not served; leave no error behind for later calls
+    }
+    if (!attr_ok) return cudaSuccess;
+    const size_t dyn_max = (size_t)optin - stat_bytes;
     const int pairs = c.batch * c.num_kv_heads;
-    const size_t stat_bytes = sizeof(AttShared<D, G>);
     int C = 1;
     while (C < 16 && (long long)pairs * C * 2 <= sms) C *= 2;
     auto smem_for = [&](int Cc) { return att_smem_bytes((a0.max_sel + Cc - 1) / Cc, c.page_size, G); };
-    while (C <= 16 && smem_for(C) + stat_bytes > kAttSmemMax) C *= 2;
+    while (C <= 16 && smem_for(C) > dyn_max) C *= 2;
     // not served (the caller takes the chunk kernels): a selection too large for 16 CTAs, or
     // clusters that would not all be resident at once
     if (C > 16 || (C > 1 && (long long)pairs * C > sms)) return cudaSuccess;
-    static bool attr_set = false;  // per instantiation
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)(kAttSmemMax - stat_bytes));
-        if (e == cudaSuccess) e = cudaFuncSetAttribute(k, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
     AttArgs a = a0;
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -504,9 +510,12 @@ static cudaError_t launch_attend_t(const AttArgs &a0, cudaStream_t st, bool pdl,
     // a smaller cluster when the GPU cannot hold every cluster of this size at once
     for (;;) {
         int active = 0;
-        if (cudaOccupancyMaxActiveClusters(&active, (const void *)k, &cfg) != cudaSuccess) active = 0;
+        if (cudaOccupancyMaxActiveClusters(&active, (const void *)k, &cfg) != cudaSuccess) {
+            cudaGetLastError();
+            active = 0;
+        }
         const int Cn = C / 2;
-        if (active >= pairs || Cn < 1 || smem_for(Cn) + stat_bytes > kAttSmemMax) break;
+        if (active >= pairs || Cn < 1 || smem_for(Cn) > dyn_max) break;
         C = Cn;
         set_c(C);
     }

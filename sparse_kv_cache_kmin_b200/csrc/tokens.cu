@@ -14,8 +14,11 @@
 
 namespace ekv {
 
-// One CTA per (8 selected pages, sequence x KV head). The group query sum Q = sum_g q_g is in
-// shared memory; a warp scores one token row at a time (lane l reads elements l, l + 32, ...).
+constexpr int kTokRowsSmem = 16384;  // kept tokens whose cache rows the attention keeps on chip
+
+// One CTA per (8 selected pages, sequence x KV head). A half-warp scores four token rows at a
+// time: lane l of the half reads the 16-byte pieces l (+16) of each row and holds the matching
+// coordinates of the group query sum Q = sum_g q_g; the partial dots are summed over the half.
 template <int DT, int D, int G>
 __global__ void __launch_bounds__(256)
 token_score_kernel(ekv_cache c, const void *__restrict__ q, int H_q, float scale,
@@ -23,10 +26,12 @@ token_score_kernel(ekv_cache c, const void *__restrict__ q, int H_q, float scale
                    int max_sel, float *__restrict__ tscores)
 {
     constexpr int PPC = 8;
-    __shared__ float qsum[D];
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    constexpr int EPC = Chunk<DT>::N, RB = D * Chunk<DT>::kBytes, W = RB / 16, PPL = (W + 15) / 16;
+    constexpr int RIF = 4;  // rows in flight per half-warp
+    __shared__ int s_blk[PPC], s_nt[PPC];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, half = lane >> 4, hl = lane & 15;
     const int bh = blockIdx.y, b = bh / c.num_kv_heads, h = bh % c.num_kv_heads;
-    const int P = c.page_size;
+    const int H = c.num_kv_heads, P = c.page_size;
     pdl_wait();
     int ns = sel_count[bh];
     ns = ns < 0 ? 0 : (ns > max_sel ? max_sel : ns);
@@ -34,35 +39,73 @@ token_score_kernel(ekv_cache c, const void *__restrict__ q, int H_q, float scale
     if (i0 >= ns) return;
     int len;
     const int np = seq_pages(c.seq_lens, b, P, c.max_pages, nullptr, &len);
-    for (int e = tid; e < D; e += 256) {
-        float s = 0.f;
-#pragma unroll
-        for (int g = 0; g < G; ++g) s += load_elem<DT>(q, ((size_t)b * H_q + (size_t)h * G + g) * D + e);
-        qsum[e] = s;
-    }
-    __syncthreads();
-    float *out = tscores + (size_t)bh * max_sel * P;
-    const int i1 = i0 + PPC < ns ? i0 + PPC : ns;
-    for (int r = warp; r < (i1 - i0) * P; r += 8) {
-        const int i = i0 + r / P, t = r % P;
-        const int j = sel_idx[(size_t)bh * max_sel + i];
-        int blk = -1;
-        if (j < 0 || j >= np) {
-            if (t == 0 && lane == 0) flag(c.dev_status, EKV_DEV_BAD_SEL);
-        } else if (j * P + t < len) {
-            blk = c.page_table[(size_t)b * c.max_pages + j];
-            if (blk < 0 || blk >= c.num_blocks) {
-                if (lane == 0) flag(c.dev_status, EKV_DEV_BAD_BLOCK);
-                blk = -1;
+    if (tid < PPC) {
+        const int i = i0 + tid;
+        int blk = -1, nt = 0;
+        if (i < ns) {
+            const int j = sel_idx[(size_t)bh * max_sel + i];
+            if (j < 0 || j >= np) {
+                flag(c.dev_status, EKV_DEV_BAD_SEL);
+            } else {
+                const int bk = c.page_table[(size_t)b * c.max_pages + j];
+                if (bk < 0 || bk >= c.num_blocks) {
+                    flag(c.dev_status, EKV_DEV_BAD_BLOCK);
+                } else {
+                    blk = bk;
+                    nt = len - j * P < P ? len - j * P : P;
+                }
             }
         }
-        float acc = 0.f;
-        if (blk >= 0) {
-            const size_t row = ((size_t)blk * c.num_kv_heads + h) * P + t;
-            for (int e = lane; e < D; e += 32) acc = fmaf(qsum[e], load_elem<DT>(c.k_cache, row * D + e), acc);
-            acc = warp_sum(acc);
+        s_blk[tid] = blk;
+        s_nt[tid] = nt;
+    }
+    auto owns = [&](int k) { return hl + 16 * k < W; };
+    float qv[PPL][EPC];
+#pragma unroll
+    for (int k = 0; k < PPL; ++k)
+#pragma unroll
+        for (int e = 0; e < EPC; ++e) {
+            float sum = 0.f;
+            if (owns(k))
+#pragma unroll
+                for (int g = 0; g < G; ++g)
+                    sum += load_elem<DT>(q, ((size_t)b * H_q + (size_t)h * G + g) * D + (hl + 16 * k) * EPC + e);
+            qv[k][e] = sum;
         }
-        if (lane == 0) out[(size_t)i * P + t] = blk >= 0 ? scale * acc : -INFINITY;
+    __syncthreads();
+    const int i1 = i0 + PPC < ns ? i0 + PPC : ns;
+    const int nrows = (i1 - i0) * P;
+    float *out = tscores + (size_t)bh * max_sel * P + (size_t)i0 * P;
+    const char *kc = static_cast<const char *>(c.k_cache);
+    for (int base = (warp * 2 + half) * RIF; base < nrows; base += 16 * RIF) {
+        float kf[RIF][PPL][EPC];
+        bool ok[RIF];
+#pragma unroll
+        for (int r = 0; r < RIF; ++r) {
+            const int rr = base + r, slot = rr / P, t = rr - slot * P;
+            ok[r] = rr < nrows && t < s_nt[slot < PPC ? slot : 0];
+            const size_t row = ((size_t)(ok[r] ? s_blk[slot] : 0) * H + h) * P + t;
+#pragma unroll
+            for (int k = 0; k < PPL; ++k) {
+                if (ok[r] && owns(k)) {
+                    Chunk<DT>::unpack(ld_stream16(kc + row * RB + (hl + 16 * k) * 16), kf[r][k]);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < EPC; ++e) kf[r][k][e] = 0.f;
+                }
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < RIF; ++r) {
+            float acc = 0.f;
+#pragma unroll
+            for (int k = 0; k < PPL; ++k)
+#pragma unroll
+                for (int e = 0; e < EPC; ++e) acc = fmaf(qv[k][e], kf[r][k][e], acc);
+#pragma unroll
+            for (int o = 1; o < 16; o <<= 1) acc += __shfl_xor_sync(kFull, acc, o);
+            if (hl == 0 && base + r < nrows) out[base + r] = ok[r] ? scale * acc : -INFINITY;
+        }
     }
     pdl_trigger();
 }
@@ -111,16 +154,60 @@ token_attend_kernel(ekv_cache c, const void *__restrict__ q, int H_q, float scal
         return ((long long)blk * c.num_kv_heads + h) * P + t;
     };
     const float alpha = attn == EKV_SOFTMAX ? 1.f : (attn == EKV_ENTMAX15 ? 1.5f : 2.f);
-    for (int i = warp; i < n; i += 8) {
-        const long long row = row_of(i);
-        float acc = 0.f;
-        if (row >= 0) {
-            for (int e = lane; e < D; e += 32) acc = fmaf(qs[e], load_elem<DT>(c.k_cache, (size_t)row * D + e), acc);
-            acc = warp_sum(acc);
+    const float zscale = scale * (attn == EKV_SOFTMAX ? 1.f : alpha - 1.f);
+    // the cache row of every kept token, resolved once (all lookups in flight together); for
+    // T beyond the shared-memory rows the lookups are repeated where needed
+    constexpr int EPC = Chunk<DT>::N, RB = D * Chunk<DT>::kBytes, W = RB / 16, PPL = (W + 15) / 16;
+    constexpr int RIF = 4;  // rows in flight per half-warp
+    const bool rows_smem = T <= kTokRowsSmem;
+    long long *rows = reinterpret_cast<long long *>(zs + ((T + 1) & ~1));  // [T] when rows_smem
+    if (rows_smem) {
+        for (int i = tid; i < n; i += 256) {
+            const long long r = row_of(i);
+            if (r < 0) flag(c.dev_status, EKV_DEV_BAD_SEL);
+            rows[i] = r;
         }
-        if (lane == 0) {
-            if (row < 0) flag(c.dev_status, EKV_DEV_BAD_SEL);
-            zs[i] = row >= 0 ? scale * acc * (attn == EKV_SOFTMAX ? 1.f : alpha - 1.f) : -INFINITY;
+    } else {
+        for (int i = tid; i < n; i += 256)
+            if (row_of(i) < 0) flag(c.dev_status, EKV_DEV_BAD_SEL);
+    }
+    __syncthreads();
+    auto row_at = [&](int i) { return rows_smem ? rows[i] : row_of(i); };
+    const int half = lane >> 4, hl = lane & 15;
+    auto owns = [&](int k) { return hl + 16 * k < W; };
+    float qv[PPL][EPC];
+#pragma unroll
+    for (int k = 0; k < PPL; ++k)
+#pragma unroll
+        for (int e = 0; e < EPC; ++e) qv[k][e] = owns(k) ? qs[(hl + 16 * k) * EPC + e] : 0.f;
+    const char *kc = static_cast<const char *>(c.k_cache), *vc = static_cast<const char *>(c.v_cache);
+    // logits: a half-warp takes RIF rows at a time, lane l reading pieces l (+16) of each
+    for (int base = (warp * 2 + half) * RIF; base < n; base += 16 * RIF) {
+        float kf[RIF][PPL][EPC];
+        long long rw[RIF];
+#pragma unroll
+        for (int r = 0; r < RIF; ++r) {
+            rw[r] = base + r < n ? row_at(base + r) : -1;
+#pragma unroll
+            for (int k = 0; k < PPL; ++k) {
+                if (rw[r] >= 0 && owns(k)) {
+                    Chunk<DT>::unpack(ld_stream16(kc + (size_t)rw[r] * RB + (hl + 16 * k) * 16), kf[r][k]);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < EPC; ++e) kf[r][k][e] = 0.f;
+                }
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < RIF; ++r) {
+            float acc = 0.f;
+#pragma unroll
+            for (int k = 0; k < PPL; ++k)
+#pragma unroll
+                for (int e = 0; e < EPC; ++e) acc = fmaf(qv[k][e], kf[r][k][e], acc);
+#pragma unroll
+            for (int o = 1; o < 16; o <<= 1) acc += __shfl_xor_sync(kFull, acc, o);
+            if (hl == 0 && base + r < n) zs[base + r] = rw[r] >= 0 ? zscale * acc : -INFINITY;
         }
     }
     __syncthreads();
@@ -200,15 +287,54 @@ token_attend_kernel(ekv_cache c, const void *__restrict__ q, int H_q, float scal
         st = (float)tau;
     }
     __syncthreads();
-    for (int a = tid; a < D; a += 256) {
-        float acc = 0.f;
-        for (int i = 0; i < n; ++i) {
-            const float p = zs[i];
-            if (p == 0.f) continue;
-            const long long row = row_of(i);
-            if (row >= 0) acc = fmaf(p, load_elem<DT>(c.v_cache, (size_t)row * D + a), acc);
+    // out = sum p_i v_i over the rows with p_i > 0: a half-warp takes RIF rows at a time, each
+    // lane accumulating its coordinates; then the halves and the warps are summed in order
+    float acc[PPL][EPC];
+#pragma unroll
+    for (int k = 0; k < PPL; ++k)
+#pragma unroll
+        for (int e = 0; e < EPC; ++e) acc[k][e] = 0.f;
+    for (int base = (warp * 2 + half) * RIF; base < n; base += 16 * RIF) {
+        float vf[RIF][PPL][EPC], pr[RIF];
+#pragma unroll
+        for (int r = 0; r < RIF; ++r) {
+            pr[r] = base + r < n ? zs[base + r] : 0.f;
+            const long long rw = pr[r] != 0.f ? row_at(base + r) : -1;
+#pragma unroll
+            for (int k = 0; k < PPL; ++k) {
+                if (rw >= 0 && owns(k)) {
+                    Chunk<DT>::unpack(ld_stream16(vc + (size_t)rw * RB + (hl + 16 * k) * 16), vf[r][k]);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < EPC; ++e) vf[r][k][e] = 0.f;
+                }
+            }
         }
-        out[bq * D + a] = acc;
+#pragma unroll
+        for (int r = 0; r < RIF; ++r)
+#pragma unroll
+            for (int k = 0; k < PPL; ++k)
+#pragma unroll
+                for (int e = 0; e < EPC; ++e) acc[k][e] = fmaf(pr[r], vf[r][k][e], acc[k][e]);
+    }
+    __shared__ float opart[8][D];
+#pragma unroll
+    for (int k = 0; k < PPL; ++k)
+#pragma unroll
+        for (int e = 0; e < EPC; ++e) acc[k][e] += __shfl_xor_sync(kFull, acc[k][e], 16);
+    if (half == 0) {
+#pragma unroll
+        for (int k = 0; k < PPL; ++k)
+            if (owns(k))
+#pragma unroll
+                for (int e = 0; e < EPC; ++e) opart[warp][(hl + 16 * k) * EPC + e] = acc[k][e];
+    }
+    __syncthreads();
+    for (int a = tid; a < D; a += 256) {
+        float sum = 0.f;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) sum += opart[w][a];
+        out[bq * D + a] = sum;
     }
     if (tid == 0) stat[bq] = st;
 }
@@ -230,7 +356,9 @@ static cudaError_t launch_attend_t(const ekv_cache &c, const void *q, int H_q, f
                                    cudaStream_t st)
 {
     auto k = token_attend_kernel<DT, D, G>;
-    const size_t smem = sizeof(float) * (size_t)T;
+    // the logits, then (up to kTokRowsSmem tokens) the kept tokens' cache rows
+    const size_t smem = sizeof(float) * (size_t)((T + 1) & ~1) +
+                        (T <= kTokRowsSmem ? sizeof(long long) * (size_t)T : 0);
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
