@@ -61,6 +61,9 @@ def parse():
                     help="override the workload's batch (smaller cases for profiler captures)")
     ap.add_argument("--no-full-cache", action="store_true",
                     help="skip the full-cache decode (every page selected) timed for comparison")
+    ap.add_argument("--fused-select", action="store_true",
+                    help="top-k scores and selection through the one-launch cluster kernel "
+                         "(ekv_score_select_pages) instead of the two calls")
     ap.add_argument("--policy", default=None, choices=["topk", "gauss", "gauss_max"],
                     help="selection policy (default: the workload's); gauss_max is the estimated-"
                          "maximum reading of the Gaussian rule")
@@ -381,7 +384,7 @@ class Step:
     """The public calls of one decode step of a variant, as (name, fn) pairs, with the buffers
     they write. Every call goes through the C ABI binding; nothing here computes."""
 
-    def __init__(self, ekv, SparseDecoder, cache, wl, attn, variant, T):
+    def __init__(self, ekv, SparseDecoder, cache, wl, attn, variant, T, fused_select=False):
         self.wl, self.variant, self.T = wl, variant, T
         dev = wl.k_cache.device
         B, H = wl.batch, wl.num_kv_heads
@@ -395,8 +398,8 @@ class Step:
             calls.append(("meta", lambda: ekv.ekv_page_meta_update(cache, ap_start, ap_count,
                                                                    wl.append[1])))
         q = wl.q
-        if wl.policy == 0:
-            # top-k: scores and selection in one launch (one cluster per sequence and KV head)
+        if wl.policy == 0 and fused_select:
+            # top-k scores and selection in one launch (one cluster per sequence and KV head)
             calls.append(("score_select", lambda: ekv.ekv_score_select_pages(
                 cache, q, wl.num_q_heads, wl.scale, wl.topk, dec.scores, dec.sel_idx,
                 dec.sel_count, dec.max_sel)))
@@ -424,7 +427,8 @@ class Step:
                 tp, tt, tc, tws)))
             calls.append(("decode_tokens", lambda: ekv.ekv_sparse_decode_tokens(
                 cache, q, wl.num_q_heads, wl.scale, attn, tp, tt, tc, T, dec.out, dec.stat)))
-            self.kernels = {"score_select": 1, "select_tokens": 2, "decode_tokens": 1}
+            self.kernels = {"score_select": 1, "score": 1, "select": 1, "select_tokens": 2,
+                            "decode_tokens": 1}
         else:
             moments = torch.zeros(ekv.ekv_moment_bytes(cache) // 4, dtype=torch.float32, device=dev)
             ekv.ekv_moment_update(cache, moments, torch.zeros(B, dtype=torch.int32, device=dev),
@@ -436,7 +440,7 @@ class Step:
             calls.append(("decode_moment", lambda: ekv.ekv_sparse_decode_moment(
                 cache, moments, q, wl.num_q_heads, wl.scale, dec.sel_idx, dec.sel_count,
                 dec.max_sel, dec.out, dec.stat, mws)))
-            self.kernels = {"score_select": 1, "decode_moment": 4}
+            self.kernels = {"score_select": 1, "score": 1, "select": 1, "decode_moment": 4}
         self.calls = calls
 
     def launches(self):
@@ -577,7 +581,7 @@ def main():
     B = wl.batch
     ekv.ekv_page_meta_update(cache, torch.zeros(B, dtype=torch.int32, device=dev), wl.seq_lens,
                              int(wl.seq_lens.max()))
-    step = Step(ekv, SparseDecoder, cache, wl, attn, args.variant, T)
+    step = Step(ekv, SparseDecoder, cache, wl, attn, args.variant, T, args.fused_select)
     dec = step.dec
     stream = torch.cuda.current_stream()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
@@ -684,9 +688,9 @@ def main():
     ms = total_s / args.steps * 1e3
     dom = max((n for n in call_us if n in by), key=lambda n: call_us[n])
     traffic = None
-    if dom == "score_select" and args.workload == "needle128k":
+    if dom == "score" and args.workload == "needle128k":
         total_pages = int(((wl.seq_lens.long() + P - 1) // P).sum())
-        traffic = ncu_traffic("step.cu", "score_select_needle128k.md", total_pages * H)
+        traffic = ncu_traffic("score.cu", "score_pages_needle128k.md", total_pages * H)
     achieved = by[dom] / (call_us[dom] / 1e6) / 1e9
     frac_step = by["required_step"] / (ms / 1e3) / 1e9 / peak
     cpu = None

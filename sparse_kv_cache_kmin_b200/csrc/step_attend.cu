@@ -14,13 +14,15 @@
 // The threshold tau solves sum_i [z_i - tau]_+^(1/(alpha-1)) = 1 over all the pair's tokens,
 // which live in the cluster's distributed shared memory:
 //   1. The tile maxima are logits, and the exact threshold of any subset of the logits is at
-//      most tau (adding tokens only raises it). Each CTA reduces its tile maxima to 256 / C
-//      group maxima; one warp per query gathers all 256 (DSMEM) and solves them exactly
+//      most tau (adding tokens only raises it). Each CTA reduces its tile maxima to 64 / C
+//      group maxima; one warp per query gathers all 64 (DSMEM) and solves them exactly
 //      (bitonic sort, closed form) for zmax and a lower bound on tau.
 //   2. Every token above the lower bound is a candidate; each CTA lists its own in token order.
-//      With at most 512 candidates in the cluster, one warp per query gathers them and solves
-//      exactly. More (nearly flat logits): an fp64 bisection whose sums are reduced over the
-//      cluster, then the closed form over the support it brackets.
+//      Up to 128 candidates in the cluster: one warp per query gathers and sorts them. Up to
+//      512: the CTA gathers them and every thread ranks one candidate against all the others,
+//      summing the values above it, which gives the closed-form threshold of every support
+//      size at once. More (nearly flat logits): an fp64 bisection whose sums are reduced over
+//      the cluster, then the closed form over the support it brackets.
 //   3. Each CTA accumulates p_i v_i over its support tokens (V rows read only for those), in a
 //      fixed order; the CTAs' partial outputs are summed over DSMEM in rank order.
 #include "cluster.cuh"
@@ -32,8 +34,9 @@ namespace ekv {
 constexpr int kAttThreads = 512;
 constexpr int kAttWarps = kAttThreads / 32;
 constexpr int kAttStageBytes = 8192;  // per warp: 16 loads of 16 bytes per lane
-constexpr int kAttGroups = 256;       // lower-bound maxima per query over the cluster
-constexpr int kAttCand = 512;         // candidates per query solved by one warp (16 per lane)
+constexpr int kAttGroups = 64;        // lower-bound maxima per query over the cluster (2 per lane)
+constexpr int kAttWarpCand = 128;     // candidates one warp solves by sorting (4 per lane)
+constexpr int kAttCand = 512;         // candidates the CTA solves by ranking
 
 struct AttArgs {
     ekv_cache c;
@@ -57,7 +60,8 @@ struct AttShared {
     int wcnt[kAttWarps];
     float zmax[G];
     double tlb[G], tau[G];
-    int fast[G];
+    int fast[G];                 // 0: bisection, 1: solved by a warp, 2: solve by ranking
+    int best_k;
     double fpart[2][G];          // bisection partial sums (read by the cluster)
     double cpart[3];             // closed-form partial sums (read by the cluster)
     double red[kAttWarps];
@@ -96,7 +100,7 @@ step_attend_kernel(AttArgs a)
     constexpr int TPS = kAttStageBytes / TB;  // tiles per warp step
     constexpr int KS = D / 16;                // MMA k-steps per tile
     static_assert(G <= 8, "one n = 8 MMA column block");
-    static_assert(G * (kAttGroups + 2 * kAttCand) * 4 <= kAttWarps * kAttStageBytes,
+    static_assert((G * (kAttGroups + 2 * kAttCand) + kAttCand) * 4 <= kAttWarps * kAttStageBytes,
                   "the lists fit on the staging buffers");
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ AttShared<D, G> sh;
@@ -116,6 +120,7 @@ step_attend_kernel(AttArgs a)
     float *gm = reinterpret_cast<float *>(smem);                 // [G][kAttGroups] group maxima
     float *cx = gm + G * kAttGroups;                             // [G][kAttCand] candidates z - zmax
     int *ct = reinterpret_cast<int *>(cx + G * kAttCand);        // [G][kAttCand] their tokens
+    float *gat = reinterpret_cast<float *>(ct + G * kAttCand);   // [kAttCand] gathered candidates
 
     pdl_wait();
     int len;
@@ -251,7 +256,7 @@ step_attend_kernel(AttArgs a)
         double lb = 0.0;
         if (zm > -INFINITY) {
             lb = warp_exact_tau<kAttGroups / 32>(v, cnt, a.sparsemax != 0);
-            // lowered a little so that the fp32 rounding of the bound (prefix sums of up to 256
+            // lowered a little so that the fp32 rounding of the bound (prefix sums of up to 64
             // values) never drops a support member
             lb -= 1e-5 * fmax(1.0, fabs(lb));
         }
@@ -293,37 +298,87 @@ step_attend_kernel(AttArgs a)
     cluster_sync();
 
     // ---------------------------------------------------------------- exact tau
-    if (warp < G) {
-        const int g = warp;
-        int offs[17];
+    int offs[17];  // per query, filled by warp g; the ranking path recomputes them
+    auto gather_offsets = [&](int g) {
         offs[0] = 0;
-        bool fits = true;
+        bool each_fits = true;
         for (uint32_t cr = 0; cr < C; ++cr) {
             const int n = ld_dsmem(dsmem(&sh.ccnt[g], cr));
-            fits = fits && n <= kAttCand;
+            each_fits = each_fits && n <= kAttCand;
             offs[cr + 1] = offs[cr] + n;
         }
-        const int total = offs[C];
-        fits = fits && total <= kAttCand;
+        return each_fits ? offs[C] : kAttCand + 1;
+    };
+    auto gathered = [&](int g, int idx) {  // candidate idx of query g, cluster-wide token order
+        uint32_t cr = 0;
+        while (idx >= offs[cr + 1]) ++cr;
+        return ld_dsmem_f32(dsmem(&cx[g * kAttCand + idx - offs[cr]], cr));
+    };
+    if (warp < G) {
+        const int g = warp;
+        const int total = gather_offsets(g);
         double tau = 0.0;
-        if (sh.zmax[g] > -INFINITY && fits) {
-            float v[kAttCand / 32];
+        int mode = 1;
+        if (sh.zmax[g] == -INFINITY) {
+            mode = 1;
+        } else if (total <= kAttWarpCand) {
+            float v[kAttWarpCand / 32];
 #pragma unroll
-            for (int r = 0; r < kAttCand / 32; ++r) {
+            for (int r = 0; r < kAttWarpCand / 32; ++r) {
                 const int idx = r * 32 + lane;
-                v[r] = -INFINITY;
-                if (idx < total) {
-                    uint32_t cr = 0;
-                    while (idx >= offs[cr + 1]) ++cr;
-                    v[r] = ld_dsmem_f32(dsmem(&cx[g * kAttCand + idx - offs[cr]], cr));
-                }
+                v[r] = idx < total ? gathered(g, idx) : -INFINITY;
             }
-            tau = warp_exact_tau<kAttCand / 32>(v, total, a.sparsemax != 0);
+            tau = warp_exact_tau<kAttWarpCand / 32>(v, total, a.sparsemax != 0);
+        } else {
+            mode = total <= kAttCand ? 2 : 0;
         }
         if (lane == 0) {
             sh.tau[g] = tau;
-            sh.fast[g] = sh.zmax[g] == -INFINITY || fits;
+            sh.fast[g] = mode;
         }
+    }
+    __syncthreads();
+    // Up to kAttCand candidates: every CTA gathers them and thread t ranks candidate t. With
+    // x_t the k-th largest (ties broken by position), S1 and S2 the sums of the k largest and
+    // of their squares give tau(k) in closed form; the support is the largest k with
+    // tau(k) <= x_(k) (the sort-based rule without the sort).
+    for (int g = 0; g < G; ++g) {
+        if (sh.fast[g] != 2) continue;
+        const int total = gather_offsets(g);
+        for (int i = tid; i < total; i += NT) gat[i] = gathered(g, i);
+        if (tid == 0) sh.best_k = 0;
+        __syncthreads();
+        int k = 0;
+        float tk = 0.f;
+        if (tid < total) {
+            const float x = gat[tid];
+            float s1 = x, s2 = x * x;
+            int rank = 0;
+            for (int j = 0; j < total; ++j) {
+                const float y = gat[j];
+                const bool before = y > x || (y == x && j < tid);
+                rank += before;
+                s1 += before ? y : 0.f;
+                s2 += before ? y * y : 0.f;
+            }
+            k = rank + 1;
+            const float kf = (float)k;
+            bool ok;
+            if (a.sparsemax) {
+                tk = (s1 - 1.0f) / kf;
+                ok = true;
+            } else {
+                const float mean = s1 / kf;
+                const float disc = (1.0f - fmaxf(s2 - s1 * mean, 0.f)) / kf;
+                ok = disc >= 0.f;
+                tk = mean - sqrtf(fmaxf(disc, 0.f));
+            }
+            if (!(ok && tk <= x)) k = 0;
+            if (k > 0) atomicMax(&sh.best_k, k);
+        }
+        __syncthreads();
+        if (k > 0 && k == sh.best_k) sh.tau[g] = (double)tk;
+        __syncthreads();  // gat is refilled for the next query
     }
     __syncthreads();
     // Too many candidates for one warp (nearly flat logits): fp64 bisection on
@@ -331,7 +386,7 @@ step_attend_kernel(AttArgs a)
     // it brackets. The decision is the same in every CTA (the same counts were read), so every
     // CTA takes the same cluster barriers.
     for (int g = 0; g < G; ++g) {
-        if (sh.fast[g]) continue;
+        if (sh.fast[g] != 0) continue;
         const float zm = sh.zmax[g];
         const float *zg = zs + (size_t)g * ntok_cap;
         double lo = sh.tlb[g], hi = 0.0;
@@ -399,7 +454,7 @@ step_attend_kernel(AttArgs a)
             }
         };
         if (zm > -INFINITY) {
-            if (sh.fast[g]) {
+            if (sh.fast[g] != 0) {
                 const int n = sh.ccnt[g];  // this CTA's candidates (<= kAttCand on this path)
                 for (int i = part * 2 + half; i < n; i += WPQ * 2) {
                     const double r = (double)cx[g * kAttCand + i] - tau;

@@ -72,15 +72,10 @@ class SparseDecoder:
 
     def step(self, q: torch.Tensor, stream=None):
         c = self.cache
-        if self.policy == ekv.EKV_SEL_TOPK:
-            # scores and selection in one launch (one cluster per sequence and KV head)
-            ekv.ekv_score_select_pages(c, q, self.num_q_heads, self.scale, self.topk, self.scores,
-                                       self.sel_idx, self.sel_count, self.max_sel, stream)
-        else:
-            ekv.ekv_score_pages(c, q, self.num_q_heads, self.scale, self.policy, self.scores, stream)
-            ekv.ekv_select_pages(c, self.num_q_heads, self.policy, self.topk, self.alpha,
-                                 self.delta, self.scores, self.sel_idx, self.sel_count,
-                                 self.max_sel, self.tau_hat, stream)
+        ekv.ekv_score_pages(c, q, self.num_q_heads, self.scale, self.policy, self.scores, stream)
+        ekv.ekv_select_pages(c, self.num_q_heads, self.policy, self.topk, self.alpha, self.delta,
+                             self.scores, self.sel_idx, self.sel_count, self.max_sel,
+                             self.tau_hat, stream)
         ekv.ekv_sparse_decode(c, q, self.num_q_heads, self.scale, self.attn, self.sel_idx,
                               self.sel_count, self.max_sel, self.out, self.stat, self.ws, stream)
         return self.out, self.stat
