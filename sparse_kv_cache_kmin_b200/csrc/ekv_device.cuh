@@ -202,8 +202,14 @@ __device__ __forceinline__ int warp_incl_scan(int v)
 }
 
 // Programmatic dependent launch: wait for the preceding grid in the stream (no-op when the
-// launch did not opt in), and let the next grid start its prologue.
-__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// launch did not opt in), then let the next grid be scheduled at once. Every libekv kernel
+// waits here before it reads anything an earlier kernel wrote, so an early start only lets
+// the next kernel's CTAs take SM slots as this grid's CTAs leave, instead of after the grid.
+__device__ __forceinline__ void pdl_wait()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;");
+}
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;"); }
 
 }  // namespace ekv

@@ -15,18 +15,18 @@
 // which live in the cluster's distributed shared memory:
 //   1. The tile maxima are logits, and the exact threshold of any subset of the logits is at
 //      most tau (adding tokens only raises it). Each CTA reduces its tile maxima to 64 / C
-//      group maxima; one warp per query gathers all 64 (DSMEM) and solves them exactly
-//      (bitonic sort, closed form) for zmax and a lower bound on tau.
+//      group maxima; the CTA gathers all 64 of every query (DSMEM) and solves them exactly
+//      (cta_exact_tau) for zmax and a lower bound on tau.
 //   2. Every token above the lower bound is a candidate; each CTA lists its own in token order.
-//      Up to 128 candidates in the cluster: one warp per query gathers and sorts them. Up to
-//      512: the CTA gathers them and every thread ranks one candidate against all the others,
-//      summing the values above it, which gives the closed-form threshold of every support
-//      size at once. More (nearly flat logits): an fp64 bisection whose sums are reduced over
-//      the cluster, then the closed form over the support it brackets.
+//      Up to 512 per query in the cluster: every CTA gathers them and each thread ranks a
+//      candidate against all the others, summing the values above it, which gives the
+//      closed-form threshold of every support size at once (cta_exact_tau). More (nearly flat
+//      logits): an fp64 bisection whose sums are reduced over the cluster, then the closed
+//      form over the support it brackets.
 //   3. Each CTA accumulates p_i v_i over its support tokens (V rows read only for those), in a
 //      fixed order; the CTAs' partial outputs are summed over DSMEM in rank order.
 #include "cluster.cuh"
-#include "warp_entmax.cuh"
+#include "warp_entmax.cuh"  // closed_form_tau
 #include "warp_mma.cuh"
 
 namespace ekv {
@@ -35,7 +35,6 @@ constexpr int kAttThreads = 512;
 constexpr int kAttWarps = kAttThreads / 32;
 constexpr int kAttStageBytes = 8192;  // per warp: 16 loads of 16 bytes per lane
 constexpr int kAttGroups = 64;        // lower-bound maxima per query over the cluster (2 per lane)
-constexpr int kAttWarpCand = 128;     // candidates one warp solves by sorting (4 per lane)
 constexpr int kAttCand = 512;         // candidates the CTA solves by ranking
 
 struct AttArgs {
@@ -60,8 +59,11 @@ struct AttShared {
     int wcnt[kAttWarps];
     float zmax[G];
     double tlb[G], tau[G];
-    int fast[G];                 // 0: bisection, 1: solved by a warp, 2: solve by ranking
-    int best_k;
+    int fast[G];                 // 0: bisection, 1: solved by ranking (or no valid token)
+    int best_k[G];
+    int nset[G];                 // values per set handed to the ranking solver
+    int cnt_tab[G][17];          // candidate counts of every CTA, then their prefix
+    float part[kAttWarps];
     double fpart[2][G];          // bisection partial sums (read by the cluster)
     double cpart[3];             // closed-form partial sums (read by the cluster)
     double red[kAttWarps];
@@ -88,6 +90,62 @@ __device__ __forceinline__ void st_shared_v4(void *p, const uint4 &v)
                  : "memory");
 }
 
+// Exact thresholds of G small value sets at once, by the whole CTA. Set g holds n[g] values
+// x = z - zmax <= 0 at vals[g * stride + i] (-inf entries are inert). Thread t serves set
+// g = t / (NT / G) and its candidates i = t % (NT / G) + k NT / G: for each it counts the values
+// above it (ties broken by index) and sums them and their squares in one short loop, which
+// gives the closed-form threshold tau(k) of the support made of the k largest values. The
+// threshold is tau(k) for the largest k with tau(k) <= x_(k) -- the sort-based rule of the
+// oracle, evaluated for every k at once without a sort. A compact loop: the unrolled
+// single-warp sorting networks it replaces ran from a cold instruction cache. tau[g] is
+// written in fp64 (sums in fp32: values in [-1, 0], at most a few hundred of them).
+template <int NT, int G>
+__device__ void cta_exact_tau(const float *vals, int stride, const int *n, bool sparsemax,
+                              double *tau, int *best_k)
+{
+    constexpr int TPG = NT / G;
+    const int tid = threadIdx.x, g = tid / TPG, it = tid - g * TPG;
+    if (tid < G) best_k[tid] = 0;
+    __syncthreads();
+    const int ng = n[g];
+    const float *v = vals + (size_t)g * stride;
+    int best = 0;
+    float best_t = 0.f;
+    for (int i = it; i < ng; i += TPG) {
+        const float x = v[i];
+        if (!(x > -INFINITY)) continue;
+        float s1 = x, s2 = x * x;
+        int rank = 0;
+        for (int j = 0; j < ng; ++j) {
+            const float y = v[j];
+            const bool before = y > x || (y == x && j < i);
+            rank += before;
+            s1 += before ? y : 0.f;
+            s2 += before ? y * y : 0.f;
+        }
+        const int k = rank + 1;
+        const float kf = (float)k;
+        float tk;
+        bool ok = true;
+        if (sparsemax) {
+            tk = (s1 - 1.0f) / kf;
+        } else {
+            const float mean = s1 / kf;
+            const float disc = (1.0f - fmaxf(s2 - s1 * mean, 0.f)) / kf;
+            ok = disc >= 0.f;
+            tk = mean - sqrtf(fmaxf(disc, 0.f));
+        }
+        if (ok && tk <= x && k > best) {
+            best = k;
+            best_t = tk;
+        }
+    }
+    if (best > 0) atomicMax(&best_k[g], best);
+    __syncthreads();
+    if (best > 0 && best == best_k[g]) tau[g] = (double)best_t;  // k is unique within a set
+    __syncthreads();
+}
+
 template <int D, int G>
 __global__ void __launch_bounds__(kAttThreads, 1)
 step_attend_kernel(AttArgs a)
@@ -100,7 +158,7 @@ step_attend_kernel(AttArgs a)
     constexpr int TPS = kAttStageBytes / TB;  // tiles per warp step
     constexpr int KS = D / 16;                // MMA k-steps per tile
     static_assert(G <= 8, "one n = 8 MMA column block");
-    static_assert((G * (kAttGroups + 2 * kAttCand) + kAttCand) * 4 <= kAttWarps * kAttStageBytes,
+    static_assert(G * (kAttGroups + 3 * kAttCand) * 4 <= kAttWarps * kAttStageBytes,
                   "the lists fit on the staging buffers");
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ AttShared<D, G> sh;
@@ -120,7 +178,7 @@ step_attend_kernel(AttArgs a)
     float *gm = reinterpret_cast<float *>(smem);                 // [G][kAttGroups] group maxima
     float *cx = gm + G * kAttGroups;                             // [G][kAttCand] candidates z - zmax
     int *ct = reinterpret_cast<int *>(cx + G * kAttCand);        // [G][kAttCand] their tokens
-    float *gat = reinterpret_cast<float *>(ct + G * kAttCand);   // [kAttCand] gathered candidates
+    float *gat = reinterpret_cast<float *>(ct + G * kAttCand);   // [G][kAttCand] gathered values
 
     pdl_wait();
     int len;
@@ -236,34 +294,33 @@ step_attend_kernel(AttArgs a)
         gm[g * kAttGroups + k] = m;
     }
     cluster_sync();
-    if (warp < G) {
-        const int g = warp;
-        float v[kAttGroups / 32];
-        float zm = -INFINITY;
+    {
+        // thread t < G * kAttGroups gathers group maximum t % kAttGroups of query t / kAttGroups
+        static_assert(G * kAttGroups <= NT && kAttGroups % 32 == 0, "one maximum per thread");
+        float x = -INFINITY;
+        if (tid < G * kAttGroups) {
+            const int g = tid / kAttGroups, i = tid - g * kAttGroups, cr = i / GM, k = i - cr * GM;
+            x = ld_dsmem_f32(dsmem(&gm[g * kAttGroups + k], (uint32_t)cr));
+        }
+        const float wm = warp_max(x);
+        if (lane == 0) sh.part[warp] = wm;
+        __syncthreads();
+        if (tid < G * kAttGroups) {
+            const int g = tid / kAttGroups;
+            float zm = -INFINITY;
 #pragma unroll
-        for (int r = 0; r < kAttGroups / 32; ++r) {
-            const int idx = r * 32 + lane, cr = idx / GM, k = idx - cr * GM;
-            v[r] = ld_dsmem_f32(dsmem(&gm[g * kAttGroups + k], (uint32_t)cr));
-            zm = fmaxf(zm, v[r]);
+            for (int w = 0; w < kAttGroups / 32; ++w) zm = fmaxf(zm, sh.part[g * (kAttGroups / 32) + w]);
+            gat[tid] = x - zm;  // -inf stays -inf (every value is -inf when zm is)
+            if (tid % kAttGroups == 0) {
+                sh.zmax[g] = zm;
+                sh.tlb[g] = 0.0;
+                sh.nset[g] = zm > -INFINITY ? kAttGroups : 0;
+            }
         }
-        zm = warp_max(zm);
-        int cnt = 0;
-#pragma unroll
-        for (int r = 0; r < kAttGroups / 32; ++r) {
-            v[r] = v[r] - zm;  // -inf stays -inf
-            cnt += __popc(__ballot_sync(kFull, v[r] > -INFINITY));
-        }
-        double lb = 0.0;
-        if (zm > -INFINITY) {
-            lb = warp_exact_tau<kAttGroups / 32>(v, cnt, a.sparsemax != 0);
-            // lowered a little so that the fp32 rounding of the bound (prefix sums of up to 64
-            // values) never drops a support member
-            lb -= 1e-5 * fmax(1.0, fabs(lb));
-        }
-        if (lane == 0) {
-            sh.zmax[g] = zm;
-            sh.tlb[g] = lb;
-        }
+        __syncthreads();
+        cta_exact_tau<NT, G>(gat, kAttGroups, sh.nset, a.sparsemax != 0, sh.tlb, sh.best_k);
+        // lowered a little so that the fp32 rounding of the bound never drops a support member
+        if (tid < G && sh.zmax[tid] > -INFINITY) sh.tlb[tid] -= 1e-5 * fmax(1.0, fabs(sh.tlb[tid]));
     }
     __syncthreads();
 
@@ -298,90 +355,39 @@ step_attend_kernel(AttArgs a)
     cluster_sync();
 
     // ---------------------------------------------------------------- exact tau
-    int offs[17];  // per query, filled by warp g; the ranking path recomputes them
-    auto gather_offsets = [&](int g) {
-        offs[0] = 0;
+    if (tid < G * (int)C) {
+        const int g = tid / C, cr = tid - g * C;
+        sh.cnt_tab[g][cr + 1] = ld_dsmem(dsmem(&sh.ccnt[g], (uint32_t)cr));
+    }
+    __syncthreads();
+    if (tid < G) {  // prefix over the CTAs; a list that overflowed sends the query to bisection
+        int run = 0;
         bool each_fits = true;
+        sh.cnt_tab[tid][0] = 0;
         for (uint32_t cr = 0; cr < C; ++cr) {
-            const int n = ld_dsmem(dsmem(&sh.ccnt[g], cr));
+            const int n = sh.cnt_tab[tid][cr + 1];
             each_fits = each_fits && n <= kAttCand;
-            offs[cr + 1] = offs[cr] + n;
+            run += n;
+            sh.cnt_tab[tid][cr + 1] = run;
         }
-        return each_fits ? offs[C] : kAttCand + 1;
-    };
-    auto gathered = [&](int g, int idx) {  // candidate idx of query g, cluster-wide token order
-        uint32_t cr = 0;
-        while (idx >= offs[cr + 1]) ++cr;
-        return ld_dsmem_f32(dsmem(&cx[g * kAttCand + idx - offs[cr]], cr));
-    };
-    if (warp < G) {
-        const int g = warp;
-        const int total = gather_offsets(g);
-        double tau = 0.0;
-        int mode = 1;
-        if (sh.zmax[g] == -INFINITY) {
-            mode = 1;
-        } else if (total <= kAttWarpCand) {
-            float v[kAttWarpCand / 32];
-#pragma unroll
-            for (int r = 0; r < kAttWarpCand / 32; ++r) {
-                const int idx = r * 32 + lane;
-                v[r] = idx < total ? gathered(g, idx) : -INFINITY;
-            }
-            tau = warp_exact_tau<kAttWarpCand / 32>(v, total, a.sparsemax != 0);
-        } else {
-            mode = total <= kAttCand ? 2 : 0;
-        }
-        if (lane == 0) {
-            sh.tau[g] = tau;
-            sh.fast[g] = mode;
+        const bool solve = sh.zmax[tid] > -INFINITY && each_fits && run <= kAttCand;
+        sh.nset[tid] = solve ? run : 0;
+        sh.fast[tid] = sh.zmax[tid] == -INFINITY || solve;
+        sh.tau[tid] = 0.0;
+    }
+    __syncthreads();
+    // every query's candidates in cluster-wide token order, then one ranking solve for all
+    for (int i = tid; i < G * kAttCand; i += NT) {
+        const int g = i / kAttCand, idx = i - g * kAttCand;
+        if (idx < sh.nset[g]) {
+            uint32_t cr = 0;
+            while (idx >= sh.cnt_tab[g][cr + 1]) ++cr;
+            gat[i] = ld_dsmem_f32(dsmem(&cx[g * kAttCand + idx - sh.cnt_tab[g][cr]], cr));
         }
     }
     __syncthreads();
-    // Up to kAttCand candidates: every CTA gathers them and thread t ranks candidate t. With
-    // x_t the k-th largest (ties broken by position), S1 and S2 the sums of the k largest and
-    // of their squares give tau(k) in closed form; the support is the largest k with
-    // tau(k) <= x_(k) (the sort-based rule without the sort).
-    for (int g = 0; g < G; ++g) {
-        if (sh.fast[g] != 2) continue;
-        const int total = gather_offsets(g);
-        for (int i = tid; i < total; i += NT) gat[i] = gathered(g, i);
-        if (tid == 0) sh.best_k = 0;
-        __syncthreads();
-        int k = 0;
-        float tk = 0.f;
-        if (tid < total) {
-            const float x = gat[tid];
-            float s1 = x, s2 = x * x;
-            int rank = 0;
-            for (int j = 0; j < total; ++j) {
-                const float y = gat[j];
-                const bool before = y > x || (y == x && j < tid);
-                rank += before;
-                s1 += before ? y : 0.f;
-                s2 += before ? y * y : 0.f;
-            }
-            k = rank + 1;
-            const float kf = (float)k;
-            bool ok;
-            if (a.sparsemax) {
-                tk = (s1 - 1.0f) / kf;
-                ok = true;
-            } else {
-                const float mean = s1 / kf;
-                const float disc = (1.0f - fmaxf(s2 - s1 * mean, 0.f)) / kf;
-                ok = disc >= 0.f;
-                tk = mean - sqrtf(fmaxf(disc, 0.f));
-            }
-            if (!(ok && tk <= x)) k = 0;
-            if (k > 0) atomicMax(&sh.best_k, k);
-        }
-        __syncthreads();
-        if (k > 0 && k == sh.best_k) sh.tau[g] = (double)tk;
-        __syncthreads();  // gat is refilled for the next query
-    }
-    __syncthreads();
-    // Too many candidates for one warp (nearly flat logits): fp64 bisection on
+    cta_exact_tau<NT, G>(gat, kAttCand, sh.nset, a.sparsemax != 0, sh.tau, sh.best_k);
+    // Too many candidates for the ranking solve (nearly flat logits): fp64 bisection on
     // f(t) = sum [x - t]_+^p over the cluster's candidates, then the closed form over the support
     // it brackets. The decision is the same in every CTA (the same counts were read), so every
     // CTA takes the same cluster barriers.
