@@ -10,12 +10,10 @@
 // Layout and traffic: a page's bbox row for one KV head is 2*d contiguous elements (512 B for
 // bf16 d=128). A warp streams whole rows with 16-byte loads (lane l owns the l-th 16 bytes,
 // i.e. eight kmin or eight kmax coordinates, and holds the matching eight Q- or Q+
-// coefficients in registers), sixteen pages per step so that each lane has sixteen
-// independent loads in flight (two CTAs of eight warps per SM: of the load structures
-// measured on this layout, the one that keeps the most bytes in flight), then a transposing
-// butterfly reduces each eight pages' partial dots in nine shuffles. The grid is persistent;
-// the flattened work list of (sequence, KV head, 16-page group) is split evenly over CTAs, so
-// ragged batches balance.
+// coefficients in registers), eight pages per step so that each lane has eight independent
+// loads in flight, then a transposing butterfly reduces the eight per-page partial dots in
+// nine shuffles. The grid is persistent (a few CTAs per SM); the flattened work list of
+// (sequence, KV head, 8-page group) is split evenly over CTAs, so ragged batches balance.
 //
 // Gaussian policy: per query, UB_gj (as above but unsummed), m_gj = scale * q_g . mean_j and
 // v_gj = scale^2 * sum_c q_gc^2 var_jc; each page reads its bbox row and its fp32 moment row.
@@ -59,7 +57,7 @@ __device__ __forceinline__ int find_seq(const int *pre, int B, long gi)
 }
 
 template <int DT, int D, int G>
-__global__ void __launch_bounds__(256, 2)
+__global__ void __launch_bounds__(256)
 score_topk_kernel(ekv_cache c, const void *__restrict__ q, int H_q, float scale,
                   float *__restrict__ scores)
 {
@@ -70,10 +68,8 @@ score_topk_kernel(ekv_cache c, const void *__restrict__ q, int H_q, float scale,
     constexpr int W = CPR < 32 ? CPR : 32;                 // lanes per row
     constexpr int LPL = CPR / W;                           // chunks per lane per row
     constexpr int RPI = 32 / W;                            // rows per warp instruction
-    constexpr int PG8 = 8;                                 // pages per reduction
-    constexpr int NPL = PG8 / RPI;                         // page slots per lane per reduction
-    constexpr int U = NPL * LPL <= 8 ? 2 : 1;              // reductions per group: 16 loads per lane
-    constexpr int PG = PG8 * U;                            // pages per work group
+    constexpr int PG = 8;                                  // pages per work group
+    constexpr int NPL = PG / RPI;                          // page slots per lane
     static_assert(NPL <= W, "one result per lane group");
 
     pdl_wait();
@@ -99,7 +95,7 @@ score_topk_kernel(ekv_cache c, const void *__restrict__ q, int H_q, float scale,
         g.j0 = (r % ng) * PG;
         return g;
     };
-    // block id of page j0 + lane % PG: -1 past the end, -2 out of range
+    // block id of page j0 + (lane & 7): -1 past the end, -2 out of range
     auto fetch_blk = [&](const Grp &g) {
         int blk = -1;
         const int jl = g.j0 + (lane & (PG - 1));
@@ -126,21 +122,18 @@ score_topk_kernel(ekv_cache c, const void *__restrict__ q, int H_q, float scale,
         const Grp cur = nxt;
         const int myblk = nxt_blk;
         const int bh = cur.bb * H + cur.hh;
-        // all 16 pages' rows in flight at once (16 loads of 16 bytes per lane)
-        uint4 x[U][NPL][LPL];
+        uint4 x[NPL][LPL];
 #pragma unroll
-        for (int u = 0; u < U; ++u)
+        for (int i = 0; i < NPL; ++i) {
+            const int blk = __shfl_sync(kFull, myblk, i * RPI + lane / W);
 #pragma unroll
-            for (int i = 0; i < NPL; ++i) {
-                const int blk = __shfl_sync(kFull, myblk, u * PG8 + i * RPI + lane / W);
-#pragma unroll
-                for (int k = 0; k < LPL; ++k) {
-                    if (blk >= 0)
-                        x[u][i][k] = ld_stream16(bbox + (((size_t)blk * H + cur.hh) * CPR + k * W + lane % W) * 16);
-                    else
-                        x[u][i][k] = make_uint4(0, 0, 0, 0);
-                }
+            for (int k = 0; k < LPL; ++k) {
+                if (blk >= 0)
+                    x[i][k] = ld_stream16(bbox + (((size_t)blk * H + cur.hh) * CPR + k * W + lane % W) * 16);
+                else
+                    x[i][k] = make_uint4(0, 0, 0, 0);
             }
+        }
         if (gi + 8 < hi) {
             nxt = locate(gi + 8);
             nxt_blk = fetch_blk(nxt);
@@ -164,27 +157,23 @@ score_topk_kernel(ekv_cache c, const void *__restrict__ q, int H_q, float scale,
                 }
             }
         }
+        float part[NPL];
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-            float part[NPL];
+        for (int i = 0; i < NPL; ++i) {
+            part[i] = 0.f;
 #pragma unroll
-            for (int i = 0; i < NPL; ++i) {
-                part[i] = 0.f;
+            for (int k = 0; k < LPL; ++k) {
+                float f[EPC];
+                Chunk<DT>::unpack(x[i][k], f);
 #pragma unroll
-                for (int k = 0; k < LPL; ++k) {
-                    float f[EPC];
-                    Chunk<DT>::unpack(x[u][i][k], f);
-#pragma unroll
-                    for (int e = 0; e < EPC; ++e) part[i] = fmaf(coef[k][e], f[e], part[i]);
-                }
+                for (int e = 0; e < EPC; ++e) part[i] = fmaf(coef[k][e], f[e], part[i]);
             }
-            transpose_reduce<NPL, W>(part, lane);
-            const int po = transpose_index<NPL, W>(lane, 0) * RPI + lane / W;
-            const int blk = __shfl_sync(kFull, myblk, u * PG8 + po);
-            const int j = cur.j0 + u * PG8 + po;
-            if (((lane % W) % (W / NPL)) == 0 && j < cur.np)
-                scores[(size_t)bh * c.max_pages + j] = blk >= 0 ? scale * part[0] : -INFINITY;
         }
+        transpose_reduce<NPL, W>(part, lane);
+        const int po = transpose_index<NPL, W>(lane, 0) * RPI + lane / W;
+        const int blk = __shfl_sync(kFull, myblk, po);
+        if (((lane % W) % (W / NPL)) == 0 && cur.j0 + po < cur.np)
+            scores[(size_t)bh * c.max_pages + cur.j0 + po] = blk >= 0 ? scale * part[0] : -INFINITY;
     }
 }
 
@@ -281,7 +270,6 @@ score_gauss_kernel(ekv_cache c, const void *__restrict__ q, int H_q, float scale
             out[2 * (size_t)c.max_pages] = ok ? scale * scale * pv[0] : 0.f;
         }
     }
-    pdl_trigger();
 }
 
 template <int DT, int D, int G>

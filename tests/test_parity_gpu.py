@@ -226,6 +226,38 @@ def test_tie_storm_prefers_lower_pages(cuda_device):
             check_head(wl, cache, dec, b, h, ekv.EKV_ENTMAX15)
 
 
+# Page counts on each side of the selection kernels' size classes: keys held in registers, 8
+# or 16 per thread (up to 8192 and 16384 pages), and keys staged in shared memory or read
+# from L2 beyond that.
+SEL_SIZES = [8192, 8193, 12000, 16384, 20000]
+
+
+@pytest.mark.parametrize("pages", SEL_SIZES, ids=["pages%d" % n for n in SEL_SIZES])
+def test_topk_selection_at_each_key_count(cuda_device, pages):
+    P = 16
+    lens = (pages * P - 3, pages * P // 3 + 5)
+    wl = make_random(B=2, H_kv=1, G=2, d=64, P=P, lens=lens, dtype=torch.bfloat16,
+                     device="cuda", seed=pages, topk=333)
+    cache, dec = run_gpu(wl, ekv.EKV_ENTMAX15)
+    assert_status_ok(cache)
+    for b in range(2):
+        check_head(wl, cache, dec, b, 0, ekv.EKV_ENTMAX15)
+
+
+@pytest.mark.parametrize("pages", [512, 12000, 20000], ids=["pages512", "pages12000", "pages20000"])
+def test_tie_storm_heavy_boundary(cuda_device, pages):
+    # every page has the same bound, so the boundary holds more ties than the exact ranking
+    # takes: the radix path decides, keeping the lowest pages
+    P = 16
+    wl = make_random(B=1, H_kv=1, G=2, d=64, P=P, lens=(pages * P,), dtype=torch.bfloat16,
+                     device="cuda", seed=7, topk=301)
+    wl.k_cache.fill_(0.5)
+    cache, dec = run_gpu(wl, ekv.EKV_SOFTMAX)
+    assert_status_ok(cache)
+    np.testing.assert_array_equal(dec.sel_idx[0, 0, :301].cpu().numpy(), np.arange(301))
+    check_head(wl, cache, dec, 0, 0, ekv.EKV_SOFTMAX)
+
+
 def test_bad_page_table_entry_is_flagged_not_trapped(cuda_device):
     wl = make_random(B=2, H_kv=2, G=2, d=64, P=16, lens=(300, 200), dtype=torch.float32,
                      device="cuda", seed=13, topk=4)
