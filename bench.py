@@ -64,6 +64,9 @@ def parse():
     ap.add_argument("--fused-select", action="store_true",
                     help="top-k scores and selection through the one-launch cluster kernel "
                          "(ekv_score_select_pages) instead of the two calls")
+    ap.add_argument("--split-select", action="store_true",
+                    help="top-k: ekv_select_pages and ekv_sparse_decode as two calls (timed "
+                         "apart) instead of the one ekv_select_decode call")
     ap.add_argument("--policy", default=None, choices=["topk", "gauss", "gauss_max"],
                     help="selection policy (default: the workload's); gauss_max is the estimated-"
                          "maximum reading of the Gaussian rule")
@@ -153,6 +156,7 @@ def step_bytes(wl, dec, attn, variant, extra):
     if variant == "pages":
         v_rows = sel_tok if attn == 0 else support_rows(wl, dec, attn)
         by["decode"] = sel_tok * row + v_rows * row + qb + out_b + ptab
+        by["select_decode"] = scores_out + sel_out + by["decode"]
         body, body_all_v = sel_tok * row + v_rows * row, 2 * sel_tok * row
         by["support_rows"] = v_rows
     elif variant == "tokens":
@@ -384,7 +388,8 @@ class Step:
     """The public calls of one decode step of a variant, as (name, fn) pairs, with the buffers
     they write. Every call goes through the C ABI binding; nothing here computes."""
 
-    def __init__(self, ekv, SparseDecoder, cache, wl, attn, variant, T, fused_select=False):
+    def __init__(self, ekv, SparseDecoder, cache, wl, attn, variant, T, fused_select=False,
+                 split_select=False):
         self.wl, self.variant, self.T = wl, variant, T
         dev = wl.k_cache.device
         B, H = wl.batch, wl.num_kv_heads
@@ -398,7 +403,12 @@ class Step:
             calls.append(("meta", lambda: ekv.ekv_page_meta_update(cache, ap_start, ap_count,
                                                                    wl.append[1])))
         q = wl.q
-        if wl.policy == 0 and fused_select:
+        # top-k pages: the selection and the attention in one call
+        joint = wl.policy == 0 and variant == "pages" and not fused_select and not split_select
+        if joint:
+            calls.append(("score", lambda: ekv.ekv_score_pages(cache, q, wl.num_q_heads, wl.scale,
+                                                               wl.policy, dec.scores)))
+        elif wl.policy == 0 and fused_select:
             # top-k scores and selection in one launch (one cluster per sequence and KV head)
             calls.append(("score_select", lambda: ekv.ekv_score_select_pages(
                 cache, q, wl.num_q_heads, wl.scale, wl.topk, dec.scores, dec.sel_idx,
@@ -410,7 +420,12 @@ class Step:
                 cache, wl.num_q_heads, wl.policy, wl.topk, wl.alpha, wl.delta, dec.scores,
                 dec.sel_idx, dec.sel_count, dec.max_sel, dec.tau_hat)))
         self.out, self.stat = dec.out, dec.stat
-        if variant == "pages":
+        if joint:
+            calls.append(("select_decode", lambda: ekv.ekv_select_decode(
+                cache, q, wl.num_q_heads, wl.scale, attn, wl.topk, dec.scores, dec.sel_idx,
+                dec.sel_count, dec.max_sel, dec.out, dec.stat, dec.ws)))
+            self.kernels = {"meta": 1, "score": 1, "select_decode": 1}
+        elif variant == "pages":
             calls.append(("decode", lambda: ekv.ekv_sparse_decode(
                 cache, q, wl.num_q_heads, wl.scale, attn, dec.sel_idx, dec.sel_count,
                 dec.max_sel, dec.out, dec.stat, dec.ws)))
@@ -451,7 +466,7 @@ class Step:
             fn()
 
     def graph(self):
-        g = torch.cuda.CUDAGraph()
+        g = torch.cuda.CUDAGraph(keep_graph=True)
         with torch.cuda.graph(g):
             self.run()
         return g
@@ -479,6 +494,21 @@ class Step:
             out_host.copy_(self.out, non_blocking=True)
             stat_host.copy_(self.stat, non_blocking=True)
         return g
+
+
+def graph_kernel_nodes(g):
+    """Kernel nodes of a captured step graph: every kernel one step launches (the captured
+    calls are the library's own, so every kernel node is one of its kernels)."""
+    from cuda.bindings import runtime as rt
+    h = rt.cudaGraph_t(init_value=int(g.raw_cuda_graph()))
+    err, _, n = rt.cudaGraphGetNodes(h, 0)
+    if err != rt.cudaError_t.cudaSuccess:
+        raise RuntimeError(str(err))
+    err, nodes, n = rt.cudaGraphGetNodes(h, n)
+    if err != rt.cudaError_t.cudaSuccess:
+        raise RuntimeError(str(err))
+    kinds = [rt.cudaGraphNodeGetType(x)[1] for x in nodes[:n]]
+    return sum(1 for k in kinds if k == rt.cudaGraphNodeType.cudaGraphNodeTypeKernel)
 
 
 def full_cache_time(ekv, cache, wl, attn, steps, flush, stream):
@@ -581,7 +611,8 @@ def main():
     B = wl.batch
     ekv.ekv_page_meta_update(cache, torch.zeros(B, dtype=torch.int32, device=dev), wl.seq_lens,
                              int(wl.seq_lens.max()))
-    step = Step(ekv, SparseDecoder, cache, wl, attn, args.variant, T, args.fused_select)
+    step = Step(ekv, SparseDecoder, cache, wl, attn, args.variant, T, args.fused_select,
+                args.split_select)
     dec = step.dec
     stream = torch.cuda.current_stream()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
@@ -595,6 +626,10 @@ def main():
     # graph A: the step as one launch (the timed loop); graph B: the same calls with an event
     # node between them (per-call durations)
     graph = step.graph()
+    try:
+        launches_per_step, launches_src = graph_kernel_nodes(graph), "kernel nodes of the step graph"
+    except Exception as exc:  # the count then comes from the calls' known kernel counts
+        launches_per_step, launches_src = step.launches(), "per-call table (%s)" % type(exc).__name__
     graph_b, evb = step.graph_with_events()
 
     for _ in range(max(args.warmup, 3)):
@@ -729,7 +764,8 @@ def main():
         "selection_quality": quality,
         "e2e": {"value": replicas.job_rate(args.steps, world, e2e_s), "unit": "steps/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": step.launches() * args.steps,
+        "gpu_launches": launches_per_step * args.steps,
+        "gpu_launches_source": launches_src,
         "launch": "one CUDA graph per step (programmatic dependent launch between its kernels)",
         "clocks": clocks.summary(),
         "cpu_baseline": cpu,

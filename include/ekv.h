@@ -193,6 +193,24 @@ ekv_status ekv_sparse_decode(const ekv_cache *c, const void *q, int32_t num_q_he
                              const int32_t *sel_count, int32_t max_sel, float *out, float *stat,
                              void *ws, size_t ws_bytes, void *stream);
 
+/*
+ * §2.B.1 and §2.C in one call: the top-k selection of ekv_select_pages (policy EKV_SEL_TOPK)
+ * followed by ekv_sparse_decode on that selection. sel_idx and sel_count are outputs, equal to
+ * those of ekv_select_pages with the same scores and topk; out and stat are those of
+ * ekv_sparse_decode on them. The two kernels run back to back on `stream`, the decode launched
+ * behind the selection (programmatic dependent launch), so the decode's thread-block clusters
+ * are placed on the GPU while the selection runs.
+ *   scores     as written by ekv_score_pages with EKV_SEL_TOPK; 16-byte aligned.
+ *   topk, sel_idx, sel_count, max_sel   as in ekv_select_pages (max_sel >= min(topk,
+ *              max_pages)).
+ *   q, attn, scale, out, stat, ws, ws_bytes   as in ekv_sparse_decode (same alignment and
+ *              workspace rules).
+ */
+ekv_status ekv_select_decode(const ekv_cache *c, const void *q, int32_t num_q_heads, float scale,
+                             int32_t attn, int32_t topk, const float *scores, int32_t *sel_idx,
+                             int32_t *sel_count, int32_t max_sel, float *out, float *stat,
+                             void *ws, size_t ws_bytes, void *stream);
+
 /* Scratch that ekv_sparse_decode_noalloc draws on: 16 MiB, held by every GPU that loads the
  * library until the process exits. */
 #define EKV_NOALLOC_WS_BYTES (16u << 20)

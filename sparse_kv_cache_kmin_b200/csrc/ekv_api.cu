@@ -228,6 +228,36 @@ ekv_status ekv_sparse_decode(const ekv_cache *c, const void *q, int32_t num_q_he
                                             static_cast<cudaStream_t>(stream), use_pdl()));
 }
 
+ekv_status ekv_select_decode(const ekv_cache *c, const void *q, int32_t num_q_heads, float scale,
+                             int32_t attn, int32_t topk, const float *scores, int32_t *sel_idx,
+                             int32_t *sel_count, int32_t max_sel, float *out, float *stat,
+                             void *ws, size_t ws_bytes, void *stream)
+{
+    ekv_status s = check_cache(c, true);
+    if (s != EKV_OK) return s;
+    if ((s = check_heads(c, num_q_heads)) != EKV_OK) return s;
+    if (attn != EKV_SOFTMAX && attn != EKV_ENTMAX15 && attn != EKV_SPARSEMAX)
+        return EKV_ERR_UNSUPPORTED;
+    if (!q || !scores || !sel_idx || !sel_count || !out || !stat || max_sel < 1 || topk < 1 ||
+        !(scale > 0.0f) || !std::isfinite(scale))
+        return EKV_ERR_INVALID_ARG;
+    if (max_sel < (topk < c->max_pages ? topk : c->max_pages)) return EKV_ERR_INVALID_ARG;
+    if (((uintptr_t)scores | (uintptr_t)q | (uintptr_t)c->k_cache | (uintptr_t)c->v_cache) & 15u)
+        return EKV_ERR_INVALID_ARG;
+    if (!ws || ws_bytes < ekv_decode_workspace_bytes(c, num_q_heads, max_sel))
+        return EKV_ERR_WORKSPACE;
+    if ((uintptr_t)ws & 15u) return EKV_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // the selection kernel, then the decode launched behind it (programmatic dependent launch):
+    // the decode's thread-block clusters are placed while the selection runs
+    cudaError_t e = launch_select_pages(*c, num_q_heads, EKV_SEL_TOPK, topk, 1.5f, 0.0f, scores, sel_idx,
+                            sel_count, max_sel, nullptr, st, use_pdl());
+    if (e == cudaSuccess)
+        e = launch_sparse_decode(*c, q, num_q_heads, scale, attn, sel_idx, sel_count, max_sel, out,
+                                 stat, ws, st, use_pdl());
+    return cuda_status(e);
+}
+
 size_t ekv_moment_bytes(const ekv_cache *c)
 {
     if (check_cache(c, true) != EKV_OK) return 0;

@@ -15,6 +15,7 @@
 // that path and are dropped before the iterations; the rest are kept in shared memory. Then a
 // block scan keeps page j iff some query g has (alpha-1) UB_gj > tau_hat_g - Delta.
 #include "ekv_device.cuh"
+#include "topk_cta.cuh"
 
 namespace ekv {
 
@@ -276,11 +277,9 @@ select_topk_kernel(const float *__restrict__ scores, int H, int max_pages, int P
 }
 
 // The same selection with each thread's keys in registers, for n <= R * kSelThreads pages:
-// thread t owns pages [t R, t R + R), loaded as float4 (R / 4 per thread, coalesced). One
-// histogram pass over 2048 bins of [min, max] finds the bin of the k-th largest key, its few
-// keys are ranked exactly (key descending, page ascending), and one block scan of the
-// threads' kept counts places every thread's kept pages, in ascending order. Heavy ties at
-// the boundary take the exact three-pass radix select over the keys staged in shared memory.
+// thread t owns pages [t R, t R + R), loaded as float4 where the rows allow it (coalesced),
+// and cta_topk finds the kept set; one block scan of the threads' kept counts places every
+// thread's kept pages, in ascending order.
 template <int R>
 __global__ void __launch_bounds__(kSelThreads)
 select_topk_reg_kernel(const float *__restrict__ scores, int H, int max_pages, int P,
@@ -288,28 +287,14 @@ select_topk_reg_kernel(const float *__restrict__ scores, int H, int max_pages, i
                        int32_t *__restrict__ sel_count, int max_sel, uint32_t *status)
 {
     constexpr int NT = kSelThreads;
-    constexpr int NB = 2048;
-    extern __shared__ uint32_t keys[];  // [R * NT], only for heavy ties
-    __shared__ int hist[NB];
-    __shared__ int warp_tot[32];
-    __shared__ int s_bin, s_above, s_cnt;
-    __shared__ uint32_t s_umin, s_umax;
-    __shared__ uint32_t bu[kBoundaryMax];
-    __shared__ int bj[kBoundaryMax];
-    __shared__ uint32_t kept_bits[R * NT / 32];
+    __shared__ TopkShared sh;
     pdl_wait();
-    const int tid = threadIdx.x, lane = tid & 31;
+    const int tid = threadIdx.x;
     const int h = blockIdx.x, b = blockIdx.y;
     const int bh = b * H + h;
-    const int n = seq_pages(seq_lens, b, P, max_pages, h == 0 ? status : nullptr, nullptr);
     const float *S = scores + (size_t)bh * max_pages;
-    int32_t *out = sel_idx + (size_t)bh * max_sel;
-    const int kk = k < n ? k : n;
-    if (kk == n) {  // every page is kept
-        for (int j = tid; j < max_sel; j += NT) out[j] = j < n ? j : -1;
-        if (tid == 0) sel_count[bh] = n;
-        return;
-    }
+    // every float4 of the row issued at once, before the sequence length is known (entries
+    // past the last page are ignored)
     const int j0 = tid * R;
     uint32_t u[R];
     if ((max_pages & 3) == 0) {
@@ -317,80 +302,30 @@ select_topk_reg_kernel(const float *__restrict__ scores, int H, int max_pages, i
 #pragma unroll
         for (int q4 = 0; q4 < R / 4; ++q4) {
             float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (j0 + 4 * q4 < n) v = __ldcg(S4 + q4);  // n <= max_pages: the float4 stays in the row
-            u[4 * q4] = order_key(v.x);
-            u[4 * q4 + 1] = order_key(v.y);
-            u[4 * q4 + 2] = order_key(v.z);
-            u[4 * q4 + 3] = order_key(v.w);
+            if (j0 + 4 * q4 < max_pages) v = __ldcg(S4 + q4);  // max_pages % 4 == 0: inside the row
+            u[4 * q4] = topk_order_key(v.x);
+            u[4 * q4 + 1] = topk_order_key(v.y);
+            u[4 * q4 + 2] = topk_order_key(v.z);
+            u[4 * q4 + 3] = topk_order_key(v.w);
         }
     } else {
 #pragma unroll
-        for (int r = 0; r < R; ++r) u[r] = j0 + r < n ? order_key(__ldcg(S + j0 + r)) : 0u;
+        for (int r = 0; r < R; ++r) u[r] = j0 + r < max_pages ? topk_order_key(__ldcg(S + j0 + r)) : 0u;
     }
-    uint32_t umin = 0xffffffffu, umax = 0;
+    const int n = seq_pages(seq_lens, b, P, max_pages, h == 0 ? status : nullptr, nullptr);
+    int32_t *out = sel_idx + (size_t)bh * max_sel;
+    const int kk = k < n ? k : n;
+    if (kk == n) {  // every page is kept
+        for (int j = tid; j < max_sel; j += NT) out[j] = j < n ? j : -1;
+        if (tid == 0) sel_count[bh] = n;
+        return;
+    }
+    bool keep[R];
+    const int mine = cta_topk<NT, R>(u, n, kk, sh, keep);
+    int pos = block_incl_scan<NT>(mine, sh.warp_tot, nullptr) - mine;
 #pragma unroll
     for (int r = 0; r < R; ++r)
-        if (j0 + r < n) { umin = min(umin, u[r]); umax = max(umax, u[r]); }
-    for (int i = tid; i < NB; i += NT) hist[i] = 0;
-    for (int i = tid; i < R * NT / 32; i += NT) kept_bits[i] = 0;
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) {
-        umin = min(umin, __shfl_xor_sync(kFull, umin, o));
-        umax = max(umax, __shfl_xor_sync(kFull, umax, o));
-    }
-    if (tid == 0) { s_umin = 0xffffffffu; s_umax = 0; s_cnt = 0; }
-    __syncthreads();
-    if (lane == 0) { atomicMin(&s_umin, umin); atomicMax(&s_umax, umax); }
-    __syncthreads();
-    umin = s_umin;
-    umax = s_umax;
-    const float bscale = (float)NB / ((float)(umax - umin) + 1.0f);
-    int bin[R];
-#pragma unroll
-    for (int r = 0; r < R; ++r) {
-        const int bb = (int)((float)(u[r] - umin) * bscale);
-        bin[r] = j0 + r < n ? (bb < NB - 1 ? bb : NB - 1) : -1;
-        if (bin[r] >= 0) atomicAdd(&hist[bin[r]], 1);
-    }
-    __syncthreads();
-    find_bin_from_top<NT, NB / NT>(hist, NB, kk, warp_tot, &s_bin, &s_above);
-    const int B = s_bin, rneed = kk - s_above, cB = hist[B];
-    if (cB > kBoundaryMax) {  // heavy ties around the k-th key: exact radix select
-#pragma unroll
-        for (int r = 0; r < R; ++r)
-            if (j0 + r < n) keys[j0 + r] = u[r];
-        __syncthreads();
-        radix_select_emit(n, kk, [&](int j) { return keys[j]; }, hist, warp_tot, &s_bin, &s_above, out);
-    } else {
-#pragma unroll
-        for (int r = 0; r < R; ++r)
-            if (bin[r] == B) {
-                const int pos = atomicAdd(&s_cnt, 1);
-                bu[pos] = u[r];
-                bj[pos] = j0 + r;
-            }
-        __syncthreads();
-        if (tid < cB) {
-            const uint32_t uu = bu[tid];
-            const int j = bj[tid];
-            int rank = 0;
-            for (int m = 0; m < cB; ++m) rank += bu[m] > uu || (bu[m] == uu && bj[m] < j);
-            if (rank < rneed) atomicOr(&kept_bits[j >> 5], 1u << (j & 31));
-        }
-        __syncthreads();
-        bool keep[R];
-        int mine = 0;
-#pragma unroll
-        for (int r = 0; r < R; ++r) {
-            const int j = j0 + r;
-            keep[r] = bin[r] > B || (bin[r] == B && ((kept_bits[j >> 5] >> (j & 31)) & 1u));
-            mine += keep[r];
-        }
-        int pos = block_incl_scan<NT>(mine, warp_tot, nullptr) - mine;
-#pragma unroll
-        for (int r = 0; r < R; ++r)
-            if (keep[r] && pos < kk) out[pos++] = j0 + r;
-    }
+        if (keep[r] && pos < kk) out[pos++] = j0 + r;
     for (int j = kk + tid; j < max_sel; j += NT) out[j] = -1;
     if (tid == 0) sel_count[bh] = kk;
 }
@@ -746,15 +681,7 @@ cudaError_t launch_select_pages(const ekv_cache &c, int H_q, int policy, int top
     if (policy == EKV_SEL_TOPK && c.max_pages <= 16 * kSelThreads) {
         // keys in registers: 8 or 16 per thread
         cudaLaunchConfig_t cfg = pdl_config(grid, dim3(kSelThreads), st, pdl, attr);
-        const bool r8 = c.max_pages <= 8 * kSelThreads;
-        cfg.dynamicSmemBytes = sizeof(uint32_t) * (size_t)(r8 ? 8 : 16) * kSelThreads;
-        static bool attr_set = false;
-        if (!attr_set) {
-            cudaFuncSetAttribute(select_topk_reg_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 16 * kSelThreads * (int)sizeof(uint32_t));
-            attr_set = true;
-        }
-        if (r8)
+        if (c.max_pages <= 8 * kSelThreads)
             return cudaLaunchKernelEx(&cfg, select_topk_reg_kernel<8>, scores, c.num_kv_heads,
                                       c.max_pages, c.page_size, c.seq_lens, topk, sel_idx, sel_count,
                                       max_sel, c.dev_status);

@@ -14,17 +14,19 @@
 // The threshold tau solves sum_i [z_i - tau]_+^(1/(alpha-1)) = 1 over all the pair's tokens,
 // which live in the cluster's distributed shared memory:
 //   1. The tile maxima are logits, and the exact threshold of any subset of the logits is at
-//      most tau (adding tokens only raises it). Each CTA reduces its tile maxima to 64 / C
-//      group maxima; the CTA gathers all 64 of every query (DSMEM) and solves them exactly
-//      (cta_exact_tau) for zmax and a lower bound on tau.
-//   2. Every token above the lower bound is a candidate; each CTA lists its own in token order.
-//      Up to 512 per query in the cluster: every CTA gathers them and each thread ranks a
-//      candidate against all the others, summing the values above it, which gives the
-//      closed-form threshold of every support size at once (cta_exact_tau). More (nearly flat
-//      logits): an fp64 bisection whose sums are reduced over the cluster, then the closed
-//      form over the support it brackets.
+//      most tau (adding tokens only raises it). Each CTA reduces its own tile maxima to 64
+//      group maxima per query and solves them exactly (cta_exact_tau): a lower bound on tau,
+//      with no exchange yet.
+//   2. Every token of the CTA above its bound is a candidate, listed in token order. One
+//      cluster barrier; then every CTA reads all CTAs' bounds, largest logits and lists,
+//      keeps the candidates above the largest bound, and -- up to 512 per query -- ranks each
+//      against all the others, summing the values above it, which gives the closed-form
+//      threshold of every support size at once (cta_exact_tau). More (nearly flat logits): an
+//      fp64 bisection whose sums are reduced over the cluster, then the closed form over the
+//      support it brackets.
 //   3. Each CTA accumulates p_i v_i over its support tokens (V rows read only for those), in a
-//      fixed order; the CTAs' partial outputs are summed over DSMEM in rank order.
+//      fixed order, and stores the sum into rank 0's shared memory; after a second cluster
+//      barrier rank 0 adds the CTAs' partial outputs in rank order and writes the output.
 #include "cluster.cuh"
 #include "warp_entmax.cuh"  // closed_form_tau
 #include "warp_mma.cuh"
@@ -36,6 +38,7 @@ constexpr int kAttWarps = kAttThreads / 32;
 constexpr int kAttStageBytes = 8192;  // per warp: 16 loads of 16 bytes per lane
 constexpr int kAttGroups = 64;        // lower-bound maxima per query over the cluster (2 per lane)
 constexpr int kAttCand = 512;         // candidates the CTA solves by ranking
+constexpr int kAttWarpSolve = 64;     // candidates one warp solves by sorting (2 per lane)
 
 struct AttArgs {
     ekv_cache c;
@@ -55,20 +58,26 @@ struct AttArgs {
 // the tile staging buffers (free once the logits are taken).
 template <int D, int G>
 struct AttShared {
-    int ccnt[G];                 // candidates of this CTA (read by the cluster)
+    // read by the cluster: this CTA's candidate count, largest logit and lower bound on tau
+    int ccnt[G];
+    float zmax_loc[G];
+    double tlb_loc[G];
     int wcnt[kAttWarps];
-    float zmax[G];
-    double tlb[G], tau[G];
+    float zmax[G];               // the pair's largest logit
+    double tlb[G];               // the pair's lower bound on tau (absolute)
+    double tau[G];               // relative to zmax
     int fast[G];                 // 0: bisection, 1: solved by ranking (or no valid token)
     int best_k[G];
-    int nset[G];                 // values per set handed to the ranking solver
+    int nset[G];                 // values per set handed to a solver
+    int nbig[G];                 // values per set handed to the CTA-wide ranking solver
     int cnt_tab[G][17];          // candidate counts of every CTA, then their prefix
+    float zm_tab[G][16];
+    double tlb_tab[G][16];
     float part[kAttWarps];
     double fpart[2][G];          // bisection partial sums (read by the cluster)
     double cpart[3];             // closed-form partial sums (read by the cluster)
     double red[kAttWarps];
     float opart[kAttWarps][D];
-    float ocat[G][D];            // this CTA's partial output (read by the cluster)
 };
 
 __device__ __forceinline__ float ld_dsmem_f32(uint32_t addr)
@@ -82,6 +91,10 @@ __device__ __forceinline__ double ld_dsmem_f64(uint32_t addr)
     double v;
     asm volatile("ld.shared::cluster.f64 %0, [%1];" : "=d"(v) : "r"(addr) : "memory");
     return v;
+}
+__device__ __forceinline__ void st_dsmem_f32(uint32_t addr, float v)
+{
+    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
 }
 __device__ __forceinline__ void st_shared_v4(void *p, const uint4 &v)
 {
@@ -116,13 +129,21 @@ __device__ void cta_exact_tau(const float *vals, int stride, const int *n, bool 
         if (!(x > -INFINITY)) continue;
         float s1 = x, s2 = x * x;
         int rank = 0;
-        for (int j = 0; j < ng; ++j) {
-            const float y = v[j];
+        auto visit = [&](float y, int j) {
             const bool before = y > x || (y == x && j < i);
             rank += before;
             s1 += before ? y : 0.f;
             s2 += before ? y * y : 0.f;
+        };
+        int j = 0;
+        for (; j + 4 <= ng; j += 4) {  // four values per shared-memory load (vals is 16-byte aligned)
+            const float4 y = *reinterpret_cast<const float4 *>(v + j);
+            visit(y.x, j);
+            visit(y.y, j + 1);
+            visit(y.z, j + 2);
+            visit(y.w, j + 3);
         }
+        for (; j < ng; ++j) visit(v[j], j);
         const int k = rank + 1;
         const float kf = (float)k;
         float tk;
@@ -158,8 +179,8 @@ step_attend_kernel(AttArgs a)
     constexpr int TPS = kAttStageBytes / TB;  // tiles per warp step
     constexpr int KS = D / 16;                // MMA k-steps per tile
     static_assert(G <= 8, "one n = 8 MMA column block");
-    static_assert(G * (kAttGroups + 3 * kAttCand) * 4 <= kAttWarps * kAttStageBytes,
-                  "the lists fit on the staging buffers");
+    static_assert(G * (3 * kAttCand + 16 * D) * 4 <= kAttWarps * kAttStageBytes,
+                  "the lists and partial outputs fit on the staging buffers");
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ AttShared<D, G> sh;
 
@@ -174,11 +195,11 @@ step_attend_kernel(AttArgs a)
     int *ent_blk = reinterpret_cast<int *>(zs + (size_t)G * ntok_cap);        // [ent_cap]
     int *ent_nt = ent_blk + ent_cap;                                            // [ent_cap]
     float *tmax = reinterpret_cast<float *>(ent_nt + ent_cap);                  // [G][tile_cap]
-    // after the logits phase, on the staging buffers (read by the cluster):
-    float *gm = reinterpret_cast<float *>(smem);                 // [G][kAttGroups] group maxima
-    float *cx = gm + G * kAttGroups;                             // [G][kAttCand] candidates z - zmax
+    // after the logits phase, on the staging buffers:
+    float *cx = reinterpret_cast<float *>(smem);                 // [G][kAttCand] candidate logits (cluster-read)
     int *ct = reinterpret_cast<int *>(cx + G * kAttCand);        // [G][kAttCand] their tokens
-    float *gat = reinterpret_cast<float *>(ct + G * kAttCand);   // [G][kAttCand] gathered values
+    float *gat = reinterpret_cast<float *>(ct + G * kAttCand);   // [G][kAttCand] values to solve
+    float *oall = gat + G * kAttCand;                            // rank 0: [C][G][D] partial outputs
 
     pdl_wait();
     int len;
@@ -186,8 +207,8 @@ step_attend_kernel(AttArgs a)
     int ns = a.sel_count[bh];
     ns = ns < 0 ? 0 : (ns > a.max_sel ? a.max_sel : ns);
     const int e0 = (int)((long long)ns * rank / C), e1 = (int)((long long)ns * (rank + 1) / C);
-    const int ne = e1 - e0, ntiles = ne * TPP, ntok = ne * P;
-    for (int i = tid; i < ne; i += NT) {
+    for (int i = tid; i < e1 - e0; i += NT) {
+        // entry i of this CTA: selected page j -> its block and valid tokens
         const int j = a.sel_idx[(size_t)bh * a.max_sel + e0 + i];
         int blk = -1, nt = 0;
         if (j < 0 || j >= np) {
@@ -204,6 +225,7 @@ step_attend_kernel(AttArgs a)
         ent_blk[i] = blk;
         ent_nt[i] = nt;
     }
+    const int ne = e1 - e0, ntiles = ne * TPP, ntok = ne * P;
     if (tid < G) sh.ccnt[tid] = 0;
     // B fragments of the group's queries: column n = lane / 4 is query n (zero past G)
     uint32_t qb[KS][2];
@@ -284,68 +306,65 @@ step_attend_kernel(AttArgs a)
     }
     __syncthreads();
 
-    // ---------------------------------------------------------------- lower bound on tau
-    const int GM = kAttGroups / (int)C;  // group maxima per CTA
-    for (int i = tid; i < G * GM; i += NT) {
-        const int g = i / GM, k = i - g * GM;
-        const int ta = (int)((long long)ntiles * k / GM), tb = (int)((long long)ntiles * (k + 1) / GM);
-        float m = -INFINITY;
-        for (int t = ta; t < tb; ++t) m = fmaxf(m, tmax[(size_t)g * tile_cap + t]);
-        gm[g * kAttGroups + k] = m;
-    }
-    cluster_sync();
+    // ---------------------------------------------------------------- local lower bound on tau
+    // The tile maxima are logits, and the threshold of any subset of the logits is at most tau
+    // (adding tokens only raises it). Each query's tiles in this CTA are grouped into
+    // kAttGroups runs; one warp per query sorts the runs' maxima and solves them exactly, which
+    // bounds the pair's tau from below with no exchange.
     {
-        // thread t < G * kAttGroups gathers group maximum t % kAttGroups of query t / kAttGroups
-        static_assert(G * kAttGroups <= NT && kAttGroups % 32 == 0, "one maximum per thread");
+        static_assert(G * kAttGroups <= NT && kAttGroups == 64, "one maximum per thread, two per lane");
         float x = -INFINITY;
         if (tid < G * kAttGroups) {
-            const int g = tid / kAttGroups, i = tid - g * kAttGroups, cr = i / GM, k = i - cr * GM;
-            x = ld_dsmem_f32(dsmem(&gm[g * kAttGroups + k], (uint32_t)cr));
+            const int g = tid / kAttGroups, k = tid - g * kAttGroups;
+            const int ta = (int)((long long)ntiles * k / kAttGroups);
+            const int tb = (int)((long long)ntiles * (k + 1) / kAttGroups);
+            for (int t = ta; t < tb; ++t) x = fmaxf(x, tmax[(size_t)g * tile_cap + t]);
+            gat[tid] = x;
         }
-        const float wm = warp_max(x);
-        if (lane == 0) sh.part[warp] = wm;
         __syncthreads();
-        if (tid < G * kAttGroups) {
-            const int g = tid / kAttGroups;
-            float zm = -INFINITY;
-#pragma unroll
-            for (int w = 0; w < kAttGroups / 32; ++w) zm = fmaxf(zm, sh.part[g * (kAttGroups / 32) + w]);
-            gat[tid] = x - zm;  // -inf stays -inf (every value is -inf when zm is)
-            if (tid % kAttGroups == 0) {
-                sh.zmax[g] = zm;
-                sh.tlb[g] = 0.0;
-                sh.nset[g] = zm > -INFINITY ? kAttGroups : 0;
+        if (warp < G) {
+            const int g = warp;
+            float v[2] = {gat[g * kAttGroups + lane], gat[g * kAttGroups + 32 + lane]};
+            const float zm = warp_max(fmaxf(v[0], v[1]));
+            double lb = -INFINITY;
+            if (zm > -INFINITY) {
+                v[0] -= zm;  // -inf stays -inf
+                v[1] -= zm;
+                const int cnt = __popc(__ballot_sync(kFull, v[0] > -INFINITY)) +
+                                __popc(__ballot_sync(kFull, v[1] > -INFINITY));
+                const double t = warp_exact_tau<2>(v, cnt, a.sparsemax != 0);
+                // lowered a little so that fp32 rounding never drops a support member
+                lb = (double)zm + t - 1e-5 * fmax(1.0, fabs(t));
+            }
+            if (lane == 0) {
+                sh.zmax_loc[g] = zm;
+                sh.tlb_loc[g] = lb;
             }
         }
         __syncthreads();
-        cta_exact_tau<NT, G>(gat, kAttGroups, sh.nset, a.sparsemax != 0, sh.tlb, sh.best_k);
-        // lowered a little so that the fp32 rounding of the bound never drops a support member
-        if (tid < G && sh.zmax[tid] > -INFINITY) sh.tlb[tid] -= 1e-5 * fmax(1.0, fabs(sh.tlb[tid]));
     }
-    __syncthreads();
 
-    // ---------------------------------------------------------------- candidates, token order
+    // ---------------------------------------------------------------- local candidates, token order
     {
         constexpr int WPQ = NW / G;  // warps per query
         const int g = warp % G, part = warp / G;
         const int ta = (int)((long long)ntok * part / WPQ), tb = (int)((long long)ntok * (part + 1) / WPQ);
-        const float zm = sh.zmax[g];
-        const double lb = sh.tlb[g];
         const float *zg = zs + (size_t)g * ntok_cap;
+        const double lb = sh.tlb_loc[g];
         int mine = 0;
         for (int i = ta + lane; i - lane < tb; i += 32)
-            mine += __popc(__ballot_sync(kFull, i < tb && (double)(zg[i] - zm) > lb));
+            mine += __popc(__ballot_sync(kFull, i < tb && (double)zg[i] > lb));
         if (lane == 0) sh.wcnt[warp] = mine;
         __syncthreads();
         int pos = 0;
         for (int p = 0; p < part; ++p) pos += sh.wcnt[p * G + g];
         for (int i = ta + lane; i - lane < tb; i += 32) {
-            const float x = i < tb ? zg[i] - zm : -INFINITY;
-            const bool keep = i < tb && (double)x > lb;
+            const float z = i < tb ? zg[i] : -INFINITY;
+            const bool keep = i < tb && (double)z > lb;
             const unsigned bal = __ballot_sync(kFull, keep);
             const int at = pos + __popc(bal & ((1u << lane) - 1u));
             if (keep && at < kAttCand) {
-                cx[g * kAttCand + at] = x;
+                cx[g * kAttCand + at] = z;
                 ct[g * kAttCand + at] = i;
             }
             pos += __popc(bal);
@@ -355,47 +374,94 @@ step_attend_kernel(AttArgs a)
     cluster_sync();
 
     // ---------------------------------------------------------------- exact tau
+    // every CTA's count, largest logit and bound; the pair's bound is the largest of them
     if (tid < G * (int)C) {
         const int g = tid / C, cr = tid - g * C;
         sh.cnt_tab[g][cr + 1] = ld_dsmem(dsmem(&sh.ccnt[g], (uint32_t)cr));
+        sh.zm_tab[g][cr] = ld_dsmem_f32(dsmem(&sh.zmax_loc[g], (uint32_t)cr));
+        sh.tlb_tab[g][cr] = ld_dsmem_f64(dsmem(&sh.tlb_loc[g], (uint32_t)cr));
     }
     __syncthreads();
     if (tid < G) {  // prefix over the CTAs; a list that overflowed sends the query to bisection
         int run = 0;
         bool each_fits = true;
+        float zm = -INFINITY;
+        double lb = -INFINITY;
         sh.cnt_tab[tid][0] = 0;
         for (uint32_t cr = 0; cr < C; ++cr) {
             const int n = sh.cnt_tab[tid][cr + 1];
+            zm = fmaxf(zm, sh.zm_tab[tid][cr]);
+            lb = fmax(lb, sh.tlb_tab[tid][cr]);
             each_fits = each_fits && n <= kAttCand;
             run += n;
             sh.cnt_tab[tid][cr + 1] = run;
         }
-        const bool solve = sh.zmax[tid] > -INFINITY && each_fits && run <= kAttCand;
+        const bool solve = zm > -INFINITY && each_fits && run <= kAttCand;
+        sh.zmax[tid] = zm;
+        sh.tlb[tid] = lb;
         sh.nset[tid] = solve ? run : 0;
-        sh.fast[tid] = sh.zmax[tid] == -INFINITY || solve;
+        sh.fast[tid] = zm == -INFINITY || solve;
         sh.tau[tid] = 0.0;
     }
     __syncthreads();
-    // every query's candidates in cluster-wide token order, then one ranking solve for all
-    for (int i = tid; i < G * kAttCand; i += NT) {
-        const int g = i / kAttCand, idx = i - g * kAttCand;
-        if (idx < sh.nset[g]) {
-            uint32_t cr = 0;
-            while (idx >= sh.cnt_tab[g][cr + 1]) ++cr;
-            gat[i] = ld_dsmem_f32(dsmem(&cx[g * kAttCand + idx - sh.cnt_tab[g][cr]], cr));
+    // every query's candidates above the pair's bound, in cluster-wide token order, then one
+    // ranking solve for all (values below the bound enter as -inf, which the solver skips)
+    {
+        // all of a thread's remote loads in flight together, then the stores
+        static_assert((G * kAttCand) % NT == 0, "whole rounds");
+        constexpr int PER = G * kAttCand / NT;
+        float zv[PER];
+#pragma unroll
+        for (int k = 0; k < PER; ++k) {
+            const int i = tid + k * NT, g = i / kAttCand, idx = i - g * kAttCand;
+            zv[k] = -INFINITY;
+            if (idx < sh.nset[g]) {
+                uint32_t cr = 0;
+                while (idx >= sh.cnt_tab[g][cr + 1]) ++cr;
+                zv[k] = ld_dsmem_f32(dsmem(&cx[g * kAttCand + idx - sh.cnt_tab[g][cr]], cr));
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < PER; ++k) {
+            const int i = tid + k * NT, g = i / kAttCand, idx = i - g * kAttCand;
+            if (idx < sh.nset[g]) gat[i] = (double)zv[k] > sh.tlb[g] ? zv[k] - sh.zmax[g] : -INFINITY;
         }
     }
     __syncthreads();
-    cta_exact_tau<NT, G>(gat, kAttCand, sh.nset, a.sparsemax != 0, sh.tau, sh.best_k);
+    {
+        // up to kAttWarpSolve candidates: one warp per query sorts them (no barrier); more: the
+        // CTA-wide ranking solve
+        bool big = false;
+#pragma unroll
+        for (int gg = 0; gg < G; ++gg) big = big || sh.nset[gg] > kAttWarpSolve;  // the same in every thread
+        if (warp < G && sh.nset[warp] > 0 && sh.nset[warp] <= kAttWarpSolve) {
+            constexpr int RW = kAttWarpSolve / 32;
+            const int g = warp, n = sh.nset[g];
+            float v[RW];
+            int cnt = 0;
+#pragma unroll
+            for (int r = 0; r < RW; ++r) {
+                const int e = r * 32 + lane;
+                v[r] = e < n ? gat[g * kAttCand + e] : -INFINITY;
+                cnt += __popc(__ballot_sync(kFull, v[r] > -INFINITY));
+            }
+            const double t = warp_exact_tau<RW>(v, cnt, a.sparsemax != 0);
+            if (lane == 0) sh.tau[g] = t;
+        }
+        if (big) {
+            if (tid < G) sh.nbig[tid] = sh.nset[tid] > kAttWarpSolve ? sh.nset[tid] : 0;
+            cta_exact_tau<NT, G>(gat, kAttCand, sh.nbig, a.sparsemax != 0, sh.tau, sh.best_k);
+        }
+    }
     // Too many candidates for the ranking solve (nearly flat logits): fp64 bisection on
-    // f(t) = sum [x - t]_+^p over the cluster's candidates, then the closed form over the support
+    // f(t) = sum [x - t]_+^p over the cluster's tokens, then the closed form over the support
     // it brackets. The decision is the same in every CTA (the same counts were read), so every
     // CTA takes the same cluster barriers.
     for (int g = 0; g < G; ++g) {
         if (sh.fast[g] != 0) continue;
         const float zm = sh.zmax[g];
         const float *zg = zs + (size_t)g * ntok_cap;
-        double lo = sh.tlb[g], hi = 0.0;
+        double lo = sh.tlb[g] - (double)zm, hi = 0.0;
         auto cluster_total = [&](double v, double *slot) {  // sum over the cluster, rank order
             v = warp_sum(v);
             if (lane == 0) sh.red[warp] = v;
@@ -437,6 +503,9 @@ step_attend_kernel(AttArgs a)
     __syncthreads();
 
     // ---------------------------------------------------------------- output
+    // p_i v_i over this CTA's support tokens (V rows read only for those), summed over the
+    // CTA's warps in a fixed order and pushed into rank 0's shared memory; rank 0 adds the CTAs'
+    // partial outputs in rank order.
     {
         constexpr int WPQ = NW / G;
         const int g = warp % G, part = warp / G;
@@ -461,10 +530,35 @@ step_attend_kernel(AttArgs a)
         };
         if (zm > -INFINITY) {
             if (sh.fast[g] != 0) {
-                const int n = sh.ccnt[g];  // this CTA's candidates (<= kAttCand on this path)
-                for (int i = part * 2 + half; i < n; i += WPQ * 2) {
-                    const double r = (double)cx[g * kAttCand + i] - tau;
-                    if (r > 0.0) add_row(ct[g * kAttCand + i], r);
+                // this CTA's candidates (<= kAttCand on this path); a half-warp takes rows
+                // i, i + 2 WPQ, ... and keeps up to four value-row loads in flight
+                const int n = sh.ccnt[g];
+                constexpr int RF = 4;
+                for (int i0 = part * 2 + half; i0 < n; i0 += RF * WPQ * 2) {
+                    uint4 vv[RF];
+                    float pr[RF];
+#pragma unroll
+                    for (int u = 0; u < RF; ++u) {
+                        const int i = i0 + u * WPQ * 2;
+                        pr[u] = 0.f;
+                        vv[u] = make_uint4(0, 0, 0, 0);
+                        if (i < n) {
+                            const double r = (double)(cx[g * kAttCand + i] - zm) - tau;
+                            const int tl = ct[g * kAttCand + i], e = tl / P, blk = ent_blk[e];
+                            if (r > 0.0 && blk >= 0) {
+                                pr[u] = (float)(a.sparsemax ? r : r * r);
+                                if (hl < W)
+                                    vv[u] = ld_stream16(vc + (((size_t)blk * H + h) * P + (tl - e * P)) * RB + hl * 16);
+                            }
+                        }
+                    }
+#pragma unroll
+                    for (int u = 0; u < RF; ++u) {
+                        float f[8];
+                        Chunk<EKV_BF16>::unpack(vv[u], f);
+#pragma unroll
+                        for (int q8 = 0; q8 < 8; ++q8) acc[q8] = fmaf(pr[u], f[q8], acc[q8]);
+                    }
                 }
             } else {
                 const float *zg = zs + (size_t)g * ntok_cap;
@@ -485,24 +579,20 @@ step_attend_kernel(AttArgs a)
             const int gg = i / D, dd = i - gg * D;
             float s = 0.f;
             for (int p = 0; p < WPQ; ++p) s += sh.opart[p * G + gg][dd];
-            sh.ocat[gg][dd] = s;
+            st_dsmem_f32(dsmem(&oall[(size_t)rank * G * D + i], 0u), s);
         }
     }
-    cluster_sync();
-    // CTA `rank` writes the slice [rank * G * D / C, (rank + 1) * G * D / C) of the outputs
-    {
-        const int o0 = (int)((long long)G * D * rank / C), o1 = (int)((long long)G * D * (rank + 1) / C);
+    cluster_sync();  // the partial outputs have landed; no CTA's shared memory is read after this
+    if (rank == 0) {
         const size_t bq0 = (size_t)b * a.H_q + (size_t)h * G;
-        for (int i = o0 + tid; i < o1; i += NT) {
-            const int gg = i / D, dd = i - gg * D;
+        for (int i = tid; i < G * D; i += NT) {
             float s = 0.f;
-            for (uint32_t cr = 0; cr < C; ++cr) s += ld_dsmem_f32(dsmem(&sh.ocat[gg][dd], cr));
-            a.out[(bq0 + gg) * D + dd] = s;
+            for (uint32_t cr = 0; cr < C; ++cr) s += oall[(size_t)cr * G * D + i];
+            a.out[bq0 * D + i] = s;
         }
-        if (rank == 0 && tid < G)
+        if (tid < G)
             a.stat[bq0 + tid] = sh.zmax[tid] == -INFINITY ? -INFINITY : (float)((double)sh.zmax[tid] + sh.tau[tid]);
     }
-    cluster_sync();  // no CTA leaves while another may still read its partial output
     pdl_trigger();
 }
 

@@ -1,4 +1,5 @@
-"""One decode step = [page metadata update] -> page scores -> page selection -> sparse attention.
+"""One decode step = [page metadata update] -> page scores -> page selection -> sparse attention
+(the last two in one call for the top-k policy).
 
 SparseDecoder owns the per-step device buffers (scores, selection, outputs, workspace) for a
 fixed cache geometry and policy, and issues the four libekv calls on one stream. It adds no
@@ -73,6 +74,12 @@ class SparseDecoder:
     def step(self, q: torch.Tensor, stream=None):
         c = self.cache
         ekv.ekv_score_pages(c, q, self.num_q_heads, self.scale, self.policy, self.scores, stream)
+        if self.policy == ekv.EKV_SEL_TOPK:
+            # selection and attention in one call (the decode launched behind the selection)
+            ekv.ekv_select_decode(c, q, self.num_q_heads, self.scale, self.attn, self.topk,
+                                  self.scores, self.sel_idx, self.sel_count, self.max_sel,
+                                  self.out, self.stat, self.ws, stream)
+            return self.out, self.stat
         ekv.ekv_select_pages(c, self.num_q_heads, self.policy, self.topk, self.alpha, self.delta,
                              self.scores, self.sel_idx, self.sel_count, self.max_sel,
                              self.tau_hat, stream)

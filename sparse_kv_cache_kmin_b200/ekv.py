@@ -240,6 +240,21 @@ def ekv_sparse_decode(cache: PagedKVCache, q: torch.Tensor, num_q_heads: int, sc
                                             _stream(stream)), "ekv_sparse_decode")
 
 
+def ekv_select_decode(cache: PagedKVCache, q: torch.Tensor, num_q_heads: int, scale: float,
+                      attn: int, topk: int, scores: torch.Tensor, sel_idx: torch.Tensor,
+                      sel_count: torch.Tensor, max_sel: int, out: torch.Tensor, stat: torch.Tensor,
+                      ws: torch.Tensor, stream=None):
+    """Top-k selection and sparse decode in one call: the results of ekv_select_pages (top-k
+    policy) followed by ekv_sparse_decode."""
+    P, I32, F = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float
+    fn = _moment_fn("ekv_select_decode", [ctypes.POINTER(EkvCacheStruct), P, I32, F, I32, I32, P,
+                                          P, P, I32, P, P, P, ctypes.c_size_t, P])
+    c = cache.struct()
+    _check(fn(ctypes.byref(c), _ptr(q), int(num_q_heads), float(scale), int(attn), int(topk),
+              _ptr(scores), _ptr(sel_idx), _ptr(sel_count), int(max_sel), _ptr(out), _ptr(stat),
+              _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)), "ekv_select_decode")
+
+
 def ekv_decode_workspace_bytes(cache: PagedKVCache, num_q_heads: int, max_sel: int) -> int:
     c = cache.struct()
     return int(load_library().ekv_decode_workspace_bytes(ctypes.byref(c), int(num_q_heads),

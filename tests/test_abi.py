@@ -241,3 +241,30 @@ def test_misaligned_scores_and_workspaces_are_refused_before_any_launch(lib):
     tneed = lib.ekv_token_workspace_bytes(C.byref(c), 256)
     assert lib.ekv_select_tokens(C.byref(c), P, 32, 1.0, P, P, 256, 512, P, P, P, P + 8,
                                  tneed + 16, None) == 1
+
+
+def test_select_decode_validation(lib):
+    # the one-call selection + decode refuses what either of its halves refuses, on the host
+    import ctypes as C
+    cp = C.POINTER(type(fake_cache()))
+    vp, i32, f32 = C.c_void_p, C.c_int32, C.c_float
+    fn = lib.ekv_select_decode
+    fn.argtypes = [cp, vp, i32, f32, i32, i32, vp, vp, vp, i32, vp, vp, vp, C.c_size_t, vp]
+    c = fake_cache()
+    P = 0x1000
+    need = lib.ekv_decode_workspace_bytes(C.byref(c), 32, 256)
+
+    def call(topk=64, scores=P, max_sel=256, attn=1, ws=P, ws_bytes=None, q=P, cache=c):
+        return fn(C.byref(cache), q, 32, 1.0, attn, topk, scores, P, P, max_sel, P, P, ws,
+                  need if ws_bytes is None else ws_bytes, None)
+
+    assert call(topk=0) == 1                      # k < 1
+    assert call(topk=200, max_sel=100) == 1       # max_sel < min(k, max_pages)
+    assert call(scores=None) == 1
+    assert call(scores=P + 4) == 1                # score rows are read as float4
+    assert call(q=P + 8) == 1                     # query rows move with 16-byte loads
+    assert call(attn=9) == 2
+    assert call(ws_bytes=need - 1) == 3
+    assert call(ws=None) == 3
+    assert call(ws=P + 4, ws_bytes=need + 16) == 1
+    assert call(cache=fake_cache(v_cache=None)) == 1
