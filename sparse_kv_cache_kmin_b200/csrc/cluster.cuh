@@ -1,5 +1,6 @@
 // cluster.cuh -- thread-block cluster primitives (sm_90+ PTX): rank and size within the
-// cluster, a cluster-wide barrier, and loads from another CTA's shared memory (DSMEM).
+// cluster, a cluster-wide barrier, and loads from and stores to another CTA's shared memory
+// (DSMEM).
 #pragma once
 
 #include "ekv_device.cuh"
@@ -36,6 +37,31 @@ __device__ __forceinline__ int ld_dsmem(uint32_t addr)
     int v;
     asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
     return v;
+}
+__device__ __forceinline__ float ld_dsmem_f32(uint32_t addr)
+{
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+    return v;
+}
+__device__ __forceinline__ double ld_dsmem_f64(uint32_t addr)
+{
+    double v;
+    asm volatile("ld.shared::cluster.f64 %0, [%1];" : "=d"(v) : "r"(addr) : "memory");
+    return v;
+}
+// Stores into another CTA's shared memory (made visible to it by the next cluster barrier).
+__device__ __forceinline__ void st_dsmem_f32(uint32_t addr, float v)
+{
+    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+__device__ __forceinline__ void st_dsmem_s32(uint32_t addr, int v)
+{
+    asm volatile("st.shared::cluster.s32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ void st_dsmem_f64(uint32_t addr, double v)
+{
+    asm volatile("st.shared::cluster.f64 [%0], %1;" ::"r"(addr), "d"(v) : "memory");
 }
 
 }  // namespace ekv

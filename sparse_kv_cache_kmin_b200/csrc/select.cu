@@ -14,7 +14,7 @@
 // with a_j + 8 b_j <= max_j a_j - 1 contribute less than 1e-16 n_j b_j^2 to F at every tau on
 // that path and are dropped before the iterations; the rest are kept in shared memory. Then a
 // block scan keeps page j iff some query g has (alpha-1) UB_gj > tau_hat_g - Delta.
-#include "ekv_device.cuh"
+#include "cluster.cuh"
 #include "topk_cta.cuh"
 
 namespace ekv {
@@ -355,6 +355,15 @@ __device__ __forceinline__ void trunc_moment(float a, float b, float tau, bool s
     }
 }
 
+// Newton step for F^(1/p) = 1 given F and F' (p = 1 sparsemax, p = 2 1.5-entmax):
+// (F^(1/p) - 1) / -(F^(1/p))'.
+__device__ __forceinline__ double newton_step(double F, double dF, bool sparsemax)
+{
+    if (sparsemax) return (F - 1.0) / -dF;
+    const double r = sqrt(F);
+    return (r - 1.0) * 2.0 * r / -dF;
+}
+
 // The same moments in fp64, for the final Newton steps.
 __device__ __forceinline__ void trunc_moment_d(double a, double b, double tau, bool sparsemax,
                                                double &E, double &dE)
@@ -378,51 +387,62 @@ __device__ __forceinline__ void trunc_moment_d(double a, double b, double tau, b
     }
 }
 
-constexpr int kGaussSmemBytes = 192 * 1024;  // survivor lists of one CTA (all G queries)
+constexpr int kGaussSmemBytes = 200 * 1024;  // dynamic shared memory of one CTA at most
+constexpr int kGaussList = 64;                // survivors gathered for warp 0 to iterate on alone
 
-// One CTA per (sequence, KV head); the G queries of the group each get 8/G warps. Each warp owns
-// a slice of the pages and a slice of the survivor list in shared memory: (a_j, b_j, n_j) with
-// a = (alpha-1) m, b = (alpha-1) sqrt(v) and n_j the page's token count. When the slice fits, the
-// warp stages its pages' model with all loads in flight; otherwise it reads them from global
-// memory for the maximum and keeps only the pages that survive the first prune (more than the
-// capacity and it walks global memory on every iteration).
+// One CTA of 4 warps per query; the G CTAs of a (sequence, KV head) form a thread-block
+// cluster. Each warp owns a slice of the pages and a slice of the survivor list in shared
+// memory: (a_j, b_j, n_j) with a = (alpha-1) m, b = (alpha-1) sqrt(v) and n_j the page's token
+// count. When the slice fits, the warp stages its pages' model with all loads in flight;
+// otherwise it reads them from global memory for the maximum and keeps only the pages that
+// survive the first prune (more than the capacity and it walks global memory on every
+// iteration).
 //
-// tau solves F(tau) = sum_j n_j E[(X_j - tau)_+^p] = 1. F is convex and decreasing, so Newton
-// from tau0 = max_j a_j - 1 (where F >= 1) rises monotonically onto the root; the sums are
-// combined over the query's warps each iteration (double-buffered partials, one named barrier).
-// Pages with a + 8 b <= tau contribute below 1e-14 of their count and are pruned every fourth
-// step. The fp32 iterates stop within about 1e-7 of the root; a few Newton steps with fp64
-// moments finish it. The union over the group then lists, in ascending page order, every page with
-// (alpha-1) UB_j > tau_g - delta for some query g.
+// tau solves F(tau) = sum_j n_j E[(X_j - tau)_+^p] = 1. F^(1/p) is convex and decreasing (an
+// L^p norm of (X - tau)_+, each term convex in tau) and close to linear well left of the root,
+// so Newton on F^(1/p) = 1 from tau0 = max_j a_j - 1 (where F >= 1) rises monotonically onto
+// the root in a few steps. Pages with a + 8 b <= tau contribute below 1e-14 of their count.
+// When the first prune at tau0 leaves at most kGaussList pages they are gathered into one list
+// that warp 0 iterates on alone (no barrier per step); larger lists keep every warp on its
+// slice, with the sums combined each step. Survivors are pruned again every fourth step. The fp32 iterates stop
+// within about 1e-5 of the root; a few Newton steps with fp64 moments finish it.
+//
+// Each CTA then stores its tau-hat into every CTA of the cluster; after a cluster barrier CTA
+// g takes the g-th slice of the pages and marks every page with (alpha-1) UB_j > tau_g - delta
+// for some query g of the group (or the Gaussian estimate of the page maximum, est_max), the
+// slices' counts are exchanged the same way, and each CTA writes its kept pages at its offset,
+// in ascending page order.
 template <int G>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(128)
 select_gauss_kernel(const float *__restrict__ scores, int H, int max_pages, int P,
                     const int32_t *__restrict__ seq_lens, float alpha, float delta,
                     int32_t *__restrict__ sel_idx, int32_t *__restrict__ sel_count, int max_sel,
                     float *__restrict__ tau_hat, uint32_t *status, int capw, bool est_max)
 {
-    constexpr int NT = 256, WPQ = 8 / G;
-    extern __shared__ float gdyn[];
-    __shared__ double s_part[2][G][WPQ][2];
-    __shared__ float s_amax[G][WPQ];
-    __shared__ double s_tau[G];
-    __shared__ int warp_tot[8];
+    constexpr int NT = 128, NW = 4;
+    extern __shared__ float gdyn[];  // [NW][3][capw] survivor slices | [3][kGaussList] list | keep bits
+    __shared__ double s_part[2][NW][2];
+    __shared__ float s_amax[NW];
+    __shared__ int s_cnt[NW];
+    __shared__ double s_tau[G];  // every query's tau-hat (stored by the cluster)
+    __shared__ int s_kept[G];    // kept pages of every CTA's slice (stored by the cluster)
     pdl_wait();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int h = blockIdx.x, b = blockIdx.y, bh = b * H + h;
-    const int H_q = H * G;
+    const int g = blockIdx.x % G, h = blockIdx.x / G, b = blockIdx.y, bh = b * H + h;
+    const int H_q = H * G, hq = h * G + g;
     int len;
-    const int n = seq_pages(seq_lens, b, P, max_pages, h == 0 ? status : nullptr, &len);
+    const int n = seq_pages(seq_lens, b, P, max_pages, h == 0 && g == 0 ? status : nullptr, &len);
     const bool sparsemax = alpha == 2.0f;
     const float am1 = alpha - 1.0f;
+    float *la = gdyn + (size_t)NW * 3 * capw, *lb = la + kGaussList, *ln = lb + kGaussList;
+    unsigned *bits = reinterpret_cast<unsigned *>(ln + kGaussList);
 
     {
-        const int g = warp / WPQ, r = warp % WPQ, hq = h * G + g;
         const float *sc = scores + ((size_t)b * H_q + hq) * 3 * max_pages;
         const float *m = sc + max_pages, *v = sc + 2 * (size_t)max_pages;
         float *sa = gdyn + (size_t)warp * 3 * capw, *sb = sa + capw, *sn = sb + capw;
-        const int per = (n + WPQ - 1) / WPQ;
-        const int p0 = min(r * per, n), p1 = min(p0 + per, n);
+        const int per = (n + NW - 1) / NW;
+        const int p0 = min(warp * per, n), p1 = min(p0 + per, n);
         const bool staged = p1 - p0 <= capw;
         auto page_n = [&](int j) { return (float)(len - j * P < P ? len - j * P : P); };
         auto model = [&](int j, float &aj, float &bj) {
@@ -431,7 +451,7 @@ select_gauss_kernel(const float *__restrict__ scores, int H, int max_pages, int 
         };
         float amax = -INFINITY;
         if (staged) {
-            for (int j0 = p0; j0 < p1; j0 += 256) {
+            for (int j0 = p0; j0 < p1; j0 += 256) {  // 8 loads of (m, v) per lane in flight
                 float av[8], bv[8];
 #pragma unroll
                 for (int u = 0; u < 8; ++u) {
@@ -461,12 +481,12 @@ select_gauss_kernel(const float *__restrict__ scores, int H, int max_pages, int 
             }
         }
         amax = warp_max(amax);
-        if (lane == 0) s_amax[g][r] = amax;
-        named_sync(1 + g, 32 * WPQ);
-        amax = s_amax[g][0];
+        if (lane == 0) s_amax[warp] = amax;
+        __syncthreads();
+        amax = s_amax[0];
 #pragma unroll
-        for (int k = 1; k < WPQ; ++k) amax = fmaxf(amax, s_amax[g][k]);
-        double tau = (double)amax - 1.0;
+        for (int k = 1; k < NW; ++k) amax = fmaxf(amax, s_amax[k]);
+        const double tau0 = (double)amax - 1.0;
 
         // first prune: pages that can still contribute at tau >= amax - 1
         int cnt = 0;
@@ -477,7 +497,7 @@ select_gauss_kernel(const float *__restrict__ scores, int H, int max_pages, int 
             if (j < p1) {
                 if (staged) { aj = sa[j - p0]; bj = sb[j - p0]; nj = sn[j - p0]; }
                 else { model(j, aj, bj); nj = page_n(j); }
-                keep = (double)aj + 8.0 * (double)bj > tau;
+                keep = (double)aj + 8.0 * (double)bj > tau0;
             }
             const unsigned bal = __ballot_sync(kFull, keep);
             const int pos = cnt + __popc(bal & ((1u << lane) - 1u));
@@ -486,33 +506,41 @@ select_gauss_kernel(const float *__restrict__ scores, int H, int max_pages, int 
             cnt += __popc(bal);
             __syncwarp();
         }
-        const bool over = cnt > capw;
-
-        int ph = 0;  // parity of the partial-sum buffer of the next combine
-        // Combine a warp's partial F, F' over the query's warps (double-buffered partials, one
-        // named barrier); every warp of the query gets the same sums.
-        auto combine = [&](double Fw, double dFw, double &Fs, double &dFs) {
-            if (lane == 0) { s_part[ph & 1][g][r][0] = Fw; s_part[ph & 1][g][r][1] = dFw; }
-            named_sync(1 + g, 32 * WPQ);
-            Fs = 0.0;
-            dFs = 0.0;
+        if (lane == 0) s_cnt[warp] = cnt;
+        __syncthreads();
+        int total = 0, before = 0;
+        bool any_over = false;
 #pragma unroll
-            for (int k = 0; k < WPQ; ++k) { Fs += s_part[ph & 1][g][k][0]; dFs += s_part[ph & 1][g][k][1]; }
-            ++ph;
-        };
-        if (n == 0) {
-            tau = -INFINITY;
-        } else {
+        for (int w = 0; w < NW; ++w) {
+            total += s_cnt[w];
+            before += w < warp ? s_cnt[w] : 0;
+            any_over = any_over || s_cnt[w] > capw;
+        }
+        const bool solo = !any_over && total <= kGaussList;  // the same in every thread
+        if (solo) {  // gather the survivors into one list
+            for (int i = lane; i < cnt; i += 32) {
+                la[before + i] = sa[i];
+                lb[before + i] = sb[i];
+                ln[before + i] = sn[i];
+            }
+            __syncthreads();
+        }
+
+        // Newton on the list (a, b, n)[0, cnt), or on the warp's pages in global memory (glob);
+        // `reduce` sums the lanes' partial F, F' over the participating threads.
+        auto newton = [&](float *xa, float *xb, float *xn, int cnt, bool glob, auto &&reduce) {
+            double tau = tau0;
+            if (n == 0) return -(double)INFINITY;
 #pragma unroll 1
             for (int it = 0; it < 48; ++it) {
                 float F = 0.f, dF = 0.f;
                 const float tf = (float)tau;
-                if (!over) {
+                if (!glob) {
                     for (int i = lane; i < cnt; i += 32) {
                         float E, dE;
-                        trunc_moment(sa[i], sb[i], tf, sparsemax, E, dE);
-                        F = fmaf(sn[i], E, F);
-                        dF = fmaf(sn[i], dE, dF);
+                        trunc_moment(xa[i], xb[i], tf, sparsemax, E, dE);
+                        F = fmaf(xn[i], E, F);
+                        dF = fmaf(xn[i], dE, dF);
                     }
                 } else {
                     for (int j = p0 + lane; j < p1; j += 32) {
@@ -524,27 +552,27 @@ select_gauss_kernel(const float *__restrict__ scores, int H, int max_pages, int 
                     }
                 }
                 double Fs, dFs;
-                combine(warp_sum((double)F), warp_sum((double)dF), Fs, dFs);
+                reduce((double)F, (double)dF, Fs, dFs);
                 if (!(dFs < 0.0)) break;
-                const double step = (Fs - 1.0) / -dFs;
-                if (!(step > 1e-7 * fmax(1.0, fabs(tau)))) break;
+                const double step = newton_step(Fs, dFs, sparsemax);
+                if (!(step > 1e-5 * fmax(1.0, fabs(tau)))) break;  // the fp64 steps finish it
                 tau += step;
                 // pages with a + 8 b below the (rising) threshold contribute nothing any more
-                if (!over && (it & 3) == 3) {
+                if (!glob && (it & 3) == 3) {
                     int kept = 0;
                     for (int i0 = 0; i0 < cnt; i0 += 32) {
                         const int i = i0 + lane;
                         float ai = 0.f, bi = 0.f, ni = 0.f;
                         bool keep = false;
                         if (i < cnt) {
-                            ai = sa[i]; bi = sb[i]; ni = sn[i];
+                            ai = xa[i]; bi = xb[i]; ni = xn[i];
                             keep = (double)ai + 8.0 * (double)bi > tau;
                         }
                         const unsigned bal = __ballot_sync(kFull, keep);
                         __syncwarp();
                         if (keep) {
                             const int pos = kept + __popc(bal & ((1u << lane) - 1u));
-                            sa[pos] = ai; sb[pos] = bi; sn[pos] = ni;
+                            xa[pos] = ai; xb[pos] = bi; xn[pos] = ni;
                         }
                         kept += __popc(bal);
                         __syncwarp();
@@ -552,19 +580,19 @@ select_gauss_kernel(const float *__restrict__ scores, int H, int max_pages, int 
                     cnt = kept;
                 }
             }
-            // fp64 finish: the fp32 moments above carry about 1e-7 relative error, which bounds
-            // how close the fp32 iterates get to the root. Newton steps on double-precision
-            // moments over the same survivors (pruned pages add below 1e-14 of their count)
-            // take the root to fp64 accuracy; each step squares the error.
+            // fp64 finish: the fp32 moments carry about 1e-7 relative error, which bounds how
+            // close the fp32 iterates can get. Newton steps on double-precision moments over the
+            // same survivors (pruned pages add below 1e-14 of their count) take the root to fp64
+            // accuracy; each step squares the error.
 #pragma unroll 1
-            for (int it = 0; it < 4; ++it) {
+            for (int it = 0; it < 6; ++it) {
                 double F = 0.0, dF = 0.0;
-                if (!over) {
+                if (!glob) {
                     for (int i = lane; i < cnt; i += 32) {
                         double E, dE;
-                        trunc_moment_d(sa[i], sb[i], tau, sparsemax, E, dE);
-                        F = fma((double)sn[i], E, F);
-                        dF = fma((double)sn[i], dE, dF);
+                        trunc_moment_d(xa[i], xb[i], tau, sparsemax, E, dE);
+                        F = fma((double)xn[i], E, F);
+                        dF = fma((double)xn[i], dE, dF);
                     }
                 } else {
                     for (int j = p0 + lane; j < p1; j += 32) {
@@ -577,84 +605,114 @@ select_gauss_kernel(const float *__restrict__ scores, int H, int max_pages, int 
                     }
                 }
                 double Fs, dFs;
-                combine(warp_sum(F), warp_sum(dF), Fs, dFs);
+                reduce(F, dF, Fs, dFs);
                 if (!(dFs < 0.0)) break;
-                const double step = (Fs - 1.0) / -dFs;
+                const double step = newton_step(Fs, dFs, sparsemax);
                 tau += step;
                 if (!(fabs(step) > 1e-13 * fmax(1.0, fabs(tau)))) break;
             }
+            return tau;
+        };
+        double tau = 0.0;
+        if (solo) {
+            if (warp == 0)
+                tau = newton(la, lb, ln, total, false, [&](double F, double dF, double &Fs, double &dFs) {
+                    Fs = warp_sum(F);
+                    dFs = warp_sum(dF);
+                });
+        } else {
+            int ph = 0;  // parity of the partial-sum buffer of the next combine
+            tau = newton(sa, sb, sn, cnt, cnt > capw, [&](double F, double dF, double &Fs, double &dFs) {
+                // the warps' partial sums (double-buffered, one barrier), added in warp order
+                F = warp_sum(F);
+                dF = warp_sum(dF);
+                if (lane == 0) { s_part[ph & 1][warp][0] = F; s_part[ph & 1][warp][1] = dF; }
+                __syncthreads();
+                Fs = 0.0;
+                dFs = 0.0;
+#pragma unroll
+                for (int k = 0; k < NW; ++k) { Fs += s_part[ph & 1][k][0]; dFs += s_part[ph & 1][k][1]; }
+                ++ph;
+            });
         }
-        if (r == 0 && lane == 0) {
-            s_tau[g] = tau;
+        if (tid == 0) {
             tau_hat[(size_t)b * H_q + hq] = (float)tau;
+#pragma unroll
+            for (int r = 0; r < G; ++r) st_dsmem_f64(dsmem(&s_tau[g], (uint32_t)r), tau);
         }
     }
-    __syncthreads();
+    cluster_sync();  // every query's tau-hat has landed in every CTA
 
-    // union over the group, ascending page order: warp w owns pages [q0, q1) in 32-page rows;
-    // the first pass counts, the second writes at the warp's offset. The page statistic is the
-    // bound UB, or (est_max) the Gaussian estimate of the page maximum capped by the bound,
-    // min(UB, m + sqrt(2 ln n) sqrt(v)), decided in fp64.
+    // this CTA's slice of the union, ascending page order: warp w owns rows of 32 pages from
+    // q0; a page's keep flags are computed once and kept as one bit word per row. The page
+    // statistic is the bound UB, or (est_max) the Gaussian estimate of the page maximum capped
+    // by the bound, min(UB, m + sqrt(2 ln n) sqrt(v)), decided in fp64.
     const float *ub0 = scores + ((size_t)b * H_q + h * G) * 3 * max_pages;
     double thr[G];
 #pragma unroll
-    for (int g = 0; g < G; ++g) thr[g] = s_tau[g] - (double)delta;
+    for (int q = 0; q < G; ++q) thr[q] = s_tau[q] - (double)delta;
+    const double zfull = est_max && P > 1 ? sqrt(2.0 * log((double)P)) : 0.0;
     auto keep_page = [&](int j) {
         bool keep = false;
         double zn = 0.0;
         if (est_max) {
             const int nj = len - j * P < P ? len - j * P : P;
-            zn = nj > 1 ? sqrt(2.0 * log((double)nj)) : 0.0;
+            zn = nj == P ? zfull : (nj > 1 ? sqrt(2.0 * log((double)nj)) : 0.0);
         }
 #pragma unroll
-        for (int g = 0; g < G; ++g) {
-            const float *row = ub0 + (size_t)g * 3 * max_pages + j;
+        for (int q = 0; q < G; ++q) {
+            const float *row = ub0 + (size_t)q * 3 * max_pages + j;
             double x = (double)__ldcg(row);
             if (est_max) {
                 const double e = (double)__ldcg(row + max_pages) +
                                  zn * sqrt(fmax((double)__ldcg(row + 2 * (size_t)max_pages), 0.0));
                 x = e < x ? e : x;
             }
-            keep |= (double)am1 * x > thr[g];
+            keep |= (double)am1 * x > thr[q];
         }
         return keep;
     };
-    const int per = ((n + 7) / 8 + 31) & ~31;
-    const int q0 = min(warp * per, n), q1 = min(q0 + per, n);
+    const int u0 = (int)((long long)n * g / G), u1 = (int)((long long)n * (g + 1) / G);
+    const int per = ((u1 - u0 + NW - 1) / NW + 31) & ~31;
+    const int q0 = min(u0 + warp * per, u1), q1 = min(q0 + per, u1);
     int mine = 0;
-    for (int j0 = q0; j0 < q1; j0 += 128) {
-        bool kp[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int j = j0 + u * 32 + lane;
-            kp[u] = j < q1 && keep_page(j);
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) mine += __popc(__ballot_sync(kFull, kp[u]));
+    for (int j0 = q0; j0 < q1; j0 += 32) {
+        const int j = j0 + lane;
+        const unsigned bal = __ballot_sync(kFull, j < q1 && keep_page(j));
+        if (lane == 0) bits[(j0 - u0) >> 5] = bal;
+        mine += __popc(bal);
     }
-    if (lane == 0) warp_tot[warp] = mine;
+    if (lane == 0) s_cnt[warp] = mine;
     __syncthreads();
-    int pos = 0, total = 0;
+    int off = 0, slice = 0;
 #pragma unroll
-    for (int w = 0; w < 8; ++w) {
-        pos += w < warp ? warp_tot[w] : 0;
-        total += warp_tot[w];
+    for (int w = 0; w < NW; ++w) {
+        off += w < warp ? s_cnt[w] : 0;
+        slice += s_cnt[w];
+    }
+    if (tid == 0) {
+#pragma unroll
+        for (int r = 0; r < G; ++r) st_dsmem_s32(dsmem(&s_kept[g], (uint32_t)r), slice);
+    }
+    cluster_sync();  // every slice's count has landed in every CTA
+    int total = 0;
+#pragma unroll
+    for (int r = 0; r < G; ++r) {
+        off += r < g ? s_kept[r] : 0;
+        total += s_kept[r];
     }
     int32_t *out = sel_idx + (size_t)bh * max_sel;
     for (int j0 = q0; j0 < q1; j0 += 32) {
-        const int j = j0 + lane;
-        const bool keep = j < q1 && keep_page(j);
-        const unsigned bal = __ballot_sync(kFull, keep);
-        const int at = pos + __popc(bal & ((1u << lane) - 1u));
-        if (keep && at < max_sel) out[at] = j;
-        pos += __popc(bal);
+        const unsigned bal = bits[(j0 - u0) >> 5];
+        const int at = off + __popc(bal & ((1u << lane) - 1u));
+        if (((bal >> lane) & 1u) && at < max_sel) out[at] = j0 + lane;
+        off += __popc(bal);
     }
-    for (int j = total + tid; j < max_sel; j += NT) out[j] = -1;
-    if (tid == 0) {
+    for (int j = total + g * NT + tid; j < max_sel; j += G * NT) out[j] = -1;
+    if (g == 0 && tid == 0) {
         if (total > max_sel) flag(status, EKV_DEV_SEL_OVERFLOW);
         sel_count[bh] = total < max_sel ? total : max_sel;
     }
-    pdl_trigger();
 }
 
 static cudaLaunchConfig_t pdl_config(dim3 grid, dim3 block, cudaStream_t st, bool pdl,
@@ -703,19 +761,37 @@ cudaError_t launch_select_pages(const ekv_cache &c, int H_q, int policy, int top
                                   c.page_size, c.seq_lens, topk, sel_idx, sel_count, max_sel,
                                   c.dev_status);
     }
-    cudaLaunchConfig_t cfg = pdl_config(grid, dim3(256), st, pdl, attr);
-    const int G = H_q / c.num_kv_heads, wpq = 8 / G;
+    // one CTA per query, the G queries of a (sequence, KV head) in one cluster
+    const int G = H_q / c.num_kv_heads;
+    cudaLaunchAttribute gattr[2];
+    gattr[0].id = cudaLaunchAttributeClusterDimension;
+    gattr[0].val.clusterDim.x = G;
+    gattr[0].val.clusterDim.y = 1;
+    gattr[0].val.clusterDim.z = 1;
+    gattr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    gattr[1].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(c.num_kv_heads * G, c.batch);
+    cfg.blockDim = dim3(128);
+    cfg.stream = st;
+    cfg.attrs = gattr;
+    cfg.numAttrs = pdl ? 2 : 1;
     // per-warp survivor capacity: a warp's whole page slice when the shared memory allows
-    const int cap_max = kGaussSmemBytes / (8 * 3 * (int)sizeof(float));
-    int capw = (c.max_pages + wpq - 1) / wpq;
-    capw = ((capw < cap_max ? capw : cap_max) + 3) & ~3;
-    cfg.dynamicSmemBytes = (size_t)8 * 3 * sizeof(float) * capw;
+    // slices | gathered list | one keep-bit word per 32 pages of a CTA's union slice
+    const size_t bit_words = (size_t)(c.max_pages / G) / 32 + 16;
+    const size_t fixed = sizeof(float) * 3 * kGaussList + sizeof(unsigned) * bit_words;
+    if (fixed + 4 * 3 * sizeof(float) * 64 > (size_t)kGaussSmemBytes) return cudaErrorInvalidValue;
+    const int cap_max = (int)(((size_t)kGaussSmemBytes - fixed) / (4 * 3 * sizeof(float))) & ~3;
+    int capw = (c.max_pages + 3) / 4;
+    capw = ((capw + 3) & ~3) < cap_max ? ((capw + 3) & ~3) : cap_max;
+    cfg.dynamicSmemBytes = sizeof(float) * (size_t)4 * 3 * capw + fixed;
 #define EKV_GSEL(GG)                                                                           \
     [&]() {                                                                                    \
         static bool attr_set = false;                                                          \
         if (!attr_set) {                                                                       \
-            cudaFuncSetAttribute(select_gauss_kernel<GG>,                                      \
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kGaussSmemBytes); \
+            const cudaError_t e = cudaFuncSetAttribute(                                        \
+                select_gauss_kernel<GG>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGaussSmemBytes); \
+            if (e != cudaSuccess) return e;                                                    \
             attr_set = true;                                                                   \
         }                                                                                      \
         return cudaLaunchKernelEx(&cfg, select_gauss_kernel<GG>, scores, c.num_kv_heads,       \

@@ -80,22 +80,6 @@ struct AttShared {
     float opart[kAttWarps][D];
 };
 
-__device__ __forceinline__ float ld_dsmem_f32(uint32_t addr)
-{
-    float v;
-    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
-    return v;
-}
-__device__ __forceinline__ double ld_dsmem_f64(uint32_t addr)
-{
-    double v;
-    asm volatile("ld.shared::cluster.f64 %0, [%1];" : "=d"(v) : "r"(addr) : "memory");
-    return v;
-}
-__device__ __forceinline__ void st_dsmem_f32(uint32_t addr, float v)
-{
-    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
-}
 __device__ __forceinline__ void st_shared_v4(void *p, const uint4 &v)
 {
     asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(smem_addr(p)), "r"(v.x), "r"(v.y),
