@@ -364,6 +364,16 @@ ekv_status ekv_device_status(const ekv_cache *c, uint32_t *bits, void *stream);
 /* Clear *c->dev_status (asynchronous). */
 ekv_status ekv_clear_device_status(const ekv_cache *c, void *stream);
 
+/*
+ * Self-test of the device-side timeout reporting. (The paper has no counterpart: this is a
+ * library diagnostic.) Every pipelined kernel bounds each of its waits with the global timer and
+ * sets EKV_DEV_TIMEOUT in *c->dev_status when a limit (2 s) runs out, instead of hanging. This
+ * call launches one thread that waits, with that same bounded wait, on a barrier nothing ever
+ * completes, for limit_ns nanoseconds (at most 2e9; larger values: EKV_ERR_INVALID_ARG), then
+ * sets EKV_DEV_TIMEOUT and returns. Asynchronous; read the bit with ekv_device_status.
+ */
+ekv_status ekv_wait_selftest(const ekv_cache *c, uint64_t limit_ns, void *stream);
+
 /* A static, human-readable name for a status code. */
 const char *ekv_status_str(ekv_status s);
 

@@ -1169,22 +1169,12 @@ static cudaError_t launch_decode_g(const DecodeArgs &a, int G, bool softmax, cud
     }
 }
 
-cudaError_t launch_step_attend(const ekv_cache &c, const void *q, int H_q, float scale, int attn,
-                               const int32_t *sel_idx, const int32_t *sel_count, int max_sel,
-                               float *out, float *stat, cudaStream_t st, bool pdl, bool *launched);
 
 cudaError_t launch_sparse_decode(const ekv_cache &c, const void *q, int H_q, float scale,
                                  int attn, const int32_t *sel_idx, const int32_t *sel_count,
                                  int max_sel, float *out, float *stat, void *ws, cudaStream_t st,
                                  bool pdl)
 {
-    // bf16 entmax: one thread-block cluster per (sequence, KV head) computes the logits, the
-    // exact threshold and the output with the logits kept on chip (step_attend.cu); other
-    // calls, or selections too large for the cluster's shared memory, take the chunk kernels
-    bool done = false;
-    cudaError_t e0 = launch_step_attend(c, q, H_q, scale, attn, sel_idx, sel_count, max_sel, out,
-                                        stat, st, pdl, &done);
-    if (e0 != cudaSuccess || done) return e0;
     DecodeArgs a;
     size_t off_o, off_logits, off_blk;
     mode_layout(c.batch, H_q, c.num_kv_heads, c.head_dim, c.page_size, c.dtype, max_sel,

@@ -49,6 +49,7 @@ cudaError_t launch_selection_quality(const ekv_cache &c, const void *q, int H_q,
                                      int32_t *support, cudaStream_t st);
 
 bool step_score_select_supported(const ekv_cache &c);
+cudaError_t launch_wait_selftest(uint32_t *status, uint64_t limit_ns, cudaStream_t st);
 cudaError_t launch_step_score_select(const ekv_cache &c, const void *q, int H_q, float scale,
                                      int topk, float *scores, int32_t *sel_idx, int32_t *sel_count,
                                      int max_sel, cudaStream_t st, bool pdl);
@@ -400,6 +401,12 @@ ekv_status ekv_clear_device_status(const ekv_cache *c, void *stream)
     if (!c || !c->dev_status) return EKV_ERR_INVALID_ARG;
     return cuda_status(cudaMemsetAsync(c->dev_status, 0, sizeof(uint32_t),
                                        static_cast<cudaStream_t>(stream)));
+}
+
+ekv_status ekv_wait_selftest(const ekv_cache *c, uint64_t limit_ns, void *stream)
+{
+    if (!c || !c->dev_status || limit_ns > 2000000000ull) return EKV_ERR_INVALID_ARG;
+    return cuda_status(launch_wait_selftest(c->dev_status, limit_ns, static_cast<cudaStream_t>(stream)));
 }
 
 const char *ekv_status_str(ekv_status s)

@@ -238,4 +238,23 @@ cudaError_t launch_page_meta_update(const ekv_cache &c, const int32_t *new_start
     return cudaGetLastError();
 }
 
+// The device-side timeout path on its own: one thread waits on an mbarrier that nothing ever
+// arrives on, with the bounded wait every pipelined kernel uses; when the limit runs out it sets
+// EKV_DEV_TIMEOUT and the kernel returns. No copy is in flight, so giving up is always safe.
+__global__ void wait_selftest_kernel(uint32_t *status, uint64_t limit_ns)
+{
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+        if (!mbar_wait_bounded(&bar, 0, limit_ns)) flag(status, EKV_DEV_TIMEOUT);
+    }
+}
+
+cudaError_t launch_wait_selftest(uint32_t *status, uint64_t limit_ns, cudaStream_t st)
+{
+    wait_selftest_kernel<<<1, 32, 0, st>>>(status, limit_ns);
+    return cudaGetLastError();
+}
+
 }  // namespace ekv

@@ -255,6 +255,15 @@ def ekv_select_decode(cache: PagedKVCache, q: torch.Tensor, num_q_heads: int, sc
               _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)), "ekv_select_decode")
 
 
+def ekv_wait_selftest(cache: PagedKVCache, limit_ns: int, stream=None):
+    """One thread waits on a barrier nothing completes, bounded by limit_ns, then sets
+    EKV_DEV_TIMEOUT in the cache's status word (the device-side timeout path on its own)."""
+    fn = _moment_fn("ekv_wait_selftest", [ctypes.POINTER(EkvCacheStruct), ctypes.c_uint64,
+                                          ctypes.c_void_p])
+    c = cache.struct()
+    _check(fn(ctypes.byref(c), int(limit_ns), _stream(stream)), "ekv_wait_selftest")
+
+
 def ekv_decode_workspace_bytes(cache: PagedKVCache, num_q_heads: int, max_sel: int) -> int:
     c = cache.struct()
     return int(load_library().ekv_decode_workspace_bytes(ctypes.byref(c), int(num_q_heads),

@@ -268,3 +268,13 @@ def test_select_decode_validation(lib):
     assert call(ws=None) == 3
     assert call(ws=P + 4, ws_bytes=need + 16) == 1
     assert call(cache=fake_cache(v_cache=None)) == 1
+
+
+def test_wait_selftest_validation(lib):
+    import ctypes as C
+    cp = C.POINTER(type(fake_cache()))
+    lib.ekv_wait_selftest.argtypes = [cp, C.c_uint64, C.c_void_p]
+    c = fake_cache()
+    assert lib.ekv_wait_selftest(C.byref(c), 2_000_000_001, None) == 1   # above the 2 s limit
+    c2 = fake_cache(dev_status=None)
+    assert lib.ekv_wait_selftest(C.byref(c2), 1000, None) == 1

@@ -274,6 +274,23 @@ def test_bad_page_table_entry_is_flagged_not_trapped(cuda_device):
     check_head(wl, cache, dec, 0, 1, ekv.EKV_SOFTMAX)
 
 
+def test_bounded_wait_gives_up_and_reports_a_timeout(cuda_device):
+    # the device-side timeout path on its own: a wait on a barrier nothing completes gives up
+    # after 1 ms, sets EKV_DEV_TIMEOUT and returns; the context stays usable
+    wl = make_random(B=2, H_kv=2, G=4, d=128, P=16, lens=(700, 300), dtype=torch.bfloat16,
+                     device="cuda", seed=14, topk=8)
+    cache = make_cache(wl)
+    prefill_metadata(cache, wl)
+    ekv.ekv_clear_device_status(cache)
+    ekv.ekv_wait_selftest(cache, 1_000_000)
+    st, bits = ekv.ekv_device_status(cache)
+    assert st == ekv.EKV_ERR_DEVICE and bits == ekv.EKV_DEV_TIMEOUT
+    ekv.ekv_clear_device_status(cache)
+    _, dec = run_gpu(wl, ekv.EKV_ENTMAX15, cache=cache)
+    assert_status_ok(cache)
+    check_head(wl, cache, dec, 1, 1, ekv.EKV_ENTMAX15)
+
+
 def test_bad_selection_is_flagged(cuda_device):
     wl = make_random(B=1, H_kv=1, G=1, d=64, P=16, lens=(100,), dtype=torch.float32,
                      device="cuda", seed=14)
