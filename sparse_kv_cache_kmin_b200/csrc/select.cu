@@ -652,7 +652,18 @@ select_gauss_kernel(const float *__restrict__ scores, int H, int max_pages, int 
 #pragma unroll
     for (int q = 0; q < G; ++q) thr[q] = s_tau[q] - (double)delta;
     const double zfull = est_max && P > 1 ? sqrt(2.0 * log((double)P)) : 0.0;
-    auto keep_page = [&](int j) {
+    // the page statistics of G queries for page j (rows past q1 read nothing)
+    struct PageStats { float ub[G], m[G], v[G]; };
+    auto load_page = [&](int j, bool in, PageStats &ps) {
+#pragma unroll
+        for (int q = 0; q < G; ++q) {
+            const float *row = ub0 + (size_t)q * 3 * max_pages + j;
+            ps.ub[q] = in ? __ldcg(row) : 0.f;
+            ps.m[q] = in && est_max ? __ldcg(row + max_pages) : 0.f;
+            ps.v[q] = in && est_max ? __ldcg(row + 2 * (size_t)max_pages) : 0.f;
+        }
+    };
+    auto keep_page = [&](int j, const PageStats &ps) {
         bool keep = false;
         double zn = 0.0;
         if (est_max) {
@@ -661,11 +672,9 @@ select_gauss_kernel(const float *__restrict__ scores, int H, int max_pages, int 
         }
 #pragma unroll
         for (int q = 0; q < G; ++q) {
-            const float *row = ub0 + (size_t)q * 3 * max_pages + j;
-            double x = (double)__ldcg(row);
+            double x = (double)ps.ub[q];
             if (est_max) {
-                const double e = (double)__ldcg(row + max_pages) +
-                                 zn * sqrt(fmax((double)__ldcg(row + 2 * (size_t)max_pages), 0.0));
+                const double e = (double)ps.m[q] + zn * sqrt(fmax((double)ps.v[q], 0.0));
                 x = e < x ? e : x;
             }
             keep |= (double)am1 * x > thr[q];
@@ -676,11 +685,18 @@ select_gauss_kernel(const float *__restrict__ scores, int H, int max_pages, int 
     const int per = ((u1 - u0 + NW - 1) / NW + 31) & ~31;
     const int q0 = min(u0 + warp * per, u1), q1 = min(q0 + per, u1);
     int mine = 0;
-    for (int j0 = q0; j0 < q1; j0 += 32) {
-        const int j = j0 + lane;
-        const unsigned bal = __ballot_sync(kFull, j < q1 && keep_page(j));
-        if (lane == 0) bits[(j0 - u0) >> 5] = bal;
-        mine += __popc(bal);
+    for (int j0 = q0; j0 < q1; j0 += 64) {  // two rows of 32 pages, all their loads in flight
+        const int ja = j0 + lane, jb = j0 + 32 + lane;
+        PageStats sa_, sb_;
+        load_page(ja, ja < q1, sa_);
+        load_page(jb, jb < q1, sb_);
+        const unsigned ba = __ballot_sync(kFull, ja < q1 && keep_page(ja, sa_));
+        const unsigned bb = __ballot_sync(kFull, jb < q1 && keep_page(jb, sb_));
+        if (lane == 0) {
+            bits[(j0 - u0) >> 5] = ba;
+            if (j0 + 32 < q1) bits[((j0 - u0) >> 5) + 1] = bb;
+        }
+        mine += __popc(ba) + __popc(bb);
     }
     if (lane == 0) s_cnt[warp] = mine;
     __syncthreads();
