@@ -112,8 +112,8 @@ token_score_kernel(ekv_cache c, const void *__restrict__ q, int H_q, float scale
 
 // One CTA per (sequence, query head), the kept tokens' logits in shared memory.
 //   softmax: p = exp(s - max) / sum, stat = log sum exp(s);
-//   entmax:  z = (alpha - 1) s; tau by bisection on f(tau) = sum [z - tau]_+^(1/(alpha-1)) - 1
-//            over [max z - 1, max z] in fp64, then recomputed in closed form over the support
+//   entmax:  z = (alpha - 1) s; tau by Newton on f(tau)^(alpha-1) = 1, f = sum [z - tau]_+^(1/(alpha-1)),
+//            from max z - 1 in fp64, then recomputed in closed form over the support
 //            {z > tau} (sparsemax: (sum_S z - 1) / |S|; 1.5-entmax: mean_S - sqrt((1 -
 //            sum_S (z - mean_S)^2) / |S|)); p = [z - tau]_+^(1/(alpha-1)), stat = tau.
 //   out = sum_i p_i v_i, reading only rows with p_i > 0.
@@ -126,7 +126,7 @@ token_attend_kernel(ekv_cache c, const void *__restrict__ q, int H_q, float scal
 {
     extern __shared__ float zs[];   // [T] logits, then weights
     __shared__ float qs[D];
-    __shared__ double dred[8];
+    __shared__ double dred[8], dred2[8];
     __shared__ float fred[8];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int hq = blockIdx.x, b = blockIdx.y, h = hq / G;
@@ -231,6 +231,18 @@ token_attend_kernel(ekv_cache c, const void *__restrict__ q, int H_q, float scal
         __syncthreads();
         return s;
     };
+    auto block_dsum2 = [&](double &v, double &w) {  // two sums in one round of barriers
+        v = warp_sum(v);
+        w = warp_sum(w);
+        if (lane == 0) { dred[warp] = v; dred2[warp] = w; }
+        __syncthreads();
+        double s = 0.0, t = 0.0;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) { s += dred[k]; t += dred2[k]; }
+        __syncthreads();
+        v = s;
+        w = t;
+    };
     float mx = -INFINITY;
     for (int i = tid; i < n; i += 256) mx = fmaxf(mx, zs[i]);
     mx = block_max(mx);
@@ -253,16 +265,31 @@ token_attend_kernel(ekv_cache c, const void *__restrict__ q, int H_q, float scal
         st = mx + (float)log(l);
     } else {
         const bool sparse = attn == EKV_SPARSEMAX;
-        double lo = (double)mx - 1.0, hi = (double)mx;  // the sum is >= 1 at lo and 0 at hi
-        for (int it = 0; it < 60; ++it) {
-            const double mid = 0.5 * (lo + hi);
-            double f = 0.0;
+        // Newton on F^(1/p) = 1, F(t) = sum [z - t]_+^p (p = 1 sparsemax, 2 1.5-entmax): F^(1/p)
+        // is an l^p norm of (z - t)_+, so it is convex and decreasing, and Newton from
+        // t = max z - 1 (where F >= 1) rises monotonically onto the root (for sparsemax F is
+        // piecewise linear and the iteration ends once the support is found)
+        double lo = (double)mx - 1.0;
+        for (int it = 0; it < 64; ++it) {
+            double f = 0.0, df = 0.0;
             for (int i = tid; i < n; i += 256) {
-                const double r = (double)zs[i] - mid;
-                if (r > 0.0) f += sparse ? r : r * r;
+                const double r = (double)zs[i] - lo;
+                if (r > 0.0) {
+                    f += sparse ? r : r * r;
+                    df -= sparse ? 1.0 : 2.0 * r;
+                }
             }
-            f = block_dsum(f);
-            if (f >= 1.0) lo = mid; else hi = mid;
+            block_dsum2(f, df);
+            if (!(df < 0.0)) break;
+            double step;
+            if (sparse) {
+                step = (f - 1.0) / -df;
+            } else {
+                const double rf = sqrt(f);
+                step = (rf - 1.0) * 2.0 * rf / -df;
+            }
+            if (!(step > 1e-13 * fmax(1.0, fabs(lo)))) break;
+            lo += step;
         }
         // closed form over the support {z > lo}
         double s1 = 0.0, s2 = 0.0, k = 0.0;
