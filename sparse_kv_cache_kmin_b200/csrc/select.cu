@@ -828,10 +828,30 @@ cudaError_t launch_select_pages(const ekv_cache &c, int H_q, int policy, int top
 
 namespace ekv {
 
+// The kk largest of n scores S[0, n) (kk < n <= R * kSelThreads), key descending then index
+// ascending, written to out[0, kk) in ascending index order: each thread holds R consecutive
+// keys in registers and cta_topk decides.
+template <int R>
+__device__ void emit_topk_reg(const float *S, int n, int kk, TopkShared &ts, int32_t *out)
+{
+    constexpr int NT = kSelThreads;
+    const int j0 = threadIdx.x * R;
+    uint32_t u[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) u[r] = j0 + r < n ? topk_order_key(__ldcg(S + j0 + r)) : 0u;
+    bool keep[R];
+    const int mine = cta_topk<NT, R>(u, n, kk, ts, keep);
+    int pos = block_incl_scan<NT>(mine, ts.warp_tot, nullptr) - mine;
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+        if (keep[r] && pos < kk) out[pos++] = j0 + r;
+}
+
 // Token-level top-T inside the selected pages, one 1024-thread CTA per (sequence, KV head).
 // The candidate scores sit at slot i * P + t (selected page i, position t; -inf past a page's
 // valid tokens); the exact radix select above keeps the T largest, ties to the lower slot, in
-// slot order -- which is the candidate order (selection order, then position). Emits
+// slot order -- which is the candidate order (selection order, then position); up to 16384
+// slots the keys are held in registers (emit_topk_reg). Emits
 // (logical page, position) pairs, -1 padded to T, and the count.
 __global__ void __launch_bounds__(kSelThreads)
 select_tokens_kernel(const float *__restrict__ tscores, int H, int P, const int32_t *__restrict__ seq_lens,
@@ -844,6 +864,7 @@ select_tokens_kernel(const float *__restrict__ tscores, int H, int P, const int3
     __shared__ int hist[2048];
     __shared__ int warp_tot[32];
     __shared__ int s_bin, s_above;
+    __shared__ TopkShared ts;
     pdl_wait();
     const int tid = threadIdx.x;
     const int bh = blockIdx.x, b = bh / H;
@@ -876,6 +897,12 @@ select_tokens_kernel(const float *__restrict__ tscores, int H, int P, const int3
                 pos += tot;
             }
             kk = pos < kk ? pos : kk;  // a non-finite score is not a candidate
+        } else if (n <= 4 * NT) {
+            emit_topk_reg<4>(S, n, kk, ts, ps);
+        } else if (n <= 8 * NT) {
+            emit_topk_reg<8>(S, n, kk, ts, ps);
+        } else if (n <= 16 * NT) {
+            emit_topk_reg<16>(S, n, kk, ts, ps);
         } else {
             radix_select_emit(n, kk, [&](int j) { return order_key(__ldcg(S + j)); }, hist, warp_tot,
                               &s_bin, &s_above, ps);
