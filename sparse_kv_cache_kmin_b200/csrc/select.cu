@@ -451,16 +451,16 @@ select_gauss_kernel(const float *__restrict__ scores, int H, int max_pages, int 
         };
         float amax = -INFINITY;
         if (staged) {
-            for (int j0 = p0; j0 < p1; j0 += 256) {  // 8 loads of (m, v) per lane in flight
-                float av[8], bv[8];
+            for (int j0 = p0; j0 < p1; j0 += 512) {  // 16 loads of (m, v) per lane in flight
+                float av[16], bv[16];
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
+                for (int u = 0; u < 16; ++u) {
                     const int j = j0 + u * 32 + lane;
                     av[u] = -INFINITY; bv[u] = 0.f;
                     if (j < p1) model(j, av[u], bv[u]);
                 }
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
+                for (int u = 0; u < 16; ++u) {
                     const int j = j0 + u * 32 + lane;
                     if (j < p1) {
                         sa[j - p0] = av[u]; sb[j - p0] = bv[u]; sn[j - p0] = page_n(j);
@@ -527,7 +527,7 @@ select_gauss_kernel(const float *__restrict__ scores, int H, int max_pages, int 
         }
 
         // Newton on the list (a, b, n)[0, cnt), or on the warp's pages in global memory (glob);
-        // `reduce` sums the lanes' partial F, F' over the participating threads.
+        // `reduce` adds the warps' totals of F, F' over the participating warps.
         auto newton = [&](float *xa, float *xb, float *xn, int cnt, bool glob, auto &&reduce) {
             double tau = tau0;
             if (n == 0) return -(double)INFINITY;
@@ -536,6 +536,7 @@ select_gauss_kernel(const float *__restrict__ scores, int H, int max_pages, int 
                 float F = 0.f, dF = 0.f;
                 const float tf = (float)tau;
                 if (!glob) {
+#pragma unroll 2
                     for (int i = lane; i < cnt; i += 32) {
                         float E, dE;
                         trunc_moment(xa[i], xb[i], tf, sparsemax, E, dE);
@@ -551,8 +552,8 @@ select_gauss_kernel(const float *__restrict__ scores, int H, int max_pages, int 
                         dF = fmaf(page_n(j), dE, dF);
                     }
                 }
-                double Fs, dFs;
-                reduce((double)F, (double)dF, Fs, dFs);
+                double Fs, dFs;  // fp32 warp sums are enough for these iterates
+                reduce((double)warp_sum(F), (double)warp_sum(dF), Fs, dFs);
                 if (!(dFs < 0.0)) break;
                 const double step = newton_step(Fs, dFs, sparsemax);
                 if (!(step > 1e-5 * fmax(1.0, fabs(tau)))) break;  // the fp64 steps finish it
@@ -605,7 +606,7 @@ select_gauss_kernel(const float *__restrict__ scores, int H, int max_pages, int 
                     }
                 }
                 double Fs, dFs;
-                reduce(F, dF, Fs, dFs);
+                reduce(warp_sum(F), warp_sum(dF), Fs, dFs);
                 if (!(dFs < 0.0)) break;
                 const double step = newton_step(Fs, dFs, sparsemax);
                 tau += step;
@@ -617,15 +618,13 @@ select_gauss_kernel(const float *__restrict__ scores, int H, int max_pages, int 
         if (solo) {
             if (warp == 0)
                 tau = newton(la, lb, ln, total, false, [&](double F, double dF, double &Fs, double &dFs) {
-                    Fs = warp_sum(F);
-                    dFs = warp_sum(dF);
+                    Fs = F;  // the warp's totals are the sums
+                    dFs = dF;
                 });
         } else {
             int ph = 0;  // parity of the partial-sum buffer of the next combine
             tau = newton(sa, sb, sn, cnt, cnt > capw, [&](double F, double dF, double &Fs, double &dFs) {
-                // the warps' partial sums (double-buffered, one barrier), added in warp order
-                F = warp_sum(F);
-                dF = warp_sum(dF);
+                // the warps' totals (double-buffered, one barrier), added in warp order
                 if (lane == 0) { s_part[ph & 1][warp][0] = F; s_part[ph & 1][warp][1] = dF; }
                 __syncthreads();
                 Fs = 0.0;
