@@ -217,7 +217,7 @@ class ClockSampler:
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.QUERY,
-                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
+                 "--format=csv,noheader,nounits", "-lms", "50"], stdout=self.f,
                 stderr=subprocess.DEVNULL)
             time.sleep(0.3)
         except Exception:
@@ -646,6 +646,15 @@ def main():
         pg.barrier()
     torch.cuda.synchronize()
     with ClockSampler(local) as clocks:
+        # The timed steps last milliseconds, shorter than the clock sampling period; the same
+        # flush-and-step loop runs for about half a second before them (untimed) so that the
+        # samples see the GPU under this load, then the timed steps follow back to back.
+        t_end = time.time() + 0.5
+        while time.time() < t_end:
+            for i in range(20):
+                flush.fill_(i & 0xff)
+                graph.replay()
+            torch.cuda.synchronize()
         for i in range(args.steps):
             flush.fill_(i & 0xff)
             ev[i][0].record(stream)

@@ -7,8 +7,9 @@
 // shrinking key range [lo, hi]: a bin is a run of 2^s consecutive keys, s the fewest bits
 // that leave at most 2048 bins (a subtraction and a shift per key, and each bin an exact key
 // interval); the bin holding the k-th largest key becomes the next range. Once that bin holds
-// at most kTopkRank keys they are ranked exactly (key descending, page ascending); once the
-// range is a single key value, the remaining ties are kept in page order by a block scan.
+// at most kTopkRank keys they are ranked exactly (key descending, page ascending) -- or all
+// kept, when the bin holds exactly the keys still needed; once the range is a single key value,
+// the remaining ties are kept in page order by a block scan.
 // Every key above the final range is kept. Three refinements always reach a single value; on
 // scores from a continuous distribution one suffices.
 #pragma once
@@ -32,7 +33,7 @@ struct __align__(16) TopkShared {
     uint32_t rk_u[kTopkRank];
     int rk_j[kTopkRank];
     uint32_t lo, hi, bin_lo, bin_hi;
-    int bin, above, cnt, mode;  // mode: 0 rank the boundary bin, 1 ties in page order
+    int bin, above, cnt, mode;  // mode: 0 rank the boundary bin, 1 ties in page order, 2 keep it
 };
 
 // Bin width 2^s for the range [lo, hi]: (hi - lo) >> s < 2048.
@@ -60,6 +61,7 @@ __device__ int cta_topk(const uint32_t (&u)[R], int n, int kk, TopkShared &s, bo
         mx = max(mx, __shfl_xor_sync(kFull, mx, o));
     }
     if (tid == 0) { s.lo = 0xffffffffu; s.hi = 0u; }
+    for (int i = tid; i < kTopkBins; i += NT) s.hist[i] = 0;  // the first pass's histogram
     __syncthreads();
     if (lane == 0) { atomicMin(&s.lo, mn); atomicMax(&s.hi, mx); }
     __syncthreads();
@@ -72,8 +74,10 @@ __device__ int cta_topk(const uint32_t (&u)[R], int n, int kk, TopkShared &s, bo
             break;
         }
         const int sh = topk_shift(lo, hi);
-        for (int i = tid; i < kTopkBins; i += NT) s.hist[i] = 0;
-        __syncthreads();
+        if (pass > 0) {
+            for (int i = tid; i < kTopkBins; i += NT) s.hist[i] = 0;
+            __syncthreads();
+        }
 #pragma unroll
         for (int r = 0; r < R; ++r)
             if (j0 + r < n && u[r] >= lo && u[r] <= hi) atomicAdd(&s.hist[(u[r] - lo) >> sh], 1);
@@ -106,6 +110,10 @@ __device__ int cta_topk(const uint32_t (&u)[R], int n, int kk, TopkShared &s, bo
         need -= s.above;
         lo = s.bin_lo;
         hi = s.bin_hi;
+        if (s.cnt == need) {  // the whole boundary bin is kept: nothing to rank
+            if (tid == 0) s.mode = 2;
+            break;
+        }
         if (s.cnt <= kTopkRank) {
             if (tid == 0) s.mode = 0;
             break;
@@ -150,6 +158,12 @@ __device__ int cta_topk(const uint32_t (&u)[R], int n, int kk, TopkShared &s, bo
             const int j = j0 + r;
             keep[r] = j < n && (u[r] > hi ||
                                 (u[r] >= lo && ((reinterpret_cast<const unsigned *>(s.hist)[j >> 5] >> (j & 31)) & 1u)));
+            mine += keep[r];
+        }
+    } else if (s.mode == 2) {
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            keep[r] = j0 + r < n && u[r] >= lo;
             mine += keep[r];
         }
     } else {
