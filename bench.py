@@ -642,19 +642,21 @@ def main():
 
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(args.steps)]
-    if pg:
-        pg.barrier()
-    torch.cuda.synchronize()
     with ClockSampler(local) as clocks:
         # The timed steps last milliseconds, shorter than the clock sampling period; the same
-        # flush-and-step loop runs for about half a second before them (untimed) so that the
-        # samples see the GPU under this load, then the timed steps follow back to back.
-        t_end = time.time() + 0.5
-        while time.time() < t_end:
+        # flush-and-step loop runs for about half a second before them (untimed; no collective
+        # inside) so that the samples see the GPU under this load, then the timed steps follow,
+        # bracketed by a barrier and a device synchronisation.
+        rounds, t_end = 0, time.time() + 0.5
+        while time.time() < t_end and rounds < 1000:
             for i in range(20):
                 flush.fill_(i & 0xff)
                 graph.replay()
             torch.cuda.synchronize()
+            rounds += 1
+        if pg:
+            pg.barrier()
+        torch.cuda.synchronize()
         for i in range(args.steps):
             flush.fill_(i & 0xff)
             ev[i][0].record(stream)
