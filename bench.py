@@ -471,17 +471,6 @@ class Step:
             self.run()
         return g
 
-    def graph_with_events(self):
-        """The same calls with an event node around each (per-call durations)."""
-        ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(self.calls) + 1)]
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            ev[0].record()
-            for i, (_, fn) in enumerate(self.calls):
-                fn()
-                ev[i + 1].record()
-        return g, ev
-
     def graph_host(self, q_host, out_host, stat_host, host_pre=None):
         """A whole host-to-host step: the query copied in from pinned host memory, the calls,
         the outputs copied back to pinned host buffers."""
@@ -623,14 +612,12 @@ def main():
         flush.fill_(1)
         step.run()
     torch.cuda.synchronize()
-    # graph A: the step as one launch (the timed loop); graph B: the same calls with an event
-    # node between them (per-call durations)
+    # the step as one graph launch (the timed loop)
     graph = step.graph()
     try:
         launches_per_step, launches_src = graph_kernel_nodes(graph), "kernel nodes of the step graph"
     except Exception as exc:  # the count then comes from the calls' known kernel counts
         launches_per_step, launches_src = step.launches(), "per-call table (%s)" % type(exc).__name__
-    graph_b, evb = step.graph_with_events()
 
     for _ in range(max(args.warmup, 3)):
         flush.fill_(1)
@@ -666,15 +653,21 @@ def main():
         if pg:
             pg.barrier()
         step_ms = [a.elapsed_time(b) for a, b in ev]
-        # per-call durations over K more steps of graph B (same work, event nodes between calls)
+        # per-call durations: each call launched on its own K more times, bracketed by events on
+        # the launching stream, behind an L2 flush that keeps the GPU busy while the host queues
+        # the call (so the events time the call's kernels, not the host)
         names = [n for n, _ in step.calls]
         part_ms = {n: [] for n in names}
-        for i in range(args.steps):
-            flush.fill_(i & 0xff)
-            graph_b.replay()
+        for n, fn in step.calls:
+            pev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(args.steps)]
+            for i in range(args.steps):
+                flush.fill_(i & 0xff)
+                pev[i][0].record(stream)
+                fn()
+                pev[i][1].record(stream)
             torch.cuda.synchronize()
-            for j, n in enumerate(names):
-                part_ms[n].append(evb[j].elapsed_time(evb[j + 1]))
+            part_ms[n] = [a.elapsed_time(b) for a, b in pev]
     total_s = replicas.max_over_ranks(sum(step_ms) / 1e3, device=dev)
     median_ms = replicas.max_over_ranks(statistics.median(step_ms), device=dev)
     st, bits = ekv.ekv_device_status(cache)
