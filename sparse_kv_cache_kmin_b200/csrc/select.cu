@@ -531,6 +531,7 @@ select_gauss_kernel(const float *__restrict__ scores, int H, int max_pages, int 
         auto newton = [&](float *xa, float *xb, float *xn, int cnt, bool glob, auto &&reduce) {
             double tau = tau0;
             if (n == 0) return -(double)INFINITY;
+            bool settled = false;  // the fp32 iterates met their step tolerance
 #pragma unroll 1
             for (int it = 0; it < 48; ++it) {
                 float F = 0.f, dF = 0.f;
@@ -556,7 +557,10 @@ select_gauss_kernel(const float *__restrict__ scores, int H, int max_pages, int 
                 reduce((double)warp_sum(F), (double)warp_sum(dF), Fs, dFs);
                 if (!(dFs < 0.0)) break;
                 const double step = newton_step(Fs, dFs, sparsemax);
-                if (!(step > 1e-5 * fmax(1.0, fabs(tau)))) break;  // the fp64 steps finish it
+                if (!(step > 1e-5 * fmax(1.0, fabs(tau)))) {  // the fp64 steps finish it
+                    settled = step > -1e-5 * fmax(1.0, fabs(tau));
+                    break;
+                }
                 tau += step;
                 // pages with a + 8 b below the (rising) threshold contribute nothing any more
                 if (!glob && (it & 3) == 3) {
@@ -584,9 +588,10 @@ select_gauss_kernel(const float *__restrict__ scores, int H, int max_pages, int 
             // fp64 finish: the fp32 moments carry about 1e-7 relative error, which bounds how
             // close the fp32 iterates can get. Newton steps on double-precision moments over the
             // same survivors (pruned pages add below 1e-14 of their count) take the root to fp64
-            // accuracy; each step squares the error.
+            // accuracy; each step squares the error, so from settled fp32 iterates (within about
+            // 1e-5) two steps reach it.
 #pragma unroll 1
-            for (int it = 0; it < 6; ++it) {
+            for (int it = 0; it < (settled ? 2 : 6); ++it) {
                 double F = 0.0, dF = 0.0;
                 if (!glob) {
                     for (int i = lane; i < cnt; i += 32) {
