@@ -91,6 +91,32 @@ def test_gauss_estimated_max_on_the_gauss_workload(cuda_device):
         check_head(wl, cache, dec, b, h, ekv.EKV_ENTMAX15)
 
 
+@pytest.mark.parametrize("policy", [GAUSS, GAUSS_MAX], ids=["gauss", "gauss_max"])
+@pytest.mark.parametrize("attn", [ekv.EKV_ENTMAX15, ekv.EKV_SPARSEMAX])
+def test_gauss_two_query_groups(cuda_device, policy, attn):
+    # G = 2: clusters of two CTAs (one per query) for the selection
+    alpha = 1.5 if attn == ekv.EKV_ENTMAX15 else 2.0
+    wl = make_random(B=3, H_kv=2, G=2, d=128, P=16, lens=(2500, 600, 17), dtype=torch.bfloat16,
+                     device="cuda", seed=31, kv_scale=1.0, q_scale=0.6, policy=policy,
+                     alpha=alpha, delta=0.1)
+    cache, dec = run_gpu(wl, attn)
+    assert_status_ok(cache)
+    for b in range(wl.batch):
+        for h in range(wl.num_kv_heads):
+            check_head(wl, cache, dec, b, h, attn)
+
+
+def test_gauss_long_sequence_beyond_the_staged_slices(cuda_device):
+    # 20000 pages: a warp's slice exceeds its shared-memory capacity, so the model is read from
+    # global memory for the maximum and, where the survivors overflow, on every Newton step
+    wl = make_random(B=1, H_kv=1, G=4, d=64, P=16, lens=(20000 * 16 - 9,), dtype=torch.bfloat16,
+                     device="cuda", seed=32, kv_scale=0.2, q_scale=0.3, policy=GAUSS_MAX,
+                     alpha=1.5, delta=0.1)
+    cache, dec = run_gpu(wl, ekv.EKV_ENTMAX15)
+    assert_status_ok(cache)
+    check_head(wl, cache, dec, 0, 0, ekv.EKV_ENTMAX15)
+
+
 def test_multi_chunk_pages(cuda_device):
     # enough selected pages that each (sequence, head) spans several multi-page chunks
     wl = make_random(B=4, H_kv=8, G=4, d=128, P=16, lens=(8000, 8000 - 3, 4100, 8000),
