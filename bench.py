@@ -67,6 +67,9 @@ def parse():
     ap.add_argument("--split-select", action="store_true",
                     help="top-k: ekv_select_pages and ekv_sparse_decode as two calls (timed "
                          "apart) instead of the one ekv_select_decode call")
+    ap.add_argument("--split-refresh", action="store_true",
+                    help="appending workloads: ekv_page_meta_update and ekv_score_pages as two "
+                         "calls instead of the one ekv_refresh_score_pages call")
     ap.add_argument("--policy", default=None, choices=["topk", "gauss", "gauss_max"],
                     help="selection policy (default: the workload's); gauss_max is the estimated-"
                          "maximum reading of the Gaussian rule")
@@ -151,6 +154,7 @@ def step_bytes(wl, dec, attn, variant, extra):
         append_b = wl.batch * H * wl.append[1] * d * esz + wl.batch * H * meta_row
     sel_out = dec.sel_idx.numel() * 4
     by = {"score": meta + ptab + qb + scores_out, "select": scores_out + sel_out,
+          "refresh_score": meta + ptab + qb + scores_out + append_b,
           "score_select": meta + ptab + qb + scores_out + sel_out,
           "selected_tokens": sel_tok, "meta_bytes": meta}
     if variant == "pages":
@@ -389,7 +393,7 @@ class Step:
     they write. Every call goes through the C ABI binding; nothing here computes."""
 
     def __init__(self, ekv, SparseDecoder, cache, wl, attn, variant, T, fused_select=False,
-                 split_select=False):
+                 split_select=False, split_refresh=False):
         self.wl, self.variant, self.T = wl, variant, T
         dev = wl.k_cache.device
         B, H = wl.batch, wl.num_kv_heads
@@ -397,17 +401,25 @@ class Step:
                                        alpha=wl.alpha, delta=wl.delta, scale=wl.scale)
         self.extra = {}
         calls = []
-        if wl.append is not None:
-            ap_start = torch.full((B,), wl.append[0], dtype=torch.int32, device=dev)
-            ap_count = torch.full((B,), wl.append[1], dtype=torch.int32, device=dev)
-            calls.append(("meta", lambda: ekv.ekv_page_meta_update(cache, ap_start, ap_count,
-                                                                   wl.append[1])))
         q = wl.q
         # top-k pages: the selection and the attention in one call
         joint = wl.policy == 0 and variant == "pages" and not fused_select and not split_select
+        refresh = wl.append is not None and joint and not split_refresh
+        if wl.append is not None:
+            ap_start = torch.full((B,), wl.append[0], dtype=torch.int32, device=dev)
+            ap_count = torch.full((B,), wl.append[1], dtype=torch.int32, device=dev)
+            if refresh:
+                # the appended page's metadata rebuilt inside the scan (one call)
+                calls.append(("refresh_score", lambda: ekv.ekv_refresh_score_pages(
+                    cache, ap_start, ap_count, wl.append[1], q, wl.num_q_heads, wl.scale,
+                    wl.policy, dec.scores)))
+            else:
+                calls.append(("meta", lambda: ekv.ekv_page_meta_update(cache, ap_start, ap_count,
+                                                                       wl.append[1])))
         if joint:
-            calls.append(("score", lambda: ekv.ekv_score_pages(cache, q, wl.num_q_heads, wl.scale,
-                                                               wl.policy, dec.scores)))
+            if not refresh:
+                calls.append(("score", lambda: ekv.ekv_score_pages(
+                    cache, q, wl.num_q_heads, wl.scale, wl.policy, dec.scores)))
         elif wl.policy == 0 and fused_select:
             # top-k scores and selection in one launch (one cluster per sequence and KV head)
             calls.append(("score_select", lambda: ekv.ekv_score_select_pages(
@@ -424,7 +436,7 @@ class Step:
             calls.append(("select_decode", lambda: ekv.ekv_select_decode(
                 cache, q, wl.num_q_heads, wl.scale, attn, wl.topk, dec.scores, dec.sel_idx,
                 dec.sel_count, dec.max_sel, dec.out, dec.stat, dec.ws)))
-            self.kernels = {"meta": 1, "score": 1, "select_decode": 1}
+            self.kernels = {"meta": 1, "refresh_score": 1, "score": 1, "select_decode": 1}
         elif variant == "pages":
             calls.append(("decode", lambda: ekv.ekv_sparse_decode(
                 cache, q, wl.num_q_heads, wl.scale, attn, dec.sel_idx, dec.sel_count,
@@ -601,7 +613,7 @@ def main():
     ekv.ekv_page_meta_update(cache, torch.zeros(B, dtype=torch.int32, device=dev), wl.seq_lens,
                              int(wl.seq_lens.max()))
     step = Step(ekv, SparseDecoder, cache, wl, attn, args.variant, T, args.fused_select,
-                args.split_select)
+                args.split_select, args.split_refresh)
     dec = step.dec
     stream = torch.cuda.current_stream()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)

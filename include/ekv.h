@@ -131,6 +131,22 @@ ekv_status ekv_score_pages(const ekv_cache *c, const void *q, int32_t num_q_head
                            int32_t policy, float *scores, void *stream);
 
 /*
+ * §2.A both steps of a decode step's start in one call: ekv_page_meta_update(c, new_start,
+ * new_count, max_new) followed by ekv_score_pages(c, q, num_q_heads, scale, policy, scores), with
+ * the results of the two calls bit for bit (metadata, scores, device status bits). Under
+ * EKV_SEL_TOPK with max_new <= 2 P and few (sequence, KV head) pairs (2 * batch * H_kv at most a
+ * sixteenth of the scan's persistent grid), one kernel does both: leading blocks rebuild the
+ * appended pages' metadata and score the 8-page groups holding them while the rest of the grid
+ * scans every other group. Otherwise the two kernels run in turn. max_new = 0 is
+ * ekv_score_pages alone.
+ * Arguments, layouts, alignment and errors: those of the two calls.
+ */
+ekv_status ekv_refresh_score_pages(const ekv_cache *c, const int32_t *new_start,
+                                   const int32_t *new_count, int32_t max_new, const void *q,
+                                   int32_t num_q_heads, float scale, int32_t policy,
+                                   float *scores, void *stream);
+
+/*
  * §2.B candidate selection, per (sequence, KV head).
  *   EKV_SEL_TOPK (§2.B.1): the min(topk, n_pages) pages with the largest S_j; equal scores go
  *     to the lower page index. alpha, delta, tau_hat are ignored (tau_hat may be NULL).

@@ -15,6 +15,10 @@ cudaError_t launch_page_meta_update(const ekv_cache &c, const int32_t *new_start
                                     const int32_t *new_count, int max_new, cudaStream_t st);
 cudaError_t launch_score_pages(const ekv_cache &c, const void *q, int H_q, float scale,
                                int policy, float *scores, cudaStream_t st, bool pdl);
+cudaError_t launch_refresh_score_pages(const ekv_cache &c, const int32_t *new_start,
+                                       const int32_t *new_count, int max_new, const void *q,
+                                       int H_q, float scale, int policy, float *scores,
+                                       cudaStream_t st, bool pdl);
 cudaError_t launch_select_pages(const ekv_cache &c, int H_q, int policy, int topk, float alpha,
                                 float delta, const float *scores, int32_t *sel_idx,
                                 int32_t *sel_count, int max_sel, float *tau_hat, cudaStream_t st,
@@ -144,6 +148,31 @@ ekv_status ekv_score_pages(const ekv_cache *c, const void *q, int32_t num_q_head
     if (gauss && ((uintptr_t)c->meta_mom & 15u)) return EKV_ERR_INVALID_ARG;
     return cuda_status(launch_score_pages(*c, q, num_q_heads, scale, policy, scores,
                                           static_cast<cudaStream_t>(stream), use_pdl()));
+}
+
+ekv_status ekv_refresh_score_pages(const ekv_cache *c, const int32_t *new_start,
+                                   const int32_t *new_count, int32_t max_new, const void *q,
+                                   int32_t num_q_heads, float scale, int32_t policy,
+                                   float *scores, void *stream)
+{
+    ekv_status s = check_cache(c, false);
+    if (s != EKV_OK) return s;
+    if ((s = check_heads(c, num_q_heads)) != EKV_OK) return s;
+    // ekv_page_meta_update's checks
+    if (!new_start || !new_count || max_new < 0) return EKV_ERR_INVALID_ARG;
+    if ((uintptr_t)c->k_cache & 15u) return EKV_ERR_INVALID_ARG;
+    if ((long long)max_new > (long long)c->max_pages * c->page_size) return EKV_ERR_INVALID_ARG;
+    // ekv_score_pages' checks
+    if (!q || !scores || !(scale > 0.0f) || !std::isfinite(scale)) return EKV_ERR_INVALID_ARG;
+    if (policy != EKV_SEL_TOPK && policy != EKV_SEL_GAUSS && policy != EKV_SEL_GAUSS_MAX)
+        return EKV_ERR_UNSUPPORTED;
+    const bool gauss = policy != EKV_SEL_TOPK;
+    if (gauss && !c->meta_mom) return EKV_ERR_INVALID_ARG;
+    if ((uintptr_t)c->meta_bbox & 15u) return EKV_ERR_INVALID_ARG;
+    if (gauss && ((uintptr_t)c->meta_mom & 15u)) return EKV_ERR_INVALID_ARG;
+    return cuda_status(launch_refresh_score_pages(*c, new_start, new_count, max_new, q,
+                                                  num_q_heads, scale, policy, scores,
+                                                  static_cast<cudaStream_t>(stream), use_pdl()));
 }
 
 ekv_status ekv_select_pages(const ekv_cache *c, int32_t num_q_heads, int32_t policy,

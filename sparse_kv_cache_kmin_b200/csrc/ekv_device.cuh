@@ -21,6 +21,16 @@ __device__ __forceinline__ uint4 ld_stream16(const void *p)
         : "l"(p));
     return r;
 }
+// 16 bytes through L2 only: for data the same kernel wrote (ordered by a barrier before it)
+__device__ __forceinline__ uint4 ld_cg16(const void *p)
+{
+    uint4 r;
+    asm volatile("ld.global.cg.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p)
+                 : "memory");
+    return r;
+}
 
 // A 16-byte chunk of stored elements, widened to fp32. bf16 is the upper half of an IEEE
 // float32, so widening is a shift; the element at the lower address is the low half.

@@ -9,6 +9,7 @@
 // (two-pass variance; the rows are still in L1/L2). kmin/kmax are stored in the cache dtype
 // (exact: they are stored values); mean and population variance in fp32.
 #include "ekv_device.cuh"
+#include "meta_refresh.cuh"
 
 namespace ekv {
 
@@ -106,107 +107,26 @@ page_meta_update_kernel(ekv_cache c, const int32_t *__restrict__ new_start,
 }
 
 // The same statistics for a short append (a page or two per sequence per step): one CTA per
-// (touched page, KV head), so the page's rows are read once, all at the same time. Warp w takes
-// rows w, w + 8, ... (at most 8 each for P <= 64) with every load in flight, keeps them in
-// registers for the variance pass, and the eight warps' partial min / max / sums are combined
-// in shared memory.
+// (touched page, KV head), so the page's rows are read once, all at the same time
+// (meta_refresh_page).
 template <int DT, int D>
 __global__ void __launch_bounds__(256)
 page_meta_wide_kernel(ekv_cache c, const int32_t *__restrict__ new_start,
                       const int32_t *__restrict__ new_count, int max_new)
 {
-    constexpr int VEC = D / 32;
-    constexpr int RPW = 8;  // rows per warp: P <= 64 = 8 warps x 8 rows
-    __shared__ float s_a[8][D], s_b[8][D], s_c[8][D];
-    __shared__ float s_mean[D];
+    __shared__ MetaPageShared<D> sm;
     pdl_wait();
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int h = blockIdx.z, b = blockIdx.y;
     const int P = c.page_size;
     int len;
     seq_pages(c.seq_lens, b, P, c.max_pages, c.dev_status, &len);
-    int s = new_start[b], n = new_count[b];
-    if (n <= 0) return;
-    if (s < 0 || s + n > len || n > max_new) {
-        if (blockIdx.x == 0 && h == 0 && threadIdx.x == 0) flag(c.dev_status, EKV_DEV_BAD_RANGE);
-        s = s < 0 ? 0 : (s > len ? len : s);
-        int e = s + n > len ? len : s + n;
-        n = e - s > max_new ? max_new : e - s;
-        if (n <= 0) return;
-    }
+    int s, n;
+    if (!append_range(c, new_start, new_count, max_new, b, len,
+                      blockIdx.x == 0 && h == 0 && threadIdx.x == 0, s, n))
+        return;
     const int p = s / P + blockIdx.x;
     if (p > (s + n - 1) / P) return;
-    const int blk = c.page_table[(size_t)b * c.max_pages + p];
-    if (blk < 0 || blk >= c.num_blocks) {
-        if (threadIdx.x == 0) flag(c.dev_status, EKV_DEV_BAD_BLOCK);
-        return;
-    }
-    const int cnt = len - p * P < P ? len - p * P : P;
-    const size_t row0 = ((size_t)blk * c.num_kv_heads + h) * P;
-    const char *krow = static_cast<const char *>(c.k_cache) +
-                       (row0 * D + lane * VEC) * (size_t)Chunk<DT>::kBytes;
-    constexpr size_t ROWB = (size_t)D * Chunk<DT>::kBytes;
-    float x[RPW][VEC];
-#pragma unroll
-    for (int u = 0; u < RPW; ++u)
-        if (warp + 8 * u < cnt) load_vec_nc<DT, VEC>(krow + (warp + 8 * u) * ROWB, x[u]);
-    float mn[VEC], mx[VEC], sum[VEC];
-#pragma unroll
-    for (int e = 0; e < VEC; ++e) { mn[e] = INFINITY; mx[e] = -INFINITY; sum[e] = 0.f; }
-#pragma unroll
-    for (int u = 0; u < RPW; ++u) {
-        if (warp + 8 * u >= cnt) break;
-#pragma unroll
-        for (int e = 0; e < VEC; ++e) {
-            mn[e] = fminf(mn[e], x[u][e]);
-            mx[e] = fmaxf(mx[e], x[u][e]);
-            sum[e] += x[u][e];
-        }
-    }
-#pragma unroll
-    for (int e = 0; e < VEC; ++e) {
-        s_a[warp][lane * VEC + e] = mn[e];
-        s_b[warp][lane * VEC + e] = mx[e];
-        s_c[warp][lane * VEC + e] = sum[e];
-    }
-    __syncthreads();
-    const size_t mbase = ((size_t)blk * c.num_kv_heads + h) * 2 * D;
-    for (int i = threadIdx.x; i < D; i += 256) {
-        float lo = s_a[0][i], hi = s_b[0][i], sm = s_c[0][i];
-#pragma unroll
-        for (int w = 1; w < 8; ++w) {
-            lo = fminf(lo, s_a[w][i]);
-            hi = fmaxf(hi, s_b[w][i]);
-            sm += s_c[w][i];
-        }
-        store_exact<DT>(c.meta_bbox, mbase + i, lo);
-        store_exact<DT>(c.meta_bbox, mbase + D + i, hi);
-        s_mean[i] = sm / (float)cnt;
-    }
-    if (!c.meta_mom) return;
-    __syncthreads();
-    float ss[VEC];
-#pragma unroll
-    for (int e = 0; e < VEC; ++e) ss[e] = 0.f;
-#pragma unroll
-    for (int u = 0; u < RPW; ++u) {
-        if (warp + 8 * u >= cnt) break;
-#pragma unroll
-        for (int e = 0; e < VEC; ++e) {
-            const float dv = x[u][e] - s_mean[lane * VEC + e];
-            ss[e] = fmaf(dv, dv, ss[e]);
-        }
-    }
-#pragma unroll
-    for (int e = 0; e < VEC; ++e) s_a[warp][lane * VEC + e] = ss[e];
-    __syncthreads();
-    for (int i = threadIdx.x; i < D; i += 256) {
-        float v = 0.f;
-#pragma unroll
-        for (int w = 0; w < 8; ++w) v += s_a[w][i];
-        c.meta_mom[mbase + i] = s_mean[i];
-        c.meta_mom[mbase + D + i] = v / (float)cnt;
-    }
+    meta_refresh_page<DT, D>(c, b, h, p, len, sm);
 }
 
 cudaError_t launch_page_meta_update(const ekv_cache &c, const int32_t *new_start,

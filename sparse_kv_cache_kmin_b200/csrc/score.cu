@@ -18,6 +18,7 @@
 // Gaussian policy: per query, UB_gj (as above but unsummed), m_gj = scale * q_g . mean_j and
 // v_gj = scale^2 * sum_c q_gc^2 var_jc; each page reads its bbox row and its fp32 moment row.
 #include "ekv_device.cuh"
+#include "meta_refresh.cuh"
 
 namespace ekv {
 
@@ -56,12 +57,19 @@ __device__ __forceinline__ int find_seq(const int *pre, int B, long gi)
     return lo;
 }
 
-template <int DT, int D, int G>
-__global__ void __launch_bounds__(256)
-score_topk_kernel(ekv_cache c, const void *__restrict__ q, int H_q, float scale,
-                  float *__restrict__ scores)
+// The appended token ranges whose pages a refreshing scan rebuilds first (the arguments of
+// ekv_page_meta_update); nr leading blocks do that, two per (sequence, KV head).
+struct RefreshArgs {
+    const int32_t *new_start, *new_count;
+    int max_new, nr;
+};
+
+template <int DT, int D, int G, bool REFRESH>
+__device__ __forceinline__ void score_topk_body(const ekv_cache &c, const void *__restrict__ q,
+                                                int H_q, float scale, float *__restrict__ scores,
+                                                const RefreshArgs &ra)
 {
-    extern __shared__ int pre[];  // [B + 1]
+    extern __shared__ int pre[];  // [B + 1], then (refresh) the touched groups [B][2]
     __shared__ int warp_tot[8];
     constexpr int EPC = Chunk<DT>::N;
     constexpr int CPR = 2 * D * Chunk<DT>::kBytes / 16;  // 16-byte chunks per bbox row
@@ -75,9 +83,51 @@ score_topk_kernel(ekv_cache c, const void *__restrict__ q, int H_q, float scale,
     pdl_wait();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int H = c.num_kv_heads, B = c.batch, P = c.page_size;
+    // Refresh: the groups holding the appended pages of sequence b are tg[2b]..tg[2b + 1]
+    // (-1: none). Blocks [0, nr) rebuild those pages' metadata and score their groups (block r:
+    // sequence and head r / 2, the first or the last touched group); the other blocks scan the
+    // rest and skip them.
+    int *tg = pre + B + 1;
+    bool fresh = false;
+    if constexpr (REFRESH) {
+        for (int b = threadIdx.x; b < B; b += blockDim.x) {
+            int len, s, n;
+            seq_pages(c.seq_lens, b, P, c.max_pages, nullptr, &len);
+            const bool any = append_range(c, ra.new_start, ra.new_count, ra.max_new, b, len,
+                                          false, s, n);
+            tg[2 * b] = any ? s / P / PG : -1;
+            tg[2 * b + 1] = any ? (s + n - 1) / P / PG : -1;
+        }
+        fresh = (int)blockIdx.x < ra.nr;
+    }
     const long TG = build_group_prefix<PG>(c, pre, warp_tot);
-    const long lo = (long)blockIdx.x * TG / gridDim.x;
-    const long hi = (long)(blockIdx.x + 1) * TG / gridDim.x;
+    long lo, hi;
+    if constexpr (REFRESH) {
+        if (fresh) {
+            __shared__ MetaPageShared<D> msm;
+            const int bh = blockIdx.x >> 1, b = bh / H, h = bh % H;
+            int len, s, n;
+            const int np = seq_pages(c.seq_lens, b, P, c.max_pages, nullptr, &len);
+            // a bad range is reported once per sequence, by its head-0 first-group block
+            if (!append_range(c, ra.new_start, ra.new_count, ra.max_new, b, len,
+                              (blockIdx.x & 1) == 0 && h == 0 && threadIdx.x == 0, s, n))
+                return;
+            const int g = tg[2 * b + (blockIdx.x & 1)];
+            if ((blockIdx.x & 1) && g == tg[2 * b]) return;  // one touched group
+            const int p0 = max(s / P, g * PG), p1 = min((s + n - 1) / P, g * PG + PG - 1);
+            for (int p = p0; p <= p1; ++p) meta_refresh_page<DT, D>(c, b, h, p, len, msm);
+            // the block's metadata stores are visible to its own threads from here on; warp 0
+            // scores the group (bbox rows read coherently, not through the read-only path)
+            lo = pre[b] + (long)h * ((np + PG - 1) / PG) + g;
+            hi = lo + 1;
+        } else {
+            lo = (long)(blockIdx.x - ra.nr) * TG / (gridDim.x - ra.nr);
+            hi = (long)(blockIdx.x - ra.nr + 1) * TG / (gridDim.x - ra.nr);
+        }
+    } else {
+        lo = (long)blockIdx.x * TG / gridDim.x;
+        hi = (long)(blockIdx.x + 1) * TG / gridDim.x;
+    }
     const char *bbox = static_cast<const char *>(c.meta_bbox);
 
     // Work group gi -> (sequence, KV head, first page); its page-table entries are fetched
@@ -122,16 +172,29 @@ score_topk_kernel(ekv_cache c, const void *__restrict__ q, int H_q, float scale,
         const Grp cur = nxt;
         const int myblk = nxt_blk;
         const int bh = cur.bb * H + cur.hh;
+        if constexpr (REFRESH) {
+            const int gg = cur.j0 / PG;  // a group a refresh block scores: not ours
+            if (!fresh && gg >= tg[2 * cur.bb] && gg <= tg[2 * cur.bb + 1]) {
+                if (gi + 8 < hi) {
+                    nxt = locate(gi + 8);
+                    nxt_blk = fetch_blk(nxt);
+                }
+                continue;
+            }
+        }
         uint4 x[NPL][LPL];
 #pragma unroll
         for (int i = 0; i < NPL; ++i) {
             const int blk = __shfl_sync(kFull, myblk, i * RPI + lane / W);
 #pragma unroll
             for (int k = 0; k < LPL; ++k) {
-                if (blk >= 0)
-                    x[i][k] = ld_stream16(bbox + (((size_t)blk * H + cur.hh) * CPR + k * W + lane % W) * 16);
-                else
+                const char *src = bbox + (((size_t)blk * H + cur.hh) * CPR + k * W + lane % W) * 16;
+                if (blk < 0)
                     x[i][k] = make_uint4(0, 0, 0, 0);
+                else if (REFRESH && fresh)
+                    x[i][k] = ld_cg16(src);
+                else
+                    x[i][k] = ld_stream16(src);
             }
         }
         if (gi + 8 < hi) {
@@ -175,6 +238,27 @@ score_topk_kernel(ekv_cache c, const void *__restrict__ q, int H_q, float scale,
         if (((lane % W) % (W / NPL)) == 0 && cur.j0 + po < cur.np)
             scores[(size_t)bh * c.max_pages + cur.j0 + po] = blk >= 0 ? scale * part[0] : -INFINITY;
     }
+}
+
+template <int DT, int D, int G>
+__global__ void __launch_bounds__(256)
+score_topk_kernel(ekv_cache c, const void *__restrict__ q, int H_q, float scale,
+                  float *__restrict__ scores)
+{
+    score_topk_body<DT, D, G, false>(c, q, H_q, scale, scores, RefreshArgs{});
+}
+
+// ekv_page_meta_update of a short append followed by the top-k scan, in one launch: blocks
+// [0, ra.nr) rebuild the appended pages' metadata (meta_refresh_page, as the short-append
+// kernel does) and score the 8-page groups holding them; the other blocks scan every other
+// group. The results are those of the two calls, bit for bit; the refresh runs under the scan
+// instead of before it.
+template <int DT, int D, int G>
+__global__ void __launch_bounds__(256, DT == EKV_BF16 ? 4 : 1)
+score_refresh_topk_kernel(ekv_cache c, const void *__restrict__ q, int H_q, float scale,
+                          float *__restrict__ scores, RefreshArgs ra)
+{
+    score_topk_body<DT, D, G, true>(c, q, H_q, scale, scores, ra);
 }
 
 template <int DT, int D, int G>
@@ -316,6 +400,75 @@ cudaError_t launch_score_pages(const ekv_cache &c, const void *q, int H_q, float
                                  : launch_score_g<EKV_BF16, 64>(c, q, H_q, scale, policy, scores, st, pdl);
     return c.head_dim == 128 ? launch_score_g<EKV_F32, 128>(c, q, H_q, scale, policy, scores, st, pdl)
                              : launch_score_g<EKV_F32, 64>(c, q, H_q, scale, policy, scores, st, pdl);
+}
+
+
+template <int DT, int D, int G>
+static cudaError_t launch_refresh_t(const ekv_cache &c, const void *q, int H_q, float scale,
+                                    float *scores, RefreshArgs ra, cudaStream_t st, bool pdl,
+                                    bool *launched)
+{
+    auto k = score_refresh_topk_kernel<DT, D, G>;
+    const size_t smem = sizeof(int) * (3 * (size_t)c.batch + 1);
+    const int grid = persistent_grid_size((const void *)k, 256, smem);
+    // The refresh blocks come out of the scan's single wave: only when they are few (at most a
+    // sixteenth of the grid) is the scan they slow down cheaper than a launch of its own.
+    ra.nr = 2 * c.batch * c.num_kv_heads;
+    *launched = (long long)ra.nr * 16 <= grid;
+    if (!*launched) return cudaSuccess;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    cfg.gridDim = dim3(grid);
+    return cudaLaunchKernelEx(&cfg, k, c, q, H_q, scale, scores, ra);
+}
+
+template <int DT, int D>
+static cudaError_t launch_refresh_g(const ekv_cache &c, const void *q, int H_q, float scale,
+                                    float *scores, RefreshArgs ra, cudaStream_t st, bool pdl,
+                                    bool *launched)
+{
+    switch (H_q / c.num_kv_heads) {
+    case 1: return launch_refresh_t<DT, D, 1>(c, q, H_q, scale, scores, ra, st, pdl, launched);
+    case 2: return launch_refresh_t<DT, D, 2>(c, q, H_q, scale, scores, ra, st, pdl, launched);
+    case 4: return launch_refresh_t<DT, D, 4>(c, q, H_q, scale, scores, ra, st, pdl, launched);
+    default: return launch_refresh_t<DT, D, 8>(c, q, H_q, scale, scores, ra, st, pdl, launched);
+    }
+}
+
+cudaError_t launch_page_meta_update(const ekv_cache &c, const int32_t *new_start,
+                                    const int32_t *new_count, int max_new, cudaStream_t st);
+
+// ekv_page_meta_update then ekv_score_pages. A short append (at most 2 P tokens per sequence)
+// under the top-k policy with few (sequence, KV head) pairs runs as one refreshing scan;
+// otherwise the two kernels run one after the other.
+cudaError_t launch_refresh_score_pages(const ekv_cache &c, const int32_t *new_start,
+                                       const int32_t *new_count, int max_new, const void *q,
+                                       int H_q, float scale, int policy, float *scores,
+                                       cudaStream_t st, bool pdl)
+{
+    if (max_new == 0) return launch_score_pages(c, q, H_q, scale, policy, scores, st, pdl);
+    if (policy == EKV_SEL_TOPK && max_new <= 2 * c.page_size) {
+        const RefreshArgs ra = {new_start, new_count, max_new, 0};
+        bool launched = false;
+        cudaError_t e;
+        if (c.dtype == EKV_BF16)
+            e = c.head_dim == 128 ? launch_refresh_g<EKV_BF16, 128>(c, q, H_q, scale, scores, ra, st, pdl, &launched)
+                                  : launch_refresh_g<EKV_BF16, 64>(c, q, H_q, scale, scores, ra, st, pdl, &launched);
+        else
+            e = c.head_dim == 128 ? launch_refresh_g<EKV_F32, 128>(c, q, H_q, scale, scores, ra, st, pdl, &launched)
+                                  : launch_refresh_g<EKV_F32, 64>(c, q, H_q, scale, scores, ra, st, pdl, &launched);
+        if (e != cudaSuccess || launched) return e;
+    }
+    cudaError_t e = launch_page_meta_update(c, new_start, new_count, max_new, st);
+    if (e != cudaSuccess) return e;
+    return launch_score_pages(c, q, H_q, scale, policy, scores, st, pdl);
 }
 
 }  // namespace ekv

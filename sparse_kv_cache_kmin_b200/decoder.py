@@ -71,9 +71,17 @@ class SparseDecoder:
             stat_host.copy_(self.stat, non_blocking=True)
         return g
 
-    def step(self, q: torch.Tensor, stream=None):
+    def step(self, q: torch.Tensor, stream=None, append=None):
+        """One decode step. `append` = (new_start, new_count, max_new), the arguments of
+        ekv_page_meta_update, refreshes the appended pages' metadata first (in the scoring call)."""
         c = self.cache
-        ekv.ekv_score_pages(c, q, self.num_q_heads, self.scale, self.policy, self.scores, stream)
+        if append is not None:
+            new_start, new_count, max_new = append
+            ekv.ekv_refresh_score_pages(c, new_start, new_count, max_new, q, self.num_q_heads,
+                                        self.scale, self.policy, self.scores, stream)
+        else:
+            ekv.ekv_score_pages(c, q, self.num_q_heads, self.scale, self.policy, self.scores,
+                                stream)
         if self.policy == ekv.EKV_SEL_TOPK:
             # selection and attention in one call (the decode launched behind the selection)
             ekv.ekv_select_decode(c, q, self.num_q_heads, self.scale, self.attn, self.topk,

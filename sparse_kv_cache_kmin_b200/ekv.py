@@ -218,6 +218,20 @@ def ekv_score_pages(cache: PagedKVCache, q: torch.Tensor, num_q_heads: int, scal
                                           _stream(stream)), "ekv_score_pages")
 
 
+def ekv_refresh_score_pages(cache: PagedKVCache, new_start: torch.Tensor, new_count: torch.Tensor,
+                            max_new: int, q: torch.Tensor, num_q_heads: int, scale: float,
+                            policy: int, scores: torch.Tensor, stream=None):
+    """ekv_page_meta_update followed by ekv_score_pages, in one call (one kernel for a short
+    top-k append over few (sequence, KV head) pairs), with the two calls' results bit for bit."""
+    P, I32, F = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float
+    fn = _moment_fn("ekv_refresh_score_pages", [ctypes.POINTER(EkvCacheStruct), P, P, I32, P, I32,
+                                                F, I32, P, P])
+    c = cache.struct()
+    _check(fn(ctypes.byref(c), _ptr(new_start), _ptr(new_count), int(max_new), _ptr(q),
+              int(num_q_heads), float(scale), int(policy), _ptr(scores), _stream(stream)),
+           "ekv_refresh_score_pages")
+
+
 def ekv_select_pages(cache: PagedKVCache, num_q_heads: int, policy: int, topk: int, alpha: float,
                      delta: float, scores: torch.Tensor, sel_idx: torch.Tensor,
                      sel_count: torch.Tensor, max_sel: int, tau_hat: Optional[torch.Tensor],

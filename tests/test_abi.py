@@ -278,3 +278,35 @@ def test_wait_selftest_validation(lib):
     assert lib.ekv_wait_selftest(C.byref(c), 2_000_000_001, None) == 1   # above the 2 s limit
     c2 = fake_cache(dev_status=None)
     assert lib.ekv_wait_selftest(C.byref(c2), 1000, None) == 1
+
+
+def test_refresh_score_validation(lib):
+    # the one-call metadata refresh + scores refuses what either of its halves refuses, on the
+    # host; every call below fails validation, so nothing is launched
+    import ctypes as C
+    cp = C.POINTER(type(fake_cache()))
+    vp, i32, f32 = C.c_void_p, C.c_int32, C.c_float
+    fn = lib.ekv_refresh_score_pages
+    fn.argtypes = [cp, vp, vp, i32, vp, i32, f32, i32, vp, vp]
+    P = 0x1000
+
+    def call(start=P, count=P, max_new=16, q=P, hq=32, scale=1.0, policy=0, scores=P, cache=None):
+        c = fake_cache() if cache is None else cache
+        return fn(C.byref(c), start, count, max_new, q, hq, scale, policy, scores, None)
+
+    assert call(start=None) == 1
+    assert call(count=None) == 1
+    assert call(max_new=-1) == 1
+    assert call(max_new=256 * 16 + 1) == 1        # longer than a whole sequence
+    assert call(cache=fake_cache(k_cache=P + 4)) == 1
+    assert call(q=None) == 1
+    assert call(scores=None) == 1
+    assert call(scale=0.0) == 1
+    assert call(scale=float("inf")) == 1
+    assert call(hq=31) == 1                       # not a multiple of H_kv
+    assert call(hq=8 * 16) == 2                   # G = 16
+    assert call(policy=7) == 2
+    assert call(policy=1, cache=fake_cache(meta_mom=None)) == 1
+    assert call(cache=fake_cache(meta_bbox=P + 8)) == 1
+    assert call(policy=2, cache=fake_cache(meta_mom=P + 4)) == 1
+    assert call(cache=fake_cache(dtype=5)) == 2
