@@ -58,6 +58,14 @@ decode_logits_direct_kernel(DecodeArgs a)
     const long long nw = (long long)gridDim.x * kDirWarps;
     const long long ck0 = (long long)blockIdx.x * kDirWarps + warp;
 
+    // The page-table rows do not depend on the selection: CTAs placed while the selection still
+    // runs bring them into L2 before waiting for it, so the resolution below hits L2.
+    {
+        const size_t lines = ((size_t)c.batch * c.max_pages * sizeof(int32_t) + 127) / 128;
+        for (size_t l = (size_t)blockIdx.x * blockDim.x + threadIdx.x; l < lines;
+             l += (size_t)gridDim.x * blockDim.x)
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<const char *>(c.page_table) + l * 128));
+    }
     pdl_wait();
     // Lane l of a batch: chunk l / CP of the batch, page l % CP of that chunk. bh < 0 past the
     // last slot; nt = valid tokens of the page (0: no page); ok: the chunk holds a selected page.

@@ -121,3 +121,14 @@ def test_select_decode_needle_workload_sampled_heads(cuda_device):
     wl = make("needle128k", device="cuda")
     cache, dec = select_decode_step(wl, ekv.EKV_ENTMAX15)
     check_all(wl, cache, dec, ekv.EKV_ENTMAX15, heads=[(0, 0), (3, 5), (7, 7)])
+
+
+def test_select_decode_many_pairs(cuda_device):
+    # 72 x 8 (sequence, KV head) pairs, two chunk slots each: one selection CTA per pair and
+    # about a quarter of the logits kernel's warps busy
+    B = 72
+    lens = tuple(16 * (30 + i % 7) + i % 5 for i in range(B))
+    wl = make_random(B=B, H_kv=8, G=4, d=128, P=16, lens=lens, dtype=torch.bfloat16,
+                     device="cuda", seed=97, topk=16)
+    cache, dec = select_decode_step(wl, ekv.EKV_ENTMAX15)
+    check_all(wl, cache, dec, ekv.EKV_ENTMAX15, heads=[(0, 0), (B - 1, 7), (35, 3), (50, 6)])
