@@ -130,6 +130,7 @@ moment_retained_kernel(ekv_cache c, const void *__restrict__ q, int H_q,
     __shared__ int s_cnt[8];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int half = lane >> 4, hl = lane & 15;
+    const unsigned hmask = 0xffffu << (16 * half);  // this half-warp's lanes
     const int bh = blockIdx.y, b = bh / c.num_kv_heads, h = bh % c.num_kv_heads;
     const int P = c.page_size;
     int ns = sel_count[bh];
@@ -203,7 +204,7 @@ moment_retained_kernel(ekv_cache c, const void *__restrict__ q, int H_q,
 #pragma unroll
                 for (int e = 0; e < EPC; ++e) acc = fmaf(qv[g][k][e], kf[k][e], acc);
 #pragma unroll
-            for (int o = 1; o < 16; o <<= 1) acc += __shfl_xor_sync(kFull, acc, o);
+            for (int o = 1; o < 16; o <<= 1) acc += __shfl_xor_sync(hmask, acc, o);
             dot[g] = acc;
         }
 #pragma unroll

@@ -30,6 +30,7 @@ token_score_kernel(ekv_cache c, const void *__restrict__ q, int H_q, float scale
     constexpr int RIF = 4;  // rows in flight per half-warp
     __shared__ int s_blk[PPC], s_nt[PPC];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, half = lane >> 4, hl = lane & 15;
+    const unsigned hmask = 0xffffu << (16 * half);  // this half-warp's lanes
     const int bh = blockIdx.y, b = bh / c.num_kv_heads, h = bh % c.num_kv_heads;
     const int H = c.num_kv_heads, P = c.page_size;
     pdl_wait();
@@ -103,7 +104,7 @@ token_score_kernel(ekv_cache c, const void *__restrict__ q, int H_q, float scale
 #pragma unroll
                 for (int e = 0; e < EPC; ++e) acc = fmaf(qv[k][e], kf[r][k][e], acc);
 #pragma unroll
-            for (int o = 1; o < 16; o <<= 1) acc += __shfl_xor_sync(kFull, acc, o);
+            for (int o = 1; o < 16; o <<= 1) acc += __shfl_xor_sync(hmask, acc, o);
             if (hl == 0 && base + r < nrows) out[base + r] = ok[r] ? scale * acc : -INFINITY;
         }
     }
@@ -174,6 +175,9 @@ token_attend_kernel(ekv_cache c, const void *__restrict__ q, int H_q, float scal
     __syncthreads();
     auto row_at = [&](int i) { return rows_smem ? rows[i] : row_of(i); };
     const int half = lane >> 4, hl = lane & 15;
+    // the two halves of a warp may take different trip counts through the row loops: their
+    // reductions synchronise only their own 16 lanes
+    const unsigned hmask = 0xffffu << (16 * half);
     auto owns = [&](int k) { return hl + 16 * k < W; };
     float qv[PPL][EPC];
 #pragma unroll
@@ -206,7 +210,7 @@ token_attend_kernel(ekv_cache c, const void *__restrict__ q, int H_q, float scal
 #pragma unroll
                 for (int e = 0; e < EPC; ++e) acc = fmaf(qv[k][e], kf[r][k][e], acc);
 #pragma unroll
-            for (int o = 1; o < 16; o <<= 1) acc += __shfl_xor_sync(kFull, acc, o);
+            for (int o = 1; o < 16; o <<= 1) acc += __shfl_xor_sync(hmask, acc, o);
             if (hl == 0 && base + r < n) zs[base + r] = rw[r] >= 0 ? zscale * acc : -INFINITY;
         }
     }

@@ -240,6 +240,18 @@ def test_edge_lengths_and_budgets(cuda_device):
                 check_head(wl, cache, dec, b, h, attn)
 
 
+@pytest.mark.parametrize("dtype,d", [(torch.float32, 64), (torch.bfloat16, 128)], ids=["f32", "bf16"])
+def test_every_sequence_empty(cuda_device, dtype, d):
+    # a batch whose sequences all hold no token: every step kernel runs with nothing to do
+    wl = make_random(B=3, H_kv=2, G=4, d=d, P=16, lens=(0, 0, 0), dtype=dtype, device="cuda",
+                     seed=14, topk=8)
+    for attn in ATTN:
+        cache, dec = run_gpu(wl, attn)
+        assert_status_ok(cache)
+        assert torch.all(dec.sel_count == 0)
+        assert torch.all(dec.out == 0) and torch.all(torch.isinf(dec.stat)) and torch.all(dec.stat < 0)
+
+
 def test_tie_storm_prefers_lower_pages(cuda_device):
     wl = make_random(B=2, H_kv=2, G=4, d=128, P=16, lens=(4096, 3000), dtype=torch.bfloat16,
                      device="cuda", seed=12, topk=37)

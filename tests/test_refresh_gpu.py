@@ -91,6 +91,7 @@ CASES = [  # B, H_kv, G, d, P, dtype, final lengths, appended tokens per sequenc
     (3, 2, 4, 128, 32, torch.bfloat16, (32 * 30, 32 * 9 + 5, 700), (16, 0, 5), False),
     (2, 2, 4, 128, 16, torch.bfloat16, (16 * 33 + 3, 16 * 16), (9, 16), True),  # with mean/var
     (2, 2, 1, 64, 32, torch.float32, (32 * 17 + 2, 32 * 9), (40, 32), False),
+    (2, 2, 4, 128, 16, torch.bfloat16, (20, 16 * 30), (20, 5), False),  # first tokens of a sequence
 ]
 
 
@@ -141,3 +142,13 @@ def test_refresh_score_bad_page_table_entry_is_flagged_alike(cuda_device):
     st, bits_ = ekv.ekv_device_status(cache)
     assert st == ekv.EKV_ERR_DEVICE and bits_ & ekv.EKV_DEV_BAD_BLOCK
     assert torch.all(scores[0, :, 20] == float("-inf"))
+
+
+def test_refresh_score_with_no_append_in_any_sequence(cuda_device):
+    # max_new > 0 but every count 0: the one-kernel path runs and refreshes nothing
+    wl = make_random(B=2, H_kv=2, G=4, d=128, P=16, lens=(16 * 12 + 3, 16 * 9), device="cuda",
+                     seed=95)
+    cache, scores, stale = run_both(wl, [0, 0], False, TOPK, max_new=16)
+    assert ekv.ekv_device_status(cache)[0] == ekv.EKV_OK
+    assert torch.equal(bits(stale), bits(cache.meta_bbox))
+    check_oracle(wl, cache, scores)
