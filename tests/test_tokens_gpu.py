@@ -21,10 +21,24 @@ CASES = list(itertools.product([torch.float32, torch.bfloat16], [64, 128], [16, 
 
 @pytest.mark.parametrize("dtype,d,P,G,attn", CASES)
 def test_token_selection_and_attention_small_ragged(cuda_device, dtype, d, P, G, attn):
-    wl = make_random(B=3, H_kv=2, G=G, d=d, P=P, lens=(900, 333, 5), dtype=dtype, device="cuda",
+    check_tokens(dtype, d, P, G, attn, T=40, lens=(900, 333, 5))
+
+
+SPLIT = [(torch.bfloat16, 128, 16, 4, ekv.EKV_ENTMAX15), (torch.float32, 64, 32, 8, ekv.EKV_SOFTMAX),
+         (torch.bfloat16, 64, 16, 1, ekv.EKV_SPARSEMAX)]
+
+
+@pytest.mark.parametrize("dtype,d,P,G,attn", SPLIT)
+def test_token_row_counts_that_split_a_warp(cuda_device, dtype, d, P, G, attn):
+    # 35 and 3 kept tokens: the two halves of a warp stream different numbers of rows (4 at a
+    # time, 8 per warp), so their reductions must not wait on each other
+    check_tokens(dtype, d, P, G, attn, T=35, lens=(900, 3, 333))
+
+
+def check_tokens(dtype, d, P, G, attn, T, lens):
+    wl = make_random(B=3, H_kv=2, G=G, d=d, P=P, lens=lens, dtype=dtype, device="cuda",
                      seed=9, topk=12)
     cache, dec = run_gpu(wl, attn)
-    T = 40
     B, H = wl.batch, wl.num_kv_heads
     ws = torch.zeros(ekv.ekv_token_workspace_bytes(cache, dec.max_sel), dtype=torch.uint8, device="cuda")
     tp = torch.empty((B, H, T), dtype=torch.int32, device="cuda")
