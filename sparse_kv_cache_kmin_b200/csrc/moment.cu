@@ -22,6 +22,7 @@ namespace ekv {
 
 constexpr int kMomTok = 4096;  // tokens per CTA of the running-sum update
 constexpr int kMomSub = 32;    // tokens staged in shared memory at a time
+constexpr int kRetPages = 64;  // selected pages per CTA of the retained sums, at most
 
 __host__ __device__ constexpr int moment_floats(int d) { return EKV_MOMENT_FLOATS(d); }
 __host__ __device__ constexpr int retained_floats(int d, int G) { return 4 + 2 * d + G * d; }
@@ -109,23 +110,23 @@ moment_update_kernel(ekv_cache c, float *__restrict__ moments, const int32_t *__
         for (int j = 0; j < RB; ++j) atomicAdd(S + (size_t)(a0 + i) * D + c0 + j, acc[i][j]);
 }
 
-// Sums over the selected tokens of one (sequence, KV head), eight selected pages per CTA:
+// Sums over the selected tokens of one (sequence, KV head), up to kRetPages selected pages per CTA:
 // n_R, sum_R k, sum_R v and u_g = sum_R v (k . q_g) for the G queries, added with atomics to a
 // zeroed [B * H_kv][retained_floats(d, G)] region. A half-warp takes one token row at a time:
 // lane l of the half reads the 16-byte pieces l of the K and V rows (8 coordinates each), the
 // G dot products k . q_g are summed over the half's lanes, and each lane keeps its coordinates
 // of sum k, sum v and u_g in registers; the CTA adds its partial sums once at the end.
 template <int DT, int D, int G>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, G <= 4 ? 2 : 1)  // G <= 4: two CTAs per SM
 moment_retained_kernel(ekv_cache c, const void *__restrict__ q, int H_q,
                        const int32_t *__restrict__ sel_idx, const int32_t *__restrict__ sel_count,
-                       int max_sel, float *__restrict__ ret)
+                       int max_sel, int ppc, float *__restrict__ ret)
 {
-    constexpr int PPC = 8;                         // selected pages per CTA
+    const int PPC = ppc;                           // selected pages per CTA (<= kRetPages)
     constexpr int EPC = Chunk<DT>::N;              // coordinates per 16-byte piece
     constexpr int W = D * Chunk<DT>::kBytes / 16;  // pieces per row
     constexpr int PPL = (W + 15) / 16;             // pieces per lane of a half-warp
-    __shared__ int s_blk[PPC], s_nt[PPC];
+    __shared__ int s_blk[kRetPages], s_nt[kRetPages];
     __shared__ float red[8][2 * D + G * D];
     __shared__ int s_cnt[8];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -180,21 +181,35 @@ moment_retained_kernel(ekv_cache c, const void *__restrict__ q, int H_q,
     __syncthreads();
     const char *kc = static_cast<const char *>(c.k_cache), *vc = static_cast<const char *>(c.v_cache);
     constexpr int RB = D * Chunk<DT>::kBytes;
-    for (int rho = warp * 2 + half; rho < PPC * P; rho += 16) {
+    // the next row's 16-byte pieces are loaded before this row is reduced, so each half-warp
+    // keeps a row in flight while it computes (every half takes the same PPC * P / 16 rows)
+    auto fetch = [&](int rho, uint4 (&kr)[PPL], uint4 (&vr)[PPL]) {
         const int slot = rho / P, t = rho - slot * P;
         const bool valid = t < s_nt[slot];
         const size_t row = ((size_t)(valid ? s_blk[slot] : 0) * c.num_kv_heads + h) * P + t;
-        float kf[PPL][EPC], vf[PPL][EPC];
 #pragma unroll
         for (int k = 0; k < PPL; ++k) {
             if (valid && owns(k)) {
-                Chunk<DT>::unpack(ld_stream16(kc + row * RB + (hl + 16 * k) * 16), kf[k]);
-                Chunk<DT>::unpack(ld_stream16(vc + row * RB + (hl + 16 * k) * 16), vf[k]);
+                kr[k] = ld_stream16(kc + row * RB + (hl + 16 * k) * 16);
+                vr[k] = ld_stream16(vc + row * RB + (hl + 16 * k) * 16);
             } else {
-#pragma unroll
-                for (int e = 0; e < EPC; ++e) { kf[k][e] = 0.f; vf[k][e] = 0.f; }
+                kr[k] = make_uint4(0, 0, 0, 0);
+                vr[k] = make_uint4(0, 0, 0, 0);
             }
         }
+        return valid;
+    };
+    uint4 kr[PPL], vr[PPL];
+    bool valid_next = fetch(warp * 2 + half, kr, vr);
+    for (int rho = warp * 2 + half; rho < PPC * P; rho += 16) {
+        const bool valid = valid_next;
+        float kf[PPL][EPC], vf[PPL][EPC];
+#pragma unroll
+        for (int k = 0; k < PPL; ++k) {
+            Chunk<DT>::unpack(kr[k], kf[k]);  // zero pieces unpack to 0
+            Chunk<DT>::unpack(vr[k], vf[k]);
+        }
+        if (rho + 16 < PPC * P) valid_next = fetch(rho + 16, kr, vr);
         float dot[G];
 #pragma unroll
         for (int g = 0; g < G; ++g) {
@@ -357,8 +372,18 @@ static cudaError_t launch_correct_t(const ekv_cache &c, const float *moments, co
     if (!after_decode) {  // retained sums (before the decode, which does not depend on them)
         cudaError_t e = cudaMemsetAsync(ret, 0, moment_retained_bytes(c.batch, c.num_kv_heads, D, G), st);
         if (e != cudaSuccess) return e;
-        const dim3 grid((max_sel + 7) / 8, c.batch * c.num_kv_heads);
-        moment_retained_kernel<DT, D, G><<<grid, 256, 0, st>>>(c, q, H_q, sel_idx, sel_count, max_sel, ret);
+        // pages per CTA: the most (up to kRetPages) that still give 1.5 CTAs per SM, so that long
+        // per-CTA row loops keep the loads flowing without leaving SMs idle
+        int dev = 0, sms = 0;
+        e = cudaGetDevice(&dev);
+        if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return e;
+        const long long pairs = (long long)c.batch * c.num_kv_heads;
+        int ppc = kRetPages;
+        while (ppc > 8 && (long long)((max_sel + ppc - 1) / ppc) * pairs * 2 < 3ll * sms) ppc >>= 1;
+        const dim3 grid((max_sel + ppc - 1) / ppc, c.batch * c.num_kv_heads);
+        moment_retained_kernel<DT, D, G><<<grid, 256, 0, st>>>(c, q, H_q, sel_idx, sel_count, max_sel,
+                                                               ppc, ret);
         return cudaGetLastError();
     }
     moment_correct_kernel<DT, D, G><<<dim3(H_q, c.batch), 256, 0, st>>>(c, moments, q, H_q, scale, ret, out, stat);

@@ -30,6 +30,21 @@ def prefill_moments(cache, wl):
 def test_moment_corrected_softmax_small_ragged(cuda_device, dtype, d, P, G):
     wl = make_random(B=3, H_kv=2, G=G, d=d, P=P, lens=(1000, 517, 1),
                      dtype=dtype, device="cuda", seed=5, topk=6)
+    check_moment(wl)
+
+
+@pytest.mark.parametrize("topk", [128, 64], ids=["pages64_per_cta", "pages32_per_cta"])
+def test_moment_many_pairs_long_retained_loops(cuda_device, topk):
+    # 16 x 8 (sequence, KV head) pairs: the retained sums take 64 or 32 selected pages per CTA
+    # (the most that leave 1.5 CTAs per SM), not the 8 of the small cases
+    lens = tuple(16 * (150 + 7 * i) + i % 5 for i in range(16))
+    wl = make_random(B=16, H_kv=8, G=4, d=128, P=16, lens=lens, dtype=torch.bfloat16,
+                     device="cuda", seed=17 + topk, topk=topk)
+    check_moment(wl, pairs=[(0, 0), (7, 3), (15, 7)])
+
+
+def check_moment(wl, pairs=None):
+    dtype, d, G = wl.k_cache.dtype, wl.head_dim, wl.num_q_heads // wl.num_kv_heads
     cache, dec = run_gpu(wl, ekv.EKV_SOFTMAX)
     mom = prefill_moments(cache, wl)
     need = ekv.ekv_moment_decode_workspace_bytes(cache, wl.num_q_heads, dec.max_sel)
@@ -43,9 +58,10 @@ def test_moment_corrected_softmax_small_ragged(cuda_device, dtype, d, P, G):
     assert st == ekv.EKV_OK, hex(bits)
     rec = mom.view(wl.batch, wl.num_kv_heads, -1).double().cpu().numpy()
     bf16 = dtype == torch.bfloat16
-    for b in range(wl.batch):
+    pairs = pairs or [(b, h) for b in range(wl.batch) for h in range(wl.num_kv_heads)]
+    for b in sorted({b for b, _ in pairs}):
         hc = HostCopy(wl, b)
-        for h in range(wl.num_kv_heads):
+        for h in [h for bb, h in pairs if bb == b]:
             n, sk, sv, S = O.moment_sums_head(hc.k, hc.v, hc.pt, hc.L, h)
             assert rec[b, h, 0] == n
             np.testing.assert_allclose(rec[b, h, 4:4 + d], sk, rtol=1e-5, atol=1e-5 * n)
