@@ -15,20 +15,22 @@
 namespace ekv {
 
 constexpr int kTokRowsSmem = 16384;  // kept tokens whose cache rows the attention keeps on chip
+constexpr int kTokPages = 64;        // selected pages per CTA of the token scores, at most
 
-// One CTA per (8 selected pages, sequence x KV head). A half-warp scores four token rows at a
-// time: lane l of the half reads the 16-byte pieces l (+16) of each row and holds the matching
-// coordinates of the group query sum Q = sum_g q_g; the partial dots are summed over the half.
+// One CTA per (up to kTokPages selected pages, sequence x KV head). A half-warp scores four
+// token rows at a time: lane l of the half reads the 16-byte pieces l (+16) of each row and
+// holds the matching coordinates of the group query sum Q = sum_g q_g; the partial dots are
+// summed over the half.
 template <int DT, int D, int G>
 __global__ void __launch_bounds__(256)
 token_score_kernel(ekv_cache c, const void *__restrict__ q, int H_q, float scale,
                    const int32_t *__restrict__ sel_idx, const int32_t *__restrict__ sel_count,
-                   int max_sel, float *__restrict__ tscores)
+                   int max_sel, int ppc, float *__restrict__ tscores)
 {
-    constexpr int PPC = 8;
+    const int PPC = ppc;  // selected pages per CTA (<= kTokPages)
     constexpr int EPC = Chunk<DT>::N, RB = D * Chunk<DT>::kBytes, W = RB / 16, PPL = (W + 15) / 16;
     constexpr int RIF = 4;  // rows in flight per half-warp
-    __shared__ int s_blk[PPC], s_nt[PPC];
+    __shared__ int s_blk[kTokPages], s_nt[kTokPages];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, half = lane >> 4, hl = lane & 15;
     const unsigned hmask = 0xffffu << (16 * half);  // this half-warp's lanes
     const int bh = blockIdx.y, b = bh / c.num_kv_heads, h = bh % c.num_kv_heads;
@@ -375,8 +377,18 @@ static cudaError_t launch_tokens_t(const ekv_cache &c, const void *q, int H_q, f
                                    const int32_t *sel_idx, const int32_t *sel_count, int max_sel,
                                    float *tscores, cudaStream_t st)
 {
-    const dim3 grid((max_sel + 7) / 8, c.batch * c.num_kv_heads);
-    token_score_kernel<DT, D, G><<<grid, 256, 0, st>>>(c, q, H_q, scale, sel_idx, sel_count, max_sel, tscores);
+    // pages per CTA: the most (up to kTokPages) that still give 3 CTAs per SM (of the 4 that fit),
+    // so that each CTA's page resolution is spent on a longer run of rows
+    int dev = 0, sms = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    const long long pairs = (long long)c.batch * c.num_kv_heads;
+    int ppc = kTokPages;
+    while (ppc > 8 && (long long)((max_sel + ppc - 1) / ppc) * pairs < 3ll * sms) ppc >>= 1;
+    const dim3 grid((max_sel + ppc - 1) / ppc, c.batch * c.num_kv_heads);
+    token_score_kernel<DT, D, G><<<grid, 256, 0, st>>>(c, q, H_q, scale, sel_idx, sel_count, max_sel,
+                                                        ppc, tscores);
     return cudaGetLastError();
 }
 

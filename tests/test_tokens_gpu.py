@@ -35,9 +35,18 @@ def test_token_row_counts_that_split_a_warp(cuda_device, dtype, d, P, G, attn):
     check_tokens(dtype, d, P, G, attn, T=35, lens=(900, 3, 333))
 
 
-def check_tokens(dtype, d, P, G, attn, T, lens):
-    wl = make_random(B=3, H_kv=2, G=G, d=d, P=P, lens=lens, dtype=dtype, device="cuda",
-                     seed=9, topk=12)
+@pytest.mark.parametrize("B,topk", [(16, 128), (32, 128)], ids=["pages32_per_cta", "pages64_per_cta"])
+def test_token_scores_with_long_per_cta_runs(cuda_device, B, topk):
+    # B x 8 (sequence, KV head) pairs with 128 selected pages: the token scores take 32 or 64
+    # selected pages per CTA (the most that leave 3 CTAs per SM), not the 8 of the small cases
+    lens = tuple(16 * (140 + 5 * i) + i % 7 for i in range(B))
+    check_tokens(torch.bfloat16, 128, 16, 4, ekv.EKV_ENTMAX15, T=512, lens=lens, H=8, topk=topk,
+                 heads=[(0, 0), (B // 2, 5), (B - 1, 7)])
+
+
+def check_tokens(dtype, d, P, G, attn, T, lens, H=2, topk=12, heads=None):
+    wl = make_random(B=len(lens), H_kv=H, G=G, d=d, P=P, lens=lens, dtype=dtype, device="cuda",
+                     seed=9, topk=topk)
     cache, dec = run_gpu(wl, attn)
     B, H = wl.batch, wl.num_kv_heads
     ws = torch.zeros(ekv.ekv_token_workspace_bytes(cache, dec.max_sel), dtype=torch.uint8, device="cuda")
@@ -53,9 +62,10 @@ def check_tokens(dtype, d, P, G, attn, T, lens):
     st, bits = ekv.ekv_device_status(cache)
     assert st == ekv.EKV_OK, hex(bits)
     bf16 = dtype == torch.bfloat16
-    for b in range(B):
+    heads = heads or [(b, h) for b in range(B) for h in range(H)]
+    for b in sorted({b for b, _ in heads}):
         hc = HostCopy(wl, b)
-        for h in range(H):
+        for h in [h for bb, h in heads if bb == b]:
             ns = int(dec.sel_count[b, h].item())
             sel = dec.sel_idx[b, h, :ns].cpu().numpy()
             pages, pos = O.token_topk_head(hc.k, hc.pt, hc.L, h, hc.q[h], wl.scale, sel, T)
