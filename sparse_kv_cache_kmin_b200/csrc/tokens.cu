@@ -80,34 +80,45 @@ token_score_kernel(ekv_cache c, const void *__restrict__ q, int H_q, float scale
     const int nrows = (i1 - i0) * P;
     float *out = tscores + (size_t)bh * max_sel * P + (size_t)i0 * P;
     const char *kc = static_cast<const char *>(c.k_cache);
-    for (int base = (warp * 2 + half) * RIF; base < nrows; base += 16 * RIF) {
-        float kf[RIF][PPL][EPC];
-        bool ok[RIF];
+    // the next RIF rows' 16-byte pieces are loaded before the current ones are reduced (kept
+    // raw and unpacked row by row), so each half-warp has two groups of rows in flight
+    auto fetch = [&](int base, uint4 (&raw)[RIF][PPL], bool (&ok)[RIF]) {
 #pragma unroll
         for (int r = 0; r < RIF; ++r) {
             const int rr = base + r, slot = rr / P, t = rr - slot * P;
             ok[r] = rr < nrows && t < s_nt[slot < PPC ? slot : 0];
             const size_t row = ((size_t)(ok[r] ? s_blk[slot] : 0) * H + h) * P + t;
 #pragma unroll
-            for (int k = 0; k < PPL; ++k) {
-                if (ok[r] && owns(k)) {
-                    Chunk<DT>::unpack(ld_stream16(kc + row * RB + (hl + 16 * k) * 16), kf[r][k]);
-                } else {
-#pragma unroll
-                    for (int e = 0; e < EPC; ++e) kf[r][k][e] = 0.f;
-                }
-            }
+            for (int k = 0; k < PPL; ++k)
+                raw[r][k] = ok[r] && owns(k) ? ld_stream16(kc + row * RB + (hl + 16 * k) * 16)
+                                             : make_uint4(0, 0, 0, 0);
         }
+    };
+    uint4 cur[RIF][PPL], nxt[RIF][PPL];
+    bool okc[RIF], okn[RIF];
+    int base = (warp * 2 + half) * RIF;
+    if (base < nrows) fetch(base, cur, okc);
+    for (; base < nrows; base += 16 * RIF) {
+        if (base + 16 * RIF < nrows) fetch(base + 16 * RIF, nxt, okn);
 #pragma unroll
         for (int r = 0; r < RIF; ++r) {
             float acc = 0.f;
 #pragma unroll
-            for (int k = 0; k < PPL; ++k)
+            for (int k = 0; k < PPL; ++k) {
+                float kf[EPC];
+                Chunk<DT>::unpack(cur[r][k], kf);  // zero pieces unpack to 0
 #pragma unroll
-                for (int e = 0; e < EPC; ++e) acc = fmaf(qv[k][e], kf[r][k][e], acc);
+                for (int e = 0; e < EPC; ++e) acc = fmaf(qv[k][e], kf[e], acc);
+            }
 #pragma unroll
             for (int o = 1; o < 16; o <<= 1) acc += __shfl_xor_sync(hmask, acc, o);
-            if (hl == 0 && base + r < nrows) out[base + r] = ok[r] ? scale * acc : -INFINITY;
+            if (hl == 0 && base + r < nrows) out[base + r] = okc[r] ? scale * acc : -INFINITY;
+        }
+#pragma unroll
+        for (int r = 0; r < RIF; ++r) {
+            okc[r] = okn[r];
+#pragma unroll
+            for (int k = 0; k < PPL; ++k) cur[r][k] = nxt[r][k];
         }
     }
     pdl_trigger();
