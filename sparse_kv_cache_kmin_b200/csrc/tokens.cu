@@ -198,33 +198,46 @@ token_attend_kernel(ekv_cache c, const void *__restrict__ q, int H_q, float scal
 #pragma unroll
         for (int e = 0; e < EPC; ++e) qv[k][e] = owns(k) ? qs[(hl + 16 * k) * EPC + e] : 0.f;
     const char *kc = static_cast<const char *>(c.k_cache), *vc = static_cast<const char *>(c.v_cache);
-    // logits: a half-warp takes RIF rows at a time, lane l reading pieces l (+16) of each
-    for (int base = (warp * 2 + half) * RIF; base < n; base += 16 * RIF) {
-        float kf[RIF][PPL][EPC];
-        long long rw[RIF];
+    // logits: a half-warp takes RIF rows at a time, lane l reading pieces l (+16) of each; the
+    // next RIF rows' pieces are loaded (kept raw) before the current ones are reduced
+    auto fetch = [&](int base, uint4 (&raw)[RIF][PPL], bool (&ok)[RIF]) {
 #pragma unroll
         for (int r = 0; r < RIF; ++r) {
-            rw[r] = base + r < n ? row_at(base + r) : -1;
-#pragma unroll
-            for (int k = 0; k < PPL; ++k) {
-                if (rw[r] >= 0 && owns(k)) {
-                    Chunk<DT>::unpack(ld_stream16(kc + (size_t)rw[r] * RB + (hl + 16 * k) * 16), kf[r][k]);
-                } else {
-#pragma unroll
-                    for (int e = 0; e < EPC; ++e) kf[r][k][e] = 0.f;
-                }
-            }
-        }
-#pragma unroll
-        for (int r = 0; r < RIF; ++r) {
-            float acc = 0.f;
+            const long long rw = base + r < n ? row_at(base + r) : -1;
+            ok[r] = rw >= 0;
 #pragma unroll
             for (int k = 0; k < PPL; ++k)
+                raw[r][k] = ok[r] && owns(k) ? ld_stream16(kc + (size_t)rw * RB + (hl + 16 * k) * 16)
+                                             : make_uint4(0, 0, 0, 0);
+        }
+    };
+    {
+        uint4 cur[RIF][PPL], nxt[RIF][PPL];
+        bool okc[RIF], okn[RIF];
+        int base = (warp * 2 + half) * RIF;
+        if (base < n) fetch(base, cur, okc);
+        for (; base < n; base += 16 * RIF) {
+            if (base + 16 * RIF < n) fetch(base + 16 * RIF, nxt, okn);
 #pragma unroll
-                for (int e = 0; e < EPC; ++e) acc = fmaf(qv[k][e], kf[r][k][e], acc);
+            for (int r = 0; r < RIF; ++r) {
+                float acc = 0.f;
 #pragma unroll
-            for (int o = 1; o < 16; o <<= 1) acc += __shfl_xor_sync(hmask, acc, o);
-            if (hl == 0 && base + r < n) zs[base + r] = rw[r] >= 0 ? zscale * acc : -INFINITY;
+                for (int k = 0; k < PPL; ++k) {
+                    float kf[EPC];
+                    Chunk<DT>::unpack(cur[r][k], kf);  // zero pieces unpack to 0
+#pragma unroll
+                    for (int e = 0; e < EPC; ++e) acc = fmaf(qv[k][e], kf[e], acc);
+                }
+#pragma unroll
+                for (int o = 1; o < 16; o <<= 1) acc += __shfl_xor_sync(hmask, acc, o);
+                if (hl == 0 && base + r < n) zs[base + r] = okc[r] ? zscale * acc : -INFINITY;
+            }
+#pragma unroll
+            for (int r = 0; r < RIF; ++r) {
+                okc[r] = okn[r];
+#pragma unroll
+                for (int k = 0; k < PPL; ++k) cur[r][k] = nxt[r][k];
+            }
         }
     }
     __syncthreads();
