@@ -281,17 +281,48 @@ score_gauss_kernel(ekv_cache c, const void *__restrict__ q, int H_q, float scale
     const long lo = (long)blockIdx.x * TG / gridDim.x;
     const long hi = (long)(blockIdx.x + 1) * TG / gridDim.x;
 
+    // Work group gi -> (sequence, KV head, first page); as in the top-k scan, a group's
+    // page-table entries are fetched one group ahead, so its metadata loads wait on one memory
+    // latency, not two.
+    struct Grp { int bb, hh, j0, np; };
+    auto locate = [&](long gi) {
+        Grp g;
+        g.bb = find_seq(pre, B, gi);
+        int len = c.seq_lens[g.bb];
+        len = len < 0 ? 0 : (len > c.max_pages * P ? c.max_pages * P : len);
+        g.np = (len + P - 1) / P;
+        const int ng = (g.np + PGG - 1) / PGG;
+        const int r = (int)(gi - pre[g.bb]);
+        g.hh = r / ng;
+        g.j0 = (r % ng) * PGG;
+        return g;
+    };
+    auto fetch_blk = [&](const Grp &g) {  // block of page j0 + lane % PGG: -1 past the end, -2 bad
+        int blk = -1;
+        const int jl = g.j0 + lane % PGG;
+        if (jl < g.np) {
+            blk = c.page_table[(size_t)g.bb * c.max_pages + jl];
+            if (blk < 0 || blk >= c.num_blocks) {
+                flag(c.dev_status, EKV_DEV_BAD_BLOCK);
+                blk = -2;
+            }
+        }
+        return blk;
+    };
+
     int cur_bh = -1;
     float qv[G][VEC];
-    for (long gi = lo + warp; gi < hi; gi += 8) {
-        const int bb = find_seq(pre, B, gi);
-        int len = c.seq_lens[bb];
-        len = len < 0 ? 0 : (len > c.max_pages * P ? c.max_pages * P : len);
-        const int np = (len + P - 1) / P;
-        const int ng = (np + PGG - 1) / PGG;
-        const int r = (int)(gi - pre[bb]);
-        const int hh = r / ng;
-        const int j0 = (r % ng) * PGG;
+    long gi = lo + warp;
+    Grp nxt = {0, 0, 0, 0};
+    int nxt_blk = -1;
+    if (gi < hi) {
+        nxt = locate(gi);
+        nxt_blk = fetch_blk(nxt);
+    }
+    for (; gi < hi; gi += 8) {
+        const Grp cur = nxt;
+        const int myblk = nxt_blk;
+        const int bb = cur.bb, hh = cur.hh, j0 = cur.j0, np = cur.np;
         const int bh = bb * H + hh;
         if (bh != cur_bh) {
             cur_bh = bh;
@@ -300,15 +331,6 @@ score_gauss_kernel(ekv_cache c, const void *__restrict__ q, int H_q, float scale
 #pragma unroll
                 for (int e = 0; e < VEC; ++e)
                     qv[g][e] = load_elem<DT>(q, ((size_t)bb * H_q + hh * G + g) * D + lane * VEC + e);
-        }
-        int myblk = -1;
-        const int jl = j0 + lane % PGG;
-        if (jl < np) {
-            myblk = c.page_table[(size_t)bb * c.max_pages + jl];
-            if (myblk < 0 || myblk >= c.num_blocks) {
-                flag(c.dev_status, EKV_DEV_BAD_BLOCK);
-                myblk = -2;
-            }
         }
         float kn[PGG][VEC], kx[PGG][VEC], mu[PGG][VEC], vr[PGG][VEC];
 #pragma unroll
@@ -324,6 +346,10 @@ score_gauss_kernel(ekv_cache c, const void *__restrict__ q, int H_q, float scale
 #pragma unroll
                 for (int e = 0; e < VEC; ++e) { kn[i][e] = 0.f; kx[i][e] = 0.f; mu[i][e] = 0.f; vr[i][e] = 0.f; }
             }
+        }
+        if (gi + 8 < hi) {
+            nxt = locate(gi + 8);
+            nxt_blk = fetch_blk(nxt);
         }
         float pu[NV], pm[NV], pv[NV];
 #pragma unroll
