@@ -289,6 +289,16 @@ moment_correct_kernel(ekv_cache c, const float *__restrict__ moments, const void
     const size_t bh = (size_t)b * c.num_kv_heads + h, bq = (size_t)b * H_q + hq;
     const float *rec = moments + bh * moment_floats(D);
     const float *r = ret + bh * retained_floats(D, G);
+    // (sum v k^T) q: warp w takes rows a = w, w + 8, ... (D / 8 of them), lane l coordinates
+    // l, l + 32, ...; every row's loads are issued first, before anything else of the
+    // correction, so they are in flight together and overlap the steps below
+    const float *S = rec + 4 + 2 * D;
+    constexpr int RPW = D / 8, CPL = D / 32;
+    float sv[RPW][CPL];
+#pragma unroll
+    for (int i = 0; i < RPW; ++i)
+#pragma unroll
+        for (int k = 0; k < CPL; ++k) sv[i][k] = __ldg(S + (size_t)(warp + 8 * i) * D + lane + 32 * k);
     const float n_e = rec[0] - r[0];
     if (!(n_e >= 0.5f)) return;  // nothing skipped: the plain softmax stands
     for (int i = tid; i < D; i += 256) {
@@ -305,16 +315,6 @@ moment_correct_kernel(ekv_cache c, const float *__restrict__ moments, const void
     float qk = 0.f;
 #pragma unroll
     for (int w = 0; w < 8; ++w) qk += red[w];
-    // (sum v k^T) q: warp w takes rows a = w, w + 8, ... (D / 8 of them), lane l coordinates
-    // l, l + 32, ...; every row's loads are issued before any product, so they are in flight
-    // together
-    const float *S = rec + 4 + 2 * D;
-    constexpr int RPW = D / 8, CPL = D / 32;
-    float sv[RPW][CPL];
-#pragma unroll
-    for (int i = 0; i < RPW; ++i)
-#pragma unroll
-        for (int k = 0; k < CPL; ++k) sv[i][k] = __ldg(S + (size_t)(warp + 8 * i) * D + lane + 32 * k);
 #pragma unroll
     for (int i = 0; i < RPW; ++i) {
         float acc = 0.f;
